@@ -1,0 +1,387 @@
+"""Decode-step benchmark of the persistent megakernel (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama1b]
+                    [--impl mk|reference] [--no-cpu-baseline]
+
+A step is one decode step (the whole hot path: every layer's fused
+RMSNorm->QKV->RoPE->KV append, split-K attention + merge, O-proj+residual,
+RMSNorm->gate/up->SiLU*up, down+residual, then final norm->LM head->argmax)
+for one sequence, run as one persistent-kernel launch through the C ABI.
+Warm-up steps feed the synthetic prompt at positions 0..W-1; the K timed
+steps continue autoregressively on the device (each step reads the token
+the previous step wrote) at positions W..W+K-1.  Weights (2.47 GB for the
+1B shape) exceed the 126 MB L2, so no flush is needed between steps.
+
+`value` is device time per token (CUDA events over the K launches on the
+launching stream, max over ranks); `e2e` is the same through host buffers:
+per step the token and position are copied from pinned host memory, the
+step launched, and the next token copied back and waited for.
+
+Multi-GPU: every rank runs an independent replica (the single-sequence step
+does not shard without a per-layer exchange); `value` is then the max rank
+time divided by all ranks' tokens.
+
+--impl reference times the oracle (the plain fp64 CPU definition in
+oracle/) on the host: each step is a bounded sample -- one decoder layer and
+1/L of the LM-head rows of the same shape, weights and positions -- and the
+reported ms/token is that sample's time times L.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from persistent_decode_megakernel_02_b200 import workloads as wl  # noqa: E402
+
+METRIC = "decode ms/token @bs1 (Llama-3.2-1B shape); achieved HBM GB/s vs roofline"
+UNIT = "ms/token"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (the roofline numerator)
+# ---------------------------------------------------------------------------
+def step_weight_bytes(shape: wl.ModelShape) -> int:
+    """bf16 bytes one decode step must read: every weight matrix once, every
+    RMSNorm gain once, one embedding row (the LM head is read in full)."""
+    H, F, V, L = shape.hidden, shape.ffn, shape.vocab, shape.layers
+    QD, KD = shape.n_q_heads * shape.head_dim, shape.n_kv_heads * shape.head_dim
+    mats = L * ((QD + 2 * KD) * H + H * QD + 3 * F * H) + V * H
+    norms = (2 * L + 1) * H
+    return 2 * (mats + norms + H)
+
+
+def step_kv_bytes(shape: wl.ModelShape, contexts) -> int:
+    """bf16 K and V bytes attention reads: C positions per sequence per layer."""
+    per_pos = 2 * shape.n_kv_heads * shape.head_dim * 2 * shape.layers
+    return int(per_pos * int(np.sum(contexts)))
+
+
+def bandwidth_bound_ms(bytes_per_step: float, gbs: float) -> float:
+    """Time to stream `bytes_per_step` at `gbs` GB/s (1 GB = 1e9 B)."""
+    return bytes_per_step / (gbs * 1e9) * 1e3
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self) -> dict:
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        pw = np.array([r[2] for r in rows])
+        load = [r for r in rows if r[2] >= np.median(pw)] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in load:
+            for n, v in zip(names, r[3][1:5]):
+                if v.lower() in ("active", "1", "yes"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median([r[0] for r in load])),
+                "sm_max_mhz": float(max(r[1] for r in rows)),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """One decoder layer plus 1/L of the LM-head rows of `shape`, built from
+    the same weights, so that a step of it costs 1/L of a full oracle step.
+    The KV prefix is seeded N(0,1) data (attention cost depends only on C)."""
+
+    def __init__(self, shape: wl.ModelShape, bits: dict, max_seq: int):
+        import oracle
+        L = shape.layers
+        self.L = L
+        vs = max(1, shape.vocab // L)
+        cfg = dict(layers=1, hidden=shape.hidden, n_q_heads=shape.n_q_heads,
+                   n_kv_heads=shape.n_kv_heads, head_dim=shape.head_dim, ffn=shape.ffn,
+                   vocab=vs, max_seq=max_seq, rope_theta=shape.rope_theta, rms_eps=shape.rms_eps)
+        w = {"embed": bits["embed"][:vs], "lm_head": bits["lm_head"][:vs],
+             "final_norm": bits["final_norm"]}
+        for k in ("attn_norm", "mlp_norm", "wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+            w[k] = [bits[k][0]]
+        self.model = oracle.OracleModel(cfg, w)
+        self.kc, self.vc = self.model.new_cache()
+        rng = np.random.default_rng(5)
+        for a in self.kc + self.vc:
+            a[...] = (rng.standard_normal(a.shape).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+        self.vs = vs
+
+    def step_ms(self, token: int, pos: int) -> float:
+        t0 = time.perf_counter()
+        self.model.decode_step(self.kc, self.vc, int(token) % self.vs, int(pos))
+        return (time.perf_counter() - t0) * 1e3 * self.L
+
+
+def cpu_cores_used() -> int:
+    return 1   # the oracle is single-threaded C
+
+
+# ---------------------------------------------------------------------------
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=512)
+    ap.add_argument("--warmup", type=int, default=39)
+    ap.add_argument("--workload", default="llama1b", choices=["llama1b", "llama8b", "longctx", "tiny"])
+    ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=64)
+    ap.add_argument("--cpu-sample-s", type=float, default=15.0)
+    ap.add_argument("--flags", type=int, default=0, help="mk_config.flags")
+    ap.add_argument("--attn-chunks", type=int, default=0)
+    return ap.parse_args()
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    W = max(3, args.warmup)
+    K = max(1, args.steps)
+    wk = wl.WORKLOADS[args.workload]
+    shape = wk.shape
+    prefill = wk.prefill_len
+    start = prefill if prefill else 0
+    max_seq = max(wk.max_seq, start + W + K + 1)
+    config = {"workload": f"{wk.name}: {shape.name} L{shape.layers} H{shape.hidden} "
+                          f"{shape.n_q_heads}/{shape.n_kv_heads} heads d{shape.head_dim} "
+                          f"F{shape.ffn} V{shape.vocab}" + (f", KV prefilled to {prefill}" if prefill else ""),
+              "batch": 1, "positions": [start + W, start + W + K - 1],
+              "l2": "weights exceed L2 (no flush needed)", "parallelism": f"replicas x{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import torch
+        w_host = wl.make_weights(shape, seed=1234, device="cuda" if torch.cuda.is_available() else "cpu")
+        bits = w_host.numpy_bits()
+        del w_host
+        samp = OracleSample(shape, bits, max_seq)
+        prompt = wl.make_prompt(shape.vocab, W, seed=42)
+        for i in range(W):
+            samp.step_ms(prompt[i], start + i)
+        times = [samp.step_ms(prompt[i % W], start + W + i) for i in range(K)]
+        total = float(np.sum(times))
+        ms = total / K
+        sample = (f"each step: 1 of {shape.layers} decoder layers + 1/{shape.layers} of the LM-head rows, "
+                  f"time x{shape.layers}")
+        out = {"impl": "reference", "metric": METRIC, "value": ms, "unit": UNIT, "n_gpus": world,
+               "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": False,
+               "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+               "config": config,
+               "cpu_baseline": {"value": ms, "unit": UNIT, "cores": cpu_cores_used(),
+                                "kind": "oracle", "sample": sample},
+               "e2e": {"value": ms, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(out), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from persistent_decode_megakernel_02_b200 import mk
+
+    weights = wl.make_weights(shape, seed=1234, device=dev)
+    kc, vc = wl.make_kv(shape, 1, max_seq, device=dev, prefill_len=prefill)
+    ctx = mk.Context(weights, kc, vc, max_seq, 1, flags=args.flags, attn_chunks=args.attn_chunks)
+    stream = torch.cuda.Stream(device=dev)
+    prompt = torch.from_numpy(wl.make_prompt(shape.vocab, W, seed=42)).to(dev)
+    toks = torch.zeros(W + K + 1, dtype=torch.int32, device=dev)
+    toks[:W] = prompt
+    pos = torch.arange(start, start + W + K + 1, dtype=torch.int32, device=dev)
+    logits = torch.empty(1, shape.vocab, dtype=torch.float32, device=dev)
+    dummy_next = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def one(i, next_slot):
+        ctx.decode_step(toks[i:i + 1], pos[i:i + 1], next_slot, logits, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(W):           # prompt, teacher-forced
+            one(i, dummy_next if i < W - 1 else toks[W:W + 1])
+        stream.synchronize()
+        st = ctx.sync(stream)
+        if st != 0:
+            raise mk.MkError(st, "warm-up")
+        if world > 1:
+            torch.distributed.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            e0.record(stream)
+            for i in range(W, W + K):
+                one(i, toks[i + 1:i + 2])
+            e1.record(stream)
+            stream.synchronize()
+        st = ctx.sync(stream)
+        if st != 0:
+            raise mk.MkError(st, "timed steps")
+        dev_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([dev_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        dev_ms = float(t.item())
+    per_launch_ms = dev_ms / K
+    value = dev_ms / (K * world)
+
+    # ---- roofline of the kernel (the only kernel in the step)
+    contexts = np.arange(start + W, start + W + K) + 1
+    wbytes = step_weight_bytes(shape)
+    kvbytes = step_kv_bytes(shape, contexts) / K
+    alg_bytes = wbytes + kvbytes
+    peaks = measured_peaks()
+    achieved = alg_bytes / (per_launch_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "peak_source": peaks["source"], "bytes_per_launch": int(alg_bytes),
+                "bound_ms": round(bandwidth_bound_ms(alg_bytes, peaks["hbm_gbs"]), 4)}
+
+    # ---- end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_tok = torch.zeros(1, dtype=torch.int32).pin_memory()
+        h_pos = torch.zeros(1, dtype=torch.int32).pin_memory()
+        h_next = torch.zeros(1, dtype=torch.int32).pin_memory()
+        d_tok = torch.zeros(1, dtype=torch.int32, device=dev)
+        d_pos = torch.zeros(1, dtype=torch.int32, device=dev)
+        d_next = torch.zeros(1, dtype=torch.int32, device=dev)
+        n = min(args.e2e_steps, K)
+        h_tok[0] = int(toks[W].item())
+        p0 = start + W
+        with torch.cuda.stream(stream):
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            f0 = torch.cuda.Event(enable_timing=True)
+            f1 = torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for i in range(n):
+                h_pos[0] = p0 + i
+                d_tok.copy_(h_tok, non_blocking=True)
+                d_pos.copy_(h_pos, non_blocking=True)
+                ctx.decode_step(d_tok, d_pos, d_next, logits, stream=stream)
+                h_next.copy_(d_next, non_blocking=True)
+                stream.synchronize()
+                h_tok[0] = h_next[0]
+            f1.record(stream)
+            stream.synchronize()
+            st = ctx.sync(stream)
+            if st != 0:
+                raise mk.MkError(st, "e2e steps")
+            e2e_ms = f0.elapsed_time(f1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(e2e_ms / (n * world), 5), "unit": UNIT, "h2d_bytes_per_step": 8,
+               "d2h_bytes_per_step": 4, "steps": n}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        bits = weights.numpy_bits()
+        samp = OracleSample(shape, bits, max_seq)
+        times = []
+        t_end = time.perf_counter() + args.cpu_sample_s
+        i = 0
+        while time.perf_counter() < t_end or i < 3:
+            times.append(samp.step_ms(int(toks[W + (i % K)].item()), start + W + (i % K)))
+            i += 1
+        cpu = {"value": round(float(np.mean(times)), 3), "unit": UNIT, "cores": cpu_cores_used(),
+               "kind": "oracle",
+               "sample": f"{i} oracle steps of 1 of {shape.layers} layers + 1/{shape.layers} of the "
+                         f"LM-head rows at positions {start + W}.., time x{shape.layers}; "
+                         f"host has {os.cpu_count()} cores"}
+
+    if rank == 0:
+        out = {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world,
+               "steps": K, "warmup": W, "ms_per_step": round(per_launch_ms, 5),
+               "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+               "dtype": "bf16 weights/KV, fp32 accumulate", "data": "synthetic",
+               "config": config, "roofline": roofline, "cpu_baseline": cpu,
+               "e2e": e2e, "gpu_launches": K, "clocks": clk.summary(),
+               "achieved_gbs": round(achieved, 1)}
+        print(json.dumps(out), flush=True)
+    ctx.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

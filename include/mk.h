@@ -1,0 +1,233 @@
+/*
+ * mk.h -- C ABI of the B200 persistent decode megakernel.
+ *
+ * One call of mk_decode_step runs the single-token decode step of a
+ * Llama-style decoder for up to max_batch independent sequences as ONE
+ * persistent kernel launch on a B200 (sm_100a).  Inside the launch, a static
+ * task graph built by mk_create splits the rows of every matrix-vector op
+ * into per-SM tasks; tasks wait on and bump event counters in global memory
+ * (no grid-wide barrier between layers), a loader warp per SM streams the
+ * weights of upcoming tasks into paged shared memory ahead of their
+ * dependencies, a scheduler warp per SM activates tasks when their events
+ * fire, and worker warps run the fused task bodies.
+ *
+ * Where the operations are defined (reference pages on the persistent
+ * decode megakernel topic):
+ *  - task / event model (a task runs on one SM, bumps its triggering event
+ *    when done; a task may start once its dependent event has fired, i.e.
+ *    its counter reached the threshold): "显著提升小LLM的性能，所有kernel集成一个
+ *    巨大kernel！" (zejuncao.github.io, 2025-06-26), Figure 2 and Figure 3 text;
+ *  - worker loop (fetch task, run, notify) and scheduler warps: same page,
+ *    MPK runtime section; warp specialisation: zizhi168.cn/news/174794,
+ *    section 2.2;
+ *  - fused ops of one decoder layer and the model tail: the Hazy megakernel
+ *    news page (sfrk.com.cn/ruanjian/202506/86466), paragraph listing the
+ *    fused instructions, and the MPK walkthrough's per-layer *_layer calls
+ *    (zizhi168.cn/news/174794, section 3.3.1);
+ *  - paged shared memory with early weight preload: the Hazy page, paragraph
+ *    on static plans and paged shared memory.
+ *
+ * Conventions for every entry point:
+ *  - Pointers documented "device" must be device pointers of the current
+ *    CUDA device; "host" pointers are ordinary host memory.
+ *  - The caller owns every weight, KV-cache, token, position and output
+ *    buffer and keeps it alive while a context that uses it exists; the
+ *    library never frees them.  The library owns its scratch (activations,
+ *    partial results, event counters, task tables, error word, trace).
+ *  - Return value: MK_OK (0) or one of the MK_ERR_* codes below;
+ *    mk_status_string() names them.  Invalid arguments are reported
+ *    synchronously with MK_ERR_INVALID and nothing is launched.
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (NULL = the legacy default stream). */
+typedef struct CUstream_st *mk_stream_t;
+
+enum mk_status {
+    MK_OK = 0,
+    MK_ERR_INVALID = 1,  /* bad argument or unsupported shape             */
+    MK_ERR_CUDA = 2,     /* a CUDA runtime call failed                     */
+    MK_ERR_TIMEOUT = 3,  /* a device-side wait exceeded timeout_ns         */
+    MK_ERR_OOM = 4,      /* device or pinned host allocation failed        */
+    MK_ERR_STATE = 5     /* context unusable after an earlier device error */
+};
+
+enum mk_flags {
+    MK_FLAG_TRACE = 1,        /* record a per-task timing trace (globaltimer) */
+    MK_FLAG_NO_L2_PREFETCH = 2 /* loader does not prefetch ahead into L2     */
+};
+
+/* Upper bounds of the shapes the kernel tiles. */
+#define MK_MAX_BATCH 1
+#define MK_MAX_K 16384      /* max of hidden, n_q_heads*head_dim and ffn */
+#define MK_MAX_HEAD_DIM 256
+
+/*
+ * Model shape and run options.
+ *  hidden, ffn, n_q_heads*head_dim: multiples of 8, at most MK_MAX_K.
+ *  head_dim: multiple of 8, at most MK_MAX_HEAD_DIM; n_kv_heads divides
+ *  n_q_heads.  max_seq: KV capacity per sequence (positions 0..max_seq-1).
+ *  max_batch: 1..MK_MAX_BATCH.  rms_eps > 0, rope_theta > 1.
+ *  attn_chunks: split-K chunks per (sequence, KV head) in the attention
+ *  op; 0 picks one chunk count so that the attention tasks cover the SMs.
+ *  timeout_ns: bound on every device-side wait; 0 means 2 s.
+ */
+typedef struct mk_config {
+    int layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+    int max_seq, max_batch;
+    float rope_theta, rms_eps;
+    int flags;
+    int attn_chunks;
+    long long timeout_ns;
+} mk_config;
+
+/*
+ * Weights, all bf16, row-major, 16-byte aligned, in device memory.  The
+ * per-layer members are HOST arrays of `layers` device pointers (copied by
+ * mk_create; the arrays themselves may be freed after it returns).
+ *   embed      [vocab][hidden]
+ *   lm_head    [vocab][hidden]          (may equal embed: tied head)
+ *   final_norm [hidden]
+ *   attn_norm, mlp_norm  [layers] -> [hidden]        RMSNorm gains
+ *   wq [layers] -> [n_q_heads*head_dim][hidden]
+ *   wk, wv [layers] -> [n_kv_heads*head_dim][hidden]
+ *   wo [layers] -> [hidden][n_q_heads*head_dim]
+ *   wg, wu [layers] -> [ffn][hidden]    (gate, up)
+ *   wd [layers] -> [hidden][ffn]        (down)
+ */
+typedef struct mk_weights {
+    const void *embed, *lm_head, *final_norm;
+    const void *const *attn_norm, *const *mlp_norm;
+    const void *const *wq, *const *wk, *const *wv, *const *wo;
+    const void *const *wg, *const *wu, *const *wd;
+} mk_weights;
+
+/*
+ * KV cache: per layer, device bf16 [max_batch][n_kv_heads][max_seq][head_dim]
+ * (keys stored after RoPE).  k, v are HOST arrays of `layers` device
+ * pointers.  Sequence b of a step uses batch slot b.
+ */
+typedef struct mk_kv {
+    void *const *k, *const *v;
+} mk_kv;
+
+typedef struct mk_ctx mk_ctx;
+
+/*
+ * Validate the shape, build the static task graph for this device (one
+ * persistent CTA per SM), allocate scratch and upload the tables.  Blocks
+ * the host.  *out receives the context (NULL on error).
+ * Errors: MK_ERR_INVALID (shape or pointer checks), MK_ERR_OOM, MK_ERR_CUDA.
+ */
+int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx **out);
+
+/*
+ * One decode step for sequences 0..batch-1, enqueued on `stream` (one
+ * kernel launch; asynchronous).
+ *   tokens    device int32 [batch]: input token of each sequence.
+ *   positions device int32 [batch]: position of that token; its K/V entry
+ *             is written at that slot of every layer's cache and attention
+ *             covers positions 0..positions[b].
+ *   logits_out   device float [batch][vocab], or NULL to skip writing.
+ *   next_tok_out device int32 [batch]: argmax of each row of logits
+ *                (lowest index on ties).
+ * 1 <= batch <= max_batch.  A token outside [0, vocab) or a position
+ * outside [0, max_seq) is detected on the device: the step then does no
+ * work and the context reports MK_ERR_INVALID from mk_sync.  A device
+ * timeout is reported as MK_ERR_TIMEOUT by mk_sync.  After a device error
+ * every call returns MK_ERR_STATE until mk_reset.
+ * Not thread-safe with respect to the same context.
+ */
+int mk_decode_step(mk_ctx *ctx, const int32_t *tokens, const int32_t *positions, int batch,
+                   float *logits_out, int32_t *next_tok_out, mk_stream_t stream);
+
+/* Wait for `stream`, then return the device status of the context
+ * (MK_OK, MK_ERR_INVALID, MK_ERR_TIMEOUT) or MK_ERR_CUDA. */
+int mk_sync(mk_ctx *ctx, mk_stream_t stream);
+
+/* Clear the device error state and the event counters (blocks the host;
+ * no step may be in flight). */
+int mk_reset(mk_ctx *ctx);
+
+/* Free the context's scratch (blocks the host).  NULL is accepted. */
+int mk_destroy(mk_ctx *ctx);
+
+const char *mk_status_string(int status);
+
+/* ---- introspection (tests, tracing) ------------------------------------ */
+
+typedef struct mk_info {
+    int num_sms;        /* persistent CTAs = SMs used */
+    int num_tasks;
+    int num_events;
+    int num_ops;
+    int attn_chunks;
+    int max_queue;      /* longest per-SM task queue */
+    int page_bytes, num_pages;
+    long long steps_run; /* completed mk_decode_step launches since create/reset */
+    unsigned int err_code, err_info; /* device error word (0 = none) */
+} mk_info;
+
+int mk_get_info(mk_ctx *ctx, mk_info *out);
+
+/* Copy the event counters (uint32 [num_events]) and thresholds to host.
+ * After s successful steps every counter equals threshold * s (mod 2^32).
+ * Blocks the host. */
+int mk_get_event_counts(mk_ctx *ctx, uint32_t *counts_out, uint32_t *thresholds_out, int n);
+
+/* Scratch buffers readable after a step (host copy, blocks the host):
+ * MK_BUF_HIDDEN float [max_batch][hidden] residual stream after the last
+ * layer; MK_BUF_Q float [max_batch][nq*head_dim] last layer's rotated q;
+ * MK_BUF_ATTN float [max_batch][nq*head_dim] last layer's attention output;
+ * MK_BUF_ACT float [max_batch][ffn] last layer's SiLU(gate)*up. */
+enum mk_buffer { MK_BUF_HIDDEN = 0, MK_BUF_Q = 1, MK_BUF_ATTN = 2, MK_BUF_ACT = 3 };
+int mk_read_buffer(mk_ctx *ctx, int which, float *host_out, size_t count);
+
+/* Per-task trace of the last step (MK_FLAG_TRACE).  Records are
+ * mk_trace_rec [num_tasks], indexed by task id. */
+typedef struct mk_trace_rec {
+    unsigned long long t_ready;  /* globaltimer ns: scheduler saw the dependency fire */
+    unsigned long long t_start;  /* workers began the task body */
+    unsigned long long t_end;    /* workers finished and signalled */
+    int sm;                      /* CTA that ran it */
+    int kind;                    /* op kind (MK_OP_*) */
+    int layer;
+    int trig_event;
+} mk_trace_rec;
+enum mk_op_kind { MK_OP_QKV = 0, MK_OP_ATTN = 1, MK_OP_OPROJ = 2, MK_OP_GATEUP = 3,
+                  MK_OP_DOWN = 4, MK_OP_LMHEAD = 5 };
+int mk_get_trace(mk_ctx *ctx, mk_trace_rec *host_out, int n);
+
+/* Static task graph as built by mk_create (host copy).  task_out: int32
+ * [num_tasks][8] = {kind, layer, dep_event (-1 none), trig_event, begin,
+ * end, sm, slot}; queue_out: int32 [num_tasks] task ids grouped by SM in
+ * execution order; qoff_out: int32 [num_sms+1] offsets into queue_out. */
+int mk_get_graph(mk_ctx *ctx, int32_t *task_out, int32_t *queue_out, int32_t *qoff_out);
+
+/* Host-only planning (no GPU needed): build the task graph for `cfg` on a
+ * machine with `num_sms` SMs and return its sizes in *info (num_tasks,
+ * num_events, num_ops, attn_chunks, max_queue, page sizes), then fill the
+ * arrays as mk_get_graph does (any of them may be NULL) plus thresholds_out
+ * uint32 [num_events] and the per-task weight bytes bytes_out int64
+ * [num_tasks].  Used to test the graph builder without a device. */
+int mk_plan(const mk_config *cfg, int num_sms, mk_info *info,
+            int32_t *task_out, int32_t *queue_out, int32_t *qoff_out,
+            uint32_t *thresholds_out, int64_t *bytes_out);
+
+/* Test hook: overwrite the threshold of one event (simulates a graph
+ * whose event can never fire; the next step then ends in MK_ERR_TIMEOUT).
+ * Blocks the host. */
+int mk_debug_set_threshold(mk_ctx *ctx, int event, uint32_t threshold);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H */

@@ -1,0 +1,161 @@
+// mk_graph.cpp -- host-side builder of the static task graph.
+//
+// The graph follows the MPK task/event model described on the page
+// "显著提升小LLM的性能，所有kernel集成一个巨大kernel！" (Figure 2 / Figure 3 text):
+// every op is split into tasks, each task runs on one SM, has one dependent
+// event it waits for and one triggering event it bumps when done; an event
+// fires when its counter reaches its threshold (the number of tasks that
+// trigger it).  Tasks are placed in static per-SM queues (the Hazy page's
+// per-SM "execution plan"), ops in model order, so every queue is
+// dependency-ordered and the graph cannot deadlock.
+//
+// Placement balances weight bytes per SM across the whole step rather than
+// per op: each op's tiles go to the SMs that have streamed the fewest bytes
+// so far, so the per-SM loaders see equal totals.
+//
+// No heap allocation: the caller sizes the arrays with plan_sizes().
+#include "mk_internal.h"
+
+namespace mk {
+
+static constexpr int kMaxSms = 1024;
+
+int default_attn_chunks(int num_sms, int Bmax, int nkv, int S) {
+    int per = Bmax * nkv;
+    int nc = per > 0 ? num_sms / per : 1;
+    if (nc < 1) nc = 1;
+    int cap = (S + 15) / 16;            // at least ~16 positions per chunk at capacity
+    if (cap < 1) cap = 1;
+    if (nc > cap) nc = cap;
+    return nc;
+}
+
+PlanSizes plan_sizes(const Shape &s, int num_sms) {
+    OpTiles t = op_tiles(s);
+    auto ntask = [&](int tiles) { return tiles < num_sms ? tiles : num_sms; };
+    PlanSizes z;
+    int per_layer = ntask(t.qkv_pair + t.qkv_v) + t.attn_items + ntask(t.oproj) +
+                    ntask(t.gateup) + ntask(t.down);
+    z.num_tasks = s.L * per_layer + ntask(t.lmhead);
+    z.num_events = 5 * s.L + 1;
+    z.num_ops = 5 * s.L + 1;
+    return z;
+}
+
+namespace {
+
+struct Builder {
+    const Shape &s;
+    Plan &p;
+    int64_t load[kMaxSms];
+    int order[kMaxSms];
+    int nt = 0;
+
+    Builder(const Shape &s_, Plan &p_) : s(s_), p(p_) {
+        for (int i = 0; i < p.num_sms; ++i) load[i] = 0;
+    }
+
+    // SMs sorted by bytes assigned so far (ties: lower index first).
+    void sort_by_load() {
+        int n = p.num_sms;
+        for (int i = 0; i < n; ++i) order[i] = i;
+        for (int i = 1; i < n; ++i) {  // insertion sort, stable
+            int v = order[i];
+            int j = i - 1;
+            while (j >= 0 && load[order[j]] > load[v]) { order[j + 1] = order[j]; --j; }
+            order[j + 1] = v;
+        }
+    }
+
+    Task &add(int kind, int layer, int dep, int trig, int begin, int end, int sm, int slot,
+              int64_t bytes) {
+        Task &t = p.tasks[nt];
+        t.kind = kind; t.layer = layer; t.dep = dep; t.trig = trig;
+        t.begin = begin; t.end = end; t.sm = sm; t.slot = slot;
+        if (p.bytes) p.bytes[nt] = bytes;
+        load[sm] += bytes;
+        ++nt;
+        return t;
+    }
+
+    // Split `ntiles` tiles of `tile_bytes` (last tile `last_bytes`) over the
+    // least-loaded SMs, one contiguous tile range per task.  Returns the
+    // number of tasks.
+    int gemv_op(int kind, int layer, int dep, int trig, int ntiles, int64_t tile_bytes,
+                int64_t last_bytes) {
+        int T = ntiles < p.num_sms ? ntiles : p.num_sms;
+        int base = ntiles / T, extra = ntiles % T;
+        sort_by_load();
+        int tile = 0;
+        for (int i = 0; i < T; ++i) {
+            int n = base + (i < extra ? 1 : 0);
+            int64_t b = (int64_t)n * tile_bytes;
+            if (tile + n == ntiles) b += last_bytes - tile_bytes;
+            add(kind, layer, dep, trig, tile, tile + n, order[i], i, b);
+            tile += n;
+        }
+        return T;
+    }
+
+    int attn_op(int layer, int dep, int trig) {
+        OpTiles t = op_tiles(s);
+        int per_chunk = (s.S + s.NC - 1) / s.NC;
+        int64_t est = (int64_t)4 * s.d * per_chunk;   // K + V bf16 of one chunk at capacity
+        for (int i = 0; i < t.attn_items; ++i) {
+            int best = 0;   // least-loaded SM (lowest index on ties)
+            for (int k = 1; k < p.num_sms; ++k)
+                if (load[k] < load[best]) best = k;
+            add(OP_ATTN, layer, dep, trig, i, i + 1, best, i, est);
+        }
+        return t.attn_items;
+    }
+};
+
+}  // namespace
+
+void plan_build(const Shape &s, int num_sms, Plan &p) {
+    p.s = s;
+    p.num_sms = num_sms;
+    PlanSizes z = plan_sizes(s, num_sms);
+    p.num_events = z.num_events;
+    p.num_ops = z.num_ops;
+    Builder b(s, p);
+    OpTiles t = op_tiles(s);
+    const int64_t H2 = 2LL * s.H;
+    for (int l = 0; l < s.L; ++l) {
+        int e_qkv = 5 * l, e_attn = e_qkv + 1, e_o = e_qkv + 2, e_gu = e_qkv + 3, e_down = e_qkv + 4;
+        int dep_in = l == 0 ? -1 : e_qkv - 1;   // previous layer's down projection
+        p.thresholds[e_qkv] = b.gemv_op(OP_QKV, l, dep_in, e_qkv, t.qkv_pair + t.qkv_v,
+                                        8 * H2, 8 * H2);
+        p.thresholds[e_attn] = b.attn_op(l, e_qkv, e_attn);
+        p.thresholds[e_o] = b.gemv_op(OP_OPROJ, l, e_attn, e_o, t.oproj, 16LL * s.QD, 16LL * s.QD);
+        p.thresholds[e_gu] = b.gemv_op(OP_GATEUP, l, e_o, e_gu, t.gateup, 8 * H2, 8 * H2);
+        p.thresholds[e_down] = b.gemv_op(OP_DOWN, l, e_gu, e_down, t.down, 16LL * s.F, 16LL * s.F);
+    }
+    int e_lm = 5 * s.L;
+    int last_rows = s.V - 8 * (t.lmhead - 1);
+    p.thresholds[e_lm] = b.gemv_op(OP_LMHEAD, s.L, e_lm - 1, e_lm, t.lmhead, 8 * H2,
+                                   (int64_t)last_rows * H2);
+    p.num_lm_tasks = (int)p.thresholds[e_lm];
+    p.num_tasks = b.nt;
+
+    // group by SM, keeping op order inside each queue
+    for (int i = 0; i <= num_sms; ++i) p.qoff[i] = 0;
+    for (int i = 0; i < p.num_tasks; ++i) p.qoff[p.tasks[i].sm + 1]++;
+    for (int i = 0; i < num_sms; ++i) p.qoff[i + 1] += p.qoff[i];
+    int max_q = 0;
+    for (int i = 0; i < num_sms; ++i) {
+        int n = p.qoff[i + 1] - p.qoff[i];
+        if (n > max_q) max_q = n;
+    }
+    p.max_queue = max_q;
+    // stable fill: use the tail of qoff as a cursor by walking tasks in order
+    // (cursor per SM kept in `b.load`, reused as scratch)
+    for (int i = 0; i < num_sms; ++i) b.load[i] = p.qoff[i];
+    for (int i = 0; i < p.num_tasks; ++i) {
+        int sm = p.tasks[i].sm;
+        p.queue[b.load[sm]++] = i;
+    }
+}
+
+}  // namespace mk

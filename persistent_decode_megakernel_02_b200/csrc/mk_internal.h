@@ -1,0 +1,185 @@
+// mk_internal.h -- layout of the task graph and the kernel parameters,
+// shared by the host runtime (mk_runtime.cpp, mk_graph.cpp) and the
+// persistent kernel (mk_kernel.cu).  Not part of the public ABI.
+#pragma once
+
+#include <stdint.h>
+#include <stddef.h>
+#include <vector_types.h>   // float2
+
+#if defined(__CUDACC__)
+#define MK_HD __host__ __device__
+#else
+#define MK_HD
+#endif
+
+namespace mk {
+
+// ---- CTA shape ---------------------------------------------------------------
+constexpr int kWorkerWarps = 8;                     // run task bodies
+constexpr int kWorkerThreads = kWorkerWarps * 32;   // 256
+constexpr int kLoaderWarp = kWorkerWarps;           // streams weight pages
+constexpr int kSchedWarp = kWorkerWarps + 1;        // waits on events, activates tasks
+constexpr int kThreads = (kWorkerWarps + 2) * 32;   // 320
+
+// ---- tiling ------------------------------------------------------------------
+constexpr int kTileRows = 8;        // output rows per GEMV tile
+constexpr int kPageBytes = 32768;   // one shared-memory page
+constexpr int kNumPages = 6;        // pages in the per-SM ring
+constexpr int kVecMax = 8;          // 16-byte vectors per thread per row (K <= 8*8*256)
+constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 16384
+constexpr int kMaxGroup = 8;        // q heads per KV head handled by one attention task
+constexpr int kMaxHeadDim = 256;
+constexpr long long kL2Lookahead = 256 * 1024;  // bytes the L2 prefetch runs ahead of the ring
+
+// ---- ops ---------------------------------------------------------------------
+enum OpKind : int32_t { OP_QKV = 0, OP_ATTN = 1, OP_OPROJ = 2, OP_GATEUP = 3, OP_DOWN = 4, OP_LMHEAD = 5 };
+
+// One task: a contiguous range of tiles of one op (GEMV ops), or one
+// attention work item (b, kv head, chunk), assigned to one SM.
+struct Task {
+    int32_t kind;
+    int32_t layer;
+    int32_t dep;      // event waited on (-1: none)
+    int32_t trig;     // event bumped when done
+    int32_t begin;    // first tile (GEMV) / item index (ATTN)
+    int32_t end;      // one past the last tile / item
+    int32_t sm;       // CTA whose queue holds it
+    int32_t slot;     // index of the task within its op
+};
+static_assert(sizeof(Task) == 32, "Task is 8 int32");
+
+// Device pointers of one layer (bf16 as uint16_t on the host side).
+struct LayerW {
+    const uint16_t *wq, *wk, *wv, *wo, *wg, *wu, *wd;
+    const uint16_t *g_attn, *g_mlp;
+    uint16_t *kc, *vc;
+};
+
+// Sizes derived from the model shape.
+struct Shape {
+    int L, H, nq, nkv, d, F, V, S, Bmax, NC;
+    int G;            // nq / nkv
+    int QD, KD;       // nq*d, nkv*d
+    float theta, eps;
+};
+
+// Tile counts of each op (identical on host and device).
+struct OpTiles {
+    int qkv_pair;     // (nq + nkv) * d / 8 tiles of 4 RoPE pairs
+    int qkv_v;        // nkv * d / 8 tiles of 8 value rows
+    int oproj;        // H / 8
+    int gateup;       // F / 4 (4 gate rows + 4 up rows)
+    int down;         // H / 8
+    int lmhead;       // ceil(V / 8)
+    int attn_items;   // Bmax * nkv * NC
+};
+
+MK_HD inline OpTiles op_tiles(const Shape &s) {
+    OpTiles t;
+    t.qkv_pair = (s.nq + s.nkv) * s.d / 8;
+    t.qkv_v = s.nkv * s.d / 8;
+    t.oproj = s.H / 8;
+    t.gateup = s.F / 4;
+    t.down = s.H / 8;
+    t.lmhead = (s.V + 7) / 8;
+    t.attn_items = s.Bmax * s.nkv * s.NC;
+    return t;
+}
+
+// Reduction dimension (columns) of a GEMV op.
+MK_HD inline int op_k(const Shape &s, int kind) {
+    return kind == OP_OPROJ ? s.QD : (kind == OP_DOWN ? s.F : s.H);
+}
+
+// Rows of one tile held by one page: the largest power of two <= 8 whose
+// rows (K bf16 each) fit in a page.
+MK_HD inline int rows_per_page(int K) {
+    int r = kPageBytes / (2 * K);
+    int p = 1;
+    while (p * 2 <= r && p * 2 <= kTileRows) p *= 2;
+    return p;
+}
+
+// Attention positions per page (K block and V block of `n` positions).
+MK_HD inline int attn_pos_per_page(int d) { return kPageBytes / (4 * d); }
+
+// Device-side error word (mapped pinned host memory).
+struct ErrWord {
+    uint32_t code;    // MK_ERR_* (0 = none)
+    uint32_t task;    // task id where it happened (or 0xffffffff)
+    uint32_t where;   // which wait: 1 dep event, 2 ready, 3 page full, 4 page empty,
+                      // 5 worker barrier, 6 input check, 7 drain
+    uint32_t info;    // extra (event index, bad value)
+};
+
+struct TraceRec {
+    unsigned long long t_ready, t_start, t_end;
+    int32_t sm, kind, layer, trig;
+};
+static_assert(sizeof(TraceRec) == 40, "trace record layout");
+
+struct Params {
+    Shape s;
+    // graph
+    const Task *tasks;
+    const int32_t *queue;
+    const int32_t *qoff;         // [num_sms + 1]
+    const uint32_t *thresholds;  // [num_events]
+    uint32_t *events;            // [num_events]
+    uint32_t *merge_cnt;         // [L][Bmax][nkv]
+    uint32_t *lm_cnt;            // [1]
+    uint32_t *epoch;             // [1]: steps completed
+    uint32_t *done_cnt;          // [1]: CTAs that have read the epoch
+    uint32_t *abort_flag;        // [1]
+    int num_lm_tasks;
+    // model
+    const LayerW *layers;
+    const uint16_t *embed, *lm_head, *g_final;
+    const float2 *rope;          // [S][d/2] (cos, sin)
+    // step inputs / outputs
+    const int32_t *tokens, *positions;
+    int batch;
+    float *logits;               // may be null
+    int32_t *next_tok;
+    // scratch
+    float *x;                    // [Bmax][H] residual stream
+    float *q;                    // [Bmax][QD]
+    float *attn;                 // [Bmax][QD]
+    float *part;                 // [Bmax][nq][NC][d + 2]
+    float *act;                  // [Bmax][F]
+    float *amax_val;             // [Bmax][num_lm_tasks]
+    int32_t *amax_idx;           // [Bmax][num_lm_tasks]
+    // control
+    ErrWord *err;                // device view of mapped host memory
+    TraceRec *trace;             // null unless tracing
+    unsigned long long timeout_ns;
+    int l2_prefetch;
+};
+
+// ---- host planning -------------------------------------------------------------
+struct Plan {
+    Shape s;
+    int num_sms = 0;
+    int num_events = 0;
+    int num_ops = 0;
+    int max_queue = 0;
+    int num_lm_tasks = 0;
+    // tasks in op order; queue grouped by SM
+    Task *tasks = nullptr; int num_tasks = 0;
+    int32_t *queue = nullptr;
+    int32_t *qoff = nullptr;
+    uint32_t *thresholds = nullptr;
+    int64_t *bytes = nullptr;    // weight bytes per task (attention: estimate)
+};
+
+// Build the plan into caller-sized storage.  plan_sizes() returns the
+// element counts needed; plan_build() fills arrays of at least those sizes.
+struct PlanSizes { int num_tasks, num_events, num_ops; };
+PlanSizes plan_sizes(const Shape &s, int num_sms);
+void plan_build(const Shape &s, int num_sms, Plan &p);
+
+// Default number of attention chunks for a shape on `num_sms` SMs.
+int default_attn_chunks(int num_sms, int Bmax, int nkv, int S);
+
+}  // namespace mk

@@ -1,0 +1,1012 @@
+// mk_kernel.cu -- the persistent decode-step kernel for B200 (sm_100a).
+//
+// One CTA per SM, launched cooperatively so that every CTA is resident.
+// Each CTA owns a static queue of tasks (built on the host, see
+// mk_graph.cpp) and runs three roles in separate warps:
+//
+//  * loader warp (one thread): walks the queue ahead of the workers and,
+//    for every page of every upcoming task, waits for a free page of the
+//    shared-memory ring and issues 1-D bulk async copies (cp.async.bulk) of
+//    the task's weight rows (or KV-cache prefix) into it, completing on the
+//    page's mbarrier.  Weights do not depend on activations, so this runs
+//    ahead of the task dependencies (the Hazy page's "paged shared memory,
+//    next stage preloads its weights early").  It also issues
+//    cp.async.bulk.prefetch.L2 a bounded distance further ahead so HBM keeps
+//    streaming while the ring is full.
+//  * scheduler warp (one thread): for each queued task, spins (bounded) on
+//    the task's dependent event counter in global memory until it reaches
+//    threshold * epoch, then activates the task for the workers (MPK's
+//    event/threshold model, "显著提升小LLM的性能..." page, Figure 3 text).
+//  * worker warps (8): run the task bodies on CUDA cores and bump the
+//    task's triggering event with a release add when done.
+//
+// Task bodies (the fused instruction list of the Hazy megakernel page and
+// the per-layer *_layer calls of the MPK walkthrough, section 3.3.1):
+//   QKV    RMSNorm -> q/k/v GEMV rows -> RoPE -> q to scratch, k/v appended
+//          to the bf16 cache at the token's position
+//   ATTN   GQA decode attention over one chunk of positions of one KV head
+//          (split-K partial softmax); the last chunk to finish merges the
+//          partials of its KV head
+//   OPROJ  O-projection GEMV rows + residual
+//   GATEUP RMSNorm -> gate and up GEMV rows -> SiLU(gate) * up
+//   DOWN   down-projection GEMV rows + residual
+//   LMHEAD final RMSNorm -> LM-head GEMV rows -> per-task argmax; the last
+//          task to finish reduces the partial argmaxes to the next token
+//
+// Every wait is bounded by timeout_ns (globaltimer); on expiry the CTA
+// records MK_ERR_TIMEOUT in the error word, raises the abort flag that all
+// other waits poll, lets its in-flight bulk copies land, and returns.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "mk_internal.h"
+
+namespace mk {
+
+// status codes (same values as the public header's enum)
+constexpr uint32_t kErrInvalid = 1, kErrTimeout = 3;
+enum Where : uint32_t { W_DEP = 1, W_READY = 2, W_FULL = 3, W_EMPTY = 4, W_WBAR = 5,
+                        W_INPUT = 6, W_DRAIN = 7 };
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu(uint32_t *p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_add_acqrel_gpu(uint32_t *p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ uint32_t ld_acquire_cta_shared(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta_shared(uint32_t *p, uint32_t v) {
+    asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t *p) {
+    return *(const volatile uint32_t *)p;
+}
+__device__ __forceinline__ uint4 ld_shared_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_addr(p)));
+    return v;
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+__device__ __forceinline__ uint16_t f2bf(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+__device__ __forceinline__ float dot8(const uint4 w, const float *x) {
+    float a = bf_lo(w.x) * x[0];
+    a = fmaf(bf_hi(w.x), x[1], a);
+    a = fmaf(bf_lo(w.y), x[2], a);
+    a = fmaf(bf_hi(w.y), x[3], a);
+    a = fmaf(bf_lo(w.z), x[4], a);
+    a = fmaf(bf_hi(w.z), x[5], a);
+    a = fmaf(bf_lo(w.w), x[6], a);
+    a = fmaf(bf_hi(w.w), x[7], a);
+    return a;
+}
+
+// ---------------------------------------------------------------------------
+// shared memory
+// ---------------------------------------------------------------------------
+constexpr int kAttnCombine = 512;   // G * head_dim handled by the warp combine
+
+struct __align__(16) SmemCtl {
+    uint64_t full[kNumPages];
+    uint64_t empty[kNumPages];
+    uint64_t wbar;              // worker barrier, one arrival per worker warp
+    uint32_t ready_upto;        // tasks of this queue activated by the scheduler
+    uint32_t abort;             // this CTA is bailing out
+    uint32_t ep;                // epoch of this launch (steps completed + 1)
+    uint32_t last_flag;         // broadcast of "this task arrived last"
+    float red[2][kWorkerWarps][kTileRows];
+    float scal[kWorkerWarps];
+    float att_m[kWorkerWarps][kMaxGroup];
+    float att_l[kWorkerWarps][kMaxGroup];
+    float att_o[kWorkerWarps][kAttnCombine];
+};
+constexpr size_t kSmemBytes = (size_t)kNumPages * kPageBytes + sizeof(SmemCtl);
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+// ---------------------------------------------------------------------------
+// bounded waiting
+// ---------------------------------------------------------------------------
+struct Spin {
+    unsigned long long t0 = 0;
+    uint32_t n = 0;
+};
+
+// Record the first device error (later ones are dropped) and raise both
+// abort flags.
+__device__ void raise_error(const Params &p, SmemCtl *ctl, uint32_t code, uint32_t where,
+                            uint32_t task, uint32_t info) {
+    if (atomicCAS(&p.err->code, 0u, code) == 0u) {
+        p.err->task = task;
+        p.err->where = where;
+        p.err->info = info;
+    }
+    *(volatile uint32_t *)&ctl->abort = 1;
+    atomicExch(p.abort_flag, 1u);
+    __threadfence();
+}
+
+// Returns false when the wait must be abandoned: this CTA or another one
+// aborted, or the wait exceeded the time budget (then the error is raised).
+__device__ __forceinline__ bool spin_ok(Spin &s, const Params &p, SmemCtl *ctl, uint32_t where,
+                                        uint32_t task, uint32_t info) {
+    if ((++s.n & 127u) != 0u) return true;
+    if (*(volatile uint32_t *)&ctl->abort) return false;
+    if (ld_volatile_u32(p.abort_flag)) {
+        *(volatile uint32_t *)&ctl->abort = 1;
+        return false;
+    }
+    unsigned long long now = globaltimer();
+    if (s.t0 == 0) {
+        s.t0 = now;
+        return true;
+    }
+    if (now - s.t0 > p.timeout_ns) {
+        raise_error(p, ctl, kErrTimeout, where, task, info);
+        return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ bool wait_mbar(uint64_t *bar, uint32_t parity, const Params &p,
+                                          SmemCtl *ctl, uint32_t where, uint32_t task) {
+    Spin s;
+    while (!mbar_try_wait(bar, parity))
+        if (!spin_ok(s, p, ctl, where, task, parity)) return false;
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// task geometry shared by the loader and the workers
+// ---------------------------------------------------------------------------
+struct Seg {
+    const void *src;
+    uint32_t dst;     // byte offset in the page
+    uint32_t bytes;
+};
+struct PageDesc {
+    Seg seg[kTileRows];
+    int nseg;
+    uint32_t bytes;
+};
+
+// Attention chunk of one work item.
+struct AttnChunk {
+    int b, kvh, c;
+    bool active;      // sequence b takes part in this step
+    int P;            // position of the new token
+    int c0, c1;       // positions [c0, c1) of this chunk (c1 <= P + 1)
+    int npre;         // cached positions loaded by pages: [c0, c0 + npre), all < P
+    bool has_new;     // P is in [c0, c1)
+};
+
+__device__ __forceinline__ AttnChunk attn_chunk(const Params &p, int item) {
+    const Shape &s = p.s;
+    AttnChunk a;
+    a.b = item / (s.nkv * s.NC);
+    a.kvh = (item / s.NC) % s.nkv;
+    a.c = item % s.NC;
+    a.active = a.b < p.batch;
+    a.P = 0; a.c0 = 0; a.c1 = 0; a.npre = 0; a.has_new = false;
+    if (a.active) {
+        a.P = p.positions[a.b];
+        int C = a.P + 1;
+        int Lc = (C + s.NC - 1) / s.NC;
+        a.c0 = a.c * Lc;
+        a.c1 = min(a.c0 + Lc, C);
+        if (a.c0 >= C) { a.c0 = C; a.c1 = C; }
+        int pend = min(a.c1, a.P);
+        a.npre = max(0, pend - a.c0);
+        a.has_new = a.c0 <= a.P && a.P < a.c1;
+    }
+    return a;
+}
+
+__device__ __forceinline__ int task_pages(const Params &p, const Task &t) {
+    if (t.kind == OP_ATTN) {
+        AttnChunk a = attn_chunk(p, t.begin);
+        int npp = attn_pos_per_page(p.s.d);
+        return (a.npre + npp - 1) / npp;
+    }
+    int K = op_k(p.s, t.kind);
+    return (t.end - t.begin) * (kTileRows / rows_per_page(K));
+}
+
+// Source row r (0..7) of GEMV tile `tile`, or null when the row is past
+// the end of the matrix (ragged LM-head tile).
+__device__ __forceinline__ const uint16_t *gemv_row(const Params &p, int kind, int layer, int tile,
+                                                    int r) {
+    const Shape &s = p.s;
+    const size_t H = (size_t)s.H;
+    if (kind == OP_LMHEAD) {
+        int row = tile * 8 + r;
+        return row < s.V ? p.lm_head + (size_t)row * H : nullptr;
+    }
+    const LayerW &L = p.layers[layer];
+    switch (kind) {
+    case OP_QKV: {
+        int npair = (s.nq + s.nkv) * s.d / 8;
+        if (tile < npair) {
+            int per_head = s.d / 8;
+            int head = tile / per_head;
+            int j4 = (tile % per_head) * 4;
+            const uint16_t *base = head < s.nq ? L.wq + (size_t)head * s.d * H
+                                               : L.wk + (size_t)(head - s.nq) * s.d * H;
+            int row = r < 4 ? j4 + r : s.d / 2 + j4 + (r - 4);
+            return base + (size_t)row * H;
+        }
+        return L.wv + (size_t)((tile - npair) * 8 + r) * H;
+    }
+    case OP_OPROJ: return L.wo + (size_t)(tile * 8 + r) * (size_t)s.QD;
+    case OP_GATEUP:
+        return r < 4 ? L.wg + (size_t)(tile * 4 + r) * H : L.wu + (size_t)(tile * 4 + r - 4) * H;
+    default: /* OP_DOWN */ return L.wd + (size_t)(tile * 8 + r) * (size_t)s.F;
+    }
+}
+
+__device__ void page_desc(const Params &p, const Task &t, int pidx, PageDesc &pd) {
+    const Shape &s = p.s;
+    pd.nseg = 0;
+    pd.bytes = 0;
+    if (t.kind == OP_ATTN) {
+        AttnChunk a = attn_chunk(p, t.begin);
+        const LayerW &L = p.layers[t.layer];
+        int npp = attn_pos_per_page(s.d);
+        int pos0 = a.c0 + pidx * npp;
+        int n = min(npp, a.npre - pidx * npp);
+        size_t off = (((size_t)a.b * s.nkv + a.kvh) * s.S + pos0) * s.d;
+        uint32_t bytes = (uint32_t)n * s.d * 2;
+        pd.seg[0] = Seg{L.kc + off, 0u, bytes};
+        pd.seg[1] = Seg{L.vc + off, (uint32_t)(npp * s.d * 2), bytes};
+        pd.nseg = 2;
+        pd.bytes = 2 * bytes;
+        return;
+    }
+    const int K = op_k(s, t.kind);
+    const int rpp = rows_per_page(K);
+    const int ppt = kTileRows / rpp;
+    const int tile = t.begin + pidx / ppt;
+    const int r0 = (pidx % ppt) * rpp;
+    const uint32_t row_bytes = (uint32_t)K * 2u;
+    const char *run_end = nullptr;
+    for (int i = 0; i < rpp; ++i) {
+        const uint16_t *src = gemv_row(p, t.kind, t.layer, tile, r0 + i);
+        if (!src) break;
+        if ((const char *)src == run_end && pd.nseg > 0) {
+            pd.seg[pd.nseg - 1].bytes += row_bytes;
+        } else {
+            pd.seg[pd.nseg++] = Seg{src, (uint32_t)i * row_bytes, row_bytes};
+        }
+        run_end = (const char *)src + row_bytes;
+        pd.bytes += row_bytes;
+    }
+}
+
+// Iterates (task, page) over one SM's queue in execution order.
+struct PageCursor {
+    int qi, q1, pidx, npages;
+    Task t;
+    __device__ PageCursor(int q0, int q1_) : qi(q0 - 1), q1(q1_), pidx(0), npages(0) {}
+    __device__ bool next(const Params &p, PageDesc &pd) {
+        while (pidx >= npages) {
+            if (++qi >= q1) return false;
+            t = p.tasks[p.queue[qi]];
+            npages = task_pages(p, t);
+            pidx = 0;
+        }
+        page_desc(p, t, pidx++, pd);
+        return true;
+    }
+};
+
+// ---------------------------------------------------------------------------
+// loader role (one thread)
+// ---------------------------------------------------------------------------
+__device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
+    const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
+    PageCursor fill(q0, q1), pf(q0, q1);
+    PageDesc pd, pp;
+    uint32_t seq = 0;
+    long long fill_bytes = 0, pf_bytes = 0;
+    bool pf_more = p.l2_prefetch != 0;
+    bool ok = true;
+    while (fill.next(p, pd)) {
+        // keep HBM busy beyond the ring: prefetch later pages into L2
+        while (pf_more && pf_bytes < fill_bytes + kL2Lookahead) {
+            if (!pf.next(p, pp)) { pf_more = false; break; }
+            if (pf_bytes >= fill_bytes) {
+                for (int i = 0; i < pp.nseg; ++i) prefetch_l2(pp.seg[i].src, pp.seg[i].bytes);
+            }
+            pf_bytes += pp.bytes;
+        }
+        const uint32_t slot = seq % kNumPages;
+        const uint32_t par = ((seq / kNumPages) & 1u) ^ 1u;
+        if (!wait_mbar(&ctl->empty[slot], par, p, ctl, W_EMPTY, (uint32_t)p.queue[fill.qi])) {
+            ok = false;
+            break;
+        }
+        mbar_arrive_expect_tx(&ctl->full[slot], pd.bytes);
+        unsigned char *dst = pages + (size_t)slot * kPageBytes;
+        for (int i = 0; i < pd.nseg; ++i) bulk_g2s(dst + pd.seg[i].dst, pd.seg[i].src, pd.seg[i].bytes, &ctl->full[slot]);
+        fill_bytes += pd.bytes;
+        ++seq;
+    }
+    (void)ok;
+    {
+        // let every copy already issued land before this thread returns, so
+        // no bulk copy can still be writing shared memory when the CTA exits
+        uint32_t first = seq > (uint32_t)kNumPages ? seq - kNumPages : 0u;
+        for (uint32_t k = first; k < seq; ++k) {
+            Spin s;
+            while (!mbar_try_wait(&ctl->full[k % kNumPages], (k / kNumPages) & 1u)) {
+                if ((++s.n & 127u) == 0u) {
+                    unsigned long long now = globaltimer();
+                    if (s.t0 == 0) s.t0 = now;
+                    else if (now - s.t0 > p.timeout_ns) break;
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// scheduler role (one thread)
+// ---------------------------------------------------------------------------
+__device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
+    const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
+    for (int qi = q0; qi < q1; ++qi) {
+        const int id = p.queue[qi];
+        const int dep = p.tasks[id].dep;
+        if (dep >= 0) {
+            const uint32_t target = p.thresholds[dep] * ep;
+            Spin s;
+            while ((int32_t)(ld_acquire_gpu(&p.events[dep]) - target) < 0)
+                if (!spin_ok(s, p, ctl, W_DEP, (uint32_t)id, (uint32_t)dep)) return;
+        }
+        if (p.trace) p.trace[id].t_ready = globaltimer();
+        st_release_cta_shared(&ctl->ready_upto, (uint32_t)(qi - q0 + 1));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// worker helpers
+// ---------------------------------------------------------------------------
+struct WState {
+    uint32_t page_seq = 0;   // pages consumed
+    uint32_t wphase = 0;     // worker-barrier phase
+    int red_buf = 0;
+    int task_id = 0;
+};
+
+// All worker warps meet; bounded.
+__device__ __forceinline__ bool worker_sync(const Params &p, SmemCtl *ctl, WState &w) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&ctl->wbar);
+    bool ok = wait_mbar(&ctl->wbar, w.wphase, p, ctl, W_WBAR, (uint32_t)w.task_id);
+    w.wphase ^= 1u;
+    return ok;
+}
+
+__device__ __forceinline__ bool wait_page(const Params &p, SmemCtl *ctl, WState &w, uint32_t &slot) {
+    slot = w.page_seq % kNumPages;
+    return wait_mbar(&ctl->full[slot], (w.page_seq / kNumPages) & 1u, p, ctl, W_FULL,
+                     (uint32_t)w.task_id);
+}
+
+__device__ __forceinline__ void release_page(SmemCtl *ctl, WState &w, uint32_t slot) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&ctl->empty[slot]);
+    ++w.page_seq;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Reduce acc[8] over the 32 lanes; afterwards every lane holds the warp
+// total of row (lane >> 2) & 7.
+__device__ __forceinline__ float warp_reduce_rows8(const float (&acc)[8], int lane) {
+    float b0[4], b1[2];
+    const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float send = u16 ? acc[i] : acc[i + 4];
+        float keep = u16 ? acc[i + 4] : acc[i];
+        b0[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        float send = u8 ? b0[i] : b0[i + 2];
+        float keep = u8 ? b0[i + 2] : b0[i];
+        b1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float send = u4 ? b1[0] : b1[1];
+    float keep = u4 ? b1[1] : b1[0];
+    float c = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    c += __shfl_xor_sync(0xffffffffu, c, 2);
+    c += __shfl_xor_sync(0xffffffffu, c, 1);
+    return c;
+}
+
+// Sum of one float over the 256 worker threads (bounded barrier inside).
+__device__ __forceinline__ bool worker_block_sum(const Params &p, SmemCtl *ctl, WState &w, float v,
+                                                 float &out) {
+    v = warp_sum(v);
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) ctl->scal[warp] = v;
+    if (!worker_sync(p, ctl, w)) return false;
+    float t = 0.f;
+#pragma unroll
+    for (int i = 0; i < kWorkerWarps; ++i) t += ctl->scal[i];
+    out = t;
+    return true;
+}
+
+// Signal the task's triggering event after every worker's writes.
+__device__ __forceinline__ void signal_event(const Params &p, const Task &t) {
+    __threadfence();
+    red_release_gpu(&p.events[t.trig], 1u);
+}
+
+// ---------------------------------------------------------------------------
+// GEMV task body: tiles of 8 rows x K, NV 16-byte vectors per thread per row
+// ---------------------------------------------------------------------------
+template <int NV>
+__device__ bool gemv_task(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
+                          WState &w) {
+    const Shape &s = p.s;
+    const int kind = t.kind, layer = t.layer;
+    const int K = op_k(s, kind);
+    const int K8 = K >> 3;
+    const int rpp = rows_per_page(K);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = 0;
+
+    // ---- the task's input vector slice, normalised if the op has a norm
+    const float *src = nullptr;
+    const uint16_t *src_bf = nullptr;
+    const uint16_t *gain = nullptr;
+    switch (kind) {
+    case OP_QKV:
+        if (layer == 0) src_bf = p.embed + (size_t)p.tokens[b] * s.H;
+        else src = p.x + (size_t)b * s.H;
+        gain = p.layers[layer].g_attn;
+        break;
+    case OP_GATEUP: src = p.x + (size_t)b * s.H; gain = p.layers[layer].g_mlp; break;
+    case OP_LMHEAD: src = p.x + (size_t)b * s.H; gain = p.g_final; break;
+    case OP_OPROJ: src = p.attn + (size_t)b * s.QD; break;
+    default: src = p.act + (size_t)b * s.F; break;
+    }
+    float xr[NV][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        const int v = tid + j * kWorkerThreads;
+        if (v < K8) {
+            if (src_bf) {
+                uint4 e = __ldg(reinterpret_cast<const uint4 *>(src_bf) + v);
+                xr[j][0] = bf_lo(e.x); xr[j][1] = bf_hi(e.x); xr[j][2] = bf_lo(e.y); xr[j][3] = bf_hi(e.y);
+                xr[j][4] = bf_lo(e.z); xr[j][5] = bf_hi(e.z); xr[j][6] = bf_lo(e.w); xr[j][7] = bf_hi(e.w);
+            } else {
+                float4 a0 = __ldcg(reinterpret_cast<const float4 *>(src) + 2 * v);
+                float4 a1 = __ldcg(reinterpret_cast<const float4 *>(src) + 2 * v + 1);
+                xr[j][0] = a0.x; xr[j][1] = a0.y; xr[j][2] = a0.z; xr[j][3] = a0.w;
+                xr[j][4] = a1.x; xr[j][5] = a1.y; xr[j][6] = a1.z; xr[j][7] = a1.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
+        }
+    }
+    if (gain) {
+        float tot;
+        if (!worker_block_sum(p, ctl, w, ss, tot)) return false;
+        const float sc = 1.0f / sqrtf(tot / (float)s.H + s.eps);
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int v = tid + j * kWorkerThreads;
+            if (v < K8) {
+                uint4 g = __ldg(reinterpret_cast<const uint4 *>(gain) + v);
+                xr[j][0] *= sc * bf_lo(g.x); xr[j][1] *= sc * bf_hi(g.x);
+                xr[j][2] *= sc * bf_lo(g.y); xr[j][3] *= sc * bf_hi(g.y);
+                xr[j][4] *= sc * bf_lo(g.z); xr[j][5] *= sc * bf_hi(g.z);
+                xr[j][6] *= sc * bf_lo(g.w); xr[j][7] *= sc * bf_hi(g.w);
+            }
+        }
+    }
+
+    // ---- tiles
+    const int P = p.positions[b];
+    float best_v = -INFINITY;
+    int best_i = 0;
+    const size_t row_bytes = (size_t)K * 2;
+    for (int tile = t.begin; tile < t.end; ++tile) {
+        float acc[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+        uint32_t slot = 0;
+        const unsigned char *page = pages;
+#pragma unroll
+        for (int r = 0; r < kTileRows; ++r) {
+            if ((r & (rpp - 1)) == 0) {
+                if (!wait_page(p, ctl, w, slot)) return false;
+                page = pages + (size_t)slot * kPageBytes;
+            }
+            const unsigned char *row = page + (size_t)(r & (rpp - 1)) * row_bytes;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                const int v = tid + j * kWorkerThreads;
+                if (v < K8) acc[r] += dot8(ld_shared_v4(row + (size_t)v * 16), xr[j]);
+            }
+            if (((r + 1) & (rpp - 1)) == 0) release_page(ctl, w, slot);
+        }
+        const float rsum = warp_reduce_rows8(acc, lane);
+        if ((lane & 3) == 0) ctl->red[w.red_buf][warp][(lane >> 2) & 7] = rsum;
+        if (!worker_sync(p, ctl, w)) return false;
+        if (tid < 8) {
+            const float(*red)[kTileRows] = ctl->red[w.red_buf];
+            auto rs = [&](int r) {
+                float a = 0.f;
+#pragma unroll
+                for (int i = 0; i < kWorkerWarps; ++i) a += red[i][r];
+                return a;
+            };
+            switch (kind) {
+            case OP_QKV: {
+                const int npair = (s.nq + s.nkv) * s.d / 8;
+                if (tile < npair) {
+                    if (tid < 4) {
+                        const int per_head = s.d / 8;
+                        const int head = tile / per_head;
+                        const int i = (tile % per_head) * 4 + tid;
+                        const float a = rs(tid), c = rs(tid + 4);
+                        const float2 cs = p.rope[(size_t)P * (s.d / 2) + i];
+                        const float ra = a * cs.x - c * cs.y;
+                        const float rc = c * cs.x + a * cs.y;
+                        if (head < s.nq) {
+                            float *qh = p.q + (size_t)b * s.QD + (size_t)head * s.d;
+                            qh[i] = ra;
+                            qh[i + s.d / 2] = rc;
+                        } else {
+                            const LayerW &L = p.layers[layer];
+                            uint16_t *kh = L.kc + (((size_t)b * s.nkv + (head - s.nq)) * s.S + P) * s.d;
+                            kh[i] = f2bf(ra);
+                            kh[i + s.d / 2] = f2bf(rc);
+                        }
+                    }
+                } else {
+                    const int row = (tile - npair) * 8 + tid;
+                    const int kvh = row / s.d, dd = row % s.d;
+                    const LayerW &L = p.layers[layer];
+                    L.vc[(((size_t)b * s.nkv + kvh) * s.S + P) * s.d + dd] = f2bf(rs(tid));
+                }
+                break;
+            }
+            case OP_OPROJ: {
+                const int row = tile * 8 + tid;
+                float *xp = p.x + (size_t)b * s.H + row;
+                const float resid = layer == 0 ? bf2f(p.embed[(size_t)p.tokens[b] * s.H + row]) : __ldcg(xp);
+                *xp = resid + rs(tid);
+                break;
+            }
+            case OP_GATEUP:
+                if (tid < 4) {
+                    const float g = rs(tid), u = rs(tid + 4);
+                    p.act[(size_t)b * s.F + tile * 4 + tid] = g / (1.0f + expf(-g)) * u;
+                }
+                break;
+            case OP_DOWN: {
+                const int row = tile * 8 + tid;
+                float *xp = p.x + (size_t)b * s.H + row;
+                *xp = __ldcg(xp) + rs(tid);
+                break;
+            }
+            default: {  // OP_LMHEAD
+                const int row = tile * 8 + tid;
+                float val = -INFINITY;
+                if (row < s.V) {
+                    val = rs(tid);
+                    if (p.logits) p.logits[(size_t)b * s.V + row] = val;
+                }
+                int idx = row;
+#pragma unroll
+                for (int o = 4; o > 0; o >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffu, val, o);
+                    const int oi = __shfl_xor_sync(0xffu, idx, o);
+                    if (ov > val || (ov == val && oi < idx)) { val = ov; idx = oi; }
+                }
+                if (tid == 0 && (val > best_v || (val == best_v && idx < best_i))) {
+                    best_v = val;
+                    best_i = idx;
+                }
+                break;
+            }
+            }
+        }
+        w.red_buf ^= 1;
+    }
+    if (kind == OP_LMHEAD && tid == 0) {
+        p.amax_val[(size_t)b * p.num_lm_tasks + t.slot] = best_v;
+        p.amax_idx[(size_t)b * p.num_lm_tasks + t.slot] = best_i;
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// attention task body: one chunk of positions of one KV head, G q heads
+// ---------------------------------------------------------------------------
+template <int G, int DPL>   // q heads per KV head, head dims per lane (d = 32 * DPL)
+__device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
+                          WState &w) {
+    const Shape &s = p.s;
+    constexpr int d = 32 * DPL;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const AttnChunk a = attn_chunk(p, t.begin);
+    const int npp = attn_pos_per_page(d);
+    const int npages = (a.npre + npp - 1) / npp;
+
+    float m[G], l[G], o[G][DPL], qr[G][DPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        m[g] = -INFINITY;
+        l[g] = 0.f;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) { o[g][i] = 0.f; qr[g][i] = 0.f; }
+    }
+    if (a.active) {
+        const float scale = 1.0f / sqrtf((float)d);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float *qh = p.q + (size_t)a.b * s.QD + (size_t)(a.kvh * G + g) * d + lane * DPL;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) qr[g][i] = __ldcg(qh + i) * scale;
+        }
+    }
+
+    auto visit = [&](const uint16_t *krow, const uint16_t *vrow, bool global_mem) {
+        float kv[DPL], vv[DPL];
+#pragma unroll
+        for (int i = 0; i < DPL; i += 2) {
+            uint32_t kw, vw;
+            if (global_mem) {
+                kw = __ldcg(reinterpret_cast<const unsigned int *>(krow + lane * DPL + i));
+                vw = __ldcg(reinterpret_cast<const unsigned int *>(vrow + lane * DPL + i));
+            } else {
+                kw = *reinterpret_cast<const uint32_t *>(krow + lane * DPL + i);
+                vw = *reinterpret_cast<const uint32_t *>(vrow + lane * DPL + i);
+            }
+            kv[i] = bf_lo(kw); kv[i + 1] = bf_hi(kw);
+            vv[i] = bf_lo(vw); vv[i + 1] = bf_hi(vw);
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float sc = 0.f;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) sc = fmaf(qr[g][i], kv[i], sc);
+            sc = warp_sum(sc);
+            const float mn = fmaxf(m[g], sc);
+            const float corr = expf(m[g] - mn);
+            const float pe = expf(sc - mn);
+            l[g] = l[g] * corr + pe;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) o[g][i] = fmaf(o[g][i], corr, pe * vv[i]);
+            m[g] = mn;
+        }
+    };
+
+    for (int pg = 0; pg < npages; ++pg) {
+        uint32_t slot;
+        if (!wait_page(p, ctl, w, slot)) return false;
+        const uint16_t *Kp = reinterpret_cast<const uint16_t *>(pages + (size_t)slot * kPageBytes);
+        const uint16_t *Vp = Kp + (size_t)npp * d;
+        const int n = min(npp, a.npre - pg * npp);
+        for (int j = warp; j < n; j += kWorkerWarps) visit(Kp + (size_t)j * d, Vp + (size_t)j * d, false);
+        release_page(ctl, w, slot);
+    }
+    if (a.has_new && warp == (a.npre % kWorkerWarps)) {
+        const LayerW &L = p.layers[t.layer];
+        const size_t off = (((size_t)a.b * s.nkv + a.kvh) * s.S + a.P) * d;
+        visit(L.kc + off, L.vc + off, true);
+    }
+
+    // ---- combine the warps' running states into this chunk's partial
+    if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) { ctl->att_m[warp][g] = m[g]; ctl->att_l[warp][g] = l[g]; }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) ctl->att_o[warp][g * d + lane * DPL + i] = o[g][i];
+    if (!worker_sync(p, ctl, w)) return false;
+    if (a.active) {
+        for (int e = tid; e < G * d; e += kWorkerThreads) {
+            const int g = e / d, i = e % d;
+            float M = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < kWorkerWarps; ++k) M = fmaxf(M, ctl->att_m[k][g]);
+            float O = 0.f, Lsum = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int k = 0; k < kWorkerWarps; ++k) {
+                    const float f = expf(ctl->att_m[k][g] - M);
+                    O = fmaf(f, ctl->att_o[k][e], O);
+                    Lsum = fmaf(f, ctl->att_l[k][g], Lsum);
+                }
+            }
+            float *dst = p.part + (((size_t)a.b * s.nq + a.kvh * G + g) * s.NC + a.c) * (d + 2);
+            dst[i] = O;
+            if (i == 0) { dst[d] = M; dst[d + 1] = Lsum; }
+        }
+    }
+    // every partial of this task is written
+    if (!worker_sync(p, ctl, w)) return false;
+    if (tid == 0) {
+        __threadfence();
+        uint32_t *cnt = p.merge_cnt + ((size_t)t.layer * s.Bmax + a.b) * s.nkv + a.kvh;
+        const uint32_t old = atom_add_acqrel_gpu(cnt, 1u);
+        const uint32_t last = (old + 1u == (uint32_t)s.NC * ctl->ep) ? 1u : 0u;
+        ctl->last_flag = last;
+        if (!last) red_release_gpu(&p.events[t.trig], 1u);
+    }
+    if (!worker_sync(p, ctl, w)) return false;
+    if (ctl->last_flag) {
+        __threadfence();
+        if (a.active) {
+            for (int e = tid; e < G * d; e += kWorkerThreads) {
+                const int g = e / d, i = e % d;
+                const int hq = a.kvh * G + g;
+                const float *base = p.part + ((size_t)a.b * s.nq + hq) * s.NC * (d + 2);
+                float M = -INFINITY;
+                for (int c = 0; c < s.NC; ++c) M = fmaxf(M, __ldcg(base + (size_t)c * (d + 2) + d));
+                float num = 0.f, den = 0.f;
+                for (int c = 0; c < s.NC; ++c) {
+                    const float *pc = base + (size_t)c * (d + 2);
+                    const float mc = __ldcg(pc + d);
+                    if (mc == -INFINITY) continue;
+                    const float f = expf(mc - M);
+                    num = fmaf(f, __ldcg(pc + i), num);
+                    den = fmaf(f, __ldcg(pc + d + 1), den);
+                }
+                p.attn[(size_t)a.b * s.QD + (size_t)hq * d + i] = num / den;
+            }
+        }
+        if (!worker_sync(p, ctl, w)) return false;
+        if (tid == 0) signal_event(p, t);
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// worker role
+// ---------------------------------------------------------------------------
+template <int G>
+__device__ bool attn_dispatch_d(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
+                                WState &w) {
+    if (p.s.d == 64) return attn_task<G, 2>(p, t, pages, ctl, w);
+    return attn_task<G, 4>(p, t, pages, ctl, w);
+}
+
+__device__ bool run_task(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
+                         WState &w) {
+    if (t.kind == OP_ATTN) {
+        switch (p.s.G) {
+        case 1: return attn_dispatch_d<1>(p, t, pages, ctl, w);
+        case 2: return attn_dispatch_d<2>(p, t, pages, ctl, w);
+        case 4: return attn_dispatch_d<4>(p, t, pages, ctl, w);
+        default: return attn_dispatch_d<8>(p, t, pages, ctl, w);
+        }
+    }
+    const int K = op_k(p.s, t.kind);
+    const int nv = (K / 8 + kWorkerThreads - 1) / kWorkerThreads;
+    switch (nv) {
+    case 1: return gemv_task<1>(p, t, pages, ctl, w);
+    case 2: return gemv_task<2>(p, t, pages, ctl, w);
+    case 3: return gemv_task<3>(p, t, pages, ctl, w);
+    case 4: return gemv_task<4>(p, t, pages, ctl, w);
+    case 5: return gemv_task<5>(p, t, pages, ctl, w);
+    case 6: return gemv_task<6>(p, t, pages, ctl, w);
+    case 7: return gemv_task<7>(p, t, pages, ctl, w);
+    default: return gemv_task<8>(p, t, pages, ctl, w);
+    }
+}
+
+__device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
+    const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
+    const int tid = threadIdx.x;
+    WState w;
+    for (int qi = q0; qi < q1; ++qi) {
+        const int id = p.queue[qi];
+        const Task t = p.tasks[id];
+        w.task_id = id;
+        {
+            Spin s;
+            const uint32_t need = (uint32_t)(qi - q0 + 1);
+            while (ld_acquire_cta_shared(&ctl->ready_upto) < need)
+                if (!spin_ok(s, p, ctl, W_READY, (uint32_t)id, 0u)) return;
+        }
+        if (p.trace && tid == 0) p.trace[id].t_start = globaltimer();
+        if (!run_task(p, t, pages, ctl, w)) return;
+        if (t.kind != OP_ATTN) {
+            // every output of the task is written (tile epilogues by threads < 8)
+            if (!worker_sync(p, ctl, w)) return;
+            if (t.kind == OP_LMHEAD) {
+                if (tid == 0) {
+                    __threadfence();
+                    const uint32_t old = atom_add_acqrel_gpu(p.lm_cnt, 1u);
+                    const uint32_t last = (old + 1u == (uint32_t)p.num_lm_tasks * ctl->ep) ? 1u : 0u;
+                    ctl->last_flag = last;
+                }
+                if (!worker_sync(p, ctl, w)) return;
+                if (ctl->last_flag && tid < 32) {
+                    __threadfence();
+                    for (int b = 0; b < p.batch; ++b) {
+                        float bv = -INFINITY;
+                        int bi = 0x7fffffff;
+                        for (int k = tid; k < p.num_lm_tasks; k += 32) {
+                            const float v = __ldcg(p.amax_val + (size_t)b * p.num_lm_tasks + k);
+                            const int i = __ldcg(p.amax_idx + (size_t)b * p.num_lm_tasks + k);
+                            if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+                        }
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) {
+                            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+                        }
+                        if (tid == 0) p.next_tok[b] = bi;
+                    }
+                }
+            }
+            if (tid == 0) signal_event(p, t);
+        }
+        if (p.trace && tid == 0) p.trace[id].t_end = globaltimer();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_constant__ Params p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    unsigned char *pages = smem;
+    SmemCtl *ctl = reinterpret_cast<SmemCtl *>(smem + (size_t)kNumPages * kPageBytes);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        for (int i = 0; i < kNumPages; ++i) {
+            mbar_init(&ctl->full[i], 1);
+            mbar_init(&ctl->empty[i], kWorkerWarps);
+        }
+        mbar_init(&ctl->wbar, kWorkerWarps);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        ctl->ready_upto = 0;
+        ctl->last_flag = 0;
+        ctl->ep = ld_volatile_u32(p.epoch) + 1u;
+        uint32_t stop = ld_volatile_u32(p.abort_flag) ? 1u : 0u;
+        for (int b = 0; b < p.batch && !stop; ++b) {
+            const int tok = p.tokens[b], pos = p.positions[b];
+            if (tok < 0 || tok >= p.s.V || pos < 0 || pos >= p.s.S) {
+                if (atomicCAS(&p.err->code, 0u, kErrInvalid) == 0u) {
+                    p.err->task = 0xffffffffu;
+                    p.err->where = W_INPUT;
+                    p.err->info = (uint32_t)b;
+                }
+                stop = 1u;
+            }
+        }
+        ctl->abort = stop;
+    }
+    __syncthreads();
+    if (ctl->abort) return;   // nothing was started
+    if (tid == 0) {
+        // the last CTA to read the epoch publishes it for the next launch
+        const uint32_t ep = ctl->ep;
+        const uint32_t old = atomicAdd(p.done_cnt, 1u);
+        if (old + 1u == gridDim.x * ep) atomicExch(p.epoch, ep);
+    }
+    if (warp < kWorkerWarps) {
+        worker_role(p, pages, ctl);
+    } else if (warp == kLoaderWarp) {
+        if (lane == 0) loader_role(p, pages, ctl);
+    } else {
+        if (lane == 0) scheduler_role(p, ctl, ctl->ep);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host-side launch helpers (called from mk_runtime.cpp)
+// ---------------------------------------------------------------------------
+size_t kernel_smem_bytes() { return kSmemBytes; }
+
+cudaError_t kernel_prepare() {
+    return cudaFuncSetAttribute(mk_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSmemBytes);
+}
+
+cudaError_t kernel_occupancy(int *blocks_per_sm) {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, mk_step_kernel, kThreads,
+                                                         kSmemBytes);
+}
+
+cudaError_t kernel_launch(const Params &p, int grid, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, mk_step_kernel, p);
+}
+
+}  // namespace mk

@@ -1,0 +1,434 @@
+// mk_runtime.cpp -- implementation of the C ABI declared in include/mk.h:
+// argument validation, task-graph construction (mk_graph.cpp), scratch
+// allocation, and the one cooperative launch per decode step.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/mk.h"
+#include "mk_internal.h"
+
+namespace mk {
+size_t kernel_smem_bytes();
+cudaError_t kernel_prepare();
+cudaError_t kernel_occupancy(int *blocks_per_sm);
+cudaError_t kernel_launch(const Params &p, int grid, cudaStream_t stream);
+}  // namespace mk
+
+using namespace mk;
+
+struct mk_ctx {
+    int device = 0;
+    mk_config cfg{};
+    Shape s{};
+    int num_sms = 0;
+    int num_tasks = 0, num_events = 0, num_ops = 0, max_queue = 0, num_lm_tasks = 0;
+    std::vector<Task> h_tasks;
+    std::vector<int32_t> h_queue, h_qoff;
+    std::vector<uint32_t> h_thresholds;
+    // device allocations
+    std::vector<void *> allocs;
+    Params p{};            // template: step inputs filled per call
+    ErrWord *d_err = nullptr;
+    long long steps = 0;
+    bool failed = false;   // a device error was observed by mk_sync
+};
+
+namespace {
+
+template <class T>
+cudaError_t dalloc(mk_ctx *c, T **out, size_t count) {
+    void *ptr = nullptr;
+    size_t bytes = count * sizeof(T);
+    if (bytes == 0) bytes = 16;
+    cudaError_t e = cudaMalloc(&ptr, bytes);
+    if (e != cudaSuccess) return e;
+    c->allocs.push_back(ptr);
+    *out = static_cast<T *>(ptr);
+    return cudaSuccess;
+}
+
+bool aligned16(const void *p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
+    if (!c) return MK_ERR_INVALID;
+    if (c->layers < 1 || c->hidden < 8 || c->n_q_heads < 1 || c->n_kv_heads < 1 ||
+        c->head_dim < 1 || c->ffn < 8 || c->vocab < 1 || c->max_seq < 1 || c->max_batch < 1)
+        return MK_ERR_INVALID;
+    if (c->max_batch > MK_MAX_BATCH) return MK_ERR_INVALID;
+    if (c->n_q_heads % c->n_kv_heads != 0) return MK_ERR_INVALID;
+    const int G = c->n_q_heads / c->n_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return MK_ERR_INVALID;
+    if (c->head_dim != 64 && c->head_dim != 128) return MK_ERR_INVALID;
+    if (G * c->head_dim > 512) return MK_ERR_INVALID;
+    const long long QD = (long long)c->n_q_heads * c->head_dim;
+    if (c->hidden % 8 || c->ffn % 8 || QD % 8) return MK_ERR_INVALID;
+    if (c->hidden > kMaxK || c->ffn > kMaxK || QD > kMaxK) return MK_ERR_INVALID;
+    if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return MK_ERR_INVALID;
+    if (c->attn_chunks < 0 || c->timeout_ns < 0) return MK_ERR_INVALID;
+    if ((long long)c->max_seq * c->head_dim > (1LL << 40)) return MK_ERR_INVALID;
+    if (num_sms < 1 || num_sms > 1024) return MK_ERR_INVALID;
+    s.L = c->layers; s.H = c->hidden; s.nq = c->n_q_heads; s.nkv = c->n_kv_heads;
+    s.d = c->head_dim; s.F = c->ffn; s.V = c->vocab; s.S = c->max_seq; s.Bmax = c->max_batch;
+    s.G = G; s.QD = (int)QD; s.KD = c->n_kv_heads * c->head_dim;
+    s.theta = c->rope_theta; s.eps = c->rms_eps;
+    s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nkv, s.S);
+    if (s.NC > 4096) return MK_ERR_INVALID;
+    return MK_OK;
+}
+
+int map_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return MK_OK;
+    if (e == cudaErrorMemoryAllocation) return MK_ERR_OOM;
+    return MK_ERR_CUDA;
+}
+
+void free_ctx(mk_ctx *c) {
+    if (!c) return;
+    for (void *p : c->allocs) cudaFree(p);
+    delete c;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mk_status_string(int status) {
+    switch (status) {
+    case MK_OK: return "ok";
+    case MK_ERR_INVALID: return "invalid argument";
+    case MK_ERR_CUDA: return "CUDA error";
+    case MK_ERR_TIMEOUT: return "device wait timed out";
+    case MK_ERR_OOM: return "out of memory";
+    case MK_ERR_STATE: return "context unusable after a device error (call mk_reset)";
+    default: return "unknown status";
+    }
+}
+
+int mk_plan(const mk_config *cfg, int num_sms, mk_info *info, int32_t *task_out,
+            int32_t *queue_out, int32_t *qoff_out, uint32_t *thresholds_out, int64_t *bytes_out) {
+    Shape s;
+    int st = shape_from_config(cfg, num_sms, s);
+    if (st != MK_OK) return st;
+    PlanSizes z = plan_sizes(s, num_sms);
+    std::vector<Task> tasks(z.num_tasks);
+    std::vector<int32_t> queue(z.num_tasks), qoff(num_sms + 1);
+    std::vector<uint32_t> thr(z.num_events);
+    std::vector<int64_t> bytes(z.num_tasks);
+    Plan p;
+    p.tasks = tasks.data(); p.queue = queue.data(); p.qoff = qoff.data();
+    p.thresholds = thr.data(); p.bytes = bytes.data();
+    plan_build(s, num_sms, p);
+    if (info) {
+        std::memset(info, 0, sizeof *info);
+        info->num_sms = num_sms;
+        info->num_tasks = p.num_tasks;
+        info->num_events = p.num_events;
+        info->num_ops = p.num_ops;
+        info->attn_chunks = s.NC;
+        info->max_queue = p.max_queue;
+        info->page_bytes = kPageBytes;
+        info->num_pages = kNumPages;
+    }
+    for (int i = 0; i < p.num_tasks; ++i) {
+        const Task &t = tasks[i];
+        if (task_out) {
+            int32_t *o = task_out + 8 * i;
+            o[0] = t.kind; o[1] = t.layer; o[2] = t.dep; o[3] = t.trig;
+            o[4] = t.begin; o[5] = t.end; o[6] = t.sm; o[7] = t.slot;
+        }
+        if (bytes_out) bytes_out[i] = bytes[i];
+    }
+    if (queue_out) std::memcpy(queue_out, queue.data(), sizeof(int32_t) * p.num_tasks);
+    if (qoff_out) std::memcpy(qoff_out, qoff.data(), sizeof(int32_t) * (num_sms + 1));
+    if (thresholds_out) std::memcpy(thresholds_out, thr.data(), sizeof(uint32_t) * p.num_events);
+    return MK_OK;
+}
+
+int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx **out) {
+    if (!out) return MK_ERR_INVALID;
+    *out = nullptr;
+    if (!cfg || !w || !kv) return MK_ERR_INVALID;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MK_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MK_ERR_CUDA;
+    if (prop.major < 10) return MK_ERR_INVALID;     // built for sm_100a only
+    if (!prop.cooperativeLaunch) return MK_ERR_INVALID;
+    if ((size_t)prop.sharedMemPerBlockOptin < kernel_smem_bytes()) return MK_ERR_INVALID;
+    Shape s;
+    int st = shape_from_config(cfg, prop.multiProcessorCount, s);
+    if (st != MK_OK) return st;
+
+    // pointer checks
+    if (!aligned16(w->embed) || !aligned16(w->lm_head) || !aligned16(w->final_norm)) return MK_ERR_INVALID;
+    if (!w->attn_norm || !w->mlp_norm || !w->wq || !w->wk || !w->wv || !w->wo || !w->wg ||
+        !w->wu || !w->wd || !kv->k || !kv->v)
+        return MK_ERR_INVALID;
+    for (int l = 0; l < s.L; ++l) {
+        const void *ps[] = {w->attn_norm[l], w->mlp_norm[l], w->wq[l], w->wk[l], w->wv[l],
+                            w->wo[l], w->wg[l], w->wu[l], w->wd[l], kv->k[l], kv->v[l]};
+        for (const void *q : ps)
+            if (!aligned16(q)) return MK_ERR_INVALID;
+    }
+
+    mk_ctx *c = new (std::nothrow) mk_ctx;
+    if (!c) return MK_ERR_OOM;
+    c->device = dev;
+    c->cfg = *cfg;
+    c->s = s;
+    c->num_sms = prop.multiProcessorCount;
+
+    // ---- task graph (host)
+    PlanSizes z = plan_sizes(s, c->num_sms);
+    c->h_tasks.resize(z.num_tasks);
+    c->h_queue.resize(z.num_tasks);
+    c->h_qoff.resize(c->num_sms + 1);
+    c->h_thresholds.resize(z.num_events);
+    Plan plan;
+    plan.tasks = c->h_tasks.data(); plan.queue = c->h_queue.data(); plan.qoff = c->h_qoff.data();
+    plan.thresholds = c->h_thresholds.data(); plan.bytes = nullptr;
+    plan_build(s, c->num_sms, plan);
+    c->num_tasks = plan.num_tasks;
+    c->num_events = plan.num_events;
+    c->num_ops = plan.num_ops;
+    c->max_queue = plan.max_queue;
+    c->num_lm_tasks = plan.num_lm_tasks;
+
+    // ---- RoPE table: cos/sin of pos * theta^(-2i/d), computed in double
+    const int half = s.d / 2;
+    std::vector<float> rope((size_t)s.S * half * 2);
+    for (int pos = 0; pos < s.S; ++pos)
+        for (int i = 0; i < half; ++i) {
+            double inv = std::pow((double)cfg->rope_theta, -2.0 * i / (double)s.d);
+            double ang = (double)pos * inv;
+            rope[((size_t)pos * half + i) * 2 + 0] = (float)std::cos(ang);
+            rope[((size_t)pos * half + i) * 2 + 1] = (float)std::sin(ang);
+        }
+
+    std::vector<LayerW> lw(s.L);
+    for (int l = 0; l < s.L; ++l) {
+        lw[l].wq = (const uint16_t *)w->wq[l]; lw[l].wk = (const uint16_t *)w->wk[l];
+        lw[l].wv = (const uint16_t *)w->wv[l]; lw[l].wo = (const uint16_t *)w->wo[l];
+        lw[l].wg = (const uint16_t *)w->wg[l]; lw[l].wu = (const uint16_t *)w->wu[l];
+        lw[l].wd = (const uint16_t *)w->wd[l];
+        lw[l].g_attn = (const uint16_t *)w->attn_norm[l]; lw[l].g_mlp = (const uint16_t *)w->mlp_norm[l];
+        lw[l].kc = (uint16_t *)kv->k[l]; lw[l].vc = (uint16_t *)kv->v[l];
+    }
+
+    // ---- device memory
+    Params &p = c->p;
+    p.s = s;
+    cudaError_t e = cudaSuccess;
+    Task *d_tasks; int32_t *d_queue, *d_qoff; uint32_t *d_thr, *d_ev, *d_merge, *d_ctrl;
+    LayerW *d_layers; float2 *d_rope;
+    float *d_x, *d_q, *d_attn, *d_part, *d_act, *d_aval; int32_t *d_aidx;
+    const size_t B = s.Bmax;
+    const size_t n_merge = (size_t)s.L * B * s.nkv;
+#define MK_TRY(expr) do { e = (expr); if (e != cudaSuccess) { free_ctx(c); return map_cuda(e); } } while (0)
+    MK_TRY(dalloc(c, &d_tasks, c->num_tasks));
+    MK_TRY(dalloc(c, &d_queue, c->num_tasks));
+    MK_TRY(dalloc(c, &d_qoff, c->num_sms + 1));
+    MK_TRY(dalloc(c, &d_thr, c->num_events));
+    MK_TRY(dalloc(c, &d_ev, c->num_events));
+    MK_TRY(dalloc(c, &d_merge, n_merge));
+    MK_TRY(dalloc(c, &d_ctrl, 8));             // lm_cnt, epoch, done_cnt, abort
+    MK_TRY(dalloc(c, &c->d_err, 1));
+    MK_TRY(dalloc(c, &d_layers, s.L));
+    MK_TRY(dalloc(c, &d_rope, (size_t)s.S * half));
+    MK_TRY(dalloc(c, &d_x, B * s.H));
+    MK_TRY(dalloc(c, &d_q, B * s.QD));
+    MK_TRY(dalloc(c, &d_attn, B * s.QD));
+    MK_TRY(dalloc(c, &d_part, B * s.nq * (size_t)s.NC * (s.d + 2)));
+    MK_TRY(dalloc(c, &d_act, B * s.F));
+    MK_TRY(dalloc(c, &d_aval, B * c->num_lm_tasks));
+    MK_TRY(dalloc(c, &d_aidx, B * c->num_lm_tasks));
+    TraceRec *d_trace = nullptr;
+    if (cfg->flags & MK_FLAG_TRACE) MK_TRY(dalloc(c, &d_trace, c->num_tasks));
+
+    MK_TRY(cudaMemcpy(d_tasks, c->h_tasks.data(), sizeof(Task) * c->num_tasks, cudaMemcpyHostToDevice));
+    MK_TRY(cudaMemcpy(d_queue, c->h_queue.data(), sizeof(int32_t) * c->num_tasks, cudaMemcpyHostToDevice));
+    MK_TRY(cudaMemcpy(d_qoff, c->h_qoff.data(), sizeof(int32_t) * (c->num_sms + 1), cudaMemcpyHostToDevice));
+    MK_TRY(cudaMemcpy(d_thr, c->h_thresholds.data(), sizeof(uint32_t) * c->num_events, cudaMemcpyHostToDevice));
+    MK_TRY(cudaMemcpy(d_layers, lw.data(), sizeof(LayerW) * s.L, cudaMemcpyHostToDevice));
+    MK_TRY(cudaMemcpy(d_rope, rope.data(), sizeof(float) * rope.size(), cudaMemcpyHostToDevice));
+    MK_TRY(cudaMemset(d_ev, 0, sizeof(uint32_t) * c->num_events));
+    MK_TRY(cudaMemset(d_merge, 0, sizeof(uint32_t) * n_merge));
+    MK_TRY(cudaMemset(d_ctrl, 0, sizeof(uint32_t) * 8));
+    MK_TRY(cudaMemset(c->d_err, 0, sizeof(ErrWord)));
+    MK_TRY(cudaMemset(d_x, 0, sizeof(float) * B * s.H));
+    MK_TRY(cudaMemset(d_q, 0, sizeof(float) * B * s.QD));
+    MK_TRY(cudaMemset(d_attn, 0, sizeof(float) * B * s.QD));
+    MK_TRY(cudaMemset(d_act, 0, sizeof(float) * B * s.F));
+    if (d_trace) {
+        std::vector<TraceRec> tr(c->num_tasks);
+        for (int i = 0; i < c->num_tasks; ++i) {
+            const Task &t = c->h_tasks[i];
+            tr[i] = TraceRec{0, 0, 0, t.sm, t.kind, t.layer, t.trig};
+        }
+        MK_TRY(cudaMemcpy(d_trace, tr.data(), sizeof(TraceRec) * c->num_tasks, cudaMemcpyHostToDevice));
+    }
+    MK_TRY(kernel_prepare());
+    int per_sm = 0;
+    MK_TRY(kernel_occupancy(&per_sm));
+    if (per_sm < 1) { free_ctx(c); return MK_ERR_INVALID; }
+#undef MK_TRY
+
+    p.tasks = d_tasks; p.queue = d_queue; p.qoff = d_qoff; p.thresholds = d_thr; p.events = d_ev;
+    p.merge_cnt = d_merge;
+    p.lm_cnt = d_ctrl + 0; p.epoch = d_ctrl + 1; p.done_cnt = d_ctrl + 2; p.abort_flag = d_ctrl + 3;
+    p.num_lm_tasks = c->num_lm_tasks;
+    p.layers = d_layers;
+    p.embed = (const uint16_t *)w->embed; p.lm_head = (const uint16_t *)w->lm_head;
+    p.g_final = (const uint16_t *)w->final_norm;
+    p.rope = d_rope;
+    p.x = d_x; p.q = d_q; p.attn = d_attn; p.part = d_part; p.act = d_act;
+    p.amax_val = d_aval; p.amax_idx = d_aidx;
+    p.err = c->d_err;
+    p.trace = d_trace;
+    p.timeout_ns = cfg->timeout_ns > 0 ? (unsigned long long)cfg->timeout_ns : 2000000000ull;
+    p.l2_prefetch = (cfg->flags & MK_FLAG_NO_L2_PREFETCH) ? 0 : 1;
+    *out = c;
+    return MK_OK;
+}
+
+int mk_decode_step(mk_ctx *c, const int32_t *tokens, const int32_t *positions, int batch,
+                   float *logits_out, int32_t *next_tok_out, mk_stream_t stream) {
+    if (!c) return MK_ERR_INVALID;
+    if (c->failed) return MK_ERR_STATE;
+    if (batch < 1 || batch > c->s.Bmax) return MK_ERR_INVALID;
+    if (!tokens || !positions || !next_tok_out) return MK_ERR_INVALID;
+    if (((uintptr_t)tokens & 3u) || ((uintptr_t)positions & 3u) || ((uintptr_t)next_tok_out & 3u) ||
+        ((uintptr_t)logits_out & 3u))
+        return MK_ERR_INVALID;
+    Params p = c->p;
+    p.tokens = tokens;
+    p.positions = positions;
+    p.batch = batch;
+    p.logits = logits_out;
+    p.next_tok = next_tok_out;
+    cudaError_t e = kernel_launch(p, c->num_sms, (cudaStream_t)stream);
+    if (e != cudaSuccess) return MK_ERR_CUDA;
+    c->steps++;
+    return MK_OK;
+}
+
+int mk_sync(mk_ctx *c, mk_stream_t stream) {
+    if (!c) return MK_ERR_INVALID;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MK_ERR_CUDA;
+    ErrWord ew;
+    if (cudaMemcpy(&ew, c->d_err, sizeof ew, cudaMemcpyDeviceToHost) != cudaSuccess) return MK_ERR_CUDA;
+    if (ew.code != 0) {
+        c->failed = true;
+        return (int)ew.code;
+    }
+    return MK_OK;
+}
+
+int mk_reset(mk_ctx *c) {
+    if (!c) return MK_ERR_INVALID;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MK_ERR_CUDA;
+    const Params &p = c->p;
+    if (cudaMemset(p.events, 0, sizeof(uint32_t) * c->num_events) != cudaSuccess ||
+        cudaMemset(p.merge_cnt, 0, sizeof(uint32_t) * (size_t)c->s.L * c->s.Bmax * c->s.nkv) != cudaSuccess ||
+        cudaMemset(p.lm_cnt, 0, sizeof(uint32_t) * 4) != cudaSuccess ||
+        cudaMemset(c->d_err, 0, sizeof(ErrWord)) != cudaSuccess ||
+        cudaMemcpy(const_cast<uint32_t *>(p.thresholds), c->h_thresholds.data(), sizeof(uint32_t) * c->num_events,
+                   cudaMemcpyHostToDevice) != cudaSuccess)
+        return MK_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MK_ERR_CUDA;
+    c->steps = 0;
+    c->failed = false;
+    return MK_OK;
+}
+
+int mk_destroy(mk_ctx *c) {
+    if (!c) return MK_OK;
+    cudaDeviceSynchronize();
+    free_ctx(c);
+    return MK_OK;
+}
+
+int mk_get_info(mk_ctx *c, mk_info *out) {
+    if (!c || !out) return MK_ERR_INVALID;
+    std::memset(out, 0, sizeof *out);
+    out->num_sms = c->num_sms;
+    out->num_tasks = c->num_tasks;
+    out->num_events = c->num_events;
+    out->num_ops = c->num_ops;
+    out->attn_chunks = c->s.NC;
+    out->max_queue = c->max_queue;
+    out->page_bytes = kPageBytes;
+    out->num_pages = kNumPages;
+    out->steps_run = c->steps;
+    ErrWord ew;
+    if (cudaMemcpy(&ew, c->d_err, sizeof ew, cudaMemcpyDeviceToHost) != cudaSuccess) return MK_ERR_CUDA;
+    out->err_code = ew.code;
+    out->err_info = ew.where << 24 | (ew.info & 0xffffffu);
+    return MK_OK;
+}
+
+int mk_get_event_counts(mk_ctx *c, uint32_t *counts_out, uint32_t *thresholds_out, int n) {
+    if (!c || n < 0 || n > c->num_events) return MK_ERR_INVALID;
+    if (counts_out &&
+        cudaMemcpy(counts_out, c->p.events, sizeof(uint32_t) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MK_ERR_CUDA;
+    if (thresholds_out &&
+        cudaMemcpy(thresholds_out, c->p.thresholds, sizeof(uint32_t) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MK_ERR_CUDA;
+    return MK_OK;
+}
+
+int mk_read_buffer(mk_ctx *c, int which, float *host_out, size_t count) {
+    if (!c || !host_out) return MK_ERR_INVALID;
+    const Shape &s = c->s;
+    const float *src = nullptr;
+    size_t n = 0;
+    switch (which) {
+    case MK_BUF_HIDDEN: src = c->p.x; n = (size_t)s.Bmax * s.H; break;
+    case MK_BUF_Q: src = c->p.q; n = (size_t)s.Bmax * s.QD; break;
+    case MK_BUF_ATTN: src = c->p.attn; n = (size_t)s.Bmax * s.QD; break;
+    case MK_BUF_ACT: src = c->p.act; n = (size_t)s.Bmax * s.F; break;
+    default: return MK_ERR_INVALID;
+    }
+    if (count > n) return MK_ERR_INVALID;
+    if (cudaMemcpy(host_out, src, sizeof(float) * count, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MK_ERR_CUDA;
+    return MK_OK;
+}
+
+int mk_get_trace(mk_ctx *c, mk_trace_rec *host_out, int n) {
+    if (!c || !host_out || n < 0 || n > c->num_tasks) return MK_ERR_INVALID;
+    if (!c->p.trace) return MK_ERR_INVALID;
+    static_assert(sizeof(mk_trace_rec) == sizeof(TraceRec), "trace record layout");
+    if (cudaMemcpy(host_out, c->p.trace, sizeof(TraceRec) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MK_ERR_CUDA;
+    return MK_OK;
+}
+
+int mk_get_graph(mk_ctx *c, int32_t *task_out, int32_t *queue_out, int32_t *qoff_out) {
+    if (!c) return MK_ERR_INVALID;
+    for (int i = 0; i < c->num_tasks && task_out; ++i) {
+        const Task &t = c->h_tasks[i];
+        int32_t *o = task_out + 8 * i;
+        o[0] = t.kind; o[1] = t.layer; o[2] = t.dep; o[3] = t.trig;
+        o[4] = t.begin; o[5] = t.end; o[6] = t.sm; o[7] = t.slot;
+    }
+    if (queue_out) std::memcpy(queue_out, c->h_queue.data(), sizeof(int32_t) * c->num_tasks);
+    if (qoff_out) std::memcpy(qoff_out, c->h_qoff.data(), sizeof(int32_t) * (c->num_sms + 1));
+    return MK_OK;
+}
+
+int mk_debug_set_threshold(mk_ctx *c, int event, uint32_t threshold) {
+    if (!c || event < 0 || event >= c->num_events) return MK_ERR_INVALID;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MK_ERR_CUDA;
+    if (cudaMemcpy(const_cast<uint32_t *>(c->p.thresholds) + event, &threshold, sizeof threshold, cudaMemcpyHostToDevice) != cudaSuccess)
+        return MK_ERR_CUDA;
+    return MK_OK;
+}
+
+}  // extern "C"

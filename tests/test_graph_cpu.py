@@ -1,0 +1,162 @@
+"""Host-side checks of the C-ABI library and its task-graph builder (no GPU).
+
+The library is loaded and every function include/mk.h declares must be
+exported; mk_plan builds the static task graph on the host, which is checked
+for coverage, event thresholds, dependency order, load balance, and by a
+simulator that runs the per-SM queues in random interleavings with event
+counters the way the persistent kernel does.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+from persistent_decode_megakernel_02_b200 import workloads as wl
+
+mk = pytest.importorskip("persistent_decode_megakernel_02_b200.mk")
+
+QKV, ATTN, OPROJ, GATEUP, DOWN, LMHEAD = range(6)
+SMS = 148
+
+
+def test_library_exports_every_declared_function():
+    names = mk.header_functions()
+    assert "mk_create" in names and "mk_decode_step" in names and "mk_destroy" in names
+    lib = ctypes.CDLL(mk.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in mk.h but not exported"
+
+
+def test_status_strings():
+    assert mk.status_string(0) == "ok"
+    for s in range(1, 6):
+        assert mk.status_string(s) != "unknown status"
+    assert mk.status_string(99) == "unknown status"
+
+
+def _tiles(shape):
+    d, H, F, V = shape.head_dim, shape.hidden, shape.ffn, shape.vocab
+    return {QKV: (shape.n_q_heads + shape.n_kv_heads) * d // 8 + shape.n_kv_heads * d // 8,
+            OPROJ: H // 8, GATEUP: F // 4, DOWN: H // 8, LMHEAD: (V + 7) // 8}
+
+
+CASES = [("tiny", wl.TINY, 64), ("1b", wl.LLAMA_1B, 560), ("8b", wl.LLAMA_8B, 560),
+         ("longctx", wl.LLAMA_1B, 16640)]
+
+
+@pytest.fixture(scope="module", params=CASES, ids=[c[0] for c in CASES])
+def planned(request):
+    name, shape, S = request.param
+    cfg = mk.make_config(shape, S, 1)
+    return shape, cfg, mk.plan(cfg, SMS)
+
+
+def test_every_row_and_item_covered_once(planned):
+    shape, cfg, pl = planned
+    tasks = pl["tasks"]
+    tiles = _tiles(shape)
+    nc = pl["info"].attn_chunks
+    for layer in range(shape.layers + 1):
+        for kind in (QKV, ATTN, OPROJ, GATEUP, DOWN, LMHEAD):
+            sel = tasks[(tasks[:, 0] == kind) & (tasks[:, 1] == layer)]
+            if (kind == LMHEAD) != (layer == shape.layers):
+                assert len(sel) == 0
+                continue
+            n = shape.n_kv_heads * nc if kind == ATTN else tiles[kind]
+            cover = np.zeros(n, np.int32)
+            for t in sel:
+                cover[t[4]:t[5]] += 1
+            assert np.all(cover == 1), (kind, layer)
+            # slots number the op's tasks 0..T-1
+            assert sorted(sel[:, 7].tolist()) == list(range(len(sel)))
+
+
+def test_thresholds_equal_triggering_tasks_and_deps_form_a_chain(planned):
+    shape, cfg, pl = planned
+    tasks, thr = pl["tasks"], pl["thresholds"]
+    E = len(thr)
+    assert E == 5 * shape.layers + 1
+    counts = np.bincount(tasks[:, 3], minlength=E)
+    assert np.array_equal(counts, thr.astype(np.int64))
+    for t in tasks:
+        # each op waits on the event of the op right before it (none for the first)
+        assert t[2] == t[3] - 1
+    # one op per event: all tasks triggering an event share kind and layer
+    for e in range(E):
+        sel = tasks[tasks[:, 3] == e]
+        assert len(set(map(tuple, sel[:, :2].tolist()))) == 1
+
+
+def test_queues_partition_tasks_in_op_order(planned):
+    shape, cfg, pl = planned
+    tasks, queue, qoff = pl["tasks"], pl["queue"], pl["qoff"]
+    assert qoff[0] == 0 and qoff[-1] == len(tasks)
+    assert sorted(queue.tolist()) == list(range(len(tasks)))
+    for sm in range(SMS):
+        q = queue[qoff[sm]:qoff[sm + 1]]
+        assert np.all(tasks[q, 6] == sm)
+        assert np.all(np.diff(tasks[q, 3]) >= 0)     # events (= op order) never go back
+        assert np.all(np.diff(q) > 0)
+
+
+def test_weight_bytes_balanced_and_complete(planned):
+    shape, cfg, pl = planned
+    tasks, nbytes = pl["tasks"], pl["bytes"]
+    gemv = tasks[:, 0] != ATTN
+    H, F, V = shape.hidden, shape.ffn, shape.vocab
+    QD, KD = shape.n_q_heads * shape.head_dim, shape.n_kv_heads * shape.head_dim
+    matrices = 2 * (shape.layers * ((QD + 2 * KD) * H + H * QD + 3 * F * H) + V * H)
+    assert int(nbytes[gemv].sum()) == matrices
+    if shape.layers >= 16:
+        per_sm = np.bincount(tasks[:, 6], weights=nbytes.astype(np.float64), minlength=SMS)
+        assert per_sm.max() / per_sm.mean() < 1.02
+
+
+def _simulate(tasks, queue, qoff, thr, steps, rng):
+    """Run the per-SM queues in random interleavings; returns event counts."""
+    ev = np.zeros(len(thr), np.int64)
+    for ep in range(1, steps + 1):
+        pos = [int(qoff[s]) for s in range(SMS)]
+        live = [s for s in range(SMS) if pos[s] < qoff[s + 1]]
+        while live:
+            progressed = False
+            for s in rng.permutation(live):
+                t = tasks[queue[pos[s]]]
+                if t[2] < 0 or ev[t[2]] >= thr[t[2]] * ep:
+                    ev[t[3]] += 1
+                    pos[s] += 1
+                    progressed = True
+            live = [s for s in live if pos[s] < qoff[s + 1]]
+            assert progressed, "schedule deadlocked"
+    return ev
+
+
+def test_schedule_runs_to_completion_with_exact_event_counts(planned):
+    shape, cfg, pl = planned
+    if shape.layers > 16:
+        pytest.skip("covered by the smaller shapes")
+    rng = np.random.default_rng(0)
+    ev = _simulate(pl["tasks"], pl["queue"], pl["qoff"], pl["thresholds"], 2, rng)
+    assert np.array_equal(ev, 2 * pl["thresholds"].astype(np.int64))
+
+
+@pytest.mark.parametrize("bad", [
+    dict(head_dim=96), dict(n_q_heads=12, n_kv_heads=4), dict(hidden=2044),
+    dict(ffn=20000), dict(max_batch=99), dict(vocab=0), dict(max_seq=0),
+])
+def test_plan_rejects_unsupported_shapes(bad):
+    base = dict(layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=768,
+                vocab=4096, tied=True, rope_theta=1e4)
+    run = {k: bad[k] for k in ("max_seq", "max_batch") if k in bad}
+    base.update({k: v for k, v in bad.items() if k not in run})
+    shape = wl.ModelShape("bad", **base)
+    cfg = mk.make_config(shape, bad.get("max_seq", 64), bad.get("max_batch", 1))
+    with pytest.raises(mk.MkError) as ei:
+        mk.plan(cfg, SMS)
+    assert ei.value.status == mk.MK_ERR_INVALID
+
+
+def test_default_attention_chunks():
+    assert mk.plan(mk.make_config(wl.LLAMA_1B, 16640), SMS)["info"].attn_chunks == 18
+    assert mk.plan(mk.make_config(wl.TINY, 64), SMS)["info"].attn_chunks == 4
+    assert mk.plan(mk.make_config(wl.TINY, 64, attn_chunks=7), SMS)["info"].attn_chunks == 7
