@@ -125,6 +125,11 @@ typedef struct mk_ctx mk_ctx;
  * Validate the shape, build the static task graph for this device (one
  * persistent CTA per SM), allocate scratch and upload the tables.  Blocks
  * the host.  *out receives the context (NULL on error).
+ * The q/k/v and gate/up matrices are copied into a library-owned layout
+ * (rows in the order the kernel streams them, so every task reads one
+ * contiguous range): later changes to those caller buffers are not seen,
+ * and device memory grows by their size.  The other weights and the KV
+ * cache are used in place.
  * Errors: MK_ERR_INVALID (shape or pointer checks), MK_ERR_OOM, MK_ERR_CUDA.
  */
 int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx **out);

@@ -24,13 +24,30 @@ def _nvcc() -> str:
     return "nvcc"
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
-        return True
-    t = os.path.getmtime(LIB)
+STAMP = LIB + ".sha256"
+
+
+def _digest() -> str:
+    """Hash of every input of the build (sources, headers, flags)."""
+    import hashlib
+    h = hashlib.sha256()
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps.append(os.path.join(ROOT, "include", "mk.h"))
-    return any(os.path.getmtime(f) > t for f in deps)
+    for f in deps:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    h.update(" ".join(ARCH).encode())
+    return h.hexdigest()
+
+
+def _stale() -> bool:
+    # content-based: copies of the tree (which may not keep mtimes) reuse the
+    # library as long as its inputs are unchanged
+    if not os.path.exists(LIB) or not os.path.exists(STAMP):
+        return True
+    with open(STAMP) as f:
+        return f.read().strip() != _digest()
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
@@ -42,6 +59,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
     subprocess.check_call(cmd)
+    with open(STAMP, "w") as f:
+        f.write(_digest())
     return LIB
 
 

@@ -97,15 +97,18 @@ struct Builder {
         return T;
     }
 
+    // One task per attention item.  Items go to distinct SMs (the least
+    // loaded ones) so an SM runs a second item of the same op only when
+    // there are more items than SMs.
     int attn_op(int layer, int dep, int trig) {
         OpTiles t = op_tiles(s);
         int per_chunk = (s.S + s.NC - 1) / s.NC;
         int64_t est = (int64_t)4 * s.d * per_chunk;   // K + V bf16 of one chunk at capacity
-        for (int i = 0; i < t.attn_items; ++i) {
-            int best = 0;   // least-loaded SM (lowest index on ties)
-            for (int k = 1; k < p.num_sms; ++k)
-                if (load[k] < load[best]) best = k;
-            add(OP_ATTN, layer, dep, trig, i, i + 1, best, i, est);
+        for (int i = 0; i < t.attn_items; i += p.num_sms) {
+            sort_by_load();
+            int n = t.attn_items - i < p.num_sms ? t.attn_items - i : p.num_sms;
+            for (int k = 0; k < n; ++k)
+                add(OP_ATTN, layer, dep, trig, i + k, i + k + 1, order[k], i + k, est);
         }
         return t.attn_items;
     }

@@ -31,6 +31,7 @@ constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 16384
 constexpr int kMaxGroup = 8;        // q heads per KV head handled by one attention task
 constexpr int kMaxHeadDim = 256;
 constexpr long long kL2Lookahead = 256 * 1024;  // bytes the L2 prefetch runs ahead of the ring
+constexpr int kL2Chunk = 64 * 1024;             // bytes per L2 prefetch instruction
 
 // ---- ops ---------------------------------------------------------------------
 enum OpKind : int32_t { OP_QKV = 0, OP_ATTN = 1, OP_OPROJ = 2, OP_GATEUP = 3, OP_DOWN = 4, OP_LMHEAD = 5 };
@@ -50,8 +51,15 @@ struct Task {
 static_assert(sizeof(Task) == 32, "Task is 8 int32");
 
 // Device pointers of one layer (bf16 as uint16_t on the host side).
+//  qkv: library-owned [(nq + 2 nkv) d][H] in QKV tile order: for every q
+//       head then every k head, d/8 tiles of 8 rows (4 rows of the first
+//       half of the head, then the 4 rows d/2 later that RoPE pairs them
+//       with), then the value rows in their own order.
+//  gu:  library-owned [2F][H] in gate/up tile order: 4 gate rows, then the
+//       4 up rows with the same indices.
+//  wo, wd: the caller's matrices, read in place.
 struct LayerW {
-    const uint16_t *wq, *wk, *wv, *wo, *wg, *wu, *wd;
+    const uint16_t *qkv, *gu, *wo, *wd;
     const uint16_t *g_attn, *g_mlp;
     uint16_t *kc, *vc;
 };

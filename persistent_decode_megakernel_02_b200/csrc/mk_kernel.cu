@@ -220,17 +220,6 @@ __device__ __forceinline__ bool wait_mbar(uint64_t *bar, uint32_t parity, const 
 // ---------------------------------------------------------------------------
 // task geometry shared by the loader and the workers
 // ---------------------------------------------------------------------------
-struct Seg {
-    const void *src;
-    uint32_t dst;     // byte offset in the page
-    uint32_t bytes;
-};
-struct PageDesc {
-    Seg seg[kTileRows];
-    int nseg;
-    uint32_t bytes;
-};
-
 // Attention chunk of one work item.
 struct AttnChunk {
     int b, kvh, c;
@@ -263,148 +252,139 @@ __device__ __forceinline__ AttnChunk attn_chunk(const Params &p, int item) {
     return a;
 }
 
-__device__ __forceinline__ int task_pages(const Params &p, const Task &t) {
-    if (t.kind == OP_ATTN) {
-        AttnChunk a = attn_chunk(p, t.begin);
-        int npp = attn_pos_per_page(p.s.d);
-        return (a.npre + npp - 1) / npp;
-    }
-    int K = op_k(p.s, t.kind);
-    return (t.end - t.begin) * (kTileRows / rows_per_page(K));
-}
+// Weights of every GEMV op are laid out so that tile t's 8 rows are
+// contiguous at base + t * 8 * K (bf16 elements): the q/k/v and gate/up
+// matrices are repacked into that order by mk_create, the O-projection,
+// down-projection and LM head already are in it.  A task (tiles [begin,
+// end)) is therefore one contiguous byte range, streamed page by page.
+struct GemvStream {
+    const char *src;      // next byte to load
+    long long left;       // bytes of real rows still to load
+    uint32_t page_bytes;  // rows_per_page * K * 2
+    int npages;
+};
 
-// Source row r (0..7) of GEMV tile `tile`, or null when the row is past
-// the end of the matrix (ragged LM-head tile).
-__device__ __forceinline__ const uint16_t *gemv_row(const Params &p, int kind, int layer, int tile,
-                                                    int r) {
-    const Shape &s = p.s;
-    const size_t H = (size_t)s.H;
-    if (kind == OP_LMHEAD) {
-        int row = tile * 8 + r;
-        return row < s.V ? p.lm_head + (size_t)row * H : nullptr;
-    }
+__device__ __forceinline__ const uint16_t *gemv_base(const Params &p, int kind, int layer) {
+    if (kind == OP_LMHEAD) return p.lm_head;
     const LayerW &L = p.layers[layer];
     switch (kind) {
-    case OP_QKV: {
-        int npair = (s.nq + s.nkv) * s.d / 8;
-        if (tile < npair) {
-            int per_head = s.d / 8;
-            int head = tile / per_head;
-            int j4 = (tile % per_head) * 4;
-            const uint16_t *base = head < s.nq ? L.wq + (size_t)head * s.d * H
-                                               : L.wk + (size_t)(head - s.nq) * s.d * H;
-            int row = r < 4 ? j4 + r : s.d / 2 + j4 + (r - 4);
-            return base + (size_t)row * H;
-        }
-        return L.wv + (size_t)((tile - npair) * 8 + r) * H;
-    }
-    case OP_OPROJ: return L.wo + (size_t)(tile * 8 + r) * (size_t)s.QD;
-    case OP_GATEUP:
-        return r < 4 ? L.wg + (size_t)(tile * 4 + r) * H : L.wu + (size_t)(tile * 4 + r - 4) * H;
-    default: /* OP_DOWN */ return L.wd + (size_t)(tile * 8 + r) * (size_t)s.F;
+    case OP_QKV: return L.qkv;
+    case OP_OPROJ: return L.wo;
+    case OP_GATEUP: return L.gu;
+    default: return L.wd;
     }
 }
 
-__device__ void page_desc(const Params &p, const Task &t, int pidx, PageDesc &pd) {
-    const Shape &s = p.s;
-    pd.nseg = 0;
-    pd.bytes = 0;
-    if (t.kind == OP_ATTN) {
-        AttnChunk a = attn_chunk(p, t.begin);
-        const LayerW &L = p.layers[t.layer];
-        int npp = attn_pos_per_page(s.d);
-        int pos0 = a.c0 + pidx * npp;
-        int n = min(npp, a.npre - pidx * npp);
-        size_t off = (((size_t)a.b * s.nkv + a.kvh) * s.S + pos0) * s.d;
-        uint32_t bytes = (uint32_t)n * s.d * 2;
-        pd.seg[0] = Seg{L.kc + off, 0u, bytes};
-        pd.seg[1] = Seg{L.vc + off, (uint32_t)(npp * s.d * 2), bytes};
-        pd.nseg = 2;
-        pd.bytes = 2 * bytes;
-        return;
-    }
-    const int K = op_k(s, t.kind);
+__device__ __forceinline__ GemvStream gemv_stream(const Params &p, const Task &t) {
+    const int K = op_k(p.s, t.kind);
     const int rpp = rows_per_page(K);
-    const int ppt = kTileRows / rpp;
-    const int tile = t.begin + pidx / ppt;
-    const int r0 = (pidx % ppt) * rpp;
-    const uint32_t row_bytes = (uint32_t)K * 2u;
-    const char *run_end = nullptr;
-    for (int i = 0; i < rpp; ++i) {
-        const uint16_t *src = gemv_row(p, t.kind, t.layer, tile, r0 + i);
-        if (!src) break;
-        if ((const char *)src == run_end && pd.nseg > 0) {
-            pd.seg[pd.nseg - 1].bytes += row_bytes;
-        } else {
-            pd.seg[pd.nseg++] = Seg{src, (uint32_t)i * row_bytes, row_bytes};
-        }
-        run_end = (const char *)src + row_bytes;
-        pd.bytes += row_bytes;
-    }
+    const long long row_bytes = 2LL * K;
+    GemvStream g;
+    g.src = reinterpret_cast<const char *>(gemv_base(p, t.kind, t.layer)) + (long long)t.begin * 8 * row_bytes;
+    long long rows = (long long)(t.end - t.begin) * 8;
+    if (t.kind == OP_LMHEAD) rows = min(rows, (long long)p.s.V - (long long)t.begin * 8);
+    g.left = rows * row_bytes;
+    g.page_bytes = (uint32_t)(rpp * row_bytes);
+    g.npages = (t.end - t.begin) * (kTileRows / rpp);
+    return g;
 }
-
-// Iterates (task, page) over one SM's queue in execution order.
-struct PageCursor {
-    int qi, q1, pidx, npages;
-    Task t;
-    __device__ PageCursor(int q0, int q1_) : qi(q0 - 1), q1(q1_), pidx(0), npages(0) {}
-    __device__ bool next(const Params &p, PageDesc &pd) {
-        while (pidx >= npages) {
-            if (++qi >= q1) return false;
-            t = p.tasks[p.queue[qi]];
-            npages = task_pages(p, t);
-            pidx = 0;
-        }
-        page_desc(p, t, pidx++, pd);
-        return true;
-    }
-};
 
 // ---------------------------------------------------------------------------
 // loader role (one thread)
 // ---------------------------------------------------------------------------
+struct Ring {
+    uint32_t seq = 0;     // pages issued
+};
+
+// Wait for a free page, then arm its full barrier for `bytes`.
+__device__ __forceinline__ bool ring_acquire(const Params &p, SmemCtl *ctl, Ring &r, uint32_t bytes,
+                                             uint32_t task, uint32_t &slot) {
+    slot = r.seq % kNumPages;
+    const uint32_t par = ((r.seq / kNumPages) & 1u) ^ 1u;
+    if (!wait_mbar(&ctl->empty[slot], par, p, ctl, W_EMPTY, task)) return false;
+    mbar_arrive_expect_tx(&ctl->full[slot], bytes);
+    ++r.seq;
+    return true;
+}
+
+// L2 prefetch cursor: walks the GEMV byte ranges of the queue ahead of the
+// ring so HBM keeps streaming while the ring is full.
+struct Prefetcher {
+    int qi, q1;
+    const char *src = nullptr;
+    long long left = 0;
+    long long done = 0;   // GEMV bytes prefetched so far
+    bool more = true;
+    __device__ Prefetcher(int q0, int q1_) : qi(q0 - 1), q1(q1_) {}
+    __device__ void run(const Params &p, long long limit) {
+        while (more && done < limit) {
+            if (left <= 0) {
+                if (++qi >= q1) { more = false; return; }
+                const Task t = p.tasks[p.queue[qi]];
+                if (t.kind == OP_ATTN) continue;
+                GemvStream g = gemv_stream(p, t);
+                src = g.src;
+                left = g.left;
+                continue;
+            }
+            const uint32_t chunk = (uint32_t)min(left, (long long)kL2Chunk);
+            prefetch_l2(src, chunk);
+            src += chunk;
+            left -= chunk;
+            done += chunk;
+        }
+    }
+};
+
 __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
-    PageCursor fill(q0, q1), pf(q0, q1);
-    PageDesc pd, pp;
-    uint32_t seq = 0;
-    long long fill_bytes = 0, pf_bytes = 0;
-    bool pf_more = p.l2_prefetch != 0;
-    bool ok = true;
-    while (fill.next(p, pd)) {
-        // keep HBM busy beyond the ring: prefetch later pages into L2
-        while (pf_more && pf_bytes < fill_bytes + kL2Lookahead) {
-            if (!pf.next(p, pp)) { pf_more = false; break; }
-            if (pf_bytes >= fill_bytes) {
-                for (int i = 0; i < pp.nseg; ++i) prefetch_l2(pp.seg[i].src, pp.seg[i].bytes);
+    Ring ring;
+    Prefetcher pf(q0, q1);
+    long long issued = 0;   // GEMV bytes copied into the ring so far
+    bool ok = true;         // false when a wait was abandoned
+    for (int qi = q0; qi < q1 && ok; ++qi) {
+        const int id = p.queue[qi];
+        const Task t = p.tasks[id];
+        if (t.kind == OP_ATTN) {
+            const AttnChunk a = attn_chunk(p, t.begin);
+            const int npp = attn_pos_per_page(p.s.d);
+            const LayerW &L = p.layers[t.layer];
+            const size_t head_off = ((size_t)a.b * p.s.nkv + a.kvh) * p.s.S;
+            for (int pos0 = a.c0; pos0 < a.c0 + a.npre; pos0 += npp) {
+                const int n = min(npp, a.c0 + a.npre - pos0);
+                const uint32_t bytes = (uint32_t)n * p.s.d * 2;
+                uint32_t slot;
+                if (!ring_acquire(p, ctl, ring, 2 * bytes, (uint32_t)id, slot)) { ok = false; break; }
+                unsigned char *dst = pages + (size_t)slot * kPageBytes;
+                const size_t off = (head_off + pos0) * p.s.d;
+                bulk_g2s(dst, L.kc + off, bytes, &ctl->full[slot]);
+                bulk_g2s(dst + (size_t)npp * p.s.d * 2, L.vc + off, bytes, &ctl->full[slot]);
             }
-            pf_bytes += pp.bytes;
+            continue;
         }
-        const uint32_t slot = seq % kNumPages;
-        const uint32_t par = ((seq / kNumPages) & 1u) ^ 1u;
-        if (!wait_mbar(&ctl->empty[slot], par, p, ctl, W_EMPTY, (uint32_t)p.queue[fill.qi])) {
-            ok = false;
-            break;
+        GemvStream g = gemv_stream(p, t);
+        for (int k = 0; k < g.npages; ++k) {
+            if (p.l2_prefetch) pf.run(p, issued + kL2Lookahead);
+            const uint32_t bytes = (uint32_t)max(0LL, min((long long)g.page_bytes, g.left));
+            uint32_t slot;
+            if (!ring_acquire(p, ctl, ring, bytes, (uint32_t)id, slot)) { ok = false; break; }
+            if (bytes) bulk_g2s(pages + (size_t)slot * kPageBytes, g.src, bytes, &ctl->full[slot]);
+            g.src += g.page_bytes;
+            g.left -= bytes;
+            issued += bytes;
         }
-        mbar_arrive_expect_tx(&ctl->full[slot], pd.bytes);
-        unsigned char *dst = pages + (size_t)slot * kPageBytes;
-        for (int i = 0; i < pd.nseg; ++i) bulk_g2s(dst + pd.seg[i].dst, pd.seg[i].src, pd.seg[i].bytes, &ctl->full[slot]);
-        fill_bytes += pd.bytes;
-        ++seq;
     }
-    (void)ok;
-    {
-        // let every copy already issued land before this thread returns, so
-        // no bulk copy can still be writing shared memory when the CTA exits
-        uint32_t first = seq > (uint32_t)kNumPages ? seq - kNumPages : 0u;
-        for (uint32_t k = first; k < seq; ++k) {
-            Spin s;
-            while (!mbar_try_wait(&ctl->full[k % kNumPages], (k / kNumPages) & 1u)) {
-                if ((++s.n & 127u) == 0u) {
-                    unsigned long long now = globaltimer();
-                    if (s.t0 == 0) s.t0 = now;
-                    else if (now - s.t0 > p.timeout_ns) break;
-                }
+    // Let every copy already issued land before this thread returns, so no
+    // bulk copy can still be writing shared memory when the CTA exits.
+    const uint32_t seq = ring.seq;
+    const uint32_t first = seq > (uint32_t)kNumPages ? seq - kNumPages : 0u;
+    for (uint32_t k = first; k < seq; ++k) {
+        Spin s;
+        while (!mbar_try_wait(&ctl->full[k % kNumPages], (k / kNumPages) & 1u)) {
+            if ((++s.n & 127u) == 0u) {
+                unsigned long long now = globaltimer();
+                if (s.t0 == 0) s.t0 = now;
+                else if (now - s.t0 > p.timeout_ns) break;
             }
         }
     }

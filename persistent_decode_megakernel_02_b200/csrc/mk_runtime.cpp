@@ -212,9 +212,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
 
     std::vector<LayerW> lw(s.L);
     for (int l = 0; l < s.L; ++l) {
-        lw[l].wq = (const uint16_t *)w->wq[l]; lw[l].wk = (const uint16_t *)w->wk[l];
-        lw[l].wv = (const uint16_t *)w->wv[l]; lw[l].wo = (const uint16_t *)w->wo[l];
-        lw[l].wg = (const uint16_t *)w->wg[l]; lw[l].wu = (const uint16_t *)w->wu[l];
+        lw[l].wo = (const uint16_t *)w->wo[l];
         lw[l].wd = (const uint16_t *)w->wd[l];
         lw[l].g_attn = (const uint16_t *)w->attn_norm[l]; lw[l].g_mlp = (const uint16_t *)w->mlp_norm[l];
         lw[l].kc = (uint16_t *)kv->k[l]; lw[l].vc = (uint16_t *)kv->v[l];
@@ -249,6 +247,34 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     MK_TRY(dalloc(c, &d_aidx, B * c->num_lm_tasks));
     TraceRec *d_trace = nullptr;
     if (cfg->flags & MK_FLAG_TRACE) MK_TRY(dalloc(c, &d_trace, c->num_tasks));
+
+    // ---- repack q/k/v and gate/up into tile order (see LayerW)
+    {
+        const size_t rb = 2 * (size_t)s.H;          // bytes of one row of K = H
+        const size_t tile = 8 * rb;
+        const int per_head = s.d / 8;
+        for (int l = 0; l < s.L; ++l) {
+            uint16_t *qkv, *gu;
+            MK_TRY(dalloc(c, &qkv, (size_t)(s.QD + 2 * s.KD) * s.H));
+            MK_TRY(dalloc(c, &gu, (size_t)2 * s.F * s.H));
+            char *dq = (char *)qkv;
+            for (int h = 0; h < s.nq + s.nkv; ++h) {
+                const char *src = h < s.nq ? (const char *)w->wq[l] + (size_t)h * s.d * rb
+                                           : (const char *)w->wk[l] + (size_t)(h - s.nq) * s.d * rb;
+                char *dst = dq + (size_t)h * per_head * tile;
+                MK_TRY(cudaMemcpy2D(dst, tile, src, 4 * rb, 4 * rb, per_head, cudaMemcpyDeviceToDevice));
+                MK_TRY(cudaMemcpy2D(dst + 4 * rb, tile, src + (size_t)(s.d / 2) * rb, 4 * rb, 4 * rb,
+                                    per_head, cudaMemcpyDeviceToDevice));
+            }
+            MK_TRY(cudaMemcpy(dq + (size_t)(s.nq + s.nkv) * per_head * tile, w->wv[l],
+                              (size_t)s.KD * rb, cudaMemcpyDeviceToDevice));
+            MK_TRY(cudaMemcpy2D(gu, tile, w->wg[l], 4 * rb, 4 * rb, s.F / 4, cudaMemcpyDeviceToDevice));
+            MK_TRY(cudaMemcpy2D((char *)gu + 4 * rb, tile, w->wu[l], 4 * rb, 4 * rb, s.F / 4,
+                                cudaMemcpyDeviceToDevice));
+            lw[l].qkv = qkv;
+            lw[l].gu = gu;
+        }
+    }
 
     MK_TRY(cudaMemcpy(d_tasks, c->h_tasks.data(), sizeof(Task) * c->num_tasks, cudaMemcpyHostToDevice));
     MK_TRY(cudaMemcpy(d_queue, c->h_queue.data(), sizeof(int32_t) * c->num_tasks, cudaMemcpyHostToDevice));
