@@ -78,20 +78,23 @@ struct Builder {
         return t;
     }
 
-    // Split `ntiles` tiles of `tile_bytes` (last tile `last_bytes`) over the
-    // least-loaded SMs, one contiguous tile range per task.  Returns the
-    // number of tasks.
-    int gemv_op(int kind, int layer, int dep, int trig, int ntiles, int64_t tile_bytes,
-                int64_t last_bytes) {
+    // Split the op's `ntiles` tiles over the least-loaded SMs, one
+    // contiguous tile range per task, with equal tile counts (+-1).
+    // Returns the number of tasks.
+    int gemv_op(int kind, int layer, int dep, int trig, int ntiles) {
+        const int K = op_k(s, kind);
         int T = ntiles < p.num_sms ? ntiles : p.num_sms;
         int base = ntiles / T, extra = ntiles % T;
         sort_by_load();
         int tile = 0;
         for (int i = 0; i < T; ++i) {
             int n = base + (i < extra ? 1 : 0);
-            int64_t b = (int64_t)n * tile_bytes;
-            if (tile + n == ntiles) b += last_bytes - tile_bytes;
-            add(kind, layer, dep, trig, tile, tile + n, order[i], i, b);
+            long long rows = tile_row_offset(s, kind, tile + n) - tile_row_offset(s, kind, tile);
+            if (kind == OP_LMHEAD) {
+                long long valid = (long long)s.V - tile_row_offset(s, kind, tile);
+                if (rows > valid) rows = valid;
+            }
+            add(kind, layer, dep, trig, tile, tile + n, order[i], i, rows * 2LL * K);
             tile += n;
         }
         return T;
@@ -124,21 +127,17 @@ void plan_build(const Shape &s, int num_sms, Plan &p) {
     p.num_ops = z.num_ops;
     Builder b(s, p);
     OpTiles t = op_tiles(s);
-    const int64_t H2 = 2LL * s.H;
     for (int l = 0; l < s.L; ++l) {
         int e_qkv = 5 * l, e_attn = e_qkv + 1, e_o = e_qkv + 2, e_gu = e_qkv + 3, e_down = e_qkv + 4;
         int dep_in = l == 0 ? -1 : e_qkv - 1;   // previous layer's down projection
-        p.thresholds[e_qkv] = b.gemv_op(OP_QKV, l, dep_in, e_qkv, t.qkv_pair + t.qkv_v,
-                                        8 * H2, 8 * H2);
+        p.thresholds[e_qkv] = b.gemv_op(OP_QKV, l, dep_in, e_qkv, t.qkv_pair + t.qkv_v);
         p.thresholds[e_attn] = b.attn_op(l, e_qkv, e_attn);
-        p.thresholds[e_o] = b.gemv_op(OP_OPROJ, l, e_attn, e_o, t.oproj, 16LL * s.QD, 16LL * s.QD);
-        p.thresholds[e_gu] = b.gemv_op(OP_GATEUP, l, e_o, e_gu, t.gateup, 8 * H2, 8 * H2);
-        p.thresholds[e_down] = b.gemv_op(OP_DOWN, l, e_gu, e_down, t.down, 16LL * s.F, 16LL * s.F);
+        p.thresholds[e_o] = b.gemv_op(OP_OPROJ, l, e_attn, e_o, t.oproj);
+        p.thresholds[e_gu] = b.gemv_op(OP_GATEUP, l, e_o, e_gu, t.gateup);
+        p.thresholds[e_down] = b.gemv_op(OP_DOWN, l, e_gu, e_down, t.down);
     }
     int e_lm = 5 * s.L;
-    int last_rows = s.V - 8 * (t.lmhead - 1);
-    p.thresholds[e_lm] = b.gemv_op(OP_LMHEAD, s.L, e_lm - 1, e_lm, t.lmhead, 8 * H2,
-                                   (int64_t)last_rows * H2);
+    p.thresholds[e_lm] = b.gemv_op(OP_LMHEAD, s.L, e_lm - 1, e_lm, t.lmhead);
     p.num_lm_tasks = (int)p.thresholds[e_lm];
     p.num_tasks = b.nt;
 

@@ -73,22 +73,27 @@ struct Shape {
 };
 
 // Tile counts of each op (identical on host and device).
+//  QKV:    (nq + nkv) * d / 16 "pair" tiles of 16 rows (8 rows of the first
+//          half of a head + the 8 rows d/2 later that RoPE pairs them with),
+//          then nkv * d / 8 value tiles of 8 rows
+//  GATEUP: F / 8 pair tiles of 16 rows (8 gate rows + the same 8 up rows)
+//  OPROJ, DOWN: H / 8 tiles of 8 rows; LMHEAD: ceil(V / 8) tiles of 8 rows
 struct OpTiles {
-    int qkv_pair;     // (nq + nkv) * d / 8 tiles of 4 RoPE pairs
-    int qkv_v;        // nkv * d / 8 tiles of 8 value rows
-    int oproj;        // H / 8
-    int gateup;       // F / 4 (4 gate rows + 4 up rows)
-    int down;         // H / 8
-    int lmhead;       // ceil(V / 8)
+    int qkv_pair;
+    int qkv_v;
+    int oproj;
+    int gateup;
+    int down;
+    int lmhead;
     int attn_items;   // Bmax * nkv * NC
 };
 
 MK_HD inline OpTiles op_tiles(const Shape &s) {
     OpTiles t;
-    t.qkv_pair = (s.nq + s.nkv) * s.d / 8;
+    t.qkv_pair = (s.nq + s.nkv) * s.d / 16;
     t.qkv_v = s.nkv * s.d / 8;
     t.oproj = s.H / 8;
-    t.gateup = s.F / 4;
+    t.gateup = s.F / 8;
     t.down = s.H / 8;
     t.lmhead = (s.V + 7) / 8;
     t.attn_items = s.Bmax * s.nkv * s.NC;
@@ -100,8 +105,28 @@ MK_HD inline int op_k(const Shape &s, int kind) {
     return kind == OP_OPROJ ? s.QD : (kind == OP_DOWN ? s.F : s.H);
 }
 
-// Rows of one tile held by one page: the largest power of two <= 8 whose
-// rows (K bf16 each) fit in a page.
+// Row offset of tile `tile` in its op's weight buffer (rows of tiles are
+// contiguous and in tile order) -- also the rows of tiles [0, tile).
+MK_HD inline long long tile_row_offset(const Shape &s, int kind, int tile) {
+    if (kind == OP_GATEUP) return 16LL * tile;
+    if (kind == OP_QKV) {
+        const int np = (s.nq + s.nkv) * s.d / 16;
+        return tile <= np ? 16LL * tile : 16LL * np + 8LL * (tile - np);
+    }
+    return 8LL * tile;
+}
+
+MK_HD inline int tile_rows(const Shape &s, int kind, int tile) {
+    return (int)(tile_row_offset(s, kind, tile + 1) - tile_row_offset(s, kind, tile));
+}
+
+// GEMVs with K <= kRowK run one row per warp with the whole input vector in
+// registers; larger K splits columns across warps.
+constexpr int kRowK = 2048;
+constexpr int kMaxHidden = 4096;   // pair tiles in the column split hold 2 vectors per thread
+
+// Rows of one page: the largest power of two <= 8 whose rows (K bf16 each)
+// fit in a page.
 MK_HD inline int rows_per_page(int K) {
     int r = kPageBytes / (2 * K);
     int p = 1;

@@ -156,7 +156,7 @@ struct __align__(16) SmemCtl {
     uint32_t abort;             // this CTA is bailing out
     uint32_t ep;                // epoch of this launch (steps completed + 1)
     uint32_t last_flag;         // broadcast of "this task arrived last"
-    float red[2][kWorkerWarps][kTileRows];
+    float red[2][kWorkerWarps][2 * kTileRows];
     float scal[kWorkerWarps];
     float att_m[kWorkerWarps][kMaxGroup];
     float att_l[kWorkerWarps][kMaxGroup];
@@ -279,13 +279,15 @@ __device__ __forceinline__ GemvStream gemv_stream(const Params &p, const Task &t
     const int K = op_k(p.s, t.kind);
     const int rpp = rows_per_page(K);
     const long long row_bytes = 2LL * K;
+    const long long r0 = tile_row_offset(p.s, t.kind, t.begin);
+    const long long r1 = tile_row_offset(p.s, t.kind, t.end);
     GemvStream g;
-    g.src = reinterpret_cast<const char *>(gemv_base(p, t.kind, t.layer)) + (long long)t.begin * 8 * row_bytes;
-    long long rows = (long long)(t.end - t.begin) * 8;
-    if (t.kind == OP_LMHEAD) rows = min(rows, (long long)p.s.V - (long long)t.begin * 8);
+    g.src = reinterpret_cast<const char *>(gemv_base(p, t.kind, t.layer)) + r0 * row_bytes;
+    long long rows = r1 - r0;
+    if (t.kind == OP_LMHEAD) rows = min(rows, (long long)p.s.V - r0);
     g.left = rows * row_bytes;
     g.page_bytes = (uint32_t)(rpp * row_bytes);
-    g.npages = (t.end - t.begin) * (kTileRows / rpp);
+    g.npages = (int)((r1 - r0) / rpp);
     return g;
 }
 
@@ -492,10 +494,242 @@ __device__ __forceinline__ void signal_event(const Params &p, const Task &t) {
 }
 
 // ---------------------------------------------------------------------------
-// GEMV task body: tiles of 8 rows x K, NV 16-byte vectors per thread per row
+// GEMV task bodies
 // ---------------------------------------------------------------------------
-template <int NV>
-__device__ bool gemv_task(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
+// Input vector of a GEMV op (fp32 scratch, or the bf16 embedding row for the
+// first layer's QKV) and the RMSNorm gain applied to it, if any.
+struct GemvInput {
+    const float *src;
+    const uint16_t *src_bf;
+    const uint16_t *gain;
+};
+
+__device__ __forceinline__ GemvInput gemv_input(const Params &p, int kind, int layer, int b) {
+    const Shape &s = p.s;
+    GemvInput in{nullptr, nullptr, nullptr};
+    switch (kind) {
+    case OP_QKV:
+        if (layer == 0) in.src_bf = p.embed + (size_t)p.tokens[b] * s.H;
+        else in.src = p.x + (size_t)b * s.H;
+        in.gain = p.layers[layer].g_attn;
+        break;
+    case OP_GATEUP: in.src = p.x + (size_t)b * s.H; in.gain = p.layers[layer].g_mlp; break;
+    case OP_LMHEAD: in.src = p.x + (size_t)b * s.H; in.gain = p.g_final; break;
+    case OP_OPROJ: in.src = p.attn + (size_t)b * s.QD; break;
+    default: in.src = p.act + (size_t)b * s.F; break;
+    }
+    return in;
+}
+
+__device__ __forceinline__ void load_vec8(const GemvInput &in, int v, float *x) {
+    if (in.src_bf) {
+        const uint4 e = __ldg(reinterpret_cast<const uint4 *>(in.src_bf) + v);
+        x[0] = bf_lo(e.x); x[1] = bf_hi(e.x); x[2] = bf_lo(e.y); x[3] = bf_hi(e.y);
+        x[4] = bf_lo(e.z); x[5] = bf_hi(e.z); x[6] = bf_lo(e.w); x[7] = bf_hi(e.w);
+    } else {
+        const float4 a0 = __ldcg(reinterpret_cast<const float4 *>(in.src) + 2 * v);
+        const float4 a1 = __ldcg(reinterpret_cast<const float4 *>(in.src) + 2 * v + 1);
+        x[0] = a0.x; x[1] = a0.y; x[2] = a0.z; x[3] = a0.w;
+        x[4] = a1.x; x[5] = a1.y; x[6] = a1.z; x[7] = a1.w;
+    }
+}
+
+__device__ __forceinline__ void scale_vec8(float *x, float sc, const uint16_t *gain, int v) {
+    const uint4 g = __ldg(reinterpret_cast<const uint4 *>(gain) + v);
+    x[0] *= sc * bf_lo(g.x); x[1] *= sc * bf_hi(g.x); x[2] *= sc * bf_lo(g.y); x[3] *= sc * bf_hi(g.y);
+    x[4] *= sc * bf_lo(g.z); x[5] *= sc * bf_hi(g.z); x[6] *= sc * bf_lo(g.w); x[7] *= sc * bf_hi(g.w);
+}
+
+// Output of one finished row (or RoPE / gate-up pair), written by one lane.
+//   a: the row's dot product (first-half row of a pair tile);
+//   c: the partner row's (second-half q/k row, or the up row), pair tiles only.
+__device__ __forceinline__ void gemv_epilogue_row(const Params &p, int kind, int layer, int tile,
+                                                  int r, float a, float c, int b, int P,
+                                                  float &best_v, int &best_i) {
+    const Shape &s = p.s;
+    switch (kind) {
+    case OP_QKV: {
+        const int npair = (s.nq + s.nkv) * s.d / 16;
+        if (tile < npair) {
+            const int per_head = s.d / 16;
+            const int head = tile / per_head;
+            const int i = (tile % per_head) * 8 + r;
+            const float2 cs = p.rope[(size_t)P * (s.d / 2) + i];
+            const float ra = a * cs.x - c * cs.y;
+            const float rc = c * cs.x + a * cs.y;
+            if (head < s.nq) {
+                float *qh = p.q + (size_t)b * s.QD + (size_t)head * s.d;
+                qh[i] = ra;
+                qh[i + s.d / 2] = rc;
+            } else {
+                uint16_t *kh = p.layers[layer].kc + (((size_t)b * s.nkv + (head - s.nq)) * s.S + P) * s.d;
+                kh[i] = f2bf(ra);
+                kh[i + s.d / 2] = f2bf(rc);
+            }
+        } else {
+            const int row = (tile - npair) * 8 + r;
+            const int kvh = row / s.d, dd = row % s.d;
+            p.layers[layer].vc[(((size_t)b * s.nkv + kvh) * s.S + P) * s.d + dd] = f2bf(a);
+        }
+        break;
+    }
+    case OP_GATEUP:
+        p.act[(size_t)b * s.F + tile * 8 + r] = a / (1.0f + expf(-a)) * c;
+        break;
+    case OP_OPROJ: {
+        const int row = tile * 8 + r;
+        float *xp = p.x + (size_t)b * s.H + row;
+        const float resid = layer == 0 ? bf2f(p.embed[(size_t)p.tokens[b] * s.H + row]) : __ldcg(xp);
+        *xp = resid + a;
+        break;
+    }
+    case OP_DOWN: {
+        float *xp = p.x + (size_t)b * s.H + tile * 8 + r;
+        *xp = __ldcg(xp) + a;
+        break;
+    }
+    default: {  // OP_LMHEAD
+        const int row = tile * 8 + r;
+        if (row < s.V) {
+            if (p.logits) p.logits[(size_t)b * s.V + row] = a;
+            if (a > best_v || (a == best_v && row < best_i)) { best_v = a; best_i = row; }
+        }
+        break;
+    }
+    }
+}
+
+// One warp per row.  Each lane keeps NVL 8-element vectors of the input
+// (vectors lane, lane+32, ...), so a warp holds the whole input vector and
+// computes its RMSNorm itself; tiles need no cross-warp reduction.  Warp w
+// computes row w of every 8-row tile, and rows w and 8+w of a 16-row pair
+// tile (RoPE partners, or the gate and up rows of one FFN index).
+template <int NVL>
+__device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
+                          WState &w) {
+    const Shape &s = p.s;
+    const int kind = t.kind, layer = t.layer;
+    const int K = op_k(s, kind);
+    const int K8 = K >> 3;
+    const int rpp = rows_per_page(K);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = 0;
+    const size_t row_bytes = (size_t)K * 2;
+
+    const GemvInput in = gemv_input(p, kind, layer, b);
+    float xr[NVL][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+        const int v = lane + 32 * j;
+        if (v < K8) {
+            load_vec8(in, v, xr[j]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
+        }
+    }
+    if (in.gain) {
+        const float sc = 1.0f / sqrtf(warp_sum(ss) / (float)s.H + s.eps);
+#pragma unroll
+        for (int j = 0; j < NVL; ++j) {
+            const int v = lane + 32 * j;
+            if (v < K8) scale_vec8(xr[j], sc, in.gain, v);
+        }
+    }
+
+    const int P = p.positions[b];
+    float best_v = -INFINITY;
+    int best_i = 0x7fffffff;
+    for (int tile = t.begin; tile < t.end; ++tile) {
+        const int rows = tile_rows(s, kind, tile);     // 8 or 16
+        const int ra = warp, rc = 8 + warp;            // my rows in the tile
+        float acc_a = 0.f, acc_c = 0.f;
+        for (int r0 = 0; r0 < rows; r0 += rpp) {
+            uint32_t slot;
+            if (!wait_page(p, ctl, w, slot)) return false;
+            const unsigned char *page = pages + (size_t)slot * kPageBytes;
+            const bool mine_a = ra >= r0 && ra < r0 + rpp;
+            const bool mine_c = rows == 16 && rc >= r0 && rc < r0 + rpp;
+            if (mine_a || mine_c) {
+                const unsigned char *row = page + (size_t)((mine_a ? ra : rc) - r0) * row_bytes;
+                float acc = 0.f;
+#pragma unroll
+                for (int j = 0; j < NVL; ++j) {
+                    const int v = lane + 32 * j;
+                    if (v < K8) acc += dot8(ld_shared_v4(row + (size_t)v * 16), xr[j]);
+                }
+                if (mine_a) acc_a = acc;
+                else acc_c = acc;
+            }
+            release_page(ctl, w, slot);
+        }
+        acc_a = warp_sum(acc_a);
+        if (rows == 16) acc_c = warp_sum(acc_c);
+        if (lane == 0) gemv_epilogue_row(p, kind, layer, tile, warp, acc_a, acc_c, b, P, best_v, best_i);
+    }
+    if (kind == OP_LMHEAD) {
+        if (lane == 0) { ctl->att_m[warp][0] = best_v; ctl->att_l[warp][0] = __int_as_float(best_i); }
+        if (!worker_sync(p, ctl, w)) return false;
+        if (threadIdx.x == 0) {
+            for (int k = 1; k < kWorkerWarps; ++k) {
+                const float v = ctl->att_m[k][0];
+                const int i = __float_as_int(ctl->att_l[k][0]);
+                if (v > best_v || (v == best_v && i < best_i)) { best_v = v; best_i = i; }
+            }
+            p.amax_val[(size_t)b * p.num_lm_tasks + t.slot] = best_v;
+            p.amax_idx[(size_t)b * p.num_lm_tasks + t.slot] = best_i;
+        }
+    }
+    return true;
+}
+
+// Column split, for K > kRowK: thread t owns 16-byte vectors t, t+256, ...
+// of every row of a tile (up to RMAX rows: 8, or 16 for pair tiles); per
+// tile the partial sums are reduced across lanes, then across warps through
+// shared memory, and warp 0's lanes 0..7 run the epilogues.
+template <int RMAX>
+__device__ __forceinline__ float warp_reduce_rows(const float (&acc)[RMAX], int lane);
+
+template <>
+__device__ __forceinline__ float warp_reduce_rows<8>(const float (&acc)[8], int lane) {
+    return warp_reduce_rows8(acc, lane);   // lane holds row (lane >> 2) & 7
+}
+
+// 16 partial sums over 32 lanes; afterwards lane holds row (lane >> 1) & 15.
+template <>
+__device__ __forceinline__ float warp_reduce_rows<16>(const float (&acc)[16], int lane) {
+    float b0[8], b1[4], b2[2];
+    const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4, u2 = lane & 2;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float send = u16 ? acc[i] : acc[i + 8];
+        const float keep = u16 ? acc[i + 8] : acc[i];
+        b0[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = u8 ? b0[i] : b0[i + 4];
+        const float keep = u8 ? b0[i + 4] : b0[i];
+        b1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = u4 ? b1[i] : b1[i + 2];
+        const float keep = u4 ? b1[i + 2] : b1[i];
+        b2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    const float send = u2 ? b2[0] : b2[1];
+    const float keep = u2 ? b2[1] : b2[0];
+    float c = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    c += __shfl_xor_sync(0xffffffffu, c, 1);
+    return c;
+}
+
+template <int NV, int RMAX>
+__device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                           WState &w) {
     const Shape &s = p.s;
     const int kind = t.kind, layer = t.layer;
@@ -504,38 +738,14 @@ __device__ bool gemv_task(const Params &p, const Task &t, unsigned char *pages, 
     const int rpp = rows_per_page(K);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = 0;
-
-    // ---- the task's input vector slice, normalised if the op has a norm
-    const float *src = nullptr;
-    const uint16_t *src_bf = nullptr;
-    const uint16_t *gain = nullptr;
-    switch (kind) {
-    case OP_QKV:
-        if (layer == 0) src_bf = p.embed + (size_t)p.tokens[b] * s.H;
-        else src = p.x + (size_t)b * s.H;
-        gain = p.layers[layer].g_attn;
-        break;
-    case OP_GATEUP: src = p.x + (size_t)b * s.H; gain = p.layers[layer].g_mlp; break;
-    case OP_LMHEAD: src = p.x + (size_t)b * s.H; gain = p.g_final; break;
-    case OP_OPROJ: src = p.attn + (size_t)b * s.QD; break;
-    default: src = p.act + (size_t)b * s.F; break;
-    }
+    const GemvInput in = gemv_input(p, kind, layer, b);
     float xr[NV][8];
     float ss = 0.f;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
         const int v = tid + j * kWorkerThreads;
         if (v < K8) {
-            if (src_bf) {
-                uint4 e = __ldg(reinterpret_cast<const uint4 *>(src_bf) + v);
-                xr[j][0] = bf_lo(e.x); xr[j][1] = bf_hi(e.x); xr[j][2] = bf_lo(e.y); xr[j][3] = bf_hi(e.y);
-                xr[j][4] = bf_lo(e.z); xr[j][5] = bf_hi(e.z); xr[j][6] = bf_lo(e.w); xr[j][7] = bf_hi(e.w);
-            } else {
-                float4 a0 = __ldcg(reinterpret_cast<const float4 *>(src) + 2 * v);
-                float4 a1 = __ldcg(reinterpret_cast<const float4 *>(src) + 2 * v + 1);
-                xr[j][0] = a0.x; xr[j][1] = a0.y; xr[j][2] = a0.z; xr[j][3] = a0.w;
-                xr[j][4] = a1.x; xr[j][5] = a1.y; xr[j][6] = a1.z; xr[j][7] = a1.w;
-            }
+            load_vec8(in, v, xr[j]);
 #pragma unroll
             for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
         } else {
@@ -543,136 +753,69 @@ __device__ bool gemv_task(const Params &p, const Task &t, unsigned char *pages, 
             for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
         }
     }
-    if (gain) {
+    if (in.gain) {
         float tot;
         if (!worker_block_sum(p, ctl, w, ss, tot)) return false;
         const float sc = 1.0f / sqrtf(tot / (float)s.H + s.eps);
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
             const int v = tid + j * kWorkerThreads;
-            if (v < K8) {
-                uint4 g = __ldg(reinterpret_cast<const uint4 *>(gain) + v);
-                xr[j][0] *= sc * bf_lo(g.x); xr[j][1] *= sc * bf_hi(g.x);
-                xr[j][2] *= sc * bf_lo(g.y); xr[j][3] *= sc * bf_hi(g.y);
-                xr[j][4] *= sc * bf_lo(g.z); xr[j][5] *= sc * bf_hi(g.z);
-                xr[j][6] *= sc * bf_lo(g.w); xr[j][7] *= sc * bf_hi(g.w);
-            }
+            if (v < K8) scale_vec8(xr[j], sc, in.gain, v);
         }
     }
-
-    // ---- tiles
     const int P = p.positions[b];
     float best_v = -INFINITY;
-    int best_i = 0;
+    int best_i = 0x7fffffff;
     const size_t row_bytes = (size_t)K * 2;
+    constexpr int kLanesPerRow = 32 / RMAX;   // lanes holding one row after the reduction
     for (int tile = t.begin; tile < t.end; ++tile) {
-        float acc[8];
+        const int rows = RMAX == 16 ? tile_rows(s, kind, tile) : 8;
+        float acc[RMAX];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+        for (int r = 0; r < RMAX; ++r) acc[r] = 0.f;
         uint32_t slot = 0;
         const unsigned char *page = pages;
 #pragma unroll
-        for (int r = 0; r < kTileRows; ++r) {
-            if ((r & (rpp - 1)) == 0) {
-                if (!wait_page(p, ctl, w, slot)) return false;
-                page = pages + (size_t)slot * kPageBytes;
-            }
-            const unsigned char *row = page + (size_t)(r & (rpp - 1)) * row_bytes;
+        for (int r = 0; r < RMAX; ++r) {
+            if (r < rows) {
+                if ((r & (rpp - 1)) == 0) {
+                    if (!wait_page(p, ctl, w, slot)) return false;
+                    page = pages + (size_t)slot * kPageBytes;
+                }
+                const unsigned char *row = page + (size_t)(r & (rpp - 1)) * row_bytes;
 #pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                const int v = tid + j * kWorkerThreads;
-                if (v < K8) acc[r] += dot8(ld_shared_v4(row + (size_t)v * 16), xr[j]);
+                for (int j = 0; j < NV; ++j) {
+                    const int v = tid + j * kWorkerThreads;
+                    if (v < K8) acc[r] += dot8(ld_shared_v4(row + (size_t)v * 16), xr[j]);
+                }
+                if (((r + 1) & (rpp - 1)) == 0) release_page(ctl, w, slot);
             }
-            if (((r + 1) & (rpp - 1)) == 0) release_page(ctl, w, slot);
         }
-        const float rsum = warp_reduce_rows8(acc, lane);
-        if ((lane & 3) == 0) ctl->red[w.red_buf][warp][(lane >> 2) & 7] = rsum;
+        const float rsum = warp_reduce_rows<RMAX>(acc, lane);
+        if ((lane & (kLanesPerRow - 1)) == 0) ctl->red[w.red_buf][warp][lane / kLanesPerRow] = rsum;
         if (!worker_sync(p, ctl, w)) return false;
-        if (tid < 8) {
-            const float(*red)[kTileRows] = ctl->red[w.red_buf];
-            auto rs = [&](int r) {
-                float a = 0.f;
+        if (warp == 0 && lane < 8) {
+            float a = 0.f, c = 0.f;
 #pragma unroll
-                for (int i = 0; i < kWorkerWarps; ++i) a += red[i][r];
-                return a;
-            };
-            switch (kind) {
-            case OP_QKV: {
-                const int npair = (s.nq + s.nkv) * s.d / 8;
-                if (tile < npair) {
-                    if (tid < 4) {
-                        const int per_head = s.d / 8;
-                        const int head = tile / per_head;
-                        const int i = (tile % per_head) * 4 + tid;
-                        const float a = rs(tid), c = rs(tid + 4);
-                        const float2 cs = p.rope[(size_t)P * (s.d / 2) + i];
-                        const float ra = a * cs.x - c * cs.y;
-                        const float rc = c * cs.x + a * cs.y;
-                        if (head < s.nq) {
-                            float *qh = p.q + (size_t)b * s.QD + (size_t)head * s.d;
-                            qh[i] = ra;
-                            qh[i + s.d / 2] = rc;
-                        } else {
-                            const LayerW &L = p.layers[layer];
-                            uint16_t *kh = L.kc + (((size_t)b * s.nkv + (head - s.nq)) * s.S + P) * s.d;
-                            kh[i] = f2bf(ra);
-                            kh[i + s.d / 2] = f2bf(rc);
-                        }
-                    }
-                } else {
-                    const int row = (tile - npair) * 8 + tid;
-                    const int kvh = row / s.d, dd = row % s.d;
-                    const LayerW &L = p.layers[layer];
-                    L.vc[(((size_t)b * s.nkv + kvh) * s.S + P) * s.d + dd] = f2bf(rs(tid));
-                }
-                break;
+            for (int i = 0; i < kWorkerWarps; ++i) {
+                a += ctl->red[w.red_buf][i][lane];
+                if (RMAX == 16) c += ctl->red[w.red_buf][i][8 + lane];
             }
-            case OP_OPROJ: {
-                const int row = tile * 8 + tid;
-                float *xp = p.x + (size_t)b * s.H + row;
-                const float resid = layer == 0 ? bf2f(p.embed[(size_t)p.tokens[b] * s.H + row]) : __ldcg(xp);
-                *xp = resid + rs(tid);
-                break;
-            }
-            case OP_GATEUP:
-                if (tid < 4) {
-                    const float g = rs(tid), u = rs(tid + 4);
-                    p.act[(size_t)b * s.F + tile * 4 + tid] = g / (1.0f + expf(-g)) * u;
-                }
-                break;
-            case OP_DOWN: {
-                const int row = tile * 8 + tid;
-                float *xp = p.x + (size_t)b * s.H + row;
-                *xp = __ldcg(xp) + rs(tid);
-                break;
-            }
-            default: {  // OP_LMHEAD
-                const int row = tile * 8 + tid;
-                float val = -INFINITY;
-                if (row < s.V) {
-                    val = rs(tid);
-                    if (p.logits) p.logits[(size_t)b * s.V + row] = val;
-                }
-                int idx = row;
-#pragma unroll
-                for (int o = 4; o > 0; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffu, val, o);
-                    const int oi = __shfl_xor_sync(0xffu, idx, o);
-                    if (ov > val || (ov == val && oi < idx)) { val = ov; idx = oi; }
-                }
-                if (tid == 0 && (val > best_v || (val == best_v && idx < best_i))) {
-                    best_v = val;
-                    best_i = idx;
-                }
-                break;
-            }
-            }
+            gemv_epilogue_row(p, kind, layer, tile, lane, a, c, b, P, best_v, best_i);
         }
         w.red_buf ^= 1;
     }
-    if (kind == OP_LMHEAD && tid == 0) {
-        p.amax_val[(size_t)b * p.num_lm_tasks + t.slot] = best_v;
-        p.amax_idx[(size_t)b * p.num_lm_tasks + t.slot] = best_i;
+    if (kind == OP_LMHEAD && warp == 0 && lane < 8) {
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffu, best_v, o);
+            const int oi = __shfl_xor_sync(0xffu, best_i, o);
+            if (ov > best_v || (ov == best_v && oi < best_i)) { best_v = ov; best_i = oi; }
+        }
+        if (lane == 0) {
+            p.amax_val[(size_t)b * p.num_lm_tasks + t.slot] = best_v;
+            p.amax_idx[(size_t)b * p.num_lm_tasks + t.slot] = best_i;
+        }
     }
     return true;
 }
@@ -843,16 +986,23 @@ __device__ bool run_task(const Params &p, const Task &t, unsigned char *pages, S
         }
     }
     const int K = op_k(p.s, t.kind);
-    const int nv = (K / 8 + kWorkerThreads - 1) / kWorkerThreads;
-    switch (nv) {
-    case 1: return gemv_task<1>(p, t, pages, ctl, w);
-    case 2: return gemv_task<2>(p, t, pages, ctl, w);
-    case 3: return gemv_task<3>(p, t, pages, ctl, w);
-    case 4: return gemv_task<4>(p, t, pages, ctl, w);
-    case 5: return gemv_task<5>(p, t, pages, ctl, w);
-    case 6: return gemv_task<6>(p, t, pages, ctl, w);
-    case 7: return gemv_task<7>(p, t, pages, ctl, w);
-    default: return gemv_task<8>(p, t, pages, ctl, w);
+    if (K <= kRowK) {
+        switch ((K / 8 + 31) / 32) {   // 16-byte vectors per lane
+        case 1: return gemv_rows<1>(p, t, pages, ctl, w);
+        case 2: return gemv_rows<2>(p, t, pages, ctl, w);
+        case 3: return gemv_rows<3>(p, t, pages, ctl, w);
+        case 4: return gemv_rows<4>(p, t, pages, ctl, w);
+        case 5: case 6: return gemv_rows<6>(p, t, pages, ctl, w);
+        default: return gemv_rows<8>(p, t, pages, ctl, w);
+        }
+    }
+    if (t.kind == OP_QKV || t.kind == OP_GATEUP)   // K = hidden <= kMaxHidden
+        return gemv_cols<2, 16>(p, t, pages, ctl, w);
+    switch ((K / 8 + kWorkerThreads - 1) / kWorkerThreads) {
+    case 1: case 2: return gemv_cols<2, 8>(p, t, pages, ctl, w);
+    case 3: case 4: return gemv_cols<4, 8>(p, t, pages, ctl, w);
+    case 5: case 6: return gemv_cols<6, 8>(p, t, pages, ctl, w);
+    default: return gemv_cols<8, 8>(p, t, pages, ctl, w);
     }
 }
 

@@ -64,6 +64,7 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     const int G = c->n_q_heads / c->n_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return MK_ERR_INVALID;
     if (c->head_dim != 64 && c->head_dim != 128) return MK_ERR_INVALID;
+    if (c->hidden > kMaxHidden) return MK_ERR_INVALID;
     if (G * c->head_dim > 512) return MK_ERR_INVALID;
     const long long QD = (long long)c->n_q_heads * c->head_dim;
     if (c->hidden % 8 || c->ffn % 8 || QD % 8) return MK_ERR_INVALID;
@@ -248,11 +249,11 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     TraceRec *d_trace = nullptr;
     if (cfg->flags & MK_FLAG_TRACE) MK_TRY(dalloc(c, &d_trace, c->num_tasks));
 
-    // ---- repack q/k/v and gate/up into tile order (see LayerW)
+    // ---- repack q/k/v and gate/up into tile order (see LayerW / OpTiles)
     {
         const size_t rb = 2 * (size_t)s.H;          // bytes of one row of K = H
-        const size_t tile = 8 * rb;
-        const int per_head = s.d / 8;
+        const size_t tile = 16 * rb;                 // one pair tile
+        const int per_head = s.d / 16;               // pair tiles per head
         for (int l = 0; l < s.L; ++l) {
             uint16_t *qkv, *gu;
             MK_TRY(dalloc(c, &qkv, (size_t)(s.QD + 2 * s.KD) * s.H));
@@ -262,19 +263,20 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
                 const char *src = h < s.nq ? (const char *)w->wq[l] + (size_t)h * s.d * rb
                                            : (const char *)w->wk[l] + (size_t)(h - s.nq) * s.d * rb;
                 char *dst = dq + (size_t)h * per_head * tile;
-                MK_TRY(cudaMemcpy2D(dst, tile, src, 4 * rb, 4 * rb, per_head, cudaMemcpyDeviceToDevice));
-                MK_TRY(cudaMemcpy2D(dst + 4 * rb, tile, src + (size_t)(s.d / 2) * rb, 4 * rb, 4 * rb,
+                MK_TRY(cudaMemcpy2D(dst, tile, src, 8 * rb, 8 * rb, per_head, cudaMemcpyDeviceToDevice));
+                MK_TRY(cudaMemcpy2D(dst + 8 * rb, tile, src + (size_t)(s.d / 2) * rb, 8 * rb, 8 * rb,
                                     per_head, cudaMemcpyDeviceToDevice));
             }
             MK_TRY(cudaMemcpy(dq + (size_t)(s.nq + s.nkv) * per_head * tile, w->wv[l],
                               (size_t)s.KD * rb, cudaMemcpyDeviceToDevice));
-            MK_TRY(cudaMemcpy2D(gu, tile, w->wg[l], 4 * rb, 4 * rb, s.F / 4, cudaMemcpyDeviceToDevice));
-            MK_TRY(cudaMemcpy2D((char *)gu + 4 * rb, tile, w->wu[l], 4 * rb, 4 * rb, s.F / 4,
+            MK_TRY(cudaMemcpy2D(gu, tile, w->wg[l], 8 * rb, 8 * rb, s.F / 8, cudaMemcpyDeviceToDevice));
+            MK_TRY(cudaMemcpy2D((char *)gu + 8 * rb, tile, w->wu[l], 8 * rb, 8 * rb, s.F / 8,
                                 cudaMemcpyDeviceToDevice));
             lw[l].qkv = qkv;
             lw[l].gu = gu;
         }
     }
+    MK_TRY(cudaDeviceSynchronize());
 
     MK_TRY(cudaMemcpy(d_tasks, c->h_tasks.data(), sizeof(Task) * c->num_tasks, cudaMemcpyHostToDevice));
     MK_TRY(cudaMemcpy(d_queue, c->h_queue.data(), sizeof(int32_t) * c->num_tasks, cudaMemcpyHostToDevice));

@@ -36,8 +36,10 @@ def test_status_strings():
 
 def _tiles(shape):
     d, H, F, V = shape.head_dim, shape.hidden, shape.ffn, shape.vocab
-    return {QKV: (shape.n_q_heads + shape.n_kv_heads) * d // 8 + shape.n_kv_heads * d // 8,
-            OPROJ: H // 8, GATEUP: F // 4, DOWN: H // 8, LMHEAD: (V + 7) // 8}
+    # q/k tiles hold 8 RoPE pairs (16 rows), value tiles 8 rows, gate/up tiles
+    # 8 gate + 8 up rows, the others 8 rows
+    return {QKV: (shape.n_q_heads + shape.n_kv_heads) * d // 16 + shape.n_kv_heads * d // 8,
+            OPROJ: H // 8, GATEUP: F // 8, DOWN: H // 8, LMHEAD: (V + 7) // 8}
 
 
 CASES = [("tiny", wl.TINY, 64), ("1b", wl.LLAMA_1B, 560), ("8b", wl.LLAMA_8B, 560),
@@ -142,7 +144,7 @@ def test_schedule_runs_to_completion_with_exact_event_counts(planned):
 
 @pytest.mark.parametrize("bad", [
     dict(head_dim=96), dict(n_q_heads=12, n_kv_heads=4), dict(hidden=2044),
-    dict(ffn=20000), dict(max_batch=99), dict(vocab=0), dict(max_seq=0),
+    dict(ffn=20000), dict(max_batch=99), dict(vocab=0), dict(max_seq=0), dict(hidden=8192),
 ])
 def test_plan_rejects_unsupported_shapes(bad):
     base = dict(layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=768,
