@@ -211,6 +211,13 @@ enum mk_op_kind { MK_OP_QKV = 0, MK_OP_ATTN = 1, MK_OP_OPROJ = 2, MK_OP_GATEUP =
                   MK_OP_DOWN = 4, MK_OP_LMHEAD = 5 };
 int mk_get_trace(mk_ctx *ctx, mk_trace_rec *host_out, int n);
 
+/* Per-SM wait accounting of the last step (MK_FLAG_TRACE): uint64
+ * [num_sms][8] = {loader ns waiting for a free page, pages issued, loader
+ * ns total, worker ns waiting for loaded pages, worker ns waiting for the
+ * scheduler, worker ns in worker barriers, worker ns total, scheduler ns
+ * waiting on event counters} (the worker figures are those of warp 0). */
+int mk_get_sm_stats(mk_ctx *ctx, uint64_t *host_out, int n);
+
 /* Static task graph as built by mk_create (host copy).  task_out: int32
  * [num_tasks][8] = {kind, layer, dep_event (-1 none), trig_event, begin,
  * end, sm, slot}; queue_out: int32 [num_tasks] task ids grouped by SM in

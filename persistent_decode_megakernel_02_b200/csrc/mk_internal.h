@@ -146,6 +146,19 @@ struct ErrWord {
     uint32_t info;    // extra (event index, bad value)
 };
 
+// Per-SM wait accounting (trace mode), in globaltimer ns unless noted.
+enum StatSlot {
+    ST_LOADER_EMPTY = 0,  // loader waiting for a free page
+    ST_LOADER_PAGES = 1,  // pages issued (count)
+    ST_LOADER_TOTAL = 2,  // loader role start to end
+    ST_WORKER_FULL = 3,   // worker warp 0 waiting for a loaded page
+    ST_WORKER_READY = 4,  // worker warp 0 waiting for the scheduler
+    ST_WORKER_SYNC = 5,   // worker warp 0 in worker barriers
+    ST_WORKER_TOTAL = 6,  // worker role start to end
+    ST_SCHED_DEP = 7,     // scheduler waiting on event counters
+    kStatSlots = 8
+};
+
 struct TraceRec {
     unsigned long long t_ready, t_start, t_end;
     int32_t sm, kind, layer, trig;
@@ -186,6 +199,7 @@ struct Params {
     // control
     ErrWord *err;                // device view of mapped host memory
     TraceRec *trace;             // null unless tracing
+    unsigned long long *sm_stats; // [num_sms][kStatSlots] wait times (ns), null unless tracing
     unsigned long long timeout_ns;
     int l2_prefetch;
 };

@@ -296,6 +296,8 @@ __device__ __forceinline__ GemvStream gemv_stream(const Params &p, const Task &t
 // ---------------------------------------------------------------------------
 struct Ring {
     uint32_t seq = 0;     // pages issued
+    bool stats = false;
+    unsigned long long t_empty = 0;
 };
 
 // Wait for a free page, then arm its full barrier for `bytes`.
@@ -303,7 +305,10 @@ __device__ __forceinline__ bool ring_acquire(const Params &p, SmemCtl *ctl, Ring
                                              uint32_t task, uint32_t &slot) {
     slot = r.seq % kNumPages;
     const uint32_t par = ((r.seq / kNumPages) & 1u) ^ 1u;
-    if (!wait_mbar(&ctl->empty[slot], par, p, ctl, W_EMPTY, task)) return false;
+    const unsigned long long t0 = r.stats ? globaltimer() : 0ull;
+    const bool ok = wait_mbar(&ctl->empty[slot], par, p, ctl, W_EMPTY, task);
+    if (r.stats) r.t_empty += globaltimer() - t0;
+    if (!ok) return false;
     mbar_arrive_expect_tx(&ctl->full[slot], bytes);
     ++r.seq;
     return true;
@@ -341,6 +346,8 @@ struct Prefetcher {
 __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     Ring ring;
+    ring.stats = p.sm_stats != nullptr;
+    const unsigned long long t_begin = ring.stats ? globaltimer() : 0ull;
     Prefetcher pf(q0, q1);
     long long issued = 0;   // GEMV bytes copied into the ring so far
     bool ok = true;         // false when a wait was abandoned
@@ -390,6 +397,12 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
             }
         }
     }
+    if (ring.stats) {
+        unsigned long long *st = p.sm_stats + (size_t)blockIdx.x * kStatSlots;
+        st[ST_LOADER_EMPTY] = ring.t_empty;
+        st[ST_LOADER_PAGES] = ring.seq;
+        st[ST_LOADER_TOTAL] = globaltimer() - t_begin;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -397,18 +410,22 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
 // ---------------------------------------------------------------------------
 __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
+    unsigned long long t_dep = 0;
     for (int qi = q0; qi < q1; ++qi) {
         const int id = p.queue[qi];
         const int dep = p.tasks[id].dep;
         if (dep >= 0) {
             const uint32_t target = p.thresholds[dep] * ep;
             Spin s;
+            const unsigned long long t0 = p.sm_stats ? globaltimer() : 0ull;
             while ((int32_t)(ld_acquire_gpu(&p.events[dep]) - target) < 0)
                 if (!spin_ok(s, p, ctl, W_DEP, (uint32_t)id, (uint32_t)dep)) return;
+            if (p.sm_stats) t_dep += globaltimer() - t0;
         }
         if (p.trace) p.trace[id].t_ready = globaltimer();
         st_release_cta_shared(&ctl->ready_upto, (uint32_t)(qi - q0 + 1));
     }
+    if (p.sm_stats) p.sm_stats[(size_t)blockIdx.x * kStatSlots + ST_SCHED_DEP] = t_dep;
 }
 
 // ---------------------------------------------------------------------------
@@ -419,21 +436,28 @@ struct WState {
     uint32_t wphase = 0;     // worker-barrier phase
     int red_buf = 0;
     int task_id = 0;
+    bool stats = false;      // accumulate wait times (trace mode)
+    unsigned long long t_full = 0, t_ready = 0, t_sync = 0;
 };
 
 // All worker warps meet; bounded.
 __device__ __forceinline__ bool worker_sync(const Params &p, SmemCtl *ctl, WState &w) {
     __syncwarp();
+    const unsigned long long t0 = w.stats ? globaltimer() : 0ull;
     if ((threadIdx.x & 31) == 0) mbar_arrive(&ctl->wbar);
     bool ok = wait_mbar(&ctl->wbar, w.wphase, p, ctl, W_WBAR, (uint32_t)w.task_id);
     w.wphase ^= 1u;
+    if (w.stats) w.t_sync += globaltimer() - t0;
     return ok;
 }
 
 __device__ __forceinline__ bool wait_page(const Params &p, SmemCtl *ctl, WState &w, uint32_t &slot) {
     slot = w.page_seq % kNumPages;
-    return wait_mbar(&ctl->full[slot], (w.page_seq / kNumPages) & 1u, p, ctl, W_FULL,
-                     (uint32_t)w.task_id);
+    const unsigned long long t0 = w.stats ? globaltimer() : 0ull;
+    const bool ok = wait_mbar(&ctl->full[slot], (w.page_seq / kNumPages) & 1u, p, ctl, W_FULL,
+                              (uint32_t)w.task_id);
+    if (w.stats) w.t_full += globaltimer() - t0;
+    return ok;
 }
 
 __device__ __forceinline__ void release_page(SmemCtl *ctl, WState &w, uint32_t slot) {
@@ -1010,6 +1034,8 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     const int tid = threadIdx.x;
     WState w;
+    w.stats = p.sm_stats != nullptr && tid == 0;
+    const unsigned long long t_begin = w.stats ? globaltimer() : 0ull;
     for (int qi = q0; qi < q1; ++qi) {
         const int id = p.queue[qi];
         const Task t = p.tasks[id];
@@ -1017,8 +1043,10 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         {
             Spin s;
             const uint32_t need = (uint32_t)(qi - q0 + 1);
+            const unsigned long long t0 = w.stats ? globaltimer() : 0ull;
             while (ld_acquire_cta_shared(&ctl->ready_upto) < need)
                 if (!spin_ok(s, p, ctl, W_READY, (uint32_t)id, 0u)) return;
+            if (w.stats) w.t_ready += globaltimer() - t0;
         }
         if (p.trace && tid == 0) p.trace[id].t_start = globaltimer();
         if (!run_task(p, t, pages, ctl, w)) return;
@@ -1056,6 +1084,13 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
             if (tid == 0) signal_event(p, t);
         }
         if (p.trace && tid == 0) p.trace[id].t_end = globaltimer();
+    }
+    if (w.stats) {
+        unsigned long long *st = p.sm_stats + (size_t)blockIdx.x * kStatSlots;
+        st[ST_WORKER_FULL] = w.t_full;
+        st[ST_WORKER_READY] = w.t_ready;
+        st[ST_WORKER_SYNC] = w.t_sync;
+        st[ST_WORKER_TOTAL] = globaltimer() - t_begin;
     }
 }
 

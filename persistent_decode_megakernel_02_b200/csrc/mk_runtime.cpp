@@ -247,7 +247,12 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     MK_TRY(dalloc(c, &d_aval, B * c->num_lm_tasks));
     MK_TRY(dalloc(c, &d_aidx, B * c->num_lm_tasks));
     TraceRec *d_trace = nullptr;
-    if (cfg->flags & MK_FLAG_TRACE) MK_TRY(dalloc(c, &d_trace, c->num_tasks));
+    unsigned long long *d_stats = nullptr;
+    if (cfg->flags & MK_FLAG_TRACE) {
+        MK_TRY(dalloc(c, &d_trace, c->num_tasks));
+        MK_TRY(dalloc(c, &d_stats, (size_t)c->num_sms * kStatSlots));
+        MK_TRY(cudaMemset(d_stats, 0, sizeof(unsigned long long) * c->num_sms * kStatSlots));
+    }
 
     // ---- repack q/k/v and gate/up into tile order (see LayerW / OpTiles)
     {
@@ -318,6 +323,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     p.amax_val = d_aval; p.amax_idx = d_aidx;
     p.err = c->d_err;
     p.trace = d_trace;
+    p.sm_stats = d_stats;
     p.timeout_ns = cfg->timeout_ns > 0 ? (unsigned long long)cfg->timeout_ns : 2000000000ull;
     p.l2_prefetch = (cfg->flags & MK_FLAG_NO_L2_PREFETCH) ? 0 : 1;
     *out = c;
@@ -434,6 +440,14 @@ int mk_get_trace(mk_ctx *c, mk_trace_rec *host_out, int n) {
     if (!c->p.trace) return MK_ERR_INVALID;
     static_assert(sizeof(mk_trace_rec) == sizeof(TraceRec), "trace record layout");
     if (cudaMemcpy(host_out, c->p.trace, sizeof(TraceRec) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MK_ERR_CUDA;
+    return MK_OK;
+}
+
+int mk_get_sm_stats(mk_ctx *c, uint64_t *host_out, int n) {
+    if (!c || !host_out || n < 0 || n > c->num_sms * kStatSlots) return MK_ERR_INVALID;
+    if (!c->p.sm_stats) return MK_ERR_INVALID;
+    if (cudaMemcpy(host_out, c->p.sm_stats, sizeof(uint64_t) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
         return MK_ERR_CUDA;
     return MK_OK;
 }

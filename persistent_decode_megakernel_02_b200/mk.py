@@ -83,10 +83,12 @@ _lib.mk_get_event_counts.argtypes = [_P, _P, _P, C.c_int]
 _lib.mk_read_buffer.argtypes = [_P, C.c_int, _P, C.c_size_t]
 _lib.mk_get_trace.argtypes = [_P, _P, C.c_int]
 _lib.mk_get_graph.argtypes = [_P, _P, _P, _P]
+_lib.mk_get_sm_stats.argtypes = [_P, _P, C.c_int]
 _lib.mk_plan.argtypes = [C.POINTER(Config), C.c_int, C.POINTER(Info), _P, _P, _P, _P, _P]
 _lib.mk_debug_set_threshold.argtypes = [_P, C.c_int, C.c_uint]
 for _f in ("mk_create", "mk_decode_step", "mk_sync", "mk_reset", "mk_destroy", "mk_get_info",
            "mk_get_event_counts", "mk_read_buffer", "mk_get_trace", "mk_get_graph", "mk_plan",
+           "mk_get_sm_stats",
            "mk_debug_set_threshold"):
     getattr(_lib, _f).restype = C.c_int
 
@@ -233,6 +235,16 @@ class Context:
                        ("sm", np.int32), ("kind", np.int32), ("layer", np.int32),
                        ("trig_event", np.int32)])
         return np.frombuffer(bytes(recs), dtype=dt).copy()
+
+    STAT_NAMES = ["loader_empty_ns", "loader_pages", "loader_total_ns", "worker_full_ns",
+                  "worker_ready_ns", "worker_sync_ns", "worker_total_ns", "sched_dep_ns"]
+
+    def sm_stats(self) -> np.ndarray:
+        """Per-SM wait accounting of the last step (trace mode): [num_sms][8]."""
+        n = self.info().num_sms
+        out = np.zeros((n, 8), np.uint64)
+        _check(_lib.mk_get_sm_stats(self._h, out.ctypes.data, n * 8), "mk_get_sm_stats")
+        return out
 
     def graph(self) -> dict:
         i = self.info()
