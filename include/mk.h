@@ -211,11 +211,15 @@ enum mk_op_kind { MK_OP_QKV = 0, MK_OP_ATTN = 1, MK_OP_OPROJ = 2, MK_OP_GATEUP =
                   MK_OP_DOWN = 4, MK_OP_LMHEAD = 5 };
 int mk_get_trace(mk_ctx *ctx, mk_trace_rec *host_out, int n);
 
-/* Per-SM wait accounting of the last step (MK_FLAG_TRACE): uint64
- * [num_sms][8] = {loader ns waiting for a free page, pages issued, loader
+/* Per-SM time accounting of the last step (MK_FLAG_TRACE): uint64
+ * [num_sms][16] = {loader ns waiting for a free page, pages issued, loader
  * ns total, worker ns waiting for loaded pages, worker ns waiting for the
  * scheduler, worker ns in worker barriers, worker ns total, scheduler ns
- * waiting on event counters} (the worker figures are those of warp 0). */
+ * waiting on event counters, worker ns in task prologues (input vector
+ * load, RMSNorm), worker ns in dot products, worker ns in per-tile
+ * reductions and epilogues, worker ns in task ends (barrier, fence, event,
+ * merges), tasks run, 3 unused}.  Worker figures are those of warp 0 and
+ * some phases overlap the waits they contain. */
 int mk_get_sm_stats(mk_ctx *ctx, uint64_t *host_out, int n);
 
 /* Static task graph as built by mk_create (host copy).  task_out: int32

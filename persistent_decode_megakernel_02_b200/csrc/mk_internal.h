@@ -156,7 +156,12 @@ enum StatSlot {
     ST_WORKER_SYNC = 5,   // worker warp 0 in worker barriers
     ST_WORKER_TOTAL = 6,  // worker role start to end
     ST_SCHED_DEP = 7,     // scheduler waiting on event counters
-    kStatSlots = 8
+    ST_WORKER_PROLOGUE = 8,  // worker warp 0: task start to its first page (input load, norm)
+    ST_WORKER_DOT = 9,       // worker warp 0: dot products on loaded pages
+    ST_WORKER_EPI = 10,      // worker warp 0: per-tile reductions and epilogues
+    ST_WORKER_END = 11,      // worker warp 0: task end (barrier, fence, event, merges)
+    ST_WORKER_TASKS = 12,    // tasks run (count)
+    kStatSlots = 16
 };
 
 struct TraceRec {

@@ -89,6 +89,9 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
 __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
+__device__ __forceinline__ void prefetch_l1(const void *p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -161,6 +164,7 @@ struct __align__(16) SmemCtl {
     float att_m[kWorkerWarps][kMaxGroup];
     float att_l[kWorkerWarps][kMaxGroup];
     float att_o[kWorkerWarps][kAttnCombine];
+    unsigned long long wstat[8];   // trace-mode time accounting of worker thread 0
 };
 constexpr size_t kSmemBytes = (size_t)kNumPages * kPageBytes + sizeof(SmemCtl);
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -432,38 +436,58 @@ __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
 // worker helpers
 // ---------------------------------------------------------------------------
 struct WState {
-    uint32_t page_seq = 0;   // pages consumed
+    uint32_t slot = 0;       // ring slot of the next page to consume
+    uint32_t phase = 0;      // its full-barrier parity
     uint32_t wphase = 0;     // worker-barrier phase
+    uint32_t need = 0;       // ready_upto value that activates the current task
     int red_buf = 0;
     int task_id = 0;
-    bool stats = false;      // accumulate wait times (trace mode)
-    unsigned long long t_full = 0, t_ready = 0, t_sync = 0;
+    unsigned long long *stat = nullptr;   // per-phase accumulators in shared memory (trace mode, thread 0)
 };
+// Trace-mode time accounting of worker thread 0, accumulated in shared memory
+// so it costs no registers across the task bodies.
+enum WStat { WS_FULL = 0, WS_READY, WS_SYNC, WS_PRO, WS_DOT, WS_EPI, WS_END, WS_TASKS, kWStats };
+__device__ __forceinline__ unsigned long long phase_begin(const WState &w) {
+    return w.stat ? globaltimer() : 0ull;
+}
+__device__ __forceinline__ void phase_end(const WState &w, unsigned long long t0, int which) {
+    if (w.stat) w.stat[which] += globaltimer() - t0;
+}
 
 // All worker warps meet; bounded.
 __device__ __forceinline__ bool worker_sync(const Params &p, SmemCtl *ctl, WState &w) {
     __syncwarp();
-    const unsigned long long t0 = w.stats ? globaltimer() : 0ull;
+    const unsigned long long t0 = phase_begin(w);
     if ((threadIdx.x & 31) == 0) mbar_arrive(&ctl->wbar);
     bool ok = wait_mbar(&ctl->wbar, w.wphase, p, ctl, W_WBAR, (uint32_t)w.task_id);
     w.wphase ^= 1u;
-    if (w.stats) w.t_sync += globaltimer() - t0;
+    phase_end(w, t0, WS_SYNC);
     return ok;
 }
 
+// Wait until the scheduler has activated the current task (its dependent
+// event fired); bounded.
+__device__ __forceinline__ bool wait_ready(const Params &p, SmemCtl *ctl, WState &w) {
+    Spin s;
+    const unsigned long long t0 = phase_begin(w);
+    while (ld_acquire_cta_shared(&ctl->ready_upto) < w.need)
+        if (!spin_ok(s, p, ctl, W_READY, (uint32_t)w.task_id, 0u)) return false;
+    phase_end(w, t0, WS_READY);
+    return true;
+}
+
 __device__ __forceinline__ bool wait_page(const Params &p, SmemCtl *ctl, WState &w, uint32_t &slot) {
-    slot = w.page_seq % kNumPages;
-    const unsigned long long t0 = w.stats ? globaltimer() : 0ull;
-    const bool ok = wait_mbar(&ctl->full[slot], (w.page_seq / kNumPages) & 1u, p, ctl, W_FULL,
-                              (uint32_t)w.task_id);
-    if (w.stats) w.t_full += globaltimer() - t0;
+    slot = w.slot;
+    const unsigned long long t0 = phase_begin(w);
+    const bool ok = wait_mbar(&ctl->full[slot], w.phase, p, ctl, W_FULL, (uint32_t)w.task_id);
+    phase_end(w, t0, WS_FULL);
     return ok;
 }
 
 __device__ __forceinline__ void release_page(SmemCtl *ctl, WState &w, uint32_t slot) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(&ctl->empty[slot]);
-    ++w.page_seq;
+    if (++w.slot == (uint32_t)kNumPages) { w.slot = 0; w.phase ^= 1u; }
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -512,8 +536,10 @@ __device__ __forceinline__ bool worker_block_sum(const Params &p, SmemCtl *ctl, 
 }
 
 // Signal the task's triggering event after every worker's writes.
+// The CTA-scope worker barrier before this call orders every worker's
+// output stores before it; the gpu-scope release add publishes them with
+// the event.
 __device__ __forceinline__ void signal_event(const Params &p, const Task &t) {
-    __threadfence();
     red_release_gpu(&p.events[t.trig], 1u);
 }
 
@@ -623,11 +649,39 @@ __device__ __forceinline__ void gemv_epilogue_row(const Params &p, int kind, int
     }
 }
 
+// Two partial sums per lane -> lanes 0..15 hold the warp total of `a`,
+// lanes 16..31 the total of `c`.
+__device__ __forceinline__ float dual_reduce(float a, float c, int lane) {
+    const bool hi = lane & 16;
+    float v = (hi ? c : a) + __shfl_xor_sync(0xffffffffu, hi ? a : c, 16);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    return v;
+}
+
+template <int NVL>
+__device__ __forceinline__ float dot_row(const uint4 *row, const float (&xr)[NVL][8], int K8, int lane) {
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+        const int v = lane + 32 * j;
+        if (v < K8) acc += dot8(row[v], xr[j]);
+    }
+    return acc;
+}
+
 // One warp per row.  Each lane keeps NVL 8-element vectors of the input
 // (vectors lane, lane+32, ...), so a warp holds the whole input vector and
-// computes its RMSNorm itself; tiles need no cross-warp reduction.  Warp w
-// computes row w of every 8-row tile, and rows w and 8+w of a 16-row pair
-// tile (RoPE partners, or the gate and up rows of one FFN index).
+// computes its RMSNorm itself: tiles need no cross-warp reduction.  Work
+// goes in units of two pages (16 rows): a pair tile (the 8 first-half q/k
+// rows and their RoPE partners, or 8 gate rows and the matching up rows),
+// or two consecutive 8-row tiles.  Warp w takes row w of both pages.
+// Everything that does not depend on the activation (gains, RoPE cos/sin,
+// the first layer's embedding row) is loaded before the task's dependency
+// is waited on; after it, one round trip loads the input vector and the
+// residual values.
 template <int NVL>
 __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                           WState &w) {
@@ -635,66 +689,182 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     const int kind = t.kind, layer = t.layer;
     const int K = op_k(s, kind);
     const int K8 = K >> 3;
-    const int rpp = rows_per_page(K);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = 0;
     const size_t row_bytes = (size_t)K * 2;
+    const int P = p.positions[b];
+    const int tok = p.tokens[b];
+    // pair tiles: every GATEUP tile, and QKV tiles below npair
+    const int npair = kind == OP_GATEUP ? 0x7fffffff
+                    : kind == OP_QKV ? (s.nq + s.nkv) * s.d / 16 : 0;
+    const int per_head = s.d / 16;
 
-    const GemvInput in = gemv_input(p, kind, layer, b);
+    // ---- before the dependency
+    const uint16_t *gain = kind == OP_QKV ? p.layers[layer].g_attn
+                         : kind == OP_GATEUP ? p.layers[layer].g_mlp
+                         : kind == OP_LMHEAD ? p.g_final : nullptr;
     float xr[NVL][8];
-    float ss = 0.f;
+    const bool embed_in = kind == OP_QKV && layer == 0;
 #pragma unroll
     for (int j = 0; j < NVL; ++j) {
         const int v = lane + 32 * j;
-        if (v < K8) {
-            load_vec8(in, v, xr[j]);
+        // gains: pulled into L1 now, read after the dependency (no registers held)
+        if (gain && v < K8 && (v & 7) == 0) prefetch_l1(reinterpret_cast<const uint4 *>(gain) + v);
+        if (embed_in && v < K8) {
+            const uint4 e = __ldg(reinterpret_cast<const uint4 *>(p.embed + (size_t)tok * s.H) + v);
+            xr[j][0] = bf_lo(e.x); xr[j][1] = bf_hi(e.x); xr[j][2] = bf_lo(e.y); xr[j][3] = bf_hi(e.y);
+            xr[j][4] = bf_lo(e.z); xr[j][5] = bf_hi(e.z); xr[j][6] = bf_lo(e.w); xr[j][7] = bf_hi(e.w);
+        }
+    }
+    // per-tile values, lane L holding those of tile begin + L (row `warp`)
+    float pre0 = 0.f, pre1 = 0.f;
+    const int my_tile = t.begin + lane;
+    if (kind == OP_QKV && my_tile < t.end && my_tile < npair) {
+        const int i = (my_tile % per_head) * 8 + warp;
+        const float2 cs = p.rope[(size_t)P * (s.d / 2) + i];
+        pre0 = cs.x;
+        pre1 = cs.y;
+    }
+    if (kind == OP_OPROJ && layer == 0 && my_tile < t.end)
+        pre0 = bf2f(p.embed[(size_t)tok * s.H + my_tile * 8 + warp]);
+
+    // ---- the dependency, then the activation
+    if (!wait_ready(p, ctl, w)) return false;
+    unsigned long long tp = phase_begin(w);
+    if (!embed_in) {
+        const float *src = kind == OP_OPROJ ? p.attn + (size_t)b * s.QD
+                         : kind == OP_DOWN ? p.act + (size_t)b * s.F : p.x + (size_t)b * s.H;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
-        } else {
+        for (int j = 0; j < NVL; ++j) {
+            const int v = lane + 32 * j;
+            if (v < K8) {
+                const float4 a0 = __ldcg(reinterpret_cast<const float4 *>(src) + 2 * v);
+                const float4 a1 = __ldcg(reinterpret_cast<const float4 *>(src) + 2 * v + 1);
+                xr[j][0] = a0.x; xr[j][1] = a0.y; xr[j][2] = a0.z; xr[j][3] = a0.w;
+                xr[j][4] = a1.x; xr[j][5] = a1.y; xr[j][6] = a1.z; xr[j][7] = a1.w;
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NVL; ++j)
+        if (lane + 32 * j >= K8) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
         }
-    }
-    if (in.gain) {
+    if (((kind == OP_OPROJ && layer > 0) || kind == OP_DOWN) && my_tile < t.end)
+        pre0 = __ldcg(p.x + (size_t)b * s.H + my_tile * 8 + warp);
+    if (gain) {
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < NVL; ++j)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
         const float sc = 1.0f / sqrtf(warp_sum(ss) / (float)s.H + s.eps);
 #pragma unroll
         for (int j = 0; j < NVL; ++j) {
             const int v = lane + 32 * j;
-            if (v < K8) scale_vec8(xr[j], sc, in.gain, v);
+            const uint4 g = v < K8 ? __ldg(reinterpret_cast<const uint4 *>(gain) + v) : make_uint4(0, 0, 0, 0);
+            xr[j][0] *= sc * bf_lo(g.x); xr[j][1] *= sc * bf_hi(g.x);
+            xr[j][2] *= sc * bf_lo(g.y); xr[j][3] *= sc * bf_hi(g.y);
+            xr[j][4] *= sc * bf_lo(g.z); xr[j][5] *= sc * bf_hi(g.z);
+            xr[j][6] *= sc * bf_lo(g.w); xr[j][7] *= sc * bf_hi(g.w);
         }
     }
+    phase_end(w, tp, WS_PRO);
 
-    const int P = p.positions[b];
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
-    for (int tile = t.begin; tile < t.end; ++tile) {
-        const int rows = tile_rows(s, kind, tile);     // 8 or 16
-        const int ra = warp, rc = 8 + warp;            // my rows in the tile
+    int tile = t.begin;
+    while (tile < t.end) {
+        const bool pair = tile < npair;
+        const bool two = pair || tile + 1 < t.end;
         float acc_a = 0.f, acc_c = 0.f;
-        for (int r0 = 0; r0 < rows; r0 += rpp) {
-            uint32_t slot;
+        uint32_t slot;
+        if (!wait_page(p, ctl, w, slot)) return false;
+        tp = phase_begin(w);
+        acc_a = dot_row<NVL>(reinterpret_cast<const uint4 *>(pages + (size_t)slot * kPageBytes + warp * row_bytes),
+                        xr, K8, lane);
+        release_page(ctl, w, slot);
+        phase_end(w, tp, WS_DOT);
+        if (two) {
             if (!wait_page(p, ctl, w, slot)) return false;
-            const unsigned char *page = pages + (size_t)slot * kPageBytes;
-            const bool mine_a = ra >= r0 && ra < r0 + rpp;
-            const bool mine_c = rows == 16 && rc >= r0 && rc < r0 + rpp;
-            if (mine_a || mine_c) {
-                const unsigned char *row = page + (size_t)((mine_a ? ra : rc) - r0) * row_bytes;
-                float acc = 0.f;
-#pragma unroll
-                for (int j = 0; j < NVL; ++j) {
-                    const int v = lane + 32 * j;
-                    if (v < K8) acc += dot8(ld_shared_v4(row + (size_t)v * 16), xr[j]);
-                }
-                if (mine_a) acc_a = acc;
-                else acc_c = acc;
-            }
+            tp = phase_begin(w);
+            acc_c = dot_row<NVL>(reinterpret_cast<const uint4 *>(pages + (size_t)slot * kPageBytes + warp * row_bytes),
+                            xr, K8, lane);
             release_page(ctl, w, slot);
+            phase_end(w, tp, WS_DOT);
         }
-        acc_a = warp_sum(acc_a);
-        if (rows == 16) acc_c = warp_sum(acc_c);
-        if (lane == 0) gemv_epilogue_row(p, kind, layer, tile, warp, acc_a, acc_c, b, P, best_v, best_i);
+        tp = phase_begin(w);
+        const float v = dual_reduce(acc_a, acc_c, lane);
+        // tile handled by this lane: lanes 0..15 the first page's, 16..31 the second's
+        const int my = (lane < 16 || pair) ? tile : tile + 1;
+        const int off = my - t.begin;
+        const float q0 = __shfl_sync(0xffffffffu, pre0, off & 31);
+        const float q1 = __shfl_sync(0xffffffffu, pre1, off & 31);
+        if (pair) {
+            const float c = __shfl_sync(0xffffffffu, v, 16);
+            if (lane == 0) {
+                if (kind == OP_GATEUP) {
+                    p.act[(size_t)b * s.F + tile * 8 + warp] = v / (1.0f + expf(-v)) * c;
+                } else {
+                    const int head = tile / per_head;
+                    const int i = (tile % per_head) * 8 + warp;
+                    float cs = q0, sn = q1;
+                    if (off >= 32) {
+                        const float2 r = p.rope[(size_t)P * (s.d / 2) + i];
+                        cs = r.x;
+                        sn = r.y;
+                    }
+                    const float ra = v * cs - c * sn;
+                    const float rc = c * cs + v * sn;
+                    if (head < s.nq) {
+                        float *qh = p.q + (size_t)b * s.QD + (size_t)head * s.d;
+                        qh[i] = ra;
+                        qh[i + s.d / 2] = rc;
+                    } else {
+                        uint16_t *kh = p.layers[layer].kc +
+                                       (((size_t)b * s.nkv + (head - s.nq)) * s.S + P) * s.d;
+                        kh[i] = f2bf(ra);
+                        kh[i + s.d / 2] = f2bf(rc);
+                    }
+                }
+            }
+            tile += 1;
+        } else {
+            if ((lane == 0) || (lane == 16 && two)) {
+                const int row = my * 8 + warp;
+                switch (kind) {
+                case OP_QKV: {
+                    const int vr = (my - npair) * 8 + warp;
+                    const int kvh = vr / s.d, dd = vr % s.d;
+                    p.layers[layer].vc[(((size_t)b * s.nkv + kvh) * s.S + P) * s.d + dd] = f2bf(v);
+                    break;
+                }
+                case OP_OPROJ:
+                case OP_DOWN: {
+                    float resid = q0;
+                    if (off >= 32)
+                        resid = (kind == OP_OPROJ && layer == 0) ? bf2f(p.embed[(size_t)tok * s.H + row])
+                                                                 : __ldcg(p.x + (size_t)b * s.H + row);
+                    p.x[(size_t)b * s.H + row] = resid + v;
+                    break;
+                }
+                default:   // OP_LMHEAD
+                    if (row < s.V) {
+                        if (p.logits) p.logits[(size_t)b * s.V + row] = v;
+                        if (v > best_v || (v == best_v && row < best_i)) { best_v = v; best_i = row; }
+                    }
+                    break;
+                }
+            }
+            tile += two ? 2 : 1;
+        }
+        phase_end(w, tp, WS_EPI);
     }
     if (kind == OP_LMHEAD) {
+        const float ov = __shfl_sync(0xffffffffu, best_v, 16);
+        const int oi = __shfl_sync(0xffffffffu, best_i, 16);
+        if (ov > best_v || (ov == best_v && oi < best_i)) { best_v = ov; best_i = oi; }
         if (lane == 0) { ctl->att_m[warp][0] = best_v; ctl->att_l[warp][0] = __int_as_float(best_i); }
         if (!worker_sync(p, ctl, w)) return false;
         if (threadIdx.x == 0) {
@@ -762,6 +932,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
     const int rpp = rows_per_page(K);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = 0;
+    if (!wait_ready(p, ctl, w)) return false;
     const GemvInput in = gemv_input(p, kind, layer, b);
     float xr[NV][8];
     float ss = 0.f;
@@ -855,6 +1026,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const AttnChunk a = attn_chunk(p, t.begin);
     const int npp = attn_pos_per_page(d);
+    if (!wait_ready(p, ctl, w)) return false;
     const int npages = (a.npre + npp - 1) / npp;
 
     float m[G], l[G], o[G][DPL], qr[G][DPL];
@@ -995,7 +1167,8 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
 template <int G>
 __device__ bool attn_dispatch_d(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                                 WState &w) {
-    if (p.s.d == 64) return attn_task<G, 2>(p, t, pages, ctl, w);
+    // head_dim 64 or 128, with G * head_dim <= 512 (checked by mk_create)
+    if (G == 8 || p.s.d == 64) return attn_task<G, 2>(p, t, pages, ctl, w);
     return attn_task<G, 4>(p, t, pages, ctl, w);
 }
 
@@ -1009,47 +1182,33 @@ __device__ bool run_task(const Params &p, const Task &t, unsigned char *pages, S
         default: return attn_dispatch_d<8>(p, t, pages, ctl, w);
         }
     }
+    // Few instantiations on purpose: every body is inlined into the one
+    // kernel, and more variants raise the register pressure of the whole.
     const int K = op_k(p.s, t.kind);
-    if (K <= kRowK) {
-        switch ((K / 8 + 31) / 32) {   // 16-byte vectors per lane
-        case 1: return gemv_rows<1>(p, t, pages, ctl, w);
-        case 2: return gemv_rows<2>(p, t, pages, ctl, w);
-        case 3: return gemv_rows<3>(p, t, pages, ctl, w);
-        case 4: return gemv_rows<4>(p, t, pages, ctl, w);
-        case 5: case 6: return gemv_rows<6>(p, t, pages, ctl, w);
-        default: return gemv_rows<8>(p, t, pages, ctl, w);
-        }
-    }
+    if (K <= kRowK) return gemv_rows<kRowK / 256>(p, t, pages, ctl, w);
     if (t.kind == OP_QKV || t.kind == OP_GATEUP)   // K = hidden <= kMaxHidden
-        return gemv_cols<2, 16>(p, t, pages, ctl, w);
-    switch ((K / 8 + kWorkerThreads - 1) / kWorkerThreads) {
-    case 1: case 2: return gemv_cols<2, 8>(p, t, pages, ctl, w);
-    case 3: case 4: return gemv_cols<4, 8>(p, t, pages, ctl, w);
-    case 5: case 6: return gemv_cols<6, 8>(p, t, pages, ctl, w);
-    default: return gemv_cols<8, 8>(p, t, pages, ctl, w);
-    }
+        return gemv_cols<kMaxHidden / 2048, 16>(p, t, pages, ctl, w);
+    if (K <= kMaxHidden) return gemv_cols<kMaxHidden / 2048, 8>(p, t, pages, ctl, w);
+    return gemv_cols<kMaxK / 2048, 8>(p, t, pages, ctl, w);
 }
 
 __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     const int tid = threadIdx.x;
     WState w;
-    w.stats = p.sm_stats != nullptr && tid == 0;
-    const unsigned long long t_begin = w.stats ? globaltimer() : 0ull;
+    if (p.sm_stats && tid == 0) {
+        w.stat = ctl->wstat;
+        for (int i = 0; i < kWStats; ++i) ctl->wstat[i] = 0;
+    }
+    const unsigned long long t_begin = phase_begin(w);
     for (int qi = q0; qi < q1; ++qi) {
         const int id = p.queue[qi];
         const Task t = p.tasks[id];
         w.task_id = id;
-        {
-            Spin s;
-            const uint32_t need = (uint32_t)(qi - q0 + 1);
-            const unsigned long long t0 = w.stats ? globaltimer() : 0ull;
-            while (ld_acquire_cta_shared(&ctl->ready_upto) < need)
-                if (!spin_ok(s, p, ctl, W_READY, (uint32_t)id, 0u)) return;
-            if (w.stats) w.t_ready += globaltimer() - t0;
-        }
+        w.need = (uint32_t)(qi - q0 + 1);   // the task body waits for it
         if (p.trace && tid == 0) p.trace[id].t_start = globaltimer();
         if (!run_task(p, t, pages, ctl, w)) return;
+        const unsigned long long te = phase_begin(w);
         if (t.kind != OP_ATTN) {
             // every output of the task is written (tile epilogues by threads < 8)
             if (!worker_sync(p, ctl, w)) return;
@@ -1084,12 +1243,19 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
             if (tid == 0) signal_event(p, t);
         }
         if (p.trace && tid == 0) p.trace[id].t_end = globaltimer();
+        phase_end(w, te, WS_END);
+        if (w.stat) w.stat[WS_TASKS] += 1;
     }
-    if (w.stats) {
+    if (w.stat) {
         unsigned long long *st = p.sm_stats + (size_t)blockIdx.x * kStatSlots;
-        st[ST_WORKER_FULL] = w.t_full;
-        st[ST_WORKER_READY] = w.t_ready;
-        st[ST_WORKER_SYNC] = w.t_sync;
+        st[ST_WORKER_FULL] = w.stat[WS_FULL];
+        st[ST_WORKER_READY] = w.stat[WS_READY];
+        st[ST_WORKER_SYNC] = w.stat[WS_SYNC];
+        st[ST_WORKER_PROLOGUE] = w.stat[WS_PRO];
+        st[ST_WORKER_DOT] = w.stat[WS_DOT];
+        st[ST_WORKER_EPI] = w.stat[WS_EPI];
+        st[ST_WORKER_END] = w.stat[WS_END];
+        st[ST_WORKER_TASKS] = w.stat[WS_TASKS];
         st[ST_WORKER_TOTAL] = globaltimer() - t_begin;
     }
 }

@@ -237,13 +237,15 @@ class Context:
         return np.frombuffer(bytes(recs), dtype=dt).copy()
 
     STAT_NAMES = ["loader_empty_ns", "loader_pages", "loader_total_ns", "worker_full_ns",
-                  "worker_ready_ns", "worker_sync_ns", "worker_total_ns", "sched_dep_ns"]
+                  "worker_ready_ns", "worker_sync_ns", "worker_total_ns", "sched_dep_ns",
+                  "worker_prologue_ns", "worker_dot_ns", "worker_epi_ns", "worker_end_ns",
+                  "worker_tasks", "unused13", "unused14", "unused15"]
 
     def sm_stats(self) -> np.ndarray:
-        """Per-SM wait accounting of the last step (trace mode): [num_sms][8]."""
+        """Per-SM wait accounting of the last step (trace mode): [num_sms][16]."""
         n = self.info().num_sms
-        out = np.zeros((n, 8), np.uint64)
-        _check(_lib.mk_get_sm_stats(self._h, out.ctypes.data, n * 8), "mk_get_sm_stats")
+        out = np.zeros((n, 16), np.uint64)
+        _check(_lib.mk_get_sm_stats(self._h, out.ctypes.data, n * 16), "mk_get_sm_stats")
         return out
 
     def graph(self) -> dict:
