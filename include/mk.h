@@ -200,7 +200,8 @@ int mk_read_buffer(mk_ctx *ctx, int which, float *host_out, size_t count);
  * mk_trace_rec [num_tasks], indexed by task id. */
 typedef struct mk_trace_rec {
     unsigned long long t_ready;  /* globaltimer ns: scheduler saw the dependency fire */
-    unsigned long long t_start;  /* workers began the task body */
+    unsigned long long t_start;  /* workers passed the dependency (loads that do not
+                                    depend on it may start earlier) */
     unsigned long long t_end;    /* workers finished and signalled */
     int sm;                      /* CTA that ran it */
     int kind;                    /* op kind (MK_OP_*) */

@@ -473,6 +473,7 @@ __device__ __forceinline__ bool wait_ready(const Params &p, SmemCtl *ctl, WState
     while (ld_acquire_cta_shared(&ctl->ready_upto) < w.need)
         if (!spin_ok(s, p, ctl, W_READY, (uint32_t)w.task_id, 0u)) return false;
     phase_end(w, t0, WS_READY);
+    if (p.trace && threadIdx.x == 0) p.trace[w.task_id].t_start = globaltimer();
     return true;
 }
 
@@ -1206,7 +1207,6 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         const Task t = p.tasks[id];
         w.task_id = id;
         w.need = (uint32_t)(qi - q0 + 1);   // the task body waits for it
-        if (p.trace && tid == 0) p.trace[id].t_start = globaltimer();
         if (!run_task(p, t, pages, ctl, w)) return;
         const unsigned long long te = phase_begin(w);
         if (t.kind != OP_ATTN) {
