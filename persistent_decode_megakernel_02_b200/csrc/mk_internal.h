@@ -16,11 +16,23 @@
 namespace mk {
 
 // ---- CTA shape ---------------------------------------------------------------
+// Three warpgroups: two of workers, one of control warps (loader, scheduler
+// and two idle warps).  The CTA launches at kLaunchRegs registers per thread
+// (65536 / 384, rounded down to 8); setmaxnreg then moves registers from the
+// control warpgroup to the workers.  The shares must add up to the launch
+// total exactly or setmaxnreg.inc would wait forever:
+//   256 * kWorkerRegs + 128 * kControlRegs == 384 * kLaunchRegs.
 constexpr int kWorkerWarps = 8;                     // run task bodies
 constexpr int kWorkerThreads = kWorkerWarps * 32;   // 256
 constexpr int kLoaderWarp = kWorkerWarps;           // streams weight pages
 constexpr int kSchedWarp = kWorkerWarps + 1;        // waits on events, activates tasks
-constexpr int kThreads = (kWorkerWarps + 2) * 32;   // 320
+constexpr int kThreads = (kWorkerWarps + 4) * 32;   // 384
+constexpr int kLaunchRegs = 168;
+constexpr int kWorkerRegs = 224;
+constexpr int kControlRegs = 56;
+static_assert(kWorkerThreads * kWorkerRegs + (kThreads - kWorkerThreads) * kControlRegs ==
+                  kThreads * kLaunchRegs,
+              "register split must equal the launch allocation");
 
 // ---- tiling ------------------------------------------------------------------
 constexpr int kTileRows = 8;        // output rows per GEMV tile

@@ -159,7 +159,7 @@ struct __align__(16) SmemCtl {
     uint32_t abort;             // this CTA is bailing out
     uint32_t ep;                // epoch of this launch (steps completed + 1)
     uint32_t last_flag;         // broadcast of "this task arrived last"
-    float red[2][kWorkerWarps][2 * kTileRows];
+    float red[2][kWorkerWarps][16];
     float scal[kWorkerWarps];
     float att_m[kWorkerWarps][kMaxGroup];
     float att_l[kWorkerWarps][kMaxGroup];
@@ -673,6 +673,25 @@ __device__ __forceinline__ float dot_row(const uint4 *row, const float (&xr)[NVL
     return acc;
 }
 
+// Two rows against the same input slice (two independent load/FMA streams).
+template <int NVL>
+__device__ __forceinline__ void dot_rows2(const uint4 *ra, const uint4 *rc, const float (&xr)[NVL][8],
+                                          int K8, int lane, float &acc_a, float &acc_c) {
+    float a = 0.f, c = 0.f;
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+        const int v = lane + 32 * j;
+        if (v < K8) {
+            const uint4 wa = ra[v];
+            const uint4 wc = rc[v];
+            a += dot8(wa, xr[j]);
+            c += dot8(wc, xr[j]);
+        }
+    }
+    acc_a = a;
+    acc_c = c;
+}
+
 // One warp per row.  Each lane keeps NVL 8-element vectors of the input
 // (vectors lane, lane+32, ...), so a warp holds the whole input vector and
 // computes its RMSNorm itself: tiles need no cross-warp reduction.  Work
@@ -780,21 +799,28 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
         const bool pair = tile < npair;
         const bool two = pair || tile + 1 < t.end;
         float acc_a = 0.f, acc_c = 0.f;
-        uint32_t slot;
-        if (!wait_page(p, ctl, w, slot)) return false;
-        tp = phase_begin(w);
-        acc_a = dot_row<NVL>(reinterpret_cast<const uint4 *>(pages + (size_t)slot * kPageBytes + warp * row_bytes),
-                        xr, K8, lane);
-        release_page(ctl, w, slot);
-        phase_end(w, tp, WS_DOT);
+        uint32_t slot_a, slot_c;
+        if (!wait_page(p, ctl, w, slot_a)) return false;
+        const uint4 *row_a = reinterpret_cast<const uint4 *>(pages + (size_t)slot_a * kPageBytes + warp * row_bytes);
         if (two) {
-            if (!wait_page(p, ctl, w, slot)) return false;
+            // the unit's second page is the ring's next one
+            const uint32_t s0 = w.slot, p0 = w.phase;
+            if (++w.slot == (uint32_t)kNumPages) { w.slot = 0; w.phase ^= 1u; }
+            if (!wait_page(p, ctl, w, slot_c)) return false;
+            w.slot = s0;
+            w.phase = p0;
             tp = phase_begin(w);
-            acc_c = dot_row<NVL>(reinterpret_cast<const uint4 *>(pages + (size_t)slot * kPageBytes + warp * row_bytes),
-                            xr, K8, lane);
-            release_page(ctl, w, slot);
-            phase_end(w, tp, WS_DOT);
+            dot_rows2<NVL>(row_a,
+                           reinterpret_cast<const uint4 *>(pages + (size_t)slot_c * kPageBytes + warp * row_bytes),
+                           xr, K8, lane, acc_a, acc_c);
+            release_page(ctl, w, slot_a);
+            release_page(ctl, w, slot_c);
+        } else {
+            tp = phase_begin(w);
+            acc_a = dot_row<NVL>(row_a, xr, K8, lane);
+            release_page(ctl, w, slot_a);
         }
+        phase_end(w, tp, WS_DOT);
         tp = phase_begin(w);
         const float v = dual_reduce(acc_a, acc_c, lane);
         // tile handled by this lane: lanes 0..15 the first page's, 16..31 the second's
@@ -923,7 +949,7 @@ __device__ __forceinline__ float warp_reduce_rows<16>(const float (&acc)[16], in
     return c;
 }
 
-template <int NV, int RMAX>
+template <int NV>
 __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                           WState &w) {
     const Shape &s = p.s;
@@ -933,7 +959,19 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
     const int rpp = rows_per_page(K);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = 0;
+    const int npair = kind == OP_GATEUP ? 0x7fffffff
+                    : kind == OP_QKV ? (s.nq + s.nkv) * s.d / 16 : 0;
+    const int P = p.positions[b];
+    const int tok = p.tokens[b];
+    // residual of row 8 * begin + lane (warp 0), for the O / down projections
+    const bool resid_op = kind == OP_OPROJ || kind == OP_DOWN;
+    const int task_rows = 8 * (t.end - t.begin);
+    float resid = 0.f;
+    if (kind == OP_OPROJ && layer == 0 && warp == 0 && lane < task_rows)
+        resid = bf2f(p.embed[(size_t)tok * s.H + 8 * t.begin + lane]);
     if (!wait_ready(p, ctl, w)) return false;
+    if (resid_op && !(kind == OP_OPROJ && layer == 0) && warp == 0 && lane < task_rows)
+        resid = __ldcg(p.x + (size_t)b * s.H + 8 * t.begin + lane);
     const GemvInput in = gemv_input(p, kind, layer, b);
     float xr[NV][8];
     float ss = 0.f;
@@ -959,53 +997,72 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
             if (v < K8) scale_vec8(xr[j], sc, in.gain, v);
         }
     }
-    const int P = p.positions[b];
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
     const size_t row_bytes = (size_t)K * 2;
-    constexpr int kLanesPerRow = 32 / RMAX;   // lanes holding one row after the reduction
-    for (int tile = t.begin; tile < t.end; ++tile) {
-        const int rows = RMAX == 16 ? tile_rows(s, kind, tile) : 8;
-        float acc[RMAX];
+    // groups of 16 rows: one pair tile, or two consecutive 8-row tiles
+    int tile = t.begin;
+    while (tile < t.end) {
+        const bool pair = tile < npair;
+        const int rows = pair ? 16 : (tile + 1 < t.end ? 16 : 8);
+        float acc[16];
 #pragma unroll
-        for (int r = 0; r < RMAX; ++r) acc[r] = 0.f;
+        for (int r = 0; r < 16; ++r) acc[r] = 0.f;
         uint32_t slot = 0;
         const unsigned char *page = pages;
 #pragma unroll
-        for (int r = 0; r < RMAX; ++r) {
+        for (int r = 0; r < 16; ++r) {
             if (r < rows) {
                 if ((r & (rpp - 1)) == 0) {
                     if (!wait_page(p, ctl, w, slot)) return false;
                     page = pages + (size_t)slot * kPageBytes;
                 }
-                const unsigned char *row = page + (size_t)(r & (rpp - 1)) * row_bytes;
+                const uint4 *row = reinterpret_cast<const uint4 *>(page + (size_t)(r & (rpp - 1)) * row_bytes);
 #pragma unroll
                 for (int j = 0; j < NV; ++j) {
                     const int v = tid + j * kWorkerThreads;
-                    if (v < K8) acc[r] += dot8(ld_shared_v4(row + (size_t)v * 16), xr[j]);
+                    if (v < K8) acc[r] += dot8(row[v], xr[j]);
                 }
-                if (((r + 1) & (rpp - 1)) == 0) release_page(ctl, w, slot);
+                if (((r + 1) & (rpp - 1)) == 0 || r + 1 == rows) release_page(ctl, w, slot);
             }
         }
-        const float rsum = warp_reduce_rows<RMAX>(acc, lane);
-        if ((lane & (kLanesPerRow - 1)) == 0) ctl->red[w.red_buf][warp][lane / kLanesPerRow] = rsum;
+        const float rsum = warp_reduce_rows<16>(acc, lane);   // lane holds row (lane >> 1) & 15
+        if ((lane & 1) == 0) ctl->red[w.red_buf][warp][lane >> 1] = rsum;
         if (!worker_sync(p, ctl, w)) return false;
-        if (warp == 0 && lane < 8) {
+        if (warp == 0) {
+            const int e = lane & 15;                      // row within the group
             float a = 0.f, c = 0.f;
 #pragma unroll
             for (int i = 0; i < kWorkerWarps; ++i) {
-                a += ctl->red[w.red_buf][i][lane];
-                if (RMAX == 16) c += ctl->red[w.red_buf][i][8 + lane];
+                a += ctl->red[w.red_buf][i][e];
+                c += ctl->red[w.red_buf][i][(e + 8) & 15];
             }
-            gemv_epilogue_row(p, kind, layer, tile, lane, a, c, b, P, best_v, best_i);
+            const int grp_row = 8 * (tile - t.begin) + e;   // row within the task
+            const float rres = __shfl_sync(0xffffffffu, resid, grp_row & 31);
+            if (pair) {
+                if (lane < 8) gemv_epilogue_row(p, kind, layer, tile, lane, a, c, b, P, best_v, best_i);
+            } else if (lane < rows) {
+                const int tl = tile + (e >> 3), r = e & 7;
+                if (resid_op) {
+                    const int row = tl * 8 + r;
+                    const float base = grp_row < 32 ? rres
+                                     : (kind == OP_OPROJ && layer == 0)
+                                           ? bf2f(p.embed[(size_t)tok * s.H + row])
+                                           : __ldcg(p.x + (size_t)b * s.H + row);
+                    p.x[(size_t)b * s.H + row] = base + a;
+                } else {
+                    gemv_epilogue_row(p, kind, layer, tl, r, a, 0.f, b, P, best_v, best_i);
+                }
+            }
         }
         w.red_buf ^= 1;
+        tile += pair ? 1 : (rows == 16 ? 2 : 1);
     }
-    if (kind == OP_LMHEAD && warp == 0 && lane < 8) {
+    if (kind == OP_LMHEAD && warp == 0) {
 #pragma unroll
-        for (int o = 4; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffu, best_v, o);
-            const int oi = __shfl_xor_sync(0xffu, best_i, o);
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, best_i, o);
             if (ov > best_v || (ov == best_v && oi < best_i)) { best_v = ov; best_i = oi; }
         }
         if (lane == 0) {
@@ -1187,10 +1244,9 @@ __device__ bool run_task(const Params &p, const Task &t, unsigned char *pages, S
     // kernel, and more variants raise the register pressure of the whole.
     const int K = op_k(p.s, t.kind);
     if (K <= kRowK) return gemv_rows<kRowK / 256>(p, t, pages, ctl, w);
-    if (t.kind == OP_QKV || t.kind == OP_GATEUP)   // K = hidden <= kMaxHidden
-        return gemv_cols<kMaxHidden / 2048, 16>(p, t, pages, ctl, w);
-    if (K <= kMaxHidden) return gemv_cols<kMaxHidden / 2048, 8>(p, t, pages, ctl, w);
-    return gemv_cols<kMaxK / 2048, 8>(p, t, pages, ctl, w);
+    if (K <= kMaxHidden) return gemv_cols<kMaxHidden / 2048>(p, t, pages, ctl, w);
+    if (K <= 4 * 2048) return gemv_cols<4>(p, t, pages, ctl, w);
+    return gemv_cols<kMaxK / 2048>(p, t, pages, ctl, w);
 }
 
 __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
@@ -1303,11 +1359,15 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
         if (old + 1u == gridDim.x * ep) atomicExch(p.epoch, ep);
     }
     if (warp < kWorkerWarps) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kWorkerRegs));
         worker_role(p, pages, ctl);
-    } else if (warp == kLoaderWarp) {
-        if (lane == 0) loader_role(p, pages, ctl);
     } else {
-        if (lane == 0) scheduler_role(p, ctl, ctl->ep);
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+        if (warp == kLoaderWarp) {
+            if (lane == 0) loader_role(p, pages, ctl);
+        } else if (warp == kSchedWarp) {
+            if (lane == 0) scheduler_role(p, ctl, ctl->ep);
+        }
     }
 }
 
@@ -1315,6 +1375,14 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
 // host-side launch helpers (called from mk_runtime.cpp)
 // ---------------------------------------------------------------------------
 size_t kernel_smem_bytes() { return kSmemBytes; }
+
+// Registers per thread the kernel was compiled to launch with; the register
+// split (setmaxnreg) is only valid when this equals kLaunchRegs.
+int kernel_launch_regs() {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, mk_step_kernel) != cudaSuccess) return -1;
+    return a.numRegs;
+}
 
 cudaError_t kernel_prepare() {
     return cudaFuncSetAttribute(mk_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

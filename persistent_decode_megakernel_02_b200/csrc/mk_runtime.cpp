@@ -14,6 +14,7 @@
 
 namespace mk {
 size_t kernel_smem_bytes();
+int kernel_launch_regs();
 cudaError_t kernel_prepare();
 cudaError_t kernel_occupancy(int *blocks_per_sm);
 cudaError_t kernel_launch(const Params &p, int grid, cudaStream_t stream);
@@ -161,6 +162,9 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     if (prop.major < 10) return MK_ERR_INVALID;     // built for sm_100a only
     if (!prop.cooperativeLaunch) return MK_ERR_INVALID;
     if ((size_t)prop.sharedMemPerBlockOptin < kernel_smem_bytes()) return MK_ERR_INVALID;
+    // The worker/control register split is only safe with the launch
+    // allocation it was computed for; refuse to launch anything else.
+    if (kernel_launch_regs() != kLaunchRegs) return MK_ERR_INVALID;
     Shape s;
     int st = shape_from_config(cfg, prop.multiProcessorCount, s);
     if (st != MK_OK) return st;
