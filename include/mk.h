@@ -219,7 +219,8 @@ int mk_get_trace(mk_ctx *ctx, mk_trace_rec *host_out, int n);
  * waiting on event counters, worker ns in task prologues (input vector
  * load, RMSNorm), worker ns in dot products, worker ns in per-tile
  * reductions and epilogues, worker ns in task ends (barrier, fence, event,
- * merges), tasks run, 3 unused}.  Worker figures are those of warp 0 and
+ * merges), tasks run, worker ns in attention combine/merge tails,
+ * 2 unused}.  Worker figures are those of warp 0 and
  * some phases overlap the waits they contain. */
 int mk_get_sm_stats(mk_ctx *ctx, uint64_t *host_out, int n);
 

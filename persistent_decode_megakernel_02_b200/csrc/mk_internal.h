@@ -173,6 +173,7 @@ enum StatSlot {
     ST_WORKER_EPI = 10,      // worker warp 0: per-tile reductions and epilogues
     ST_WORKER_END = 11,      // worker warp 0: task end (barrier, fence, event, merges)
     ST_WORKER_TASKS = 12,    // tasks run (count)
+    ST_WORKER_ATTN_TAIL = 13, // worker warp 0: attention combine, partial write and merge
     kStatSlots = 16
 };
 

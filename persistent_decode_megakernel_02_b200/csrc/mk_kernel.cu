@@ -164,7 +164,7 @@ struct __align__(16) SmemCtl {
     float att_m[kWorkerWarps][kMaxGroup];
     float att_l[kWorkerWarps][kMaxGroup];
     float att_o[kWorkerWarps][kAttnCombine];
-    unsigned long long wstat[8];   // trace-mode time accounting of worker thread 0
+    unsigned long long wstat[16];   // trace-mode time accounting of worker thread 0
 };
 constexpr size_t kSmemBytes = (size_t)kNumPages * kPageBytes + sizeof(SmemCtl);
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -446,7 +446,7 @@ struct WState {
 };
 // Trace-mode time accounting of worker thread 0, accumulated in shared memory
 // so it costs no registers across the task bodies.
-enum WStat { WS_FULL = 0, WS_READY, WS_SYNC, WS_PRO, WS_DOT, WS_EPI, WS_END, WS_TASKS, kWStats };
+enum WStat { WS_FULL = 0, WS_READY, WS_SYNC, WS_PRO, WS_DOT, WS_EPI, WS_END, WS_TASKS, WS_ATT, kWStats };
 __device__ __forceinline__ unsigned long long phase_begin(const WState &w) {
     return w.stat ? globaltimer() : 0ull;
 }
@@ -970,6 +970,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
     if (kind == OP_OPROJ && layer == 0 && warp == 0 && lane < task_rows)
         resid = bf2f(p.embed[(size_t)tok * s.H + 8 * t.begin + lane]);
     if (!wait_ready(p, ctl, w)) return false;
+    unsigned long long tp = phase_begin(w);
     if (resid_op && !(kind == OP_OPROJ && layer == 0) && warp == 0 && lane < task_rows)
         resid = __ldcg(p.x + (size_t)b * s.H + 8 * t.begin + lane);
     const GemvInput in = gemv_input(p, kind, layer, b);
@@ -997,6 +998,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
             if (v < K8) scale_vec8(xr[j], sc, in.gain, v);
         }
     }
+    phase_end(w, tp, WS_PRO);
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
     const size_t row_bytes = (size_t)K * 2;
@@ -1016,6 +1018,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
                 if ((r & (rpp - 1)) == 0) {
                     if (!wait_page(p, ctl, w, slot)) return false;
                     page = pages + (size_t)slot * kPageBytes;
+                    tp = phase_begin(w);
                 }
                 const uint4 *row = reinterpret_cast<const uint4 *>(page + (size_t)(r & (rpp - 1)) * row_bytes);
 #pragma unroll
@@ -1023,9 +1026,13 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
                     const int v = tid + j * kWorkerThreads;
                     if (v < K8) acc[r] += dot8(row[v], xr[j]);
                 }
-                if (((r + 1) & (rpp - 1)) == 0 || r + 1 == rows) release_page(ctl, w, slot);
+                if (((r + 1) & (rpp - 1)) == 0 || r + 1 == rows) {
+                    release_page(ctl, w, slot);
+                    phase_end(w, tp, WS_DOT);
+                }
             }
         }
+        tp = phase_begin(w);
         const float rsum = warp_reduce_rows<16>(acc, lane);   // lane holds row (lane >> 1) & 15
         if ((lane & 1) == 0) ctl->red[w.red_buf][warp][lane >> 1] = rsum;
         if (!worker_sync(p, ctl, w)) return false;
@@ -1057,6 +1064,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
         }
         w.red_buf ^= 1;
         tile += pair ? 1 : (rows == 16 ? 2 : 1);
+        phase_end(w, tp, WS_EPI);
     }
     if (kind == OP_LMHEAD && warp == 0) {
 #pragma unroll
@@ -1085,6 +1093,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     const AttnChunk a = attn_chunk(p, t.begin);
     const int npp = attn_pos_per_page(d);
     if (!wait_ready(p, ctl, w)) return false;
+    unsigned long long tp = phase_begin(w);
     const int npages = (a.npre + npp - 1) / npp;
 
     float m[G], l[G], o[G][DPL], qr[G][DPL];
@@ -1136,15 +1145,19 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
         }
     };
 
+    phase_end(w, tp, WS_PRO);
     for (int pg = 0; pg < npages; ++pg) {
         uint32_t slot;
         if (!wait_page(p, ctl, w, slot)) return false;
+        tp = phase_begin(w);
         const uint16_t *Kp = reinterpret_cast<const uint16_t *>(pages + (size_t)slot * kPageBytes);
         const uint16_t *Vp = Kp + (size_t)npp * d;
         const int n = min(npp, a.npre - pg * npp);
         for (int j = warp; j < n; j += kWorkerWarps) visit(Kp + (size_t)j * d, Vp + (size_t)j * d, false);
         release_page(ctl, w, slot);
+        phase_end(w, tp, WS_DOT);
     }
+    tp = phase_begin(w);
     if (a.has_new && warp == (a.npre % kWorkerWarps)) {
         const LayerW &L = p.layers[t.layer];
         const size_t off = (((size_t)a.b * s.nkv + a.kvh) * s.S + a.P) * d;
@@ -1216,6 +1229,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
         if (!worker_sync(p, ctl, w)) return false;
         if (tid == 0) signal_event(p, t);
     }
+    phase_end(w, tp, WS_ATT);
     return true;
 }
 
@@ -1312,6 +1326,7 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         st[ST_WORKER_EPI] = w.stat[WS_EPI];
         st[ST_WORKER_END] = w.stat[WS_END];
         st[ST_WORKER_TASKS] = w.stat[WS_TASKS];
+        st[ST_WORKER_ATTN_TAIL] = w.stat[WS_ATT];
         st[ST_WORKER_TOTAL] = globaltimer() - t_begin;
     }
 }
