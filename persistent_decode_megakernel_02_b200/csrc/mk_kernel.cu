@@ -446,7 +446,7 @@ struct WState {
 };
 // Trace-mode time accounting of worker thread 0, accumulated in shared memory
 // so it costs no registers across the task bodies.
-enum WStat { WS_FULL = 0, WS_READY, WS_SYNC, WS_PRO, WS_DOT, WS_EPI, WS_END, WS_TASKS, WS_ATT, kWStats };
+enum WStat { WS_FULL = 0, WS_READY, WS_SYNC, WS_PRO, WS_DOT, WS_EPI, WS_END, WS_TASKS, WS_ATT, WS_FIRST, kWStats };
 __device__ __forceinline__ unsigned long long phase_begin(const WState &w) {
     return w.stat ? globaltimer() : 0ull;
 }
@@ -999,42 +999,52 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
         }
     }
     phase_end(w, tp, WS_PRO);
+    bool first_page = true;
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
     const size_t row_bytes = (size_t)K * 2;
-    // groups of 16 rows: one pair tile, or two consecutive 8-row tiles
+    // groups of 16 rows: one pair tile, or two consecutive 8-row tiles.  Rows
+    // go two at a time in page order (rows 2k and 2k + 1), each pair reduced
+    // across the warp right away and its warp partials parked in shared
+    // memory, so the loop stays rolled: compact code that stays in the
+    // instruction cache instead of 16 unrolled rows.
     int tile = t.begin;
+    uint32_t slot = 0;
+    const unsigned char *page = pages;
     while (tile < t.end) {
         const bool pair = tile < npair;
         const int rows = pair ? 16 : (tile + 1 < t.end ? 16 : 8);
-        float acc[16];
+        float *red = ctl->red[w.red_buf][warp];
+#pragma unroll 1
+        for (int k = 0; k < rows; k += 2) {
+            float acc2[2];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) acc[r] = 0.f;
-        uint32_t slot = 0;
-        const unsigned char *page = pages;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            if (r < rows) {
-                if ((r & (rpp - 1)) == 0) {
+            for (int h = 0; h < 2; ++h) {
+                const int rr = k + h;
+                if ((rr & (rpp - 1)) == 0) {
                     if (!wait_page(p, ctl, w, slot)) return false;
                     page = pages + (size_t)slot * kPageBytes;
                     tp = phase_begin(w);
                 }
-                const uint4 *row = reinterpret_cast<const uint4 *>(page + (size_t)(r & (rpp - 1)) * row_bytes);
+                const uint4 *row = reinterpret_cast<const uint4 *>(page + (size_t)(rr & (rpp - 1)) * row_bytes);
+                float acc = 0.f;
 #pragma unroll
                 for (int j = 0; j < NV; ++j) {
                     const int v = tid + j * kWorkerThreads;
-                    if (v < K8) acc[r] += dot8(row[v], xr[j]);
+                    if (v < K8) acc += dot8(row[v], xr[j]);
                 }
-                if (((r + 1) & (rpp - 1)) == 0 || r + 1 == rows) {
+                acc2[h] = acc;
+                if (((rr + 1) & (rpp - 1)) == 0 || rr + 1 == rows) {
                     release_page(ctl, w, slot);
-                    phase_end(w, tp, WS_DOT);
+                    phase_end(w, tp, first_page ? WS_FIRST : WS_DOT);
+                    first_page = false;
                 }
             }
+            const float v = dual_reduce(acc2[0], acc2[1], lane);
+            if (lane == 0) red[k] = v;
+            if (lane == 16) red[k + 1] = v;
         }
         tp = phase_begin(w);
-        const float rsum = warp_reduce_rows<16>(acc, lane);   // lane holds row (lane >> 1) & 15
-        if ((lane & 1) == 0) ctl->red[w.red_buf][warp][lane >> 1] = rsum;
         if (!worker_sync(p, ctl, w)) return false;
         if (warp == 0) {
             const int e = lane & 15;                      // row within the group
@@ -1327,6 +1337,7 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         st[ST_WORKER_END] = w.stat[WS_END];
         st[ST_WORKER_TASKS] = w.stat[WS_TASKS];
         st[ST_WORKER_ATTN_TAIL] = w.stat[WS_ATT];
+        st[14] = w.stat[WS_FIRST];
         st[ST_WORKER_TOTAL] = globaltimer() - t_begin;
     }
 }

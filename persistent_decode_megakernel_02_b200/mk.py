@@ -239,7 +239,7 @@ class Context:
     STAT_NAMES = ["loader_empty_ns", "loader_pages", "loader_total_ns", "worker_full_ns",
                   "worker_ready_ns", "worker_sync_ns", "worker_total_ns", "sched_dep_ns",
                   "worker_prologue_ns", "worker_dot_ns", "worker_epi_ns", "worker_end_ns",
-                  "worker_tasks", "worker_attn_tail_ns", "unused14", "unused15"]
+                  "worker_tasks", "worker_attn_tail_ns", "cols_first_page_ns", "unused15"]
 
     def sm_stats(self) -> np.ndarray:
         """Per-SM wait accounting of the last step (trace mode): [num_sms][16]."""
