@@ -79,6 +79,8 @@ enum mk_flags {
  *  attn_chunks: split-K chunks per (sequence, KV head) in the attention
  *  op; 0 picks one chunk count so that the attention tasks cover the SMs.
  *  timeout_ns: bound on every device-side wait; 0 means 2 s.
+ *  l2_lookahead_kb: how far (KiB of weights per SM) the loader prefetches
+ *  into L2 beyond its shared-memory ring; 0 picks the default (256).
  */
 typedef struct mk_config {
     int layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
@@ -87,6 +89,7 @@ typedef struct mk_config {
     int flags;
     int attn_chunks;
     long long timeout_ns;
+    int l2_lookahead_kb;
 } mk_config;
 
 /*
@@ -202,6 +205,8 @@ typedef struct mk_trace_rec {
     unsigned long long t_ready;  /* globaltimer ns: scheduler saw the dependency fire */
     unsigned long long t_start;  /* workers passed the dependency (loads that do not
                                     depend on it may start earlier) */
+    unsigned long long t_input;  /* the task's input vector is loaded (and normalised) */
+    unsigned long long t_done;   /* all rows computed, before the task-end barrier */
     unsigned long long t_end;    /* workers finished and signalled */
     int sm;                      /* CTA that ran it */
     int kind;                    /* op kind (MK_OP_*) */

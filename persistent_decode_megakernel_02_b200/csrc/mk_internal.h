@@ -42,7 +42,8 @@ constexpr int kVecMax = 8;          // 16-byte vectors per thread per row (K <= 
 constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 16384
 constexpr int kMaxGroup = 8;        // q heads per KV head handled by one attention task
 constexpr int kMaxHeadDim = 256;
-constexpr long long kL2Lookahead = 256 * 1024;  // bytes the L2 prefetch runs ahead of the ring
+constexpr long long kL2Lookahead = 256 * 1024;  // default bytes the L2 prefetch runs ahead of the ring
+constexpr int kStageFloats = 6144;  // shared staging: a GEMV input vector, or attention partials
 constexpr int kL2Chunk = 64 * 1024;             // bytes per L2 prefetch instruction
 
 // ---- ops ---------------------------------------------------------------------
@@ -178,10 +179,10 @@ enum StatSlot {
 };
 
 struct TraceRec {
-    unsigned long long t_ready, t_start, t_end;
+    unsigned long long t_ready, t_start, t_input, t_done, t_end;
     int32_t sm, kind, layer, trig;
 };
-static_assert(sizeof(TraceRec) == 40, "trace record layout");
+static_assert(sizeof(TraceRec) == 56, "trace record layout");
 
 struct Params {
     Shape s;
@@ -219,7 +220,7 @@ struct Params {
     TraceRec *trace;             // null unless tracing
     unsigned long long *sm_stats; // [num_sms][kStatSlots] wait times (ns), null unless tracing
     unsigned long long timeout_ns;
-    int l2_prefetch;
+    long long l2_lookahead;      // bytes the L2 prefetch runs ahead of the ring (0: off)
 };
 
 // ---- host planning -------------------------------------------------------------

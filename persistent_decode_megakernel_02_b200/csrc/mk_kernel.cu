@@ -39,6 +39,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <math.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "mk_internal.h"
@@ -150,6 +151,8 @@ __device__ __forceinline__ float dot8(const uint4 w, const float *x) {
 // shared memory
 // ---------------------------------------------------------------------------
 constexpr int kAttnCombine = 512;   // G * head_dim handled by the warp combine
+static_assert(kWorkerWarps * kAttnCombine <= kStageFloats, "combine fits the staging area");
+constexpr int kMinChunk = 32;       // fewest positions per active attention chunk
 
 struct __align__(16) SmemCtl {
     uint64_t full[kNumPages];
@@ -163,10 +166,15 @@ struct __align__(16) SmemCtl {
     float scal[kWorkerWarps];
     float att_m[kWorkerWarps][kMaxGroup];
     float att_l[kWorkerWarps][kMaxGroup];
-    float att_o[kWorkerWarps][kAttnCombine];
+    // staging area: a GEMV task's input vector (read as float4); an attention
+    // task's per-warp running outputs (kWorkerWarps x kAttnCombine), later
+    // its merge inputs
+    __align__(16) float stage[kStageFloats];
     unsigned long long wstat[16];   // trace-mode time accounting of worker thread 0
 };
 constexpr size_t kSmemBytes = (size_t)kNumPages * kPageBytes + sizeof(SmemCtl);
+static_assert(offsetof(SmemCtl, stage) % 16 == 0, "float4 access to the staging area");
+static_assert((kNumPages * kPageBytes) % 16 == 0, "SmemCtl placement");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 // ---------------------------------------------------------------------------
@@ -232,6 +240,7 @@ struct AttnChunk {
     int c0, c1;       // positions [c0, c1) of this chunk (c1 <= P + 1)
     int npre;         // cached positions loaded by pages: [c0, c0 + npre), all < P
     bool has_new;     // P is in [c0, c1)
+    int nc;           // chunks with positions for this sequence (the others are empty)
 };
 
 __device__ __forceinline__ AttnChunk attn_chunk(const Params &p, int item) {
@@ -241,11 +250,15 @@ __device__ __forceinline__ AttnChunk attn_chunk(const Params &p, int item) {
     a.kvh = (item / s.NC) % s.nkv;
     a.c = item % s.NC;
     a.active = a.b < p.batch;
-    a.P = 0; a.c0 = 0; a.c1 = 0; a.npre = 0; a.has_new = false;
+    a.P = 0; a.c0 = 0; a.c1 = 0; a.npre = 0; a.has_new = false; a.nc = 0;
     if (a.active) {
         a.P = p.positions[a.b];
         int C = a.P + 1;
-        int Lc = (C + s.NC - 1) / s.NC;
+        // at most NC chunks, but no fewer than kMinChunk positions per chunk:
+        // short contexts use few chunks (fewer partials to merge)
+        const int nc = min(s.NC, (C + kMinChunk - 1) / kMinChunk);
+        int Lc = (C + nc - 1) / nc;
+        a.nc = nc;
         a.c0 = a.c * Lc;
         a.c1 = min(a.c0 + Lc, C);
         if (a.c0 >= C) { a.c0 = C; a.c1 = C; }
@@ -377,7 +390,7 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         }
         GemvStream g = gemv_stream(p, t);
         for (int k = 0; k < g.npages; ++k) {
-            if (p.l2_prefetch) pf.run(p, issued + kL2Lookahead);
+            if (p.l2_lookahead) pf.run(p, issued + p.l2_lookahead);
             const uint32_t bytes = (uint32_t)max(0LL, min((long long)g.page_bytes, g.left));
             uint32_t slot;
             if (!ring_acquire(p, ctl, ring, bytes, (uint32_t)id, slot)) { ok = false; break; }
@@ -452,6 +465,13 @@ __device__ __forceinline__ unsigned long long phase_begin(const WState &w) {
 }
 __device__ __forceinline__ void phase_end(const WState &w, unsigned long long t0, int which) {
     if (w.stat) w.stat[which] += globaltimer() - t0;
+}
+// Trace stamps of the current task (thread 0 only).
+__device__ __forceinline__ void stamp_input(const Params &p, const WState &w) {
+    if (p.trace && threadIdx.x == 0) p.trace[w.task_id].t_input = globaltimer();
+}
+__device__ __forceinline__ void stamp_done(const Params &p, const WState &w) {
+    if (p.trace && threadIdx.x == 0) p.trace[w.task_id].t_done = globaltimer();
 }
 
 // All worker warps meet; bounded.
@@ -751,9 +771,36 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     // ---- the dependency, then the activation
     if (!wait_ready(p, ctl, w)) return false;
     unsigned long long tp = phase_begin(w);
-    if (!embed_in) {
+    if (((kind == OP_OPROJ && layer > 0) || kind == OP_DOWN) && my_tile < t.end)
+        pre0 = __ldcg(p.x + (size_t)b * s.H + my_tile * 8 + warp);
+    if (embed_in) {
+        // the embedding row needs no dependency: each warp holds it already
+        if (gain) {
+            float ss = 0.f;
+#pragma unroll
+            for (int j = 0; j < NVL; ++j)
+                if (lane + 32 * j < K8) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
+                }
+            const float sc = 1.0f / sqrtf(warp_sum(ss) / (float)s.H + s.eps);
+#pragma unroll
+            for (int j = 0; j < NVL; ++j) {
+                const int v = lane + 32 * j;
+                const uint4 g = v < K8 ? __ldg(reinterpret_cast<const uint4 *>(gain) + v) : make_uint4(0, 0, 0, 0);
+                xr[j][0] *= sc * bf_lo(g.x); xr[j][1] *= sc * bf_hi(g.x);
+                xr[j][2] *= sc * bf_lo(g.y); xr[j][3] *= sc * bf_hi(g.y);
+                xr[j][4] *= sc * bf_lo(g.z); xr[j][5] *= sc * bf_hi(g.z);
+                xr[j][6] *= sc * bf_lo(g.w); xr[j][7] *= sc * bf_hi(g.w);
+            }
+        }
+    } else {
+        // the activation, straight from L2 into every warp (each warp holds
+        // the whole vector and normalises it itself: no block barrier, so a
+        // warp still finishing the previous task delays nobody)
         const float *src = kind == OP_OPROJ ? p.attn + (size_t)b * s.QD
                          : kind == OP_DOWN ? p.act + (size_t)b * s.F : p.x + (size_t)b * s.H;
+        float ss = 0.f;
 #pragma unroll
         for (int j = 0; j < NVL; ++j) {
             const int v = lane + 32 * j;
@@ -762,35 +809,30 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
                 const float4 a1 = __ldcg(reinterpret_cast<const float4 *>(src) + 2 * v + 1);
                 xr[j][0] = a0.x; xr[j][1] = a0.y; xr[j][2] = a0.z; xr[j][3] = a0.w;
                 xr[j][4] = a1.x; xr[j][5] = a1.y; xr[j][6] = a1.z; xr[j][7] = a1.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
+            }
+        }
+        if (gain) {
+#pragma unroll
+            for (int j = 0; j < NVL; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
+            const float sc = 1.0f / sqrtf(warp_sum(ss) / (float)s.H + s.eps);
+#pragma unroll
+            for (int j = 0; j < NVL; ++j) {
+                const int v = lane + 32 * j;
+                const uint4 g = v < K8 ? __ldg(reinterpret_cast<const uint4 *>(gain) + v) : make_uint4(0, 0, 0, 0);
+                xr[j][0] *= sc * bf_lo(g.x); xr[j][1] *= sc * bf_hi(g.x);
+                xr[j][2] *= sc * bf_lo(g.y); xr[j][3] *= sc * bf_hi(g.y);
+                xr[j][4] *= sc * bf_lo(g.z); xr[j][5] *= sc * bf_hi(g.z);
+                xr[j][6] *= sc * bf_lo(g.w); xr[j][7] *= sc * bf_hi(g.w);
             }
         }
     }
-#pragma unroll
-    for (int j = 0; j < NVL; ++j)
-        if (lane + 32 * j >= K8) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
-        }
-    if (((kind == OP_OPROJ && layer > 0) || kind == OP_DOWN) && my_tile < t.end)
-        pre0 = __ldcg(p.x + (size_t)b * s.H + my_tile * 8 + warp);
-    if (gain) {
-        float ss = 0.f;
-#pragma unroll
-        for (int j = 0; j < NVL; ++j)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
-        const float sc = 1.0f / sqrtf(warp_sum(ss) / (float)s.H + s.eps);
-#pragma unroll
-        for (int j = 0; j < NVL; ++j) {
-            const int v = lane + 32 * j;
-            const uint4 g = v < K8 ? __ldg(reinterpret_cast<const uint4 *>(gain) + v) : make_uint4(0, 0, 0, 0);
-            xr[j][0] *= sc * bf_lo(g.x); xr[j][1] *= sc * bf_hi(g.x);
-            xr[j][2] *= sc * bf_lo(g.y); xr[j][3] *= sc * bf_hi(g.y);
-            xr[j][4] *= sc * bf_lo(g.z); xr[j][5] *= sc * bf_hi(g.z);
-            xr[j][6] *= sc * bf_lo(g.w); xr[j][7] *= sc * bf_hi(g.w);
-        }
-    }
     phase_end(w, tp, WS_PRO);
+    stamp_input(p, w);
 
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
@@ -888,6 +930,7 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
         }
         phase_end(w, tp, WS_EPI);
     }
+    stamp_done(p, w);
     if (kind == OP_LMHEAD) {
         const float ov = __shfl_sync(0xffffffffu, best_v, 16);
         const int oi = __shfl_sync(0xffffffffu, best_i, 16);
@@ -999,6 +1042,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
         }
     }
     phase_end(w, tp, WS_PRO);
+    stamp_input(p, w);
     bool first_page = true;
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
@@ -1076,6 +1120,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
         tile += pair ? 1 : (rows == 16 ? 2 : 1);
         phase_end(w, tp, WS_EPI);
     }
+    stamp_done(p, w);
     if (kind == OP_LMHEAD && warp == 0) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -1156,6 +1201,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     };
 
     phase_end(w, tp, WS_PRO);
+    stamp_input(p, w);
     for (int pg = 0; pg < npages; ++pg) {
         uint32_t slot;
         if (!wait_page(p, ctl, w, slot)) return false;
@@ -1182,7 +1228,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) ctl->att_o[warp][g * d + lane * DPL + i] = o[g][i];
+        for (int i = 0; i < DPL; ++i) ctl->stage[warp * kAttnCombine + g * d + lane * DPL + i] = o[g][i];
     if (!worker_sync(p, ctl, w)) return false;
     if (a.active) {
         for (int e = tid; e < G * d; e += kWorkerThreads) {
@@ -1195,7 +1241,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
 #pragma unroll
                 for (int k = 0; k < kWorkerWarps; ++k) {
                     const float f = expf(ctl->att_m[k][g] - M);
-                    O = fmaf(f, ctl->att_o[k][e], O);
+                    O = fmaf(f, ctl->stage[k * kAttnCombine + e], O);
                     Lsum = fmaf(f, ctl->att_l[k][g], Lsum);
                 }
             }
@@ -1205,6 +1251,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
         }
     }
     // every partial of this task is written
+    stamp_done(p, w);
     if (!worker_sync(p, ctl, w)) return false;
     if (tid == 0) {
         __threadfence();
@@ -1218,22 +1265,36 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     if (ctl->last_flag) {
         __threadfence();
         if (a.active) {
-            for (int e = tid; e < G * d; e += kWorkerThreads) {
-                const int g = e / d, i = e % d;
-                const int hq = a.kvh * G + g;
-                const float *base = p.part + ((size_t)a.b * s.nq + hq) * s.NC * (d + 2);
-                float M = -INFINITY;
-                for (int c = 0; c < s.NC; ++c) M = fmaxf(M, __ldcg(base + (size_t)c * (d + 2) + d));
-                float num = 0.f, den = 0.f;
-                for (int c = 0; c < s.NC; ++c) {
-                    const float *pc = base + (size_t)c * (d + 2);
-                    const float mc = __ldcg(pc + d);
-                    if (mc == -INFINITY) continue;
-                    const float f = expf(mc - M);
-                    num = fmaf(f, __ldcg(pc + i), num);
-                    den = fmaf(f, __ldcg(pc + d + 1), den);
+            // merge this KV head's chunk partials: stage them in shared memory
+            // with independent loads (one L2 round trip), then combine there
+            const int nc = a.nc;
+            const int per = nc * (d + 2);                       // floats per q head
+            const int hb = min(G, kStageFloats / per);          // q heads per batch
+            const float *blk = p.part + ((size_t)a.b * s.nq + (size_t)a.kvh * G) * s.NC * (d + 2);
+            for (int g0 = 0; g0 < G; g0 += hb) {
+                const int nh = min(hb, G - g0);
+#pragma unroll 4
+                for (int i = tid; i < nh * per; i += kWorkerThreads) {
+                    const int g = i / per, r = i - g * per;
+                    ctl->stage[i] = __ldcg(blk + (size_t)(g0 + g) * s.NC * (d + 2) + r);
                 }
-                p.attn[(size_t)a.b * s.QD + (size_t)hq * d + i] = num / den;
+                if (!worker_sync(p, ctl, w)) return false;
+                for (int e = tid; e < nh * d; e += kWorkerThreads) {
+                    const int g = e / d, i = e - g * d;
+                    const float *sg = ctl->stage + g * per;
+                    float M = -INFINITY;
+                    for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (d + 2) + d]);
+                    float num = 0.f, den = 0.f;
+                    for (int c = 0; c < nc; ++c) {
+                        const float mc = sg[c * (d + 2) + d];
+                        if (mc == -INFINITY) continue;
+                        const float f = expf(mc - M);
+                        num = fmaf(f, sg[c * (d + 2) + i], num);
+                        den = fmaf(f, sg[c * (d + 2) + d + 1], den);
+                    }
+                    p.attn[(size_t)a.b * s.QD + (size_t)(a.kvh * G + g0 + g) * d + i] = num / den;
+                }
+                if (g0 + hb < G && !worker_sync(p, ctl, w)) return false;
             }
         }
         if (!worker_sync(p, ctl, w)) return false;

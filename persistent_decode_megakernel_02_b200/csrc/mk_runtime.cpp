@@ -71,7 +71,7 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     if (c->hidden % 8 || c->ffn % 8 || QD % 8) return MK_ERR_INVALID;
     if (c->hidden > kMaxK || c->ffn > kMaxK || QD > kMaxK) return MK_ERR_INVALID;
     if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return MK_ERR_INVALID;
-    if (c->attn_chunks < 0 || c->timeout_ns < 0) return MK_ERR_INVALID;
+    if (c->attn_chunks < 0 || c->timeout_ns < 0 || c->l2_lookahead_kb < 0) return MK_ERR_INVALID;
     if ((long long)c->max_seq * c->head_dim > (1LL << 40)) return MK_ERR_INVALID;
     if (num_sms < 1 || num_sms > 1024) return MK_ERR_INVALID;
     s.L = c->layers; s.H = c->hidden; s.nq = c->n_q_heads; s.nkv = c->n_kv_heads;
@@ -80,6 +80,8 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     s.theta = c->rope_theta; s.eps = c->rms_eps;
     s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nkv, s.S);
     if (s.NC > 4096) return MK_ERR_INVALID;
+    // one q head's chunk partials must fit the merge's shared staging area
+    if ((long long)s.NC * (s.d + 2) > kStageFloats) return MK_ERR_INVALID;
     return MK_OK;
 }
 
@@ -305,7 +307,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
         std::vector<TraceRec> tr(c->num_tasks);
         for (int i = 0; i < c->num_tasks; ++i) {
             const Task &t = c->h_tasks[i];
-            tr[i] = TraceRec{0, 0, 0, t.sm, t.kind, t.layer, t.trig};
+            tr[i] = TraceRec{0, 0, 0, 0, 0, t.sm, t.kind, t.layer, t.trig};
         }
         MK_TRY(cudaMemcpy(d_trace, tr.data(), sizeof(TraceRec) * c->num_tasks, cudaMemcpyHostToDevice));
     }
@@ -329,7 +331,8 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     p.trace = d_trace;
     p.sm_stats = d_stats;
     p.timeout_ns = cfg->timeout_ns > 0 ? (unsigned long long)cfg->timeout_ns : 2000000000ull;
-    p.l2_prefetch = (cfg->flags & MK_FLAG_NO_L2_PREFETCH) ? 0 : 1;
+    p.l2_lookahead = (cfg->flags & MK_FLAG_NO_L2_PREFETCH) ? 0
+                   : cfg->l2_lookahead_kb > 0 ? 1024LL * cfg->l2_lookahead_kb : kL2Lookahead;
     *out = c;
     return MK_OK;
 }

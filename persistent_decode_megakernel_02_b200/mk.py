@@ -41,6 +41,7 @@ class Config(C.Structure):
         ("max_seq", C.c_int), ("max_batch", C.c_int),
         ("rope_theta", C.c_float), ("rms_eps", C.c_float),
         ("flags", C.c_int), ("attn_chunks", C.c_int), ("timeout_ns", C.c_longlong),
+        ("l2_lookahead_kb", C.c_int),
     ]
 
 
@@ -66,7 +67,8 @@ class Info(C.Structure):
 
 
 class TraceRec(C.Structure):
-    _fields_ = [("t_ready", C.c_ulonglong), ("t_start", C.c_ulonglong), ("t_end", C.c_ulonglong),
+    _fields_ = [("t_ready", C.c_ulonglong), ("t_start", C.c_ulonglong), ("t_input", C.c_ulonglong),
+                ("t_done", C.c_ulonglong), ("t_end", C.c_ulonglong),
                 ("sm", C.c_int), ("kind", C.c_int), ("layer", C.c_int), ("trig_event", C.c_int)]
 
 
@@ -110,12 +112,12 @@ def header_functions() -> list[str]:
 
 
 def make_config(shape, max_seq: int, max_batch: int = 1, flags: int = 0,
-                attn_chunks: int = 0, timeout_ns: int = 0) -> Config:
+                attn_chunks: int = 0, timeout_ns: int = 0, l2_lookahead_kb: int = 0) -> Config:
     """`shape`: a workloads.ModelShape (or anything with the same fields)."""
     return Config(shape.layers, shape.hidden, shape.n_q_heads, shape.n_kv_heads,
                   shape.head_dim, shape.ffn, shape.vocab, int(max_seq), int(max_batch),
                   float(shape.rope_theta), float(shape.rms_eps), int(flags),
-                  int(attn_chunks), int(timeout_ns))
+                  int(attn_chunks), int(timeout_ns), int(l2_lookahead_kb))
 
 
 def plan(cfg: Config, num_sms: int) -> dict:
@@ -153,9 +155,11 @@ class Context:
     `kcache`/`vcache`: per-layer bf16 CUDA tensors [max_batch][nkv][max_seq][d]."""
 
     def __init__(self, weights, kcache, vcache, max_seq: int, max_batch: int = 1,
-                 flags: int = 0, attn_chunks: int = 0, timeout_ns: int = 0):
+                 flags: int = 0, attn_chunks: int = 0, timeout_ns: int = 0,
+                 l2_lookahead_kb: int = 0):
         shape = weights.shape
-        self.cfg = make_config(shape, max_seq, max_batch, flags, attn_chunks, timeout_ns)
+        self.cfg = make_config(shape, max_seq, max_batch, flags, attn_chunks, timeout_ns,
+                               l2_lookahead_kb)
         L = shape.layers
         self._keep = [weights, kcache, vcache]
 
@@ -231,7 +235,8 @@ class Context:
         n = self.info().num_tasks
         recs = (TraceRec * n)()
         _check(_lib.mk_get_trace(self._h, C.cast(recs, C.c_void_p), n), "mk_get_trace")
-        dt = np.dtype([("t_ready", np.uint64), ("t_start", np.uint64), ("t_end", np.uint64),
+        dt = np.dtype([("t_ready", np.uint64), ("t_start", np.uint64), ("t_input", np.uint64),
+                       ("t_done", np.uint64), ("t_end", np.uint64),
                        ("sm", np.int32), ("kind", np.int32), ("layer", np.int32),
                        ("trig_event", np.int32)])
         return np.frombuffer(bytes(recs), dtype=dt).copy()
