@@ -79,8 +79,8 @@ enum mk_flags {
  *  attn_chunks: split-K chunks per (sequence, KV head) in the attention
  *  op; 0 picks one chunk count so that the attention tasks cover the SMs.
  *  timeout_ns: bound on every device-side wait; 0 means 2 s.
- *  l2_lookahead_kb: how far (KiB of weights per SM) the loader prefetches
- *  into L2 beyond its shared-memory ring; 0 picks the default (256).
+ *  l2_lookahead_kb: how far (KiB of weights per SM) a prefetch warp runs
+ *  ahead of the shared-memory ring into L2; 0 means no L2 prefetch.
  */
 typedef struct mk_config {
     int layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
@@ -207,7 +207,8 @@ typedef struct mk_trace_rec {
                                     depend on it may start earlier) */
     unsigned long long t_input;  /* the task's input vector is loaded (and normalised) */
     unsigned long long t_done;   /* all rows computed, before the task-end barrier */
-    unsigned long long t_end;    /* workers finished and signalled */
+    unsigned long long t_end;    /* workers finished and posted the completion */
+    unsigned long long t_wait;   /* ns worker thread 0 spent waiting for pages */
     int sm;                      /* CTA that ran it */
     int kind;                    /* op kind (MK_OP_*) */
     int layer;

@@ -42,7 +42,7 @@ constexpr int kVecMax = 8;          // 16-byte vectors per thread per row (K <= 
 constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 16384
 constexpr int kMaxGroup = 8;        // q heads per KV head handled by one attention task
 constexpr int kMaxHeadDim = 256;
-constexpr long long kL2Lookahead = 256 * 1024;  // default bytes the L2 prefetch runs ahead of the ring
+constexpr long long kL2Lookahead = 0;  // default L2 prefetch distance beyond the ring (0: off; measured no gain)
 constexpr int kStageFloats = 6144;  // shared staging: a GEMV input vector, or attention partials
 constexpr int kL2Chunk = 64 * 1024;             // bytes per L2 prefetch instruction
 
@@ -179,10 +179,10 @@ enum StatSlot {
 };
 
 struct TraceRec {
-    unsigned long long t_ready, t_start, t_input, t_done, t_end;
+    unsigned long long t_ready, t_start, t_input, t_done, t_end, t_wait;
     int32_t sm, kind, layer, trig;
 };
-static_assert(sizeof(TraceRec) == 56, "trace record layout");
+static_assert(sizeof(TraceRec) == 64, "trace record layout");
 
 struct Params {
     Shape s;

@@ -87,11 +87,26 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
 }
+// Same, with an L2 cache policy (createpolicy) for the source lines.
+__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                              uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+// Weights are read once per step: their lines should leave L2 first.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
 __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void prefetch_l1(const void *p) {
-    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+__device__ __forceinline__ void prefetch_l2_line(const void *p) {
+    asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
 }
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
     uint32_t v;
@@ -153,6 +168,7 @@ __device__ __forceinline__ float dot8(const uint4 w, const float *x) {
 constexpr int kAttnCombine = 512;   // G * head_dim handled by the warp combine
 static_assert(kWorkerWarps * kAttnCombine <= kStageFloats, "combine fits the staging area");
 constexpr int kMinChunk = 32;       // fewest positions per active attention chunk
+constexpr int kSigRing = 64;        // pending task completions the signaler can hold
 
 struct __align__(16) SmemCtl {
     uint64_t full[kNumPages];
@@ -162,6 +178,12 @@ struct __align__(16) SmemCtl {
     uint32_t abort;             // this CTA is bailing out
     uint32_t ep;                // epoch of this launch (steps completed + 1)
     uint32_t last_flag;         // broadcast of "this task arrived last"
+    uint32_t loader_done;       // the loader has issued its last page
+    long long issued;           // GEMV bytes the loader has issued into the ring
+    uint64_t xbar;              // staged input vector landed (one phase per staged task)
+    uint32_t sig_post;          // task completions posted by the workers
+    uint32_t sig_done;          // completions the signaler has published
+    uint32_t sig_ev[kSigRing];  // event of each posted completion (ring)
     float red[2][kWorkerWarps][16];
     float scal[kWorkerWarps];
     float att_m[kWorkerWarps][kMaxGroup];
@@ -292,6 +314,21 @@ __device__ __forceinline__ const uint16_t *gemv_base(const Params &p, int kind, 
     }
 }
 
+// GEMV tasks whose input vector the scheduler copies into ctl->stage with
+// one bulk copy as soon as the dependency fires (row-per-warp GEMVs whose
+// input comes from another op; the first layer's QKV reads the embedding).
+__device__ __forceinline__ bool staged_input(const Shape &s, const Task &t) {
+    if (t.kind == OP_ATTN) return false;
+    if (op_k(s, t.kind) > kRowK) return false;
+    return !(t.kind == OP_QKV && t.layer == 0);
+}
+
+__device__ __forceinline__ const float *staged_src(const Params &p, const Task &t) {
+    const int b = 0;
+    return t.kind == OP_OPROJ ? p.attn + (size_t)b * p.s.QD
+         : t.kind == OP_DOWN ? p.act + (size_t)b * p.s.F : p.x + (size_t)b * p.s.H;
+}
+
 __device__ __forceinline__ GemvStream gemv_stream(const Params &p, const Task &t) {
     const int K = op_k(p.s, t.kind);
     const int rpp = rows_per_page(K);
@@ -331,43 +368,45 @@ __device__ __forceinline__ bool ring_acquire(const Params &p, SmemCtl *ctl, Ring
     return true;
 }
 
-// L2 prefetch cursor: walks the GEMV byte ranges of the queue ahead of the
-// ring so HBM keeps streaming while the ring is full.
-struct Prefetcher {
-    int qi, q1;
-    const char *src = nullptr;
-    long long left = 0;
-    long long done = 0;   // GEMV bytes prefetched so far
-    bool more = true;
-    __device__ Prefetcher(int q0, int q1_) : qi(q0 - 1), q1(q1_) {}
-    __device__ void run(const Params &p, long long limit) {
-        while (more && done < limit) {
-            if (left <= 0) {
-                if (++qi >= q1) { more = false; return; }
-                const Task t = p.tasks[p.queue[qi]];
-                if (t.kind == OP_ATTN) continue;
-                GemvStream g = gemv_stream(p, t);
-                src = g.src;
-                left = g.left;
-                continue;
+// L2 prefetcher (one warp, plain prefetch.global.L2 per 128-byte line, so it
+// never queues behind or in front of the loader's bulk copies): walks the
+// GEMV byte ranges of the queue and keeps `lookahead` bytes beyond what the
+// loader has issued into the ring, so HBM keeps streaming while the ring is
+// full.  The loader publishes its progress in ctl->issued.
+__device__ void prefetch_role(const Params &p, SmemCtl *ctl) {
+    const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
+    const int lane = threadIdx.x & 31;
+    long long done = 0;
+    for (int qi = q0; qi < q1; ++qi) {
+        const Task t = p.tasks[p.queue[qi]];
+        if (t.kind == OP_ATTN) continue;
+        GemvStream g = gemv_stream(p, t);
+        const char *src = g.src;
+        long long left = g.left;
+        while (left > 0) {
+            // wait (bounded) until the loader is close enough
+            Spin sp;
+            while (done >= *(volatile long long *)&ctl->issued + p.l2_lookahead) {
+                if (*(volatile uint32_t *)&ctl->loader_done) return;
+                if (!spin_ok(sp, p, ctl, W_EMPTY, 0xffffffffu, 0u)) return;
             }
-            const uint32_t chunk = (uint32_t)min(left, (long long)kL2Chunk);
-            prefetch_l2(src, chunk);
+            const long long chunk = min(left, 4096LL);      // 32 lanes x 128 B
+            if ((long long)lane * 128 < chunk) prefetch_l2_line(src + lane * 128);
             src += chunk;
             left -= chunk;
             done += chunk;
         }
     }
-};
+}
 
 __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     Ring ring;
     ring.stats = p.sm_stats != nullptr;
     const unsigned long long t_begin = ring.stats ? globaltimer() : 0ull;
-    Prefetcher pf(q0, q1);
     long long issued = 0;   // GEMV bytes copied into the ring so far
     bool ok = true;         // false when a wait was abandoned
+    const uint64_t wpol = policy_evict_first();
     for (int qi = q0; qi < q1 && ok; ++qi) {
         const int id = p.queue[qi];
         const Task t = p.tasks[id];
@@ -390,16 +429,17 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         }
         GemvStream g = gemv_stream(p, t);
         for (int k = 0; k < g.npages; ++k) {
-            if (p.l2_lookahead) pf.run(p, issued + p.l2_lookahead);
             const uint32_t bytes = (uint32_t)max(0LL, min((long long)g.page_bytes, g.left));
             uint32_t slot;
             if (!ring_acquire(p, ctl, ring, bytes, (uint32_t)id, slot)) { ok = false; break; }
-            if (bytes) bulk_g2s(pages + (size_t)slot * kPageBytes, g.src, bytes, &ctl->full[slot]);
+            if (bytes) bulk_g2s_hint(pages + (size_t)slot * kPageBytes, g.src, bytes, &ctl->full[slot], wpol);
             g.src += g.page_bytes;
             g.left -= bytes;
             issued += bytes;
+            *(volatile long long *)&ctl->issued = issued;
         }
     }
+    *(volatile uint32_t *)&ctl->loader_done = 1u;
     // Let every copy already issued land before this thread returns, so no
     // bulk copy can still be writing shared memory when the CTA exits.
     const uint32_t seq = ring.seq;
@@ -425,9 +465,23 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
 // ---------------------------------------------------------------------------
 // scheduler role (one thread)
 // ---------------------------------------------------------------------------
+__device__ void scheduler_drain(const Params &p, SmemCtl *ctl, uint32_t copies) {
+    // let the last staged-input copy land before this thread returns
+    if (copies == 0) return;
+    Spin s;
+    while (!mbar_try_wait(&ctl->xbar, (copies - 1u) & 1u)) {
+        if ((++s.n & 127u) == 0u) {
+            const unsigned long long now = globaltimer();
+            if (s.t0 == 0) s.t0 = now;
+            else if (now - s.t0 > p.timeout_ns) break;
+        }
+    }
+}
+
 __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     unsigned long long t_dep = 0;
+    uint32_t copies = 0;   // staged-input copies issued
     for (int qi = q0; qi < q1; ++qi) {
         const int id = p.queue[qi];
         const int dep = p.tasks[id].dep;
@@ -436,13 +490,52 @@ __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
             Spin s;
             const unsigned long long t0 = p.sm_stats ? globaltimer() : 0ull;
             while ((int32_t)(ld_acquire_gpu(&p.events[dep]) - target) < 0)
-                if (!spin_ok(s, p, ctl, W_DEP, (uint32_t)id, (uint32_t)dep)) return;
+                if (!spin_ok(s, p, ctl, W_DEP, (uint32_t)id, (uint32_t)dep)) {
+                    scheduler_drain(p, ctl, copies);
+                    return;
+                }
             if (p.sm_stats) t_dep += globaltimer() - t0;
+        }
+        const Task t = p.tasks[id];
+        if (staged_input(p.s, t)) {
+            // the previous task of this queue must be done with the staging
+            // area (its completion is posted after its last read)
+            Spin s2;
+            while (ld_acquire_cta_shared(&ctl->sig_post) < (uint32_t)(qi - q0))
+                if (!spin_ok(s2, p, ctl, W_READY, (uint32_t)id, 1u)) {
+                    scheduler_drain(p, ctl, copies);
+                    return;
+                }
+            // generic-proxy reads of the stage and the producers' generic
+            // writes of the vector, ordered before the async-proxy copy
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            const uint32_t bytes = (uint32_t)op_k(p.s, t.kind) * 4u;
+            mbar_arrive_expect_tx(&ctl->xbar, bytes);
+            bulk_g2s(ctl->stage, staged_src(p, t), bytes, &ctl->xbar);
+            ++copies;
         }
         if (p.trace) p.trace[id].t_ready = globaltimer();
         st_release_cta_shared(&ctl->ready_upto, (uint32_t)(qi - q0 + 1));
     }
+    scheduler_drain(p, ctl, copies);
     if (p.sm_stats) p.sm_stats[(size_t)blockIdx.x * kStatSlots + ST_SCHED_DEP] = t_dep;
+}
+
+// Publishes task completions: workers post the finished task's event in a
+// shared-memory ring (after the barrier that ends the task), this thread
+// performs the gpu-scope release add, so no worker stalls on the release.
+__device__ void signaler_role(const Params &p, SmemCtl *ctl) {
+    const uint32_t total = (uint32_t)(p.qoff[blockIdx.x + 1] - p.qoff[blockIdx.x]);
+    uint32_t done = 0;
+    while (done < total) {
+        Spin s;
+        uint32_t posted;
+        while ((posted = ld_acquire_cta_shared(&ctl->sig_post)) == done)
+            if (!spin_ok(s, p, ctl, W_READY, 0xfffffffeu, done)) return;
+        for (; done < posted; ++done) red_release_gpu(&p.events[ctl->sig_ev[done % kSigRing]], 1u);
+        *(volatile uint32_t *)&ctl->sig_done = done;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -453,13 +546,14 @@ struct WState {
     uint32_t phase = 0;      // its full-barrier parity
     uint32_t wphase = 0;     // worker-barrier phase
     uint32_t need = 0;       // ready_upto value that activates the current task
+    uint32_t xphase = 0;     // parity of the staged-input barrier
     int red_buf = 0;
     int task_id = 0;
     unsigned long long *stat = nullptr;   // per-phase accumulators in shared memory (trace mode, thread 0)
 };
 // Trace-mode time accounting of worker thread 0, accumulated in shared memory
 // so it costs no registers across the task bodies.
-enum WStat { WS_FULL = 0, WS_READY, WS_SYNC, WS_PRO, WS_DOT, WS_EPI, WS_END, WS_TASKS, WS_ATT, WS_FIRST, kWStats };
+enum WStat { WS_FULL = 0, WS_READY, WS_SYNC, WS_PRO, WS_DOT, WS_EPI, WS_END, WS_TASKS, WS_ATT, WS_FIRST, WS_TASKWAIT, kWStats };
 __device__ __forceinline__ unsigned long long phase_begin(const WState &w) {
     return w.stat ? globaltimer() : 0ull;
 }
@@ -502,6 +596,7 @@ __device__ __forceinline__ bool wait_page(const Params &p, SmemCtl *ctl, WState 
     const unsigned long long t0 = phase_begin(w);
     const bool ok = wait_mbar(&ctl->full[slot], w.phase, p, ctl, W_FULL, (uint32_t)w.task_id);
     phase_end(w, t0, WS_FULL);
+    phase_end(w, t0, WS_TASKWAIT);
     return ok;
 }
 
@@ -557,11 +652,18 @@ __device__ __forceinline__ bool worker_block_sum(const Params &p, SmemCtl *ctl, 
 }
 
 // Signal the task's triggering event after every worker's writes.
-// The CTA-scope worker barrier before this call orders every worker's
-// output stores before it; the gpu-scope release add publishes them with
-// the event.
-__device__ __forceinline__ void signal_event(const Params &p, const Task &t) {
-    red_release_gpu(&p.events[t.trig], 1u);
+// Post the task's completion to the signaler (thread 0, after the barrier
+// that ends the task: every worker's output stores happen before it; the
+// release store to the ring makes them visible to the signaler, whose
+// gpu-scope release add publishes them with the event).
+__device__ __forceinline__ bool signal_event(const Params &p, SmemCtl *ctl, const Task &t) {
+    const uint32_t n = ctl->sig_post;   // only thread 0 writes it
+    Spin s;
+    while (n - *(volatile uint32_t *)&ctl->sig_done >= (uint32_t)kSigRing)
+        if (!spin_ok(s, p, ctl, W_READY, 0xfffffffdu, n)) return false;
+    ctl->sig_ev[n % kSigRing] = (uint32_t)t.trig;
+    st_release_cta_shared(&ctl->sig_post, n + 1u);
+    return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -744,12 +846,12 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
                          : kind == OP_GATEUP ? p.layers[layer].g_mlp
                          : kind == OP_LMHEAD ? p.g_final : nullptr;
     float xr[NVL][8];
+    uint4 gv[NVL];   // the RMSNorm gain slice, loaded before the dependency
     const bool embed_in = kind == OP_QKV && layer == 0;
 #pragma unroll
     for (int j = 0; j < NVL; ++j) {
         const int v = lane + 32 * j;
-        // gains: pulled into L1 now, read after the dependency (no registers held)
-        if (gain && v < K8 && (v & 7) == 0) prefetch_l1(reinterpret_cast<const uint4 *>(gain) + v);
+        gv[j] = (gain && v < K8) ? __ldg(reinterpret_cast<const uint4 *>(gain) + v) : make_uint4(0, 0, 0, 0);
         if (embed_in && v < K8) {
             const uint4 e = __ldg(reinterpret_cast<const uint4 *>(p.embed + (size_t)tok * s.H) + v);
             xr[j][0] = bf_lo(e.x); xr[j][1] = bf_hi(e.x); xr[j][2] = bf_lo(e.y); xr[j][3] = bf_hi(e.y);
@@ -786,8 +888,7 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
             const float sc = 1.0f / sqrtf(warp_sum(ss) / (float)s.H + s.eps);
 #pragma unroll
             for (int j = 0; j < NVL; ++j) {
-                const int v = lane + 32 * j;
-                const uint4 g = v < K8 ? __ldg(reinterpret_cast<const uint4 *>(gain) + v) : make_uint4(0, 0, 0, 0);
+                const uint4 g = gv[j];
                 xr[j][0] *= sc * bf_lo(g.x); xr[j][1] *= sc * bf_hi(g.x);
                 xr[j][2] *= sc * bf_lo(g.y); xr[j][3] *= sc * bf_hi(g.y);
                 xr[j][4] *= sc * bf_lo(g.z); xr[j][5] *= sc * bf_hi(g.z);
@@ -795,18 +896,19 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
             }
         }
     } else {
-        // the activation, straight from L2 into every warp (each warp holds
-        // the whole vector and normalises it itself: no block barrier, so a
-        // warp still finishing the previous task delays nobody)
-        const float *src = kind == OP_OPROJ ? p.attn + (size_t)b * s.QD
-                         : kind == OP_DOWN ? p.act + (size_t)b * s.F : p.x + (size_t)b * s.H;
+        // the activation: the scheduler copied it into ctl->stage when the
+        // dependency fired; every warp takes the whole vector from there and
+        // normalises it itself (no block barrier)
+        if (!wait_mbar(&ctl->xbar, w.xphase, p, ctl, W_FULL, (uint32_t)w.task_id)) return false;
+        w.xphase ^= 1u;
+        const float4 *src = reinterpret_cast<const float4 *>(ctl->stage);
         float ss = 0.f;
 #pragma unroll
         for (int j = 0; j < NVL; ++j) {
             const int v = lane + 32 * j;
             if (v < K8) {
-                const float4 a0 = __ldcg(reinterpret_cast<const float4 *>(src) + 2 * v);
-                const float4 a1 = __ldcg(reinterpret_cast<const float4 *>(src) + 2 * v + 1);
+                const float4 a0 = src[2 * v];
+                const float4 a1 = src[2 * v + 1];
                 xr[j][0] = a0.x; xr[j][1] = a0.y; xr[j][2] = a0.z; xr[j][3] = a0.w;
                 xr[j][4] = a1.x; xr[j][5] = a1.y; xr[j][6] = a1.z; xr[j][7] = a1.w;
             } else {
@@ -822,8 +924,7 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
             const float sc = 1.0f / sqrtf(warp_sum(ss) / (float)s.H + s.eps);
 #pragma unroll
             for (int j = 0; j < NVL; ++j) {
-                const int v = lane + 32 * j;
-                const uint4 g = v < K8 ? __ldg(reinterpret_cast<const uint4 *>(gain) + v) : make_uint4(0, 0, 0, 0);
+                const uint4 g = gv[j];
                 xr[j][0] *= sc * bf_lo(g.x); xr[j][1] *= sc * bf_hi(g.x);
                 xr[j][2] *= sc * bf_lo(g.y); xr[j][3] *= sc * bf_hi(g.y);
                 xr[j][4] *= sc * bf_lo(g.z); xr[j][5] *= sc * bf_hi(g.z);
@@ -1259,7 +1360,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
         const uint32_t old = atom_add_acqrel_gpu(cnt, 1u);
         const uint32_t last = (old + 1u == (uint32_t)s.NC * ctl->ep) ? 1u : 0u;
         ctl->last_flag = last;
-        if (!last) red_release_gpu(&p.events[t.trig], 1u);
+        if (!last) signal_event(p, ctl, t);
     }
     if (!worker_sync(p, ctl, w)) return false;
     if (ctl->last_flag) {
@@ -1298,7 +1399,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
             }
         }
         if (!worker_sync(p, ctl, w)) return false;
-        if (tid == 0) signal_event(p, t);
+        if (tid == 0) signal_event(p, ctl, t);
     }
     phase_end(w, tp, WS_ATT);
     return true;
@@ -1381,9 +1482,15 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
                     }
                 }
             }
-            if (tid == 0) signal_event(p, t);
+            if (tid == 0) signal_event(p, ctl, t);
         }
-        if (p.trace && tid == 0) p.trace[id].t_end = globaltimer();
+        if (p.trace && tid == 0) {
+            p.trace[id].t_end = globaltimer();
+            if (w.stat) {
+                p.trace[id].t_wait = w.stat[WS_TASKWAIT];
+                w.stat[WS_TASKWAIT] = 0;
+            }
+        }
         phase_end(w, te, WS_END);
         if (w.stat) w.stat[WS_TASKS] += 1;
     }
@@ -1418,10 +1525,15 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
             mbar_init(&ctl->empty[i], kWorkerWarps);
         }
         mbar_init(&ctl->wbar, kWorkerWarps);
+        mbar_init(&ctl->xbar, 1);
+        ctl->sig_post = 0;
+        ctl->sig_done = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         ctl->ready_upto = 0;
         ctl->last_flag = 0;
+        ctl->loader_done = 0;
+        ctl->issued = 0;
         ctl->ep = ld_volatile_u32(p.epoch) + 1u;
         uint32_t stop = ld_volatile_u32(p.abort_flag) ? 1u : 0u;
         for (int b = 0; b < p.batch && !stop; ++b) {
@@ -1454,6 +1566,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
             if (lane == 0) loader_role(p, pages, ctl);
         } else if (warp == kSchedWarp) {
             if (lane == 0) scheduler_role(p, ctl, ctl->ep);
+        } else if (warp == kSchedWarp + 1) {
+            if (p.l2_lookahead) prefetch_role(p, ctl);
+        } else {
+            if (lane == 0) signaler_role(p, ctl);
         }
     }
 }

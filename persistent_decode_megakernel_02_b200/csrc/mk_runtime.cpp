@@ -307,7 +307,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
         std::vector<TraceRec> tr(c->num_tasks);
         for (int i = 0; i < c->num_tasks; ++i) {
             const Task &t = c->h_tasks[i];
-            tr[i] = TraceRec{0, 0, 0, 0, 0, t.sm, t.kind, t.layer, t.trig};
+            tr[i] = TraceRec{0, 0, 0, 0, 0, 0, t.sm, t.kind, t.layer, t.trig};
         }
         MK_TRY(cudaMemcpy(d_trace, tr.data(), sizeof(TraceRec) * c->num_tasks, cudaMemcpyHostToDevice));
     }

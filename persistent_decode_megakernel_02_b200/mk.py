@@ -68,7 +68,7 @@ class Info(C.Structure):
 
 class TraceRec(C.Structure):
     _fields_ = [("t_ready", C.c_ulonglong), ("t_start", C.c_ulonglong), ("t_input", C.c_ulonglong),
-                ("t_done", C.c_ulonglong), ("t_end", C.c_ulonglong),
+                ("t_done", C.c_ulonglong), ("t_end", C.c_ulonglong), ("t_wait", C.c_ulonglong),
                 ("sm", C.c_int), ("kind", C.c_int), ("layer", C.c_int), ("trig_event", C.c_int)]
 
 
@@ -236,7 +236,7 @@ class Context:
         recs = (TraceRec * n)()
         _check(_lib.mk_get_trace(self._h, C.cast(recs, C.c_void_p), n), "mk_get_trace")
         dt = np.dtype([("t_ready", np.uint64), ("t_start", np.uint64), ("t_input", np.uint64),
-                       ("t_done", np.uint64), ("t_end", np.uint64),
+                       ("t_done", np.uint64), ("t_end", np.uint64), ("t_wait", np.uint64),
                        ("sm", np.int32), ("kind", np.int32), ("layer", np.int32),
                        ("trig_event", np.int32)])
         return np.frombuffer(bytes(recs), dtype=dt).copy()
