@@ -36,8 +36,9 @@ static_assert(kWorkerThreads * kWorkerRegs + (kThreads - kWorkerThreads) * kCont
 
 // ---- tiling ------------------------------------------------------------------
 constexpr int kTileRows = 8;        // output rows per GEMV tile
-constexpr int kPageBytes = 32768;   // one shared-memory page
-constexpr int kNumPages = 6;        // pages in the per-SM ring
+constexpr int kPageRowsMax = 16;    // rows one page holds at most (a 16-row unit)
+constexpr int kPageBytes = 65536;   // one shared-memory page
+constexpr int kNumPages = 3;        // pages in the per-SM ring
 constexpr int kVecMax = 8;          // 16-byte vectors per thread per row (K <= 8*8*256)
 constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 16384
 constexpr int kMaxGroup = 8;        // q heads per KV head handled by one attention task
@@ -138,12 +139,12 @@ MK_HD inline int tile_rows(const Shape &s, int kind, int tile) {
 constexpr int kRowK = 2048;
 constexpr int kMaxHidden = 4096;   // pair tiles in the column split hold 2 vectors per thread
 
-// Rows of one page: the largest power of two <= 8 whose rows (K bf16 each)
-// fit in a page.
+// Rows of one page: the largest power of two <= 16 whose rows (K bf16 each)
+// fit in a page (16 for K <= 2048: one page holds a whole 16-row unit).
 MK_HD inline int rows_per_page(int K) {
     int r = kPageBytes / (2 * K);
     int p = 1;
-    while (p * 2 <= r && p * 2 <= kTileRows) p *= 2;
+    while (p * 2 <= r && p * 2 <= kPageRowsMax) p *= 2;
     return p;
 }
 

@@ -161,6 +161,24 @@ __device__ __forceinline__ float dot8(const uint4 w, const float *x) {
     a = fmaf(bf_hi(w.w), x[7], a);
     return a;
 }
+// Packed two-lane fp32 FMA (sm_100): d = a * b + c element-wise on pairs.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+// acc += w (8 bf16) . x (8 fp32), two interleaved partial sums (even, odd)
+__device__ __forceinline__ float2 dot8x2(const uint4 w, const float *x, float2 acc) {
+    acc = ffma2(make_float2(bf_lo(w.x), bf_hi(w.x)), make_float2(x[0], x[1]), acc);
+    acc = ffma2(make_float2(bf_lo(w.y), bf_hi(w.y)), make_float2(x[2], x[3]), acc);
+    acc = ffma2(make_float2(bf_lo(w.z), bf_hi(w.z)), make_float2(x[4], x[5]), acc);
+    acc = ffma2(make_float2(bf_lo(w.w), bf_hi(w.w)), make_float2(x[6], x[7]), acc);
+    return acc;
+}
 
 // ---------------------------------------------------------------------------
 // shared memory
@@ -341,7 +359,7 @@ __device__ __forceinline__ GemvStream gemv_stream(const Params &p, const Task &t
     if (t.kind == OP_LMHEAD) rows = min(rows, (long long)p.s.V - r0);
     g.left = rows * row_bytes;
     g.page_bytes = (uint32_t)(rpp * row_bytes);
-    g.npages = (int)((r1 - r0) / rpp);
+    g.npages = (int)((r1 - r0 + rpp - 1) / rpp);   // a trailing 8-row tile gets a partial page
     return g;
 }
 
@@ -786,32 +804,33 @@ __device__ __forceinline__ float dual_reduce(float a, float c, int lane) {
 
 template <int NVL>
 __device__ __forceinline__ float dot_row(const uint4 *row, const float (&xr)[NVL][8], int K8, int lane) {
-    float acc = 0.f;
+    float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < NVL; ++j) {
         const int v = lane + 32 * j;
-        if (v < K8) acc += dot8(row[v], xr[j]);
+        if (v < K8) acc = dot8x2(row[v], xr[j], acc);
     }
-    return acc;
+    return acc.x + acc.y;
 }
 
-// Two rows against the same input slice (two independent load/FMA streams).
+// Two rows against the same input slice (two independent load/FMA streams,
+// packed two-lane FMAs).
 template <int NVL>
 __device__ __forceinline__ void dot_rows2(const uint4 *ra, const uint4 *rc, const float (&xr)[NVL][8],
                                           int K8, int lane, float &acc_a, float &acc_c) {
-    float a = 0.f, c = 0.f;
+    float2 a = make_float2(0.f, 0.f), c = make_float2(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < NVL; ++j) {
         const int v = lane + 32 * j;
         if (v < K8) {
             const uint4 wa = ra[v];
             const uint4 wc = rc[v];
-            a += dot8(wa, xr[j]);
-            c += dot8(wc, xr[j]);
+            a = dot8x2(wa, xr[j], a);
+            c = dot8x2(wc, xr[j], c);
         }
     }
-    acc_a = a;
-    acc_c = c;
+    acc_a = a.x + a.y;
+    acc_c = c.x + c.y;
 }
 
 // One warp per row.  Each lane keeps NVL 8-element vectors of the input
@@ -942,27 +961,19 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
         const bool pair = tile < npair;
         const bool two = pair || tile + 1 < t.end;
         float acc_a = 0.f, acc_c = 0.f;
-        uint32_t slot_a, slot_c;
-        if (!wait_page(p, ctl, w, slot_a)) return false;
-        const uint4 *row_a = reinterpret_cast<const uint4 *>(pages + (size_t)slot_a * kPageBytes + warp * row_bytes);
+        // the unit's 16 (or 8) rows are one page: rows warp and 8 + warp
+        uint32_t slot;
+        if (!wait_page(p, ctl, w, slot)) return false;
+        tp = phase_begin(w);
+        const unsigned char *pg = pages + (size_t)slot * kPageBytes;
+        const uint4 *row_a = reinterpret_cast<const uint4 *>(pg + warp * row_bytes);
         if (two) {
-            // the unit's second page is the ring's next one
-            const uint32_t s0 = w.slot, p0 = w.phase;
-            if (++w.slot == (uint32_t)kNumPages) { w.slot = 0; w.phase ^= 1u; }
-            if (!wait_page(p, ctl, w, slot_c)) return false;
-            w.slot = s0;
-            w.phase = p0;
-            tp = phase_begin(w);
-            dot_rows2<NVL>(row_a,
-                           reinterpret_cast<const uint4 *>(pages + (size_t)slot_c * kPageBytes + warp * row_bytes),
-                           xr, K8, lane, acc_a, acc_c);
-            release_page(ctl, w, slot_a);
-            release_page(ctl, w, slot_c);
+            dot_rows2<NVL>(row_a, reinterpret_cast<const uint4 *>(pg + (8 + warp) * row_bytes), xr, K8,
+                           lane, acc_a, acc_c);
         } else {
-            tp = phase_begin(w);
             acc_a = dot_row<NVL>(row_a, xr, K8, lane);
-            release_page(ctl, w, slot_a);
         }
+        release_page(ctl, w, slot);
         phase_end(w, tp, WS_DOT);
         tp = phase_begin(w);
         const float v = dual_reduce(acc_a, acc_c, lane);
