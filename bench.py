@@ -72,6 +72,21 @@ def bandwidth_bound_ms(bytes_per_step: float, gbs: float) -> float:
     return bytes_per_step / (gbs * 1e9) * 1e3
 
 
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu capture, only while the
+    library build is the one that was profiled (else None)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        with open(os.path.join(ROOT, "persistent_decode_megakernel_02_b200", "libmk.so.sha256")) as f:
+            digest = f.read().strip()
+    except (OSError, ValueError):
+        return None
+    if t.get("workload") != workload or t.get("build_digest") != digest:
+        return None
+    return int(t["dram_bytes_read_per_launch"]) + int(t["dram_bytes_write_per_launch"])
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -308,7 +323,8 @@ def main():
     peaks = measured_peaks()
     achieved = alg_bytes / (per_launch_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": profiled_traffic(args.workload),
                 "peak_source": peaks["source"], "bytes_per_launch": int(alg_bytes),
                 "bound_ms": round(bandwidth_bound_ms(alg_bytes, peaks["hbm_gbs"]), 4)}
 
