@@ -246,6 +246,54 @@ int mk_plan(const mk_config *cfg, int num_sms, mk_info *info,
             int32_t *task_out, int32_t *queue_out, int32_t *qoff_out,
             uint32_t *thresholds_out, int64_t *bytes_out);
 
+/* ---- decode without allocating --------------------------------------- */
+
+/*
+ * For callers that cannot allocate device memory where they decode (an
+ * arena that owns all device memory, an allocation-free serving loop):
+ * mk_decode_step_static runs the same decode step as mk_decode_step without
+ * a context and without allocating anything.  The pages describing this
+ * method have no counterpart of it; it is an addition of this library.
+ *
+ * Its scratch (task tables, RoPE table, activations, attention partials,
+ * counters, error word) lives in one fixed device array of
+ * MK_STATIC_SCRATCH_BYTES that every GPU which loads the library holds
+ * until the process exits.  Shapes whose scratch does not fit are rejected
+ * with MK_ERR_INVALID (the 1B shape at max_seq 16640 uses about 5 MiB).
+ * Every call shares that array and leaves its last contents there: calls
+ * that overlap on the GPU (several streams or host threads) race.  The
+ * first call on a device looks up the array's address and sets up the
+ * kernel for that device (and uploads the task tables when the shape
+ * changes, synchronising the stream); make that first call before any
+ * stream capture.  MK_FLAG_TRACE is not supported here.
+ *
+ * Weights come already in the kernel's streaming layout (mk_create makes
+ * this copy itself; this entry point cannot allocate one):
+ *   qkv [layers] -> bf16 [(n_q_heads + 2*n_kv_heads)*head_dim][hidden]:
+ *       for each q head, then each k head, head_dim/16 tiles of 16 rows
+ *       (rows 8j..8j+7 of the head, then rows head_dim/2+8j..+7), then the
+ *       n_kv_heads*head_dim value rows in their own order;
+ *   gu  [layers] -> bf16 [2*ffn][hidden]: for each j < ffn/8, gate rows
+ *       8j..8j+7 then up rows 8j..8j+7;
+ *   the other members as in mk_weights.
+ * tokens, positions, logits_out, next_tok_out, stream: as mk_decode_step.
+ * status_out: device int32 [1] or NULL; receives the step's device status
+ * (MK_OK, MK_ERR_INVALID for an out-of-range token/position,
+ * MK_ERR_TIMEOUT) in stream order.
+ */
+#define MK_STATIC_SCRATCH_BYTES (8u << 20)
+
+typedef struct mk_packed_weights {
+    const void *embed, *lm_head, *final_norm;
+    const void *const *attn_norm, *const *mlp_norm;
+    const void *const *qkv, *const *wo, *const *gu, *const *wd;
+} mk_packed_weights;
+
+int mk_decode_step_static(const mk_config *cfg, const mk_packed_weights *w, const mk_kv *kv,
+                          const int32_t *tokens, const int32_t *positions, int batch,
+                          float *logits_out, int32_t *next_tok_out, int32_t *status_out,
+                          mk_stream_t stream);
+
 /* Test hook: overwrite the threshold of one event (simulates a graph
  * whose event can never fire; the next step then ends in MK_ERR_TIMEOUT).
  * Blocks the host. */

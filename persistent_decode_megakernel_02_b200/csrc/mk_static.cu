@@ -1,0 +1,290 @@
+// mk_static.cu -- mk_decode_step_static: one decode step that allocates
+// nothing.
+//
+// Some callers cannot allocate device memory at the point where they want
+// to decode: code running inside a memory arena that owns all of the
+// device's memory, allocation-free real-time serving loops, or hosts whose
+// allocator must not be entered on the decode path.  This entry point takes
+// everything per call (shape, weights in the kernel's packed layout, KV
+// cache, inputs, outputs) and keeps all of its own scratch -- task tables,
+// RoPE table, activations, attention partials, event counters, error word --
+// in one file-scope device array of fixed size, MK_STATIC_SCRATCH_BYTES,
+// that every GPU which loads the library holds until the process exits.
+// It calls no cudaMalloc, cudaFree or allocating library routine; host
+// staging of the tables uses static host storage.
+//
+// Every call shares that array and leaves the last call's contents in it;
+// calls that overlap on the GPU (different streams, or several host threads)
+// race on it.  The first call on a device looks up the array's device
+// address with cudaGetSymbolAddress (with that device current) and sets the
+// kernel's shared-memory attribute; make that first call before any stream
+// capture.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/mk.h"
+#include "mk_internal.h"
+
+namespace mk {
+size_t kernel_smem_bytes();
+int kernel_launch_regs();
+cudaError_t kernel_prepare();
+cudaError_t kernel_launch(const Params &p, int grid, cudaStream_t stream);
+}  // namespace mk
+
+using namespace mk;
+
+// The scratch of mk_decode_step_static.  In host code this name is only a
+// stand-in for the device array: never pass it to a kernel, pass the address
+// from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_static_scratch[MK_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceSetup {
+    bool ready = false;
+    unsigned char *scratch = nullptr;   // device address of g_static_scratch
+    int num_sms = 0;
+};
+DeviceSetup g_dev[kMaxDevices];
+
+// Host staging of the tables (static storage; no allocation).
+alignas(256) unsigned char g_host[MK_STATIC_SCRATCH_BYTES];
+
+// What the tables currently in a device's scratch were built from: a hash of
+// the shape (task graph, RoPE table) and a hash of the layer pointer table.
+struct Signature {
+    bool valid = false;
+    uint64_t shape_key = 0;
+    uint64_t layer_key = 0;
+};
+Signature g_sig[kMaxDevices];
+
+uint64_t fnv1a(uint64_t h, const void *data, size_t n) {
+    const unsigned char *b = static_cast<const unsigned char *>(data);
+    for (size_t i = 0; i < n; ++i) { h ^= b[i]; h *= 1099511628211ull; }
+    return h;
+}
+
+uint64_t shape_key(const mk_config *c, int num_sms) {
+    const long long f[] = {c->layers, c->hidden, c->n_q_heads, c->n_kv_heads, c->head_dim, c->ffn,
+                           c->vocab, c->max_seq, c->max_batch, c->attn_chunks, num_sms};
+    uint64_t h = fnv1a(1469598103934665603ull, f, sizeof f);
+    const float g[] = {c->rope_theta, c->rms_eps};
+    return fnv1a(h, g, sizeof g);
+}
+
+struct Layout {
+    size_t tasks, queue, qoff, thr, events, merge, ctrl, err, layers, rope;
+    size_t x, q, attn, part, act, aval, aidx, end;
+};
+
+size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
+
+bool shape_ok(const mk_config *c, int num_sms, Shape &s) {
+    if (!c) return false;
+    if (c->layers < 1 || c->hidden < 8 || c->n_q_heads < 1 || c->n_kv_heads < 1 ||
+        c->head_dim < 1 || c->ffn < 8 || c->vocab < 1 || c->max_seq < 1 || c->max_batch < 1)
+        return false;
+    if (c->max_batch > MK_MAX_BATCH || c->n_q_heads % c->n_kv_heads != 0) return false;
+    const int G = c->n_q_heads / c->n_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return false;
+    if (c->head_dim != 64 && c->head_dim != 128) return false;
+    if (G * c->head_dim > 512) return false;
+    const long long QD = (long long)c->n_q_heads * c->head_dim;
+    if (c->hidden % 8 || c->ffn % 8 || QD % 8) return false;
+    if (c->hidden > kMaxHidden || c->ffn > kMaxK || QD > kMaxK) return false;
+    if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return false;
+    if (c->attn_chunks < 0 || c->timeout_ns < 0 || c->l2_lookahead_kb < 0) return false;
+    if (c->flags & MK_FLAG_TRACE) return false;   // no trace buffer in the static scratch
+    s.L = c->layers; s.H = c->hidden; s.nq = c->n_q_heads; s.nkv = c->n_kv_heads;
+    s.d = c->head_dim; s.F = c->ffn; s.V = c->vocab; s.S = c->max_seq; s.Bmax = c->max_batch;
+    s.G = G; s.QD = (int)QD; s.KD = c->n_kv_heads * c->head_dim;
+    s.theta = c->rope_theta; s.eps = c->rms_eps;
+    s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nkv, s.S);
+    if (s.NC > 4096 || (long long)s.NC * (s.d + 2) > kStageFloats) return false;
+    return true;
+}
+
+Layout layout_for(const Shape &s, const PlanSizes &z, int num_sms, int num_lm_tasks) {
+    Layout l;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+    const size_t B = s.Bmax;
+    l.tasks = take(sizeof(Task) * z.num_tasks);
+    l.queue = take(sizeof(int32_t) * z.num_tasks);
+    l.qoff = take(sizeof(int32_t) * (num_sms + 1));
+    l.thr = take(sizeof(uint32_t) * z.num_events);
+    l.events = take(sizeof(uint32_t) * z.num_events);
+    l.merge = take(sizeof(uint32_t) * (size_t)s.L * B * s.nkv);
+    l.ctrl = take(sizeof(uint32_t) * 8);
+    l.err = take(sizeof(ErrWord));
+    l.layers = take(sizeof(LayerW) * s.L);
+    l.rope = take(sizeof(float2) * (size_t)s.S * (s.d / 2));
+    l.x = take(sizeof(float) * B * s.H);
+    l.q = take(sizeof(float) * B * s.QD);
+    l.attn = take(sizeof(float) * B * s.QD);
+    l.part = take(sizeof(float) * B * s.nq * (size_t)s.NC * (s.d + 2));
+    l.act = take(sizeof(float) * B * s.F);
+    l.aval = take(sizeof(float) * B * num_lm_tasks);
+    l.aidx = take(sizeof(int32_t) * B * num_lm_tasks);
+    l.end = o;
+    return l;
+}
+
+bool aligned16(const void *p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+
+extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weights *w,
+                                     const mk_kv *kv, const int32_t *tokens,
+                                     const int32_t *positions, int batch, float *logits_out,
+                                     int32_t *next_tok_out, int32_t *status_out,
+                                     mk_stream_t stream) {
+    if (!cfg || !w || !kv || !tokens || !positions || !next_tok_out) return MK_ERR_INVALID;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MK_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MK_ERR_INVALID;
+    DeviceSetup &ds = g_dev[dev];
+    if (!ds.ready) {
+        // once per device, with that device current
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return MK_ERR_CUDA;
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MK_ERR_CUDA;
+        if (prop.major < 10 || !prop.cooperativeLaunch) return MK_ERR_INVALID;
+        if ((size_t)prop.sharedMemPerBlockOptin < kernel_smem_bytes()) return MK_ERR_INVALID;
+        if (kernel_launch_regs() != kLaunchRegs) return MK_ERR_INVALID;
+        if (kernel_prepare() != cudaSuccess) return MK_ERR_CUDA;
+        ds.scratch = static_cast<unsigned char *>(ptr);
+        ds.num_sms = prop.multiProcessorCount;
+        ds.ready = true;
+    }
+
+    Shape s;
+    if (!shape_ok(cfg, ds.num_sms, s)) return MK_ERR_INVALID;
+    if (batch < 1 || batch > s.Bmax) return MK_ERR_INVALID;
+    if (((uintptr_t)tokens & 3u) || ((uintptr_t)positions & 3u) || ((uintptr_t)next_tok_out & 3u) ||
+        ((uintptr_t)logits_out & 3u) || ((uintptr_t)status_out & 3u))
+        return MK_ERR_INVALID;
+    if (!aligned16(w->embed) || !aligned16(w->lm_head) || !aligned16(w->final_norm)) return MK_ERR_INVALID;
+    if (!w->attn_norm || !w->mlp_norm || !w->qkv || !w->wo || !w->gu || !w->wd || !kv->k || !kv->v)
+        return MK_ERR_INVALID;
+    for (int l = 0; l < s.L; ++l) {
+        const void *ps[] = {w->attn_norm[l], w->mlp_norm[l], w->qkv[l], w->wo[l], w->gu[l],
+                            w->wd[l], kv->k[l], kv->v[l]};
+        for (const void *q : ps)
+            if (!aligned16(q)) return MK_ERR_INVALID;
+    }
+
+    const PlanSizes z = plan_sizes(s, ds.num_sms);
+    const int num_lm = (s.V + 7) / 8 < ds.num_sms ? (s.V + 7) / 8 : ds.num_sms;
+    const Layout lay = layout_for(s, z, ds.num_sms, num_lm);
+    if (lay.end > MK_STATIC_SCRATCH_BYTES) return MK_ERR_INVALID;   // shape too large for the fixed scratch
+
+    unsigned char *d = ds.scratch;
+    cudaStream_t st = (cudaStream_t)stream;
+    Signature &sig = g_sig[dev];
+    // the layer pointer table, built every call (small) and uploaded when it
+    // differs from the one in the scratch
+    LayerW *lw = reinterpret_cast<LayerW *>(g_host + lay.layers);
+    for (int l = 0; l < s.L; ++l) {
+        lw[l].qkv = (const uint16_t *)w->qkv[l];
+        lw[l].gu = (const uint16_t *)w->gu[l];
+        lw[l].wo = (const uint16_t *)w->wo[l];
+        lw[l].wd = (const uint16_t *)w->wd[l];
+        lw[l].g_attn = (const uint16_t *)w->attn_norm[l];
+        lw[l].g_mlp = (const uint16_t *)w->mlp_norm[l];
+        lw[l].kc = (uint16_t *)kv->k[l];
+        lw[l].vc = (uint16_t *)kv->v[l];
+    }
+    const uint64_t skey = shape_key(cfg, ds.num_sms);
+    const uint64_t lkey = fnv1a(skey, lw, sizeof(LayerW) * s.L);
+    if (!sig.valid || sig.shape_key != skey) {
+        // task graph and RoPE table for this shape, in static host storage
+        sig.valid = false;
+        Plan plan;
+        plan.tasks = reinterpret_cast<Task *>(g_host + lay.tasks);
+        plan.queue = reinterpret_cast<int32_t *>(g_host + lay.queue);
+        plan.qoff = reinterpret_cast<int32_t *>(g_host + lay.qoff);
+        plan.thresholds = reinterpret_cast<uint32_t *>(g_host + lay.thr);
+        plan.bytes = nullptr;
+        plan_build(s, ds.num_sms, plan);
+        float2 *rope = reinterpret_cast<float2 *>(g_host + lay.rope);
+        const int half = s.d / 2;
+        for (int pos = 0; pos < s.S; ++pos)
+            for (int i = 0; i < half; ++i) {
+                const double ang = (double)pos * std::pow((double)cfg->rope_theta, -2.0 * i / (double)s.d);
+                rope[(size_t)pos * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+            }
+        if (cudaMemcpyAsync(d + lay.tasks, g_host + lay.tasks, lay.events - lay.tasks,
+                            cudaMemcpyHostToDevice, st) != cudaSuccess ||
+            cudaMemcpyAsync(d + lay.rope, g_host + lay.rope, lay.x - lay.rope,
+                            cudaMemcpyHostToDevice, st) != cudaSuccess ||
+            cudaStreamSynchronize(st) != cudaSuccess)
+            return MK_ERR_CUDA;
+        sig.shape_key = skey;
+        sig.layer_key = 0;
+        sig.valid = true;
+    }
+    if (sig.layer_key != lkey) {
+        if (cudaMemcpyAsync(d + lay.layers, lw, sizeof(LayerW) * s.L, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+            cudaStreamSynchronize(st) != cudaSuccess) {
+            sig.valid = false;
+            return MK_ERR_CUDA;
+        }
+        sig.layer_key = lkey;
+    }
+    // what must start at zero: event and merge counters, the epoch / done /
+    // abort words and the error word (everything else is written before it
+    // is read within the step)
+    if (cudaMemsetAsync(d + lay.events, 0, lay.layers - lay.events, st) != cudaSuccess) return MK_ERR_CUDA;
+
+    Params p{};
+    p.s = s;
+    p.tasks = reinterpret_cast<const Task *>(d + lay.tasks);
+    p.queue = reinterpret_cast<const int32_t *>(d + lay.queue);
+    p.qoff = reinterpret_cast<const int32_t *>(d + lay.qoff);
+    p.thresholds = reinterpret_cast<const uint32_t *>(d + lay.thr);
+    p.events = reinterpret_cast<uint32_t *>(d + lay.events);
+    p.merge_cnt = reinterpret_cast<uint32_t *>(d + lay.merge);
+    uint32_t *ctrl = reinterpret_cast<uint32_t *>(d + lay.ctrl);
+    p.lm_cnt = ctrl + 0;
+    p.epoch = ctrl + 1;
+    p.done_cnt = ctrl + 2;
+    p.abort_flag = ctrl + 3;
+    p.num_lm_tasks = num_lm;
+    p.layers = reinterpret_cast<const LayerW *>(d + lay.layers);
+    p.embed = (const uint16_t *)w->embed;
+    p.lm_head = (const uint16_t *)w->lm_head;
+    p.g_final = (const uint16_t *)w->final_norm;
+    p.rope = reinterpret_cast<const float2 *>(d + lay.rope);
+    p.tokens = tokens;
+    p.positions = positions;
+    p.batch = batch;
+    p.logits = logits_out;
+    p.next_tok = next_tok_out;
+    p.x = reinterpret_cast<float *>(d + lay.x);
+    p.q = reinterpret_cast<float *>(d + lay.q);
+    p.attn = reinterpret_cast<float *>(d + lay.attn);
+    p.part = reinterpret_cast<float *>(d + lay.part);
+    p.act = reinterpret_cast<float *>(d + lay.act);
+    p.amax_val = reinterpret_cast<float *>(d + lay.aval);
+    p.amax_idx = reinterpret_cast<int32_t *>(d + lay.aidx);
+    p.err = reinterpret_cast<ErrWord *>(d + lay.err);
+    p.trace = nullptr;
+    p.sm_stats = nullptr;
+    p.timeout_ns = cfg->timeout_ns > 0 ? (unsigned long long)cfg->timeout_ns : 2000000000ull;
+    p.l2_lookahead = (cfg->flags & MK_FLAG_NO_L2_PREFETCH) ? 0
+                   : cfg->l2_lookahead_kb > 0 ? 1024LL * cfg->l2_lookahead_kb : kL2Lookahead;
+    if (kernel_launch(p, ds.num_sms, st) != cudaSuccess) return MK_ERR_CUDA;
+    if (status_out &&
+        cudaMemcpyAsync(status_out, d + lay.err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return MK_ERR_CUDA;
+    return MK_OK;
+}

@@ -59,6 +59,12 @@ class KV(C.Structure):
     _fields_ = [("k", _VPP), ("v", _VPP)]
 
 
+class PackedWeights(C.Structure):
+    _fields_ = [("embed", C.c_void_p), ("lm_head", C.c_void_p), ("final_norm", C.c_void_p),
+                ("attn_norm", _VPP), ("mlp_norm", _VPP),
+                ("qkv", _VPP), ("wo", _VPP), ("gu", _VPP), ("wd", _VPP)]
+
+
 class Info(C.Structure):
     _fields_ = [("num_sms", C.c_int), ("num_tasks", C.c_int), ("num_events", C.c_int),
                 ("num_ops", C.c_int), ("attn_chunks", C.c_int), ("max_queue", C.c_int),
@@ -88,9 +94,11 @@ _lib.mk_get_graph.argtypes = [_P, _P, _P, _P]
 _lib.mk_get_sm_stats.argtypes = [_P, _P, C.c_int]
 _lib.mk_plan.argtypes = [C.POINTER(Config), C.c_int, C.POINTER(Info), _P, _P, _P, _P, _P]
 _lib.mk_debug_set_threshold.argtypes = [_P, C.c_int, C.c_uint]
+_lib.mk_decode_step_static.argtypes = [C.POINTER(Config), C.POINTER(PackedWeights), C.POINTER(KV),
+                                       _P, _P, C.c_int, _P, _P, _P, _P]
 for _f in ("mk_create", "mk_decode_step", "mk_sync", "mk_reset", "mk_destroy", "mk_get_info",
            "mk_get_event_counts", "mk_read_buffer", "mk_get_trace", "mk_get_graph", "mk_plan",
-           "mk_get_sm_stats",
+           "mk_get_sm_stats", "mk_decode_step_static",
            "mk_debug_set_threshold"):
     getattr(_lib, _f).restype = C.c_int
 
@@ -141,6 +149,32 @@ def plan(cfg: Config, num_sms: int) -> dict:
 
 def _ptr(t) -> int:
     return int(t.data_ptr())
+
+
+def decode_step_static(cfg: Config, packed: dict, kcache, vcache, tokens, positions, next_tok,
+                       logits=None, status=None, stream=None, batch=None) -> int:
+    """mk_decode_step_static: one step without a context and without any
+    allocation.  `packed`: dict of CUDA tensors embed, lm_head, final_norm and
+    per-layer lists attn_norm, mlp_norm, qkv, wo, gu, wd (qkv and gu in the
+    packed tile order documented in mk.h).  Returns the status code."""
+    L = len(packed["qkv"])
+    keep = []
+
+    def arr(ts):
+        a = (C.c_void_p * L)(*[_ptr(t) for t in ts])
+        keep.append(a)
+        return C.cast(a, _VPP)
+
+    w = PackedWeights(_ptr(packed["embed"]), _ptr(packed["lm_head"]), _ptr(packed["final_norm"]),
+                      arr(packed["attn_norm"]), arr(packed["mlp_norm"]), arr(packed["qkv"]),
+                      arr(packed["wo"]), arr(packed["gu"]), arr(packed["wd"]))
+    kv = KV(arr(kcache), arr(vcache))
+    b = int(tokens.numel()) if batch is None else int(batch)
+    return _lib.mk_decode_step_static(C.byref(cfg), C.byref(w), C.byref(kv), _ptr(tokens),
+                                      _ptr(positions), b,
+                                      _ptr(logits) if logits is not None else None,
+                                      _ptr(next_tok), _ptr(status) if status is not None else None,
+                                      _stream_ptr(stream))
 
 
 def _stream_ptr(stream) -> int | None:
