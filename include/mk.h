@@ -61,13 +61,20 @@ enum mk_status {
 };
 
 enum mk_flags {
-    MK_FLAG_TRACE = 1,        /* record a per-task timing trace (globaltimer) */
-    MK_FLAG_NO_L2_PREFETCH = 2 /* loader does not prefetch ahead into L2     */
+    MK_FLAG_TRACE = 1,          /* record a per-task timing trace (globaltimer) */
+    MK_FLAG_NO_L2_PREFETCH = 2, /* loader does not prefetch ahead into L2     */
+    /* Gate every task on its dependency's event counter (a scheduler warp
+     * spins until counter >= threshold * epoch, the scheduling of MPK's
+     * event model, "显著提升小LLM的性能..." page, Figure 3 text).  Without
+     * it tasks wait on their inputs directly: every activation is stored
+     * with the step's tag in the same 64-bit word and readers poll the tags.
+     * Results are identical either way; the counters are bumped either way. */
+    MK_FLAG_EVENT_WAIT = 4
 };
 
 /* Upper bounds of the shapes the kernel tiles. */
 #define MK_MAX_BATCH 1
-#define MK_MAX_K 16384      /* max of hidden, n_q_heads*head_dim and ffn */
+#define MK_MAX_K 14336      /* max of hidden, n_q_heads*head_dim and ffn */
 #define MK_MAX_HEAD_DIM 256
 
 /*
@@ -202,9 +209,13 @@ int mk_read_buffer(mk_ctx *ctx, int which, float *host_out, size_t count);
 /* Per-task trace of the last step (MK_FLAG_TRACE).  Records are
  * mk_trace_rec [num_tasks], indexed by task id. */
 typedef struct mk_trace_rec {
-    unsigned long long t_ready;  /* globaltimer ns: scheduler saw the dependency fire */
+    unsigned long long t_ready;  /* globaltimer ns: the dependency was seen met (the
+                                    scheduler saw the event fire; without
+                                    MK_FLAG_EVENT_WAIT: every input word the
+                                    task reads carried this step's tag) */
     unsigned long long t_start;  /* workers passed the dependency (loads that do not
-                                    depend on it may start earlier) */
+                                    depend on it may start earlier); without
+                                    MK_FLAG_EVENT_WAIT equal to t_ready */
     unsigned long long t_input;  /* the task's input vector is loaded (and normalised) */
     unsigned long long t_done;   /* all rows computed, before the task-end barrier */
     unsigned long long t_end;    /* workers finished and posted the completion */
@@ -298,6 +309,13 @@ int mk_decode_step_static(const mk_config *cfg, const mk_packed_weights *w, cons
  * whose event can never fire; the next step then ends in MK_ERR_TIMEOUT).
  * Blocks the host. */
 int mk_debug_set_threshold(mk_ctx *ctx, int event, uint32_t threshold);
+
+/* Test hook for the tagged-input waits: from the next step on, the tasks
+ * that trigger `event` store their outputs with a stale tag, so the tasks
+ * reading them wait until timeout_ns and the step ends in MK_ERR_TIMEOUT
+ * (every wait is bounded; nothing faults).  event = -1 turns it off;
+ * mk_reset turns it off too.  Host-side only (applies to later launches). */
+int mk_debug_withhold_event(mk_ctx *ctx, int event);
 
 #ifdef __cplusplus
 }

@@ -103,15 +103,24 @@ struct Builder {
     // One task per attention item.  Items go to distinct SMs (the least
     // loaded ones) so an SM runs a second item of the same op only when
     // there are more items than SMs.
+    // Work items (sequence, KV head, chunk) in descending chunk order: chunk
+    // 0's task merges its KV head's partials and waits for the other chunks,
+    // so on every queue it must come after any other chunk it could wait for
+    // (the queues keep this order); chunks > 0 wait on nothing in the op.
     int attn_op(int layer, int dep, int trig) {
         OpTiles t = op_tiles(s);
         int per_chunk = (s.S + s.NC - 1) / s.NC;
         int64_t est = (int64_t)4 * s.d * per_chunk;   // K + V bf16 of one chunk at capacity
+        const int heads = s.Bmax * s.nkv;             // items per chunk index
         for (int i = 0; i < t.attn_items; i += p.num_sms) {
             sort_by_load();
             int n = t.attn_items - i < p.num_sms ? t.attn_items - i : p.num_sms;
-            for (int k = 0; k < n; ++k)
-                add(OP_ATTN, layer, dep, trig, i + k, i + k + 1, order[k], i + k, est);
+            for (int k = 0; k < n; ++k) {
+                const int ord = i + k;
+                const int c = s.NC - 1 - ord / heads;
+                const int item = (ord % heads) * s.NC + c;
+                add(OP_ATTN, layer, dep, trig, item, item + 1, order[k], ord, est);
+            }
         }
         return t.attn_items;
     }

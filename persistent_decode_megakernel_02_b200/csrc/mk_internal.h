@@ -25,7 +25,7 @@ namespace mk {
 constexpr int kWorkerWarps = 8;                     // run task bodies
 constexpr int kWorkerThreads = kWorkerWarps * 32;   // 256
 constexpr int kLoaderWarp = kWorkerWarps;           // streams weight pages
-constexpr int kSchedWarp = kWorkerWarps + 1;        // waits on events, activates tasks
+constexpr int kSchedWarp = kWorkerWarps + 1;        // waits on events (when gating by events)
 constexpr int kThreads = (kWorkerWarps + 4) * 32;   // 384
 constexpr int kLaunchRegs = 168;
 constexpr int kWorkerRegs = 224;
@@ -39,8 +39,8 @@ constexpr int kTileRows = 8;        // output rows per GEMV tile
 constexpr int kPageRowsMax = 16;    // rows one page holds at most (a 16-row unit)
 constexpr int kPageBytes = 65536;   // one shared-memory page
 constexpr int kNumPages = 3;        // pages in the per-SM ring
-constexpr int kVecMax = 8;          // 16-byte vectors per thread per row (K <= 8*8*256)
-constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 16384
+constexpr int kVecMax = 7;          // 16-byte vectors per thread per row (K <= 7*8*256)
+constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 14336
 constexpr int kMaxGroup = 8;        // q heads per KV head handled by one attention task
 constexpr int kMaxHeadDim = 256;
 constexpr long long kL2Lookahead = 0;  // default L2 prefetch distance beyond the ring (0: off; measured no gain)
@@ -151,6 +151,45 @@ MK_HD inline int rows_per_page(int K) {
 // Attention positions per page (K block and V block of `n` positions).
 MK_HD inline int attn_pos_per_page(int d) { return kPageBytes / (4 * d); }
 
+// ---- tagged activations -------------------------------------------------------
+// Every activation one task hands to another lives in a "tagged" buffer: one
+// 64-bit word per fp32 value, the value's bits in the low half and the step
+// tag (the launch's epoch) in the high half, written with one 64-bit store.
+// A consumer polls the words it needs until every tag equals the current
+// epoch, so the data carries its own readiness: no fence, counter or extra
+// copy sits between a producer's store and the consumer's read.  Each layer
+// owns its own buffers (nothing is overwritten within a step), so a word's tag
+// is either this step's or an older one.
+//   xa: residual after the O-projection   [Bmax][H]
+//   xb: residual after the down projection [Bmax][H] (layer L-1: final hidden)
+//   q:  rotated queries                    [Bmax][nq * d]
+//   kn, vn: the new position's key (rotated) and value, rounded to bf16
+//                                          [Bmax][nkv * d]
+//   part: split-K attention partials, per q head and chunk o[d], m, l
+//                                          [Bmax][nq][NC][d + 2]
+//   attn: merged attention output          [Bmax][nq * d]
+//   act:  SiLU(gate) * up                  [Bmax][F]
+struct TagLayout {
+    size_t xa, xb, q, kn, vn, part, attn, act;   // word offsets within a layer's block
+    size_t layer;                                // words per layer
+};
+
+MK_HD inline TagLayout tag_layout(const Shape &s) {
+    TagLayout t;
+    const size_t B = (size_t)s.Bmax;
+    size_t o = 0;
+    t.xa = o; o += B * s.H;
+    t.xb = o; o += B * s.H;
+    t.q = o; o += B * s.QD;
+    t.kn = o; o += B * s.KD;
+    t.vn = o; o += B * s.KD;
+    t.part = o; o += B * s.nq * (size_t)s.NC * (s.d + 2);
+    t.attn = o; o += B * s.QD;
+    t.act = o; o += B * s.F;
+    t.layer = (o + 1) & ~(size_t)1;   // keep every block 16-byte aligned
+    return t;
+}
+
 // Device-side error word (mapped pinned host memory).
 struct ErrWord {
     uint32_t code;    // MK_ERR_* (0 = none)
@@ -193,7 +232,6 @@ struct Params {
     const int32_t *qoff;         // [num_sms + 1]
     const uint32_t *thresholds;  // [num_events]
     uint32_t *events;            // [num_events]
-    uint32_t *merge_cnt;         // [L][Bmax][nkv]
     uint32_t *lm_cnt;            // [1]
     uint32_t *epoch;             // [1]: steps completed
     uint32_t *done_cnt;          // [1]: CTAs that have read the epoch
@@ -209,11 +247,8 @@ struct Params {
     float *logits;               // may be null
     int32_t *next_tok;
     // scratch
-    float *x;                    // [Bmax][H] residual stream
-    float *q;                    // [Bmax][QD]
-    float *attn;                 // [Bmax][QD]
-    float *part;                 // [Bmax][nq][NC][d + 2]
-    float *act;                  // [Bmax][F]
+    uint64_t *tag;               // [L][TagLayout::layer] tagged activations
+    TagLayout tl;
     float *amax_val;             // [Bmax][num_lm_tasks]
     int32_t *amax_idx;           // [Bmax][num_lm_tasks]
     // control
@@ -222,6 +257,8 @@ struct Params {
     unsigned long long *sm_stats; // [num_sms][kStatSlots] wait times (ns), null unless tracing
     unsigned long long timeout_ns;
     long long l2_lookahead;      // bytes the L2 prefetch runs ahead of the ring (0: off)
+    int event_wait;              // 1: the scheduler gates tasks on event counters
+    int debug_withhold;          // test hook: tasks triggering this event write stale tags (-1: off)
 };
 
 // ---- host planning -------------------------------------------------------------

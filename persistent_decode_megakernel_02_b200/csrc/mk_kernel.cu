@@ -2,7 +2,7 @@
 //
 // One CTA per SM, launched cooperatively so that every CTA is resident.
 // Each CTA owns a static queue of tasks (built on the host, see
-// mk_graph.cpp) and runs three roles in separate warps:
+// mk_graph.cpp) and runs these roles in separate warps:
 //
 //  * loader warp (one thread): walks the queue ahead of the workers and,
 //    for every page of every upcoming task, waits for a free page of the
@@ -10,15 +10,19 @@
 //    the task's weight rows (or KV-cache prefix) into it, completing on the
 //    page's mbarrier.  Weights do not depend on activations, so this runs
 //    ahead of the task dependencies (the Hazy page's "paged shared memory,
-//    next stage preloads its weights early").  It also issues
-//    cp.async.bulk.prefetch.L2 a bounded distance further ahead so HBM keeps
-//    streaming while the ring is full.
-//  * scheduler warp (one thread): for each queued task, spins (bounded) on
-//    the task's dependent event counter in global memory until it reaches
-//    threshold * epoch, then activates the task for the workers (MPK's
-//    event/threshold model, "显著提升小LLM的性能..." page, Figure 3 text).
-//  * worker warps (8): run the task bodies on CUDA cores and bump the
-//    task's triggering event with a release add when done.
+//    next stage preloads its weights early").
+//  * worker warps (8): run the task bodies on CUDA cores.  A task's input
+//    activations are "tagged" words (value + step tag in one 64-bit store,
+//    see TagLayout); the workers poll the words they read until every tag is
+//    this step's, which is the task's dependency wait.
+//  * signaler warp (one thread): bumps each finished task's triggering event
+//    counter in global memory with a release add (MPK's event/threshold
+//    model, "显著提升小LLM的性能..." page, Figure 3 text), off the workers'
+//    path.
+//  * scheduler warp (one thread, only with MK_FLAG_EVENT_WAIT): spins on each
+//    queued task's dependent event counter until it reaches threshold *
+//    epoch and only then lets the workers start the task -- the pages' own
+//    gating, kept as an option; the tagged words make it redundant.
 //
 // Task bodies (the fused instruction list of the Hazy megakernel page and
 // the per-layer *_layer calls of the MPK walkthrough, section 3.3.1):
@@ -49,7 +53,7 @@ namespace mk {
 // status codes (same values as the public header's enum)
 constexpr uint32_t kErrInvalid = 1, kErrTimeout = 3;
 enum Where : uint32_t { W_DEP = 1, W_READY = 2, W_FULL = 3, W_EMPTY = 4, W_WBAR = 5,
-                        W_INPUT = 6, W_DRAIN = 7 };
+                        W_INPUT = 6, W_DRAIN = 7, W_TAG = 8 };
 
 // ---------------------------------------------------------------------------
 // PTX helpers
@@ -144,6 +148,31 @@ __device__ __forceinline__ uint4 ld_shared_v4(const void *p) {
                  : "r"(smem_addr(p)));
     return v;
 }
+// Tagged activation words: value bits low, step tag high, one 64-bit access
+// (single-copy atomic), so a reader that sees the tag sees the value.
+__device__ __forceinline__ void st_tag(uint64_t *p, float v, uint32_t ep) {
+    const uint64_t w = ((uint64_t)ep << 32) | __float_as_uint(v);
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ ulonglong2 ld_tag2(const uint64_t *p) {
+    ulonglong2 v;
+    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint64_t ld_tag1(const uint64_t *p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+// The tag half of a tagged word alone (polling without keeping values).
+__device__ __forceinline__ uint32_t ld_tag_hi(const uint64_t *p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(reinterpret_cast<const char *>(p) + 4) : "memory");
+    return v;
+}
+__device__ __forceinline__ bool tag_ok(uint64_t w, uint32_t ep) { return (uint32_t)(w >> 32) == ep; }
+__device__ __forceinline__ float tag_val(uint64_t w) { return __uint_as_float((uint32_t)w); }
+
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
@@ -198,7 +227,6 @@ struct __align__(16) SmemCtl {
     uint32_t last_flag;         // broadcast of "this task arrived last"
     uint32_t loader_done;       // the loader has issued its last page
     long long issued;           // GEMV bytes the loader has issued into the ring
-    uint64_t xbar;              // staged input vector landed (one phase per staged task)
     uint32_t sig_post;          // task completions posted by the workers
     uint32_t sig_done;          // completions the signaler has published
     uint32_t sig_ev[kSigRing];  // event of each posted completion (ring)
@@ -206,9 +234,9 @@ struct __align__(16) SmemCtl {
     float scal[kWorkerWarps];
     float att_m[kWorkerWarps][kMaxGroup];
     float att_l[kWorkerWarps][kMaxGroup];
-    // staging area: a GEMV task's input vector (read as float4); an attention
-    // task's per-warp running outputs (kWorkerWarps x kAttnCombine), later
-    // its merge inputs
+    // staging area: a row-per-warp GEMV task's input vector (read as
+    // float4); an attention task's per-warp running outputs (kWorkerWarps x
+    // kAttnCombine), later its merge inputs
     __align__(16) float stage[kStageFloats];
     unsigned long long wstat[16];   // trace-mode time accounting of worker thread 0
 };
@@ -267,6 +295,32 @@ __device__ __forceinline__ bool wait_mbar(uint64_t *bar, uint32_t parity, const 
     while (!mbar_try_wait(bar, parity))
         if (!spin_ok(s, p, ctl, where, task, parity)) return false;
     return true;
+}
+
+// Warp-wide verdict of a bounded wait: lane 0 keeps the budget and raises the
+// error, every lane gets the same answer, so the warp leaves a poll together.
+__device__ __forceinline__ bool warp_spin_ok(Spin &s, const Params &p, SmemCtl *ctl, uint32_t task,
+                                             uint32_t info) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = spin_ok(s, p, ctl, W_TAG, task, info) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// One tagged value, polled by a single thread (rare paths); on an abandoned
+// wait the error is raised and the stale value returned.
+__device__ __forceinline__ float wait_tag1(const Params &p, SmemCtl *ctl, const uint64_t *src, uint32_t ep,
+                                        uint32_t task) {
+    uint64_t v = ld_tag1(src);
+    Spin s;
+    while (!tag_ok(v, ep)) {
+        if (!spin_ok(s, p, ctl, W_TAG, task, 1u)) break;
+        v = ld_tag1(src);
+    }
+    return tag_val(v);
+}
+
+__device__ __forceinline__ uint64_t *tag_buf(const Params &p, int layer, size_t off) {
+    return p.tag + (size_t)layer * p.tl.layer + off;
 }
 
 // ---------------------------------------------------------------------------
@@ -330,21 +384,6 @@ __device__ __forceinline__ const uint16_t *gemv_base(const Params &p, int kind, 
     case OP_GATEUP: return L.gu;
     default: return L.wd;
     }
-}
-
-// GEMV tasks whose input vector the scheduler copies into ctl->stage with
-// one bulk copy as soon as the dependency fires (row-per-warp GEMVs whose
-// input comes from another op; the first layer's QKV reads the embedding).
-__device__ __forceinline__ bool staged_input(const Shape &s, const Task &t) {
-    if (t.kind == OP_ATTN) return false;
-    if (op_k(s, t.kind) > kRowK) return false;
-    return !(t.kind == OP_QKV && t.layer == 0);
-}
-
-__device__ __forceinline__ const float *staged_src(const Params &p, const Task &t) {
-    const int b = 0;
-    return t.kind == OP_OPROJ ? p.attn + (size_t)b * p.s.QD
-         : t.kind == OP_DOWN ? p.act + (size_t)b * p.s.F : p.x + (size_t)b * p.s.H;
 }
 
 __device__ __forceinline__ GemvStream gemv_stream(const Params &p, const Task &t) {
@@ -483,23 +522,11 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
 // ---------------------------------------------------------------------------
 // scheduler role (one thread)
 // ---------------------------------------------------------------------------
-__device__ void scheduler_drain(const Params &p, SmemCtl *ctl, uint32_t copies) {
-    // let the last staged-input copy land before this thread returns
-    if (copies == 0) return;
-    Spin s;
-    while (!mbar_try_wait(&ctl->xbar, (copies - 1u) & 1u)) {
-        if ((++s.n & 127u) == 0u) {
-            const unsigned long long now = globaltimer();
-            if (s.t0 == 0) s.t0 = now;
-            else if (now - s.t0 > p.timeout_ns) break;
-        }
-    }
-}
-
+// Gates the queue on event counters (only when tasks wait on events): task
+// qi becomes ready once its dependency's counter reaches threshold x epoch.
 __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     unsigned long long t_dep = 0;
-    uint32_t copies = 0;   // staged-input copies issued
     for (int qi = q0; qi < q1; ++qi) {
         const int id = p.queue[qi];
         const int dep = p.tasks[id].dep;
@@ -508,35 +535,12 @@ __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
             Spin s;
             const unsigned long long t0 = p.sm_stats ? globaltimer() : 0ull;
             while ((int32_t)(ld_acquire_gpu(&p.events[dep]) - target) < 0)
-                if (!spin_ok(s, p, ctl, W_DEP, (uint32_t)id, (uint32_t)dep)) {
-                    scheduler_drain(p, ctl, copies);
-                    return;
-                }
+                if (!spin_ok(s, p, ctl, W_DEP, (uint32_t)id, (uint32_t)dep)) return;
             if (p.sm_stats) t_dep += globaltimer() - t0;
-        }
-        const Task t = p.tasks[id];
-        if (staged_input(p.s, t)) {
-            // the previous task of this queue must be done with the staging
-            // area (its completion is posted after its last read)
-            Spin s2;
-            while (ld_acquire_cta_shared(&ctl->sig_post) < (uint32_t)(qi - q0))
-                if (!spin_ok(s2, p, ctl, W_READY, (uint32_t)id, 1u)) {
-                    scheduler_drain(p, ctl, copies);
-                    return;
-                }
-            // generic-proxy reads of the stage and the producers' generic
-            // writes of the vector, ordered before the async-proxy copy
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            const uint32_t bytes = (uint32_t)op_k(p.s, t.kind) * 4u;
-            mbar_arrive_expect_tx(&ctl->xbar, bytes);
-            bulk_g2s(ctl->stage, staged_src(p, t), bytes, &ctl->xbar);
-            ++copies;
         }
         if (p.trace) p.trace[id].t_ready = globaltimer();
         st_release_cta_shared(&ctl->ready_upto, (uint32_t)(qi - q0 + 1));
     }
-    scheduler_drain(p, ctl, copies);
     if (p.sm_stats) p.sm_stats[(size_t)blockIdx.x * kStatSlots + ST_SCHED_DEP] = t_dep;
 }
 
@@ -564,7 +568,8 @@ struct WState {
     uint32_t phase = 0;      // its full-barrier parity
     uint32_t wphase = 0;     // worker-barrier phase
     uint32_t need = 0;       // ready_upto value that activates the current task
-    uint32_t xphase = 0;     // parity of the staged-input barrier
+    uint32_t ep = 0;         // this launch's epoch: the tag of this step's activations
+    uint32_t ep_out = 0;     // tag the current task stores (ep, or stale under the test hook)
     int red_buf = 0;
     int task_id = 0;
     unsigned long long *stat = nullptr;   // per-phase accumulators in shared memory (trace mode, thread 0)
@@ -597,9 +602,11 @@ __device__ __forceinline__ bool worker_sync(const Params &p, SmemCtl *ctl, WStat
     return ok;
 }
 
-// Wait until the scheduler has activated the current task (its dependent
-// event fired); bounded.
+// With MK_FLAG_EVENT_WAIT: wait until the scheduler has activated the
+// current task (its dependent event fired); bounded.  Otherwise tasks start
+// at once and wait on their tagged inputs.
 __device__ __forceinline__ bool wait_ready(const Params &p, SmemCtl *ctl, WState &w) {
+    if (!p.event_wait) return true;
     Spin s;
     const unsigned long long t0 = phase_begin(w);
     while (ld_acquire_cta_shared(&ctl->ready_upto) < w.need)
@@ -607,6 +614,16 @@ __device__ __forceinline__ bool wait_ready(const Params &p, SmemCtl *ctl, WState
     phase_end(w, t0, WS_READY);
     if (p.trace && threadIdx.x == 0) p.trace[w.task_id].t_start = globaltimer();
     return true;
+}
+
+// Trace stamps when tasks wait on their tagged inputs: the task counts as
+// ready (and started) once every input word it needs carried this step's tag.
+__device__ __forceinline__ void stamp_ready(const Params &p, const WState &w) {
+    if (p.trace && !p.event_wait && threadIdx.x == 0) {
+        const unsigned long long t = globaltimer();
+        p.trace[w.task_id].t_ready = t;
+        p.trace[w.task_id].t_start = t;
+    }
 }
 
 __device__ __forceinline__ bool wait_page(const Params &p, SmemCtl *ctl, WState &w, uint32_t &slot) {
@@ -684,45 +701,149 @@ __device__ __forceinline__ bool signal_event(const Params &p, SmemCtl *ctl, cons
     return true;
 }
 
+// Copy a tagged vector of n values (n a multiple of 8, n <= 2 * 256 * NP)
+// into ctl->stage, polling every word until it carries this step's tag.  The
+// 256 worker threads take 16-byte pairs round-robin (coalesced), only stale
+// pairs are reloaded.  ss returns the thread's partial sum of squares.  The
+// caller's worker barrier publishes the stage to every warp.
+// Stage layout: the first four values of every 8-value vector v at float4
+// slot v, the last four at slot n/8 + v, so that a warp reading vectors
+// lane + 32 j touches consecutive 16-byte slots (no bank conflicts).
+template <int NP>
+__device__ __forceinline__ bool stage_tagged(const Params &p, SmemCtl *ctl, const WState &w,
+                                             const uint64_t *src, int n, float &ss) {
+    const int tid = threadIdx.x;
+    const int npairs = n >> 1;
+    float2 v[NP];
+    uint32_t pend = 0;
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const int i = tid + j * kWorkerThreads;
+        v[j] = make_float2(0.f, 0.f);
+        if (i < npairs) {
+            const ulonglong2 t = ld_tag2(src + 2 * i);
+            v[j] = make_float2(tag_val(t.x), tag_val(t.y));
+            if (!tag_ok(t.x, w.ep) || !tag_ok(t.y, w.ep)) pend |= 1u << j;
+        }
+    }
+    Spin s;
+    while (__any_sync(0xffffffffu, pend != 0u)) {
+        if (!warp_spin_ok(s, p, ctl, (uint32_t)w.task_id, 0u)) return false;
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            if (pend & (1u << j)) {
+                const ulonglong2 t = ld_tag2(src + 2 * (tid + j * kWorkerThreads));
+                v[j] = make_float2(tag_val(t.x), tag_val(t.y));
+                if (tag_ok(t.x, w.ep) && tag_ok(t.y, w.ep)) pend &= ~(1u << j);
+            }
+        }
+    }
+    float acc = 0.f;
+    float2 *st = reinterpret_cast<float2 *>(ctl->stage);
+    const int n8 = n >> 3;
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const int i = tid + j * kWorkerThreads;
+        if (i < npairs) {
+            st[2 * (((i >> 1) & 1) * n8 + (i >> 2)) + (i & 1)] = v[j];
+            acc = fmaf(v[j].x, v[j].x, fmaf(v[j].y, v[j].y, acc));
+        }
+    }
+    ss = acc;
+    return true;
+}
+
+// Poll nh q heads' partials of one KV head into ctl->stage, densely: head g
+// takes `per` words (its chunks' o[d], m, l) at src + g * stride.  Pairs of
+// words go round-robin over the 256 worker threads; a fresh pair is stored
+// to shared memory at once, so only stale pairs are reloaded and no values
+// stay in registers across the poll.
+__device__ __forceinline__ bool stage_partials(const Params &p, SmemCtl *ctl, const WState &w,
+                                               const uint64_t *src, int nh, int per, int stride) {
+    constexpr int NP = kStageFloats / 2 / kWorkerThreads;   // pairs per thread at most
+    const int tid = threadIdx.x;
+    const int hp = per >> 1, npairs = nh * hp;
+    float2 *st = reinterpret_cast<float2 *>(ctl->stage);
+    uint32_t pend = 0;
+    auto load = [&](int j) {
+        const int i = tid + j * kWorkerThreads;
+        const int g = i / hp;
+        const ulonglong2 q = ld_tag2(src + (size_t)g * stride + 2 * (i - g * hp));
+        if (tag_ok(q.x, w.ep) && tag_ok(q.y, w.ep)) {
+            st[i] = make_float2(tag_val(q.x), tag_val(q.y));
+            pend &= ~(1u << j);
+        } else {
+            pend |= 1u << j;
+        }
+    };
+#pragma unroll
+    for (int j = 0; j < NP; ++j)
+        if (tid + j * kWorkerThreads < npairs) load(j);
+    Spin sp;
+    while (__any_sync(0xffffffffu, pend != 0u)) {
+        if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 5u)) return false;
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+            if (pend & (1u << j)) load(j);
+    }
+    return true;
+}
+
+// One tagged value per lane (lanes with `want`), polled by the whole warp.
+__device__ __forceinline__ bool warp_tag1(const Params &p, SmemCtl *ctl, const WState &w,
+                                          const uint64_t *src, bool want, float &out) {
+    uint64_t v = want ? ld_tag1(src) : 0ull;
+    bool pend = want && !tag_ok(v, w.ep);
+    Spin s;
+    while (__any_sync(0xffffffffu, pend)) {
+        if (!warp_spin_ok(s, p, ctl, (uint32_t)w.task_id, 2u)) return false;
+        if (pend) {
+            v = ld_tag1(src);
+            pend = !tag_ok(v, w.ep);
+        }
+    }
+    out = tag_val(v);
+    return true;
+}
+
 // ---------------------------------------------------------------------------
 // GEMV task bodies
 // ---------------------------------------------------------------------------
-// Input vector of a GEMV op (fp32 scratch, or the bf16 embedding row for the
-// first layer's QKV) and the RMSNorm gain applied to it, if any.
+// Input vector of a GEMV op (a tagged buffer, or the bf16 embedding row for
+// the first layer's QKV) and the RMSNorm gain applied to it, if any.
 struct GemvInput {
-    const float *src;
+    const uint64_t *src;
     const uint16_t *src_bf;
     const uint16_t *gain;
 };
 
 __device__ __forceinline__ GemvInput gemv_input(const Params &p, int kind, int layer, int b) {
     const Shape &s = p.s;
+    const TagLayout &tl = p.tl;
     GemvInput in{nullptr, nullptr, nullptr};
     switch (kind) {
     case OP_QKV:
         if (layer == 0) in.src_bf = p.embed + (size_t)p.tokens[b] * s.H;
-        else in.src = p.x + (size_t)b * s.H;
+        else in.src = tag_buf(p, layer - 1, tl.xb) + (size_t)b * s.H;
         in.gain = p.layers[layer].g_attn;
         break;
-    case OP_GATEUP: in.src = p.x + (size_t)b * s.H; in.gain = p.layers[layer].g_mlp; break;
-    case OP_LMHEAD: in.src = p.x + (size_t)b * s.H; in.gain = p.g_final; break;
-    case OP_OPROJ: in.src = p.attn + (size_t)b * s.QD; break;
-    default: in.src = p.act + (size_t)b * s.F; break;
+    case OP_GATEUP: in.src = tag_buf(p, layer, tl.xa) + (size_t)b * s.H; in.gain = p.layers[layer].g_mlp; break;
+    case OP_LMHEAD: in.src = tag_buf(p, s.L - 1, tl.xb) + (size_t)b * s.H; in.gain = p.g_final; break;
+    case OP_OPROJ: in.src = tag_buf(p, layer, tl.attn) + (size_t)b * s.QD; break;
+    default: in.src = tag_buf(p, layer, tl.act) + (size_t)b * s.F; break;
     }
     return in;
 }
 
-__device__ __forceinline__ void load_vec8(const GemvInput &in, int v, float *x) {
-    if (in.src_bf) {
-        const uint4 e = __ldg(reinterpret_cast<const uint4 *>(in.src_bf) + v);
-        x[0] = bf_lo(e.x); x[1] = bf_hi(e.x); x[2] = bf_lo(e.y); x[3] = bf_hi(e.y);
-        x[4] = bf_lo(e.z); x[5] = bf_hi(e.z); x[6] = bf_lo(e.w); x[7] = bf_hi(e.w);
-    } else {
-        const float4 a0 = __ldcg(reinterpret_cast<const float4 *>(in.src) + 2 * v);
-        const float4 a1 = __ldcg(reinterpret_cast<const float4 *>(in.src) + 2 * v + 1);
-        x[0] = a0.x; x[1] = a0.y; x[2] = a0.z; x[3] = a0.w;
-        x[4] = a1.x; x[5] = a1.y; x[6] = a1.z; x[7] = a1.w;
-    }
+// Residual stream read by the O projection (layer > 0: the previous layer's
+// down output) and the down projection (this layer's O output), and the
+// buffer each writes.
+__device__ __forceinline__ const uint64_t *resid_in(const Params &p, int kind, int layer, int b) {
+    return kind == OP_DOWN ? tag_buf(p, layer, p.tl.xa) + (size_t)b * p.s.H
+                           : tag_buf(p, layer - 1, p.tl.xb) + (size_t)b * p.s.H;
+}
+__device__ __forceinline__ uint64_t *resid_out(const Params &p, int kind, int layer, int b) {
+    return tag_buf(p, layer, kind == OP_DOWN ? p.tl.xb : p.tl.xa) + (size_t)b * p.s.H;
 }
 
 __device__ __forceinline__ void scale_vec8(float *x, float sc, const uint16_t *gain, int v) {
@@ -731,11 +852,43 @@ __device__ __forceinline__ void scale_vec8(float *x, float sc, const uint16_t *g
     x[4] *= sc * bf_lo(g.z); x[5] *= sc * bf_hi(g.z); x[6] *= sc * bf_lo(g.w); x[7] *= sc * bf_hi(g.w);
 }
 
-// Output of one finished row (or RoPE / gate-up pair), written by one lane.
+// Outputs of a rotated q/k row pair (ra: row i of the head, rc: row i + d/2):
+// q goes to its tagged buffer; k is appended to the bf16 cache and, rounded
+// the same way, to the tagged new-key buffer the attention reads.
+__device__ __forceinline__ void qk_store(const Params &p, int layer, int head, int i, float ra, float rc,
+                                         int b, int P, uint32_t ep) {
+    const Shape &s = p.s;
+    if (head < s.nq) {
+        uint64_t *qh = tag_buf(p, layer, p.tl.q) + (size_t)b * s.QD + (size_t)head * s.d;
+        st_tag(qh + i, ra, ep);
+        st_tag(qh + i + s.d / 2, rc, ep);
+    } else {
+        const int kvh = head - s.nq;
+        uint16_t *kh = p.layers[layer].kc + (((size_t)b * s.nkv + kvh) * s.S + P) * s.d;
+        const uint16_t ka = f2bf(ra), kc = f2bf(rc);
+        kh[i] = ka;
+        kh[i + s.d / 2] = kc;
+        uint64_t *kn = tag_buf(p, layer, p.tl.kn) + (size_t)b * s.KD + (size_t)kvh * s.d;
+        st_tag(kn + i, bf2f(ka), ep);
+        st_tag(kn + i + s.d / 2, bf2f(kc), ep);
+    }
+}
+// Value row vr (kv head vr / d, dim vr % d): cache append + tagged copy.
+__device__ __forceinline__ void v_store(const Params &p, int layer, int vr, float a, int b, int P, uint32_t ep) {
+    const Shape &s = p.s;
+    const int kvh = vr / s.d, dd = vr % s.d;
+    const uint16_t vb = f2bf(a);
+    p.layers[layer].vc[(((size_t)b * s.nkv + kvh) * s.S + P) * s.d + dd] = vb;
+    st_tag(tag_buf(p, layer, p.tl.vn) + (size_t)b * s.KD + vr, bf2f(vb), ep);
+}
+
+// Output of one finished row (or RoPE / gate-up pair) of the column-split
+// GEMV, written by one lane (the O and down projections are handled by the
+// caller, which owns the residual).
 //   a: the row's dot product (first-half row of a pair tile);
 //   c: the partner row's (second-half q/k row, or the up row), pair tiles only.
 __device__ __forceinline__ void gemv_epilogue_row(const Params &p, int kind, int layer, int tile,
-                                                  int r, float a, float c, int b, int P,
+                                                  int r, float a, float c, int b, int P, uint32_t ep,
                                                   float &best_v, int &best_i) {
     const Shape &s = p.s;
     switch (kind) {
@@ -746,39 +899,15 @@ __device__ __forceinline__ void gemv_epilogue_row(const Params &p, int kind, int
             const int head = tile / per_head;
             const int i = (tile % per_head) * 8 + r;
             const float2 cs = p.rope[(size_t)P * (s.d / 2) + i];
-            const float ra = a * cs.x - c * cs.y;
-            const float rc = c * cs.x + a * cs.y;
-            if (head < s.nq) {
-                float *qh = p.q + (size_t)b * s.QD + (size_t)head * s.d;
-                qh[i] = ra;
-                qh[i + s.d / 2] = rc;
-            } else {
-                uint16_t *kh = p.layers[layer].kc + (((size_t)b * s.nkv + (head - s.nq)) * s.S + P) * s.d;
-                kh[i] = f2bf(ra);
-                kh[i + s.d / 2] = f2bf(rc);
-            }
+            qk_store(p, layer, head, i, a * cs.x - c * cs.y, c * cs.x + a * cs.y, b, P, ep);
         } else {
-            const int row = (tile - npair) * 8 + r;
-            const int kvh = row / s.d, dd = row % s.d;
-            p.layers[layer].vc[(((size_t)b * s.nkv + kvh) * s.S + P) * s.d + dd] = f2bf(a);
+            v_store(p, layer, (tile - npair) * 8 + r, a, b, P, ep);
         }
         break;
     }
     case OP_GATEUP:
-        p.act[(size_t)b * s.F + tile * 8 + r] = a / (1.0f + expf(-a)) * c;
+        st_tag(tag_buf(p, layer, p.tl.act) + (size_t)b * s.F + tile * 8 + r, a / (1.0f + expf(-a)) * c, ep);
         break;
-    case OP_OPROJ: {
-        const int row = tile * 8 + r;
-        float *xp = p.x + (size_t)b * s.H + row;
-        const float resid = layer == 0 ? bf2f(p.embed[(size_t)p.tokens[b] * s.H + row]) : __ldcg(xp);
-        *xp = resid + a;
-        break;
-    }
-    case OP_DOWN: {
-        float *xp = p.x + (size_t)b * s.H + tile * 8 + r;
-        *xp = __ldcg(xp) + a;
-        break;
-    }
     default: {  // OP_LMHEAD
         const int row = tile * 8 + r;
         if (row < s.V) {
@@ -889,13 +1018,13 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     if (kind == OP_OPROJ && layer == 0 && my_tile < t.end)
         pre0 = bf2f(p.embed[(size_t)tok * s.H + my_tile * 8 + warp]);
 
-    // ---- the dependency, then the activation
+    // ---- the dependency (tagged inputs), then the activation
     if (!wait_ready(p, ctl, w)) return false;
     unsigned long long tp = phase_begin(w);
-    if (((kind == OP_OPROJ && layer > 0) || kind == OP_DOWN) && my_tile < t.end)
-        pre0 = __ldcg(p.x + (size_t)b * s.H + my_tile * 8 + warp);
+    const bool resid_op = (kind == OP_OPROJ && layer > 0) || kind == OP_DOWN;
     if (embed_in) {
         // the embedding row needs no dependency: each warp holds it already
+        stamp_ready(p, w);
         if (gain) {
             float ss = 0.f;
 #pragma unroll
@@ -915,19 +1044,26 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
             }
         }
     } else {
-        // the activation: the scheduler copied it into ctl->stage when the
-        // dependency fired; every warp takes the whole vector from there and
-        // normalises it itself (no block barrier)
-        if (!wait_mbar(&ctl->xbar, w.xphase, p, ctl, W_FULL, (uint32_t)w.task_id)) return false;
-        w.xphase ^= 1u;
-        const float4 *src = reinterpret_cast<const float4 *>(ctl->stage);
+        // the activation: the worker threads copy the tagged vector into
+        // ctl->stage together (waiting for this step's tags), meet, and then
+        // every warp takes the whole vector from there
+        const GemvInput in = gemv_input(p, kind, layer, b);
         float ss = 0.f;
+        if (!stage_tagged<kRowK / 512>(p, ctl, w, in.src, K, ss)) return false;
+        if (resid_op && !warp_tag1(p, ctl, w, resid_in(p, kind, layer, b) + my_tile * 8 + warp,
+                                   my_tile < t.end, pre0))
+            return false;
+        ss = warp_sum(ss);
+        if (lane == 0) ctl->scal[warp] = ss;
+        if (!worker_sync(p, ctl, w)) return false;
+        stamp_ready(p, w);
+        const float4 *src = reinterpret_cast<const float4 *>(ctl->stage);
 #pragma unroll
         for (int j = 0; j < NVL; ++j) {
             const int v = lane + 32 * j;
             if (v < K8) {
-                const float4 a0 = src[2 * v];
-                const float4 a1 = src[2 * v + 1];
+                const float4 a0 = src[v];
+                const float4 a1 = src[K8 + v];
                 xr[j][0] = a0.x; xr[j][1] = a0.y; xr[j][2] = a0.z; xr[j][3] = a0.w;
                 xr[j][4] = a1.x; xr[j][5] = a1.y; xr[j][6] = a1.z; xr[j][7] = a1.w;
             } else {
@@ -936,11 +1072,10 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
             }
         }
         if (gain) {
+            float tot = 0.f;
 #pragma unroll
-            for (int j = 0; j < NVL; ++j)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
-            const float sc = 1.0f / sqrtf(warp_sum(ss) / (float)s.H + s.eps);
+            for (int i = 0; i < kWorkerWarps; ++i) tot += ctl->scal[i];
+            const float sc = 1.0f / sqrtf(tot / (float)s.H + s.eps);
 #pragma unroll
             for (int j = 0; j < NVL; ++j) {
                 const uint4 g = gv[j];
@@ -986,7 +1121,8 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
             const float c = __shfl_sync(0xffffffffu, v, 16);
             if (lane == 0) {
                 if (kind == OP_GATEUP) {
-                    p.act[(size_t)b * s.F + tile * 8 + warp] = v / (1.0f + expf(-v)) * c;
+                    st_tag(tag_buf(p, layer, p.tl.act) + (size_t)b * s.F + tile * 8 + warp,
+                           v / (1.0f + expf(-v)) * c, w.ep_out);
                 } else {
                     const int head = tile / per_head;
                     const int i = (tile % per_head) * 8 + warp;
@@ -996,18 +1132,7 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
                         cs = r.x;
                         sn = r.y;
                     }
-                    const float ra = v * cs - c * sn;
-                    const float rc = c * cs + v * sn;
-                    if (head < s.nq) {
-                        float *qh = p.q + (size_t)b * s.QD + (size_t)head * s.d;
-                        qh[i] = ra;
-                        qh[i + s.d / 2] = rc;
-                    } else {
-                        uint16_t *kh = p.layers[layer].kc +
-                                       (((size_t)b * s.nkv + (head - s.nq)) * s.S + P) * s.d;
-                        kh[i] = f2bf(ra);
-                        kh[i + s.d / 2] = f2bf(rc);
-                    }
+                    qk_store(p, layer, head, i, v * cs - c * sn, c * cs + v * sn, b, P, w.ep_out);
                 }
             }
             tile += 1;
@@ -1015,19 +1140,17 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
             if ((lane == 0) || (lane == 16 && two)) {
                 const int row = my * 8 + warp;
                 switch (kind) {
-                case OP_QKV: {
-                    const int vr = (my - npair) * 8 + warp;
-                    const int kvh = vr / s.d, dd = vr % s.d;
-                    p.layers[layer].vc[(((size_t)b * s.nkv + kvh) * s.S + P) * s.d + dd] = f2bf(v);
+                case OP_QKV:
+                    v_store(p, layer, (my - npair) * 8 + warp, v, b, P, w.ep_out);
                     break;
-                }
                 case OP_OPROJ:
                 case OP_DOWN: {
                     float resid = q0;
                     if (off >= 32)
-                        resid = (kind == OP_OPROJ && layer == 0) ? bf2f(p.embed[(size_t)tok * s.H + row])
-                                                                 : __ldcg(p.x + (size_t)b * s.H + row);
-                    p.x[(size_t)b * s.H + row] = resid + v;
+                        resid = (kind == OP_OPROJ && layer == 0)
+                                    ? bf2f(p.embed[(size_t)tok * s.H + row])
+                                    : wait_tag1(p, ctl, resid_in(p, kind, layer, b) + row, w.ep, (uint32_t)w.task_id);
+                    st_tag(resid_out(p, kind, layer, b) + row, resid + v, w.ep_out);
                     break;
                 }
                 default:   // OP_LMHEAD
@@ -1126,32 +1249,100 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
         resid = bf2f(p.embed[(size_t)tok * s.H + 8 * t.begin + lane]);
     if (!wait_ready(p, ctl, w)) return false;
     unsigned long long tp = phase_begin(w);
-    if (resid_op && !(kind == OP_OPROJ && layer == 0) && warp == 0 && lane < task_rows)
-        resid = __ldcg(p.x + (size_t)b * s.H + 8 * t.begin + lane);
     const GemvInput in = gemv_input(p, kind, layer, b);
+    // thread tid takes 16-byte vectors tid, tid + 256, ... of the input: from
+    // the embedding row, or as 4 tagged pairs each, stale pairs reloaded
+    // until every tag is this step's
     float xr[NV][8];
-    float ss = 0.f;
+    uint32_t pend = 0;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
         const int v = tid + j * kWorkerThreads;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
         if (v < K8) {
-            load_vec8(in, v, xr[j]);
+            if (in.src_bf) {
+                const uint4 e = __ldg(reinterpret_cast<const uint4 *>(in.src_bf) + v);
+                xr[j][0] = bf_lo(e.x); xr[j][1] = bf_hi(e.x); xr[j][2] = bf_lo(e.y); xr[j][3] = bf_hi(e.y);
+                xr[j][4] = bf_lo(e.z); xr[j][5] = bf_hi(e.z); xr[j][6] = bf_lo(e.w); xr[j][7] = bf_hi(e.w);
+            } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
+                for (int h = 0; h < 4; ++h) {
+                    const ulonglong2 q = ld_tag2(in.src + 8 * v + 2 * h);
+                    xr[j][2 * h] = tag_val(q.x);
+                    xr[j][2 * h + 1] = tag_val(q.y);
+                    if (!tag_ok(q.x, w.ep) || !tag_ok(q.y, w.ep)) pend |= 1u << (4 * j + h);
+                }
+            }
         }
     }
+    if (__any_sync(0xffffffffu, pend != 0u)) {
+        Spin sp;
+        if constexpr (NV <= 2) {
+            // few vectors: reload stale pairs with their values
+            while (__any_sync(0xffffffffu, pend != 0u)) {
+                if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 3u)) return false;
+#pragma unroll
+                for (int j = 0; j < NV; ++j)
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        if (pend & (1u << (4 * j + h))) {
+                            const ulonglong2 q = ld_tag2(in.src + 8 * (tid + j * kWorkerThreads) + 2 * h);
+                            xr[j][2 * h] = tag_val(q.x);
+                            xr[j][2 * h + 1] = tag_val(q.y);
+                            if (tag_ok(q.x, w.ep) && tag_ok(q.y, w.ep)) pend &= ~(1u << (4 * j + h));
+                        }
+            }
+        } else {
+            // many vectors: poll only the tag halves of the stale pairs (one
+            // register each), then load the values once more -- a word whose
+            // tag was seen reads back this step's value
+            while (__any_sync(0xffffffffu, pend != 0u)) {
+                if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 3u)) return false;
+#pragma unroll
+                for (int j = 0; j < NV; ++j)
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        if (pend & (1u << (4 * j + h))) {
+                            const uint64_t *q = in.src + 8 * (tid + j * kWorkerThreads) + 2 * h;
+                            if (ld_tag_hi(q) == w.ep && ld_tag_hi(q + 1) == w.ep) pend &= ~(1u << (4 * j + h));
+                        }
+            }
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                const int v = tid + j * kWorkerThreads;
+                if (v < K8)
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const ulonglong2 q = ld_tag2(in.src + 8 * v + 2 * h);
+                        xr[j][2 * h] = tag_val(q.x);
+                        xr[j][2 * h + 1] = tag_val(q.y);
+                    }
+            }
+        }
+    }
+    if (resid_op && !(kind == OP_OPROJ && layer == 0) && warp == 0 &&
+        !warp_tag1(p, ctl, w, resid_in(p, kind, layer, b) + 8 * t.begin + lane, lane < task_rows, resid))
+        return false;
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(xr[j][e], xr[j][e], ss);
     if (in.gain) {
         float tot;
         if (!worker_block_sum(p, ctl, w, ss, tot)) return false;
+        stamp_ready(p, w);
         const float sc = 1.0f / sqrtf(tot / (float)s.H + s.eps);
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
             const int v = tid + j * kWorkerThreads;
             if (v < K8) scale_vec8(xr[j], sc, in.gain, v);
         }
+    } else {
+        // trace mode: the stamp marks the moment every thread has its input
+        if (p.trace && !p.event_wait && !worker_sync(p, ctl, w)) return false;
+        stamp_ready(p, w);
     }
     phase_end(w, tp, WS_PRO);
     stamp_input(p, w);
@@ -1213,7 +1404,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
             const int grp_row = 8 * (tile - t.begin) + e;   // row within the task
             const float rres = __shfl_sync(0xffffffffu, resid, grp_row & 31);
             if (pair) {
-                if (lane < 8) gemv_epilogue_row(p, kind, layer, tile, lane, a, c, b, P, best_v, best_i);
+                if (lane < 8) gemv_epilogue_row(p, kind, layer, tile, lane, a, c, b, P, w.ep_out, best_v, best_i);
             } else if (lane < rows) {
                 const int tl = tile + (e >> 3), r = e & 7;
                 if (resid_op) {
@@ -1221,10 +1412,11 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
                     const float base = grp_row < 32 ? rres
                                      : (kind == OP_OPROJ && layer == 0)
                                            ? bf2f(p.embed[(size_t)tok * s.H + row])
-                                           : __ldcg(p.x + (size_t)b * s.H + row);
-                    p.x[(size_t)b * s.H + row] = base + a;
+                                           : wait_tag1(p, ctl, resid_in(p, kind, layer, b) + row, w.ep,
+                                                       (uint32_t)w.task_id);
+                    st_tag(resid_out(p, kind, layer, b) + row, base + a, w.ep_out);
                 } else {
-                    gemv_epilogue_row(p, kind, layer, tl, r, a, 0.f, b, P, best_v, best_i);
+                    gemv_epilogue_row(p, kind, layer, tl, r, a, 0.f, b, P, w.ep_out, best_v, best_i);
                 }
             }
         }
@@ -1271,31 +1463,61 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
 #pragma unroll
         for (int i = 0; i < DPL; ++i) { o[g][i] = 0.f; qr[g][i] = 0.f; }
     }
-    if (a.active) {
+    // q of the group's heads (every warp) and the new position's key and
+    // value (the warp that visits it): tagged pairs, polled until fresh
+    const bool new_warp = a.has_new && warp == (a.npre % kWorkerWarps);
+    float kn[DPL], vn[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) { kn[i] = 0.f; vn[i] = 0.f; }
+    {
+        constexpr int QP = G * DPL / 2, KP = DPL / 2;   // pairs per lane
+        const uint64_t *qsrc = tag_buf(p, t.layer, p.tl.q) + (size_t)a.b * s.QD + (size_t)a.kvh * G * d + lane * DPL;
+        const uint64_t *ksrc = tag_buf(p, t.layer, p.tl.kn) + (size_t)a.b * s.KD + (size_t)a.kvh * d + lane * DPL;
+        const uint64_t *vsrc = tag_buf(p, t.layer, p.tl.vn) + (size_t)a.b * s.KD + (size_t)a.kvh * d + lane * DPL;
+        uint32_t pend = 0;
+        auto load = [&](int bit) {
+            // bits [0, QP): q pairs (head g = bit / KP); then KP key pairs, KP value pairs
+            ulonglong2 v;
+            if (bit < QP) {
+                const int g = bit / KP, h = bit % KP;
+                v = ld_tag2(qsrc + (size_t)g * d + 2 * h);
+                qr[g][2 * h] = tag_val(v.x);
+                qr[g][2 * h + 1] = tag_val(v.y);
+            } else if (bit < QP + KP) {
+                const int h = bit - QP;
+                v = ld_tag2(ksrc + 2 * h);
+                kn[2 * h] = tag_val(v.x);
+                kn[2 * h + 1] = tag_val(v.y);
+            } else {
+                const int h = bit - QP - KP;
+                v = ld_tag2(vsrc + 2 * h);
+                vn[2 * h] = tag_val(v.x);
+                vn[2 * h + 1] = tag_val(v.y);
+            }
+            if (!tag_ok(v.x, w.ep) || !tag_ok(v.y, w.ep)) pend |= 1u << bit;
+            else pend &= ~(1u << bit);
+        };
+        if (a.active) {
+#pragma unroll
+            for (int bit = 0; bit < QP + 2 * KP; ++bit)
+                if (bit < QP || new_warp) load(bit);
+        }
+        Spin sp;
+        while (__any_sync(0xffffffffu, pend != 0u)) {
+            if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 4u)) return false;
+#pragma unroll
+            for (int bit = 0; bit < QP + 2 * KP; ++bit)
+                if (pend & (1u << bit)) load(bit);
+        }
         const float scale = 1.0f / sqrtf((float)d);
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float *qh = p.q + (size_t)a.b * s.QD + (size_t)(a.kvh * G + g) * d + lane * DPL;
+        for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) qr[g][i] = __ldcg(qh + i) * scale;
-        }
+            for (int i = 0; i < DPL; ++i) qr[g][i] *= scale;
     }
+    stamp_ready(p, w);
 
-    auto visit = [&](const uint16_t *krow, const uint16_t *vrow, bool global_mem) {
-        float kv[DPL], vv[DPL];
-#pragma unroll
-        for (int i = 0; i < DPL; i += 2) {
-            uint32_t kw, vw;
-            if (global_mem) {
-                kw = __ldcg(reinterpret_cast<const unsigned int *>(krow + lane * DPL + i));
-                vw = __ldcg(reinterpret_cast<const unsigned int *>(vrow + lane * DPL + i));
-            } else {
-                kw = *reinterpret_cast<const uint32_t *>(krow + lane * DPL + i);
-                vw = *reinterpret_cast<const uint32_t *>(vrow + lane * DPL + i);
-            }
-            kv[i] = bf_lo(kw); kv[i + 1] = bf_hi(kw);
-            vv[i] = bf_lo(vw); vv[i + 1] = bf_hi(vw);
-        }
+    auto visit = [&](const float (&kv)[DPL], const float (&vv)[DPL]) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             float sc = 0.f;
@@ -1321,16 +1543,22 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
         const uint16_t *Kp = reinterpret_cast<const uint16_t *>(pages + (size_t)slot * kPageBytes);
         const uint16_t *Vp = Kp + (size_t)npp * d;
         const int n = min(npp, a.npre - pg * npp);
-        for (int j = warp; j < n; j += kWorkerWarps) visit(Kp + (size_t)j * d, Vp + (size_t)j * d, false);
+        for (int j = warp; j < n; j += kWorkerWarps) {
+            float kv[DPL], vv[DPL];
+#pragma unroll
+            for (int i = 0; i < DPL; i += 2) {
+                const uint32_t kw = *reinterpret_cast<const uint32_t *>(Kp + (size_t)j * d + lane * DPL + i);
+                const uint32_t vw = *reinterpret_cast<const uint32_t *>(Vp + (size_t)j * d + lane * DPL + i);
+                kv[i] = bf_lo(kw); kv[i + 1] = bf_hi(kw);
+                vv[i] = bf_lo(vw); vv[i + 1] = bf_hi(vw);
+            }
+            visit(kv, vv);
+        }
         release_page(ctl, w, slot);
         phase_end(w, tp, WS_DOT);
     }
     tp = phase_begin(w);
-    if (a.has_new && warp == (a.npre % kWorkerWarps)) {
-        const LayerW &L = p.layers[t.layer];
-        const size_t off = (((size_t)a.b * s.nkv + a.kvh) * s.S + a.P) * d;
-        visit(L.kc + off, L.vc + off, true);
-    }
+    if (new_warp) visit(kn, vn);
 
     // ---- combine the warps' running states into this chunk's partial
     if (lane == 0) {
@@ -1342,6 +1570,8 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
 #pragma unroll
         for (int i = 0; i < DPL; ++i) ctl->stage[warp * kAttnCombine + g * d + lane * DPL + i] = o[g][i];
     if (!worker_sync(p, ctl, w)) return false;
+    // this chunk's partial (per q head: o[d], m, l) as tagged words
+    uint64_t *part = tag_buf(p, t.layer, p.tl.part) + ((size_t)a.b * s.nq + (size_t)a.kvh * G) * s.NC * (d + 2);
     if (a.active) {
         for (int e = tid; e < G * d; e += kWorkerThreads) {
             const int g = e / d, i = e % d;
@@ -1357,61 +1587,51 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
                     Lsum = fmaf(f, ctl->att_l[k][g], Lsum);
                 }
             }
-            float *dst = p.part + (((size_t)a.b * s.nq + a.kvh * G + g) * s.NC + a.c) * (d + 2);
-            dst[i] = O;
-            if (i == 0) { dst[d] = M; dst[d + 1] = Lsum; }
-        }
-    }
-    // every partial of this task is written
-    stamp_done(p, w);
-    if (!worker_sync(p, ctl, w)) return false;
-    if (tid == 0) {
-        __threadfence();
-        uint32_t *cnt = p.merge_cnt + ((size_t)t.layer * s.Bmax + a.b) * s.nkv + a.kvh;
-        const uint32_t old = atom_add_acqrel_gpu(cnt, 1u);
-        const uint32_t last = (old + 1u == (uint32_t)s.NC * ctl->ep) ? 1u : 0u;
-        ctl->last_flag = last;
-        if (!last) signal_event(p, ctl, t);
-    }
-    if (!worker_sync(p, ctl, w)) return false;
-    if (ctl->last_flag) {
-        __threadfence();
-        if (a.active) {
-            // merge this KV head's chunk partials: stage them in shared memory
-            // with independent loads (one L2 round trip), then combine there
-            const int nc = a.nc;
-            const int per = nc * (d + 2);                       // floats per q head
-            const int hb = min(G, kStageFloats / per);          // q heads per batch
-            const float *blk = p.part + ((size_t)a.b * s.nq + (size_t)a.kvh * G) * s.NC * (d + 2);
-            for (int g0 = 0; g0 < G; g0 += hb) {
-                const int nh = min(hb, G - g0);
-#pragma unroll 4
-                for (int i = tid; i < nh * per; i += kWorkerThreads) {
-                    const int g = i / per, r = i - g * per;
-                    ctl->stage[i] = __ldcg(blk + (size_t)(g0 + g) * s.NC * (d + 2) + r);
-                }
-                if (!worker_sync(p, ctl, w)) return false;
-                for (int e = tid; e < nh * d; e += kWorkerThreads) {
-                    const int g = e / d, i = e - g * d;
-                    const float *sg = ctl->stage + g * per;
-                    float M = -INFINITY;
-                    for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (d + 2) + d]);
-                    float num = 0.f, den = 0.f;
-                    for (int c = 0; c < nc; ++c) {
-                        const float mc = sg[c * (d + 2) + d];
-                        if (mc == -INFINITY) continue;
-                        const float f = expf(mc - M);
-                        num = fmaf(f, sg[c * (d + 2) + i], num);
-                        den = fmaf(f, sg[c * (d + 2) + d + 1], den);
-                    }
-                    p.attn[(size_t)a.b * s.QD + (size_t)(a.kvh * G + g0 + g) * d + i] = num / den;
-                }
-                if (g0 + hb < G && !worker_sync(p, ctl, w)) return false;
+            uint64_t *dst = part + ((size_t)g * s.NC + a.c) * (d + 2);
+            st_tag(dst + i, O, w.ep_out);
+            if (i == 0) {
+                st_tag(dst + d, M, w.ep_out);
+                st_tag(dst + d + 1, Lsum, w.ep_out);
             }
         }
-        if (!worker_sync(p, ctl, w)) return false;
-        if (tid == 0) signal_event(p, ctl, t);
     }
+    stamp_done(p, w);
+    if (a.active && a.c == 0) {
+        // chunk 0's task merges the KV head's partials: it polls them into
+        // shared memory (tagged, so it waits for exactly the chunks it
+        // reads), then combines them there.  No fence or counter: the tags
+        // carry the readiness.
+        const int nc = a.nc;
+        const int per = nc * (d + 2);                       // words per q head
+        const int hb = min(G, kStageFloats / per);          // q heads per batch
+        for (int g0 = 0; g0 < G; g0 += hb) {
+            const int nh = min(hb, G - g0);
+            // every thread is done reading the stage (the combine above, or
+            // the previous batch's merge) before it is refilled
+            if (!worker_sync(p, ctl, w)) return false;
+            if (!stage_partials(p, ctl, w, part + (size_t)g0 * s.NC * (d + 2), nh, per, s.NC * (d + 2)))
+                return false;
+            if (!worker_sync(p, ctl, w)) return false;
+            for (int e = tid; e < nh * d; e += kWorkerThreads) {
+                const int g = e / d, i = e - g * d;
+                const float *sg = ctl->stage + g * per;
+                float M = -INFINITY;
+                for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (d + 2) + d]);
+                float num = 0.f, den = 0.f;
+                for (int c = 0; c < nc; ++c) {
+                    const float mc = sg[c * (d + 2) + d];
+                    if (mc == -INFINITY) continue;
+                    const float f = expf(mc - M);
+                    num = fmaf(f, sg[c * (d + 2) + i], num);
+                    den = fmaf(f, sg[c * (d + 2) + d + 1], den);
+                }
+                st_tag(tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)(a.kvh * G + g0 + g) * d + i,
+                       num / den, w.ep_out);
+            }
+        }
+    }
+    if (!worker_sync(p, ctl, w)) return false;
+    if (tid == 0) signal_event(p, ctl, t);
     phase_end(w, tp, WS_ATT);
     return true;
 }
@@ -1454,11 +1674,13 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         w.stat = ctl->wstat;
         for (int i = 0; i < kWStats; ++i) ctl->wstat[i] = 0;
     }
+    w.ep = ctl->ep;
     const unsigned long long t_begin = phase_begin(w);
     for (int qi = q0; qi < q1; ++qi) {
         const int id = p.queue[qi];
         const Task t = p.tasks[id];
         w.task_id = id;
+        w.ep_out = t.trig == p.debug_withhold ? w.ep - 1u : w.ep;
         w.need = (uint32_t)(qi - q0 + 1);   // the task body waits for it
         if (!run_task(p, t, pages, ctl, w)) return;
         const unsigned long long te = phase_begin(w);
@@ -1536,7 +1758,6 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
             mbar_init(&ctl->empty[i], kWorkerWarps);
         }
         mbar_init(&ctl->wbar, kWorkerWarps);
-        mbar_init(&ctl->xbar, 1);
         ctl->sig_post = 0;
         ctl->sig_done = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1576,7 +1797,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
         if (warp == kLoaderWarp) {
             if (lane == 0) loader_role(p, pages, ctl);
         } else if (warp == kSchedWarp) {
-            if (lane == 0) scheduler_role(p, ctl, ctl->ep);
+            if (lane == 0 && p.event_wait) scheduler_role(p, ctl, ctl->ep);
         } else if (warp == kSchedWarp + 1) {
             if (p.l2_lookahead) prefetch_role(p, ctl);
         } else {

@@ -229,27 +229,22 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     Params &p = c->p;
     p.s = s;
     cudaError_t e = cudaSuccess;
-    Task *d_tasks; int32_t *d_queue, *d_qoff; uint32_t *d_thr, *d_ev, *d_merge, *d_ctrl;
+    Task *d_tasks; int32_t *d_queue, *d_qoff; uint32_t *d_thr, *d_ev, *d_ctrl;
     LayerW *d_layers; float2 *d_rope;
-    float *d_x, *d_q, *d_attn, *d_part, *d_act, *d_aval; int32_t *d_aidx;
+    uint64_t *d_tag; float *d_aval; int32_t *d_aidx;
+    const TagLayout tl = tag_layout(s);
     const size_t B = s.Bmax;
-    const size_t n_merge = (size_t)s.L * B * s.nkv;
 #define MK_TRY(expr) do { e = (expr); if (e != cudaSuccess) { free_ctx(c); return map_cuda(e); } } while (0)
     MK_TRY(dalloc(c, &d_tasks, c->num_tasks));
     MK_TRY(dalloc(c, &d_queue, c->num_tasks));
     MK_TRY(dalloc(c, &d_qoff, c->num_sms + 1));
     MK_TRY(dalloc(c, &d_thr, c->num_events));
     MK_TRY(dalloc(c, &d_ev, c->num_events));
-    MK_TRY(dalloc(c, &d_merge, n_merge));
     MK_TRY(dalloc(c, &d_ctrl, 8));             // lm_cnt, epoch, done_cnt, abort
     MK_TRY(dalloc(c, &c->d_err, 1));
     MK_TRY(dalloc(c, &d_layers, s.L));
     MK_TRY(dalloc(c, &d_rope, (size_t)s.S * half));
-    MK_TRY(dalloc(c, &d_x, B * s.H));
-    MK_TRY(dalloc(c, &d_q, B * s.QD));
-    MK_TRY(dalloc(c, &d_attn, B * s.QD));
-    MK_TRY(dalloc(c, &d_part, B * s.nq * (size_t)s.NC * (s.d + 2)));
-    MK_TRY(dalloc(c, &d_act, B * s.F));
+    MK_TRY(dalloc(c, &d_tag, tl.layer * s.L));
     MK_TRY(dalloc(c, &d_aval, B * c->num_lm_tasks));
     MK_TRY(dalloc(c, &d_aidx, B * c->num_lm_tasks));
     TraceRec *d_trace = nullptr;
@@ -296,13 +291,9 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     MK_TRY(cudaMemcpy(d_layers, lw.data(), sizeof(LayerW) * s.L, cudaMemcpyHostToDevice));
     MK_TRY(cudaMemcpy(d_rope, rope.data(), sizeof(float) * rope.size(), cudaMemcpyHostToDevice));
     MK_TRY(cudaMemset(d_ev, 0, sizeof(uint32_t) * c->num_events));
-    MK_TRY(cudaMemset(d_merge, 0, sizeof(uint32_t) * n_merge));
     MK_TRY(cudaMemset(d_ctrl, 0, sizeof(uint32_t) * 8));
     MK_TRY(cudaMemset(c->d_err, 0, sizeof(ErrWord)));
-    MK_TRY(cudaMemset(d_x, 0, sizeof(float) * B * s.H));
-    MK_TRY(cudaMemset(d_q, 0, sizeof(float) * B * s.QD));
-    MK_TRY(cudaMemset(d_attn, 0, sizeof(float) * B * s.QD));
-    MK_TRY(cudaMemset(d_act, 0, sizeof(float) * B * s.F));
+    MK_TRY(cudaMemset(d_tag, 0, sizeof(uint64_t) * tl.layer * s.L));   // tag 0: never a step's
     if (d_trace) {
         std::vector<TraceRec> tr(c->num_tasks);
         for (int i = 0; i < c->num_tasks; ++i) {
@@ -318,14 +309,13 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
 #undef MK_TRY
 
     p.tasks = d_tasks; p.queue = d_queue; p.qoff = d_qoff; p.thresholds = d_thr; p.events = d_ev;
-    p.merge_cnt = d_merge;
     p.lm_cnt = d_ctrl + 0; p.epoch = d_ctrl + 1; p.done_cnt = d_ctrl + 2; p.abort_flag = d_ctrl + 3;
     p.num_lm_tasks = c->num_lm_tasks;
     p.layers = d_layers;
     p.embed = (const uint16_t *)w->embed; p.lm_head = (const uint16_t *)w->lm_head;
     p.g_final = (const uint16_t *)w->final_norm;
     p.rope = d_rope;
-    p.x = d_x; p.q = d_q; p.attn = d_attn; p.part = d_part; p.act = d_act;
+    p.tag = d_tag; p.tl = tl;
     p.amax_val = d_aval; p.amax_idx = d_aidx;
     p.err = c->d_err;
     p.trace = d_trace;
@@ -333,6 +323,8 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     p.timeout_ns = cfg->timeout_ns > 0 ? (unsigned long long)cfg->timeout_ns : 2000000000ull;
     p.l2_lookahead = (cfg->flags & MK_FLAG_NO_L2_PREFETCH) ? 0
                    : cfg->l2_lookahead_kb > 0 ? 1024LL * cfg->l2_lookahead_kb : kL2Lookahead;
+    p.event_wait = (cfg->flags & MK_FLAG_EVENT_WAIT) ? 1 : 0;
+    p.debug_withhold = -1;
     *out = c;
     return MK_OK;
 }
@@ -375,15 +367,18 @@ int mk_reset(mk_ctx *c) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MK_ERR_CUDA;
     const Params &p = c->p;
     if (cudaMemset(p.events, 0, sizeof(uint32_t) * c->num_events) != cudaSuccess ||
-        cudaMemset(p.merge_cnt, 0, sizeof(uint32_t) * (size_t)c->s.L * c->s.Bmax * c->s.nkv) != cudaSuccess ||
         cudaMemset(p.lm_cnt, 0, sizeof(uint32_t) * 4) != cudaSuccess ||
         cudaMemset(c->d_err, 0, sizeof(ErrWord)) != cudaSuccess ||
+        // the epoch restarts at 0: tags written before the reset must not
+        // pass for the next steps'
+        cudaMemset(p.tag, 0, sizeof(uint64_t) * p.tl.layer * c->s.L) != cudaSuccess ||
         cudaMemcpy(const_cast<uint32_t *>(p.thresholds), c->h_thresholds.data(), sizeof(uint32_t) * c->num_events,
                    cudaMemcpyHostToDevice) != cudaSuccess)
         return MK_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) return MK_ERR_CUDA;
     c->steps = 0;
     c->failed = false;
+    c->p.debug_withhold = -1;
     return MK_OK;
 }
 
@@ -427,18 +422,25 @@ int mk_get_event_counts(mk_ctx *c, uint32_t *counts_out, uint32_t *thresholds_ou
 int mk_read_buffer(mk_ctx *c, int which, float *host_out, size_t count) {
     if (!c || !host_out) return MK_ERR_INVALID;
     const Shape &s = c->s;
-    const float *src = nullptr;
-    size_t n = 0;
+    const TagLayout &tl = c->p.tl;
+    const size_t last = (size_t)(s.L - 1) * tl.layer;
+    size_t off = 0, n = 0;
     switch (which) {
-    case MK_BUF_HIDDEN: src = c->p.x; n = (size_t)s.Bmax * s.H; break;
-    case MK_BUF_Q: src = c->p.q; n = (size_t)s.Bmax * s.QD; break;
-    case MK_BUF_ATTN: src = c->p.attn; n = (size_t)s.Bmax * s.QD; break;
-    case MK_BUF_ACT: src = c->p.act; n = (size_t)s.Bmax * s.F; break;
+    case MK_BUF_HIDDEN: off = tl.xb; n = (size_t)s.Bmax * s.H; break;
+    case MK_BUF_Q: off = tl.q; n = (size_t)s.Bmax * s.QD; break;
+    case MK_BUF_ATTN: off = tl.attn; n = (size_t)s.Bmax * s.QD; break;
+    case MK_BUF_ACT: off = tl.act; n = (size_t)s.Bmax * s.F; break;
     default: return MK_ERR_INVALID;
     }
     if (count > n) return MK_ERR_INVALID;
-    if (cudaMemcpy(host_out, src, sizeof(float) * count, cudaMemcpyDeviceToHost) != cudaSuccess)
+    std::vector<uint64_t> words(count);
+    if (count && cudaMemcpy(words.data(), c->p.tag + last + off, sizeof(uint64_t) * count,
+                            cudaMemcpyDeviceToHost) != cudaSuccess)
         return MK_ERR_CUDA;
+    for (size_t i = 0; i < count; ++i) {
+        const uint32_t bits = (uint32_t)words[i];
+        std::memcpy(host_out + i, &bits, sizeof bits);
+    }
     return MK_OK;
 }
 
@@ -477,6 +479,12 @@ int mk_debug_set_threshold(mk_ctx *c, int event, uint32_t threshold) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MK_ERR_CUDA;
     if (cudaMemcpy(const_cast<uint32_t *>(c->p.thresholds) + event, &threshold, sizeof threshold, cudaMemcpyHostToDevice) != cudaSuccess)
         return MK_ERR_CUDA;
+    return MK_OK;
+}
+
+int mk_debug_withhold_event(mk_ctx *c, int event) {
+    if (!c || event < -1 || event >= c->num_events) return MK_ERR_INVALID;
+    c->p.debug_withhold = event;
     return MK_OK;
 }
 

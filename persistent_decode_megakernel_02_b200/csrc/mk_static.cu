@@ -80,8 +80,8 @@ uint64_t shape_key(const mk_config *c, int num_sms) {
 }
 
 struct Layout {
-    size_t tasks, queue, qoff, thr, events, merge, ctrl, err, layers, rope;
-    size_t x, q, attn, part, act, aval, aidx, end;
+    size_t tasks, queue, qoff, thr, events, ctrl, err, tag, layers, rope;
+    size_t aval, aidx, end;
 };
 
 size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -121,16 +121,11 @@ Layout layout_for(const Shape &s, const PlanSizes &z, int num_sms, int num_lm_ta
     l.qoff = take(sizeof(int32_t) * (num_sms + 1));
     l.thr = take(sizeof(uint32_t) * z.num_events);
     l.events = take(sizeof(uint32_t) * z.num_events);
-    l.merge = take(sizeof(uint32_t) * (size_t)s.L * B * s.nkv);
     l.ctrl = take(sizeof(uint32_t) * 8);
     l.err = take(sizeof(ErrWord));
+    l.tag = take(sizeof(uint64_t) * tag_layout(s).layer * s.L);
     l.layers = take(sizeof(LayerW) * s.L);
     l.rope = take(sizeof(float2) * (size_t)s.S * (s.d / 2));
-    l.x = take(sizeof(float) * B * s.H);
-    l.q = take(sizeof(float) * B * s.QD);
-    l.attn = take(sizeof(float) * B * s.QD);
-    l.part = take(sizeof(float) * B * s.nq * (size_t)s.NC * (s.d + 2));
-    l.act = take(sizeof(float) * B * s.F);
     l.aval = take(sizeof(float) * B * num_lm_tasks);
     l.aidx = take(sizeof(int32_t) * B * num_lm_tasks);
     l.end = o;
@@ -224,7 +219,7 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
             }
         if (cudaMemcpyAsync(d + lay.tasks, g_host + lay.tasks, lay.events - lay.tasks,
                             cudaMemcpyHostToDevice, st) != cudaSuccess ||
-            cudaMemcpyAsync(d + lay.rope, g_host + lay.rope, lay.x - lay.rope,
+            cudaMemcpyAsync(d + lay.rope, g_host + lay.rope, lay.aval - lay.rope,
                             cudaMemcpyHostToDevice, st) != cudaSuccess ||
             cudaStreamSynchronize(st) != cudaSuccess)
             return MK_ERR_CUDA;
@@ -240,9 +235,11 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
         }
         sig.layer_key = lkey;
     }
-    // what must start at zero: event and merge counters, the epoch / done /
-    // abort words and the error word (everything else is written before it
-    // is read within the step)
+    // what must start at zero: event counters, the epoch / done /
+    // abort words, the error word and the tagged activations (the epoch
+    // restarts at 0 every call, so tags left by the previous call must not
+    // pass for this one's; everything else is written before it is read
+    // within the step)
     if (cudaMemsetAsync(d + lay.events, 0, lay.layers - lay.events, st) != cudaSuccess) return MK_ERR_CUDA;
 
     Params p{};
@@ -252,7 +249,6 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
     p.qoff = reinterpret_cast<const int32_t *>(d + lay.qoff);
     p.thresholds = reinterpret_cast<const uint32_t *>(d + lay.thr);
     p.events = reinterpret_cast<uint32_t *>(d + lay.events);
-    p.merge_cnt = reinterpret_cast<uint32_t *>(d + lay.merge);
     uint32_t *ctrl = reinterpret_cast<uint32_t *>(d + lay.ctrl);
     p.lm_cnt = ctrl + 0;
     p.epoch = ctrl + 1;
@@ -269,11 +265,8 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
     p.batch = batch;
     p.logits = logits_out;
     p.next_tok = next_tok_out;
-    p.x = reinterpret_cast<float *>(d + lay.x);
-    p.q = reinterpret_cast<float *>(d + lay.q);
-    p.attn = reinterpret_cast<float *>(d + lay.attn);
-    p.part = reinterpret_cast<float *>(d + lay.part);
-    p.act = reinterpret_cast<float *>(d + lay.act);
+    p.tag = reinterpret_cast<uint64_t *>(d + lay.tag);
+    p.tl = tag_layout(s);
     p.amax_val = reinterpret_cast<float *>(d + lay.aval);
     p.amax_idx = reinterpret_cast<int32_t *>(d + lay.aidx);
     p.err = reinterpret_cast<ErrWord *>(d + lay.err);
@@ -282,6 +275,8 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
     p.timeout_ns = cfg->timeout_ns > 0 ? (unsigned long long)cfg->timeout_ns : 2000000000ull;
     p.l2_lookahead = (cfg->flags & MK_FLAG_NO_L2_PREFETCH) ? 0
                    : cfg->l2_lookahead_kb > 0 ? 1024LL * cfg->l2_lookahead_kb : kL2Lookahead;
+    p.event_wait = (cfg->flags & MK_FLAG_EVENT_WAIT) ? 1 : 0;
+    p.debug_withhold = -1;
     if (kernel_launch(p, ds.num_sms, st) != cudaSuccess) return MK_ERR_CUDA;
     if (status_out &&
         cudaMemcpyAsync(status_out, d + lay.err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)

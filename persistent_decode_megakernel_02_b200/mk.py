@@ -19,6 +19,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "mk.h")
 MK_OK, MK_ERR_INVALID, MK_ERR_CUDA, MK_ERR_TIMEOUT, MK_ERR_OOM, MK_ERR_STATE = range(6)
 MK_FLAG_TRACE = 1
 MK_FLAG_NO_L2_PREFETCH = 2
+MK_FLAG_EVENT_WAIT = 4
 MK_BUF_HIDDEN, MK_BUF_Q, MK_BUF_ATTN, MK_BUF_ACT = range(4)
 OP_NAMES = ["qkv", "attn", "oproj", "gateup", "down", "lmhead"]
 
@@ -94,12 +95,13 @@ _lib.mk_get_graph.argtypes = [_P, _P, _P, _P]
 _lib.mk_get_sm_stats.argtypes = [_P, _P, C.c_int]
 _lib.mk_plan.argtypes = [C.POINTER(Config), C.c_int, C.POINTER(Info), _P, _P, _P, _P, _P]
 _lib.mk_debug_set_threshold.argtypes = [_P, C.c_int, C.c_uint]
+_lib.mk_debug_withhold_event.argtypes = [_P, C.c_int]
 _lib.mk_decode_step_static.argtypes = [C.POINTER(Config), C.POINTER(PackedWeights), C.POINTER(KV),
                                        _P, _P, C.c_int, _P, _P, _P, _P]
 for _f in ("mk_create", "mk_decode_step", "mk_sync", "mk_reset", "mk_destroy", "mk_get_info",
            "mk_get_event_counts", "mk_read_buffer", "mk_get_trace", "mk_get_graph", "mk_plan",
            "mk_get_sm_stats", "mk_decode_step_static",
-           "mk_debug_set_threshold"):
+           "mk_debug_set_threshold", "mk_debug_withhold_event"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -299,3 +301,6 @@ class Context:
     def debug_set_threshold(self, event: int, value: int):
         _check(_lib.mk_debug_set_threshold(self._h, int(event), int(value)),
                "mk_debug_set_threshold")
+
+    def debug_withhold_event(self, event: int):
+        _check(_lib.mk_debug_withhold_event(self._h, int(event)), "mk_debug_withhold_event")

@@ -162,3 +162,51 @@ def test_default_attention_chunks():
     assert mk.plan(mk.make_config(wl.LLAMA_1B, 16640), SMS)["info"].attn_chunks == 18
     assert mk.plan(mk.make_config(wl.TINY, 64), SMS)["info"].attn_chunks == 4
     assert mk.plan(mk.make_config(wl.TINY, 64, attn_chunks=7), SMS)["info"].attn_chunks == 7
+
+
+@pytest.mark.parametrize("sms,chunks", [(5, 7), (16, 8), (SMS, 0)])
+def test_attention_merger_runs_after_its_chunks(sms, chunks):
+    """Chunk 0's task of every (sequence, KV head) merges the partials and
+    waits for the other chunks' tagged outputs: on every queue it must come
+    after each other chunk of its head, and the whole graph must run to
+    completion when tasks wait on exactly their inputs."""
+    shape = wl.TINY
+    cfg = mk.make_config(shape, 256, 1, attn_chunks=chunks)
+    pl = mk.plan(cfg, sms)
+    tasks, queue, qoff = pl["tasks"], pl["queue"], pl["qoff"]
+    NC = pl["info"].attn_chunks
+    for s in range(sms):
+        q = list(queue[qoff[s]:qoff[s + 1]])
+        for k, i in enumerate(q):
+            t = tasks[i]
+            if t[0] == ATTN and t[4] % NC == 0:
+                later = tasks[q[k + 1:]]
+                assert not np.any((later[:, 0] == ATTN) & (later[:, 1] == t[1]) &
+                                  (later[:, 4] // NC == t[4] // NC))
+    # run the queues with data dependencies: a task needs every task of the
+    # op before it, except that attention chunks need only the QKV op and
+    # chunk 0 additionally needs the other chunks of its head
+    rng = np.random.default_rng(1)
+    done = np.zeros(len(tasks), bool)
+    by_event = {e: np.where(tasks[:, 3] == e)[0] for e in np.unique(tasks[:, 3])}
+    pos = [int(qoff[s]) for s in range(sms)]
+
+    def runnable(i):
+        t = tasks[i]
+        if t[2] >= 0 and not done[by_event[t[2]]].all():
+            return False
+        if t[0] == ATTN and t[4] % NC == 0:
+            mates = by_event[t[3]]
+            mates = mates[(tasks[mates, 4] // NC == t[4] // NC) & (mates != i)]
+            return bool(done[mates].all())
+        return True
+
+    while any(pos[s] < qoff[s + 1] for s in range(sms)):
+        progressed = False
+        for s in rng.permutation(sms):
+            if pos[s] < qoff[s + 1] and runnable(queue[pos[s]]):
+                done[queue[pos[s]]] = True
+                pos[s] += 1
+                progressed = True
+        assert progressed, "tasks wait on each other in a cycle"
+    assert done.all()

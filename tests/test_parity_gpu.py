@@ -32,9 +32,15 @@ def _check_events(pair, steps):
     assert np.array_equal(counts.astype(np.uint64), (thr.astype(np.uint64) * steps) % (1 << 32))
 
 
-def test_tiny_teacher_forced_prompt_and_decode():
+# 0: tasks wait on their tagged inputs; 4 (MK_FLAG_EVENT_WAIT): a scheduler
+# warp gates every task on its dependency's event counter first
+WAIT_MODES = [0, 4]
+
+
+@pytest.mark.parametrize("flags", WAIT_MODES)
+def test_tiny_teacher_forced_prompt_and_decode(flags):
     shape = wl.TINY
-    pair = Pair(shape, max_seq=64)
+    pair = Pair(shape, max_seq=64, flags=flags)
     prompt = wl.make_prompt(shape.vocab, 16, seed=42)
     n = 0
     for step, pos, g_tok, g_log, ref in pair.teacher_forced(prompt, 32):
@@ -50,9 +56,10 @@ def test_tiny_teacher_forced_prompt_and_decode():
         assert np.abs(kg - kr).max() <= 2e-2 * np.abs(kr).max()
 
 
-def test_tiny_random_gains_untied_head_and_intermediates():
+@pytest.mark.parametrize("flags", WAIT_MODES)
+def test_tiny_random_gains_untied_head_and_intermediates(flags):
     shape = wl.ModelShape("tiny-untied", 2, 256, 4, 2, 64, 768, 4096, False, 1e4)
-    pair = Pair(shape, max_seq=40, gains="random", std=0.05)
+    pair = Pair(shape, max_seq=40, gains="random", std=0.05, flags=flags)
     toks = wl.make_prompt(shape.vocab, 20, seed=9)
     for pos, t in enumerate(toks):
         g_tok, g_log = pair.gpu_step(int(t), pos)
@@ -113,7 +120,8 @@ def test_invalid_inputs_reported_then_reset():
 
 def test_event_that_never_fires_times_out_and_context_recovers():
     shape = wl.TINY
-    pair = Pair(shape, max_seq=16, timeout_ns=50_000_000)   # 50 ms bound per wait
+    # counter-gated scheduling: the scheduler's wait on event 3 never ends
+    pair = Pair(shape, max_seq=16, timeout_ns=50_000_000, flags=4)   # 50 ms bound per wait
     mk = pair.mk
     g_tok, _ = pair.gpu_step(1, 0)
     _, thr = pair.ctx.event_counts()
@@ -132,20 +140,47 @@ def test_event_that_never_fires_times_out_and_context_recovers():
     _check_step(pair, 1, g_tok, g_log, ref)
 
 
-def test_trace_records_respect_dependencies():
+def test_withheld_outputs_time_out_and_context_recovers():
     shape = wl.TINY
-    pair = Pair(shape, max_seq=32, flags=1)
+    # tagged-input waits: the gate/up tasks of layer 0 (event 3) store stale
+    # tags, the down projection's poll of its input never succeeds
+    pair = Pair(shape, max_seq=16, timeout_ns=50_000_000)
+    mk = pair.mk
+    pair.gpu_step(1, 0)
+    pair.ctx.debug_withhold_event(3)
+    pair.tok.fill_(2)
+    pair.pos.fill_(1)
+    pair.ctx.decode_step(pair.tok, pair.pos, pair.nxt, pair.logits)
+    assert pair.ctx.sync() == mk.MK_ERR_TIMEOUT
+    assert pair.ctx.info().err_code == mk.MK_ERR_TIMEOUT
+    pair.ctx.reset()
+    pair.ref_step(1, 0)
+    g_tok, g_log = pair.gpu_step(2, 1)
+    ref = pair.ref_step(2, 1)
+    _check_step(pair, 1, g_tok, g_log, ref)
+    g_tok, g_log = pair.gpu_step(3, 2)
+    ref = pair.ref_step(3, 2)
+    _check_step(pair, 2, g_tok, g_log, ref)
+
+
+@pytest.mark.parametrize("flags", WAIT_MODES)
+def test_trace_records_respect_dependencies(flags):
+    shape = wl.TINY
+    pair = Pair(shape, max_seq=32, flags=1 | flags)
     for pos, t in enumerate([5, 6, 7]):
         pair.gpu_step(t, pos)
     tr = pair.ctx.trace()
     g = pair.ctx.graph()
     tasks = g["tasks"]
-    assert np.all(tr["t_start"] >= tr["t_ready"]) and np.all(tr["t_end"] >= tr["t_start"])
+    assert np.all(tr["t_start"] >= tr["t_ready"]) and np.all(tr["t_input"] >= tr["t_start"])
+    assert np.all(tr["t_done"] >= tr["t_input"]) and np.all(tr["t_end"] >= tr["t_done"])
     fire = {}
     for e in np.unique(tasks[:, 3]):
         fire[e] = tr["t_end"][tasks[:, 3] == e].max()
     for i, t in enumerate(tasks):
-        if t[2] >= 0:
+        # an attention task waiting on its inputs needs only its own KV
+        # head's q/k/v, not the whole QKV op (the event's other tasks)
+        if t[2] >= 0 and (flags or t[0] != 1):
             # a task becomes ready only after every task of its dependency
             # signalled (t_end is stamped just after the signal; allow 5 us)
             assert int(tr["t_ready"][i]) + 5000 >= int(fire[t[2]])
