@@ -88,6 +88,8 @@ enum mk_flags {
  *  timeout_ns: bound on every device-side wait; 0 means 2 s.
  *  l2_lookahead_kb: how far (KiB of weights per SM) a prefetch warp runs
  *  ahead of the shared-memory ring into L2; 0 means no L2 prefetch.
+ *  poll_ns: pause (ns) between two polls of a task's not yet ready input
+ *  words; 0 polls back to back.
  */
 typedef struct mk_config {
     int layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
@@ -97,6 +99,7 @@ typedef struct mk_config {
     int attn_chunks;
     long long timeout_ns;
     int l2_lookahead_kb;
+    int poll_ns;
 } mk_config;
 
 /*
@@ -233,12 +236,13 @@ int mk_get_trace(mk_ctx *ctx, mk_trace_rec *host_out, int n);
  * [num_sms][16] = {loader ns waiting for a free page, pages issued, loader
  * ns total, worker ns waiting for loaded pages, worker ns waiting for the
  * scheduler, worker ns in worker barriers, worker ns total, scheduler ns
- * waiting on event counters, worker ns in task prologues (input vector
- * load, RMSNorm), worker ns in dot products, worker ns in per-tile
- * reductions and epilogues, worker ns in task ends (barrier, fence, event,
- * merges), tasks run, worker ns in attention combine/merge tails,
- * 2 unused}.  Worker figures are those of warp 0 and
- * some phases overlap the waits they contain. */
+ * waiting on event counters, worker ns in task prologues (waiting for and
+ * loading the input vector, RMSNorm), worker ns in row-per-warp dot
+ * products, worker ns in per-tile reductions and epilogues, worker ns in
+ * task ends (barrier, completion post, argmax), tasks run, worker ns in
+ * attention combine/merge tails, worker ns in the first page of each
+ * column-split task, worker ns in its later pages}.  Worker figures are
+ * those of thread 0 and some phases overlap the waits they contain. */
 int mk_get_sm_stats(mk_ctx *ctx, uint64_t *host_out, int n);
 
 /* Static task graph as built by mk_create (host copy).  task_out: int32

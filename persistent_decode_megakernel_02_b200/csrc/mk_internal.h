@@ -44,7 +44,7 @@ constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 14336
 constexpr int kMaxGroup = 8;        // q heads per KV head handled by one attention task
 constexpr int kMaxHeadDim = 256;
 constexpr long long kL2Lookahead = 0;  // default L2 prefetch distance beyond the ring (0: off; measured no gain)
-constexpr int kStageFloats = 6144;  // shared staging: a GEMV input vector, or attention partials
+constexpr int kStageFloats = 8192;  // shared staging: a GEMV input vector, or attention partials
 constexpr int kL2Chunk = 64 * 1024;             // bytes per L2 prefetch instruction
 
 // ---- ops ---------------------------------------------------------------------
@@ -135,8 +135,10 @@ MK_HD inline int tile_rows(const Shape &s, int kind, int tile) {
 }
 
 // GEMVs with K <= kRowK run one row per warp with the whole input vector in
-// registers; larger K splits columns across warps.
+// registers; K = 2 or 4 x kRowK run one 2048-column segment of a row per
+// warp; other K split columns across all worker threads.
 constexpr int kRowK = 2048;
+MK_HD inline bool rows_gemv(int K) { return K <= kRowK || K == 2 * kRowK || K == 4 * kRowK; }
 constexpr int kMaxHidden = 4096;   // pair tiles in the column split hold 2 vectors per thread
 
 // Rows of one page: the largest power of two <= 16 whose rows (K bf16 each)
@@ -160,32 +162,43 @@ MK_HD inline int attn_pos_per_page(int d) { return kPageBytes / (4 * d); }
 // copy sits between a producer's store and the consumer's read.  Each layer
 // owns its own buffers (nothing is overwritten within a step), so a word's tag
 // is either this step's or an older one.
-//   xa: residual after the O-projection   [Bmax][H]
-//   xb: residual after the down projection [Bmax][H] (layer L-1: final hidden)
+// The vectors every SM reads whole (the two residual streams, the attention
+// output and SiLU(gate) * up) are written kReplicas times, and SM i reads
+// copy i % kReplicas: when 148 SMs read the same few hundred L2 lines at
+// once the lines' L2 slices serialise the requests; copies at different
+// addresses spread them over more slices.  Producers write a few hundred
+// words per task, so the extra stores cost little.
+//   xa: residual after the O-projection   [R][Bmax][H]
+//   xb: residual after the down projection [R][Bmax][H] (layer L-1: final hidden)
 //   q:  rotated queries                    [Bmax][nq * d]
 //   kn, vn: the new position's key (rotated) and value, rounded to bf16
 //                                          [Bmax][nkv * d]
 //   part: split-K attention partials, per q head and chunk o[d], m, l
 //                                          [Bmax][nq][NC][d + 2]
-//   attn: merged attention output          [Bmax][nq * d]
-//   act:  SiLU(gate) * up                  [Bmax][F]
+//   attn: merged attention output          [R][Bmax][nq * d]
+//   act:  SiLU(gate) * up                  [R][Bmax][F]
+constexpr int kReplicas = 8;
 struct TagLayout {
     size_t xa, xb, q, kn, vn, part, attn, act;   // word offsets within a layer's block
+    size_t rep_h, rep_qd, rep_f;                 // distance between copies (words)
     size_t layer;                                // words per layer
 };
 
 MK_HD inline TagLayout tag_layout(const Shape &s) {
     TagLayout t;
     const size_t B = (size_t)s.Bmax;
+    t.rep_h = B * s.H;
+    t.rep_qd = B * s.QD;
+    t.rep_f = B * s.F;
     size_t o = 0;
-    t.xa = o; o += B * s.H;
-    t.xb = o; o += B * s.H;
+    t.xa = o; o += kReplicas * t.rep_h;
+    t.xb = o; o += kReplicas * t.rep_h;
     t.q = o; o += B * s.QD;
     t.kn = o; o += B * s.KD;
     t.vn = o; o += B * s.KD;
     t.part = o; o += B * s.nq * (size_t)s.NC * (s.d + 2);
-    t.attn = o; o += B * s.QD;
-    t.act = o; o += B * s.F;
+    t.attn = o; o += kReplicas * t.rep_qd;
+    t.act = o; o += kReplicas * t.rep_f;
     t.layer = (o + 1) & ~(size_t)1;   // keep every block 16-byte aligned
     return t;
 }
@@ -259,6 +272,7 @@ struct Params {
     long long l2_lookahead;      // bytes the L2 prefetch runs ahead of the ring (0: off)
     int event_wait;              // 1: the scheduler gates tasks on event counters
     int debug_withhold;          // test hook: tasks triggering this event write stale tags (-1: off)
+    unsigned int poll_ns;        // pause between polls of stale input words
 };
 
 // ---- host planning -------------------------------------------------------------

@@ -149,25 +149,33 @@ __device__ __forceinline__ uint4 ld_shared_v4(const void *p) {
     return v;
 }
 // Tagged activation words: value bits low, step tag high, one 64-bit access
-// (single-copy atomic), so a reader that sees the tag sees the value.
+// (single-copy atomic), so a reader that sees the tag sees the value.  The
+// loads are volatile (re-issued on every poll, kept in order among
+// themselves) but carry no memory clobber, so the compiler may issue a
+// batch of them before the shared-memory stores that consume the results.
 __device__ __forceinline__ void st_tag(uint64_t *p, float v, uint32_t ep) {
     const uint64_t w = ((uint64_t)ep << 32) | __float_as_uint(v);
     asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
+// The same value into every copy of a replicated tagged vector.
+__device__ __forceinline__ void st_tag_rep(uint64_t *p, size_t stride, float v, uint32_t ep) {
+#pragma unroll 1
+    for (int r = 0; r < kReplicas; ++r) st_tag(p + r * stride, v, ep);
+}
 __device__ __forceinline__ ulonglong2 ld_tag2(const uint64_t *p) {
     ulonglong2 v;
-    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p));
     return v;
 }
 __device__ __forceinline__ uint64_t ld_tag1(const uint64_t *p) {
     uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p));
     return v;
 }
 // The tag half of a tagged word alone (polling without keeping values).
 __device__ __forceinline__ uint32_t ld_tag_hi(const uint64_t *p) {
     uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(reinterpret_cast<const char *>(p) + 4) : "memory");
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(reinterpret_cast<const char *>(p) + 4));
     return v;
 }
 __device__ __forceinline__ bool tag_ok(uint64_t w, uint32_t ep) { return (uint32_t)(w >> 32) == ep; }
@@ -303,6 +311,7 @@ __device__ __forceinline__ bool warp_spin_ok(Spin &s, const Params &p, SmemCtl *
                                              uint32_t info) {
     int ok = 1;
     if ((threadIdx.x & 31) == 0) ok = spin_ok(s, p, ctl, W_TAG, task, info) ? 1 : 0;
+    if (p.poll_ns) __nanosleep(p.poll_ns);
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -322,6 +331,8 @@ __device__ __forceinline__ float wait_tag1(const Params &p, SmemCtl *ctl, const 
 __device__ __forceinline__ uint64_t *tag_buf(const Params &p, int layer, size_t off) {
     return p.tag + (size_t)layer * p.tl.layer + off;
 }
+// The copy of the replicated vectors this SM reads.
+__device__ __forceinline__ size_t my_copy(size_t stride) { return (size_t)(blockIdx.x % kReplicas) * stride; }
 
 // ---------------------------------------------------------------------------
 // task geometry shared by the loader and the workers
@@ -576,7 +587,7 @@ struct WState {
 };
 // Trace-mode time accounting of worker thread 0, accumulated in shared memory
 // so it costs no registers across the task bodies.
-enum WStat { WS_FULL = 0, WS_READY, WS_SYNC, WS_PRO, WS_DOT, WS_EPI, WS_END, WS_TASKS, WS_ATT, WS_FIRST, WS_TASKWAIT, kWStats };
+enum WStat { WS_FULL = 0, WS_READY, WS_SYNC, WS_PRO, WS_DOT, WS_EPI, WS_END, WS_TASKS, WS_ATT, WS_FIRST, WS_TASKWAIT, WS_COLS, kWStats };
 __device__ __forceinline__ unsigned long long phase_begin(const WState &w) {
     return w.stat ? globaltimer() : 0ull;
 }
@@ -712,42 +723,41 @@ __device__ __forceinline__ bool signal_event(const Params &p, SmemCtl *ctl, cons
 template <int NP>
 __device__ __forceinline__ bool stage_tagged(const Params &p, SmemCtl *ctl, const WState &w,
                                              const uint64_t *src, int n, float &ss) {
+    constexpr int NB = NP < 8 ? NP : 8;   // loads in flight per thread
     const int tid = threadIdx.x;
-    const int npairs = n >> 1;
-    float2 v[NP];
+    const int npairs = n >> 1, n8 = n >> 3;
+    float2 *st = reinterpret_cast<float2 *>(ctl->stage);
+    float acc = 0.f;
     uint32_t pend = 0;
+    // pairs j = jb .. jb + NB - 1 of the thread: issue all loads, then store
+    // the fresh ones (one round trip per batch); stale ones are polled after
+    auto batch = [&](int jb, bool only_pending) {
+        ulonglong2 q[NB];
 #pragma unroll
-    for (int j = 0; j < NP; ++j) {
-        const int i = tid + j * kWorkerThreads;
-        v[j] = make_float2(0.f, 0.f);
-        if (i < npairs) {
-            const ulonglong2 t = ld_tag2(src + 2 * i);
-            v[j] = make_float2(tag_val(t.x), tag_val(t.y));
-            if (!tag_ok(t.x, w.ep) || !tag_ok(t.y, w.ep)) pend |= 1u << j;
+        for (int k = 0; k < NB; ++k) {
+            const int j = jb + k, i = tid + j * kWorkerThreads;
+            const bool want = i < npairs && (!only_pending || (pend & (1u << j)));
+            q[k] = want ? ld_tag2(src + 2 * i) : make_ulonglong2(0ull, 0ull);
+            if (want) pend |= 1u << j;
         }
-    }
-    Spin s;
-    while (__any_sync(0xffffffffu, pend != 0u)) {
-        if (!warp_spin_ok(s, p, ctl, (uint32_t)w.task_id, 0u)) return false;
 #pragma unroll
-        for (int j = 0; j < NP; ++j) {
-            if (pend & (1u << j)) {
-                const ulonglong2 t = ld_tag2(src + 2 * (tid + j * kWorkerThreads));
-                v[j] = make_float2(tag_val(t.x), tag_val(t.y));
-                if (tag_ok(t.x, w.ep) && tag_ok(t.y, w.ep)) pend &= ~(1u << j);
+        for (int k = 0; k < NB; ++k) {
+            const int j = jb + k, i = tid + j * kWorkerThreads;
+            if ((pend & (1u << j)) && tag_ok(q[k].x, w.ep) && tag_ok(q[k].y, w.ep)) {
+                const float2 v = make_float2(tag_val(q[k].x), tag_val(q[k].y));
+                st[2 * (((i >> 1) & 1) * n8 + (i >> 2)) + (i & 1)] = v;
+                acc = fmaf(v.x, v.x, fmaf(v.y, v.y, acc));
+                pend &= ~(1u << j);
             }
         }
-    }
-    float acc = 0.f;
-    float2 *st = reinterpret_cast<float2 *>(ctl->stage);
-    const int n8 = n >> 3;
+    };
 #pragma unroll
-    for (int j = 0; j < NP; ++j) {
-        const int i = tid + j * kWorkerThreads;
-        if (i < npairs) {
-            st[2 * (((i >> 1) & 1) * n8 + (i >> 2)) + (i & 1)] = v[j];
-            acc = fmaf(v[j].x, v[j].x, fmaf(v[j].y, v[j].y, acc));
-        }
+    for (int jb = 0; jb < NP; jb += NB) batch(jb, false);
+    Spin sp;
+    while (__any_sync(0xffffffffu, pend != 0u)) {
+        if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 0u)) return false;
+#pragma unroll
+        for (int jb = 0; jb < NP; jb += NB) batch(jb, true);
     }
     ss = acc;
     return true;
@@ -765,26 +775,32 @@ __device__ __forceinline__ bool stage_partials(const Params &p, SmemCtl *ctl, co
     const int hp = per >> 1, npairs = nh * hp;
     float2 *st = reinterpret_cast<float2 *>(ctl->stage);
     uint32_t pend = 0;
-    auto load = [&](int j) {
+    // all loads of a pass are issued before any result is looked at
+    auto addr = [&](int j) {
         const int i = tid + j * kWorkerThreads;
         const int g = i / hp;
-        const ulonglong2 q = ld_tag2(src + (size_t)g * stride + 2 * (i - g * hp));
-        if (tag_ok(q.x, w.ep) && tag_ok(q.y, w.ep)) {
-            st[i] = make_float2(tag_val(q.x), tag_val(q.y));
-            pend &= ~(1u << j);
-        } else {
-            pend |= 1u << j;
-        }
+        return src + (size_t)g * stride + 2 * (i - g * hp);
     };
+    ulonglong2 q[NP];
 #pragma unroll
-    for (int j = 0; j < NP; ++j)
-        if (tid + j * kWorkerThreads < npairs) load(j);
+    for (int j = 0; j < NP; ++j) {
+        const bool in = tid + j * kWorkerThreads < npairs;
+        q[j] = in ? ld_tag2(addr(j)) : make_ulonglong2(0ull, 0ull);
+        if (in) pend |= 1u << j;
+    }
     Spin sp;
-    while (__any_sync(0xffffffffu, pend != 0u)) {
+    while (true) {
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+            if ((pend & (1u << j)) && tag_ok(q[j].x, w.ep) && tag_ok(q[j].y, w.ep)) {
+                st[tid + j * kWorkerThreads] = make_float2(tag_val(q[j].x), tag_val(q[j].y));
+                pend &= ~(1u << j);
+            }
+        if (!__any_sync(0xffffffffu, pend != 0u)) break;
         if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 5u)) return false;
 #pragma unroll
         for (int j = 0; j < NP; ++j)
-            if (pend & (1u << j)) load(j);
+            if (pend & (1u << j)) q[j] = ld_tag2(addr(j));
     }
     return true;
 }
@@ -824,13 +840,13 @@ __device__ __forceinline__ GemvInput gemv_input(const Params &p, int kind, int l
     switch (kind) {
     case OP_QKV:
         if (layer == 0) in.src_bf = p.embed + (size_t)p.tokens[b] * s.H;
-        else in.src = tag_buf(p, layer - 1, tl.xb) + (size_t)b * s.H;
+        else in.src = tag_buf(p, layer - 1, tl.xb) + my_copy(tl.rep_h) + (size_t)b * s.H;
         in.gain = p.layers[layer].g_attn;
         break;
-    case OP_GATEUP: in.src = tag_buf(p, layer, tl.xa) + (size_t)b * s.H; in.gain = p.layers[layer].g_mlp; break;
-    case OP_LMHEAD: in.src = tag_buf(p, s.L - 1, tl.xb) + (size_t)b * s.H; in.gain = p.g_final; break;
-    case OP_OPROJ: in.src = tag_buf(p, layer, tl.attn) + (size_t)b * s.QD; break;
-    default: in.src = tag_buf(p, layer, tl.act) + (size_t)b * s.F; break;
+    case OP_GATEUP: in.src = tag_buf(p, layer, tl.xa) + my_copy(tl.rep_h) + (size_t)b * s.H; in.gain = p.layers[layer].g_mlp; break;
+    case OP_LMHEAD: in.src = tag_buf(p, s.L - 1, tl.xb) + my_copy(tl.rep_h) + (size_t)b * s.H; in.gain = p.g_final; break;
+    case OP_OPROJ: in.src = tag_buf(p, layer, tl.attn) + my_copy(tl.rep_qd) + (size_t)b * s.QD; break;
+    default: in.src = tag_buf(p, layer, tl.act) + my_copy(tl.rep_f) + (size_t)b * s.F; break;
     }
     return in;
 }
@@ -839,8 +855,8 @@ __device__ __forceinline__ GemvInput gemv_input(const Params &p, int kind, int l
 // down output) and the down projection (this layer's O output), and the
 // buffer each writes.
 __device__ __forceinline__ const uint64_t *resid_in(const Params &p, int kind, int layer, int b) {
-    return kind == OP_DOWN ? tag_buf(p, layer, p.tl.xa) + (size_t)b * p.s.H
-                           : tag_buf(p, layer - 1, p.tl.xb) + (size_t)b * p.s.H;
+    return (kind == OP_DOWN ? tag_buf(p, layer, p.tl.xa) : tag_buf(p, layer - 1, p.tl.xb)) +
+           my_copy(p.tl.rep_h) + (size_t)b * p.s.H;
 }
 __device__ __forceinline__ uint64_t *resid_out(const Params &p, int kind, int layer, int b) {
     return tag_buf(p, layer, kind == OP_DOWN ? p.tl.xb : p.tl.xa) + (size_t)b * p.s.H;
@@ -906,7 +922,7 @@ __device__ __forceinline__ void gemv_epilogue_row(const Params &p, int kind, int
         break;
     }
     case OP_GATEUP:
-        st_tag(tag_buf(p, layer, p.tl.act) + (size_t)b * s.F + tile * 8 + r, a / (1.0f + expf(-a)) * c, ep);
+        st_tag_rep(tag_buf(p, layer, p.tl.act) + (size_t)b * s.F + tile * 8 + r, p.tl.rep_f, a / (1.0f + expf(-a)) * c, ep);
         break;
     default: {  // OP_LMHEAD
         const int row = tile * 8 + r;
@@ -962,32 +978,85 @@ __device__ __forceinline__ void dot_rows2(const uint4 *ra, const uint4 *rc, cons
     acc_c = c.x + c.y;
 }
 
-// One warp per row.  Each lane keeps NVL 8-element vectors of the input
-// (vectors lane, lane+32, ...), so a warp holds the whole input vector and
-// computes its RMSNorm itself: tiles need no cross-warp reduction.  Work
-// goes in units of two pages (16 rows): a pair tile (the 8 first-half q/k
-// rows and their RoPE partners, or 8 gate rows and the matching up rows),
-// or two consecutive 8-row tiles.  Warp w takes row w of both pages.
-// Everything that does not depend on the activation (gains, RoPE cos/sin,
-// the first layer's embedding row) is loaded before the task's dependency
-// is waited on; after it, one round trip loads the input vector and the
-// residual values.
+// Epilogue of one unit (16 rows: a pair tile or two 8-row tiles; or one
+// 8-row tile) whose row sums warp 0 holds: lane e (< rows) has row e's dot
+// product `a`, and for pair tiles `c` is row e + 8's.  `resid` is lane L's
+// residual of task row L (O / down projections).  Warp 0 calls it whole.
+__device__ __forceinline__ void unit_epilogue(const Params &p, SmemCtl *ctl, const WState &w, const Task &t,
+                                              int tile, bool pair, int rows, float a, float c, float resid,
+                                              int tok, int P, float &best_v, int &best_i) {
+    const Shape &s = p.s;
+    const int kind = t.kind, layer = t.layer, b = 0;
+    const int lane = threadIdx.x & 31, e = lane & 15;
+    const int grp_row = 8 * (tile - t.begin) + e;   // row within the task
+    const float rres = __shfl_sync(0xffffffffu, resid, grp_row & 31);
+    if (pair) {
+        if (lane < 8) gemv_epilogue_row(p, kind, layer, tile, lane, a, c, b, P, w.ep_out, best_v, best_i);
+    } else if (lane < rows) {
+        const int tl = tile + (e >> 3), r = e & 7;
+        if (kind == OP_OPROJ || kind == OP_DOWN) {
+            const int row = tl * 8 + r;
+            const float base = grp_row < 32 ? rres
+                             : (kind == OP_OPROJ && layer == 0)
+                                   ? bf2f(p.embed[(size_t)tok * s.H + row])
+                                   : wait_tag1(p, ctl, resid_in(p, kind, layer, b) + row, w.ep, (uint32_t)w.task_id);
+            st_tag_rep(resid_out(p, kind, layer, b) + row, p.tl.rep_h, base + a, w.ep_out);
+        } else {
+            gemv_epilogue_row(p, kind, layer, tl, r, a, 0.f, b, P, w.ep_out, best_v, best_i);
+        }
+    }
+}
+
+// Convert a bf16 vector of n values (n a multiple of 8) into ctl->stage in
+// the layout stage_tagged writes; ss returns the thread's sum of squares.
+__device__ __forceinline__ void stage_embed(SmemCtl *ctl, const uint16_t *src, int n, float &ss) {
+    float2 *st = reinterpret_cast<float2 *>(ctl->stage);
+    const int n8 = n >> 3;
+    float acc = 0.f;
+    for (int i = threadIdx.x; i < (n >> 1); i += kWorkerThreads) {
+        const uint32_t wd = __ldg(reinterpret_cast<const uint32_t *>(src) + i);
+        const float2 v = make_float2(bf_lo(wd), bf_hi(wd));
+        st[2 * (((i >> 1) & 1) * n8 + (i >> 2)) + (i & 1)] = v;
+        acc = fmaf(v.x, v.x, fmaf(v.y, v.y, acc));
+    }
+    ss = acc;
+}
+
+// One warp per row of 2048 (or fewer) columns.  Each lane keeps NVL
+// 8-element vectors of its input (vectors lane, lane+32, ...).  A 64 KB page
+// holds 16 such rows and warp w takes rows w and 8 + w of every page.
+//  * K <= 2048: a page is a unit of 16 matrix rows (a pair tile -- the 8
+//    first-half q/k rows and their RoPE partners, or 8 gate rows and the
+//    matching up rows -- or two consecutive 8-row tiles); every warp holds
+//    the whole input and finishes its rows itself (no cross-warp reduction).
+//  * K = 2048 * nseg (nseg = 2 or 4): each matrix row is nseg 2048-column
+//    segments, so a page holds 16 / nseg matrix rows and its row w is
+//    segment w % nseg of a row; warp w keeps only that segment of the input.
+//    The segment sums of a unit go to shared memory and warp 0 adds them up
+//    once the unit's nseg pages are done.
+// The input vector is staged once per task in shared memory by all worker
+// threads (tagged loads, waiting for this step's tags); everything that does
+// not depend on it (gains, RoPE cos/sin) is loaded before.
 template <int NVL>
 __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                           WState &w) {
     const Shape &s = p.s;
     const int kind = t.kind, layer = t.layer;
     const int K = op_k(s, kind);
-    const int K8 = K >> 3;
+    const int nseg = K > kRowK ? K / kRowK : 1;
+    const int K8 = nseg > 1 ? kRowK / 8 : K >> 3;     // vectors per page row
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int seg = warp % nseg;
     const int b = 0;
-    const size_t row_bytes = (size_t)K * 2;
+    const size_t row_bytes = (size_t)K8 * 16;          // one page row
     const int P = p.positions[b];
     const int tok = p.tokens[b];
     // pair tiles: every GATEUP tile, and QKV tiles below npair
     const int npair = kind == OP_GATEUP ? 0x7fffffff
                     : kind == OP_QKV ? (s.nq + s.nkv) * s.d / 16 : 0;
     const int per_head = s.d / 16;
+    const bool resid_op = kind == OP_OPROJ || kind == OP_DOWN;
+    const int task_rows = 8 * (t.end - t.begin);
 
     // ---- before the dependency
     const uint16_t *gain = kind == OP_QKV ? p.layers[layer].g_attn
@@ -996,33 +1065,38 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     float xr[NVL][8];
     uint4 gv[NVL];   // the RMSNorm gain slice, loaded before the dependency
     const bool embed_in = kind == OP_QKV && layer == 0;
+    const bool embed_regs = embed_in && nseg == 1;      // warps read the embedding row themselves
 #pragma unroll
     for (int j = 0; j < NVL; ++j) {
         const int v = lane + 32 * j;
-        gv[j] = (gain && v < K8) ? __ldg(reinterpret_cast<const uint4 *>(gain) + v) : make_uint4(0, 0, 0, 0);
-        if (embed_in && v < K8) {
+        const int vg = seg * K8 + v;                    // vector index in the whole input
+        gv[j] = (gain && v < K8) ? __ldg(reinterpret_cast<const uint4 *>(gain) + vg) : make_uint4(0, 0, 0, 0);
+        if (embed_regs && v < K8) {
             const uint4 e = __ldg(reinterpret_cast<const uint4 *>(p.embed + (size_t)tok * s.H) + v);
             xr[j][0] = bf_lo(e.x); xr[j][1] = bf_hi(e.x); xr[j][2] = bf_lo(e.y); xr[j][3] = bf_hi(e.y);
             xr[j][4] = bf_lo(e.z); xr[j][5] = bf_hi(e.z); xr[j][6] = bf_lo(e.w); xr[j][7] = bf_hi(e.w);
         }
     }
-    // per-tile values, lane L holding those of tile begin + L (row `warp`)
+    // per-tile values.  Whole rows per warp: lane L holds those of tile
+    // begin + L, row `warp`.  Segments: warp 0's lane L holds the residual of
+    // task row L.
     float pre0 = 0.f, pre1 = 0.f;
     const int my_tile = t.begin + lane;
-    if (kind == OP_QKV && my_tile < t.end && my_tile < npair) {
+    if (nseg == 1 && kind == OP_QKV && my_tile < t.end && my_tile < npair) {
         const int i = (my_tile % per_head) * 8 + warp;
         const float2 cs = p.rope[(size_t)P * (s.d / 2) + i];
         pre0 = cs.x;
         pre1 = cs.y;
     }
-    if (kind == OP_OPROJ && layer == 0 && my_tile < t.end)
-        pre0 = bf2f(p.embed[(size_t)tok * s.H + my_tile * 8 + warp]);
+    if (kind == OP_OPROJ && layer == 0) {
+        if (nseg == 1 && my_tile < t.end) pre0 = bf2f(p.embed[(size_t)tok * s.H + my_tile * 8 + warp]);
+        if (nseg > 1 && warp == 0 && lane < task_rows) pre0 = bf2f(p.embed[(size_t)tok * s.H + 8 * t.begin + lane]);
+    }
 
     // ---- the dependency (tagged inputs), then the activation
     if (!wait_ready(p, ctl, w)) return false;
     unsigned long long tp = phase_begin(w);
-    const bool resid_op = (kind == OP_OPROJ && layer > 0) || kind == OP_DOWN;
-    if (embed_in) {
+    if (embed_regs) {
         // the embedding row needs no dependency: each warp holds it already
         stamp_ready(p, w);
         if (gain) {
@@ -1044,26 +1118,33 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
             }
         }
     } else {
-        // the activation: the worker threads copy the tagged vector into
-        // ctl->stage together (waiting for this step's tags), meet, and then
-        // every warp takes the whole vector from there
+        // the activation: the worker threads copy the input vector into
+        // ctl->stage together (tagged: waiting for this step's tags), meet,
+        // and then every warp takes its part from there
         const GemvInput in = gemv_input(p, kind, layer, b);
         float ss = 0.f;
-        if (!stage_tagged<kRowK / 512>(p, ctl, w, in.src, K, ss)) return false;
-        if (resid_op && !warp_tag1(p, ctl, w, resid_in(p, kind, layer, b) + my_tile * 8 + warp,
-                                   my_tile < t.end, pre0))
-            return false;
+        if (in.src_bf) stage_embed(ctl, in.src_bf, K, ss);
+        else if (!(K <= kRowK ? stage_tagged<kRowK / 512>(p, ctl, w, in.src, K, ss) : stage_tagged<kStageFloats / 512>(p, ctl, w, in.src, K, ss))) return false;
+        if (resid_op && !(kind == OP_OPROJ && layer == 0)) {
+            const uint64_t *rs = resid_in(p, kind, layer, b);
+            if (nseg == 1) {
+                if (!warp_tag1(p, ctl, w, rs + my_tile * 8 + warp, my_tile < t.end, pre0)) return false;
+            } else if (warp == 0) {
+                if (!warp_tag1(p, ctl, w, rs + 8 * t.begin + lane, lane < task_rows, pre0)) return false;
+            }
+        }
         ss = warp_sum(ss);
         if (lane == 0) ctl->scal[warp] = ss;
         if (!worker_sync(p, ctl, w)) return false;
         stamp_ready(p, w);
         const float4 *src = reinterpret_cast<const float4 *>(ctl->stage);
+        const int n8 = K >> 3;
 #pragma unroll
         for (int j = 0; j < NVL; ++j) {
             const int v = lane + 32 * j;
             if (v < K8) {
-                const float4 a0 = src[v];
-                const float4 a1 = src[K8 + v];
+                const float4 a0 = src[seg * K8 + v];
+                const float4 a1 = src[n8 + seg * K8 + v];
                 xr[j][0] = a0.x; xr[j][1] = a0.y; xr[j][2] = a0.z; xr[j][3] = a0.w;
                 xr[j][4] = a1.x; xr[j][5] = a1.y; xr[j][6] = a1.z; xr[j][7] = a1.w;
             } else {
@@ -1092,17 +1173,18 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
     int tile = t.begin;
+    int pu = 0;   // page of the current unit (segments)
     while (tile < t.end) {
         const bool pair = tile < npair;
         const bool two = pair || tile + 1 < t.end;
         float acc_a = 0.f, acc_c = 0.f;
-        // the unit's 16 (or 8) rows are one page: rows warp and 8 + warp
+        // rows warp and 8 + warp of the page
         uint32_t slot;
         if (!wait_page(p, ctl, w, slot)) return false;
         tp = phase_begin(w);
         const unsigned char *pg = pages + (size_t)slot * kPageBytes;
         const uint4 *row_a = reinterpret_cast<const uint4 *>(pg + warp * row_bytes);
-        if (two) {
+        if (two || nseg > 1) {
             dot_rows2<NVL>(row_a, reinterpret_cast<const uint4 *>(pg + (8 + warp) * row_bytes), xr, K8,
                            lane, acc_a, acc_c);
         } else {
@@ -1112,6 +1194,30 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
         phase_end(w, tp, WS_DOT);
         tp = phase_begin(w);
         const float v = dual_reduce(acc_a, acc_c, lane);
+        if (nseg > 1) {
+            // segment sums in page-row order: matrix row r, segment q at r * nseg + q
+            float *red = &ctl->red[w.red_buf][0][0];
+            if (lane == 0) red[pu * 16 + warp] = v;
+            if (lane == 16) red[pu * 16 + 8 + warp] = v;
+            const int rows = two ? 16 : 8;
+            if (++pu == rows * nseg / 16) {
+                pu = 0;
+                if (!worker_sync(p, ctl, w)) return false;
+                if (warp == 0) {
+                    const int e = lane & 15;
+                    float a = 0.f, c = 0.f;
+                    for (int q = 0; q < nseg; ++q) {
+                        a += red[e * nseg + q];
+                        c += red[((e + 8) & 15) * nseg + q];
+                    }
+                    unit_epilogue(p, ctl, w, t, tile, pair, rows, a, c, pre0, tok, P, best_v, best_i);
+                }
+                w.red_buf ^= 1;
+                tile += pair ? 1 : (two ? 2 : 1);
+            }
+            phase_end(w, tp, WS_EPI);
+            continue;
+        }
         // tile handled by this lane: lanes 0..15 the first page's, 16..31 the second's
         const int my = (lane < 16 || pair) ? tile : tile + 1;
         const int off = my - t.begin;
@@ -1121,8 +1227,8 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
             const float c = __shfl_sync(0xffffffffu, v, 16);
             if (lane == 0) {
                 if (kind == OP_GATEUP) {
-                    st_tag(tag_buf(p, layer, p.tl.act) + (size_t)b * s.F + tile * 8 + warp,
-                           v / (1.0f + expf(-v)) * c, w.ep_out);
+                    st_tag_rep(tag_buf(p, layer, p.tl.act) + (size_t)b * s.F + tile * 8 + warp, p.tl.rep_f,
+                               v / (1.0f + expf(-v)) * c, w.ep_out);
                 } else {
                     const int head = tile / per_head;
                     const int i = (tile % per_head) * 8 + warp;
@@ -1150,7 +1256,7 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
                         resid = (kind == OP_OPROJ && layer == 0)
                                     ? bf2f(p.embed[(size_t)tok * s.H + row])
                                     : wait_tag1(p, ctl, resid_in(p, kind, layer, b) + row, w.ep, (uint32_t)w.task_id);
-                    st_tag(resid_out(p, kind, layer, b) + row, resid + v, w.ep_out);
+                    st_tag_rep(resid_out(p, kind, layer, b) + row, p.tl.rep_h, resid + v, w.ep_out);
                     break;
                 }
                 default:   // OP_LMHEAD
@@ -1167,9 +1273,20 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     }
     stamp_done(p, w);
     if (kind == OP_LMHEAD) {
-        const float ov = __shfl_sync(0xffffffffu, best_v, 16);
-        const int oi = __shfl_sync(0xffffffffu, best_i, 16);
-        if (ov > best_v || (ov == best_v && oi < best_i)) { best_v = ov; best_i = oi; }
+        // segments: warp 0 holds the candidates (lanes 0..15); whole rows:
+        // lanes 0 and 16 of every warp
+        if (nseg == 1) {
+            const float ov = __shfl_sync(0xffffffffu, best_v, 16);
+            const int oi = __shfl_sync(0xffffffffu, best_i, 16);
+            if (ov > best_v || (ov == best_v && oi < best_i)) { best_v = ov; best_i = oi; }
+        } else {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+                if (ov > best_v || (ov == best_v && oi < best_i)) { best_v = ov; best_i = oi; }
+            }
+        }
         if (lane == 0) { ctl->att_m[warp][0] = best_v; ctl->att_l[warp][0] = __int_as_float(best_i); }
         if (!worker_sync(p, ctl, w)) return false;
         if (threadIdx.x == 0) {
@@ -1383,7 +1500,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
                 acc2[h] = acc;
                 if (((rr + 1) & (rpp - 1)) == 0 || rr + 1 == rows) {
                     release_page(ctl, w, slot);
-                    phase_end(w, tp, first_page ? WS_FIRST : WS_DOT);
+                    phase_end(w, tp, first_page ? WS_FIRST : WS_COLS);
                     first_page = false;
                 }
             }
@@ -1401,24 +1518,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
                 a += ctl->red[w.red_buf][i][e];
                 c += ctl->red[w.red_buf][i][(e + 8) & 15];
             }
-            const int grp_row = 8 * (tile - t.begin) + e;   // row within the task
-            const float rres = __shfl_sync(0xffffffffu, resid, grp_row & 31);
-            if (pair) {
-                if (lane < 8) gemv_epilogue_row(p, kind, layer, tile, lane, a, c, b, P, w.ep_out, best_v, best_i);
-            } else if (lane < rows) {
-                const int tl = tile + (e >> 3), r = e & 7;
-                if (resid_op) {
-                    const int row = tl * 8 + r;
-                    const float base = grp_row < 32 ? rres
-                                     : (kind == OP_OPROJ && layer == 0)
-                                           ? bf2f(p.embed[(size_t)tok * s.H + row])
-                                           : wait_tag1(p, ctl, resid_in(p, kind, layer, b) + row, w.ep,
-                                                       (uint32_t)w.task_id);
-                    st_tag(resid_out(p, kind, layer, b) + row, base + a, w.ep_out);
-                } else {
-                    gemv_epilogue_row(p, kind, layer, tl, r, a, 0.f, b, P, w.ep_out, best_v, best_i);
-                }
-            }
+            unit_epilogue(p, ctl, w, t, tile, pair, rows, a, c, resid, tok, P, best_v, best_i);
         }
         w.red_buf ^= 1;
         tile += pair ? 1 : (rows == 16 ? 2 : 1);
@@ -1625,8 +1725,8 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
                     num = fmaf(f, sg[c * (d + 2) + i], num);
                     den = fmaf(f, sg[c * (d + 2) + d + 1], den);
                 }
-                st_tag(tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)(a.kvh * G + g0 + g) * d + i,
-                       num / den, w.ep_out);
+                st_tag_rep(tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)(a.kvh * G + g0 + g) * d + i,
+                           p.tl.rep_qd, num / den, w.ep_out);
             }
         }
     }
@@ -1658,11 +1758,9 @@ __device__ bool run_task(const Params &p, const Task &t, unsigned char *pages, S
         }
     }
     // Few instantiations on purpose: every body is inlined into the one
-    // kernel, and more variants raise the register pressure of the whole.
-    const int K = op_k(p.s, t.kind);
-    if (K <= kRowK) return gemv_rows<kRowK / 256>(p, t, pages, ctl, w);
-    if (K <= kMaxHidden) return gemv_cols<kMaxHidden / 2048>(p, t, pages, ctl, w);
-    if (K <= 4 * 2048) return gemv_cols<4>(p, t, pages, ctl, w);
+    // kernel, and more variants raise the register pressure of the whole and
+    // spread the hot loop over more instruction-cache lines.
+    if (rows_gemv(op_k(p.s, t.kind))) return gemv_rows<kRowK / 256>(p, t, pages, ctl, w);
     return gemv_cols<kMaxK / 2048>(p, t, pages, ctl, w);
 }
 
@@ -1739,6 +1837,7 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         st[ST_WORKER_TASKS] = w.stat[WS_TASKS];
         st[ST_WORKER_ATTN_TAIL] = w.stat[WS_ATT];
         st[14] = w.stat[WS_FIRST];
+        st[15] = w.stat[WS_COLS];
         st[ST_WORKER_TOTAL] = globaltimer() - t_begin;
     }
 }

@@ -72,6 +72,7 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     if (c->hidden > kMaxK || c->ffn > kMaxK || QD > kMaxK) return MK_ERR_INVALID;
     if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return MK_ERR_INVALID;
     if (c->attn_chunks < 0 || c->timeout_ns < 0 || c->l2_lookahead_kb < 0) return MK_ERR_INVALID;
+    if (c->poll_ns < 0 || c->poll_ns > 1000000) return MK_ERR_INVALID;
     if ((long long)c->max_seq * c->head_dim > (1LL << 40)) return MK_ERR_INVALID;
     if (num_sms < 1 || num_sms > 1024) return MK_ERR_INVALID;
     s.L = c->layers; s.H = c->hidden; s.nq = c->n_q_heads; s.nkv = c->n_kv_heads;
@@ -325,6 +326,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
                    : cfg->l2_lookahead_kb > 0 ? 1024LL * cfg->l2_lookahead_kb : kL2Lookahead;
     p.event_wait = (cfg->flags & MK_FLAG_EVENT_WAIT) ? 1 : 0;
     p.debug_withhold = -1;
+    p.poll_ns = (unsigned int)cfg->poll_ns;
     *out = c;
     return MK_OK;
 }

@@ -101,6 +101,7 @@ bool shape_ok(const mk_config *c, int num_sms, Shape &s) {
     if (c->hidden > kMaxHidden || c->ffn > kMaxK || QD > kMaxK) return false;
     if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return false;
     if (c->attn_chunks < 0 || c->timeout_ns < 0 || c->l2_lookahead_kb < 0) return false;
+    if (c->poll_ns < 0 || c->poll_ns > 1000000) return false;
     if (c->flags & MK_FLAG_TRACE) return false;   // no trace buffer in the static scratch
     s.L = c->layers; s.H = c->hidden; s.nq = c->n_q_heads; s.nkv = c->n_kv_heads;
     s.d = c->head_dim; s.F = c->ffn; s.V = c->vocab; s.S = c->max_seq; s.Bmax = c->max_batch;
@@ -277,6 +278,7 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
                    : cfg->l2_lookahead_kb > 0 ? 1024LL * cfg->l2_lookahead_kb : kL2Lookahead;
     p.event_wait = (cfg->flags & MK_FLAG_EVENT_WAIT) ? 1 : 0;
     p.debug_withhold = -1;
+    p.poll_ns = (unsigned int)cfg->poll_ns;
     if (kernel_launch(p, ds.num_sms, st) != cudaSuccess) return MK_ERR_CUDA;
     if (status_out &&
         cudaMemcpyAsync(status_out, d + lay.err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)

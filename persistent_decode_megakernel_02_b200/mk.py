@@ -42,7 +42,7 @@ class Config(C.Structure):
         ("max_seq", C.c_int), ("max_batch", C.c_int),
         ("rope_theta", C.c_float), ("rms_eps", C.c_float),
         ("flags", C.c_int), ("attn_chunks", C.c_int), ("timeout_ns", C.c_longlong),
-        ("l2_lookahead_kb", C.c_int),
+        ("l2_lookahead_kb", C.c_int), ("poll_ns", C.c_int),
     ]
 
 
@@ -122,12 +122,13 @@ def header_functions() -> list[str]:
 
 
 def make_config(shape, max_seq: int, max_batch: int = 1, flags: int = 0,
-                attn_chunks: int = 0, timeout_ns: int = 0, l2_lookahead_kb: int = 0) -> Config:
+                attn_chunks: int = 0, timeout_ns: int = 0, l2_lookahead_kb: int = 0,
+                poll_ns: int = 0) -> Config:
     """`shape`: a workloads.ModelShape (or anything with the same fields)."""
     return Config(shape.layers, shape.hidden, shape.n_q_heads, shape.n_kv_heads,
                   shape.head_dim, shape.ffn, shape.vocab, int(max_seq), int(max_batch),
                   float(shape.rope_theta), float(shape.rms_eps), int(flags),
-                  int(attn_chunks), int(timeout_ns), int(l2_lookahead_kb))
+                  int(attn_chunks), int(timeout_ns), int(l2_lookahead_kb), int(poll_ns))
 
 
 def plan(cfg: Config, num_sms: int) -> dict:
@@ -192,10 +193,10 @@ class Context:
 
     def __init__(self, weights, kcache, vcache, max_seq: int, max_batch: int = 1,
                  flags: int = 0, attn_chunks: int = 0, timeout_ns: int = 0,
-                 l2_lookahead_kb: int = 0):
+                 l2_lookahead_kb: int = 0, poll_ns: int = 0):
         shape = weights.shape
         self.cfg = make_config(shape, max_seq, max_batch, flags, attn_chunks, timeout_ns,
-                               l2_lookahead_kb)
+                               l2_lookahead_kb, poll_ns)
         L = shape.layers
         self._keep = [weights, kcache, vcache]
 
@@ -280,7 +281,7 @@ class Context:
     STAT_NAMES = ["loader_empty_ns", "loader_pages", "loader_total_ns", "worker_full_ns",
                   "worker_ready_ns", "worker_sync_ns", "worker_total_ns", "sched_dep_ns",
                   "worker_prologue_ns", "worker_dot_ns", "worker_epi_ns", "worker_end_ns",
-                  "worker_tasks", "worker_attn_tail_ns", "cols_first_page_ns", "unused15"]
+                  "worker_tasks", "worker_attn_tail_ns", "cols_first_page_ns", "cols_dot_ns"]
 
     def sm_stats(self) -> np.ndarray:
         """Per-SM wait accounting of the last step (trace mode): [num_sms][16]."""
