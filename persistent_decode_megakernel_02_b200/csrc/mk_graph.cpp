@@ -20,11 +20,11 @@ namespace mk {
 
 static constexpr int kMaxSms = 1024;
 
-int default_attn_chunks(int num_sms, int Bmax, int nkv, int S) {
-    int per = Bmax * nkv;
+int default_attn_chunks(int num_sms, int Bmax, int nq, int S) {
+    int per = Bmax * nq;
     int nc = per > 0 ? num_sms / per : 1;
     if (nc < 1) nc = 1;
-    int cap = (S + 15) / 16;            // at least ~16 positions per chunk at capacity
+    int cap = (S + kAttnChunkPositions - 1) / kAttnChunkPositions;   // chunks a full cache needs
     if (cap < 1) cap = 1;
     if (nc > cap) nc = cap;
     return nc;
@@ -111,7 +111,7 @@ struct Builder {
         OpTiles t = op_tiles(s);
         int per_chunk = (s.S + s.NC - 1) / s.NC;
         int64_t est = (int64_t)4 * s.d * per_chunk;   // K + V bf16 of one chunk at capacity
-        const int heads = s.Bmax * s.nkv;             // items per chunk index
+        const int heads = s.Bmax * s.nq;              // items per chunk index
         for (int i = 0; i < t.attn_items; i += p.num_sms) {
             sort_by_load();
             int n = t.attn_items - i < p.num_sms ? t.attn_items - i : p.num_sms;

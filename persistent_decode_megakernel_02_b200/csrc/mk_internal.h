@@ -41,7 +41,11 @@ constexpr int kPageBytes = 65536;   // one shared-memory page
 constexpr int kNumPages = 3;        // pages in the per-SM ring
 constexpr int kVecMax = 7;          // 16-byte vectors per thread per row (K <= 7*8*256)
 constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 14336
-constexpr int kMaxGroup = 8;        // q heads per KV head handled by one attention task
+constexpr int kMaxGroup = 8;        // q heads per KV head
+// Attention chunking: a sequence's positions are split into at most NC
+// chunks of at least this many positions (shorter contexts use fewer chunks;
+// one chunk needs no merge).
+constexpr int kAttnChunkPositions = 1024;
 constexpr int kMaxHeadDim = 256;
 constexpr long long kL2Lookahead = 0;  // default L2 prefetch distance beyond the ring (0: off; measured no gain)
 constexpr int kStageFloats = 8192;  // shared staging: a GEMV input vector, or attention partials
@@ -51,7 +55,7 @@ constexpr int kL2Chunk = 64 * 1024;             // bytes per L2 prefetch instruc
 enum OpKind : int32_t { OP_QKV = 0, OP_ATTN = 1, OP_OPROJ = 2, OP_GATEUP = 3, OP_DOWN = 4, OP_LMHEAD = 5 };
 
 // One task: a contiguous range of tiles of one op (GEMV ops), or one
-// attention work item (b, kv head, chunk), assigned to one SM.
+// attention work item (b, q head, chunk), assigned to one SM.
 struct Task {
     int32_t kind;
     int32_t layer;
@@ -99,7 +103,7 @@ struct OpTiles {
     int gateup;
     int down;
     int lmhead;
-    int attn_items;   // Bmax * nkv * NC
+    int attn_items;   // Bmax * nq * NC
 };
 
 MK_HD inline OpTiles op_tiles(const Shape &s) {
@@ -110,7 +114,7 @@ MK_HD inline OpTiles op_tiles(const Shape &s) {
     t.gateup = s.F / 8;
     t.down = s.H / 8;
     t.lmhead = (s.V + 7) / 8;
-    t.attn_items = s.Bmax * s.nkv * s.NC;
+    t.attn_items = s.Bmax * s.nq * s.NC;
     return t;
 }
 
@@ -298,6 +302,6 @@ PlanSizes plan_sizes(const Shape &s, int num_sms);
 void plan_build(const Shape &s, int num_sms, Plan &p);
 
 // Default number of attention chunks for a shape on `num_sms` SMs.
-int default_attn_chunks(int num_sms, int Bmax, int nkv, int S);
+int default_attn_chunks(int num_sms, int Bmax, int nq, int S);
 
 }  // namespace mk

@@ -220,9 +220,8 @@ __device__ __forceinline__ float2 dot8x2(const uint4 w, const float *x, float2 a
 // ---------------------------------------------------------------------------
 // shared memory
 // ---------------------------------------------------------------------------
-constexpr int kAttnCombine = 512;   // G * head_dim handled by the warp combine
-static_assert(kWorkerWarps * kAttnCombine <= kStageFloats, "combine fits the staging area");
-constexpr int kMinChunk = 32;       // fewest positions per active attention chunk
+constexpr int kAttnCombine = kMaxHeadDim + 8;   // per-warp slot of the attention combine
+static_assert(kWorkerWarps * kAttnCombine + 16 * 12 <= kStageFloats, "combine fits the staging area");
 constexpr int kSigRing = 64;        // pending task completions the signaler can hold
 
 struct __align__(16) SmemCtl {
@@ -337,9 +336,9 @@ __device__ __forceinline__ size_t my_copy(size_t stride) { return (size_t)(block
 // ---------------------------------------------------------------------------
 // task geometry shared by the loader and the workers
 // ---------------------------------------------------------------------------
-// Attention chunk of one work item.
+// Attention chunk of one work item (sequence b, q head h, chunk c).
 struct AttnChunk {
-    int b, kvh, c;
+    int b, h, kvh, c;
     bool active;      // sequence b takes part in this step
     int P;            // position of the new token
     int c0, c1;       // positions [c0, c1) of this chunk (c1 <= P + 1)
@@ -351,17 +350,18 @@ struct AttnChunk {
 __device__ __forceinline__ AttnChunk attn_chunk(const Params &p, int item) {
     const Shape &s = p.s;
     AttnChunk a;
-    a.b = item / (s.nkv * s.NC);
-    a.kvh = (item / s.NC) % s.nkv;
+    a.b = item / (s.nq * s.NC);
+    a.h = (item / s.NC) % s.nq;
+    a.kvh = a.h / s.G;
     a.c = item % s.NC;
     a.active = a.b < p.batch;
     a.P = 0; a.c0 = 0; a.c1 = 0; a.npre = 0; a.has_new = false; a.nc = 0;
     if (a.active) {
         a.P = p.positions[a.b];
         int C = a.P + 1;
-        // at most NC chunks, but no fewer than kMinChunk positions per chunk:
-        // short contexts use few chunks (fewer partials to merge)
-        const int nc = min(s.NC, (C + kMinChunk - 1) / kMinChunk);
+        // at most NC chunks, but no fewer than kAttnChunkPositions positions
+        // per chunk: short contexts use one chunk (nothing to merge)
+        const int nc = min(s.NC, (C + kAttnChunkPositions - 1) / kAttnChunkPositions);
         int Lc = (C + nc - 1) / nc;
         a.nc = nc;
         a.c0 = a.c * Lc;
@@ -1541,193 +1541,220 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
 }
 
 // ---------------------------------------------------------------------------
-// attention task body: one chunk of positions of one KV head, G q heads
+// attention task body: one chunk of positions of one q head
 // ---------------------------------------------------------------------------
-template <int G, int DPL>   // q heads per KV head, head dims per lane (d = 32 * DPL)
+// Prefix K/V rows of the chunk arrive through the ring (a page holds the K
+// block then the V block of up to 256 / 128 positions).  Each warp takes
+// blocks of 32 positions: lanes compute the 32 scores at once (lane j reads
+// K row j in a rotated chunk order, so the 8 lanes of a shared-memory phase
+// hit different banks; q sits in shared memory padded the same way), the
+// warp updates its online-softmax state (max, sum) with two reductions,
+// and accumulates P·V with lanes over head dims.  The new position's k/v
+// come from tagged words (warp 0).  The warps' states are combined through
+// shared memory; a single-chunk task writes the q head's output directly,
+// otherwise the chunk's (o, m, l) partial goes out tagged and chunk 0's task
+// merges the partials of its q head.
+template <int D>   // head_dim: 64 or 128
 __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                           WState &w) {
     const Shape &s = p.s;
-    constexpr int d = 32 * DPL;
+    constexpr int DPL = D / 32;   // head dims per lane in P·V
+    constexpr int NCH = D / 8;    // 16-byte chunks of a K row
+    constexpr int KP = DPL / 2;   // tagged pairs of the new k (and v) per lane
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const AttnChunk a = attn_chunk(p, t.begin);
-    const int npp = attn_pos_per_page(d);
+    const int npp = attn_pos_per_page(D);
     if (!wait_ready(p, ctl, w)) return false;
     unsigned long long tp = phase_begin(w);
     const int npages = (a.npre + npp - 1) / npp;
+    float *qs = ctl->stage + kWorkerWarps * kAttnCombine;   // q: chunk c (8 values) at qs + 12 c
 
-    float m[G], l[G], o[G][DPL], qr[G][DPL];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        m[g] = -INFINITY;
-        l[g] = 0.f;
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) { o[g][i] = 0.f; qr[g][i] = 0.f; }
-    }
-    // q of the group's heads (every warp) and the new position's key and
-    // value (the warp that visits it): tagged pairs, polled until fresh
-    const bool new_warp = a.has_new && warp == (a.npre % kWorkerWarps);
+    // ---- q (threads 0 .. D/2-1, one pair each) and the new k / v (warp 0),
+    // tagged, polled until fresh
+    const bool new_warp = a.has_new && warp == 0;
     float kn[DPL], vn[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) { kn[i] = 0.f; vn[i] = 0.f; }
-    {
-        constexpr int QP = G * DPL / 2, KP = DPL / 2;   // pairs per lane
-        const uint64_t *qsrc = tag_buf(p, t.layer, p.tl.q) + (size_t)a.b * s.QD + (size_t)a.kvh * G * d + lane * DPL;
-        const uint64_t *ksrc = tag_buf(p, t.layer, p.tl.kn) + (size_t)a.b * s.KD + (size_t)a.kvh * d + lane * DPL;
-        const uint64_t *vsrc = tag_buf(p, t.layer, p.tl.vn) + (size_t)a.b * s.KD + (size_t)a.kvh * d + lane * DPL;
+    if (a.active) {
+        const uint64_t *qsrc = tag_buf(p, t.layer, p.tl.q) + (size_t)a.b * s.QD + (size_t)a.h * D;
+        const uint64_t *ksrc = tag_buf(p, t.layer, p.tl.kn) + (size_t)a.b * s.KD + (size_t)a.kvh * D + lane * DPL;
+        const uint64_t *vsrc = tag_buf(p, t.layer, p.tl.vn) + (size_t)a.b * s.KD + (size_t)a.kvh * D + lane * DPL;
+        float2 qv = make_float2(0.f, 0.f);
         uint32_t pend = 0;
+        // bit 0: this thread's q pair; bits 1 .. KP: new k pairs; then new v pairs
         auto load = [&](int bit) {
-            // bits [0, QP): q pairs (head g = bit / KP); then KP key pairs, KP value pairs
             ulonglong2 v;
-            if (bit < QP) {
-                const int g = bit / KP, h = bit % KP;
-                v = ld_tag2(qsrc + (size_t)g * d + 2 * h);
-                qr[g][2 * h] = tag_val(v.x);
-                qr[g][2 * h + 1] = tag_val(v.y);
-            } else if (bit < QP + KP) {
-                const int h = bit - QP;
-                v = ld_tag2(ksrc + 2 * h);
-                kn[2 * h] = tag_val(v.x);
-                kn[2 * h + 1] = tag_val(v.y);
+            if (bit == 0) {
+                v = ld_tag2(qsrc + 2 * tid);
+                qv = make_float2(tag_val(v.x), tag_val(v.y));
+            } else if (bit <= KP) {
+                v = ld_tag2(ksrc + 2 * (bit - 1));
+                kn[2 * (bit - 1)] = tag_val(v.x);
+                kn[2 * (bit - 1) + 1] = tag_val(v.y);
             } else {
-                const int h = bit - QP - KP;
-                v = ld_tag2(vsrc + 2 * h);
-                vn[2 * h] = tag_val(v.x);
-                vn[2 * h + 1] = tag_val(v.y);
+                v = ld_tag2(vsrc + 2 * (bit - 1 - KP));
+                vn[2 * (bit - 1 - KP)] = tag_val(v.x);
+                vn[2 * (bit - 1 - KP) + 1] = tag_val(v.y);
             }
-            if (!tag_ok(v.x, w.ep) || !tag_ok(v.y, w.ep)) pend |= 1u << bit;
-            else pend &= ~(1u << bit);
+            if (tag_ok(v.x, w.ep) && tag_ok(v.y, w.ep)) pend &= ~(1u << bit);
+            else pend |= 1u << bit;
         };
-        if (a.active) {
 #pragma unroll
-            for (int bit = 0; bit < QP + 2 * KP; ++bit)
-                if (bit < QP || new_warp) load(bit);
-        }
+        for (int bit = 0; bit <= 2 * KP; ++bit)
+            if ((bit == 0 && tid < D / 2) || (bit > 0 && new_warp)) load(bit);
         Spin sp;
         while (__any_sync(0xffffffffu, pend != 0u)) {
             if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 4u)) return false;
 #pragma unroll
-            for (int bit = 0; bit < QP + 2 * KP; ++bit)
+            for (int bit = 0; bit <= 2 * KP; ++bit)
                 if (pend & (1u << bit)) load(bit);
         }
-        const float scale = 1.0f / sqrtf((float)d);
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) qr[g][i] *= scale;
-    }
-    stamp_ready(p, w);
-
-    auto visit = [&](const float (&kv)[DPL], const float (&vv)[DPL]) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float sc = 0.f;
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) sc = fmaf(qr[g][i], kv[i], sc);
-            sc = warp_sum(sc);
-            const float mn = fmaxf(m[g], sc);
-            const float corr = expf(m[g] - mn);
-            const float pe = expf(sc - mn);
-            l[g] = l[g] * corr + pe;
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) o[g][i] = fmaf(o[g][i], corr, pe * vv[i]);
-            m[g] = mn;
+        if (tid < D / 2) {
+            const float scale = 1.0f / sqrtf((float)D);
+            const int e = 2 * tid;
+            qs[12 * (e >> 3) + (e & 7)] = qv.x * scale;
+            qs[12 * (e >> 3) + (e & 7) + 1] = qv.y * scale;
         }
-    };
-
+    }
+    if (!worker_sync(p, ctl, w)) return false;   // q visible to every warp
+    stamp_ready(p, w);
     phase_end(w, tp, WS_PRO);
     stamp_input(p, w);
+
+    float m = -INFINITY, l = 0.f, o[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) o[i] = 0.f;
     for (int pg = 0; pg < npages; ++pg) {
         uint32_t slot;
         if (!wait_page(p, ctl, w, slot)) return false;
         tp = phase_begin(w);
         const uint16_t *Kp = reinterpret_cast<const uint16_t *>(pages + (size_t)slot * kPageBytes);
-        const uint16_t *Vp = Kp + (size_t)npp * d;
+        const uint16_t *Vp = Kp + (size_t)npp * D;
         const int n = min(npp, a.npre - pg * npp);
-        for (int j = warp; j < n; j += kWorkerWarps) {
-            float kv[DPL], vv[DPL];
+        for (int j0 = warp * 32; j0 < n; j0 += kWorkerWarps * 32) {
+            const int j = j0 + lane;
+            float sc = -INFINITY;
+            if (j < n) {
+                const uint4 *krow = reinterpret_cast<const uint4 *>(Kp + (size_t)j * D);
+                float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < DPL; i += 2) {
-                const uint32_t kw = *reinterpret_cast<const uint32_t *>(Kp + (size_t)j * d + lane * DPL + i);
-                const uint32_t vw = *reinterpret_cast<const uint32_t *>(Vp + (size_t)j * d + lane * DPL + i);
-                kv[i] = bf_lo(kw); kv[i + 1] = bf_hi(kw);
-                vv[i] = bf_lo(vw); vv[i + 1] = bf_hi(vw);
+                for (int c = 0; c < NCH; ++c) {
+                    const int cc = (c + lane) & (NCH - 1);
+                    const uint4 kw = krow[cc];
+                    const float4 q0 = *reinterpret_cast<const float4 *>(qs + 12 * cc);
+                    const float4 q1 = *reinterpret_cast<const float4 *>(qs + 12 * cc + 4);
+                    acc = ffma2(make_float2(bf_lo(kw.x), bf_hi(kw.x)), make_float2(q0.x, q0.y), acc);
+                    acc = ffma2(make_float2(bf_lo(kw.y), bf_hi(kw.y)), make_float2(q0.z, q0.w), acc);
+                    acc = ffma2(make_float2(bf_lo(kw.z), bf_hi(kw.z)), make_float2(q1.x, q1.y), acc);
+                    acc = ffma2(make_float2(bf_lo(kw.w), bf_hi(kw.w)), make_float2(q1.z, q1.w), acc);
+                }
+                sc = acc.x + acc.y;
             }
-            visit(kv, vv);
+            float mb = sc;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
+            const float mn = fmaxf(m, mb);             // finite: lane 0's position is valid
+            const float corr = expf(m - mn);
+            const float pe = j < n ? expf(sc - mn) : 0.f;
+            l = l * corr + warp_sum(pe);
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) o[i] *= corr;
+            m = mn;
+            const int cnt = min(32, n - j0);
+            const uint16_t *vb = Vp + (size_t)j0 * D + lane * DPL;
+            for (int k = 0; k < cnt; ++k) {
+                const float pk = __shfl_sync(0xffffffffu, pe, k);
+                if constexpr (DPL == 2) {
+                    const uint32_t vw = *reinterpret_cast<const uint32_t *>(vb + (size_t)k * D);
+                    o[0] = fmaf(pk, bf_lo(vw), o[0]);
+                    o[1] = fmaf(pk, bf_hi(vw), o[1]);
+                } else {
+                    const uint2 vw = *reinterpret_cast<const uint2 *>(vb + (size_t)k * D);
+                    o[0] = fmaf(pk, bf_lo(vw.x), o[0]);
+                    o[1] = fmaf(pk, bf_hi(vw.x), o[1]);
+                    o[2] = fmaf(pk, bf_lo(vw.y), o[2]);
+                    o[3] = fmaf(pk, bf_hi(vw.y), o[3]);
+                }
+            }
         }
         release_page(ctl, w, slot);
         phase_end(w, tp, WS_DOT);
     }
     tp = phase_begin(w);
-    if (new_warp) visit(kn, vn);
-
-    // ---- combine the warps' running states into this chunk's partial
-    if (lane == 0) {
+    if (new_warp) {
+        float sc = 0.f;
 #pragma unroll
-        for (int g = 0; g < G; ++g) { ctl->att_m[warp][g] = m[g]; ctl->att_l[warp][g] = l[g]; }
+        for (int i = 0; i < DPL; ++i) {
+            const int e = lane * DPL + i;
+            sc = fmaf(qs[12 * (e >> 3) + (e & 7)], kn[i], sc);
+        }
+        sc = warp_sum(sc);
+        const float mn = fmaxf(m, sc);
+        const float corr = expf(m - mn);
+        const float pe = expf(sc - mn);
+        l = l * corr + pe;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) o[i] = fmaf(o[i], corr, pe * vn[i]);
+        m = mn;
     }
+
+    // ---- combine the warps' states
+    float *cw = ctl->stage + warp * kAttnCombine;
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) ctl->stage[warp * kAttnCombine + g * d + lane * DPL + i] = o[g][i];
+    for (int i = 0; i < DPL; ++i) cw[lane * DPL + i] = o[i];
+    if (lane == 0) { cw[D] = m; cw[D + 1] = l; }
     if (!worker_sync(p, ctl, w)) return false;
-    // this chunk's partial (per q head: o[d], m, l) as tagged words
-    uint64_t *part = tag_buf(p, t.layer, p.tl.part) + ((size_t)a.b * s.nq + (size_t)a.kvh * G) * s.NC * (d + 2);
-    if (a.active) {
-        for (int e = tid; e < G * d; e += kWorkerThreads) {
-            const int g = e / d, i = e % d;
-            float M = -INFINITY;
+    uint64_t *part = tag_buf(p, t.layer, p.tl.part) + ((size_t)a.b * s.nq + a.h) * s.NC * (D + 2);
+    // chunks at or past nc hold no positions and write nothing
+    if (a.active && a.c < a.nc && tid < D) {
+        float M = -INFINITY;
 #pragma unroll
-            for (int k = 0; k < kWorkerWarps; ++k) M = fmaxf(M, ctl->att_m[k][g]);
-            float O = 0.f, Lsum = 0.f;
-            if (M != -INFINITY) {
+        for (int k = 0; k < kWorkerWarps; ++k) M = fmaxf(M, ctl->stage[k * kAttnCombine + D]);
+        float O = 0.f, L = 0.f;
+        if (M != -INFINITY) {
 #pragma unroll
-                for (int k = 0; k < kWorkerWarps; ++k) {
-                    const float f = expf(ctl->att_m[k][g] - M);
-                    O = fmaf(f, ctl->stage[k * kAttnCombine + e], O);
-                    Lsum = fmaf(f, ctl->att_l[k][g], Lsum);
-                }
+            for (int k = 0; k < kWorkerWarps; ++k) {
+                const float *ck = ctl->stage + k * kAttnCombine;
+                const float f = expf(ck[D] - M);
+                O = fmaf(f, ck[tid], O);
+                L = fmaf(f, ck[D + 1], L);
             }
-            uint64_t *dst = part + ((size_t)g * s.NC + a.c) * (d + 2);
-            st_tag(dst + i, O, w.ep_out);
-            if (i == 0) {
-                st_tag(dst + d, M, w.ep_out);
-                st_tag(dst + d + 1, Lsum, w.ep_out);
+        }
+        if (a.nc == 1) {
+            st_tag_rep(tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)a.h * D + tid,
+                       p.tl.rep_qd, O / L, w.ep_out);
+        } else {
+            uint64_t *dst = part + (size_t)a.c * (D + 2);
+            st_tag(dst + tid, O, w.ep_out);
+            if (tid == 0) {
+                st_tag(dst + D, M, w.ep_out);
+                st_tag(dst + D + 1, L, w.ep_out);
             }
         }
     }
     stamp_done(p, w);
-    if (a.active && a.c == 0) {
-        // chunk 0's task merges the KV head's partials: it polls them into
-        // shared memory (tagged, so it waits for exactly the chunks it
-        // reads), then combines them there.  No fence or counter: the tags
-        // carry the readiness.
+    if (a.active && a.nc > 1 && a.c == 0) {
+        // chunk 0's task merges its q head's partials: polls them into shared
+        // memory (tagged, so it waits for exactly the chunks it reads), then
+        // combines them there
         const int nc = a.nc;
-        const int per = nc * (d + 2);                       // words per q head
-        const int hb = min(G, kStageFloats / per);          // q heads per batch
-        for (int g0 = 0; g0 < G; g0 += hb) {
-            const int nh = min(hb, G - g0);
-            // every thread is done reading the stage (the combine above, or
-            // the previous batch's merge) before it is refilled
-            if (!worker_sync(p, ctl, w)) return false;
-            if (!stage_partials(p, ctl, w, part + (size_t)g0 * s.NC * (d + 2), nh, per, s.NC * (d + 2)))
-                return false;
-            if (!worker_sync(p, ctl, w)) return false;
-            for (int e = tid; e < nh * d; e += kWorkerThreads) {
-                const int g = e / d, i = e - g * d;
-                const float *sg = ctl->stage + g * per;
-                float M = -INFINITY;
-                for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (d + 2) + d]);
-                float num = 0.f, den = 0.f;
-                for (int c = 0; c < nc; ++c) {
-                    const float mc = sg[c * (d + 2) + d];
-                    if (mc == -INFINITY) continue;
-                    const float f = expf(mc - M);
-                    num = fmaf(f, sg[c * (d + 2) + i], num);
-                    den = fmaf(f, sg[c * (d + 2) + d + 1], den);
-                }
-                st_tag_rep(tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)(a.kvh * G + g0 + g) * d + i,
-                           p.tl.rep_qd, num / den, w.ep_out);
+        if (!worker_sync(p, ctl, w)) return false;   // the combine above is done with the stage
+        if (!stage_partials(p, ctl, w, part, 1, nc * (D + 2), s.NC * (D + 2))) return false;
+        if (!worker_sync(p, ctl, w)) return false;
+        if (tid < D) {
+            const float *sg = ctl->stage;
+            float M = -INFINITY;
+            for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (D + 2) + D]);
+            float num = 0.f, den = 0.f;
+            for (int c = 0; c < nc; ++c) {
+                const float mc = sg[c * (D + 2) + D];
+                if (mc == -INFINITY) continue;
+                const float f = expf(mc - M);
+                num = fmaf(f, sg[c * (D + 2) + tid], num);
+                den = fmaf(f, sg[c * (D + 2) + D + 1], den);
             }
+            st_tag_rep(tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)a.h * D + tid,
+                       p.tl.rep_qd, num / den, w.ep_out);
         }
     }
     if (!worker_sync(p, ctl, w)) return false;
@@ -1739,24 +1766,10 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
 // ---------------------------------------------------------------------------
 // worker role
 // ---------------------------------------------------------------------------
-template <int G>
-__device__ bool attn_dispatch_d(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
-                                WState &w) {
-    // head_dim 64 or 128, with G * head_dim <= 512 (checked by mk_create)
-    if (G == 8 || p.s.d == 64) return attn_task<G, 2>(p, t, pages, ctl, w);
-    return attn_task<G, 4>(p, t, pages, ctl, w);
-}
-
 __device__ bool run_task(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                          WState &w) {
-    if (t.kind == OP_ATTN) {
-        switch (p.s.G) {
-        case 1: return attn_dispatch_d<1>(p, t, pages, ctl, w);
-        case 2: return attn_dispatch_d<2>(p, t, pages, ctl, w);
-        case 4: return attn_dispatch_d<4>(p, t, pages, ctl, w);
-        default: return attn_dispatch_d<8>(p, t, pages, ctl, w);
-        }
-    }
+    if (t.kind == OP_ATTN)   // head_dim 64 or 128 (checked by mk_create)
+        return p.s.d == 64 ? attn_task<64>(p, t, pages, ctl, w) : attn_task<128>(p, t, pages, ctl, w);
     // Few instantiations on purpose: every body is inlined into the one
     // kernel, and more variants raise the register pressure of the whole and
     // spread the hot loop over more instruction-cache lines.

@@ -66,7 +66,6 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     if (G != 1 && G != 2 && G != 4 && G != 8) return MK_ERR_INVALID;
     if (c->head_dim != 64 && c->head_dim != 128) return MK_ERR_INVALID;
     if (c->hidden > kMaxHidden) return MK_ERR_INVALID;
-    if (G * c->head_dim > 512) return MK_ERR_INVALID;
     const long long QD = (long long)c->n_q_heads * c->head_dim;
     if (c->hidden % 8 || c->ffn % 8 || QD % 8) return MK_ERR_INVALID;
     if (c->hidden > kMaxK || c->ffn > kMaxK || QD > kMaxK) return MK_ERR_INVALID;
@@ -79,7 +78,7 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     s.d = c->head_dim; s.F = c->ffn; s.V = c->vocab; s.S = c->max_seq; s.Bmax = c->max_batch;
     s.G = G; s.QD = (int)QD; s.KD = c->n_kv_heads * c->head_dim;
     s.theta = c->rope_theta; s.eps = c->rms_eps;
-    s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nkv, s.S);
+    s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nq, s.S);
     if (s.NC > 4096) return MK_ERR_INVALID;
     // one q head's chunk partials must fit the merge's shared staging area
     if ((long long)s.NC * (s.d + 2) > kStageFloats) return MK_ERR_INVALID;

@@ -95,7 +95,6 @@ bool shape_ok(const mk_config *c, int num_sms, Shape &s) {
     const int G = c->n_q_heads / c->n_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return false;
     if (c->head_dim != 64 && c->head_dim != 128) return false;
-    if (G * c->head_dim > 512) return false;
     const long long QD = (long long)c->n_q_heads * c->head_dim;
     if (c->hidden % 8 || c->ffn % 8 || QD % 8) return false;
     if (c->hidden > kMaxHidden || c->ffn > kMaxK || QD > kMaxK) return false;
@@ -107,7 +106,7 @@ bool shape_ok(const mk_config *c, int num_sms, Shape &s) {
     s.d = c->head_dim; s.F = c->ffn; s.V = c->vocab; s.S = c->max_seq; s.Bmax = c->max_batch;
     s.G = G; s.QD = (int)QD; s.KD = c->n_kv_heads * c->head_dim;
     s.theta = c->rope_theta; s.eps = c->rms_eps;
-    s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nkv, s.S);
+    s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nq, s.S);
     if (s.NC > 4096 || (long long)s.NC * (s.d + 2) > kStageFloats) return false;
     return true;
 }

@@ -64,7 +64,7 @@ def test_every_row_and_item_covered_once(planned):
             if (kind == LMHEAD) != (layer == shape.layers):
                 assert len(sel) == 0
                 continue
-            n = shape.n_kv_heads * nc if kind == ATTN else tiles[kind]
+            n = shape.n_q_heads * nc if kind == ATTN else tiles[kind]
             cover = np.zeros(n, np.int32)
             for t in sel:
                 cover[t[4]:t[5]] += 1
@@ -159,8 +159,13 @@ def test_plan_rejects_unsupported_shapes(bad):
 
 
 def test_default_attention_chunks():
-    assert mk.plan(mk.make_config(wl.LLAMA_1B, 16640), SMS)["info"].attn_chunks == 18
-    assert mk.plan(mk.make_config(wl.TINY, 64), SMS)["info"].attn_chunks == 4
+    # one task per (sequence, q head, chunk): as many chunks as fill the SMs
+    # (148 // 32 q heads = 4), but no more than a full cache needs at 1024
+    # positions per chunk
+    assert mk.plan(mk.make_config(wl.LLAMA_1B, 16640), SMS)["info"].attn_chunks == 4
+    assert mk.plan(mk.make_config(wl.LLAMA_1B, 560), SMS)["info"].attn_chunks == 1
+    assert mk.plan(mk.make_config(wl.TINY, 64), SMS)["info"].attn_chunks == 1
+    assert mk.plan(mk.make_config(wl.TINY, 4096), SMS)["info"].attn_chunks == 4
     assert mk.plan(mk.make_config(wl.TINY, 64, attn_chunks=7), SMS)["info"].attn_chunks == 7
 
 

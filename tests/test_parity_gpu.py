@@ -83,6 +83,23 @@ def test_attention_chunking_does_not_change_results(chunks):
         _check_step(pair, pos, g_tok, g_log, ref)
 
 
+@pytest.mark.parametrize("chunks", [3, 5])
+def test_long_prefix_split_into_chunks_and_merged(chunks):
+    # 2600+ positions: ceil(C / 1024) = 3 active chunks per q head, merged by
+    # chunk 0's task (with 5 chunks, two are empty)
+    shape = wl.TINY
+    S = 2624
+    pair = Pair(shape, max_seq=S, prefill_len=2600, attn_chunks=chunks)
+    toks = wl.make_prompt(shape.vocab, 4, seed=13)
+    for i, t in enumerate(toks):
+        pos = 2600 + i
+        g_tok, g_log = pair.gpu_step(int(t), pos)
+        ref = pair.ref_step(int(t), pos, intermediates=True)
+        _check_step(pair, pos, g_tok, g_log, ref)
+    got = pair.ctx.read_buffer(pair.mk.MK_BUF_ATTN, ref["attn"].size).astype(np.float64)
+    assert rel_l2(got, ref["attn"]) <= 5e-3
+
+
 def test_edge_positions_tokens_and_null_logits():
     shape = wl.TINY
     S = 24
