@@ -41,6 +41,7 @@ constexpr int kPageBytes = 65536;   // one shared-memory page
 constexpr int kNumPages = 3;        // pages in the per-SM ring
 constexpr int kVecMax = 7;          // 16-byte vectors per thread per row (K <= 7*8*256)
 constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 14336
+constexpr int kMaxBatch = 1;        // sequences per step (MK_MAX_BATCH)
 constexpr int kMaxGroup = 8;        // q heads per KV head
 // Attention chunking: a sequence's positions are split into at most NC
 // chunks of at least this many positions (shorter contexts use fewer chunks;
@@ -181,7 +182,7 @@ MK_HD inline int attn_pos_per_page(int d) { return kPageBytes / (4 * d); }
 //                                          [Bmax][nq][NC][d + 2]
 //   attn: merged attention output          [R][Bmax][nq * d]
 //   act:  SiLU(gate) * up                  [R][Bmax][F]
-constexpr int kReplicas = 8;
+constexpr int kReplicas = 1;
 struct TagLayout {
     size_t xa, xb, q, kn, vn, part, attn, act;   // word offsets within a layer's block
     size_t rep_h, rep_qd, rep_f;                 // distance between copies (words)
@@ -244,8 +245,7 @@ static_assert(sizeof(TraceRec) == 64, "trace record layout");
 struct Params {
     Shape s;
     // graph
-    const Task *tasks;
-    const int32_t *queue;
+    const Task *qtasks;          // [num_tasks] the tasks in queue order, `sm` holding the task id
     const int32_t *qoff;         // [num_sms + 1]
     const uint32_t *thresholds;  // [num_events]
     uint32_t *events;            // [num_events]

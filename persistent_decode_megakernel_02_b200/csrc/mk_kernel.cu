@@ -109,9 +109,6 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
 __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void prefetch_l2_line(const void *p) {
-    asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
-}
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -224,6 +221,14 @@ constexpr int kAttnCombine = kMaxHeadDim + 8;   // per-warp slot of the attentio
 static_assert(kWorkerWarps * kAttnCombine + 16 * 12 <= kStageFloats, "combine fits the staging area");
 constexpr int kSigRing = 64;        // pending task completions the signaler can hold
 
+// A task record as the loader publishes it to the workers: the task and the
+// RMSNorm gain its input takes (null if none).
+struct TaskRec {
+    Task t;
+    const uint16_t *gain;
+};
+constexpr int kTaskRing = 8;        // task records the loader may publish ahead
+
 struct __align__(16) SmemCtl {
     uint64_t full[kNumPages];
     uint64_t empty[kNumPages];
@@ -233,6 +238,11 @@ struct __align__(16) SmemCtl {
     uint32_t ep;                // epoch of this launch (steps completed + 1)
     uint32_t last_flag;         // broadcast of "this task arrived last"
     uint32_t loader_done;       // the loader has issued its last page
+    uint32_t tq_pub;            // task records published by the loader
+    uint32_t tq_reads;          // worker warps done reading a record (8 per task)
+    int32_t tok[kMaxBatch];     // this launch's tokens and positions, read once
+    int32_t pos[kMaxBatch];
+    TaskRec tq[kTaskRing];      // records of the next tasks of this queue
     long long issued;           // GEMV bytes the loader has issued into the ring
     uint32_t sig_post;          // task completions posted by the workers
     uint32_t sig_done;          // completions the signaler has published
@@ -347,7 +357,7 @@ struct AttnChunk {
     int nc;           // chunks with positions for this sequence (the others are empty)
 };
 
-__device__ __forceinline__ AttnChunk attn_chunk(const Params &p, int item) {
+__device__ __forceinline__ AttnChunk attn_chunk(const Params &p, const SmemCtl *ctl, int item) {
     const Shape &s = p.s;
     AttnChunk a;
     a.b = item / (s.nq * s.NC);
@@ -357,7 +367,7 @@ __device__ __forceinline__ AttnChunk attn_chunk(const Params &p, int item) {
     a.active = a.b < p.batch;
     a.P = 0; a.c0 = 0; a.c1 = 0; a.npre = 0; a.has_new = false; a.nc = 0;
     if (a.active) {
-        a.P = p.positions[a.b];
+        a.P = ctl->pos[a.b];
         int C = a.P + 1;
         // at most NC chunks, but no fewer than kAttnChunkPositions positions
         // per chunk: short contexts use one chunk (nothing to merge)
@@ -436,37 +446,6 @@ __device__ __forceinline__ bool ring_acquire(const Params &p, SmemCtl *ctl, Ring
     return true;
 }
 
-// L2 prefetcher (one warp, plain prefetch.global.L2 per 128-byte line, so it
-// never queues behind or in front of the loader's bulk copies): walks the
-// GEMV byte ranges of the queue and keeps `lookahead` bytes beyond what the
-// loader has issued into the ring, so HBM keeps streaming while the ring is
-// full.  The loader publishes its progress in ctl->issued.
-__device__ void prefetch_role(const Params &p, SmemCtl *ctl) {
-    const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
-    const int lane = threadIdx.x & 31;
-    long long done = 0;
-    for (int qi = q0; qi < q1; ++qi) {
-        const Task t = p.tasks[p.queue[qi]];
-        if (t.kind == OP_ATTN) continue;
-        GemvStream g = gemv_stream(p, t);
-        const char *src = g.src;
-        long long left = g.left;
-        while (left > 0) {
-            // wait (bounded) until the loader is close enough
-            Spin sp;
-            while (done >= *(volatile long long *)&ctl->issued + p.l2_lookahead) {
-                if (*(volatile uint32_t *)&ctl->loader_done) return;
-                if (!spin_ok(sp, p, ctl, W_EMPTY, 0xffffffffu, 0u)) return;
-            }
-            const long long chunk = min(left, 4096LL);      // 32 lanes x 128 B
-            if ((long long)lane * 128 < chunk) prefetch_l2_line(src + lane * 128);
-            src += chunk;
-            left -= chunk;
-            done += chunk;
-        }
-    }
-}
-
 __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     Ring ring;
@@ -475,11 +454,50 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
     long long issued = 0;   // GEMV bytes copied into the ring so far
     bool ok = true;         // false when a wait was abandoned
     const uint64_t wpol = policy_evict_first();
+    // L2 prefetch cursor: GEMV weight bytes of the queue, bulk-prefetched
+    // into L2 up to l2_lookahead bytes beyond what the ring has taken, so
+    // HBM keeps streaming while the ring is full (one instruction per 64 KB)
+    int pf_qi = q0 - 1;
+    const char *pf_src = nullptr;
+    long long pf_left = 0, pf_done = 0;
+    auto prefetch_to = [&](long long target) {
+        while (pf_done < target) {
+            if (pf_left <= 0) {
+                do { ++pf_qi; } while (pf_qi < q1 && p.qtasks[pf_qi].kind == OP_ATTN);
+                if (pf_qi >= q1) { pf_done = 0x7fffffffffffffffLL; return; }
+                const GemvStream g = gemv_stream(p, p.qtasks[pf_qi]);
+                pf_src = g.src;
+                pf_left = g.left;
+                continue;
+            }
+            const uint32_t n = (uint32_t)min(pf_left, (long long)kPageBytes);
+            prefetch_l2(pf_src, n);
+            pf_src += n;
+            pf_left -= n;
+            pf_done += n;
+        }
+    };
     for (int qi = q0; qi < q1 && ok; ++qi) {
-        const int id = p.queue[qi];
-        const Task t = p.tasks[id];
+        const Task t = p.qtasks[qi];
+        const int id = t.sm;
+        {
+            // publish the task's record to the workers (ring of kTaskRing:
+            // wait until every warp has read the record this slot held)
+            const int k = qi - q0;
+            Spin sr;
+            while (k >= kTaskRing &&
+                   *(volatile uint32_t *)&ctl->tq_reads < (uint32_t)kWorkerWarps * (uint32_t)(k - kTaskRing + 1))
+                if (!spin_ok(sr, p, ctl, W_READY, (uint32_t)id, 4u)) { ok = false; break; }
+            if (!ok) break;
+            TaskRec &r = ctl->tq[k % kTaskRing];
+            r.t = t;
+            r.gain = t.kind == OP_QKV ? p.layers[t.layer].g_attn
+                   : t.kind == OP_GATEUP ? p.layers[t.layer].g_mlp
+                   : t.kind == OP_LMHEAD ? p.g_final : nullptr;
+            st_release_cta_shared(&ctl->tq_pub, (uint32_t)(k + 1));
+        }
         if (t.kind == OP_ATTN) {
-            const AttnChunk a = attn_chunk(p, t.begin);
+            const AttnChunk a = attn_chunk(p, ctl, t.begin);
             const int npp = attn_pos_per_page(p.s.d);
             const LayerW &L = p.layers[t.layer];
             const size_t head_off = ((size_t)a.b * p.s.nkv + a.kvh) * p.s.S;
@@ -498,6 +516,7 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         GemvStream g = gemv_stream(p, t);
         for (int k = 0; k < g.npages; ++k) {
             const uint32_t bytes = (uint32_t)max(0LL, min((long long)g.page_bytes, g.left));
+            if (p.l2_lookahead) prefetch_to(issued + bytes + p.l2_lookahead);
             uint32_t slot;
             if (!ring_acquire(p, ctl, ring, bytes, (uint32_t)id, slot)) { ok = false; break; }
             if (bytes) bulk_g2s_hint(pages + (size_t)slot * kPageBytes, g.src, bytes, &ctl->full[slot], wpol);
@@ -539,8 +558,8 @@ __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     unsigned long long t_dep = 0;
     for (int qi = q0; qi < q1; ++qi) {
-        const int id = p.queue[qi];
-        const int dep = p.tasks[id].dep;
+        const int id = p.qtasks[qi].sm;
+        const int dep = p.qtasks[qi].dep;
         if (dep >= 0) {
             const uint32_t target = p.thresholds[dep] * ep;
             Spin s;
@@ -581,6 +600,7 @@ struct WState {
     uint32_t need = 0;       // ready_upto value that activates the current task
     uint32_t ep = 0;         // this launch's epoch: the tag of this step's activations
     uint32_t ep_out = 0;     // tag the current task stores (ep, or stale under the test hook)
+    const uint16_t *gain = nullptr;   // RMSNorm gain of the current task's input (null if none)
     int red_buf = 0;
     int task_id = 0;
     unsigned long long *stat = nullptr;   // per-phase accumulators in shared memory (trace mode, thread 0)
@@ -805,10 +825,10 @@ __device__ __forceinline__ bool stage_partials(const Params &p, SmemCtl *ctl, co
     return true;
 }
 
-// One tagged value per lane (lanes with `want`), polled by the whole warp.
+// One tagged value per lane (lanes with `want`), polled by the whole warp;
+// `v` is a first load the caller issued earlier.
 __device__ __forceinline__ bool warp_tag1(const Params &p, SmemCtl *ctl, const WState &w,
-                                          const uint64_t *src, bool want, float &out) {
-    uint64_t v = want ? ld_tag1(src) : 0ull;
+                                          const uint64_t *src, bool want, uint64_t v, float &out) {
     bool pend = want && !tag_ok(v, w.ep);
     Spin s;
     while (__any_sync(0xffffffffu, pend)) {
@@ -833,18 +853,18 @@ struct GemvInput {
     const uint16_t *gain;
 };
 
-__device__ __forceinline__ GemvInput gemv_input(const Params &p, int kind, int layer, int b) {
+__device__ __forceinline__ GemvInput gemv_input(const Params &p, const SmemCtl *ctl, const WState &w,
+                                                int kind, int layer, int b) {
     const Shape &s = p.s;
     const TagLayout &tl = p.tl;
-    GemvInput in{nullptr, nullptr, nullptr};
+    GemvInput in{nullptr, nullptr, w.gain};
     switch (kind) {
     case OP_QKV:
-        if (layer == 0) in.src_bf = p.embed + (size_t)p.tokens[b] * s.H;
+        if (layer == 0) in.src_bf = p.embed + (size_t)ctl->tok[b] * s.H;
         else in.src = tag_buf(p, layer - 1, tl.xb) + my_copy(tl.rep_h) + (size_t)b * s.H;
-        in.gain = p.layers[layer].g_attn;
         break;
-    case OP_GATEUP: in.src = tag_buf(p, layer, tl.xa) + my_copy(tl.rep_h) + (size_t)b * s.H; in.gain = p.layers[layer].g_mlp; break;
-    case OP_LMHEAD: in.src = tag_buf(p, s.L - 1, tl.xb) + my_copy(tl.rep_h) + (size_t)b * s.H; in.gain = p.g_final; break;
+    case OP_GATEUP: in.src = tag_buf(p, layer, tl.xa) + my_copy(tl.rep_h) + (size_t)b * s.H; break;
+    case OP_LMHEAD: in.src = tag_buf(p, s.L - 1, tl.xb) + my_copy(tl.rep_h) + (size_t)b * s.H; break;
     case OP_OPROJ: in.src = tag_buf(p, layer, tl.attn) + my_copy(tl.rep_qd) + (size_t)b * s.QD; break;
     default: in.src = tag_buf(p, layer, tl.act) + my_copy(tl.rep_f) + (size_t)b * s.F; break;
     }
@@ -1049,8 +1069,8 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     const int seg = warp % nseg;
     const int b = 0;
     const size_t row_bytes = (size_t)K8 * 16;          // one page row
-    const int P = p.positions[b];
-    const int tok = p.tokens[b];
+    const int P = ctl->pos[b];
+    const int tok = ctl->tok[b];
     // pair tiles: every GATEUP tile, and QKV tiles below npair
     const int npair = kind == OP_GATEUP ? 0x7fffffff
                     : kind == OP_QKV ? (s.nq + s.nkv) * s.d / 16 : 0;
@@ -1059,9 +1079,7 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     const int task_rows = 8 * (t.end - t.begin);
 
     // ---- before the dependency
-    const uint16_t *gain = kind == OP_QKV ? p.layers[layer].g_attn
-                         : kind == OP_GATEUP ? p.layers[layer].g_mlp
-                         : kind == OP_LMHEAD ? p.g_final : nullptr;
+    const uint16_t *gain = w.gain;
     float xr[NVL][8];
     uint4 gv[NVL];   // the RMSNorm gain slice, loaded before the dependency
     const bool embed_in = kind == OP_QKV && layer == 0;
@@ -1121,18 +1139,19 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
         // the activation: the worker threads copy the input vector into
         // ctl->stage together (tagged: waiting for this step's tags), meet,
         // and then every warp takes its part from there
-        const GemvInput in = gemv_input(p, kind, layer, b);
+        const GemvInput in = gemv_input(p, ctl, w, kind, layer, b);
+        // the residual word goes out first, so its round trip overlaps the
+        // input's: whole rows: lane L's of tile begin + L, row `warp`;
+        // segments: warp 0 lane L's of task row L
+        const bool resid_wait = resid_op && !(kind == OP_OPROJ && layer == 0) && (nseg == 1 || warp == 0);
+        const uint64_t *rsrc = resid_wait ? resid_in(p, kind, layer, b) + (nseg == 1 ? my_tile * 8 + warp : 8 * t.begin + lane)
+                                          : nullptr;
+        const bool rwant = resid_wait && (nseg == 1 ? my_tile < t.end : lane < task_rows);
+        const uint64_t rfirst = rwant ? ld_tag1(rsrc) : 0ull;
         float ss = 0.f;
         if (in.src_bf) stage_embed(ctl, in.src_bf, K, ss);
         else if (!(K <= kRowK ? stage_tagged<kRowK / 512>(p, ctl, w, in.src, K, ss) : stage_tagged<kStageFloats / 512>(p, ctl, w, in.src, K, ss))) return false;
-        if (resid_op && !(kind == OP_OPROJ && layer == 0)) {
-            const uint64_t *rs = resid_in(p, kind, layer, b);
-            if (nseg == 1) {
-                if (!warp_tag1(p, ctl, w, rs + my_tile * 8 + warp, my_tile < t.end, pre0)) return false;
-            } else if (warp == 0) {
-                if (!warp_tag1(p, ctl, w, rs + 8 * t.begin + lane, lane < task_rows, pre0)) return false;
-            }
-        }
+        if (resid_wait && !warp_tag1(p, ctl, w, rsrc, rwant, rfirst, pre0)) return false;
         ss = warp_sum(ss);
         if (lane == 0) ctl->scal[warp] = ss;
         if (!worker_sync(p, ctl, w)) return false;
@@ -1356,8 +1375,8 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
     const int b = 0;
     const int npair = kind == OP_GATEUP ? 0x7fffffff
                     : kind == OP_QKV ? (s.nq + s.nkv) * s.d / 16 : 0;
-    const int P = p.positions[b];
-    const int tok = p.tokens[b];
+    const int P = ctl->pos[b];
+    const int tok = ctl->tok[b];
     // residual of row 8 * begin + lane (warp 0), for the O / down projections
     const bool resid_op = kind == OP_OPROJ || kind == OP_DOWN;
     const int task_rows = 8 * (t.end - t.begin);
@@ -1366,7 +1385,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
         resid = bf2f(p.embed[(size_t)tok * s.H + 8 * t.begin + lane]);
     if (!wait_ready(p, ctl, w)) return false;
     unsigned long long tp = phase_begin(w);
-    const GemvInput in = gemv_input(p, kind, layer, b);
+    const GemvInput in = gemv_input(p, ctl, w, kind, layer, b);
     // thread tid takes 16-byte vectors tid, tid + 256, ... of the input: from
     // the embedding row, or as 4 tagged pairs each, stale pairs reloaded
     // until every tag is this step's
@@ -1438,9 +1457,11 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
             }
         }
     }
-    if (resid_op && !(kind == OP_OPROJ && layer == 0) && warp == 0 &&
-        !warp_tag1(p, ctl, w, resid_in(p, kind, layer, b) + 8 * t.begin + lane, lane < task_rows, resid))
-        return false;
+    if (resid_op && !(kind == OP_OPROJ && layer == 0) && warp == 0) {
+        const uint64_t *rsrc = resid_in(p, kind, layer, b) + 8 * t.begin + lane;
+        if (!warp_tag1(p, ctl, w, rsrc, lane < task_rows, lane < task_rows ? ld_tag1(rsrc) : 0ull, resid))
+            return false;
+    }
     float ss = 0.f;
 #pragma unroll
     for (int j = 0; j < NV; ++j)
@@ -1562,7 +1583,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     constexpr int NCH = D / 8;    // 16-byte chunks of a K row
     constexpr int KP = DPL / 2;   // tagged pairs of the new k (and v) per lane
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const AttnChunk a = attn_chunk(p, t.begin);
+    const AttnChunk a = attn_chunk(p, ctl, t.begin);
     const int npp = attn_pos_per_page(D);
     if (!wait_ready(p, ctl, w)) return false;
     unsigned long long tp = phase_begin(w);
@@ -1787,9 +1808,22 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
     }
     w.ep = ctl->ep;
     const unsigned long long t_begin = phase_begin(w);
+    // task records in queue order; the next one is loaded while the current
+    // one runs, so no task starts with a descriptor round trip
     for (int qi = q0; qi < q1; ++qi) {
-        const int id = p.queue[qi];
-        const Task t = p.tasks[id];
+        // the task's record, published by the loader (normally well ahead)
+        const int k = qi - q0;
+        {
+            Spin sr;
+            while (ld_acquire_cta_shared(&ctl->tq_pub) <= (uint32_t)k)
+                if (!spin_ok(sr, p, ctl, W_READY, 0xfffffffcu, (uint32_t)k)) return;
+        }
+        const TaskRec &rec = ctl->tq[k % kTaskRing];
+        const Task t = rec.t;
+        w.gain = rec.gain;
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) atomicAdd(&ctl->tq_reads, 1u);
+        const int id = t.sm;
         w.task_id = id;
         w.ep_out = t.trig == p.debug_withhold ? w.ep - 1u : w.ep;
         w.need = (uint32_t)(qi - q0 + 1);   // the task body waits for it
@@ -1880,8 +1914,13 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
         ctl->issued = 0;
         ctl->ep = ld_volatile_u32(p.epoch) + 1u;
         uint32_t stop = ld_volatile_u32(p.abort_flag) ? 1u : 0u;
+        ctl->tq_pub = 0;
+        ctl->tq_reads = 0;
+        for (int b = 0; b < kMaxBatch; ++b) { ctl->tok[b] = 0; ctl->pos[b] = 0; }
         for (int b = 0; b < p.batch && !stop; ++b) {
             const int tok = p.tokens[b], pos = p.positions[b];
+            ctl->tok[b] = tok;
+            ctl->pos[b] = pos;
             if (tok < 0 || tok >= p.s.V || pos < 0 || pos >= p.s.S) {
                 if (atomicCAS(&p.err->code, 0u, kErrInvalid) == 0u) {
                     p.err->task = 0xffffffffu;
@@ -1911,7 +1950,6 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
         } else if (warp == kSchedWarp) {
             if (lane == 0 && p.event_wait) scheduler_role(p, ctl, ctl->ep);
         } else if (warp == kSchedWarp + 1) {
-            if (p.l2_lookahead) prefetch_role(p, ctl);
         } else {
             if (lane == 0) signaler_role(p, ctl);
         }

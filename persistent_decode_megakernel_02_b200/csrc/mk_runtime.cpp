@@ -229,14 +229,13 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     Params &p = c->p;
     p.s = s;
     cudaError_t e = cudaSuccess;
-    Task *d_tasks; int32_t *d_queue, *d_qoff; uint32_t *d_thr, *d_ev, *d_ctrl;
+    Task *d_qtasks; int32_t *d_qoff; uint32_t *d_thr, *d_ev, *d_ctrl;
     LayerW *d_layers; float2 *d_rope;
     uint64_t *d_tag; float *d_aval; int32_t *d_aidx;
     const TagLayout tl = tag_layout(s);
     const size_t B = s.Bmax;
 #define MK_TRY(expr) do { e = (expr); if (e != cudaSuccess) { free_ctx(c); return map_cuda(e); } } while (0)
-    MK_TRY(dalloc(c, &d_tasks, c->num_tasks));
-    MK_TRY(dalloc(c, &d_queue, c->num_tasks));
+    MK_TRY(dalloc(c, &d_qtasks, c->num_tasks));
     MK_TRY(dalloc(c, &d_qoff, c->num_sms + 1));
     MK_TRY(dalloc(c, &d_thr, c->num_events));
     MK_TRY(dalloc(c, &d_ev, c->num_events));
@@ -284,8 +283,16 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     }
     MK_TRY(cudaDeviceSynchronize());
 
-    MK_TRY(cudaMemcpy(d_tasks, c->h_tasks.data(), sizeof(Task) * c->num_tasks, cudaMemcpyHostToDevice));
-    MK_TRY(cudaMemcpy(d_queue, c->h_queue.data(), sizeof(int32_t) * c->num_tasks, cudaMemcpyHostToDevice));
+    {
+        // the device reads the tasks in queue order, each record's `sm` field
+        // replaced by the task id (one load per task, no indirection)
+        std::vector<Task> qt(c->num_tasks);
+        for (int i = 0; i < c->num_tasks; ++i) {
+            qt[i] = c->h_tasks[c->h_queue[i]];
+            qt[i].sm = c->h_queue[i];
+        }
+        MK_TRY(cudaMemcpy(d_qtasks, qt.data(), sizeof(Task) * c->num_tasks, cudaMemcpyHostToDevice));
+    }
     MK_TRY(cudaMemcpy(d_qoff, c->h_qoff.data(), sizeof(int32_t) * (c->num_sms + 1), cudaMemcpyHostToDevice));
     MK_TRY(cudaMemcpy(d_thr, c->h_thresholds.data(), sizeof(uint32_t) * c->num_events, cudaMemcpyHostToDevice));
     MK_TRY(cudaMemcpy(d_layers, lw.data(), sizeof(LayerW) * s.L, cudaMemcpyHostToDevice));
@@ -308,7 +315,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     if (per_sm < 1) { free_ctx(c); return MK_ERR_INVALID; }
 #undef MK_TRY
 
-    p.tasks = d_tasks; p.queue = d_queue; p.qoff = d_qoff; p.thresholds = d_thr; p.events = d_ev;
+    p.qtasks = d_qtasks; p.qoff = d_qoff; p.thresholds = d_thr; p.events = d_ev;
     p.lm_cnt = d_ctrl + 0; p.epoch = d_ctrl + 1; p.done_cnt = d_ctrl + 2; p.abort_flag = d_ctrl + 3;
     p.num_lm_tasks = c->num_lm_tasks;
     p.layers = d_layers;

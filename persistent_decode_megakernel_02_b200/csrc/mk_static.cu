@@ -80,7 +80,7 @@ uint64_t shape_key(const mk_config *c, int num_sms) {
 }
 
 struct Layout {
-    size_t tasks, queue, qoff, thr, events, ctrl, err, tag, layers, rope;
+    size_t tasks, queue, qtasks, qoff, thr, events, ctrl, err, tag, layers, rope;
     size_t aval, aidx, end;
 };
 
@@ -118,6 +118,7 @@ Layout layout_for(const Shape &s, const PlanSizes &z, int num_sms, int num_lm_ta
     const size_t B = s.Bmax;
     l.tasks = take(sizeof(Task) * z.num_tasks);
     l.queue = take(sizeof(int32_t) * z.num_tasks);
+    l.qtasks = take(sizeof(Task) * z.num_tasks);
     l.qoff = take(sizeof(int32_t) * (num_sms + 1));
     l.thr = take(sizeof(uint32_t) * z.num_events);
     l.events = take(sizeof(uint32_t) * z.num_events);
@@ -210,6 +211,12 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
         plan.thresholds = reinterpret_cast<uint32_t *>(g_host + lay.thr);
         plan.bytes = nullptr;
         plan_build(s, ds.num_sms, plan);
+        // the device reads the tasks in queue order, `sm` holding the task id
+        Task *qt = reinterpret_cast<Task *>(g_host + lay.qtasks);
+        for (int i = 0; i < plan.num_tasks; ++i) {
+            qt[i] = plan.tasks[plan.queue[i]];
+            qt[i].sm = plan.queue[i];
+        }
         float2 *rope = reinterpret_cast<float2 *>(g_host + lay.rope);
         const int half = s.d / 2;
         for (int pos = 0; pos < s.S; ++pos)
@@ -244,8 +251,7 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
 
     Params p{};
     p.s = s;
-    p.tasks = reinterpret_cast<const Task *>(d + lay.tasks);
-    p.queue = reinterpret_cast<const int32_t *>(d + lay.queue);
+    p.qtasks = reinterpret_cast<const Task *>(d + lay.qtasks);
     p.qoff = reinterpret_cast<const int32_t *>(d + lay.qoff);
     p.thresholds = reinterpret_cast<const uint32_t *>(d + lay.thr);
     p.events = reinterpret_cast<uint32_t *>(d + lay.events);
