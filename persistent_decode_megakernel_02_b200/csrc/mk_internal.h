@@ -263,6 +263,12 @@ struct Params {
     int batch;
     float *logits;               // may be null
     int32_t *next_tok;
+    // generation (once-per-generation launch): n_steps decode steps back to
+    // back, each step's argmax the next step's token
+    int n_steps;                 // 1 for a single decode step
+    int32_t eos;                 // a sequence stops at its first eos (-1: never)
+    int32_t *tokens_out;         // [n_steps][batch] generated tokens (null: single step)
+    uint64_t *tok_tag;           // [Bmax][2] tagged words: next step's token, sequence done
     // scratch
     uint64_t *tag;               // [L][TagLayout::layer] tagged activations
     TagLayout tl;

@@ -240,8 +240,10 @@ struct __align__(16) SmemCtl {
     uint32_t loader_done;       // the loader has issued its last page
     uint32_t tq_pub;            // task records published by the loader
     uint32_t tq_reads;          // worker warps done reading a record (8 per task)
-    int32_t tok[kMaxBatch];     // this launch's tokens and positions, read once
-    int32_t pos[kMaxBatch];
+    int32_t tok[kMaxBatch];     // the workers' current step's tokens (first step: read once)
+    int32_t pos[kMaxBatch];     // the first step's positions (step s runs at pos + s)
+    int32_t wstep;              // the workers' current step
+    uint32_t stop;              // generation ended early: every role leaves its loop
     TaskRec tq[kTaskRing];      // records of the next tasks of this queue
     long long issued;           // GEMV bytes the loader has issued into the ring
     uint32_t sig_post;          // task completions posted by the workers
@@ -290,6 +292,7 @@ __device__ __forceinline__ bool spin_ok(Spin &s, const Params &p, SmemCtl *ctl, 
                                         uint32_t task, uint32_t info) {
     if ((++s.n & 127u) != 0u) return true;
     if (*(volatile uint32_t *)&ctl->abort) return false;
+    if (*(volatile uint32_t *)&ctl->stop) return false;
     if (ld_volatile_u32(p.abort_flag)) {
         *(volatile uint32_t *)&ctl->abort = 1;
         return false;
@@ -357,7 +360,7 @@ struct AttnChunk {
     int nc;           // chunks with positions for this sequence (the others are empty)
 };
 
-__device__ __forceinline__ AttnChunk attn_chunk(const Params &p, const SmemCtl *ctl, int item) {
+__device__ __forceinline__ AttnChunk attn_chunk(const Params &p, const SmemCtl *ctl, int step, int item) {
     const Shape &s = p.s;
     AttnChunk a;
     a.b = item / (s.nq * s.NC);
@@ -367,7 +370,7 @@ __device__ __forceinline__ AttnChunk attn_chunk(const Params &p, const SmemCtl *
     a.active = a.b < p.batch;
     a.P = 0; a.c0 = 0; a.c1 = 0; a.npre = 0; a.has_new = false; a.nc = 0;
     if (a.active) {
-        a.P = ctl->pos[a.b];
+        a.P = ctl->pos[a.b] + step;
         int C = a.P + 1;
         // at most NC chunks, but no fewer than kAttnChunkPositions positions
         // per chunk: short contexts use one chunk (nothing to merge)
@@ -457,15 +460,17 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
     // L2 prefetch cursor: GEMV weight bytes of the queue, bulk-prefetched
     // into L2 up to l2_lookahead bytes beyond what the ring has taken, so
     // HBM keeps streaming while the ring is full (one instruction per 64 KB)
-    int pf_qi = q0 - 1;
+    const int qlen = q1 - q0;
+    const long long pf_end = (long long)qlen * p.n_steps;   // queue positions over all steps
+    long long pf_k = -1;
     const char *pf_src = nullptr;
     long long pf_left = 0, pf_done = 0;
     auto prefetch_to = [&](long long target) {
         while (pf_done < target) {
             if (pf_left <= 0) {
-                do { ++pf_qi; } while (pf_qi < q1 && p.qtasks[pf_qi].kind == OP_ATTN);
-                if (pf_qi >= q1) { pf_done = 0x7fffffffffffffffLL; return; }
-                const GemvStream g = gemv_stream(p, p.qtasks[pf_qi]);
+                do { ++pf_k; } while (pf_k < pf_end && p.qtasks[q0 + pf_k % qlen].kind == OP_ATTN);
+                if (pf_k >= pf_end) { pf_done = 0x7fffffffffffffffLL; return; }
+                const GemvStream g = gemv_stream(p, p.qtasks[q0 + pf_k % qlen]);
                 pf_src = g.src;
                 pf_left = g.left;
                 continue;
@@ -477,13 +482,15 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
             pf_done += n;
         }
     };
+    for (int step = 0; step < p.n_steps && ok; ++step)
     for (int qi = q0; qi < q1 && ok; ++qi) {
+        if (*(volatile uint32_t *)&ctl->stop) { ok = false; break; }   // generation ended
         const Task t = p.qtasks[qi];
         const int id = t.sm;
         {
             // publish the task's record to the workers (ring of kTaskRing:
             // wait until every warp has read the record this slot held)
-            const int k = qi - q0;
+            const int k = step * qlen + (qi - q0);
             Spin sr;
             while (k >= kTaskRing &&
                    *(volatile uint32_t *)&ctl->tq_reads < (uint32_t)kWorkerWarps * (uint32_t)(k - kTaskRing + 1))
@@ -497,7 +504,7 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
             st_release_cta_shared(&ctl->tq_pub, (uint32_t)(k + 1));
         }
         if (t.kind == OP_ATTN) {
-            const AttnChunk a = attn_chunk(p, ctl, t.begin);
+            const AttnChunk a = attn_chunk(p, ctl, step, t.begin);
             const int npp = attn_pos_per_page(p.s.d);
             const LayerW &L = p.layers[t.layer];
             const size_t head_off = ((size_t)a.b * p.s.nkv + a.kvh) * p.s.S;
@@ -557,11 +564,13 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
 __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     unsigned long long t_dep = 0;
+    const int qlen = q1 - q0;
+    for (int step = 0; step < p.n_steps; ++step)
     for (int qi = q0; qi < q1; ++qi) {
         const int id = p.qtasks[qi].sm;
         const int dep = p.qtasks[qi].dep;
         if (dep >= 0) {
-            const uint32_t target = p.thresholds[dep] * ep;
+            const uint32_t target = p.thresholds[dep] * (ep + (uint32_t)step);
             Spin s;
             const unsigned long long t0 = p.sm_stats ? globaltimer() : 0ull;
             while ((int32_t)(ld_acquire_gpu(&p.events[dep]) - target) < 0)
@@ -569,7 +578,7 @@ __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
             if (p.sm_stats) t_dep += globaltimer() - t0;
         }
         if (p.trace) p.trace[id].t_ready = globaltimer();
-        st_release_cta_shared(&ctl->ready_upto, (uint32_t)(qi - q0 + 1));
+        st_release_cta_shared(&ctl->ready_upto, (uint32_t)(step * qlen + qi - q0 + 1));
     }
     if (p.sm_stats) p.sm_stats[(size_t)blockIdx.x * kStatSlots + ST_SCHED_DEP] = t_dep;
 }
@@ -578,7 +587,7 @@ __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
 // shared-memory ring (after the barrier that ends the task), this thread
 // performs the gpu-scope release add, so no worker stalls on the release.
 __device__ void signaler_role(const Params &p, SmemCtl *ctl) {
-    const uint32_t total = (uint32_t)(p.qoff[blockIdx.x + 1] - p.qoff[blockIdx.x]);
+    const uint32_t total = (uint32_t)(p.qoff[blockIdx.x + 1] - p.qoff[blockIdx.x]) * (uint32_t)p.n_steps;
     uint32_t done = 0;
     while (done < total) {
         Spin s;
@@ -1069,7 +1078,7 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     const int seg = warp % nseg;
     const int b = 0;
     const size_t row_bytes = (size_t)K8 * 16;          // one page row
-    const int P = ctl->pos[b];
+    const int P = ctl->pos[b] + ctl->wstep;
     const int tok = ctl->tok[b];
     // pair tiles: every GATEUP tile, and QKV tiles below npair
     const int npair = kind == OP_GATEUP ? 0x7fffffff
@@ -1375,7 +1384,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
     const int b = 0;
     const int npair = kind == OP_GATEUP ? 0x7fffffff
                     : kind == OP_QKV ? (s.nq + s.nkv) * s.d / 16 : 0;
-    const int P = ctl->pos[b];
+    const int P = ctl->pos[b] + ctl->wstep;
     const int tok = ctl->tok[b];
     // residual of row 8 * begin + lane (warp 0), for the O / down projections
     const bool resid_op = kind == OP_OPROJ || kind == OP_DOWN;
@@ -1583,7 +1592,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     constexpr int NCH = D / 8;    // 16-byte chunks of a K row
     constexpr int KP = DPL / 2;   // tagged pairs of the new k (and v) per lane
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const AttnChunk a = attn_chunk(p, ctl, t.begin);
+    const AttnChunk a = attn_chunk(p, ctl, ctl->wstep, t.begin);
     const int npp = attn_pos_per_page(D);
     if (!wait_ready(p, ctl, w)) return false;
     unsigned long long tp = phase_begin(w);
@@ -1798,21 +1807,84 @@ __device__ bool run_task(const Params &p, const Task &t, unsigned char *pages, S
     return gemv_cols<kMaxK / 2048>(p, t, pages, ctl, w);
 }
 
+// The last LM-head task of a step (warp 0 of its CTA): reduce the tasks'
+// partial argmaxes to each sequence's next token; when generating, record
+// it and publish the next step's input token (and whether the sequence is
+// done) as tagged words.  Kept out of line: it runs once per step.
+__device__ __noinline__ bool lm_reduce(const Params &p, SmemCtl *ctl, int step, uint32_t ep, int task_id) {
+    const int tid = threadIdx.x;
+    __threadfence();
+    int nxt[kMaxBatch] = {};
+    bool all_done = true;
+    for (int b = 0; b < p.batch; ++b) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int k = tid; k < p.num_lm_tasks; k += 32) {
+            const float v = __ldcg(p.amax_val + (size_t)b * p.num_lm_tasks + k);
+            const int i = __ldcg(p.amax_idx + (size_t)b * p.num_lm_tasks + k);
+            if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        if (tid == 0) {
+            p.next_tok[b] = bi;
+            nxt[b] = bi;
+            if (p.tokens_out) {
+                // a sequence that produced eos earlier keeps reporting eos
+                const bool done_before =
+                    step > 0 && __float_as_int(wait_tag1(p, ctl, p.tok_tag + 2 * b + 1, ep,
+                                                         (uint32_t)task_id)) != 0;
+                const bool done = done_before || (p.eos >= 0 && bi == p.eos);
+                p.tokens_out[(size_t)step * p.batch + b] = done_before ? p.eos : bi;
+                all_done = all_done && done;
+                if (step + 1 < p.n_steps)
+                    st_tag(p.tok_tag + 2 * b + 1, __int_as_float(done ? 1 : 0), ep + 1u);
+            }
+        }
+    }
+    if (tid == 0 && p.tokens_out && step + 1 < p.n_steps)
+        for (int b = 0; b < p.batch; ++b)
+            st_tag(p.tok_tag + 2 * b, __int_as_float(all_done ? -1 : nxt[b]), ep + 1u);
+    return true;
+}
+
 __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
+    const int qlen = q1 - q0;
     const int tid = threadIdx.x;
     WState w;
     if (p.sm_stats && tid == 0) {
         w.stat = ctl->wstat;
         for (int i = 0; i < kWStats; ++i) ctl->wstat[i] = 0;
     }
-    w.ep = ctl->ep;
     const unsigned long long t_begin = phase_begin(w);
-    // task records in queue order; the next one is loaded while the current
-    // one runs, so no task starts with a descriptor round trip
+    for (int step = 0; step < p.n_steps; ++step) {
+        w.ep = ctl->ep + (uint32_t)step;
+        if (step > 0) {
+            // this step's tokens: the previous step's argmax, published as
+            // tagged words by the task that reduced it (-1: generation over);
+            // warp 0 takes them into shared memory, the barrier publishes them
+            if (tid < 32) {
+                for (int b = 0; b < p.batch; ++b) {
+                    float v;
+                    if (!warp_tag1(p, ctl, w, p.tok_tag + 2 * b, true, ld_tag1(p.tok_tag + 2 * b), v)) return;
+                    if (tid == 0) {
+                        ctl->tok[b] = __float_as_int(v);
+                        if (__float_as_int(v) < 0) *(volatile uint32_t *)&ctl->stop = 1u;
+                    }
+                }
+                if (tid == 0) ctl->wstep = step;
+            }
+            if (!worker_sync(p, ctl, w)) return;
+            if (*(volatile uint32_t *)&ctl->stop) break;
+        }
     for (int qi = q0; qi < q1; ++qi) {
         // the task's record, published by the loader (normally well ahead)
-        const int k = qi - q0;
+        const int k = step * qlen + (qi - q0);
         {
             Spin sr;
             while (ld_acquire_cta_shared(&ctl->tq_pub) <= (uint32_t)k)
@@ -1826,7 +1898,7 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         const int id = t.sm;
         w.task_id = id;
         w.ep_out = t.trig == p.debug_withhold ? w.ep - 1u : w.ep;
-        w.need = (uint32_t)(qi - q0 + 1);   // the task body waits for it
+        w.need = (uint32_t)(k + 1);   // the task body waits for it (counter-gated mode)
         if (!run_task(p, t, pages, ctl, w)) return;
         const unsigned long long te = phase_begin(w);
         if (t.kind != OP_ATTN) {
@@ -1836,29 +1908,11 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
                 if (tid == 0) {
                     __threadfence();
                     const uint32_t old = atom_add_acqrel_gpu(p.lm_cnt, 1u);
-                    const uint32_t last = (old + 1u == (uint32_t)p.num_lm_tasks * ctl->ep) ? 1u : 0u;
+                    const uint32_t last = (old + 1u == (uint32_t)p.num_lm_tasks * w.ep) ? 1u : 0u;
                     ctl->last_flag = last;
                 }
                 if (!worker_sync(p, ctl, w)) return;
-                if (ctl->last_flag && tid < 32) {
-                    __threadfence();
-                    for (int b = 0; b < p.batch; ++b) {
-                        float bv = -INFINITY;
-                        int bi = 0x7fffffff;
-                        for (int k = tid; k < p.num_lm_tasks; k += 32) {
-                            const float v = __ldcg(p.amax_val + (size_t)b * p.num_lm_tasks + k);
-                            const int i = __ldcg(p.amax_idx + (size_t)b * p.num_lm_tasks + k);
-                            if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
-                        }
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) {
-                            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-                        }
-                        if (tid == 0) p.next_tok[b] = bi;
-                    }
-                }
+                if (ctl->last_flag && tid < 32 && !lm_reduce(p, ctl, step, w.ep, w.task_id)) return;
             }
             if (tid == 0) signal_event(p, ctl, t);
         }
@@ -1871,6 +1925,7 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         }
         phase_end(w, te, WS_END);
         if (w.stat) w.stat[WS_TASKS] += 1;
+    }
     }
     if (w.stat) {
         unsigned long long *st = p.sm_stats + (size_t)blockIdx.x * kStatSlots;
@@ -1916,12 +1971,14 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
         uint32_t stop = ld_volatile_u32(p.abort_flag) ? 1u : 0u;
         ctl->tq_pub = 0;
         ctl->tq_reads = 0;
+        ctl->stop = 0;
+        ctl->wstep = 0;
         for (int b = 0; b < kMaxBatch; ++b) { ctl->tok[b] = 0; ctl->pos[b] = 0; }
         for (int b = 0; b < p.batch && !stop; ++b) {
             const int tok = p.tokens[b], pos = p.positions[b];
             ctl->tok[b] = tok;
             ctl->pos[b] = pos;
-            if (tok < 0 || tok >= p.s.V || pos < 0 || pos >= p.s.S) {
+            if (tok < 0 || tok >= p.s.V || pos < 0 || pos > p.s.S - p.n_steps) {
                 if (atomicCAS(&p.err->code, 0u, kErrInvalid) == 0u) {
                     p.err->task = 0xffffffffu;
                     p.err->where = W_INPUT;
@@ -1935,10 +1992,12 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     __syncthreads();
     if (ctl->abort) return;   // nothing was started
     if (tid == 0) {
-        // the last CTA to read the epoch publishes it for the next launch
-        const uint32_t ep = ctl->ep;
-        const uint32_t old = atomicAdd(p.done_cnt, 1u);
-        if (old + 1u == gridDim.x * ep) atomicExch(p.epoch, ep);
+        // the last CTA to read the epoch publishes the launch's last step's
+        // epoch for the next launch (steps take epochs ep .. ep + n_steps - 1)
+        const uint32_t n = (uint32_t)p.n_steps;
+        const uint32_t ep_last = ctl->ep + n - 1u;
+        const uint32_t old = atomicAdd(p.done_cnt, n);
+        if (old + n == gridDim.x * ep_last) atomicExch(p.epoch, ep_last);
     }
     if (warp < kWorkerWarps) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kWorkerRegs));

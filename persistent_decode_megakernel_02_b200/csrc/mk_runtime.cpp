@@ -231,7 +231,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     cudaError_t e = cudaSuccess;
     Task *d_qtasks; int32_t *d_qoff; uint32_t *d_thr, *d_ev, *d_ctrl;
     LayerW *d_layers; float2 *d_rope;
-    uint64_t *d_tag; float *d_aval; int32_t *d_aidx;
+    uint64_t *d_tag, *d_toktag; float *d_aval; int32_t *d_aidx;
     const TagLayout tl = tag_layout(s);
     const size_t B = s.Bmax;
 #define MK_TRY(expr) do { e = (expr); if (e != cudaSuccess) { free_ctx(c); return map_cuda(e); } } while (0)
@@ -246,6 +246,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     MK_TRY(dalloc(c, &d_tag, tl.layer * s.L));
     MK_TRY(dalloc(c, &d_aval, B * c->num_lm_tasks));
     MK_TRY(dalloc(c, &d_aidx, B * c->num_lm_tasks));
+    MK_TRY(dalloc(c, &d_toktag, 2 * B));
     TraceRec *d_trace = nullptr;
     unsigned long long *d_stats = nullptr;
     if (cfg->flags & MK_FLAG_TRACE) {
@@ -301,6 +302,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     MK_TRY(cudaMemset(d_ctrl, 0, sizeof(uint32_t) * 8));
     MK_TRY(cudaMemset(c->d_err, 0, sizeof(ErrWord)));
     MK_TRY(cudaMemset(d_tag, 0, sizeof(uint64_t) * tl.layer * s.L));   // tag 0: never a step's
+    MK_TRY(cudaMemset(d_toktag, 0, sizeof(uint64_t) * 2 * B));
     if (d_trace) {
         std::vector<TraceRec> tr(c->num_tasks);
         for (int i = 0; i < c->num_tasks; ++i) {
@@ -324,6 +326,10 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     p.rope = d_rope;
     p.tag = d_tag; p.tl = tl;
     p.amax_val = d_aval; p.amax_idx = d_aidx;
+    p.tok_tag = d_toktag;
+    p.n_steps = 1;
+    p.eos = -1;
+    p.tokens_out = nullptr;
     p.err = c->d_err;
     p.trace = d_trace;
     p.sm_stats = d_stats;
@@ -358,6 +364,30 @@ int mk_decode_step(mk_ctx *c, const int32_t *tokens, const int32_t *positions, i
     return MK_OK;
 }
 
+int mk_generate(mk_ctx *c, const int32_t *tokens, const int32_t *positions, int batch, int n_steps,
+                int32_t eos, int32_t *tokens_out, int32_t *next_tok_out, mk_stream_t stream) {
+    if (!c) return MK_ERR_INVALID;
+    if (c->failed) return MK_ERR_STATE;
+    if (batch < 1 || batch > c->s.Bmax || n_steps < 1 || n_steps > c->s.S) return MK_ERR_INVALID;
+    if (!tokens || !positions || !tokens_out || !next_tok_out) return MK_ERR_INVALID;
+    if (((uintptr_t)tokens & 3u) || ((uintptr_t)positions & 3u) || ((uintptr_t)tokens_out & 3u) ||
+        ((uintptr_t)next_tok_out & 3u))
+        return MK_ERR_INVALID;
+    Params p = c->p;
+    p.tokens = tokens;
+    p.positions = positions;
+    p.batch = batch;
+    p.logits = nullptr;
+    p.next_tok = next_tok_out;
+    p.n_steps = n_steps;
+    p.eos = eos < 0 ? -1 : eos;
+    p.tokens_out = tokens_out;
+    cudaError_t e = kernel_launch(p, c->num_sms, (cudaStream_t)stream);
+    if (e != cudaSuccess) return MK_ERR_CUDA;
+    c->steps += n_steps;
+    return MK_OK;
+}
+
 int mk_sync(mk_ctx *c, mk_stream_t stream) {
     if (!c) return MK_ERR_INVALID;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MK_ERR_CUDA;
@@ -380,6 +410,7 @@ int mk_reset(mk_ctx *c) {
         // the epoch restarts at 0: tags written before the reset must not
         // pass for the next steps'
         cudaMemset(p.tag, 0, sizeof(uint64_t) * p.tl.layer * c->s.L) != cudaSuccess ||
+        cudaMemset(p.tok_tag, 0, sizeof(uint64_t) * 2 * c->s.Bmax) != cudaSuccess ||
         cudaMemcpy(const_cast<uint32_t *>(p.thresholds), c->h_thresholds.data(), sizeof(uint32_t) * c->num_events,
                    cudaMemcpyHostToDevice) != cudaSuccess)
         return MK_ERR_CUDA;

@@ -80,7 +80,7 @@ uint64_t shape_key(const mk_config *c, int num_sms) {
 }
 
 struct Layout {
-    size_t tasks, queue, qtasks, qoff, thr, events, ctrl, err, tag, layers, rope;
+    size_t tasks, queue, qtasks, qoff, thr, events, ctrl, err, tag, toktag, layers, rope;
     size_t aval, aidx, end;
 };
 
@@ -125,6 +125,7 @@ Layout layout_for(const Shape &s, const PlanSizes &z, int num_sms, int num_lm_ta
     l.ctrl = take(sizeof(uint32_t) * 8);
     l.err = take(sizeof(ErrWord));
     l.tag = take(sizeof(uint64_t) * tag_layout(s).layer * s.L);
+    l.toktag = take(sizeof(uint64_t) * 2 * B);
     l.layers = take(sizeof(LayerW) * s.L);
     l.rope = take(sizeof(float2) * (size_t)s.S * (s.d / 2));
     l.aval = take(sizeof(float) * B * num_lm_tasks);
@@ -272,6 +273,10 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
     p.logits = logits_out;
     p.next_tok = next_tok_out;
     p.tag = reinterpret_cast<uint64_t *>(d + lay.tag);
+    p.tok_tag = reinterpret_cast<uint64_t *>(d + lay.toktag);
+    p.n_steps = 1;
+    p.eos = -1;
+    p.tokens_out = nullptr;
     p.tl = tag_layout(s);
     p.amax_val = reinterpret_cast<float *>(d + lay.aval);
     p.amax_idx = reinterpret_cast<int32_t *>(d + lay.aidx);

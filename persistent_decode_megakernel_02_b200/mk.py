@@ -96,12 +96,13 @@ _lib.mk_get_sm_stats.argtypes = [_P, _P, C.c_int]
 _lib.mk_plan.argtypes = [C.POINTER(Config), C.c_int, C.POINTER(Info), _P, _P, _P, _P, _P]
 _lib.mk_debug_set_threshold.argtypes = [_P, C.c_int, C.c_uint]
 _lib.mk_debug_withhold_event.argtypes = [_P, C.c_int]
+_lib.mk_generate.argtypes = [_P, _P, _P, C.c_int, C.c_int, C.c_int, _P, _P, _P]
 _lib.mk_decode_step_static.argtypes = [C.POINTER(Config), C.POINTER(PackedWeights), C.POINTER(KV),
                                        _P, _P, C.c_int, _P, _P, _P, _P]
 for _f in ("mk_create", "mk_decode_step", "mk_sync", "mk_reset", "mk_destroy", "mk_get_info",
            "mk_get_event_counts", "mk_read_buffer", "mk_get_trace", "mk_get_graph", "mk_plan",
            "mk_get_sm_stats", "mk_decode_step_static",
-           "mk_debug_set_threshold", "mk_debug_withhold_event"):
+           "mk_debug_set_threshold", "mk_debug_withhold_event", "mk_generate"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -231,6 +232,16 @@ class Context:
         return _lib.mk_decode_step(self._h, _ptr(tokens), _ptr(positions), b,
                                    _ptr(logits) if logits is not None else None,
                                    _ptr(next_tok), _stream_ptr(stream))
+
+    def generate(self, tokens, positions, n_steps: int, tokens_out, next_tok, eos: int = -1,
+                 stream=None, batch=None):
+        """Enqueue `n_steps` greedy steps in one launch.  tokens/positions:
+        int32 CUDA tensors [batch] (first step's input); tokens_out: int32
+        CUDA tensor [n_steps][batch]; next_tok: int32 CUDA tensor [batch]."""
+        b = int(tokens.numel()) if batch is None else int(batch)
+        st = _lib.mk_generate(self._h, _ptr(tokens), _ptr(positions), b, int(n_steps), int(eos),
+                              _ptr(tokens_out), _ptr(next_tok), _stream_ptr(stream))
+        _check(st, "mk_generate")
 
     def sync(self, stream=None) -> int:
         return _lib.mk_sync(self._h, _stream_ptr(stream))
