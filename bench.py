@@ -15,7 +15,9 @@ the previous step wrote) at positions W..W+K-1.  Weights (2.47 GB for the
 `value` is device time per token (CUDA events over the K launches on the
 launching stream, max over ranks); `e2e` is the same through host buffers:
 per step the token and position are copied from pinned host memory, the
-step launched, and the next token copied back and waited for.
+step launched, and the next token copied back and waited for.  `generate`
+times the same K steps as ONE launch (mk_generate: the kernel runs the
+steps back to back, each step's argmax feeding the next on the device).
 
 Multi-GPU: every rank runs an independent replica (the single-sequence step
 does not shard without a per-layer exchange); `value` is then the max rank
@@ -206,6 +208,8 @@ def parse():
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-generate", action="store_true",
+                    help="skip the one-launch generation measurement")
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
     ap.add_argument("--flags", type=int, default=0, help="mk_config.flags")
@@ -368,6 +372,33 @@ def main():
         e2e = {"value": round(e2e_ms / (n * world), 5), "unit": UNIT, "h2d_bytes_per_step": 8,
                "d2h_bytes_per_step": 4, "steps": n}
 
+    # ---- the same K steps as one launch (mk_generate: each step's argmax
+    # feeds the next on the device; same positions, free-running tokens)
+    gen = None
+    if not args.no_generate:
+        g_out = torch.zeros(K, 1, dtype=torch.int32, device=dev)
+        g_next = torch.zeros(1, dtype=torch.int32, device=dev)
+        with torch.cuda.stream(stream):
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            g0 = torch.cuda.Event(enable_timing=True)
+            g1 = torch.cuda.Event(enable_timing=True)
+            g0.record(stream)
+            ctx.generate(toks[W:W + 1], pos[W:W + 1], K, g_out, g_next, stream=stream)
+            g1.record(stream)
+            stream.synchronize()
+            st = ctx.sync(stream)
+            if st != 0:
+                raise mk.MkError(st, "generate")
+            gen_ms = g0.elapsed_time(g1)
+        if world > 1:
+            t = torch.tensor([gen_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            gen_ms = float(t.item())
+        gen = {"value": round(gen_ms / (K * world), 5), "unit": UNIT, "steps": K, "launches": 1,
+               "api": "mk_generate"}
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -391,7 +422,7 @@ def main():
                "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
                "dtype": "bf16 weights/KV, fp32 accumulate", "data": "synthetic",
                "config": config, "roofline": roofline, "cpu_baseline": cpu,
-               "e2e": e2e, "gpu_launches": K, "clocks": clk.summary(),
+               "e2e": e2e, "generate": gen, "gpu_launches": K, "clocks": clk.summary(),
                "achieved_gbs": round(achieved, 1)}
         print(json.dumps(out), flush=True)
     ctx.close()
