@@ -168,28 +168,36 @@ int mk_decode_step(mk_ctx *ctx, const int32_t *tokens, const int32_t *positions,
                    float *logits_out, int32_t *next_tok_out, mk_stream_t stream);
 
 /*
- * Greedy generation in one launch (MPK's once-per-generation mode: the
- * persistent kernel keeps running while the tokens are produced, "显著提升
- * 小LLM的性能..." page, section on the decode loop and its step tensor).
- * Step 0 decodes tokens[b] at positions[b]; step s decodes step s-1's
- * argmax at positions[b] + s, writing each step's K/V slot.  The steps run
- * back to back inside the kernel: each step's argmax is published on the
- * device and feeds the next step's embedding, and the next step's weights
- * stream into shared memory while the current step's LM head finishes.
- *   tokens, positions  device int32 [batch]: the first step's input.
- *   n_steps            steps to run, 1..max_seq; positions[b] + n_steps
- *                      must not exceed max_seq (checked on the device:
+ * Prompt and greedy generation in one launch (MPK's once-per-generation
+ * mode: the persistent kernel keeps running while the tokens are produced,
+ * "显著提升小LLM的性能..." page, section on the decode loop and its step
+ * tensor).  Step s decodes one token per sequence at positions[b] + s,
+ * writing that K/V slot: for s < n_prompt the prompt's token tokens[s][b],
+ * afterwards step s-1's argmax.  The steps run back to back inside the
+ * kernel: each step's next token is published on the device and feeds the
+ * next step's embedding, and the next step's weights stream into shared
+ * memory while the current step's LM head finishes.  (The prompt is fed
+ * one token per step, like the decode steps, not as a multi-token
+ * contraction.)
+ *   tokens             device int32 [n_prompt][batch]: the prompt (n_prompt
+ *                      = 1: just the first step's token).
+ *   positions          device int32 [batch]: the first step's positions.
+ *   n_steps            steps to run, n_prompt..max_seq; positions[b] +
+ *                      n_steps must not exceed max_seq and every prompt
+ *                      token must lie in [0, vocab) (checked on the device:
  *                      MK_ERR_INVALID from mk_sync, nothing run).
- *   eos                a sequence stops at its first eos token (< 0: never);
- *                      once every sequence has stopped the launch ends.
+ *   eos                a sequence stops at the first eos it generates
+ *                      (steps >= n_prompt - 1; < 0: never); once every
+ *                      sequence has stopped the launch ends.
  *   tokens_out         device int32 [n_steps][batch]: step s's argmax for
- *                      sequence b (eos after the sequence stopped); entries
- *                      of steps not run (early stop) are left untouched.
+ *                      sequence b (eos after the sequence stopped); the
+ *                      generated tokens start at row n_prompt - 1; rows of
+ *                      steps not run (early stop) are left untouched.
  *   next_tok_out       device int32 [batch]: the last step's argmax.
  * Logits are not written.  Errors as for mk_decode_step.
  */
-int mk_generate(mk_ctx *ctx, const int32_t *tokens, const int32_t *positions, int batch, int n_steps,
-                int32_t eos, int32_t *tokens_out, int32_t *next_tok_out, mk_stream_t stream);
+int mk_generate(mk_ctx *ctx, const int32_t *tokens, int n_prompt, const int32_t *positions, int batch,
+                int n_steps, int32_t eos, int32_t *tokens_out, int32_t *next_tok_out, mk_stream_t stream);
 
 /* Wait for `stream`, then return the device status of the context
  * (MK_OK, MK_ERR_INVALID, MK_ERR_TIMEOUT) or MK_ERR_CUDA. */

@@ -266,6 +266,7 @@ struct Params {
     // generation (once-per-generation launch): n_steps decode steps back to
     // back, each step's argmax the next step's token
     int n_steps;                 // 1 for a single decode step
+    int n_prompt;                // steps 0 .. n_prompt-1 take their token from `tokens` ([n_prompt][batch])
     int32_t eos;                 // a sequence stops at its first eos (-1: never)
     int32_t *tokens_out;         // [n_steps][batch] generated tokens (null: single step)
     uint64_t *tok_tag;           // [Bmax][2] tagged words: next step's token, sequence done

@@ -1834,13 +1834,17 @@ __device__ __noinline__ bool lm_reduce(const Params &p, SmemCtl *ctl, int step, 
             p.next_tok[b] = bi;
             nxt[b] = bi;
             if (p.tokens_out) {
-                // a sequence that produced eos earlier keeps reporting eos
+                // while the prompt is fed the next token is the prompt's; after
+                // it, the argmax.  A sequence that produced eos keeps reporting
+                // eos (eos counts only once generation has begun)
+                const bool prompting = step + 1 < p.n_prompt;
                 const bool done_before =
                     step > 0 && __float_as_int(wait_tag1(p, ctl, p.tok_tag + 2 * b + 1, ep,
                                                          (uint32_t)task_id)) != 0;
-                const bool done = done_before || (p.eos >= 0 && bi == p.eos);
+                const bool done = done_before || (!prompting && p.eos >= 0 && bi == p.eos);
                 p.tokens_out[(size_t)step * p.batch + b] = done_before ? p.eos : bi;
                 all_done = all_done && done;
+                if (prompting) nxt[b] = p.tokens[(size_t)(step + 1) * p.batch + b];
                 if (step + 1 < p.n_steps)
                     st_tag(p.tok_tag + 2 * b + 1, __int_as_float(done ? 1 : 0), ep + 1u);
             }
@@ -1978,7 +1982,12 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
             const int tok = p.tokens[b], pos = p.positions[b];
             ctl->tok[b] = tok;
             ctl->pos[b] = pos;
-            if (tok < 0 || tok >= p.s.V || pos < 0 || pos > p.s.S - p.n_steps) {
+            bool bad = tok < 0 || tok >= p.s.V || pos < 0 || pos > p.s.S - p.n_steps;
+            for (int i = 1; i < p.n_prompt && !bad; ++i) {
+                const int ti = p.tokens[(size_t)i * p.batch + b];
+                bad = ti < 0 || ti >= p.s.V;
+            }
+            if (bad) {
                 if (atomicCAS(&p.err->code, 0u, kErrInvalid) == 0u) {
                     p.err->task = 0xffffffffu;
                     p.err->where = W_INPUT;

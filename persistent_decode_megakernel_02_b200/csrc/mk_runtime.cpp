@@ -328,6 +328,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     p.amax_val = d_aval; p.amax_idx = d_aidx;
     p.tok_tag = d_toktag;
     p.n_steps = 1;
+    p.n_prompt = 1;
     p.eos = -1;
     p.tokens_out = nullptr;
     p.err = c->d_err;
@@ -364,11 +365,12 @@ int mk_decode_step(mk_ctx *c, const int32_t *tokens, const int32_t *positions, i
     return MK_OK;
 }
 
-int mk_generate(mk_ctx *c, const int32_t *tokens, const int32_t *positions, int batch, int n_steps,
-                int32_t eos, int32_t *tokens_out, int32_t *next_tok_out, mk_stream_t stream) {
+int mk_generate(mk_ctx *c, const int32_t *tokens, int n_prompt, const int32_t *positions, int batch,
+                int n_steps, int32_t eos, int32_t *tokens_out, int32_t *next_tok_out, mk_stream_t stream) {
     if (!c) return MK_ERR_INVALID;
     if (c->failed) return MK_ERR_STATE;
     if (batch < 1 || batch > c->s.Bmax || n_steps < 1 || n_steps > c->s.S) return MK_ERR_INVALID;
+    if (n_prompt < 1 || n_prompt > n_steps) return MK_ERR_INVALID;
     if (!tokens || !positions || !tokens_out || !next_tok_out) return MK_ERR_INVALID;
     if (((uintptr_t)tokens & 3u) || ((uintptr_t)positions & 3u) || ((uintptr_t)tokens_out & 3u) ||
         ((uintptr_t)next_tok_out & 3u))
@@ -380,6 +382,7 @@ int mk_generate(mk_ctx *c, const int32_t *tokens, const int32_t *positions, int 
     p.logits = nullptr;
     p.next_tok = next_tok_out;
     p.n_steps = n_steps;
+    p.n_prompt = n_prompt;
     p.eos = eos < 0 ? -1 : eos;
     p.tokens_out = tokens_out;
     cudaError_t e = kernel_launch(p, c->num_sms, (cudaStream_t)stream);

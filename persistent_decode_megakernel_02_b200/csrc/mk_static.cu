@@ -275,6 +275,7 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
     p.tag = reinterpret_cast<uint64_t *>(d + lay.tag);
     p.tok_tag = reinterpret_cast<uint64_t *>(d + lay.toktag);
     p.n_steps = 1;
+    p.n_prompt = 1;
     p.eos = -1;
     p.tokens_out = nullptr;
     p.tl = tag_layout(s);

@@ -96,7 +96,7 @@ _lib.mk_get_sm_stats.argtypes = [_P, _P, C.c_int]
 _lib.mk_plan.argtypes = [C.POINTER(Config), C.c_int, C.POINTER(Info), _P, _P, _P, _P, _P]
 _lib.mk_debug_set_threshold.argtypes = [_P, C.c_int, C.c_uint]
 _lib.mk_debug_withhold_event.argtypes = [_P, C.c_int]
-_lib.mk_generate.argtypes = [_P, _P, _P, C.c_int, C.c_int, C.c_int, _P, _P, _P]
+_lib.mk_generate.argtypes = [_P, _P, C.c_int, _P, C.c_int, C.c_int, C.c_int, _P, _P, _P]
 _lib.mk_decode_step_static.argtypes = [C.POINTER(Config), C.POINTER(PackedWeights), C.POINTER(KV),
                                        _P, _P, C.c_int, _P, _P, _P, _P]
 for _f in ("mk_create", "mk_decode_step", "mk_sync", "mk_reset", "mk_destroy", "mk_get_info",
@@ -235,12 +235,14 @@ class Context:
 
     def generate(self, tokens, positions, n_steps: int, tokens_out, next_tok, eos: int = -1,
                  stream=None, batch=None):
-        """Enqueue `n_steps` greedy steps in one launch.  tokens/positions:
-        int32 CUDA tensors [batch] (first step's input); tokens_out: int32
-        CUDA tensor [n_steps][batch]; next_tok: int32 CUDA tensor [batch]."""
-        b = int(tokens.numel()) if batch is None else int(batch)
-        st = _lib.mk_generate(self._h, _ptr(tokens), _ptr(positions), b, int(n_steps), int(eos),
-                              _ptr(tokens_out), _ptr(next_tok), _stream_ptr(stream))
+        """Enqueue a prompt plus greedy steps, `n_steps` in all, in one launch.
+        tokens: int32 CUDA tensor [n_prompt][batch] (or [batch] for one
+        token); positions: int32 CUDA tensor [batch] (first step's);
+        tokens_out: int32 CUDA tensor [n_steps][batch]; next_tok: [batch]."""
+        b = int(positions.numel()) if batch is None else int(batch)
+        n_prompt = int(tokens.numel()) // b
+        st = _lib.mk_generate(self._h, _ptr(tokens), n_prompt, _ptr(positions), b, int(n_steps),
+                              int(eos), _ptr(tokens_out), _ptr(next_tok), _stream_ptr(stream))
         _check(st, "mk_generate")
 
     def sync(self, stream=None) -> int:

@@ -132,3 +132,51 @@ def test_llama1b_generate_equals_step_by_step():
         t, _ = b.gpu_step(t, pos0 + i, want_logits=False)
         steps.append(t)
     assert gen.tolist() == steps
+
+
+@pytest.mark.parametrize("flags", [0, 4])
+def test_prompt_and_generation_in_one_launch(flags):
+    """The prompt (teacher-forced) and the generation in ONE launch equal the
+    same sequence of single-step launches; every generated token is an
+    argmax of the oracle's logits."""
+    shape = wl.TINY
+    n_prompt, n_gen = 11, 13
+    n = n_prompt + n_gen - 1            # the last prompt step yields the first generated token
+    prompt = wl.make_prompt(shape.vocab, n_prompt, seed=77)
+    a = Pair(shape, max_seq=64, flags=flags)
+    b = Pair(shape, max_seq=64, flags=flags)
+    out = torch.full((n, 1), -7, dtype=torch.int32, device="cuda")
+    toks = torch.from_numpy(prompt.astype(np.int32)).cuda().view(n_prompt, 1)
+    a.pos.fill_(0)
+    a.ctx.generate(toks, a.pos, n, out, a.nxt)
+    assert a.ctx.sync() == 0
+    gen = out[:, 0].cpu().numpy()
+    # single steps: the prompt, then the argmax fed back
+    ref_argmax = []
+    t = int(prompt[0])
+    for s in range(n):
+        g, _ = b.gpu_step(t, s, want_logits=False)
+        ref_argmax.append(g)
+        t = int(prompt[s + 1]) if s + 1 < n_prompt else g
+    assert gen.tolist() == ref_argmax
+    for l in range(shape.layers):
+        assert torch.equal(a.k_gpu[l][0, :, :n], b.k_gpu[l][0, :, :n])
+    # the oracle, fed the prompt and then the GPU's tokens
+    t = int(prompt[0])
+    for s in range(n):
+        ref = a.ref_step(t, s)
+        if s >= n_prompt - 1:
+            assert token_ok(int(gen[s]), ref["logits"]), f"step {s}"
+        t = int(prompt[s + 1]) if s + 1 < n_prompt else int(gen[s])
+
+
+def test_prompt_token_out_of_range_is_refused():
+    shape = wl.TINY
+    a = Pair(shape, max_seq=32)
+    mk = a.mk
+    toks = torch.tensor([[1], [2], [shape.vocab]], dtype=torch.int32, device="cuda")
+    out = torch.zeros((6, 1), dtype=torch.int32, device="cuda")
+    a.pos.fill_(0)
+    a.ctx.generate(toks, a.pos, 6, out, a.nxt)
+    assert a.ctx.sync() == mk.MK_ERR_INVALID
+    a.ctx.reset()
