@@ -235,7 +235,8 @@ int mk_get_event_counts(mk_ctx *ctx, uint32_t *counts_out, uint32_t *thresholds_
 
 /* Scratch buffers readable after a step (host copy, blocks the host):
  * MK_BUF_HIDDEN float [max_batch][hidden] residual stream after the last
- * layer; MK_BUF_Q float [max_batch][nq*head_dim] last layer's rotated q;
+ * layer; MK_BUF_Q float [max_batch][nq*head_dim] last layer's q before RoPE
+ * (the attention tasks rotate it);
  * MK_BUF_ATTN float [max_batch][nq*head_dim] last layer's attention output;
  * MK_BUF_ACT float [max_batch][ffn] last layer's SiLU(gate)*up. */
 enum mk_buffer { MK_BUF_HIDDEN = 0, MK_BUF_Q = 1, MK_BUF_ATTN = 2, MK_BUF_ACT = 3 };
@@ -317,9 +318,7 @@ int mk_plan(const mk_config *cfg, int num_sms, mk_info *info,
  * Weights come already in the kernel's streaming layout (mk_create makes
  * this copy itself; this entry point cannot allocate one):
  *   qkv [layers] -> bf16 [(n_q_heads + 2*n_kv_heads)*head_dim][hidden]:
- *       for each q head, then each k head, head_dim/16 tiles of 16 rows
- *       (rows 8j..8j+7 of the head, then rows head_dim/2+8j..+7), then the
- *       n_kv_heads*head_dim value rows in their own order;
+ *       the wq rows, then the wk rows, then the wv rows (one buffer);
  *   gu  [layers] -> bf16 [2*ffn][hidden]: for each j < ffn/8, gate rows
  *       8j..8j+7 then up rows 8j..8j+7;
  *   the other members as in mk_weights.

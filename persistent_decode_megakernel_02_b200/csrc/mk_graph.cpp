@@ -34,7 +34,7 @@ PlanSizes plan_sizes(const Shape &s, int num_sms) {
     OpTiles t = op_tiles(s);
     auto ntask = [&](int tiles) { return tiles < num_sms ? tiles : num_sms; };
     PlanSizes z;
-    int per_layer = ntask(t.qkv_pair + t.qkv_v) + t.attn_items + ntask(t.oproj) +
+    int per_layer = ntask(t.qkv) + t.attn_items + ntask(t.oproj) +
                     ntask(t.gateup) + ntask(t.down);
     z.num_tasks = s.L * per_layer + ntask(t.lmhead);
     z.num_events = 5 * s.L + 1;
@@ -139,7 +139,7 @@ void plan_build(const Shape &s, int num_sms, Plan &p) {
     for (int l = 0; l < s.L; ++l) {
         int e_qkv = 5 * l, e_attn = e_qkv + 1, e_o = e_qkv + 2, e_gu = e_qkv + 3, e_down = e_qkv + 4;
         int dep_in = l == 0 ? -1 : e_qkv - 1;   // previous layer's down projection
-        p.thresholds[e_qkv] = b.gemv_op(OP_QKV, l, dep_in, e_qkv, t.qkv_pair + t.qkv_v);
+        p.thresholds[e_qkv] = b.gemv_op(OP_QKV, l, dep_in, e_qkv, t.qkv);
         p.thresholds[e_attn] = b.attn_op(l, e_qkv, e_attn);
         p.thresholds[e_o] = b.gemv_op(OP_OPROJ, l, e_attn, e_o, t.oproj);
         p.thresholds[e_gu] = b.gemv_op(OP_GATEUP, l, e_o, e_gu, t.gateup);

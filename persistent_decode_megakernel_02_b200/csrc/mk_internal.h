@@ -70,10 +70,9 @@ struct Task {
 static_assert(sizeof(Task) == 32, "Task is 8 int32");
 
 // Device pointers of one layer (bf16 as uint16_t on the host side).
-//  qkv: library-owned [(nq + 2 nkv) d][H] in QKV tile order: for every q
-//       head then every k head, d/8 tiles of 8 rows (4 rows of the first
-//       half of the head, then the 4 rows d/2 later that RoPE pairs them
-//       with), then the value rows in their own order.
+//  qkv: library-owned [(nq + 2 nkv) d][H]: the q rows, then the k rows,
+//       then the v rows (each in the caller's order), so a QKV task's
+//       rows are one contiguous range.
 //  gu:  library-owned [2F][H] in gate/up tile order: 4 gate rows, then the
 //       4 up rows with the same indices.
 //  wo, wd: the caller's matrices, read in place.
@@ -92,14 +91,13 @@ struct Shape {
 };
 
 // Tile counts of each op (identical on host and device).
-//  QKV:    (nq + nkv) * d / 16 "pair" tiles of 16 rows (8 rows of the first
-//          half of a head + the 8 rows d/2 later that RoPE pairs them with),
-//          then nkv * d / 8 value tiles of 8 rows
+//  QKV:    (nq + 2 nkv) * d / 8 tiles of 8 rows (q, then k, then v rows;
+//          RoPE is applied by the attention tasks, so no tile needs its
+//          rotation partner rows and 8-row tiles balance the SMs)
 //  GATEUP: F / 8 pair tiles of 16 rows (8 gate rows + the same 8 up rows)
 //  OPROJ, DOWN: H / 8 tiles of 8 rows; LMHEAD: ceil(V / 8) tiles of 8 rows
 struct OpTiles {
-    int qkv_pair;
-    int qkv_v;
+    int qkv;
     int oproj;
     int gateup;
     int down;
@@ -109,8 +107,7 @@ struct OpTiles {
 
 MK_HD inline OpTiles op_tiles(const Shape &s) {
     OpTiles t;
-    t.qkv_pair = (s.nq + s.nkv) * s.d / 16;
-    t.qkv_v = s.nkv * s.d / 8;
+    t.qkv = (s.QD + 2 * s.KD) / 8;
     t.oproj = s.H / 8;
     t.gateup = s.F / 8;
     t.down = s.H / 8;
@@ -127,12 +124,8 @@ MK_HD inline int op_k(const Shape &s, int kind) {
 // Row offset of tile `tile` in its op's weight buffer (rows of tiles are
 // contiguous and in tile order) -- also the rows of tiles [0, tile).
 MK_HD inline long long tile_row_offset(const Shape &s, int kind, int tile) {
-    if (kind == OP_GATEUP) return 16LL * tile;
-    if (kind == OP_QKV) {
-        const int np = (s.nq + s.nkv) * s.d / 16;
-        return tile <= np ? 16LL * tile : 16LL * np + 8LL * (tile - np);
-    }
-    return 8LL * tile;
+    (void)s;
+    return kind == OP_GATEUP ? 16LL * tile : 8LL * tile;
 }
 
 MK_HD inline int tile_rows(const Shape &s, int kind, int tile) {

@@ -26,11 +26,12 @@
 //
 // Task bodies (the fused instruction list of the Hazy megakernel page and
 // the per-layer *_layer calls of the MPK walkthrough, section 3.3.1):
-//   QKV    RMSNorm -> q/k/v GEMV rows -> RoPE -> q to scratch, k/v appended
-//          to the bf16 cache at the token's position
-//   ATTN   GQA decode attention over one chunk of positions of one KV head
-//          (split-K partial softmax); the last chunk to finish merges the
-//          partials of its KV head
+//   QKV    RMSNorm -> q/k/v GEMV rows -> q and k to scratch, v appended to
+//          the bf16 cache at the token's position
+//   ATTN   RoPE of q and of the new k (the group's first q head appends the
+//          rotated k to the cache) -> GQA decode attention of one q head over
+//          one chunk of positions (split-K partial softmax); chunk 0's task
+//          merges the partials when there are several chunks
 //   OPROJ  O-projection GEMV rows + residual
 //   GATEUP RMSNorm -> gate and up GEMV rows -> SiLU(gate) * up
 //   DOWN   down-projection GEMV rows + residual
@@ -897,59 +898,39 @@ __device__ __forceinline__ void scale_vec8(float *x, float sc, const uint16_t *g
     x[4] *= sc * bf_lo(g.z); x[5] *= sc * bf_hi(g.z); x[6] *= sc * bf_lo(g.w); x[7] *= sc * bf_hi(g.w);
 }
 
-// Outputs of a rotated q/k row pair (ra: row i of the head, rc: row i + d/2):
-// q goes to its tagged buffer; k is appended to the bf16 cache and, rounded
-// the same way, to the tagged new-key buffer the attention reads.
-__device__ __forceinline__ void qk_store(const Params &p, int layer, int head, int i, float ra, float rc,
-                                         int b, int P, uint32_t ep) {
+// Output row r of the fused q/k/v projection.  q and k rows go to their
+// tagged buffers as computed (the attention tasks apply RoPE and append the
+// rotated key to the cache); value rows are appended to the bf16 cache and,
+// rounded the same way, to the tagged new-value buffer.
+__device__ __forceinline__ void qkv_store_row(const Params &p, int layer, int r, float a, int b, int P,
+                                              uint32_t ep) {
     const Shape &s = p.s;
-    if (head < s.nq) {
-        uint64_t *qh = tag_buf(p, layer, p.tl.q) + (size_t)b * s.QD + (size_t)head * s.d;
-        st_tag(qh + i, ra, ep);
-        st_tag(qh + i + s.d / 2, rc, ep);
+    if (r < s.QD) {
+        st_tag(tag_buf(p, layer, p.tl.q) + (size_t)b * s.QD + r, a, ep);
+    } else if (r < s.QD + s.KD) {
+        st_tag(tag_buf(p, layer, p.tl.kn) + (size_t)b * s.KD + (r - s.QD), a, ep);
     } else {
-        const int kvh = head - s.nq;
-        uint16_t *kh = p.layers[layer].kc + (((size_t)b * s.nkv + kvh) * s.S + P) * s.d;
-        const uint16_t ka = f2bf(ra), kc = f2bf(rc);
-        kh[i] = ka;
-        kh[i + s.d / 2] = kc;
-        uint64_t *kn = tag_buf(p, layer, p.tl.kn) + (size_t)b * s.KD + (size_t)kvh * s.d;
-        st_tag(kn + i, bf2f(ka), ep);
-        st_tag(kn + i + s.d / 2, bf2f(kc), ep);
+        const int vr = r - s.QD - s.KD;
+        const int kvh = vr / s.d, dd = vr % s.d;
+        const uint16_t vb = f2bf(a);
+        p.layers[layer].vc[(((size_t)b * s.nkv + kvh) * s.S + P) * s.d + dd] = vb;
+        st_tag(tag_buf(p, layer, p.tl.vn) + (size_t)b * s.KD + vr, bf2f(vb), ep);
     }
 }
-// Value row vr (kv head vr / d, dim vr % d): cache append + tagged copy.
-__device__ __forceinline__ void v_store(const Params &p, int layer, int vr, float a, int b, int P, uint32_t ep) {
-    const Shape &s = p.s;
-    const int kvh = vr / s.d, dd = vr % s.d;
-    const uint16_t vb = f2bf(a);
-    p.layers[layer].vc[(((size_t)b * s.nkv + kvh) * s.S + P) * s.d + dd] = vb;
-    st_tag(tag_buf(p, layer, p.tl.vn) + (size_t)b * s.KD + vr, bf2f(vb), ep);
-}
 
-// Output of one finished row (or RoPE / gate-up pair) of the column-split
-// GEMV, written by one lane (the O and down projections are handled by the
-// caller, which owns the residual).
-//   a: the row's dot product (first-half row of a pair tile);
-//   c: the partner row's (second-half q/k row, or the up row), pair tiles only.
+// Output of one finished row (or gate/up pair) of a unit epilogue, written
+// by one lane (the O and down projections are handled by the caller, which
+// owns the residual).
+//   a: the row's dot product (the gate row of a pair tile);
+//   c: the up row's, pair tiles only.
 __device__ __forceinline__ void gemv_epilogue_row(const Params &p, int kind, int layer, int tile,
                                                   int r, float a, float c, int b, int P, uint32_t ep,
                                                   float &best_v, int &best_i) {
     const Shape &s = p.s;
     switch (kind) {
-    case OP_QKV: {
-        const int npair = (s.nq + s.nkv) * s.d / 16;
-        if (tile < npair) {
-            const int per_head = s.d / 16;
-            const int head = tile / per_head;
-            const int i = (tile % per_head) * 8 + r;
-            const float2 cs = p.rope[(size_t)P * (s.d / 2) + i];
-            qk_store(p, layer, head, i, a * cs.x - c * cs.y, c * cs.x + a * cs.y, b, P, ep);
-        } else {
-            v_store(p, layer, (tile - npair) * 8 + r, a, b, P, ep);
-        }
+    case OP_QKV:
+        qkv_store_row(p, layer, tile * 8 + r, a, b, P, ep);
         break;
-    }
     case OP_GATEUP:
         st_tag_rep(tag_buf(p, layer, p.tl.act) + (size_t)b * s.F + tile * 8 + r, p.tl.rep_f, a / (1.0f + expf(-a)) * c, ep);
         break;
@@ -1080,10 +1061,8 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     const size_t row_bytes = (size_t)K8 * 16;          // one page row
     const int P = ctl->pos[b] + ctl->wstep;
     const int tok = ctl->tok[b];
-    // pair tiles: every GATEUP tile, and QKV tiles below npair
-    const int npair = kind == OP_GATEUP ? 0x7fffffff
-                    : kind == OP_QKV ? (s.nq + s.nkv) * s.d / 16 : 0;
-    const int per_head = s.d / 16;
+    // pair tiles (8 gate + the 8 matching up rows): every GATEUP tile
+    const int npair = kind == OP_GATEUP ? 0x7fffffff : 0;
     const bool resid_op = kind == OP_OPROJ || kind == OP_DOWN;
     const int task_rows = 8 * (t.end - t.begin);
 
@@ -1107,14 +1086,8 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     // per-tile values.  Whole rows per warp: lane L holds those of tile
     // begin + L, row `warp`.  Segments: warp 0's lane L holds the residual of
     // task row L.
-    float pre0 = 0.f, pre1 = 0.f;
+    float pre0 = 0.f;
     const int my_tile = t.begin + lane;
-    if (nseg == 1 && kind == OP_QKV && my_tile < t.end && my_tile < npair) {
-        const int i = (my_tile % per_head) * 8 + warp;
-        const float2 cs = p.rope[(size_t)P * (s.d / 2) + i];
-        pre0 = cs.x;
-        pre1 = cs.y;
-    }
     if (kind == OP_OPROJ && layer == 0) {
         if (nseg == 1 && my_tile < t.end) pre0 = bf2f(p.embed[(size_t)tok * s.H + my_tile * 8 + warp]);
         if (nseg > 1 && warp == 0 && lane < task_rows) pre0 = bf2f(p.embed[(size_t)tok * s.H + 8 * t.begin + lane]);
@@ -1250,32 +1223,18 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
         const int my = (lane < 16 || pair) ? tile : tile + 1;
         const int off = my - t.begin;
         const float q0 = __shfl_sync(0xffffffffu, pre0, off & 31);
-        const float q1 = __shfl_sync(0xffffffffu, pre1, off & 31);
-        if (pair) {
+        if (pair) {   // gate/up: SiLU(gate) * up
             const float c = __shfl_sync(0xffffffffu, v, 16);
-            if (lane == 0) {
-                if (kind == OP_GATEUP) {
-                    st_tag_rep(tag_buf(p, layer, p.tl.act) + (size_t)b * s.F + tile * 8 + warp, p.tl.rep_f,
-                               v / (1.0f + expf(-v)) * c, w.ep_out);
-                } else {
-                    const int head = tile / per_head;
-                    const int i = (tile % per_head) * 8 + warp;
-                    float cs = q0, sn = q1;
-                    if (off >= 32) {
-                        const float2 r = p.rope[(size_t)P * (s.d / 2) + i];
-                        cs = r.x;
-                        sn = r.y;
-                    }
-                    qk_store(p, layer, head, i, v * cs - c * sn, c * cs + v * sn, b, P, w.ep_out);
-                }
-            }
+            if (lane == 0)
+                st_tag_rep(tag_buf(p, layer, p.tl.act) + (size_t)b * s.F + tile * 8 + warp, p.tl.rep_f,
+                           v / (1.0f + expf(-v)) * c, w.ep_out);
             tile += 1;
         } else {
             if ((lane == 0) || (lane == 16 && two)) {
                 const int row = my * 8 + warp;
                 switch (kind) {
                 case OP_QKV:
-                    v_store(p, layer, (my - npair) * 8 + warp, v, b, P, w.ep_out);
+                    qkv_store_row(p, layer, row, v, b, P, w.ep_out);
                     break;
                 case OP_OPROJ:
                 case OP_DOWN: {
@@ -1382,8 +1341,7 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
     const int rpp = rows_per_page(K);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = 0;
-    const int npair = kind == OP_GATEUP ? 0x7fffffff
-                    : kind == OP_QKV ? (s.nq + s.nkv) * s.d / 16 : 0;
+    const int npair = kind == OP_GATEUP ? 0x7fffffff : 0;   // gate/up pair tiles
     const int P = ctl->pos[b] + ctl->wstep;
     const int tok = ctl->tok[b];
     // residual of row 8 * begin + lane (warp 0), for the O / down projections
@@ -1599,8 +1557,9 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     const int npages = (a.npre + npp - 1) / npp;
     float *qs = ctl->stage + kWorkerWarps * kAttnCombine;   // q: chunk c (8 values) at qs + 12 c
 
-    // ---- q (threads 0 .. D/2-1, one pair each) and the new k / v (warp 0),
-    // tagged, polled until fresh
+    // ---- q (thread i < D/2 takes elements i and i + D/2, the pair RoPE
+    // rotates together) and the new k / v (warp 0), tagged, polled until
+    // fresh; RoPE at the token's position is applied here
     const bool new_warp = a.has_new && warp == 0;
     float kn[DPL], vn[DPL];
 #pragma unroll
@@ -1609,41 +1568,66 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
         const uint64_t *qsrc = tag_buf(p, t.layer, p.tl.q) + (size_t)a.b * s.QD + (size_t)a.h * D;
         const uint64_t *ksrc = tag_buf(p, t.layer, p.tl.kn) + (size_t)a.b * s.KD + (size_t)a.kvh * D + lane * DPL;
         const uint64_t *vsrc = tag_buf(p, t.layer, p.tl.vn) + (size_t)a.b * s.KD + (size_t)a.kvh * D + lane * DPL;
-        float2 qv = make_float2(0.f, 0.f);
+        float q_lo = 0.f, q_hi = 0.f;
         uint32_t pend = 0;
-        // bit 0: this thread's q pair; bits 1 .. KP: new k pairs; then new v pairs
+        // bits 0, 1: this thread's q elements i, i + D/2; bits 2 .. 1+KP: new
+        // k pairs; then new v pairs
         auto load = [&](int bit) {
-            ulonglong2 v;
-            if (bit == 0) {
-                v = ld_tag2(qsrc + 2 * tid);
-                qv = make_float2(tag_val(v.x), tag_val(v.y));
-            } else if (bit <= KP) {
-                v = ld_tag2(ksrc + 2 * (bit - 1));
-                kn[2 * (bit - 1)] = tag_val(v.x);
-                kn[2 * (bit - 1) + 1] = tag_val(v.y);
+            bool ok;
+            if (bit < 2) {
+                const uint64_t v = ld_tag1(qsrc + tid + (bit ? D / 2 : 0));
+                if (bit) q_hi = tag_val(v); else q_lo = tag_val(v);
+                ok = tag_ok(v, w.ep);
             } else {
-                v = ld_tag2(vsrc + 2 * (bit - 1 - KP));
-                vn[2 * (bit - 1 - KP)] = tag_val(v.x);
-                vn[2 * (bit - 1 - KP) + 1] = tag_val(v.y);
+                const bool isk = bit < 2 + KP;
+                const int h = isk ? bit - 2 : bit - 2 - KP;
+                const ulonglong2 v = ld_tag2((isk ? ksrc : vsrc) + 2 * h);
+                float *dst = isk ? kn : vn;
+                dst[2 * h] = tag_val(v.x);
+                dst[2 * h + 1] = tag_val(v.y);
+                ok = tag_ok(v.x, w.ep) && tag_ok(v.y, w.ep);
             }
-            if (tag_ok(v.x, w.ep) && tag_ok(v.y, w.ep)) pend &= ~(1u << bit);
+            if (ok) pend &= ~(1u << bit);
             else pend |= 1u << bit;
         };
 #pragma unroll
-        for (int bit = 0; bit <= 2 * KP; ++bit)
-            if ((bit == 0 && tid < D / 2) || (bit > 0 && new_warp)) load(bit);
+        for (int bit = 0; bit < 2 + 2 * KP; ++bit)
+            if ((bit < 2 && tid < D / 2) || (bit >= 2 && new_warp)) load(bit);
         Spin sp;
         while (__any_sync(0xffffffffu, pend != 0u)) {
             if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 4u)) return false;
 #pragma unroll
-            for (int bit = 0; bit <= 2 * KP; ++bit)
+            for (int bit = 0; bit < 2 + 2 * KP; ++bit)
                 if (pend & (1u << bit)) load(bit);
         }
         if (tid < D / 2) {
+            const float2 cs = p.rope[(size_t)a.P * (D / 2) + tid];
             const float scale = 1.0f / sqrtf((float)D);
-            const int e = 2 * tid;
-            qs[12 * (e >> 3) + (e & 7)] = qv.x * scale;
-            qs[12 * (e >> 3) + (e & 7) + 1] = qv.y * scale;
+            const int e = tid, f = tid + D / 2;
+            qs[12 * (e >> 3) + (e & 7)] = (q_lo * cs.x - q_hi * cs.y) * scale;
+            qs[12 * (f >> 3) + (f & 7)] = (q_hi * cs.x + q_lo * cs.y) * scale;
+        }
+        if (new_warp) {
+            // rotate the new key (lane L holds elements L*DPL..; the partner of
+            // an element sits D/2 further, i.e. in lane L ^ 16), round it to
+            // bf16 as the cache stores it; the group's first q head appends it
+            uint16_t kb[DPL];
+#pragma unroll
+            for (int j = 0; j < DPL; ++j) {
+                const float other = __shfl_xor_sync(0xffffffffu, kn[j], 16);
+                const int e = lane * DPL + j;
+                const int i = e % (D / 2);
+                const float2 cs = p.rope[(size_t)a.P * (D / 2) + i];
+                const float r = lane < 16 ? kn[j] * cs.x - other * cs.y : kn[j] * cs.x + other * cs.y;
+                kb[j] = f2bf(r);
+            }
+#pragma unroll
+            for (int j = 0; j < DPL; ++j) kn[j] = bf2f(kb[j]);
+            if (a.h % s.G == 0) {
+                uint16_t *kc = p.layers[t.layer].kc + (((size_t)a.b * s.nkv + a.kvh) * s.S + a.P) * D + lane * DPL;
+#pragma unroll
+                for (int j = 0; j < DPL; ++j) kc[j] = kb[j];
+            }
         }
     }
     if (!worker_sync(p, ctl, w)) return false;   // q visible to every warp

@@ -255,26 +255,19 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
         MK_TRY(cudaMemset(d_stats, 0, sizeof(unsigned long long) * c->num_sms * kStatSlots));
     }
 
-    // ---- repack q/k/v and gate/up into tile order (see LayerW / OpTiles)
+    // ---- q/k/v into one buffer, gate/up into tile order (see LayerW / OpTiles)
     {
         const size_t rb = 2 * (size_t)s.H;          // bytes of one row of K = H
-        const size_t tile = 16 * rb;                 // one pair tile
-        const int per_head = s.d / 16;               // pair tiles per head
+        const size_t tile = 16 * rb;                 // one gate/up pair tile
         for (int l = 0; l < s.L; ++l) {
             uint16_t *qkv, *gu;
             MK_TRY(dalloc(c, &qkv, (size_t)(s.QD + 2 * s.KD) * s.H));
             MK_TRY(dalloc(c, &gu, (size_t)2 * s.F * s.H));
             char *dq = (char *)qkv;
-            for (int h = 0; h < s.nq + s.nkv; ++h) {
-                const char *src = h < s.nq ? (const char *)w->wq[l] + (size_t)h * s.d * rb
-                                           : (const char *)w->wk[l] + (size_t)(h - s.nq) * s.d * rb;
-                char *dst = dq + (size_t)h * per_head * tile;
-                MK_TRY(cudaMemcpy2D(dst, tile, src, 8 * rb, 8 * rb, per_head, cudaMemcpyDeviceToDevice));
-                MK_TRY(cudaMemcpy2D(dst + 8 * rb, tile, src + (size_t)(s.d / 2) * rb, 8 * rb, 8 * rb,
-                                    per_head, cudaMemcpyDeviceToDevice));
-            }
-            MK_TRY(cudaMemcpy(dq + (size_t)(s.nq + s.nkv) * per_head * tile, w->wv[l],
-                              (size_t)s.KD * rb, cudaMemcpyDeviceToDevice));
+            MK_TRY(cudaMemcpy(dq, w->wq[l], (size_t)s.QD * rb, cudaMemcpyDeviceToDevice));
+            MK_TRY(cudaMemcpy(dq + (size_t)s.QD * rb, w->wk[l], (size_t)s.KD * rb, cudaMemcpyDeviceToDevice));
+            MK_TRY(cudaMemcpy(dq + (size_t)(s.QD + s.KD) * rb, w->wv[l], (size_t)s.KD * rb,
+                              cudaMemcpyDeviceToDevice));
             MK_TRY(cudaMemcpy2D(gu, tile, w->wg[l], 8 * rb, 8 * rb, s.F / 8, cudaMemcpyDeviceToDevice));
             MK_TRY(cudaMemcpy2D((char *)gu + 8 * rb, tile, w->wu[l], 8 * rb, 8 * rb, s.F / 8,
                                 cudaMemcpyDeviceToDevice));

@@ -36,9 +36,8 @@ def test_status_strings():
 
 def _tiles(shape):
     d, H, F, V = shape.head_dim, shape.hidden, shape.ffn, shape.vocab
-    # q/k tiles hold 8 RoPE pairs (16 rows), value tiles 8 rows, gate/up tiles
-    # 8 gate + 8 up rows, the others 8 rows
-    return {QKV: (shape.n_q_heads + shape.n_kv_heads) * d // 16 + shape.n_kv_heads * d // 8,
+    # q/k/v tiles 8 rows, gate/up tiles 8 gate + 8 up rows, the others 8 rows
+    return {QKV: (shape.n_q_heads + 2 * shape.n_kv_heads) * d // 8,
             OPROJ: H // 8, GATEUP: F // 8, DOWN: H // 8, LMHEAD: (V + 7) // 8}
 
 

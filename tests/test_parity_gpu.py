@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as orc
 from persistent_decode_megakernel_02_b200 import workloads as wl
 from harness import Pair, logit_tol, rel_l2, token_ok
 
@@ -68,6 +69,10 @@ def test_tiny_random_gains_untied_head_and_intermediates(flags):
     mk = pair.mk
     for buf, key in ((mk.MK_BUF_Q, "q"), (mk.MK_BUF_ATTN, "attn"), (mk.MK_BUF_ACT, "act")):
         got = pair.ctx.read_buffer(buf, ref[key].size).astype(np.float64)
+        if key == "q":   # the kernel keeps q before RoPE; rotate it per head like the oracle
+            d = shape.head_dim
+            got = np.concatenate([orc.rope(got[h * d:(h + 1) * d], pos, shape.rope_theta)
+                                  for h in range(shape.n_q_heads)])
         assert rel_l2(got, ref[key]) <= 5e-3, key
     _check_hidden(pair, ref)
 

@@ -25,11 +25,7 @@ def _pack(weights):
     H, d, F = s.hidden, s.head_dim, s.ffn
     qkv, gu = [], []
     for l in range(s.layers):
-        heads = torch.cat([weights.wq[l].view(s.n_q_heads, d, H), weights.wk[l].view(s.n_kv_heads, d, H)])
-        first = heads[:, : d // 2].reshape(heads.shape[0], d // 16, 8, H)
-        second = heads[:, d // 2:].reshape(heads.shape[0], d // 16, 8, H)
-        pairs = torch.stack([first, second], dim=2).reshape(-1, H)
-        qkv.append(torch.cat([pairs, weights.wv[l]]).contiguous())
+        qkv.append(torch.cat([weights.wq[l], weights.wk[l], weights.wv[l]]).contiguous())
         gu.append(torch.stack([weights.wg[l].view(F // 8, 8, H), weights.wu[l].view(F // 8, 8, H)],
                               dim=1).reshape(2 * F, H).contiguous())
     return {"embed": weights.embed, "lm_head": weights.lm_head, "final_norm": weights.final_norm,
