@@ -161,15 +161,14 @@ MK_HD inline int attn_pos_per_page(int d) { return kPageBytes / (4 * d); }
 // owns its own buffers (nothing is overwritten within a step), so a word's tag
 // is either this step's or an older one.
 // The vectors every SM reads whole (the two residual streams, the attention
-// output and SiLU(gate) * up) are written kReplicas times, and SM i reads
-// copy i % kReplicas: when 148 SMs read the same few hundred L2 lines at
-// once the lines' L2 slices serialise the requests; copies at different
-// addresses spread them over more slices.  Producers write a few hundred
-// words per task, so the extra stores cost little.
+// output and SiLU(gate) * up) can be written kReplicas times, SM i reading
+// copy i % kReplicas, so that the 148 readers spread over more L2 lines.
+// Measured: 8 copies are slower than one (the extra stores cost more than
+// the readers gain), so kReplicas is 1.
 //   xa: residual after the O-projection   [R][Bmax][H]
 //   xb: residual after the down projection [R][Bmax][H] (layer L-1: final hidden)
-//   q:  rotated queries                    [Bmax][nq * d]
-//   kn, vn: the new position's key (rotated) and value, rounded to bf16
+//   q:  queries before RoPE                [Bmax][nq * d]
+//   kn: the new position's key before RoPE; vn: its value rounded to bf16
 //                                          [Bmax][nkv * d]
 //   part: split-K attention partials, per q head and chunk o[d], m, l
 //                                          [Bmax][nq][NC][d + 2]
