@@ -42,7 +42,6 @@ constexpr int kNumPages = 3;        // pages in the per-SM ring
 constexpr int kVecMax = 7;          // 16-byte vectors per thread per row (K <= 7*8*256)
 constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 14336
 constexpr int kMaxBatch = 1;        // sequences per step (MK_MAX_BATCH)
-constexpr int kMaxGroup = 8;        // q heads per KV head
 // Attention chunking: a sequence's positions are split into at most NC
 // chunks of at least this many positions (shorter contexts use fewer chunks;
 // one chunk needs no merge).
@@ -50,7 +49,6 @@ constexpr int kAttnChunkPositions = 1024;
 constexpr int kMaxHeadDim = 256;
 constexpr long long kL2Lookahead = 0;  // default L2 prefetch distance beyond the ring (0: off; measured no gain)
 constexpr int kStageFloats = 8192;  // shared staging: a GEMV input vector, or attention partials
-constexpr int kL2Chunk = 64 * 1024;             // bytes per L2 prefetch instruction
 
 // ---- ops ---------------------------------------------------------------------
 enum OpKind : int32_t { OP_QKV = 0, OP_ATTN = 1, OP_OPROJ = 2, OP_GATEUP = 3, OP_DOWN = 4, OP_LMHEAD = 5 };

@@ -139,13 +139,6 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 __device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t *p) {
     return *(const volatile uint32_t *)p;
 }
-__device__ __forceinline__ uint4 ld_shared_v4(const void *p) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(smem_addr(p)));
-    return v;
-}
 // Tagged activation words: value bits low, step tag high, one 64-bit access
 // (single-copy atomic), so a reader that sees the tag sees the value.  The
 // loads are volatile (re-issued on every poll, kept in order among
@@ -246,14 +239,13 @@ struct __align__(16) SmemCtl {
     int32_t wstep;              // the workers' current step
     uint32_t stop;              // generation ended early: every role leaves its loop
     TaskRec tq[kTaskRing];      // records of the next tasks of this queue
-    long long issued;           // GEMV bytes the loader has issued into the ring
     uint32_t sig_post;          // task completions posted by the workers
     uint32_t sig_done;          // completions the signaler has published
     uint32_t sig_ev[kSigRing];  // event of each posted completion (ring)
     float red[2][kWorkerWarps][16];
     float scal[kWorkerWarps];
-    float att_m[kWorkerWarps][kMaxGroup];
-    float att_l[kWorkerWarps][kMaxGroup];
+    float att_m[kWorkerWarps][1];   // LM-head argmax: per-warp best value
+    float att_l[kWorkerWarps][1];   //   and its index (as float bits)
     // staging area: a row-per-warp GEMV task's input vector (read as
     // float4); an attention task's per-warp running outputs (kWorkerWarps x
     // kAttnCombine), later its merge inputs
@@ -531,7 +523,6 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
             g.src += g.page_bytes;
             g.left -= bytes;
             issued += bytes;
-            *(volatile long long *)&ctl->issued = issued;
         }
     }
     *(volatile uint32_t *)&ctl->loader_done = 1u;
@@ -686,31 +677,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
-}
-
-// Reduce acc[8] over the 32 lanes; afterwards every lane holds the warp
-// total of row (lane >> 2) & 7.
-__device__ __forceinline__ float warp_reduce_rows8(const float (&acc)[8], int lane) {
-    float b0[4], b1[2];
-    const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float send = u16 ? acc[i] : acc[i + 4];
-        float keep = u16 ? acc[i + 4] : acc[i];
-        b0[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        float send = u8 ? b0[i] : b0[i + 2];
-        float keep = u8 ? b0[i + 2] : b0[i];
-        b1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-    float send = u4 ? b1[0] : b1[1];
-    float keep = u4 ? b1[1] : b1[0];
-    float c = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    c += __shfl_xor_sync(0xffffffffu, c, 2);
-    c += __shfl_xor_sync(0xffffffffu, c, 1);
-    return c;
 }
 
 // Sum of one float over the 256 worker threads (bounded barrier inside).
@@ -1289,48 +1255,10 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     return true;
 }
 
-// Column split, for K > kRowK: thread t owns 16-byte vectors t, t+256, ...
-// of every row of a tile (up to RMAX rows: 8, or 16 for pair tiles); per
-// tile the partial sums are reduced across lanes, then across warps through
-// shared memory, and warp 0's lanes 0..7 run the epilogues.
-template <int RMAX>
-__device__ __forceinline__ float warp_reduce_rows(const float (&acc)[RMAX], int lane);
-
-template <>
-__device__ __forceinline__ float warp_reduce_rows<8>(const float (&acc)[8], int lane) {
-    return warp_reduce_rows8(acc, lane);   // lane holds row (lane >> 2) & 7
-}
-
-// 16 partial sums over 32 lanes; afterwards lane holds row (lane >> 1) & 15.
-template <>
-__device__ __forceinline__ float warp_reduce_rows<16>(const float (&acc)[16], int lane) {
-    float b0[8], b1[4], b2[2];
-    const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4, u2 = lane & 2;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float send = u16 ? acc[i] : acc[i + 8];
-        const float keep = u16 ? acc[i + 8] : acc[i];
-        b0[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float send = u8 ? b0[i] : b0[i + 4];
-        const float keep = u8 ? b0[i + 4] : b0[i];
-        b1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const float send = u4 ? b1[i] : b1[i + 2];
-        const float keep = u4 ? b1[i + 2] : b1[i];
-        b2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-    const float send = u2 ? b2[0] : b2[1];
-    const float keep = u2 ? b2[1] : b2[0];
-    float c = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-    c += __shfl_xor_sync(0xffffffffu, c, 1);
-    return c;
-}
-
+// Column split, for K other than 2048 * {1, 2, 4} (e.g. 14336): thread t
+// owns 16-byte vectors t, t+256, ... of every row; rows go two at a time,
+// each pair reduced across the warp and parked in shared memory, one
+// cross-warp sum per 16-row unit, and warp 0 runs the unit's epilogue.
 template <int NV>
 __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                           WState &w) {
@@ -1954,7 +1882,6 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
         ctl->ready_upto = 0;
         ctl->last_flag = 0;
         ctl->loader_done = 0;
-        ctl->issued = 0;
         ctl->ep = ld_volatile_u32(p.epoch) + 1u;
         uint32_t stop = ld_volatile_u32(p.abort_flag) ? 1u : 0u;
         ctl->tq_pub = 0;
