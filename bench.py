@@ -217,6 +217,24 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value: device times are taken as the max over
+    ranks (all ranks call this the same number of times, in the same order)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_ms_per_token(max_rank_ms: float, steps: int, world: int) -> float:
+    """Whole-job time per token: every rank decodes `steps` tokens of its own
+    replica in the slowest rank's time."""
+    return max_rank_ms / (steps * world)
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -312,12 +330,9 @@ def main():
         if st != 0:
             raise mk.MkError(st, "timed steps")
         dev_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([dev_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        dev_ms = float(t.item())
+    dev_ms = max_over_ranks(dev_ms, world, dev)
     per_launch_ms = dev_ms / K
-    value = dev_ms / (K * world)
+    value = job_ms_per_token(dev_ms, K, world)
 
     # ---- roofline of the kernel (the only kernel in the step)
     contexts = np.arange(start + W, start + W + K) + 1
@@ -365,11 +380,8 @@ def main():
             if st != 0:
                 raise mk.MkError(st, "e2e steps")
             e2e_ms = f0.elapsed_time(f1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": round(e2e_ms / (n * world), 5), "unit": UNIT, "h2d_bytes_per_step": 8,
+        e2e_ms = max_over_ranks(e2e_ms, world, dev)
+        e2e = {"value": round(job_ms_per_token(e2e_ms, n, world), 5), "unit": UNIT, "h2d_bytes_per_step": 8,
                "d2h_bytes_per_step": 4, "steps": n}
 
     # ---- the same K steps as one launch (mk_generate: each step's argmax
@@ -392,11 +404,8 @@ def main():
             if st != 0:
                 raise mk.MkError(st, "generate")
             gen_ms = g0.elapsed_time(g1)
-        if world > 1:
-            t = torch.tensor([gen_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            gen_ms = float(t.item())
-        gen = {"value": round(gen_ms / (K * world), 5), "unit": UNIT, "steps": K, "launches": 1,
+        gen_ms = max_over_ranks(gen_ms, world, dev)
+        gen = {"value": round(job_ms_per_token(gen_ms, K, world), 5), "unit": UNIT, "steps": K, "launches": 1,
                "api": "mk_generate"}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1)
