@@ -3,13 +3,16 @@
  *
  * One call of mk_decode_step runs the single-token decode step of a
  * Llama-style decoder for up to max_batch independent sequences as ONE
- * persistent kernel launch on a B200 (sm_100a).  Inside the launch, a static
- * task graph built by mk_create splits the rows of every matrix-vector op
- * into per-SM tasks; tasks wait on and bump event counters in global memory
- * (no grid-wide barrier between layers), a loader warp per SM streams the
- * weights of upcoming tasks into paged shared memory ahead of their
- * dependencies, a scheduler warp per SM activates tasks when their events
- * fire, and worker warps run the fused task bodies.
+ * persistent kernel launch on a B200 (sm_100a); mk_generate runs a prompt
+ * and a greedy generation in one launch.  Inside the launch, a static task
+ * graph built by mk_create splits the rows of every matrix-vector op into
+ * per-SM tasks, each bumping its op's event counter in global memory (no
+ * grid-wide barrier between layers).  A task starts when its inputs exist:
+ * by default the workers poll the step-tagged activation words they read;
+ * with MK_FLAG_EVENT_WAIT a scheduler warp per SM first waits for the
+ * dependency's counter to reach its threshold.  A loader warp per SM streams
+ * the weights of upcoming tasks into paged shared memory ahead of their
+ * dependencies, and worker warps run the fused task bodies.
  *
  * Where the operations are defined (reference pages on the persistent
  * decode megakernel topic):
@@ -62,7 +65,7 @@ enum mk_status {
 
 enum mk_flags {
     MK_FLAG_TRACE = 1,          /* record a per-task timing trace (globaltimer) */
-    MK_FLAG_NO_L2_PREFETCH = 2, /* loader does not prefetch ahead into L2     */
+    MK_FLAG_NO_L2_PREFETCH = 2, /* no L2 prefetch whatever l2_lookahead_kb says */
     /* Gate every task on its dependency's event counter (a scheduler warp
      * spins until counter >= threshold * epoch, the scheduling of MPK's
      * event model, "显著提升小LLM的性能..." page, Figure 3 text).  Without
@@ -74,20 +77,25 @@ enum mk_flags {
 
 /* Upper bounds of the shapes the kernel tiles. */
 #define MK_MAX_BATCH 1
-#define MK_MAX_K 14336      /* max of hidden, n_q_heads*head_dim and ffn */
-#define MK_MAX_HEAD_DIM 256
+#define MK_MAX_K 14336      /* max of n_q_heads*head_dim and ffn */
+#define MK_MAX_HIDDEN 4096
+#define MK_MAX_HEAD_DIM 128
 
 /*
  * Model shape and run options.
- *  hidden, ffn, n_q_heads*head_dim: multiples of 8, at most MK_MAX_K.
- *  head_dim: multiple of 8, at most MK_MAX_HEAD_DIM; n_kv_heads divides
- *  n_q_heads.  max_seq: KV capacity per sequence (positions 0..max_seq-1).
- *  max_batch: 1..MK_MAX_BATCH.  rms_eps > 0, rope_theta > 1.
- *  attn_chunks: split-K chunks per (sequence, KV head) in the attention
- *  op; 0 picks one chunk count so that the attention tasks cover the SMs.
+ *  hidden: multiple of 8, at most MK_MAX_HIDDEN; ffn, n_q_heads*head_dim:
+ *  multiples of 8, at most MK_MAX_K.  head_dim: 64 or 128; n_q_heads /
+ *  n_kv_heads: 1, 2, 4 or 8.  max_seq: KV capacity per sequence (positions
+ *  0..max_seq-1).  max_batch: 1..MK_MAX_BATCH.  rms_eps > 0, rope_theta > 1.
+ *  attn_chunks: most split-K chunks per (sequence, q head) in the
+ *  attention op (a step uses ceil(context / 1024) of them, so contexts up
+ *  to 1024 positions need no merge); 0 picks min(SMs / (max_batch *
+ *  n_q_heads), ceil(max_seq / 1024)).  At most 4096 and chunks * (head_dim
+ *  + 2) <= 8192.
  *  timeout_ns: bound on every device-side wait; 0 means 2 s.
- *  l2_lookahead_kb: how far (KiB of weights per SM) a prefetch warp runs
- *  ahead of the shared-memory ring into L2; 0 means no L2 prefetch.
+ *  l2_lookahead_kb: how far (KiB of weights per SM) the loader bulk-
+ *  prefetches into L2 beyond the pages it has copied into shared memory;
+ *  0 (the default) means none -- every distance measured slower.
  *  poll_ns: pause (ns) between two polls of a task's not yet ready input
  *  words; 0 polls back to back.
  */
@@ -203,8 +211,9 @@ int mk_generate(mk_ctx *ctx, const int32_t *tokens, int n_prompt, const int32_t 
  * (MK_OK, MK_ERR_INVALID, MK_ERR_TIMEOUT) or MK_ERR_CUDA. */
 int mk_sync(mk_ctx *ctx, mk_stream_t stream);
 
-/* Clear the device error state and the event counters (blocks the host;
- * no step may be in flight). */
+/* Clear the device error state, the event counters and the tagged
+ * activations, and restart the step count (blocks the host; no step may be
+ * in flight).  Also turns off the mk_debug_withhold_event hook. */
 int mk_reset(mk_ctx *ctx);
 
 /* Free the context's scratch (blocks the host).  NULL is accepted. */
@@ -222,7 +231,7 @@ typedef struct mk_info {
     int attn_chunks;
     int max_queue;      /* longest per-SM task queue */
     int page_bytes, num_pages;
-    long long steps_run; /* completed mk_decode_step launches since create/reset */
+    long long steps_run; /* decode steps enqueued since create/reset (mk_generate adds n_steps) */
     unsigned int err_code, err_info; /* device error word (0 = none) */
 } mk_info;
 
@@ -307,7 +316,8 @@ int mk_plan(const mk_config *cfg, int num_sms, mk_info *info,
  * counters, error word) lives in one fixed device array of
  * MK_STATIC_SCRATCH_BYTES that every GPU which loads the library holds
  * until the process exits.  Shapes whose scratch does not fit are rejected
- * with MK_ERR_INVALID (the 1B shape at max_seq 16640 uses about 5 MiB).
+ * with MK_ERR_INVALID (the 1B shape needs about 3.2 MiB at max_seq 560 and
+ * 8.0 MiB at max_seq 16640).
  * Every call shares that array and leaves its last contents there: calls
  * that overlap on the GPU (several streams or host threads) race.  The
  * first call on a device looks up the array's address and sets up the

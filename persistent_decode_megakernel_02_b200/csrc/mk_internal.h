@@ -135,7 +135,7 @@ MK_HD inline int tile_rows(const Shape &s, int kind, int tile) {
 // warp; other K split columns across all worker threads.
 constexpr int kRowK = 2048;
 MK_HD inline bool rows_gemv(int K) { return K <= kRowK || K == 2 * kRowK || K == 4 * kRowK; }
-constexpr int kMaxHidden = 4096;   // pair tiles in the column split hold 2 vectors per thread
+constexpr int kMaxHidden = 4096;   // MK_MAX_HIDDEN: the largest hidden size the tests cover
 
 // Rows of one page: the largest power of two <= 16 whose rows (K bf16 each)
 // fit in a page (16 for K <= 2048: one page holds a whole 16-row unit).

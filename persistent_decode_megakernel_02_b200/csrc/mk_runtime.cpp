@@ -65,6 +65,7 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     const int G = c->n_q_heads / c->n_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return MK_ERR_INVALID;
     if (c->head_dim != 64 && c->head_dim != 128) return MK_ERR_INVALID;
+    static_assert(kMaxHidden == MK_MAX_HIDDEN && kMaxK == MK_MAX_K, "public bounds match the kernel's");
     if (c->hidden > kMaxHidden) return MK_ERR_INVALID;
     const long long QD = (long long)c->n_q_heads * c->head_dim;
     if (c->hidden % 8 || c->ffn % 8 || QD % 8) return MK_ERR_INVALID;
