@@ -1585,6 +1585,19 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     stamp_input(p, w);
 
     const float *qh = qs + hg * QH;
+    // head_dim 64: the lane's q chunks held in registers in its rotated
+    // order (chunk (c + lane) mod NCH at qr[2c], qr[2c + 1]), so the score
+    // loop reads only K from shared memory; head_dim 128 reads q there
+    constexpr bool kQReg = D == 64;
+    float4 qr[kQReg ? 2 * NCH : 1];
+    if constexpr (kQReg) {
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int cc = (c + lane) & (NCH - 1);
+            qr[2 * c] = *reinterpret_cast<const float4 *>(qh + 12 * cc);
+            qr[2 * c + 1] = *reinterpret_cast<const float4 *>(qh + 12 * cc + 4);
+        }
+    }
     float m = -INFINITY, l = 0.f, o[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) o[i] = 0.f;
@@ -1600,19 +1613,27 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
             float sc = -INFINITY;
             if (j < n) {
                 const uint4 *krow = reinterpret_cast<const uint4 *>(Kp + (size_t)j * D);
-                float2 acc = make_float2(0.f, 0.f);
+                // two accumulators (even / odd chunks) halve the FMA chain
+                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int c = 0; c < NCH; ++c) {
                     const int cc = (c + lane) & (NCH - 1);
                     const uint4 kw = krow[cc];
-                    const float4 q0 = *reinterpret_cast<const float4 *>(qh + 12 * cc);
-                    const float4 q1 = *reinterpret_cast<const float4 *>(qh + 12 * cc + 4);
-                    acc = ffma2(make_float2(bf_lo(kw.x), bf_hi(kw.x)), make_float2(q0.x, q0.y), acc);
-                    acc = ffma2(make_float2(bf_lo(kw.y), bf_hi(kw.y)), make_float2(q0.z, q0.w), acc);
-                    acc = ffma2(make_float2(bf_lo(kw.z), bf_hi(kw.z)), make_float2(q1.x, q1.y), acc);
-                    acc = ffma2(make_float2(bf_lo(kw.w), bf_hi(kw.w)), make_float2(q1.z, q1.w), acc);
+                    float4 q0, q1;
+                    if constexpr (kQReg) {
+                        q0 = qr[2 * c];
+                        q1 = qr[2 * c + 1];
+                    } else {
+                        q0 = *reinterpret_cast<const float4 *>(qh + 12 * cc);
+                        q1 = *reinterpret_cast<const float4 *>(qh + 12 * cc + 4);
+                    }
+                    float2 &a2 = acc[c & 1];
+                    a2 = ffma2(make_float2(bf_lo(kw.x), bf_hi(kw.x)), make_float2(q0.x, q0.y), a2);
+                    a2 = ffma2(make_float2(bf_lo(kw.y), bf_hi(kw.y)), make_float2(q0.z, q0.w), a2);
+                    a2 = ffma2(make_float2(bf_lo(kw.z), bf_hi(kw.z)), make_float2(q1.x, q1.y), a2);
+                    a2 = ffma2(make_float2(bf_lo(kw.w), bf_hi(kw.w)), make_float2(q1.z, q1.w), a2);
                 }
-                sc = acc.x + acc.y;
+                sc = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
             }
             float mb = sc;
 #pragma unroll
@@ -1626,19 +1647,36 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
             m = mn;
             const int cnt = min(32, n - j0);
             const uint16_t *vb = Vp + (size_t)j0 * D + lane * DPL;
-            for (int k = 0; k < cnt; ++k) {
+            auto pv_step = [&](float *acc, int k) {
                 const float pk = __shfl_sync(0xffffffffu, pe, k);
                 if constexpr (DPL == 2) {
                     const uint32_t vw = *reinterpret_cast<const uint32_t *>(vb + (size_t)k * D);
-                    o[0] = fmaf(pk, bf_lo(vw), o[0]);
-                    o[1] = fmaf(pk, bf_hi(vw), o[1]);
+                    acc[0] = fmaf(pk, bf_lo(vw), acc[0]);
+                    acc[1] = fmaf(pk, bf_hi(vw), acc[1]);
                 } else {
                     const uint2 vw = *reinterpret_cast<const uint2 *>(vb + (size_t)k * D);
-                    o[0] = fmaf(pk, bf_lo(vw.x), o[0]);
-                    o[1] = fmaf(pk, bf_hi(vw.x), o[1]);
-                    o[2] = fmaf(pk, bf_lo(vw.y), o[2]);
-                    o[3] = fmaf(pk, bf_hi(vw.y), o[3]);
+                    acc[0] = fmaf(pk, bf_lo(vw.x), acc[0]);
+                    acc[1] = fmaf(pk, bf_hi(vw.x), acc[1]);
+                    acc[2] = fmaf(pk, bf_lo(vw.y), acc[2]);
+                    acc[3] = fmaf(pk, bf_hi(vw.y), acc[3]);
                 }
+            };
+            if (cnt == 32) {
+                // a full block: unrolled, so the shuffles and V loads of many
+                // positions are in flight together; even / odd positions go
+                // to two accumulators
+                float o2[DPL];
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) o2[i] = 0.f;
+#pragma unroll
+                for (int k = 0; k < 32; k += 2) {
+                    pv_step(o, k);
+                    pv_step(o2, k + 1);
+                }
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) o[i] += o2[i];
+            } else {
+                for (int k = 0; k < cnt; ++k) pv_step(o, k);
             }
         }
         release_page(ctl, w, slot);
