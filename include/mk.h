@@ -72,17 +72,7 @@ enum mk_flags {
      * it tasks wait on their inputs directly: every activation is stored
      * with the step's tag in the same 64-bit word and readers poll the tags.
      * Results are identical either way; the counters are bumped either way. */
-    MK_FLAG_EVENT_WAIT = 4,
-    /* Attention work items.  One item per (sequence, q head, chunk) streams
-     * its KV head's rows for that q head alone; one item per (sequence, KV
-     * head, chunk) streams them once and scores the KV head's whole group of
-     * q heads against them (GQA), so the cache is read once per step instead
-     * of n_q_heads / n_kv_heads times.  Without either flag: per KV head when
-     * max_seq > 4096 and the group fits (see attn_chunks), else per q head.
-     * Setting both is refused (MK_ERR_INVALID), as is PER_KVHEAD for a group
-     * that does not fit. */
-    MK_FLAG_ATTN_PER_QHEAD = 8,
-    MK_FLAG_ATTN_PER_KVHEAD = 16
+    MK_FLAG_EVENT_WAIT = 4
 };
 
 /* Upper bounds of the shapes the kernel tiles. */
@@ -97,15 +87,11 @@ enum mk_flags {
  *  multiples of 8, at most MK_MAX_K.  head_dim: 64 or 128; n_q_heads /
  *  n_kv_heads: 1, 2, 4 or 8.  max_seq: KV capacity per sequence (positions
  *  0..max_seq-1).  max_batch: 1..MK_MAX_BATCH.  rms_eps > 0, rope_theta > 1.
- *  attn_chunks: most split-K chunks per attention head in the attention
- *  op -- an attention head is a q head, or a KV head with its q heads (see
- *  MK_FLAG_ATTN_PER_KVHEAD; q heads per item: 1 or n_q_heads / n_kv_heads,
- *  and the latter needs (n_q_heads / n_kv_heads) * head_dim <= 512).  A step
- *  uses ceil(context / P) of them, P = 1024 / (q heads per item), so with
- *  an item per q head contexts up to 1024 positions need no merge.  0 picks
- *  min(SMs / (max_batch * heads), ceil(max_seq / P), 8192 / (q heads per
- *  item * (head_dim + 2))).  At most 4096 and q heads per item * chunks *
- *  (head_dim + 2) <= 8192.
+ *  attn_chunks: most split-K chunks per (sequence, q head) in the
+ *  attention op (a step uses ceil(context / 1024) of them, so contexts up
+ *  to 1024 positions need no merge); 0 picks min(SMs / (max_batch *
+ *  n_q_heads), ceil(max_seq / 1024)).  At most 4096 and chunks * (head_dim
+ *  + 2) <= 8192.
  *  timeout_ns: bound on every device-side wait; 0 means 2 s.
  *  l2_lookahead_kb: how far (KiB of weights per SM) the loader bulk-
  *  prefetches into L2 beyond the pages it has copied into shared memory;
@@ -247,7 +233,6 @@ typedef struct mk_info {
     int page_bytes, num_pages;
     long long steps_run; /* decode steps enqueued since create/reset (mk_generate adds n_steps) */
     unsigned int err_code, err_info; /* device error word (0 = none) */
-    int attn_q_heads;   /* q heads per attention work item: 1 or n_q_heads / n_kv_heads */
 } mk_info;
 
 int mk_get_info(mk_ctx *ctx, mk_info *out);

@@ -20,34 +20,14 @@ namespace mk {
 
 static constexpr int kMaxSms = 1024;
 
-// Chunks per attention head: enough items to give every SM one (items of
-// one chunk index: Bmax * nq / AG), no more than a full cache needs at
-// attn_chunk_positions per chunk, and few enough that one item's partials
-// (AG heads x chunks x (d + 2) floats) fit the merge's staging area.
-int default_attn_chunks(int num_sms, const Shape &s) {
-    int per = s.Bmax * (s.nq / s.AG);
+int default_attn_chunks(int num_sms, int Bmax, int nq, int S) {
+    int per = Bmax * nq;
     int nc = per > 0 ? num_sms / per : 1;
     if (nc < 1) nc = 1;
-    const int cp = attn_chunk_positions(s);
-    int cap = (s.S + cp - 1) / cp;   // chunks a full cache needs
+    int cap = (S + kAttnChunkPositions - 1) / kAttnChunkPositions;   // chunks a full cache needs
     if (cap < 1) cap = 1;
     if (nc > cap) nc = cap;
-    const int fit = kStageFloats / (s.AG * (s.d + 2));
-    if (nc > fit) nc = fit;
     return nc;
-}
-
-bool attn_geometry(Shape &s, int num_sms, bool force_qhead, bool force_kvhead, int attn_chunks) {
-    if (force_qhead && force_kvhead) return false;
-    const bool group_fits = s.G * s.d <= kAttnGroupElems;
-    if (force_kvhead && !group_fits) return false;
-    const bool per_kv = force_kvhead || (!force_qhead && group_fits && s.G > 1 && s.S > kAttnGroupMinSeq);
-    s.AG = per_kv ? s.G : 1;
-    s.NC = attn_chunks > 0 ? attn_chunks : default_attn_chunks(num_sms, s);
-    if (s.NC > 4096) return false;
-    // one item's chunk partials must fit the merge's shared staging area
-    if ((long long)s.AG * s.NC * (s.d + 2) > kStageFloats) return false;
-    return true;
 }
 
 PlanSizes plan_sizes(const Shape &s, int num_sms) {
@@ -123,15 +103,15 @@ struct Builder {
     // One task per attention item.  Items go to distinct SMs (the least
     // loaded ones) so an SM runs a second item of the same op only when
     // there are more items than SMs.
-    // Work items (sequence, attention head, chunk) in descending chunk order:
-    // chunk 0's task merges its head's partials and waits for the other chunks,
+    // Work items (sequence, KV head, chunk) in descending chunk order: chunk
+    // 0's task merges its KV head's partials and waits for the other chunks,
     // so on every queue it must come after any other chunk it could wait for
     // (the queues keep this order); chunks > 0 wait on nothing in the op.
     int attn_op(int layer, int dep, int trig) {
         OpTiles t = op_tiles(s);
         int per_chunk = (s.S + s.NC - 1) / s.NC;
         int64_t est = (int64_t)4 * s.d * per_chunk;   // K + V bf16 of one chunk at capacity
-        const int heads = s.Bmax * (s.nq / s.AG);     // items per chunk index
+        const int heads = s.Bmax * s.nq;              // items per chunk index
         for (int i = 0; i < t.attn_items; i += p.num_sms) {
             sort_by_load();
             int n = t.attn_items - i < p.num_sms ? t.attn_items - i : p.num_sms;

@@ -43,17 +43,9 @@ constexpr int kVecMax = 7;          // 16-byte vectors per thread per row (K <= 
 constexpr int kMaxK = kVecMax * 8 * kWorkerThreads;  // 14336
 constexpr int kMaxBatch = 1;        // sequences per step (MK_MAX_BATCH)
 // Attention chunking: a sequence's positions are split into at most NC
-// chunks of at least this many positions per q head the item covers
-// (shorter contexts use fewer chunks; one chunk needs no merge).
+// chunks of at least this many positions (shorter contexts use fewer chunks;
+// one chunk needs no merge).
 constexpr int kAttnChunkPositions = 1024;
-// An attention work item covers AG q heads: 1 (an item per q head) or the
-// G q heads that share a KV head (an item per KV head: its K/V rows are
-// read once for the whole group).  The group's q vectors and softmax
-// states must fit one item: AG * head_dim <= kAttnGroupElems.
-constexpr int kAttnGroupElems = 512;
-// Default: an item per KV head when the cache holds more than this many
-// positions per sequence, else an item per q head.
-constexpr int kAttnGroupMinSeq = 4096;
 constexpr int kMaxHeadDim = 256;
 constexpr long long kL2Lookahead = 0;  // default L2 prefetch distance beyond the ring (0: off; measured no gain)
 constexpr int kStageFloats = 8192;  // shared staging: a GEMV input vector, or attention partials
@@ -62,8 +54,7 @@ constexpr int kStageFloats = 8192;  // shared staging: a GEMV input vector, or a
 enum OpKind : int32_t { OP_QKV = 0, OP_ATTN = 1, OP_OPROJ = 2, OP_GATEUP = 3, OP_DOWN = 4, OP_LMHEAD = 5 };
 
 // One task: a contiguous range of tiles of one op (GEMV ops), or one
-// attention work item (b, attention head, chunk) -- an attention head is a
-// q head, or a KV head with its group of q heads -- assigned to one SM.
+// attention work item (b, q head, chunk), assigned to one SM.
 struct Task {
     int32_t kind;
     int32_t layer;
@@ -93,7 +84,6 @@ struct LayerW {
 struct Shape {
     int L, H, nq, nkv, d, F, V, S, Bmax, NC;
     int G;            // nq / nkv
-    int AG;           // q heads per attention work item: 1 or G
     int QD, KD;       // nq*d, nkv*d
     float theta, eps;
 };
@@ -110,7 +100,7 @@ struct OpTiles {
     int gateup;
     int down;
     int lmhead;
-    int attn_items;   // Bmax * (nq / AG) * NC
+    int attn_items;   // Bmax * nq * NC
 };
 
 MK_HD inline OpTiles op_tiles(const Shape &s) {
@@ -120,7 +110,7 @@ MK_HD inline OpTiles op_tiles(const Shape &s) {
     t.gateup = s.F / 8;
     t.down = s.H / 8;
     t.lmhead = (s.V + 7) / 8;
-    t.attn_items = s.Bmax * (s.nq / s.AG) * s.NC;
+    t.attn_items = s.Bmax * s.nq * s.NC;
     return t;
 }
 
@@ -158,10 +148,6 @@ MK_HD inline int rows_per_page(int K) {
 
 // Attention positions per page (K block and V block of `n` positions).
 MK_HD inline int attn_pos_per_page(int d) { return kPageBytes / (4 * d); }
-
-// Fewest positions per attention chunk: kAttnChunkPositions per q head, so
-// an item per KV head (AG q heads) splits a context AG times finer.
-MK_HD inline int attn_chunk_positions(const Shape &s) { return kAttnChunkPositions / s.AG; }
 
 // ---- tagged activations -------------------------------------------------------
 // Every activation one task hands to another lives in a "tagged" buffer: one
@@ -313,11 +299,6 @@ PlanSizes plan_sizes(const Shape &s, int num_sms);
 void plan_build(const Shape &s, int num_sms, Plan &p);
 
 // Default number of attention chunks for a shape on `num_sms` SMs.
-// Attention geometry of a shape whose other fields are set: q heads per item
-// (AG: per q head if force_qhead, per KV head if force_kvhead, else chosen
-// from the cache length) and chunks (NC: attn_chunks, or the default when
-// 0).  False when the request cannot be met.
-bool attn_geometry(Shape &s, int num_sms, bool force_qhead, bool force_kvhead, int attn_chunks);
-int default_attn_chunks(int num_sms, const Shape &s);
+int default_attn_chunks(int num_sms, int Bmax, int nq, int S);
 
 }  // namespace mk

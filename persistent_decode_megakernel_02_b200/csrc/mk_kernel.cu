@@ -211,6 +211,8 @@ __device__ __forceinline__ float2 dot8x2(const uint4 w, const float *x, float2 a
 // ---------------------------------------------------------------------------
 // shared memory
 // ---------------------------------------------------------------------------
+constexpr int kAttnCombine = kMaxHeadDim + 8;   // per-warp slot of the attention combine
+static_assert(kWorkerWarps * kAttnCombine + 16 * 12 <= kStageFloats, "combine fits the staging area");
 constexpr int kSigRing = 64;        // pending task completions the signaler can hold
 
 // A task record as the loader publishes it to the workers: the task and the
@@ -245,8 +247,8 @@ struct __align__(16) SmemCtl {
     float att_m[kWorkerWarps][1];   // LM-head argmax: per-warp best value
     float att_l[kWorkerWarps][1];   //   and its index (as float bits)
     // staging area: a row-per-warp GEMV task's input vector (read as
-    // float4); an attention task's per-warp running states and its q
-    // vectors, later its merge inputs
+    // float4); an attention task's per-warp running outputs (kWorkerWarps x
+    // kAttnCombine), later its merge inputs
     __align__(16) float stage[kStageFloats];
     unsigned long long wstat[16];   // trace-mode time accounting of worker thread 0
 };
@@ -340,8 +342,7 @@ __device__ __forceinline__ size_t my_copy(size_t stride) { return (size_t)(block
 // ---------------------------------------------------------------------------
 // task geometry shared by the loader and the workers
 // ---------------------------------------------------------------------------
-// Attention chunk of one work item (sequence b, attention head, chunk c):
-// q heads h .. h + AG - 1, all of KV head kvh.
+// Attention chunk of one work item (sequence b, q head h, chunk c).
 struct AttnChunk {
     int b, h, kvh, c;
     bool active;      // sequence b takes part in this step
@@ -355,9 +356,8 @@ struct AttnChunk {
 __device__ __forceinline__ AttnChunk attn_chunk(const Params &p, const SmemCtl *ctl, int step, int item) {
     const Shape &s = p.s;
     AttnChunk a;
-    const int na = s.nq / s.AG;   // attention heads per sequence
-    a.b = item / (na * s.NC);
-    a.h = ((item / s.NC) % na) * s.AG;
+    a.b = item / (s.nq * s.NC);
+    a.h = (item / s.NC) % s.nq;
     a.kvh = a.h / s.G;
     a.c = item % s.NC;
     a.active = a.b < p.batch;
@@ -365,10 +365,9 @@ __device__ __forceinline__ AttnChunk attn_chunk(const Params &p, const SmemCtl *
     if (a.active) {
         a.P = ctl->pos[a.b] + step;
         int C = a.P + 1;
-        // at most NC chunks, but no fewer than attn_chunk_positions(s)
-        // positions per chunk: short contexts use one chunk (nothing to merge)
-        const int cp = attn_chunk_positions(s);
-        const int nc = min(s.NC, (C + cp - 1) / cp);
+        // at most NC chunks, but no fewer than kAttnChunkPositions positions
+        // per chunk: short contexts use one chunk (nothing to merge)
+        const int nc = min(s.NC, (C + kAttnChunkPositions - 1) / kAttnChunkPositions);
         int Lc = (C + nc - 1) / nc;
         a.nc = nc;
         a.c0 = a.c * Lc;
@@ -1458,22 +1457,19 @@ __device__ bool gemv_cols(const Params &p, const Task &t, unsigned char *pages, 
 }
 
 // ---------------------------------------------------------------------------
-// attention task body: one chunk of positions of one attention head
+// attention task body: one chunk of positions of one q head
 // ---------------------------------------------------------------------------
-// An item covers ag q heads of one KV head (ag = 1, or the KV head's whole
-// group).  Prefix K/V rows of the chunk arrive through the ring once (a
-// page holds the K block then the V block of up to 256 / 128 positions);
-// warp w scores q head w % ag against every (8 / ag)-th block of 32
-// positions of each page.  Lanes compute the block's 32 scores at once
-// (lane j reads K row j in a rotated chunk order, so the 8 lanes of a
-// shared-memory phase hit different banks; q sits in shared memory padded
-// the same way), the warp updates its online-softmax state (max, sum) with
-// two reductions, and accumulates P·V with lanes over head dims.  The new
-// position's k/v come from tagged words (the first warp of each head).  The
-// states of a head's warps are combined through shared memory; a
-// single-chunk task writes the heads' outputs directly, otherwise each
-// head's (o, m, l) partial of the chunk goes out tagged and chunk 0's task
-// merges them.
+// Prefix K/V rows of the chunk arrive through the ring (a page holds the K
+// block then the V block of up to 256 / 128 positions).  Each warp takes
+// blocks of 32 positions: lanes compute the 32 scores at once (lane j reads
+// K row j in a rotated chunk order, so the 8 lanes of a shared-memory phase
+// hit different banks; q sits in shared memory padded the same way), the
+// warp updates its online-softmax state (max, sum) with two reductions,
+// and accumulates P·V with lanes over head dims.  The new position's k/v
+// come from tagged words (warp 0).  The warps' states are combined through
+// shared memory; a single-chunk task writes the q head's output directly,
+// otherwise the chunk's (o, m, l) partial goes out tagged and chunk 0's task
+// merges the partials of its q head.
 template <int D>   // head_dim: 64 or 128
 __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                           WState &w) {
@@ -1481,48 +1477,33 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     constexpr int DPL = D / 32;   // head dims per lane in P·V
     constexpr int NCH = D / 8;    // 16-byte chunks of a K row
     constexpr int KP = DPL / 2;   // tagged pairs of the new k (and v) per lane
-    constexpr int HD = D / 2;     // q element pairs RoPE rotates, per head
-    constexpr int QH = 12 * NCH;  // shared-memory floats of one head's padded q
-    constexpr int SLOT = D + 2;   // per-warp combine slot: o[D], m, l
-    constexpr int AGM = kAttnGroupElems / D;   // q heads per item at most
-    static_assert(AGM * HD <= kWorkerThreads, "a thread per q element pair");
-    static_assert(kWorkerWarps % AGM == 0, "every head gets the same number of warps");
-    static_assert(kWorkerWarps * SLOT % 4 == 0, "q is read as float4");
-    static_assert(kWorkerWarps * SLOT + AGM * QH <= kStageFloats, "combine and q fit the staging area");
-    const int ag = s.AG;          // 1, 2, 4 or 8, and ag * D <= kAttnGroupElems (checked by mk_create)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int hg = warp % ag;                 // this warp's q head within the item
-    const int wblk = warp / ag;               // its first position block
-    const int nwblk = kWorkerWarps / ag;      // warps per head: block stride
     const AttnChunk a = attn_chunk(p, ctl, ctl->wstep, t.begin);
     const int npp = attn_pos_per_page(D);
     if (!wait_ready(p, ctl, w)) return false;
     unsigned long long tp = phase_begin(w);
     const int npages = (a.npre + npp - 1) / npp;
-    float *qs = ctl->stage + kWorkerWarps * SLOT;   // head g, chunk c (8 values) at qs + g QH + 12 c
+    float *qs = ctl->stage + kWorkerWarps * kAttnCombine;   // q: chunk c (8 values) at qs + 12 c
 
-    // ---- q (thread i < ag D/2: head i / (D/2), elements e and e + D/2 with
-    // e = i % (D/2), the pair RoPE rotates together) and the new k / v (the
-    // first warp of each head), tagged, polled until fresh; RoPE at the
-    // token's position is applied here
-    const bool new_warp = a.has_new && wblk == 0;
-    const bool q_thread = tid < ag * HD;
-    const int qg = tid / HD, qe = tid % HD;
+    // ---- q (thread i < D/2 takes elements i and i + D/2, the pair RoPE
+    // rotates together) and the new k / v (warp 0), tagged, polled until
+    // fresh; RoPE at the token's position is applied here
+    const bool new_warp = a.has_new && warp == 0;
     float kn[DPL], vn[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) { kn[i] = 0.f; vn[i] = 0.f; }
     if (a.active) {
-        const uint64_t *qsrc = tag_buf(p, t.layer, p.tl.q) + (size_t)a.b * s.QD + (size_t)(a.h + qg) * D + qe;
+        const uint64_t *qsrc = tag_buf(p, t.layer, p.tl.q) + (size_t)a.b * s.QD + (size_t)a.h * D;
         const uint64_t *ksrc = tag_buf(p, t.layer, p.tl.kn) + (size_t)a.b * s.KD + (size_t)a.kvh * D + lane * DPL;
         const uint64_t *vsrc = tag_buf(p, t.layer, p.tl.vn) + (size_t)a.b * s.KD + (size_t)a.kvh * D + lane * DPL;
         float q_lo = 0.f, q_hi = 0.f;
         uint32_t pend = 0;
-        // bits 0, 1: this thread's q elements e, e + D/2; bits 2 .. 1+KP: new
+        // bits 0, 1: this thread's q elements i, i + D/2; bits 2 .. 1+KP: new
         // k pairs; then new v pairs
         auto load = [&](int bit) {
             bool ok;
             if (bit < 2) {
-                const uint64_t v = ld_tag1(qsrc + (bit ? HD : 0));
+                const uint64_t v = ld_tag1(qsrc + tid + (bit ? D / 2 : 0));
                 if (bit) q_hi = tag_val(v); else q_lo = tag_val(v);
                 ok = tag_ok(v, w.ep);
             } else {
@@ -1539,7 +1520,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
         };
 #pragma unroll
         for (int bit = 0; bit < 2 + 2 * KP; ++bit)
-            if ((bit < 2 && q_thread) || (bit >= 2 && new_warp)) load(bit);
+            if ((bit < 2 && tid < D / 2) || (bit >= 2 && new_warp)) load(bit);
         Spin sp;
         while (__any_sync(0xffffffffu, pend != 0u)) {
             if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 4u)) return false;
@@ -1547,32 +1528,30 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
             for (int bit = 0; bit < 2 + 2 * KP; ++bit)
                 if (pend & (1u << bit)) load(bit);
         }
-        if (q_thread) {
-            const float2 cs = p.rope[(size_t)a.P * HD + qe];
+        if (tid < D / 2) {
+            const float2 cs = p.rope[(size_t)a.P * (D / 2) + tid];
             const float scale = 1.0f / sqrtf((float)D);
-            const int e = qe, f = qe + HD;
-            float *qd = qs + qg * QH;
-            qd[12 * (e >> 3) + (e & 7)] = (q_lo * cs.x - q_hi * cs.y) * scale;
-            qd[12 * (f >> 3) + (f & 7)] = (q_hi * cs.x + q_lo * cs.y) * scale;
+            const int e = tid, f = tid + D / 2;
+            qs[12 * (e >> 3) + (e & 7)] = (q_lo * cs.x - q_hi * cs.y) * scale;
+            qs[12 * (f >> 3) + (f & 7)] = (q_hi * cs.x + q_lo * cs.y) * scale;
         }
         if (new_warp) {
             // rotate the new key (lane L holds elements L*DPL..; the partner of
             // an element sits D/2 further, i.e. in lane L ^ 16), round it to
-            // bf16 as the cache stores it; warp 0 of the group's first q head
-            // appends it
+            // bf16 as the cache stores it; the group's first q head appends it
             uint16_t kb[DPL];
 #pragma unroll
             for (int j = 0; j < DPL; ++j) {
                 const float other = __shfl_xor_sync(0xffffffffu, kn[j], 16);
                 const int e = lane * DPL + j;
-                const int i = e % HD;
-                const float2 cs = p.rope[(size_t)a.P * HD + i];
+                const int i = e % (D / 2);
+                const float2 cs = p.rope[(size_t)a.P * (D / 2) + i];
                 const float r = lane < 16 ? kn[j] * cs.x - other * cs.y : kn[j] * cs.x + other * cs.y;
                 kb[j] = f2bf(r);
             }
 #pragma unroll
             for (int j = 0; j < DPL; ++j) kn[j] = bf2f(kb[j]);
-            if (warp == 0 && a.h % s.G == 0) {
+            if (a.h % s.G == 0) {
                 uint16_t *kc = p.layers[t.layer].kc + (((size_t)a.b * s.nkv + a.kvh) * s.S + a.P) * D + lane * DPL;
 #pragma unroll
                 for (int j = 0; j < DPL; ++j) kc[j] = kb[j];
@@ -1584,20 +1563,6 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     phase_end(w, tp, WS_PRO);
     stamp_input(p, w);
 
-    const float *qh = qs + hg * QH;
-    // head_dim 64: the lane's q chunks held in registers in its rotated
-    // order (chunk (c + lane) mod NCH at qr[2c], qr[2c + 1]), so the score
-    // loop reads only K from shared memory; head_dim 128 reads q there
-    constexpr bool kQReg = D == 64;
-    float4 qr[kQReg ? 2 * NCH : 1];
-    if constexpr (kQReg) {
-#pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-            const int cc = (c + lane) & (NCH - 1);
-            qr[2 * c] = *reinterpret_cast<const float4 *>(qh + 12 * cc);
-            qr[2 * c + 1] = *reinterpret_cast<const float4 *>(qh + 12 * cc + 4);
-        }
-    }
     float m = -INFINITY, l = 0.f, o[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) o[i] = 0.f;
@@ -1608,32 +1573,24 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
         const uint16_t *Kp = reinterpret_cast<const uint16_t *>(pages + (size_t)slot * kPageBytes);
         const uint16_t *Vp = Kp + (size_t)npp * D;
         const int n = min(npp, a.npre - pg * npp);
-        for (int j0 = wblk * 32; j0 < n; j0 += nwblk * 32) {
+        for (int j0 = warp * 32; j0 < n; j0 += kWorkerWarps * 32) {
             const int j = j0 + lane;
             float sc = -INFINITY;
             if (j < n) {
                 const uint4 *krow = reinterpret_cast<const uint4 *>(Kp + (size_t)j * D);
-                // two accumulators (even / odd chunks) halve the FMA chain
-                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < NCH; ++c) {
                     const int cc = (c + lane) & (NCH - 1);
                     const uint4 kw = krow[cc];
-                    float4 q0, q1;
-                    if constexpr (kQReg) {
-                        q0 = qr[2 * c];
-                        q1 = qr[2 * c + 1];
-                    } else {
-                        q0 = *reinterpret_cast<const float4 *>(qh + 12 * cc);
-                        q1 = *reinterpret_cast<const float4 *>(qh + 12 * cc + 4);
-                    }
-                    float2 &a2 = acc[c & 1];
-                    a2 = ffma2(make_float2(bf_lo(kw.x), bf_hi(kw.x)), make_float2(q0.x, q0.y), a2);
-                    a2 = ffma2(make_float2(bf_lo(kw.y), bf_hi(kw.y)), make_float2(q0.z, q0.w), a2);
-                    a2 = ffma2(make_float2(bf_lo(kw.z), bf_hi(kw.z)), make_float2(q1.x, q1.y), a2);
-                    a2 = ffma2(make_float2(bf_lo(kw.w), bf_hi(kw.w)), make_float2(q1.z, q1.w), a2);
+                    const float4 q0 = *reinterpret_cast<const float4 *>(qs + 12 * cc);
+                    const float4 q1 = *reinterpret_cast<const float4 *>(qs + 12 * cc + 4);
+                    acc = ffma2(make_float2(bf_lo(kw.x), bf_hi(kw.x)), make_float2(q0.x, q0.y), acc);
+                    acc = ffma2(make_float2(bf_lo(kw.y), bf_hi(kw.y)), make_float2(q0.z, q0.w), acc);
+                    acc = ffma2(make_float2(bf_lo(kw.z), bf_hi(kw.z)), make_float2(q1.x, q1.y), acc);
+                    acc = ffma2(make_float2(bf_lo(kw.w), bf_hi(kw.w)), make_float2(q1.z, q1.w), acc);
                 }
-                sc = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
+                sc = acc.x + acc.y;
             }
             float mb = sc;
 #pragma unroll
@@ -1647,36 +1604,19 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
             m = mn;
             const int cnt = min(32, n - j0);
             const uint16_t *vb = Vp + (size_t)j0 * D + lane * DPL;
-            auto pv_step = [&](float *acc, int k) {
+            for (int k = 0; k < cnt; ++k) {
                 const float pk = __shfl_sync(0xffffffffu, pe, k);
                 if constexpr (DPL == 2) {
                     const uint32_t vw = *reinterpret_cast<const uint32_t *>(vb + (size_t)k * D);
-                    acc[0] = fmaf(pk, bf_lo(vw), acc[0]);
-                    acc[1] = fmaf(pk, bf_hi(vw), acc[1]);
+                    o[0] = fmaf(pk, bf_lo(vw), o[0]);
+                    o[1] = fmaf(pk, bf_hi(vw), o[1]);
                 } else {
                     const uint2 vw = *reinterpret_cast<const uint2 *>(vb + (size_t)k * D);
-                    acc[0] = fmaf(pk, bf_lo(vw.x), acc[0]);
-                    acc[1] = fmaf(pk, bf_hi(vw.x), acc[1]);
-                    acc[2] = fmaf(pk, bf_lo(vw.y), acc[2]);
-                    acc[3] = fmaf(pk, bf_hi(vw.y), acc[3]);
+                    o[0] = fmaf(pk, bf_lo(vw.x), o[0]);
+                    o[1] = fmaf(pk, bf_hi(vw.x), o[1]);
+                    o[2] = fmaf(pk, bf_lo(vw.y), o[2]);
+                    o[3] = fmaf(pk, bf_hi(vw.y), o[3]);
                 }
-            };
-            if (cnt == 32) {
-                // a full block: unrolled, so the shuffles and V loads of many
-                // positions are in flight together; even / odd positions go
-                // to two accumulators
-                float o2[DPL];
-#pragma unroll
-                for (int i = 0; i < DPL; ++i) o2[i] = 0.f;
-#pragma unroll
-                for (int k = 0; k < 32; k += 2) {
-                    pv_step(o, k);
-                    pv_step(o2, k + 1);
-                }
-#pragma unroll
-                for (int i = 0; i < DPL; ++i) o[i] += o2[i];
-            } else {
-                for (int k = 0; k < cnt; ++k) pv_step(o, k);
             }
         }
         release_page(ctl, w, slot);
@@ -1688,7 +1628,7 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
 #pragma unroll
         for (int i = 0; i < DPL; ++i) {
             const int e = lane * DPL + i;
-            sc = fmaf(qh[12 * (e >> 3) + (e & 7)], kn[i], sc);
+            sc = fmaf(qs[12 * (e >> 3) + (e & 7)], kn[i], sc);
         }
         sc = warp_sum(sc);
         const float mn = fmaxf(m, sc);
@@ -1700,54 +1640,51 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
         m = mn;
     }
 
-    // ---- combine the states of each head's warps (warps g, g + ag, ...)
-    float *cw = ctl->stage + warp * SLOT;
+    // ---- combine the warps' states
+    float *cw = ctl->stage + warp * kAttnCombine;
 #pragma unroll
     for (int i = 0; i < DPL; ++i) cw[lane * DPL + i] = o[i];
     if (lane == 0) { cw[D] = m; cw[D + 1] = l; }
     if (!worker_sync(p, ctl, w)) return false;
-    // partials of q head h + g at part + g NC (D + 2); chunk c at + c (D + 2)
     uint64_t *part = tag_buf(p, t.layer, p.tl.part) + ((size_t)a.b * s.nq + a.h) * s.NC * (D + 2);
     // chunks at or past nc hold no positions and write nothing
-    if (a.active && a.c < a.nc) {
-        for (int idx = tid; idx < ag * D; idx += kWorkerThreads) {
-            const int g = idx / D, e = idx % D;
-            float M = -INFINITY;
-            for (int k = g; k < kWorkerWarps; k += ag) M = fmaxf(M, ctl->stage[k * SLOT + D]);
-            float O = 0.f, L = 0.f;
-            if (M != -INFINITY) {
-                for (int k = g; k < kWorkerWarps; k += ag) {
-                    const float *ck = ctl->stage + k * SLOT;
-                    const float f = expf(ck[D] - M);
-                    O = fmaf(f, ck[e], O);
-                    L = fmaf(f, ck[D + 1], L);
-                }
+    if (a.active && a.c < a.nc && tid < D) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kWorkerWarps; ++k) M = fmaxf(M, ctl->stage[k * kAttnCombine + D]);
+        float O = 0.f, L = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int k = 0; k < kWorkerWarps; ++k) {
+                const float *ck = ctl->stage + k * kAttnCombine;
+                const float f = expf(ck[D] - M);
+                O = fmaf(f, ck[tid], O);
+                L = fmaf(f, ck[D + 1], L);
             }
-            if (a.nc == 1) {
-                st_tag_rep(tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)(a.h + g) * D + e,
-                           p.tl.rep_qd, O / L, w.ep_out);
-            } else {
-                uint64_t *dst = part + ((size_t)g * s.NC + a.c) * (D + 2);
-                st_tag(dst + e, O, w.ep_out);
-                if (e == 0) {
-                    st_tag(dst + D, M, w.ep_out);
-                    st_tag(dst + D + 1, L, w.ep_out);
-                }
+        }
+        if (a.nc == 1) {
+            st_tag_rep(tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)a.h * D + tid,
+                       p.tl.rep_qd, O / L, w.ep_out);
+        } else {
+            uint64_t *dst = part + (size_t)a.c * (D + 2);
+            st_tag(dst + tid, O, w.ep_out);
+            if (tid == 0) {
+                st_tag(dst + D, M, w.ep_out);
+                st_tag(dst + D + 1, L, w.ep_out);
             }
         }
     }
     stamp_done(p, w);
     if (a.active && a.nc > 1 && a.c == 0) {
-        // chunk 0's task merges its heads' partials: polls them into shared
-        // memory (tagged, so it waits for exactly the chunks it reads; head
-        // g's nc chunks at stage + g nc (D + 2)), then combines them there
+        // chunk 0's task merges its q head's partials: polls them into shared
+        // memory (tagged, so it waits for exactly the chunks it reads), then
+        // combines them there
         const int nc = a.nc;
         if (!worker_sync(p, ctl, w)) return false;   // the combine above is done with the stage
-        if (!stage_partials(p, ctl, w, part, ag, nc * (D + 2), s.NC * (D + 2))) return false;
+        if (!stage_partials(p, ctl, w, part, 1, nc * (D + 2), s.NC * (D + 2))) return false;
         if (!worker_sync(p, ctl, w)) return false;
-        for (int idx = tid; idx < ag * D; idx += kWorkerThreads) {
-            const int g = idx / D, e = idx % D;
-            const float *sg = ctl->stage + (size_t)g * nc * (D + 2);
+        if (tid < D) {
+            const float *sg = ctl->stage;
             float M = -INFINITY;
             for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (D + 2) + D]);
             float num = 0.f, den = 0.f;
@@ -1755,10 +1692,10 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
                 const float mc = sg[c * (D + 2) + D];
                 if (mc == -INFINITY) continue;
                 const float f = expf(mc - M);
-                num = fmaf(f, sg[c * (D + 2) + e], num);
+                num = fmaf(f, sg[c * (D + 2) + tid], num);
                 den = fmaf(f, sg[c * (D + 2) + D + 1], den);
             }
-            st_tag_rep(tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)(a.h + g) * D + e,
+            st_tag_rep(tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)a.h * D + tid,
                        p.tl.rep_qd, num / den, w.ep_out);
         }
     }

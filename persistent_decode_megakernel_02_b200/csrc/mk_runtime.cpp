@@ -79,9 +79,10 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     s.d = c->head_dim; s.F = c->ffn; s.V = c->vocab; s.S = c->max_seq; s.Bmax = c->max_batch;
     s.G = G; s.QD = (int)QD; s.KD = c->n_kv_heads * c->head_dim;
     s.theta = c->rope_theta; s.eps = c->rms_eps;
-    if (!attn_geometry(s, num_sms, (c->flags & MK_FLAG_ATTN_PER_QHEAD) != 0,
-                       (c->flags & MK_FLAG_ATTN_PER_KVHEAD) != 0, c->attn_chunks))
-        return MK_ERR_INVALID;
+    s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nq, s.S);
+    if (s.NC > 4096) return MK_ERR_INVALID;
+    // one q head's chunk partials must fit the merge's shared staging area
+    if ((long long)s.NC * (s.d + 2) > kStageFloats) return MK_ERR_INVALID;
     return MK_OK;
 }
 
@@ -134,7 +135,6 @@ int mk_plan(const mk_config *cfg, int num_sms, mk_info *info, int32_t *task_out,
         info->num_events = p.num_events;
         info->num_ops = p.num_ops;
         info->attn_chunks = s.NC;
-        info->attn_q_heads = s.AG;
         info->max_queue = p.max_queue;
         info->page_bytes = kPageBytes;
         info->num_pages = kNumPages;
@@ -433,7 +433,6 @@ int mk_get_info(mk_ctx *c, mk_info *out) {
     out->num_events = c->num_events;
     out->num_ops = c->num_ops;
     out->attn_chunks = c->s.NC;
-    out->attn_q_heads = c->s.AG;
     out->max_queue = c->max_queue;
     out->page_bytes = kPageBytes;
     out->num_pages = kNumPages;

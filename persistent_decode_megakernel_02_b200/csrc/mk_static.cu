@@ -58,10 +58,6 @@ alignas(256) unsigned char g_host[MK_STATIC_SCRATCH_BYTES];
 
 // What the tables currently in a device's scratch were built from: a hash of
 // the shape (task graph, RoPE table) and a hash of the layer pointer table.
-// The shape hash covers every input of the plan and of the scratch layout,
-// the derived attention geometry included (q heads per item and chunks:
-// flags choose it), so tables of one geometry are never read at another's
-// offsets.
 struct Signature {
     bool valid = false;
     uint64_t shape_key = 0;
@@ -75,10 +71,9 @@ uint64_t fnv1a(uint64_t h, const void *data, size_t n) {
     return h;
 }
 
-uint64_t shape_key(const mk_config *c, const Shape &s, int num_sms) {
+uint64_t shape_key(const mk_config *c, int num_sms) {
     const long long f[] = {c->layers, c->hidden, c->n_q_heads, c->n_kv_heads, c->head_dim, c->ffn,
-                           c->vocab, c->max_seq, c->max_batch, c->attn_chunks, num_sms,
-                           s.AG, s.NC};
+                           c->vocab, c->max_seq, c->max_batch, c->attn_chunks, num_sms};
     uint64_t h = fnv1a(1469598103934665603ull, f, sizeof f);
     const float g[] = {c->rope_theta, c->rms_eps};
     return fnv1a(h, g, sizeof g);
@@ -111,8 +106,9 @@ bool shape_ok(const mk_config *c, int num_sms, Shape &s) {
     s.d = c->head_dim; s.F = c->ffn; s.V = c->vocab; s.S = c->max_seq; s.Bmax = c->max_batch;
     s.G = G; s.QD = (int)QD; s.KD = c->n_kv_heads * c->head_dim;
     s.theta = c->rope_theta; s.eps = c->rms_eps;
-    return attn_geometry(s, num_sms, (c->flags & MK_FLAG_ATTN_PER_QHEAD) != 0,
-                         (c->flags & MK_FLAG_ATTN_PER_KVHEAD) != 0, c->attn_chunks);
+    s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nq, s.S);
+    if (s.NC > 4096 || (long long)s.NC * (s.d + 2) > kStageFloats) return false;
+    return true;
 }
 
 Layout layout_for(const Shape &s, const PlanSizes &z, int num_sms, int num_lm_tasks) {
@@ -204,7 +200,7 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
         lw[l].kc = (uint16_t *)kv->k[l];
         lw[l].vc = (uint16_t *)kv->v[l];
     }
-    const uint64_t skey = shape_key(cfg, s, ds.num_sms);
+    const uint64_t skey = shape_key(cfg, ds.num_sms);
     const uint64_t lkey = fnv1a(skey, lw, sizeof(LayerW) * s.L);
     if (!sig.valid || sig.shape_key != skey) {
         // task graph and RoPE table for this shape, in static host storage

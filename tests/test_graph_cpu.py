@@ -41,16 +41,14 @@ def _tiles(shape):
             OPROJ: H // 8, GATEUP: F // 8, DOWN: H // 8, LMHEAD: (V + 7) // 8}
 
 
-KVH, QH = mk.MK_FLAG_ATTN_PER_KVHEAD, mk.MK_FLAG_ATTN_PER_QHEAD
-CASES = [("tiny", wl.TINY, 64, 0), ("tiny-kvhead", wl.TINY, 64, KVH), ("1b", wl.LLAMA_1B, 560, 0),
-         ("8b", wl.LLAMA_8B, 560, 0), ("longctx", wl.LLAMA_1B, 16640, 0),
-         ("longctx-qhead", wl.LLAMA_1B, 16640, QH), ("8b-long", wl.LLAMA_8B, 16640, 0)]
+CASES = [("tiny", wl.TINY, 64), ("1b", wl.LLAMA_1B, 560), ("8b", wl.LLAMA_8B, 560),
+         ("longctx", wl.LLAMA_1B, 16640)]
 
 
 @pytest.fixture(scope="module", params=CASES, ids=[c[0] for c in CASES])
 def planned(request):
-    name, shape, S, flags = request.param
-    cfg = mk.make_config(shape, S, 1, flags=flags)
+    name, shape, S = request.param
+    cfg = mk.make_config(shape, S, 1)
     return shape, cfg, mk.plan(cfg, SMS)
 
 
@@ -59,14 +57,13 @@ def test_every_row_and_item_covered_once(planned):
     tasks = pl["tasks"]
     tiles = _tiles(shape)
     nc = pl["info"].attn_chunks
-    heads = shape.n_q_heads // pl["info"].attn_q_heads   # attention heads: q heads or KV heads
     for layer in range(shape.layers + 1):
         for kind in (QKV, ATTN, OPROJ, GATEUP, DOWN, LMHEAD):
             sel = tasks[(tasks[:, 0] == kind) & (tasks[:, 1] == layer)]
             if (kind == LMHEAD) != (layer == shape.layers):
                 assert len(sel) == 0
                 continue
-            n = heads * nc if kind == ATTN else tiles[kind]
+            n = shape.n_q_heads * nc if kind == ATTN else tiles[kind]
             cover = np.zeros(n, np.int32)
             for t in sel:
                 cover[t[4]:t[5]] += 1
@@ -160,63 +157,25 @@ def test_plan_rejects_unsupported_shapes(bad):
     assert ei.value.status == mk.MK_ERR_INVALID
 
 
-def _attn(shape, S, **kw):
-    info = mk.plan(mk.make_config(shape, S, **kw), SMS)["info"]
-    return info.attn_q_heads, info.attn_chunks
-
-
-def test_default_attention_geometry():
-    # caches up to 4096 positions: a task per (sequence, q head, chunk), as
-    # many chunks as fill the SMs but no more than a full cache needs at 1024
+def test_default_attention_chunks():
+    # one task per (sequence, q head, chunk): as many chunks as fill the SMs
+    # (148 // 32 q heads = 4), but no more than a full cache needs at 1024
     # positions per chunk
-    assert _attn(wl.LLAMA_1B, 560) == (1, 1)
-    assert _attn(wl.TINY, 64) == (1, 1)
-    assert _attn(wl.TINY, 4096) == (1, 4)
-    assert _attn(wl.TINY, 64, attn_chunks=7) == (1, 7)
-    # longer caches: a task per (sequence, KV head, chunk) covering the KV
-    # head's G q heads, chunks of at least 1024 / G positions; 148 // 8 KV
-    # heads = 18 chunks, for head_dim 128 capped at 8192 // (4 * 130) = 15
-    # (one item's partials fit the merge's staging area); tiny: 148 // 2,
-    # capped at the 8192 / 512 = 16 a full cache needs
-    assert _attn(wl.LLAMA_1B, 16640) == (4, 18)
-    assert _attn(wl.LLAMA_8B, 16640) == (4, 15)
-    assert _attn(wl.TINY, 8192) == (2, 16)
-    # either forced
-    assert _attn(wl.LLAMA_1B, 16640, flags=QH) == (1, 4)
-    assert _attn(wl.LLAMA_1B, 560, flags=KVH) == (4, 3)
-    assert _attn(wl.TINY, 64, flags=KVH, attn_chunks=62) == (2, 62)
+    assert mk.plan(mk.make_config(wl.LLAMA_1B, 16640), SMS)["info"].attn_chunks == 4
+    assert mk.plan(mk.make_config(wl.LLAMA_1B, 560), SMS)["info"].attn_chunks == 1
+    assert mk.plan(mk.make_config(wl.TINY, 64), SMS)["info"].attn_chunks == 1
+    assert mk.plan(mk.make_config(wl.TINY, 4096), SMS)["info"].attn_chunks == 4
+    assert mk.plan(mk.make_config(wl.TINY, 64, attn_chunks=7), SMS)["info"].attn_chunks == 7
 
 
-@pytest.mark.parametrize("shape_kw,S,kw", [
-    ({}, 64, dict(flags=KVH | QH)),                                   # both modes at once
-    (dict(n_q_heads=8, n_kv_heads=1, head_dim=128), 64, dict(flags=KVH)),   # 8 x 128 > 512
-    ({}, 64, dict(flags=KVH, attn_chunks=63)),                        # 2 x 63 x 66 > 8192
-    ({}, 64, dict(attn_chunks=125)),                                  # 125 x 66 > 8192
-])
-def test_plan_rejects_attention_geometry_that_does_not_fit(shape_kw, S, kw):
-    base = dict(layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=768,
-                vocab=4096, tied=True, rope_theta=1e4)
-    base.update(shape_kw)
-    cfg = mk.make_config(wl.ModelShape("geo", **base), S, 1, **kw)
-    with pytest.raises(mk.MkError) as ei:
-        mk.plan(cfg, SMS)
-    assert ei.value.status == mk.MK_ERR_INVALID
-    # the same shape plans in the other mode / with fewer chunks
-    ok = dict(kw)
-    ok["flags"] = QH if kw.get("flags") else 0
-    ok["attn_chunks"] = min(kw.get("attn_chunks", 0), 62)
-    mk.plan(mk.make_config(wl.ModelShape("geo", **base), S, 1, **ok), SMS)
-
-
-@pytest.mark.parametrize("flags", [QH, KVH])
 @pytest.mark.parametrize("sms,chunks", [(5, 7), (16, 8), (SMS, 0)])
-def test_attention_merger_runs_after_its_chunks(sms, chunks, flags):
-    """Chunk 0's task of every (sequence, attention head) merges the
-    partials and waits for the other chunks' tagged outputs: on every queue
-    it must come after each other chunk of its head, and the whole graph
-    must run to completion when tasks wait on exactly their inputs."""
+def test_attention_merger_runs_after_its_chunks(sms, chunks):
+    """Chunk 0's task of every (sequence, KV head) merges the partials and
+    waits for the other chunks' tagged outputs: on every queue it must come
+    after each other chunk of its head, and the whole graph must run to
+    completion when tasks wait on exactly their inputs."""
     shape = wl.TINY
-    cfg = mk.make_config(shape, 256, 1, flags=flags, attn_chunks=chunks)
+    cfg = mk.make_config(shape, 256, 1, attn_chunks=chunks)
     pl = mk.plan(cfg, sms)
     tasks, queue, qoff = pl["tasks"], pl["queue"], pl["qoff"]
     NC = pl["info"].attn_chunks
@@ -255,3 +214,15 @@ def test_attention_merger_runs_after_its_chunks(sms, chunks, flags):
                 progressed = True
         assert progressed, "tasks wait on each other in a cycle"
     assert done.all()
+
+
+def test_plan_refuses_partials_that_overflow_the_merge_stage():
+    # chunk 0's task stages every chunk's (o[d], m, l) of its q head in 8192
+    # floats of shared memory: 124 chunks x 66 fit, 125 do not
+    base = dict(layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=768,
+                vocab=4096, tied=True, rope_theta=1e4)
+    shape = wl.ModelShape("chunks", **base)
+    assert mk.plan(mk.make_config(shape, 64, 1, attn_chunks=124), SMS)["info"].attn_chunks == 124
+    with pytest.raises(mk.MkError) as ei:
+        mk.plan(mk.make_config(shape, 64, 1, attn_chunks=125), SMS)
+    assert ei.value.status == mk.MK_ERR_INVALID

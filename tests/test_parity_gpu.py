@@ -36,9 +36,6 @@ def _check_events(pair, steps):
 # 0: tasks wait on their tagged inputs; 4 (MK_FLAG_EVENT_WAIT): a scheduler
 # warp gates every task on its dependency's event counter first
 WAIT_MODES = [0, 4]
-# attention work items per q head (8) or per KV head with its group of q
-# heads (16)
-QH, KVH = 8, 16
 
 
 @pytest.mark.parametrize("flags", WAIT_MODES)
@@ -80,11 +77,10 @@ def test_tiny_random_gains_untied_head_and_intermediates(flags):
     _check_hidden(pair, ref)
 
 
-@pytest.mark.parametrize("mode", [QH, KVH])
-@pytest.mark.parametrize("chunks", [1, 3, 13, 62])
-def test_attention_chunking_does_not_change_results(chunks, mode):
+@pytest.mark.parametrize("chunks", [1, 3, 13, 64])
+def test_attention_chunking_does_not_change_results(chunks):
     shape = wl.TINY
-    pair = Pair(shape, max_seq=96, attn_chunks=chunks, flags=mode)
+    pair = Pair(shape, max_seq=96, attn_chunks=chunks)
     toks = wl.make_prompt(shape.vocab, 40, seed=11)
     for pos, t in enumerate(toks):
         g_tok, g_log = pair.gpu_step(int(t), pos)
@@ -92,15 +88,13 @@ def test_attention_chunking_does_not_change_results(chunks, mode):
         _check_step(pair, pos, g_tok, g_log, ref)
 
 
-@pytest.mark.parametrize("mode", [QH, KVH])
 @pytest.mark.parametrize("chunks", [3, 5])
-def test_long_prefix_split_into_chunks_and_merged(chunks, mode):
-    # 2600+ positions: per q head ceil(C / 1024) = 3 active chunks, merged by
-    # chunk 0's task (with 5 chunks, two are empty); per KV head (2 q heads)
-    # chunks of 512 positions, so every chunk holds some
+def test_long_prefix_split_into_chunks_and_merged(chunks):
+    # 2600+ positions: ceil(C / 1024) = 3 active chunks per q head, merged by
+    # chunk 0's task (with 5 chunks, two are empty)
     shape = wl.TINY
     S = 2624
-    pair = Pair(shape, max_seq=S, prefill_len=2600, attn_chunks=chunks, flags=mode)
+    pair = Pair(shape, max_seq=S, prefill_len=2600, attn_chunks=chunks)
     toks = wl.make_prompt(shape.vocab, 4, seed=13)
     for i, t in enumerate(toks):
         pos = 2600 + i
@@ -228,12 +222,10 @@ def test_llama1b_shape_teacher_forced():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("mode", [0, QH])   # default at this length: per KV head
-def test_llama1b_long_context_prefilled(mode):
+def test_llama1b_long_context_prefilled():
     shape = wl.LLAMA_1B
     S = 16640
-    pair = Pair(shape, max_seq=S, prefill_len=16384, flags=mode)
-    assert pair.ctx.info().attn_q_heads == (1 if mode == QH else 4)
+    pair = Pair(shape, max_seq=S, prefill_len=16384)
     prompt = wl.make_prompt(shape.vocab, 1, seed=5)
     for step, pos, g_tok, g_log, ref in pair.teacher_forced(prompt, 1, start_pos=16384):
         _check_step(pair, step, g_tok, g_log, ref)
@@ -241,10 +233,9 @@ def test_llama1b_long_context_prefilled(mode):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("mode", [0, KVH])
-def test_llama8b_shape_teacher_forced(mode):
+def test_llama8b_shape_teacher_forced():
     shape = wl.LLAMA_8B
-    pair = Pair(shape, max_seq=560, flags=mode)
+    pair = Pair(shape, max_seq=560)
     prompt = wl.make_prompt(shape.vocab, 1, seed=42)
     for step, pos, g_tok, g_log, ref in pair.teacher_forced(prompt, 1):
         _check_step(pair, step, g_tok, g_log, ref)

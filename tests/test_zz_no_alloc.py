@@ -33,8 +33,7 @@ def _pack(weights):
             "wo": weights.wo, "gu": gu, "wd": weights.wd}
 
 
-@pytest.mark.parametrize("flags", [0, 16])   # 16: attention items per KV head
-def test_static_step_matches_context_step_twice(flags):
+def test_static_step_matches_context_step_twice():
     from persistent_decode_megakernel_02_b200 import mk
     shape = wl.TINY
     S = 48
@@ -42,8 +41,8 @@ def test_static_step_matches_context_step_twice(flags):
     packed = _pack(w)
     k_ctx, v_ctx = wl.make_kv(shape, 1, S, device="cuda")
     k_st, v_st = wl.make_kv(shape, 1, S, device="cuda")
-    ctx = mk.Context(w, k_ctx, v_ctx, S, 1, flags=flags)
-    cfg = mk.make_config(shape, S, 1, flags=flags)
+    ctx = mk.Context(w, k_ctx, v_ctx, S, 1)
+    cfg = mk.make_config(shape, S, 1)
     tok = torch.zeros(1, dtype=torch.int32, device="cuda")
     pos = torch.zeros(1, dtype=torch.int32, device="cuda")
     nxt_a = torch.zeros(1, dtype=torch.int32, device="cuda")
