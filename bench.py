@@ -35,6 +35,7 @@ import json
 import math
 import os
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -106,14 +107,21 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, path: str | None = None):
+        """`path`: where the raw samples go (CSV); a temporary file if None."""
         self.dev = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.tmp = path is None
+        if path is None:
+            fd, path = tempfile.mkstemp(prefix=f"mk_clocks_{device_index}_", suffix=".csv")
+            os.close(fd)
+        self.path = path
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            d = os.path.dirname(self.path)
+            if d:
+                os.makedirs(d, exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
@@ -135,10 +143,16 @@ class ClockSampler:
             self.f.close()
 
     def summary(self) -> dict:
-        if self.proc is None or not os.path.exists(self.path):
+        lines = []
+        if os.path.exists(self.path):
+            with open(self.path) as f:
+                lines = f.readlines()
+            if self.tmp:
+                os.remove(self.path)
+        if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         rows = []
-        for line in open(self.path):
+        for line in lines:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -214,6 +228,9 @@ def parse():
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
     ap.add_argument("--flags", type=int, default=0, help="mk_config.flags")
     ap.add_argument("--attn-chunks", type=int, default=0)
+    ap.add_argument("--clocks-csv", default=None,
+                    help="keep the raw nvidia-smi clock samples of the timed region in this CSV "
+                         "('{rank}' is replaced by the rank); default: a temporary file")
     return ap.parse_args()
 
 
@@ -320,7 +337,10 @@ def main():
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        with ClockSampler(torch.cuda.current_device()) as clk:
+        clk_path = None
+        if args.clocks_csv:
+            clk_path = args.clocks_csv.replace("{rank}", str(rank))
+        with ClockSampler(torch.cuda.current_device(), clk_path) as clk:
             e0.record(stream)
             for i in range(W, W + K):
                 one(i, toks[i + 1:i + 2])

@@ -30,3 +30,41 @@ def test_one_b_shape_step_bytes():
     assert bench.step_weight_bytes(wl.LLAMA_1B) == 2_471_632_896
     # K and V, 8 heads x 64 dims bf16, 16 layers: 32 KiB per attended position
     assert bench.step_kv_bytes(wl.LLAMA_1B, [1]) == 32768
+
+
+def _clock_rows(path, rows):
+    # nvidia-smi csv,noheader,nounits: index, clocks.sm, clocks.max.sm,
+    # power.draw, reasons.active, hw_slowdown, hw_thermal, sw_thermal, sw_power_cap
+    with open(path, "w") as f:
+        for r in rows:
+            f.write(", ".join(str(x) for x in r) + "\n")
+
+
+def test_clock_summary_takes_the_loaded_samples_and_their_reasons(tmp_path):
+    p = str(tmp_path / "c.csv")
+    idle = [(0, 1980, 1965, 150.0, "0x0", "Not Active", "Not Active", "Not Active", "Not Active")] * 4
+    busy = [(0, 1965, 1965, 900.0, "0x4", "Not Active", "Not Active", "Not Active", "Active")] * 5
+    _clock_rows(p, idle + busy + ["garbage line"])
+    c = bench.ClockSampler(0, p)
+    c.proc = object()            # as if nvidia-smi had run
+    s = c.summary()
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 9
+    assert os.path.exists(p)     # a caller's file is kept
+
+
+def test_clock_summary_flags_thermal_slowdown_and_missing_samples(tmp_path):
+    p = str(tmp_path / "c.csv")
+    rows = [(0, 1500, 1965, 950.0, "0x20", "Not Active", "Active", "Not Active", "Not Active")] * 3
+    _clock_rows(p, rows)
+    c = bench.ClockSampler(0, p)
+    c.proc = object()
+    assert c.summary()["reasons"] == ["hw_thermal_slowdown"]
+    empty = bench.ClockSampler(0)    # temporary file, nothing sampled
+    assert empty.summary()["reasons"] == ["unsampled"]
+    assert not os.path.exists(empty.path)
+    t = bench.ClockSampler(0)
+    _clock_rows(t.path, rows)
+    t.proc = object()
+    assert t.summary()["sm_mhz"] == 1500.0
+    assert not os.path.exists(t.path)   # its own temporary file is removed
