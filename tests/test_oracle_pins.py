@@ -205,8 +205,9 @@ def test_attention_weights_sum_to_one_and_positive():
         assert np.array_equal(np.argsort(o[i, :C_], kind="stable"), np.argsort(s, kind="stable"))
 
 
-def test_attention_two_positions_sigmoid_closed_form():
-    d, S = 64, 8
+@pytest.mark.parametrize("d", [64, 128])   # the head dims of the 1B and 8B shapes
+def test_attention_two_positions_sigmoid_closed_form(d):
+    S = 8
     c, t = 1.5, 2.0
     q = np.zeros((1, d)); q[0, 0] = c
     kc = np.zeros((1, S, d), np.uint16)
