@@ -24,9 +24,12 @@ does not shard without a per-layer exchange); `value` is then the max rank
 time divided by all ranks' tokens.
 
 --impl reference times the oracle (the plain fp64 CPU definition in
-oracle/) on the host: each step is a bounded sample -- one decoder layer and
-1/L of the LM-head rows of the same shape, weights and positions -- and the
-reported ms/token is that sample's time times L.
+oracle/) on the host, single-threaded and pinned to one core: W untimed and
+then K timed FULL decode steps of the same shape, weights and positions
+(every layer, every LM-head row), stopping early once --ref-budget-s has
+passed (the line's `steps` is then the number actually timed).  The CPU
+baseline leg of the default arm times full oracle steps the same way for
+about --cpu-sample-s seconds (at least 3 steps).
 """
 from __future__ import annotations
 
@@ -178,38 +181,75 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # oracle timing (CPU baseline and the reference arm)
 # ---------------------------------------------------------------------------
-class OracleSample:
-    """One decoder layer plus 1/L of the LM-head rows of `shape`, built from
-    the same weights, so that a step of it costs 1/L of a full oracle step.
-    The KV prefix is seeded N(0,1) data (attention cost depends only on C)."""
+class OracleRunner:
+    """The oracle (the plain fp64 C decode step in oracle/) on the full model
+    of `shape`, same weights, one sequence.  Every timed step is one whole
+    decode step: every layer and every LM-head row.  The KV cache starts
+    from the same seeded prefix the GPU side uses (zeros beyond it)."""
 
-    def __init__(self, shape: wl.ModelShape, bits: dict, max_seq: int):
+    def __init__(self, shape: wl.ModelShape, bits: dict, max_seq: int, prefill: int):
         import oracle
-        L = shape.layers
-        self.L = L
-        vs = max(1, shape.vocab // L)
-        cfg = dict(layers=1, hidden=shape.hidden, n_q_heads=shape.n_q_heads,
+        cfg = dict(layers=shape.layers, hidden=shape.hidden, n_q_heads=shape.n_q_heads,
                    n_kv_heads=shape.n_kv_heads, head_dim=shape.head_dim, ffn=shape.ffn,
-                   vocab=vs, max_seq=max_seq, rope_theta=shape.rope_theta, rms_eps=shape.rms_eps)
-        w = {"embed": bits["embed"][:vs], "lm_head": bits["lm_head"][:vs],
-             "final_norm": bits["final_norm"]}
-        for k in ("attn_norm", "mlp_norm", "wq", "wk", "wv", "wo", "wg", "wu", "wd"):
-            w[k] = [bits[k][0]]
-        self.model = oracle.OracleModel(cfg, w)
+                   vocab=shape.vocab, max_seq=max_seq, rope_theta=shape.rope_theta,
+                   rms_eps=shape.rms_eps)
+        self.model = oracle.OracleModel(cfg, bits)
         self.kc, self.vc = self.model.new_cache()
-        rng = np.random.default_rng(5)
-        for a in self.kc + self.vc:
-            a[...] = (rng.standard_normal(a.shape).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
-        self.vs = vs
+        if prefill:
+            k, v = wl.make_kv(shape, 1, max_seq, device="cpu", prefill_len=prefill)
+            for l in range(shape.layers):
+                self.kc[l][...] = wl.cache_bits(k[l][0])
+                self.vc[l][...] = wl.cache_bits(v[l][0])
+        self.next = 0
 
     def step_ms(self, token: int, pos: int) -> float:
         t0 = time.perf_counter()
-        self.model.decode_step(self.kc, self.vc, int(token) % self.vs, int(pos))
-        return (time.perf_counter() - t0) * 1e3 * self.L
+        out = self.model.decode_step(self.kc, self.vc, int(token), int(pos))
+        dt = (time.perf_counter() - t0) * 1e3
+        self.next = out["next"]
+        return dt
 
 
-def cpu_cores_used() -> int:
-    return 1   # the oracle is single-threaded C
+class PinnedCore:
+    """Pin the calling thread to one core for the duration (the oracle is
+    single-threaded C called from this thread); restores the old mask."""
+
+    def __enter__(self):
+        self.old = None
+        self.core = None
+        try:
+            self.old = os.sched_getaffinity(0)
+            self.core = min(self.old)
+            os.sched_setaffinity(0, {self.core})
+        except (AttributeError, OSError):
+            pass
+        return self
+
+    def __exit__(self, *a):
+        if self.old is not None:
+            try:
+                os.sched_setaffinity(0, self.old)
+            except OSError:
+                pass
+
+
+def host_cores() -> int:
+    return os.cpu_count() or 1
+
+
+def run_oracle_steps(runner: OracleRunner, tokens, positions, n_warm: int, n_max: int,
+                     budget_s: float, min_steps: int = 3):
+    """n_warm untimed full steps, then full steps until n_max steps or the
+    time budget (at least min_steps).  Returns the per-step times (ms)."""
+    for i in range(n_warm):
+        runner.step_ms(tokens[i], positions[i])
+    times = []
+    t_end = time.perf_counter() + budget_s
+    i = n_warm
+    while len(times) < n_max and (len(times) < min_steps or time.perf_counter() < t_end):
+        times.append(runner.step_ms(tokens[i % len(tokens)], positions[i % len(positions)]))
+        i += 1
+    return times
 
 
 # ---------------------------------------------------------------------------
@@ -225,7 +265,10 @@ def parse():
     ap.add_argument("--no-generate", action="store_true",
                     help="skip the one-launch generation measurement")
     ap.add_argument("--e2e-steps", type=int, default=64)
-    ap.add_argument("--cpu-sample-s", type=float, default=15.0)
+    ap.add_argument("--cpu-sample-s", type=float, default=8.0,
+                    help="CPU baseline: time full oracle steps for about this long (at least 3)")
+    ap.add_argument("--ref-budget-s", type=float, default=180.0,
+                    help="--impl reference: stop timing oracle steps after this long")
     ap.add_argument("--flags", type=int, default=0, help="mk_config.flags")
     ap.add_argument("--attn-chunks", type=int, default=0)
     ap.add_argument("--clocks-csv", default=None,
@@ -282,21 +325,26 @@ def main():
         w_host = wl.make_weights(shape, seed=1234, device="cuda" if torch.cuda.is_available() else "cpu")
         bits = w_host.numpy_bits()
         del w_host
-        samp = OracleSample(shape, bits, max_seq)
-        prompt = wl.make_prompt(shape.vocab, W, seed=42)
-        for i in range(W):
-            samp.step_ms(prompt[i], start + i)
-        times = [samp.step_ms(prompt[i % W], start + W + i) for i in range(K)]
-        total = float(np.sum(times))
-        ms = total / K
-        sample = (f"each step: 1 of {shape.layers} decoder layers + 1/{shape.layers} of the LM-head rows, "
-                  f"time x{shape.layers}")
+        runner = OracleRunner(shape, bits, max_seq, prefill)
+        prompt = wl.make_prompt(shape.vocab, W + K, seed=42)
+        positions = np.arange(start, start + W + K)
+        with PinnedCore() as pin:
+            t_run = time.perf_counter()
+            times = run_oracle_steps(runner, prompt, positions, W, K, args.ref_budget_s)
+            t_run = time.perf_counter() - t_run
+        n = len(times)
+        ms = float(np.mean(times))
+        sample = (f"{n} full oracle decode steps (every layer, every LM-head row; fp64 C, "
+                  f"single thread pinned to core {pin.core} of {host_cores()}) after {W} untimed "
+                  f"ones, positions {start + W}..{start + W + n - 1}"
+                  + ("" if n == K else f"; {K} requested, capped by the {args.ref_budget_s:.0f} s budget"))
         out = {"impl": "reference", "metric": METRIC, "value": ms, "unit": UNIT, "n_gpus": world,
-               "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": False,
+               "steps": n, "warmup": W, "ms_per_step": ms, "higher_is_better": False,
                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                "config": config,
-               "cpu_baseline": {"value": ms, "unit": UNIT, "cores": cpu_cores_used(),
-                                "kind": "oracle", "sample": sample},
+               "cpu_baseline": {"value": ms, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": sample, "pinned_core": pin.core, "host_cores": host_cores(),
+                                "wall_s": round(t_run, 2)},
                "e2e": {"value": ms, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(out), flush=True)
         return
@@ -428,22 +476,23 @@ def main():
         gen = {"value": round(job_ms_per_token(gen_ms, K, world), 5), "unit": UNIT, "steps": K, "launches": 1,
                "api": "mk_generate"}
 
-    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1)
+    # ---- CPU baseline: full oracle steps on one pinned core (rank 0, N=1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         bits = weights.numpy_bits()
-        samp = OracleSample(shape, bits, max_seq)
-        times = []
-        t_end = time.perf_counter() + args.cpu_sample_s
-        i = 0
-        while time.perf_counter() < t_end or i < 3:
-            times.append(samp.step_ms(int(toks[W + (i % K)].item()), start + W + (i % K)))
-            i += 1
-        cpu = {"value": round(float(np.mean(times)), 3), "unit": UNIT, "cores": cpu_cores_used(),
-               "kind": "oracle",
-               "sample": f"{i} oracle steps of 1 of {shape.layers} layers + 1/{shape.layers} of the "
-                         f"LM-head rows at positions {start + W}.., time x{shape.layers}; "
-                         f"host has {os.cpu_count()} cores"}
+        runner = OracleRunner(shape, bits, max_seq, prefill)
+        ptoks = toks.cpu().numpy()
+        positions = pos.cpu().numpy()
+        with PinnedCore() as pin:
+            times = run_oracle_steps(runner, ptoks[W:W + K], positions[W:W + K], 0, K,
+                                     args.cpu_sample_s)
+        n = len(times)
+        cpu = {"value": round(float(np.mean(times)), 3), "unit": UNIT, "cores": 1,
+               "kind": "oracle", "pinned_core": pin.core, "host_cores": host_cores(),
+               "sample": f"{n} full oracle decode steps (every layer, every LM-head row; fp64 C, "
+                         f"single thread pinned to core {pin.core} of {host_cores()}) on the timed "
+                         f"steps' tokens at positions {start + W}..{start + W + n - 1}; the oracle's "
+                         f"cache holds the seeded prefix only (attention cost depends on C alone)"}
 
     if rank == 0:
         out = {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world,

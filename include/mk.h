@@ -146,6 +146,14 @@ typedef struct mk_ctx mk_ctx;
  * Validate the shape, build the static task graph for this device (one
  * persistent CTA per SM), allocate scratch and upload the tables.  Blocks
  * the host.  *out receives the context (NULL on error).
+ * The graph is MPK's compile step done once on the host: every op split into
+ * tasks, one event per op whose threshold is the number of tasks that
+ * trigger it ("显著提升小LLM的性能..." page, Figure 2 text on tasks and
+ * events; the MPK walkthrough zizhi168.cn/news/174794, section 3.3.2 on
+ * task-graph generation by compile()), with the tasks placed in static per-SM queues (the Hazy page,
+ * sfrk.com.cn/ruanjian/202506/86466, paragraph on the per-SM execution plan).
+ * The device must be compute capability 10.0 (B200; the library holds sm_100a
+ * code only): any other device gives MK_ERR_INVALID.
  * The q/k/v and gate/up matrices are copied into a library-owned layout
  * (rows in the order the kernel streams them, so every task reads one
  * contiguous range): later changes to those caller buffers are not seen,
@@ -157,7 +165,14 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
 
 /*
  * One decode step for sequences 0..batch-1, enqueued on `stream` (one
- * kernel launch; asynchronous).
+ * kernel launch; asynchronous).  The step is the decoder layer sequence of
+ * the Hazy megakernel page (sfrk.com.cn/ruanjian/202506/86466, paragraph
+ * listing the fused instructions: RMSNorm + QKV + RoPE, attention and its
+ * reduction, O-projection + residual, RMSNorm + gate/up + SiLU, down +
+ * residual) and of the MPK walkthrough's per-layer *_layer calls
+ * (zizhi168.cn/news/174794, section 3.3.1), ending in the final RMSNorm, the
+ * LM head and argmax (same walkthrough, the argmax_partial / argmax_reduce
+ * layers).
  *   tokens    device int32 [batch]: input token of each sequence.
  *   positions device int32 [batch]: position of that token; its K/V entry
  *             is written at that slot of every layer's cache and attention
@@ -319,11 +334,20 @@ int mk_plan(const mk_config *cfg, int num_sms, mk_info *info,
  * with MK_ERR_INVALID (the 1B shape needs about 3.2 MiB at max_seq 560 and
  * 8.0 MiB at max_seq 16640).
  * Every call shares that array and leaves its last contents there: calls
- * that overlap on the GPU (several streams or host threads) race.  The
- * first call on a device looks up the array's address and sets up the
- * kernel for that device (and uploads the task tables when the shape
- * changes, synchronising the stream); make that first call before any
- * stream capture.  MK_FLAG_TRACE is not supported here.
+ * on the same device that overlap on the GPU (several streams or host
+ * threads) race.  Each device has its own array; the host-side staging of
+ * the tables is serialised by a lock, so host threads driving different
+ * devices do not interfere.  The first call on a device looks up the
+ * array's address and sets up the kernel for that device; a call whose shape
+ * differs from the previous call's on that device uploads new task and RoPE
+ * tables, and a call whose weight or KV pointers differ uploads a new layer
+ * table -- both synchronise the stream, so make such calls outside stream
+ * capture (the first call on a device included).  The tables carry a key
+ * that the kernel compares with the key its launch was set up with: a
+ * launch set up for tables that have been replaced since (a replay of an
+ * earlier launch) runs nothing and reports MK_ERR_INVALID through
+ * status_out.
+ * MK_FLAG_TRACE is not supported here.
  *
  * Weights come already in the kernel's streaming layout (mk_create makes
  * this copy itself; this entry point cannot allocate one):

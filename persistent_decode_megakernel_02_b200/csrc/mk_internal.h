@@ -274,6 +274,11 @@ struct Params {
     int event_wait;              // 1: the scheduler gates tasks on event counters
     int debug_withhold;          // test hook: tasks triggering this event write stale tags (-1: off)
     unsigned int poll_ns;        // pause between polls of stale input words
+    // tables shared between calls (the no-allocation entry point): the key
+    // of the tables currently uploaded, and the key this launch was built
+    // for; a mismatch refuses the step (MK_ERR_INVALID).  Null: no check.
+    const uint64_t *table_key;
+    uint64_t expect_key;
 };
 
 // ---- host planning -------------------------------------------------------------

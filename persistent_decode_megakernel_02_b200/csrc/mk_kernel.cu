@@ -1884,6 +1884,16 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
         ctl->loader_done = 0;
         ctl->ep = ld_volatile_u32(p.epoch) + 1u;
         uint32_t stop = ld_volatile_u32(p.abort_flag) ? 1u : 0u;
+        if (!stop && p.table_key && *(const volatile uint64_t *)p.table_key != p.expect_key) {
+            // the shared tables were rebuilt for another shape or other
+            // weights since this launch was set up: run nothing
+            if (atomicCAS(&p.err->code, 0u, kErrInvalid) == 0u) {
+                p.err->task = 0xffffffffu;
+                p.err->where = W_INPUT;
+                p.err->info = 0xfffffffeu;
+            }
+            stop = 1u;
+        }
         ctl->tq_pub = 0;
         ctl->tq_reads = 0;
         ctl->stop = 0;

@@ -162,7 +162,9 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     if (cudaGetDevice(&dev) != cudaSuccess) return MK_ERR_CUDA;
     cudaDeviceProp prop;
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MK_ERR_CUDA;
-    if (prop.major < 10) return MK_ERR_INVALID;     // built for sm_100a only
+    // the binary holds sm_100a code only (arch-specific: it runs on compute
+    // capability 10.0 exactly, not on other Blackwell parts)
+    if (prop.major != 10 || prop.minor != 0) return MK_ERR_INVALID;
     if (!prop.cooperativeLaunch) return MK_ERR_INVALID;
     if ((size_t)prop.sharedMemPerBlockOptin < kernel_smem_bytes()) return MK_ERR_INVALID;
     // The worker/control register split is only safe with the launch

@@ -14,16 +14,24 @@
 // staging of the tables uses static host storage.
 //
 // Every call shares that array and leaves the last call's contents in it;
-// calls that overlap on the GPU (different streams, or several host threads)
-// race on it.  The first call on a device looks up the array's device
-// address with cudaGetSymbolAddress (with that device current) and sets the
-// kernel's shared-memory attribute; make that first call before any stream
-// capture.
+// calls on the same device that overlap on the GPU (different streams, or
+// several host threads) race on it.  Each device has its own copy of the
+// array; the host-side staging is one static buffer guarded by a mutex, so
+// host threads driving different devices do not mix their tables.  The first
+// call on a device looks up the array's device address with
+// cudaGetSymbolAddress (with that device current) and sets the kernel's
+// shared-memory attribute; a call whose shape, weights or KV cache differ
+// from the previous call's on that device uploads new tables and
+// synchronises the stream.  Make such calls outside stream capture.  The
+// uploaded tables carry a key the kernel checks against the key its launch
+// was set up with: a launch set up for tables that have been replaced since
+// (a replay of an earlier launch) runs nothing and reports MK_ERR_INVALID.
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/mk.h"
 #include "mk_internal.h"
@@ -53,8 +61,10 @@ struct DeviceSetup {
 };
 DeviceSetup g_dev[kMaxDevices];
 
-// Host staging of the tables (static storage; no allocation).
+// Host staging of the tables (static storage; no allocation), shared by all
+// devices and guarded by g_host_mutex for the whole host section of a call.
 alignas(256) unsigned char g_host[MK_STATIC_SCRATCH_BYTES];
+std::mutex g_host_mutex;
 
 // What the tables currently in a device's scratch were built from: a hash of
 // the shape (task graph, RoPE table) and a hash of the layer pointer table.
@@ -80,7 +90,8 @@ uint64_t shape_key(const mk_config *c, int num_sms) {
 }
 
 struct Layout {
-    size_t tasks, queue, qtasks, qoff, thr, events, ctrl, err, tag, toktag, layers, rope;
+    size_t key,      // uint64: key of the tables below (checked by the kernel)
+        tasks, queue, qtasks, qoff, thr, events, ctrl, err, tag, toktag, layers, rope;
     size_t aval, aidx, end;
 };
 
@@ -116,6 +127,7 @@ Layout layout_for(const Shape &s, const PlanSizes &z, int num_sms, int num_lm_ta
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
     const size_t B = s.Bmax;
+    l.key = take(sizeof(uint64_t));
     l.tasks = take(sizeof(Task) * z.num_tasks);
     l.queue = take(sizeof(int32_t) * z.num_tasks);
     l.qtasks = take(sizeof(Task) * z.num_tasks);
@@ -147,6 +159,7 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MK_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return MK_ERR_INVALID;
+    std::lock_guard<std::mutex> lock(g_host_mutex);
     DeviceSetup &ds = g_dev[dev];
     if (!ds.ready) {
         // once per device, with that device current
@@ -154,7 +167,7 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
         if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return MK_ERR_CUDA;
         cudaDeviceProp prop;
         if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MK_ERR_CUDA;
-        if (prop.major < 10 || !prop.cooperativeLaunch) return MK_ERR_INVALID;
+        if (prop.major != 10 || prop.minor != 0 || !prop.cooperativeLaunch) return MK_ERR_INVALID;
         if ((size_t)prop.sharedMemPerBlockOptin < kernel_smem_bytes()) return MK_ERR_INVALID;
         if (kernel_launch_regs() != kLaunchRegs) return MK_ERR_INVALID;
         if (kernel_prepare() != cudaSuccess) return MK_ERR_CUDA;
@@ -236,7 +249,11 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
         sig.valid = true;
     }
     if (sig.layer_key != lkey) {
+        // the layer table, then the key that names the whole table set
+        uint64_t *hkey = reinterpret_cast<uint64_t *>(g_host + lay.key);
+        *hkey = lkey;
         if (cudaMemcpyAsync(d + lay.layers, lw, sizeof(LayerW) * s.L, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+            cudaMemcpyAsync(d + lay.key, hkey, sizeof(uint64_t), cudaMemcpyHostToDevice, st) != cudaSuccess ||
             cudaStreamSynchronize(st) != cudaSuccess) {
             sig.valid = false;
             return MK_ERR_CUDA;
@@ -290,6 +307,8 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
     p.event_wait = (cfg->flags & MK_FLAG_EVENT_WAIT) ? 1 : 0;
     p.debug_withhold = -1;
     p.poll_ns = (unsigned int)cfg->poll_ns;
+    p.table_key = reinterpret_cast<const uint64_t *>(d + lay.key);
+    p.expect_key = lkey;
     if (kernel_launch(p, ds.num_sms, st) != cudaSuccess) return MK_ERR_CUDA;
     if (status_out &&
         cudaMemcpyAsync(status_out, d + lay.err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)

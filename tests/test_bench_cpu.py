@@ -2,6 +2,7 @@
 import json
 import os
 
+import numpy as np
 import torch
 
 import bench
@@ -68,3 +69,21 @@ def test_clock_summary_flags_thermal_slowdown_and_missing_samples(tmp_path):
     t.proc = object()
     assert t.summary()["sm_mhz"] == 1500.0
     assert not os.path.exists(t.path)   # its own temporary file is removed
+
+
+def test_oracle_baseline_times_full_steps_pinned_to_one_core():
+    # the CPU baseline and the reference arm time whole oracle decode steps
+    # (every layer and LM-head row), on one pinned core, and restore the mask
+    import os
+    shape = wl.TINY
+    w = wl.make_weights(shape, seed=3, device="cpu")
+    runner = bench.OracleRunner(shape, w.numpy_bits(), 32, 0)
+    before = os.sched_getaffinity(0)
+    with bench.PinnedCore() as pin:
+        assert os.sched_getaffinity(0) == {pin.core}
+        times = bench.run_oracle_steps(runner, [5, 6, 7, 8, 9], list(range(5)), 2, 10, 0.0)
+    assert os.sched_getaffinity(0) == before
+    # budget 0: the minimum of 3 timed steps after the 2 warm-up ones
+    assert len(times) == 3 and all(t > 0 for t in times)
+    # the runner's cache advanced through every step: position 4 was written
+    assert any(np.any(k[:, 4] != 0) for k in runner.kc)

@@ -77,8 +77,38 @@ def test_tiny_random_gains_untied_head_and_intermediates(flags):
     _check_hidden(pair, ref)
 
 
-@pytest.mark.parametrize("chunks", [1, 3, 13, 64])
-def test_attention_chunking_does_not_change_results(chunks):
+# Split-K attention with many ACTIVE chunks: a step uses ceil(C / 1024)
+# chunks (at most attn_chunks), so each case prefills a random cache long
+# enough that every configured chunk holds positions and chunk 0's task merges
+# all of them.  124 chunks is the most the merge stage holds at head_dim 64
+# (124 * 66 <= 8192 floats), 63 at head_dim 128.
+TINY_D128 = wl.ModelShape("tiny-d128", 2, 256, 2, 1, 128, 768, 4096, True, 1e4)
+
+
+@pytest.mark.parametrize("head_dim,chunks,prefix", [(64, 13, 13000), (64, 40, 40000),
+                                                    (64, 124, 126000), (128, 63, 64000)])
+def test_many_active_attention_chunks_merged(head_dim, chunks, prefix):
+    shape = wl.TINY if head_dim == 64 else TINY_D128
+    S = prefix + 8
+    pair = Pair(shape, max_seq=S, prefill_len=prefix, attn_chunks=chunks)
+    assert pair.ctx.info().attn_chunks == chunks
+    assert -(-(prefix + 1) // 1024) >= chunks      # every chunk is active
+    toks = wl.make_prompt(shape.vocab, 3, seed=11)
+    for i, t in enumerate(toks):
+        pos = prefix + i
+        g_tok, g_log = pair.gpu_step(int(t), pos)
+        ref = pair.ref_step(int(t), pos, intermediates=True)
+        _check_step(pair, pos, g_tok, g_log, ref)
+        got = pair.ctx.read_buffer(pair.mk.MK_BUF_ATTN, ref["attn"].size).astype(np.float64)
+        assert rel_l2(got, ref["attn"]) <= 5e-3
+    _check_hidden(pair, ref)
+
+
+@pytest.mark.parametrize("chunks", [1, 3, 64])
+def test_short_contexts_with_more_chunks_than_positions(chunks):
+    # contexts of at most 40 positions use one active chunk whatever the
+    # configured count; the other chunks' items find no positions and must
+    # write nothing (and their empty partials must not reach a merge)
     shape = wl.TINY
     pair = Pair(shape, max_seq=96, attn_chunks=chunks)
     toks = wl.make_prompt(shape.vocab, 40, seed=11)
@@ -209,16 +239,34 @@ def test_trace_records_respect_dependencies(flags):
 
 
 @pytest.mark.slow
-def test_llama1b_shape_teacher_forced():
+def test_llama1b_shape_prompt_of_39_then_decode():
+    # the benchmark's workload from its first position: a 39-token prompt
+    # teacher-forced, then decode steps at positions 39..43
     shape = wl.LLAMA_1B
     pair = Pair(shape, max_seq=560)
-    prompt = wl.make_prompt(shape.vocab, 6, seed=42)
+    prompt = wl.make_prompt(shape.vocab, 39, seed=42)
     n = 0
-    for step, pos, g_tok, g_log, ref in pair.teacher_forced(prompt, 3):
+    for step, pos, g_tok, g_log, ref in pair.teacher_forced(prompt, 5):
         _check_step(pair, step, g_tok, g_log, ref)
         n += 1
+    assert n == 44 and pos == 43
     _check_hidden(pair, ref)
     _check_events(pair, n)
+
+
+@pytest.mark.slow
+def test_llama1b_shape_at_the_end_of_the_benchmark_range():
+    # positions 540..545 (the bench's 512 decode steps end at 550) over a
+    # seeded random prefix of 540 positions
+    shape = wl.LLAMA_1B
+    pair = Pair(shape, max_seq=560, prefill_len=540)
+    prompt = wl.make_prompt(shape.vocab, 1, seed=8)
+    n = 0
+    for step, pos, g_tok, g_log, ref in pair.teacher_forced(prompt, 5, start_pos=540):
+        _check_step(pair, pos, g_tok, g_log, ref)
+        n += 1
+    assert n == 6
+    _check_hidden(pair, ref)
 
 
 @pytest.mark.slow
