@@ -72,7 +72,15 @@ enum mk_flags {
      * it tasks wait on their inputs directly: every activation is stored
      * with the step's tag in the same 64-bit word and readers poll the tags.
      * Results are identical either way; the counters are bumped either way. */
-    MK_FLAG_EVENT_WAIT = 4
+    MK_FLAG_EVENT_WAIT = 4,
+    /* Stream every weight page through shared memory only.  By default the
+     * pages of the matrix-vector ops whose rows are multiples of 2048
+     * columns (hidden, n_q_heads*head_dim or ffn of 2048, 4096 or 8192) are
+     * copied on from the shared-memory ring into tensor memory as soon as
+     * they land, which frees the ring for further prefetch (7 pages of
+     * 64 KB buffered per SM instead of 3); mk_create then keeps those
+     * weights in a library-owned copy laid out for that copy. */
+    MK_FLAG_NO_TMEM_RING = 8
 };
 
 /* Upper bounds of the shapes the kernel tiles. */
@@ -156,9 +164,12 @@ typedef struct mk_ctx mk_ctx;
  * code only): any other device gives MK_ERR_INVALID.
  * The q/k/v and gate/up matrices are copied into a library-owned layout
  * (rows in the order the kernel streams them, so every task reads one
- * contiguous range): later changes to those caller buffers are not seen,
- * and device memory grows by their size.  The other weights and the KV
- * cache are used in place.
+ * contiguous range); unless MK_FLAG_NO_TMEM_RING is set, so are the other
+ * matrices whose pages pass through tensor memory (O-projection, down
+ * projection, LM head, in the TMEM page order).  Later changes to copied
+ * caller buffers are not seen, and device memory grows by their size.  The
+ * embedding table (also when tied to the LM head), the RMSNorm gains and
+ * the KV cache are always used in place.
  * Errors: MK_ERR_INVALID (shape or pointer checks), MK_ERR_OOM, MK_ERR_CUDA.
  */
 int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx **out);
@@ -247,7 +258,8 @@ typedef struct mk_info {
     int max_queue;      /* longest per-SM task queue */
     int page_bytes, num_pages;
     long long steps_run; /* decode steps enqueued since create/reset (mk_generate adds n_steps) */
-    unsigned int err_code, err_info; /* device error word (0 = none) */
+    unsigned int err_code, err_info; /* device error word (0 = none); err_info = which wait << 24 | detail */
+    unsigned int err_task;           /* task id the device error was raised in (0xffffffff: none) */
 } mk_info;
 
 int mk_get_info(mk_ctx *ctx, mk_info *out);

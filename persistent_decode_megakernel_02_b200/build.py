@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmk.so")
 SOURCES = ["mk_kernel.cu", "mk_runtime.cpp", "mk_graph.cpp", "mk_static.cu"]
-HEADERS = ["mk_internal.h"]
+HEADERS = ["mk_internal.h", "mk_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

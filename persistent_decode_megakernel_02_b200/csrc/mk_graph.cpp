@@ -30,13 +30,26 @@ int default_attn_chunks(int num_sms, int Bmax, int nq, int S) {
     return nc;
 }
 
+// Tiles per scheduling unit of a GEMV op: tasks of ops whose pages pass
+// through tensor memory must start on a 16-page-row boundary (the TMEM page
+// order is laid out on that grid), so 8-row tiles of 2048 columns go in pairs.
+static int gemv_unit(const Shape &s, int kind) {
+    if (!tmem_page_op(s, kind)) return 1;
+    const int page_rows_per_tile = tile_rows(s, kind, 0) * (op_k(s, kind) / kRowK);
+    return page_rows_per_tile < 16 ? 16 / page_rows_per_tile : 1;
+}
+
 PlanSizes plan_sizes(const Shape &s, int num_sms) {
     OpTiles t = op_tiles(s);
-    auto ntask = [&](int tiles) { return tiles < num_sms ? tiles : num_sms; };
+    auto ntask = [&](int kind, int tiles) {
+        const int u = gemv_unit(s, kind);
+        const int units = (tiles + u - 1) / u;
+        return units < num_sms ? units : num_sms;
+    };
     PlanSizes z;
-    int per_layer = ntask(t.qkv) + t.attn_items + ntask(t.oproj) +
-                    ntask(t.gateup) + ntask(t.down);
-    z.num_tasks = s.L * per_layer + ntask(t.lmhead);
+    int per_layer = ntask(OP_QKV, t.qkv) + t.attn_items + ntask(OP_OPROJ, t.oproj) +
+                    ntask(OP_GATEUP, t.gateup) + ntask(OP_DOWN, t.down);
+    z.num_tasks = s.L * per_layer + ntask(OP_LMHEAD, t.lmhead);
     z.num_events = 5 * s.L + 1;
     z.num_ops = 5 * s.L + 1;
     return z;
@@ -79,16 +92,20 @@ struct Builder {
     }
 
     // Split the op's `ntiles` tiles over the least-loaded SMs, one
-    // contiguous tile range per task, with equal tile counts (+-1).
-    // Returns the number of tasks.
+    // contiguous tile range per task, with equal unit counts (+-1) (a unit
+    // is one tile, or two 8-row tiles when pages pass through tensor
+    // memory).  Returns the number of tasks.
     int gemv_op(int kind, int layer, int dep, int trig, int ntiles) {
         const int K = op_k(s, kind);
-        int T = ntiles < p.num_sms ? ntiles : p.num_sms;
-        int base = ntiles / T, extra = ntiles % T;
+        const int unit = gemv_unit(s, kind);
+        const int nunits = (ntiles + unit - 1) / unit;
+        int T = nunits < p.num_sms ? nunits : p.num_sms;
+        int base = nunits / T, extra = nunits % T;
         sort_by_load();
         int tile = 0;
         for (int i = 0; i < T; ++i) {
-            int n = base + (i < extra ? 1 : 0);
+            int n = (base + (i < extra ? 1 : 0)) * unit;
+            if (tile + n > ntiles) n = ntiles - tile;
             long long rows = tile_row_offset(s, kind, tile + n) - tile_row_offset(s, kind, tile);
             if (kind == OP_LMHEAD) {
                 long long valid = (long long)s.V - tile_row_offset(s, kind, tile);

@@ -26,6 +26,7 @@ constexpr int kWorkerWarps = 8;                     // run task bodies
 constexpr int kWorkerThreads = kWorkerWarps * 32;   // 256
 constexpr int kLoaderWarp = kWorkerWarps;           // streams weight pages
 constexpr int kSchedWarp = kWorkerWarps + 1;        // waits on events (when gating by events)
+constexpr int kStashWarp = kWorkerWarps + 2;        // moves landed weight pages into tensor memory
 constexpr int kThreads = (kWorkerWarps + 4) * 32;   // 384
 constexpr int kLaunchRegs = 168;
 constexpr int kWorkerRegs = 224;
@@ -49,6 +50,12 @@ constexpr int kAttnChunkPositions = 1024;
 constexpr int kMaxHeadDim = 256;
 constexpr long long kL2Lookahead = 0;  // default L2 prefetch distance beyond the ring (0: off; measured no gain)
 constexpr int kStageFloats = 8192;  // shared staging: a GEMV input vector, or attention partials
+// Tensor memory as a second level of the weight ring: the whole 512-column
+// allocation of the SM, as kTmemSlots slots of one 64 KB page each (a page of
+// 16 rows of 2048 bf16 columns occupies 128 lanes x 128 columns).
+constexpr int kTmemCols = 512;
+constexpr int kTmemSlots = 4;
+constexpr int kTmemSlotCols = kTmemCols / kTmemSlots;
 
 // ---- ops ---------------------------------------------------------------------
 enum OpKind : int32_t { OP_QKV = 0, OP_ATTN = 1, OP_OPROJ = 2, OP_GATEUP = 3, OP_DOWN = 4, OP_LMHEAD = 5 };
@@ -83,6 +90,8 @@ struct LayerW {
 // Sizes derived from the model shape.
 struct Shape {
     int L, H, nq, nkv, d, F, V, S, Bmax, NC;
+    int tmem;         // 1: GEMV pages of 2048-column rows pass through tensor memory
+                      //    (weights in the TMEM page order, tasks start on page boundaries)
     int G;            // nq / nkv
     int QD, KD;       // nq*d, nkv*d
     float theta, eps;
@@ -136,6 +145,33 @@ MK_HD inline int tile_rows(const Shape &s, int kind, int tile) {
 constexpr int kRowK = 2048;
 MK_HD inline bool rows_gemv(int K) { return K <= kRowK || K == 2 * kRowK || K == 4 * kRowK; }
 constexpr int kMaxHidden = 4096;   // MK_MAX_HIDDEN: the largest hidden size the tests cover
+
+// GEMV ops whose pages are 16 "page rows" of 2048 columns (K = 2048, 4096,
+// 8192): with Shape::tmem these pages are staged in tensor memory, and the
+// weights are stored in the TMEM page order (tmem_page_src below).
+MK_HD inline bool tmem_page_op(const Shape &s, int kind) {
+    const int K = op_k(s, kind);
+    return s.tmem && kind != OP_ATTN && K % kRowK == 0 && rows_gemv(K);
+}
+
+// The TMEM page order.  A page of 16 page rows (each 2048 bf16 = 256
+// vectors of 16 bytes) is stored as 16 blocks of 4 KB; tcgen05.cp of block c
+// (128x256b, no swizzle, stride offset 128 B, leading offset 2048 B) puts
+// the 16-byte pieces at 512p + 16L and 2048 + 512p + 16L of the block into
+// TMEM lane 32p + L, columns 8c..8c+3 and 8c+4..8c+7.  Block c holds page
+// row (c / 8) * 8 + p + 4 * ((c / 4) % 2), vectors L + 32 * (2 * (c % 4) + q)
+// for the piece q, so that worker warp w reads page rows w and 8 + w (the
+// rows the shared-memory path gives it) as 32 consecutive columns each from
+// its own lane quarter (w % 4), lane L getting vectors L, L + 32, ..., L + 224
+// in order -- and rows 0..7 sit in the first 32 KB (a trailing 8-row page is
+// one half-size copy).
+// tmem_page_src: the source (page row, vector) of destination vector u
+// (0..4095) of a page.
+MK_HD inline void tmem_page_src(int u, int &row, int &vec) {
+    const int c = u >> 8, q = (u >> 7) & 1, p = (u >> 5) & 3, L = u & 31;
+    row = (c >> 3) * 8 + p + 4 * ((c >> 2) & 1);
+    vec = L + 32 * (2 * (c & 3) + q);
+}
 
 // Rows of one page: the largest power of two <= 16 whose rows (K bf16 each)
 // fit in a page (16 for K <= 2048: one page holds a whole 16-row unit).

@@ -48,6 +48,7 @@
 #include <stdint.h>
 
 #include "mk_internal.h"
+#include "mk_ptx.cuh"
 
 namespace mk {
 
@@ -56,156 +57,10 @@ constexpr uint32_t kErrInvalid = 1, kErrTimeout = 3;
 enum Where : uint32_t { W_DEP = 1, W_READY = 2, W_FULL = 3, W_EMPTY = 4, W_WBAR = 5,
                         W_INPUT = 6, W_DRAIN = 7, W_TAG = 8 };
 
-// ---------------------------------------------------------------------------
-// PTX helpers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_addr(dst)),
-        "l"(src), "r"(bytes), "r"(smem_addr(bar))
-        : "memory");
-}
-// Same, with an L2 cache policy (createpolicy) for the source lines.
-__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
-                                              uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-            smem_addr(dst)),
-        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
-        : "memory");
-}
-// Weights are read once per step: their lines should leave L2 first.
-__device__ __forceinline__ uint64_t policy_evict_first() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void red_release_gpu(uint32_t *p, uint32_t v) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t atom_add_acqrel_gpu(uint32_t *p, uint32_t v) {
-    uint32_t old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
-}
-__device__ __forceinline__ uint32_t ld_acquire_cta_shared(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_cta_shared(uint32_t *p, uint32_t v) {
-    asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
-}
-__device__ __forceinline__ unsigned long long globaltimer() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t *p) {
-    return *(const volatile uint32_t *)p;
-}
-// Tagged activation words: value bits low, step tag high, one 64-bit access
-// (single-copy atomic), so a reader that sees the tag sees the value.  The
-// loads are volatile (re-issued on every poll, kept in order among
-// themselves) but carry no memory clobber, so the compiler may issue a
-// batch of them before the shared-memory stores that consume the results.
-__device__ __forceinline__ void st_tag(uint64_t *p, float v, uint32_t ep) {
-    const uint64_t w = ((uint64_t)ep << 32) | __float_as_uint(v);
-    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
-}
 // The same value into every copy of a replicated tagged vector.
 __device__ __forceinline__ void st_tag_rep(uint64_t *p, size_t stride, float v, uint32_t ep) {
 #pragma unroll 1
     for (int r = 0; r < kReplicas; ++r) st_tag(p + r * stride, v, ep);
-}
-__device__ __forceinline__ ulonglong2 ld_tag2(const uint64_t *p) {
-    ulonglong2 v;
-    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p));
-    return v;
-}
-__device__ __forceinline__ uint64_t ld_tag1(const uint64_t *p) {
-    uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p));
-    return v;
-}
-// The tag half of a tagged word alone (polling without keeping values).
-__device__ __forceinline__ uint32_t ld_tag_hi(const uint64_t *p) {
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(reinterpret_cast<const char *>(p) + 4));
-    return v;
-}
-__device__ __forceinline__ bool tag_ok(uint64_t w, uint32_t ep) { return (uint32_t)(w >> 32) == ep; }
-__device__ __forceinline__ float tag_val(uint64_t w) { return __uint_as_float((uint32_t)w); }
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-__device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
-__device__ __forceinline__ uint16_t f2bf(float f) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
-}
-__device__ __forceinline__ float dot8(const uint4 w, const float *x) {
-    float a = bf_lo(w.x) * x[0];
-    a = fmaf(bf_hi(w.x), x[1], a);
-    a = fmaf(bf_lo(w.y), x[2], a);
-    a = fmaf(bf_hi(w.y), x[3], a);
-    a = fmaf(bf_lo(w.z), x[4], a);
-    a = fmaf(bf_hi(w.z), x[5], a);
-    a = fmaf(bf_lo(w.w), x[6], a);
-    a = fmaf(bf_hi(w.w), x[7], a);
-    return a;
-}
-// Packed two-lane fp32 FMA (sm_100): d = a * b + c element-wise on pairs.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-// acc += w (8 bf16) . x (8 fp32), two interleaved partial sums (even, odd)
-__device__ __forceinline__ float2 dot8x2(const uint4 w, const float *x, float2 acc) {
-    acc = ffma2(make_float2(bf_lo(w.x), bf_hi(w.x)), make_float2(x[0], x[1]), acc);
-    acc = ffma2(make_float2(bf_lo(w.y), bf_hi(w.y)), make_float2(x[2], x[3]), acc);
-    acc = ffma2(make_float2(bf_lo(w.z), bf_hi(w.z)), make_float2(x[4], x[5]), acc);
-    acc = ffma2(make_float2(bf_lo(w.w), bf_hi(w.w)), make_float2(x[6], x[7]), acc);
-    return acc;
 }
 
 // ---------------------------------------------------------------------------
@@ -224,8 +79,19 @@ struct TaskRec {
 constexpr int kTaskRing = 8;        // task records the loader may publish ahead
 
 struct __align__(16) SmemCtl {
+    // Every page that lands in a slot completes exactly one of two barriers:
+    // full (a page the workers read from shared memory) or tland (a page the
+    // stasher copies on into tensor memory), so that each consumer waits on
+    // a barrier whose every phase is one of its own pages -- a consumer that
+    // skips the other kind of page can never find its barrier two phases
+    // behind (mbarrier parity waits cannot tell those apart).
     uint64_t full[kNumPages];
+    uint64_t tland[kNumPages];
     uint64_t empty[kNumPages];
+    uint64_t cpdone[kNumPages];   // a page copied on into tensor memory has been read
+    uint64_t tfull[kTmemSlots];   // a TMEM slot holds a page
+    uint64_t tempty[kTmemSlots];  // the workers are done with a TMEM slot
+    uint32_t tmem_base;           // tensor-memory address of the allocation
     uint64_t wbar;              // worker barrier, one arrival per worker warp
     uint32_t ready_upto;        // tasks of this queue activated by the scheduler
     uint32_t abort;             // this CTA is bailing out
@@ -426,18 +292,39 @@ struct Ring {
     uint32_t seq = 0;     // pages issued
     bool stats = false;
     unsigned long long t_empty = 0;
+    // per slot: how its last occupant is released (by the workers through
+    // `empty`, or -- a page moved on into tensor memory -- by the stasher's
+    // copy completion through `cpdone`), and how often each barrier has
+    // completed so far (its next wait's parity)
+    uint32_t via_tmem = 0;   // bit s: slot s's last page went to TMEM
+    uint32_t odd_empty = 0;  // bit s: pages of slot s released through `empty` so far, mod 2
+    uint32_t odd_cp = 0;     // bit s: pages of slot s released through `cpdone` so far, mod 2
 };
 
-// Wait for a free page, then arm its full barrier for `bytes`.
+// Wait until the slot's previous page has been released, then arm the
+// slot's landing barrier for `bytes` and return it in `bar` (the copies of
+// the page complete on it).  `to_tmem`: this page will be copied on into
+// tensor memory (landing on tland, released by the stasher) rather than read
+// by the workers (landing on full, released by them).
 __device__ __forceinline__ bool ring_acquire(const Params &p, SmemCtl *ctl, Ring &r, uint32_t bytes,
-                                             uint32_t task, uint32_t &slot) {
+                                             uint32_t task, uint32_t &slot, bool to_tmem, uint64_t *&bar) {
     slot = r.seq % kNumPages;
-    const uint32_t par = ((r.seq / kNumPages) & 1u) ^ 1u;
     const unsigned long long t0 = r.stats ? globaltimer() : 0ull;
-    const bool ok = wait_mbar(&ctl->empty[slot], par, p, ctl, W_EMPTY, task);
+    bool ok = true;
+    if (r.seq >= (uint32_t)kNumPages) {
+        // the m-th release through a barrier completes its phase m - 1:
+        // wait on parity (m - 1) & 1 = (m & 1) ^ 1
+        if (r.via_tmem & (1u << slot))
+            ok = wait_mbar(&ctl->cpdone[slot], ((r.odd_cp >> slot) & 1u) ^ 1u, p, ctl, W_EMPTY, task);
+        else
+            ok = wait_mbar(&ctl->empty[slot], ((r.odd_empty >> slot) & 1u) ^ 1u, p, ctl, W_EMPTY, task);
+    }
     if (r.stats) r.t_empty += globaltimer() - t0;
     if (!ok) return false;
-    mbar_arrive_expect_tx(&ctl->full[slot], bytes);
+    if (to_tmem) { r.via_tmem |= 1u << slot; r.odd_cp ^= 1u << slot; }
+    else { r.via_tmem &= ~(1u << slot); r.odd_empty ^= 1u << slot; }
+    bar = to_tmem ? &ctl->tland[slot] : &ctl->full[slot];
+    mbar_arrive_expect_tx(bar, bytes);
     ++r.seq;
     return true;
 }
@@ -505,21 +392,24 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
                 const int n = min(npp, a.c0 + a.npre - pos0);
                 const uint32_t bytes = (uint32_t)n * p.s.d * 2;
                 uint32_t slot;
-                if (!ring_acquire(p, ctl, ring, 2 * bytes, (uint32_t)id, slot)) { ok = false; break; }
+                uint64_t *bar;
+                if (!ring_acquire(p, ctl, ring, 2 * bytes, (uint32_t)id, slot, false, bar)) { ok = false; break; }
                 unsigned char *dst = pages + (size_t)slot * kPageBytes;
                 const size_t off = (head_off + pos0) * p.s.d;
-                bulk_g2s(dst, L.kc + off, bytes, &ctl->full[slot]);
-                bulk_g2s(dst + (size_t)npp * p.s.d * 2, L.vc + off, bytes, &ctl->full[slot]);
+                bulk_g2s(dst, L.kc + off, bytes, bar);
+                bulk_g2s(dst + (size_t)npp * p.s.d * 2, L.vc + off, bytes, bar);
             }
             continue;
         }
         GemvStream g = gemv_stream(p, t);
+        const bool to_tmem = tmem_page_op(p.s, t.kind);
         for (int k = 0; k < g.npages; ++k) {
             const uint32_t bytes = (uint32_t)max(0LL, min((long long)g.page_bytes, g.left));
             if (p.l2_lookahead) prefetch_to(issued + bytes + p.l2_lookahead);
             uint32_t slot;
-            if (!ring_acquire(p, ctl, ring, bytes, (uint32_t)id, slot)) { ok = false; break; }
-            if (bytes) bulk_g2s_hint(pages + (size_t)slot * kPageBytes, g.src, bytes, &ctl->full[slot], wpol);
+            uint64_t *bar;
+            if (!ring_acquire(p, ctl, ring, bytes, (uint32_t)id, slot, to_tmem, bar)) { ok = false; break; }
+            if (bytes) bulk_g2s_hint(pages + (size_t)slot * kPageBytes, g.src, bytes, bar, wpol);
             g.src += g.page_bytes;
             g.left -= bytes;
             issued += bytes;
@@ -527,12 +417,16 @@ __device__ void loader_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
     }
     *(volatile uint32_t *)&ctl->loader_done = 1u;
     // Let every copy already issued land before this thread returns, so no
-    // bulk copy can still be writing shared memory when the CTA exits.
-    const uint32_t seq = ring.seq;
-    const uint32_t first = seq > (uint32_t)kNumPages ? seq - kNumPages : 0u;
-    for (uint32_t k = first; k < seq; ++k) {
+    // bulk copy can still be writing shared memory when the CTA exits: the
+    // last page of each used slot has completed its landing barrier (the
+    // m-th arming of a barrier completes its phase m - 1).
+    const uint32_t used = ring.seq < (uint32_t)kNumPages ? ring.seq : (uint32_t)kNumPages;
+    for (uint32_t sl = 0; sl < used; ++sl) {
+        const bool t = (ring.via_tmem >> sl) & 1u;
+        uint64_t *bar = t ? &ctl->tland[sl] : &ctl->full[sl];
+        const uint32_t par = (((t ? ring.odd_cp : ring.odd_empty) >> sl) & 1u) ^ 1u;
         Spin s;
-        while (!mbar_try_wait(&ctl->full[k % kNumPages], (k / kNumPages) & 1u)) {
+        while (!mbar_try_wait(bar, par)) {
             if ((++s.n & 127u) == 0u) {
                 unsigned long long now = globaltimer();
                 if (s.t0 == 0) s.t0 = now;
@@ -575,6 +469,70 @@ __device__ void scheduler_role(const Params &p, SmemCtl *ctl, uint32_t ep) {
     if (p.sm_stats) p.sm_stats[(size_t)blockIdx.x * kStatSlots + ST_SCHED_DEP] = t_dep;
 }
 
+// ---------------------------------------------------------------------------
+// stasher role (one thread; only with Shape::tmem)
+// ---------------------------------------------------------------------------
+// Walks the same page sequence as the loader.  Every page of an op whose
+// pages pass through tensor memory (tmem_page_op) is, once it has landed in
+// its shared-memory slot, copied on into the next free TMEM slot with 16
+// tcgen05.cp (one 4 KB block each, see tmem_page_src); one commit then
+// signals the workers (tfull) and another frees the shared-memory slot for
+// the loader (cpdone) as soon as the copies have read it.  Landed weights so
+// leave the shared-memory ring at once, and the ring (3 pages in flight from
+// HBM) plus tensor memory (4 landed pages) buffer 7 pages per SM.
+__device__ void stasher_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
+    const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
+    uint32_t k = 0;    // pages of the sequence (all kinds)
+    uint32_t tk = 0;   // pages moved into tensor memory
+    uint32_t odd = 0;  // bit s: pages of slot s moved so far, mod 2 (the parity of the next tland wait)
+    const uint32_t tbase = ctl->tmem_base;
+    bool ok = true;
+    for (int step = 0; step < p.n_steps && ok; ++step)
+    for (int qi = q0; qi < q1 && ok; ++qi) {
+        const Task t = p.qtasks[qi];
+        if (t.kind == OP_ATTN) {
+            const AttnChunk a = attn_chunk(p, ctl, step, t.begin);
+            const int npp = attn_pos_per_page(p.s.d);
+            k += (uint32_t)((a.npre + npp - 1) / npp);
+            continue;
+        }
+        const GemvStream g = gemv_stream(p, t);
+        if (!tmem_page_op(p.s, t.kind)) { k += (uint32_t)g.npages; continue; }
+        for (int pg = 0; pg < g.npages; ++pg, ++k) {
+            const uint32_t slot = k % kNumPages;
+            if (!wait_mbar(&ctl->tland[slot], (odd >> slot) & 1u, p, ctl, W_FULL, (uint32_t)t.sm)) { ok = false; break; }
+            odd ^= 1u << slot;
+            const uint32_t ts = tk % kTmemSlots;
+            if (tk >= (uint32_t)kTmemSlots &&
+                !wait_mbar(&ctl->tempty[ts], ((tk / kTmemSlots) - 1u) & 1u, p, ctl, W_EMPTY, (uint32_t)t.sm)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const unsigned char *src = pages + (size_t)slot * kPageBytes;
+            const uint32_t dst = tbase + ts * kTmemSlotCols;
+#pragma unroll 1
+            for (int c = 0; c < 16; ++c) tmem_cp_128x256b(dst + 8 * c, smem_desc(src + 4096 * c, 2048, 128));
+            tc_commit(&ctl->tfull[ts]);
+            tc_commit(&ctl->cpdone[slot]);
+            ++tk;
+        }
+    }
+    // every copy issued must have completed before the CTA frees tensor
+    // memory: the last commit arrives only after all earlier copies
+    if (tk > 0) {
+        const uint32_t ts = (tk - 1) % kTmemSlots, par = ((tk - 1) / kTmemSlots) & 1u;
+        Spin sp;
+        while (!mbar_try_wait(&ctl->tfull[ts], par)) {
+            if ((++sp.n & 127u) == 0u) {
+                const unsigned long long now = globaltimer();
+                if (sp.t0 == 0) sp.t0 = now;
+                else if (now - sp.t0 > p.timeout_ns) break;
+            }
+        }
+    }
+}
+
 // Publishes task completions: workers post the finished task's event in a
 // shared-memory ring (after the barrier that ends the task), this thread
 // performs the gpu-scope release add, so no worker stalls on the release.
@@ -595,8 +553,10 @@ __device__ void signaler_role(const Params &p, SmemCtl *ctl) {
 // worker helpers
 // ---------------------------------------------------------------------------
 struct WState {
-    uint32_t slot = 0;       // ring slot of the next page to consume
-    uint32_t phase = 0;      // its full-barrier parity
+    uint32_t slot = 0;       // ring slot of the next page (of any kind)
+    uint32_t odd = 0;        // bit s: pages read from slot s so far, mod 2 (the parity of the next full wait)
+    uint32_t tslot = 0;      // tensor-memory slot of the next page that passes through it
+    uint32_t tphase = 0;     // its tfull-barrier parity
     uint32_t wphase = 0;     // worker-barrier phase
     uint32_t need = 0;       // ready_upto value that activates the current task
     uint32_t ep = 0;         // this launch's epoch: the tag of this step's activations
@@ -661,7 +621,7 @@ __device__ __forceinline__ void stamp_ready(const Params &p, const WState &w) {
 __device__ __forceinline__ bool wait_page(const Params &p, SmemCtl *ctl, WState &w, uint32_t &slot) {
     slot = w.slot;
     const unsigned long long t0 = phase_begin(w);
-    const bool ok = wait_mbar(&ctl->full[slot], w.phase, p, ctl, W_FULL, (uint32_t)w.task_id);
+    const bool ok = wait_mbar(&ctl->full[slot], (w.odd >> slot) & 1u, p, ctl, W_FULL, (uint32_t)w.task_id);
     phase_end(w, t0, WS_FULL);
     phase_end(w, t0, WS_TASKWAIT);
     return ok;
@@ -670,7 +630,28 @@ __device__ __forceinline__ bool wait_page(const Params &p, SmemCtl *ctl, WState 
 __device__ __forceinline__ void release_page(SmemCtl *ctl, WState &w, uint32_t slot) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(&ctl->empty[slot]);
-    if (++w.slot == (uint32_t)kNumPages) { w.slot = 0; w.phase ^= 1u; }
+    w.odd ^= 1u << slot;
+    if (++w.slot == (uint32_t)kNumPages) w.slot = 0;
+}
+
+// A page that passes through tensor memory: wait until the stasher's copies
+// into the next TMEM slot have completed.  The page also went through the
+// next shared-memory slot (the stasher released that one), so the
+// shared-memory position advances too.
+__device__ __forceinline__ bool wait_tpage(const Params &p, SmemCtl *ctl, WState &w) {
+    const unsigned long long t0 = phase_begin(w);
+    const bool ok = wait_mbar(&ctl->tfull[w.tslot], w.tphase, p, ctl, W_FULL, (uint32_t)w.task_id);
+    phase_end(w, t0, WS_FULL);
+    phase_end(w, t0, WS_TASKWAIT);
+    tc_fence_after();
+    if (++w.slot == (uint32_t)kNumPages) w.slot = 0;
+    return ok;
+}
+__device__ __forceinline__ void release_tpage(SmemCtl *ctl, WState &w) {
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&ctl->tempty[w.tslot]);
+    if (++w.tslot == (uint32_t)kTmemSlots) { w.tslot = 0; w.tphase ^= 1u; }
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -711,7 +692,9 @@ __device__ __forceinline__ bool signal_event(const Params &p, SmemCtl *ctl, cons
 // Copy a tagged vector of n values (n a multiple of 8, n <= 2 * 256 * NP)
 // into ctl->stage, polling every word until it carries this step's tag.  The
 // 256 worker threads take 16-byte pairs round-robin (coalesced), only stale
-// pairs are reloaded.  ss returns the thread's partial sum of squares.  The
+// pairs are reloaded.  ss returns the thread's partial sum of squares, added
+// up in pair order once every pair is in (not in the order the pairs
+// arrived), so the RMSNorm of a step does not depend on timing.  The
 // caller's worker barrier publishes the stage to every warp.
 // Stage layout: the first four values of every 8-value vector v at float4
 // slot v, the last four at slot n/8 + v, so that a warp reading vectors
@@ -742,7 +725,6 @@ __device__ __forceinline__ bool stage_tagged(const Params &p, SmemCtl *ctl, cons
             if ((pend & (1u << j)) && tag_ok(q[k].x, w.ep) && tag_ok(q[k].y, w.ep)) {
                 const float2 v = make_float2(tag_val(q[k].x), tag_val(q[k].y));
                 st[2 * (((i >> 1) & 1) * n8 + (i >> 2)) + (i & 1)] = v;
-                acc = fmaf(v.x, v.x, fmaf(v.y, v.y, acc));
                 pend &= ~(1u << j);
             }
         }
@@ -754,6 +736,15 @@ __device__ __forceinline__ bool stage_tagged(const Params &p, SmemCtl *ctl, cons
         if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 0u)) return false;
 #pragma unroll
         for (int jb = 0; jb < NP; jb += NB) batch(jb, true);
+    }
+    // this thread's own pairs, read back in order
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const int i = tid + j * kWorkerThreads;
+        if (i < npairs) {
+            const float2 v = st[2 * (((i >> 1) & 1) * n8 + (i >> 2)) + (i & 1)];
+            acc = fmaf(v.x, v.x, fmaf(v.y, v.y, acc));
+        }
     }
     ss = acc;
     return true;
@@ -954,6 +945,33 @@ __device__ __forceinline__ void dot_rows2(const uint4 *ra, const uint4 *rc, cons
     acc_c = c.x + c.y;
 }
 
+// The same two dot products for a page in tensor memory: row a's 8
+// vectors (lane + 32j, j = 0..7) are the 32 columns at `ta`, row c's the 32
+// columns at ta + 64; read in quarters of 8 columns so that only 16 row
+// words are live at a time.
+template <int NVL>
+__device__ __forceinline__ void dot_tmem2(uint32_t ta, bool two, const float (&xr)[NVL][8], float &acc_a,
+                                          float &acc_c) {
+    static_assert(NVL == 8, "a TMEM page row is 2048 columns: 8 vectors per lane");
+    float2 a = make_float2(0.f, 0.f), c = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        // the second row's columns are read even when the page has one
+        // row (a trailing 8-row page): its result is then dropped
+        uint32_t ra[8], rc[8];
+        tmem_ld8(ta + 8 * h, ra);
+        tmem_ld8(ta + 64 + 8 * h, rc);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            a = dot8x2(make_uint4(ra[4 * j], ra[4 * j + 1], ra[4 * j + 2], ra[4 * j + 3]), xr[2 * h + j], a);
+            c = dot8x2(make_uint4(rc[4 * j], rc[4 * j + 1], rc[4 * j + 2], rc[4 * j + 3]), xr[2 * h + j], c);
+        }
+    }
+    acc_a = a.x + a.y;
+    acc_c = two ? c.x + c.y : 0.f;
+}
+
 // Epilogue of one unit (16 rows: a pair tile or two 8-row tiles; or one
 // 8-row tile) whose row sums warp 0 holds: lane e (< rows) has row e's dot
 // product `a`, and for pair tiles `c` is row e + 8's.  `resid` is lane L's
@@ -1031,6 +1049,7 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
     const int npair = kind == OP_GATEUP ? 0x7fffffff : 0;
     const bool resid_op = kind == OP_OPROJ || kind == OP_DOWN;
     const int task_rows = 8 * (t.end - t.begin);
+    const bool tmem = tmem_page_op(s, kind);   // pages come through tensor memory
 
     // ---- before the dependency
     const uint16_t *gain = w.gain;
@@ -1146,18 +1165,33 @@ __device__ bool gemv_rows(const Params &p, const Task &t, unsigned char *pages, 
         const bool two = pair || tile + 1 < t.end;
         float acc_a = 0.f, acc_c = 0.f;
         // rows warp and 8 + warp of the page
-        uint32_t slot;
-        if (!wait_page(p, ctl, w, slot)) return false;
-        tp = phase_begin(w);
-        const unsigned char *pg = pages + (size_t)slot * kPageBytes;
-        const uint4 *row_a = reinterpret_cast<const uint4 *>(pg + warp * row_bytes);
-        if (two || nseg > 1) {
-            dot_rows2<NVL>(row_a, reinterpret_cast<const uint4 *>(pg + (8 + warp) * row_bytes), xr, K8,
-                           lane, acc_a, acc_c);
-        } else {
-            acc_a = dot_row<NVL>(row_a, xr, K8, lane);
+        if constexpr (NVL == 8) {
+            if (tmem) {
+                // the page sits in tensor memory: row warp at column 32 *
+                // (warp / 4) of the slot, row 8 + warp 64 columns further,
+                // both in this warp's lane quarter
+                if (!wait_tpage(p, ctl, w)) return false;
+                tp = phase_begin(w);
+                const uint32_t ta = ctl->tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) +
+                                    w.tslot * (uint32_t)kTmemSlotCols + 32u * (uint32_t)(warp >> 2);
+                dot_tmem2<NVL>(ta, two || nseg > 1, xr, acc_a, acc_c);
+                release_tpage(ctl, w);
+            }
         }
-        release_page(ctl, w, slot);
+        if (!tmem) {
+            uint32_t slot;
+            if (!wait_page(p, ctl, w, slot)) return false;
+            tp = phase_begin(w);
+            const unsigned char *pg = pages + (size_t)slot * kPageBytes;
+            const uint4 *row_a = reinterpret_cast<const uint4 *>(pg + warp * row_bytes);
+            if (two || nseg > 1) {
+                dot_rows2<NVL>(row_a, reinterpret_cast<const uint4 *>(pg + (8 + warp) * row_bytes), xr, K8,
+                               lane, acc_a, acc_c);
+            } else {
+                acc_a = dot_row<NVL>(row_a, xr, K8, lane);
+            }
+            release_page(ctl, w, slot);
+        }
         phase_end(w, tp, WS_DOT);
         tp = phase_begin(w);
         const float v = dual_reduce(acc_a, acc_c, lane);
@@ -1872,7 +1906,13 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     if (tid == 0) {
         for (int i = 0; i < kNumPages; ++i) {
             mbar_init(&ctl->full[i], 1);
+            mbar_init(&ctl->tland[i], 1);
             mbar_init(&ctl->empty[i], kWorkerWarps);
+            mbar_init(&ctl->cpdone[i], 1);
+        }
+        for (int i = 0; i < kTmemSlots; ++i) {
+            mbar_init(&ctl->tfull[i], 1);
+            mbar_init(&ctl->tempty[i], kWorkerWarps);
         }
         mbar_init(&ctl->wbar, kWorkerWarps);
         ctl->sig_post = 0;
@@ -1921,6 +1961,17 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     }
     __syncthreads();
     if (ctl->abort) return;   // nothing was started
+    // Tensor memory for the weight ring: the whole allocation of the SM
+    // (one persistent CTA per SM, so nothing else on it holds any).  It is
+    // freed at the end of the kernel, after every role has returned -- the
+    // stasher only returns once its last copies have completed.
+    const bool use_tmem = p.s.tmem != 0;
+    if (use_tmem) {
+        if (warp == kStashWarp) tmem_alloc(&ctl->tmem_base, kTmemCols);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
     if (tid == 0) {
         // the last CTA to read the epoch publishes the launch's last step's
         // epoch for the next launch (steps take epochs ep .. ep + n_steps - 1)
@@ -1938,9 +1989,18 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
             if (lane == 0) loader_role(p, pages, ctl);
         } else if (warp == kSchedWarp) {
             if (lane == 0 && p.event_wait) scheduler_role(p, ctl, ctl->ep);
-        } else if (warp == kSchedWarp + 1) {
+        } else if (warp == kStashWarp) {
+            if (lane == 0 && use_tmem) stasher_role(p, pages, ctl);
         } else {
             if (lane == 0) signaler_role(p, ctl);
+        }
+    }
+    if (use_tmem) {
+        tc_fence_before();
+        __syncthreads();
+        if (warp == kStashWarp) {
+            tc_fence_after();
+            tmem_dealloc(ctl->tmem_base, kTmemCols);
         }
     }
 }
@@ -1966,6 +2026,30 @@ cudaError_t kernel_prepare() {
 cudaError_t kernel_occupancy(int *blocks_per_sm) {
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, mk_step_kernel, kThreads,
                                                          kSmemBytes);
+}
+
+// Weights of a GEMV op into the TMEM page order (see tmem_page_src): `src`
+// is the row-major matrix viewed as `page_rows` rows of 2048 bf16, `dst`
+// receives ceil(page_rows / 16) whole 64 KB pages (rows past the end of a
+// trailing partial page are zero).  Set-up only (mk_create).
+__global__ void repack_tmem_pages_kernel(uint4 *dst, const uint4 *src, long long page_rows, long long total) {
+    for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < total;
+         u += (long long)gridDim.x * blockDim.x) {
+        int row, vec;
+        tmem_page_src((int)(u & 4095), row, vec);
+        const long long pr = (u >> 12) * 16 + row;
+        dst[u] = pr < page_rows ? src[pr * 256 + vec] : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+size_t tmem_pages_bytes(long long page_rows) { return (size_t)((page_rows + 15) / 16) * kPageBytes; }
+
+cudaError_t repack_tmem_pages(void *dst, const void *src, long long page_rows, cudaStream_t stream) {
+    const long long total = (long long)(tmem_pages_bytes(page_rows) / 16);
+    const long long blocks = (total + 255) / 256;
+    repack_tmem_pages_kernel<<<(unsigned)(blocks < 8192 ? blocks : 8192), 256, 0, stream>>>(
+        static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), page_rows, total);
+    return cudaGetLastError();
 }
 
 cudaError_t kernel_launch(const Params &p, int grid, cudaStream_t stream) {

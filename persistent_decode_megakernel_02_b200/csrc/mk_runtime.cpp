@@ -18,6 +18,8 @@ int kernel_launch_regs();
 cudaError_t kernel_prepare();
 cudaError_t kernel_occupancy(int *blocks_per_sm);
 cudaError_t kernel_launch(const Params &p, int grid, cudaStream_t stream);
+size_t tmem_pages_bytes(long long page_rows);
+cudaError_t repack_tmem_pages(void *dst, const void *src, long long page_rows, cudaStream_t stream);
 }  // namespace mk
 
 using namespace mk;
@@ -35,6 +37,7 @@ struct mk_ctx {
     std::vector<void *> allocs;
     Params p{};            // template: step inputs filled per call
     ErrWord *d_err = nullptr;
+    const uint16_t *lm_tmem = nullptr;   // library copy of the LM head in the TMEM page order
     long long steps = 0;
     bool failed = false;   // a device error was observed by mk_sync
 };
@@ -79,6 +82,7 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     s.d = c->head_dim; s.F = c->ffn; s.V = c->vocab; s.S = c->max_seq; s.Bmax = c->max_batch;
     s.G = G; s.QD = (int)QD; s.KD = c->n_kv_heads * c->head_dim;
     s.theta = c->rope_theta; s.eps = c->rms_eps;
+    s.tmem = (c->flags & MK_FLAG_NO_TMEM_RING) ? 0 : 1;
     s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nq, s.S);
     if (s.NC > 4096) return MK_ERR_INVALID;
     // one q head's chunk partials must fit the merge's shared staging area
@@ -259,24 +263,53 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     }
 
     // ---- q/k/v into one buffer, gate/up into tile order (see LayerW / OpTiles)
+    // ---- then, for ops whose pages pass through tensor memory, every
+    //      matrix into the TMEM page order (tmem_page_src), library-owned
     {
         const size_t rb = 2 * (size_t)s.H;          // bytes of one row of K = H
         const size_t tile = 16 * rb;                 // one gate/up pair tile
-        for (int l = 0; l < s.L; ++l) {
-            uint16_t *qkv, *gu;
-            MK_TRY(dalloc(c, &qkv, (size_t)(s.QD + 2 * s.KD) * s.H));
-            MK_TRY(dalloc(c, &gu, (size_t)2 * s.F * s.H));
+        // row-major source (rows x K) -> TMEM page order; returns the copy
+        auto to_tmem = [&](const void *src, long long rows, int K, const uint16_t **out) -> cudaError_t {
+            const long long page_rows = rows * (K / kRowK);
+            uint16_t *dst;
+            cudaError_t err = dalloc(c, &dst, tmem_pages_bytes(page_rows) / 2);
+            if (err == cudaSuccess) err = repack_tmem_pages(dst, src, page_rows, 0);
+            if (err == cudaSuccess) *out = dst;
+            return err;
+        };
+        void *tmp_qkv = nullptr, *tmp_gu = nullptr;   // row-major staging when repacking
+        if (tmem_page_op(s, OP_QKV)) MK_TRY(cudaMalloc(&tmp_qkv, (size_t)(s.QD + 2 * s.KD) * rb));
+        if (tmem_page_op(s, OP_GATEUP)) MK_TRY(cudaMalloc(&tmp_gu, (size_t)2 * s.F * rb));
+        for (int l = 0; l < s.L && e == cudaSuccess; ++l) {
+            uint16_t *qkv = (uint16_t *)tmp_qkv, *gu = (uint16_t *)tmp_gu;
+            if (!qkv) e = dalloc(c, &qkv, (size_t)(s.QD + 2 * s.KD) * s.H);
+            if (e == cudaSuccess && !gu) e = dalloc(c, &gu, (size_t)2 * s.F * s.H);
             char *dq = (char *)qkv;
-            MK_TRY(cudaMemcpy(dq, w->wq[l], (size_t)s.QD * rb, cudaMemcpyDeviceToDevice));
-            MK_TRY(cudaMemcpy(dq + (size_t)s.QD * rb, w->wk[l], (size_t)s.KD * rb, cudaMemcpyDeviceToDevice));
-            MK_TRY(cudaMemcpy(dq + (size_t)(s.QD + s.KD) * rb, w->wv[l], (size_t)s.KD * rb,
-                              cudaMemcpyDeviceToDevice));
-            MK_TRY(cudaMemcpy2D(gu, tile, w->wg[l], 8 * rb, 8 * rb, s.F / 8, cudaMemcpyDeviceToDevice));
-            MK_TRY(cudaMemcpy2D((char *)gu + 8 * rb, tile, w->wu[l], 8 * rb, 8 * rb, s.F / 8,
-                                cudaMemcpyDeviceToDevice));
+            if (e == cudaSuccess) e = cudaMemcpy(dq, w->wq[l], (size_t)s.QD * rb, cudaMemcpyDeviceToDevice);
+            if (e == cudaSuccess)
+                e = cudaMemcpy(dq + (size_t)s.QD * rb, w->wk[l], (size_t)s.KD * rb, cudaMemcpyDeviceToDevice);
+            if (e == cudaSuccess)
+                e = cudaMemcpy(dq + (size_t)(s.QD + s.KD) * rb, w->wv[l], (size_t)s.KD * rb,
+                               cudaMemcpyDeviceToDevice);
+            if (e == cudaSuccess)
+                e = cudaMemcpy2D(gu, tile, w->wg[l], 8 * rb, 8 * rb, s.F / 8, cudaMemcpyDeviceToDevice);
+            if (e == cudaSuccess)
+                e = cudaMemcpy2D((char *)gu + 8 * rb, tile, w->wu[l], 8 * rb, 8 * rb, s.F / 8,
+                                 cudaMemcpyDeviceToDevice);
             lw[l].qkv = qkv;
             lw[l].gu = gu;
+            if (e == cudaSuccess && tmem_page_op(s, OP_QKV)) e = to_tmem(qkv, s.QD + 2 * s.KD, s.H, &lw[l].qkv);
+            if (e == cudaSuccess && tmem_page_op(s, OP_GATEUP)) e = to_tmem(gu, 2LL * s.F, s.H, &lw[l].gu);
+            if (e == cudaSuccess && tmem_page_op(s, OP_OPROJ)) e = to_tmem(w->wo[l], s.H, s.QD, &lw[l].wo);
+            if (e == cudaSuccess && tmem_page_op(s, OP_DOWN)) e = to_tmem(w->wd[l], s.H, s.F, &lw[l].wd);
+            // the staging buffers are reused by the next layer
+            if (e == cudaSuccess && (tmp_qkv || tmp_gu)) e = cudaDeviceSynchronize();
         }
+        if (e == cudaSuccess && tmem_page_op(s, OP_LMHEAD)) e = to_tmem(w->lm_head, s.V, s.H, &c->lm_tmem);
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+        if (tmp_qkv) cudaFree(tmp_qkv);
+        if (tmp_gu) cudaFree(tmp_gu);
+        if (e != cudaSuccess) { free_ctx(c); return map_cuda(e); }
     }
     MK_TRY(cudaDeviceSynchronize());
 
@@ -317,7 +350,8 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     p.lm_cnt = d_ctrl + 0; p.epoch = d_ctrl + 1; p.done_cnt = d_ctrl + 2; p.abort_flag = d_ctrl + 3;
     p.num_lm_tasks = c->num_lm_tasks;
     p.layers = d_layers;
-    p.embed = (const uint16_t *)w->embed; p.lm_head = (const uint16_t *)w->lm_head;
+    p.embed = (const uint16_t *)w->embed;
+    p.lm_head = c->lm_tmem ? c->lm_tmem : (const uint16_t *)w->lm_head;
     p.g_final = (const uint16_t *)w->final_norm;
     p.rope = d_rope;
     p.tag = d_tag; p.tl = tl;
@@ -443,6 +477,7 @@ int mk_get_info(mk_ctx *c, mk_info *out) {
     if (cudaMemcpy(&ew, c->d_err, sizeof ew, cudaMemcpyDeviceToHost) != cudaSuccess) return MK_ERR_CUDA;
     out->err_code = ew.code;
     out->err_info = ew.where << 24 | (ew.info & 0xffffffu);
+    out->err_task = ew.code ? ew.task : 0xffffffffu;
     return MK_OK;
 }
 

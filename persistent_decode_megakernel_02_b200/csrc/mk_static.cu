@@ -117,6 +117,7 @@ bool shape_ok(const mk_config *c, int num_sms, Shape &s) {
     s.d = c->head_dim; s.F = c->ffn; s.V = c->vocab; s.S = c->max_seq; s.Bmax = c->max_batch;
     s.G = G; s.QD = (int)QD; s.KD = c->n_kv_heads * c->head_dim;
     s.theta = c->rope_theta; s.eps = c->rms_eps;
+    s.tmem = 0;   // weights come in the row-major packed layout: pages stay in shared memory
     s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nq, s.S);
     if (s.NC > 4096 || (long long)s.NC * (s.d + 2) > kStageFloats) return false;
     return true;

@@ -20,6 +20,7 @@ MK_OK, MK_ERR_INVALID, MK_ERR_CUDA, MK_ERR_TIMEOUT, MK_ERR_OOM, MK_ERR_STATE = r
 MK_FLAG_TRACE = 1
 MK_FLAG_NO_L2_PREFETCH = 2
 MK_FLAG_EVENT_WAIT = 4
+MK_FLAG_NO_TMEM_RING = 8
 MK_BUF_HIDDEN, MK_BUF_Q, MK_BUF_ATTN, MK_BUF_ACT = range(4)
 OP_NAMES = ["qkv", "attn", "oproj", "gateup", "down", "lmhead"]
 
@@ -70,7 +71,8 @@ class Info(C.Structure):
     _fields_ = [("num_sms", C.c_int), ("num_tasks", C.c_int), ("num_events", C.c_int),
                 ("num_ops", C.c_int), ("attn_chunks", C.c_int), ("max_queue", C.c_int),
                 ("page_bytes", C.c_int), ("num_pages", C.c_int),
-                ("steps_run", C.c_longlong), ("err_code", C.c_uint), ("err_info", C.c_uint)]
+                ("steps_run", C.c_longlong), ("err_code", C.c_uint), ("err_info", C.c_uint),
+                ("err_task", C.c_uint)]
 
 
 class TraceRec(C.Structure):
