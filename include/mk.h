@@ -80,11 +80,15 @@ enum mk_flags {
      * they land, which frees the ring for further prefetch (7 pages of
      * 64 KB buffered per SM instead of 3); mk_create then keeps those
      * weights in a library-owned copy laid out for that copy. */
-    MK_FLAG_NO_TMEM_RING = 8
+    MK_FLAG_NO_TMEM_RING = 8,
+    /* Run steps on the batched tensor-core kernel even with max_batch = 1,
+     * which mk_prefill needs (contexts with max_batch > 1 always use it).
+     * See "Batched steps" below. */
+    MK_FLAG_ROWS = 16
 };
 
 /* Upper bounds of the shapes the kernel tiles. */
-#define MK_MAX_BATCH 1
+#define MK_MAX_BATCH 16
 #define MK_MAX_K 14336      /* max of n_q_heads*head_dim and ffn */
 #define MK_MAX_HIDDEN 4096
 #define MK_MAX_HEAD_DIM 128
@@ -94,7 +98,8 @@ enum mk_flags {
  *  hidden: multiple of 8, at most MK_MAX_HIDDEN; ffn, n_q_heads*head_dim:
  *  multiples of 8, at most MK_MAX_K.  head_dim: 64 or 128; n_q_heads /
  *  n_kv_heads: 1, 2, 4 or 8.  max_seq: KV capacity per sequence (positions
- *  0..max_seq-1).  max_batch: 1..MK_MAX_BATCH.  rms_eps > 0, rope_theta > 1.
+ *  0..max_seq-1).  max_batch: 1..MK_MAX_BATCH (above 1 see "Batched
+ *  steps").  rms_eps > 0, rope_theta > 1.
  *  attn_chunks: most split-K chunks per (sequence, q head) in the
  *  attention op (a step uses ceil(context / 1024) of them, so contexts up
  *  to 1024 positions need no merge); 0 picks min(SMs / (max_batch *
@@ -232,6 +237,46 @@ int mk_decode_step(mk_ctx *ctx, const int32_t *tokens, const int32_t *positions,
  */
 int mk_generate(mk_ctx *ctx, const int32_t *tokens, int n_prompt, const int32_t *positions, int batch,
                 int n_steps, int32_t eos, int32_t *tokens_out, int32_t *next_tok_out, mk_stream_t stream);
+
+/*
+ * Batched steps.  A context created with max_batch > 1 (or MK_FLAG_ROWS)
+ * runs every step on a second persistent kernel: one kernel step takes up to
+ * 16 rows -- a row is one token of one sequence -- and every matrix op is a
+ * contraction of the weights with those rows on the tcgen05 tensor cores
+ * (M = 128 weight rows, N = 32: each row's fp32 input enters as its bf16
+ * high part and bf16 remainder; fp32 accumulation in tensor memory), so the
+ * weights are read once per kernel step whatever the number of rows.  The
+ * matrices are copied into a library-owned tile layout at create time.
+ * Shape limits: hidden, n_q_heads*head_dim, n_kv_heads*head_dim and ffn
+ * multiples of 128; n_q_heads / n_kv_heads = 1, 2 or 4 with (n_q_heads /
+ * n_kv_heads) * head_dim <= 512; attn_chunks: chunks of at least 1024
+ * positions per (row, KV head), default ceil(max_seq / 1024).
+ * MK_FLAG_TRACE, MK_FLAG_EVENT_WAIT (tasks always wait on event counters
+ * here), mk_generate, mk_get_trace, mk_get_sm_stats and
+ * mk_debug_withhold_event are not available on such contexts
+ * (MK_ERR_INVALID); mk_read_buffer offers MK_BUF_HIDDEN as float
+ * [16][hidden].
+ *
+ * mk_decode_step on such a context: sequence b (b < batch) is a row at its
+ * own position, in KV slot b; any mix of positions.
+ *
+ * mk_prefill: a prompt of n_tokens tokens of the sequence in KV slot `slot`,
+ * at positions start_pos .. start_pos + n_tokens - 1, in ONE launch: kernel
+ * steps of 16 consecutive tokens, each a contraction over its 16 rows with
+ * causal attention (a token attends to the slot's positions up to its own,
+ * the prompt's earlier tokens included), the LM head only for the step that
+ * holds the last token (the MPK walkthrough, zizhi168.cn/news/174794, feeds
+ * the prompt through its decode loop one token per step; this is the same
+ * computation with the prompt's tokens sharing each weight read).
+ *   tokens        device int32 [n_tokens]
+ *   logits_out    device float [vocab] for the last token, or NULL
+ *   next_tok_out  device int32 [1]: argmax of the last token's logits
+ * Positions beyond max_seq, a slot >= max_batch or a context without the
+ * batched kernel give MK_ERR_INVALID synchronously; a token outside [0,
+ * vocab) is reported by mk_sync.
+ */
+int mk_prefill(mk_ctx *ctx, const int32_t *tokens, int n_tokens, int slot, int start_pos, float *logits_out,
+               int32_t *next_tok_out, mk_stream_t stream);
 
 /* Wait for `stream`, then return the device status of the context
  * (MK_OK, MK_ERR_INVALID, MK_ERR_TIMEOUT) or MK_ERR_CUDA. */

@@ -12,8 +12,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["mk_kernel.cu", "mk_runtime.cpp", "mk_graph.cpp", "mk_static.cu"]
-HEADERS = ["mk_internal.h", "mk_ptx.cuh"]
+SOURCES = ["mk_kernel.cu", "mk_runtime.cpp", "mk_graph.cpp", "mk_static.cu", "mk_rows.cu",
+           "mk_rows_graph.cpp", "mk_rows_runtime.cpp"]
+HEADERS = ["mk_internal.h", "mk_ptx.cuh", "mk_rows.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

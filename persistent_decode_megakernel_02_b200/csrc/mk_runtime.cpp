@@ -11,6 +11,7 @@
 
 #include "../../include/mk.h"
 #include "mk_internal.h"
+#include "mk_rows.h"
 
 namespace mk {
 size_t kernel_smem_bytes();
@@ -20,6 +21,20 @@ cudaError_t kernel_occupancy(int *blocks_per_sm);
 cudaError_t kernel_launch(const Params &p, int grid, cudaStream_t stream);
 size_t tmem_pages_bytes(long long page_rows);
 cudaError_t repack_tmem_pages(void *dst, const void *src, long long page_rows, cudaStream_t stream);
+// the batched (rows) step: mk_rows_runtime.cpp
+struct RowsCtx;
+bool rows_shape_ok(const Shape &s);
+int rows_default_chunks(int S);
+int rows_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, const Shape &s, int num_sms,
+                RowsCtx **out);
+int rows_step(RowsCtx *c, const int32_t *tokens, const int32_t *positions, int batch, float *logits,
+              int32_t *next_tok, cudaStream_t stream);
+int rows_prefill(RowsCtx *c, const int32_t *tokens, int n, int slot, int start, float *logits, int32_t *next_tok,
+                 cudaStream_t stream);
+int rows_reset(RowsCtx *c);
+void rows_destroy(RowsCtx *c);
+RParams rows_params(const RowsCtx *c);
+size_t rows_smem_bytes();
 }  // namespace mk
 
 using namespace mk;
@@ -37,6 +52,8 @@ struct mk_ctx {
     std::vector<void *> allocs;
     Params p{};            // template: step inputs filled per call
     ErrWord *d_err = nullptr;
+    RowsCtx *rows = nullptr;             // the batched tensor-core step (max_batch > 1 or MK_FLAG_ROWS)
+    RParams rp{};                        // its parameter template (host copy, for introspection)
     const uint16_t *lm_tmem = nullptr;   // library copy of the LM head in the TMEM page order
     long long steps = 0;
     bool failed = false;   // a device error was observed by mk_sync
@@ -64,6 +81,7 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
         c->head_dim < 1 || c->ffn < 8 || c->vocab < 1 || c->max_seq < 1 || c->max_batch < 1)
         return MK_ERR_INVALID;
     if (c->max_batch > MK_MAX_BATCH) return MK_ERR_INVALID;
+    const bool rows = c->max_batch > 1 || (c->flags & MK_FLAG_ROWS);
     if (c->n_q_heads % c->n_kv_heads != 0) return MK_ERR_INVALID;
     const int G = c->n_q_heads / c->n_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return MK_ERR_INVALID;
@@ -83,6 +101,14 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     s.G = G; s.QD = (int)QD; s.KD = c->n_kv_heads * c->head_dim;
     s.theta = c->rope_theta; s.eps = c->rms_eps;
     s.tmem = (c->flags & MK_FLAG_NO_TMEM_RING) ? 0 : 1;
+    if (rows) {
+        // the batched step: its own tiling, chunks of at least 1024 positions
+        s.tmem = 0;
+        s.NC = c->attn_chunks > 0 ? c->attn_chunks : rows_default_chunks(s.S);
+        if (s.NC > 4096 || !rows_shape_ok(s)) return MK_ERR_INVALID;
+        if (c->flags & (MK_FLAG_TRACE | MK_FLAG_EVENT_WAIT)) return MK_ERR_INVALID;
+        return MK_OK;
+    }
     s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nq, s.S);
     if (s.NC > 4096) return MK_ERR_INVALID;
     // one q head's chunk partials must fit the merge's shared staging area
@@ -99,8 +125,11 @@ int map_cuda(cudaError_t e) {
 void free_ctx(mk_ctx *c) {
     if (!c) return;
     for (void *p : c->allocs) cudaFree(p);
+    rows_destroy(c->rows);
     delete c;
 }
+
+bool is_rows(const mk_config *c) { return c->max_batch > 1 || (c->flags & MK_FLAG_ROWS); }
 
 }  // namespace
 
@@ -123,7 +152,8 @@ int mk_plan(const mk_config *cfg, int num_sms, mk_info *info, int32_t *task_out,
     Shape s;
     int st = shape_from_config(cfg, num_sms, s);
     if (st != MK_OK) return st;
-    PlanSizes z = plan_sizes(s, num_sms);
+    const bool rows = is_rows(cfg);
+    PlanSizes z = rows ? rplan_sizes(s, num_sms) : plan_sizes(s, num_sms);
     std::vector<Task> tasks(z.num_tasks);
     std::vector<int32_t> queue(z.num_tasks), qoff(num_sms + 1);
     std::vector<uint32_t> thr(z.num_events);
@@ -131,7 +161,8 @@ int mk_plan(const mk_config *cfg, int num_sms, mk_info *info, int32_t *task_out,
     Plan p;
     p.tasks = tasks.data(); p.queue = queue.data(); p.qoff = qoff.data();
     p.thresholds = thr.data(); p.bytes = bytes.data();
-    plan_build(s, num_sms, p);
+    if (rows) rplan_build(s, num_sms, p);
+    else plan_build(s, num_sms, p);
     if (info) {
         std::memset(info, 0, sizeof *info);
         info->num_sms = num_sms;
@@ -140,8 +171,8 @@ int mk_plan(const mk_config *cfg, int num_sms, mk_info *info, int32_t *task_out,
         info->num_ops = p.num_ops;
         info->attn_chunks = s.NC;
         info->max_queue = p.max_queue;
-        info->page_bytes = kPageBytes;
-        info->num_pages = kNumPages;
+        info->page_bytes = rows ? kRPageBytes : kPageBytes;
+        info->num_pages = rows ? kRStages : kNumPages;
     }
     for (int i = 0; i < p.num_tasks; ++i) {
         const Task &t = tasks[i];
@@ -162,6 +193,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     if (!out) return MK_ERR_INVALID;
     *out = nullptr;
     if (!cfg || !w || !kv) return MK_ERR_INVALID;
+    const bool rows = is_rows(cfg);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MK_ERR_CUDA;
     cudaDeviceProp prop;
@@ -170,7 +202,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     // capability 10.0 exactly, not on other Blackwell parts)
     if (prop.major != 10 || prop.minor != 0) return MK_ERR_INVALID;
     if (!prop.cooperativeLaunch) return MK_ERR_INVALID;
-    if ((size_t)prop.sharedMemPerBlockOptin < kernel_smem_bytes()) return MK_ERR_INVALID;
+    if ((size_t)prop.sharedMemPerBlockOptin < (rows ? rows_smem_bytes() : kernel_smem_bytes())) return MK_ERR_INVALID;
     // The worker/control register split is only safe with the launch
     // allocation it was computed for; refuse to launch anything else.
     if (kernel_launch_regs() != kLaunchRegs) return MK_ERR_INVALID;
@@ -196,6 +228,30 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     c->cfg = *cfg;
     c->s = s;
     c->num_sms = prop.multiProcessorCount;
+    if (rows) {
+        st = rows_create(cfg, w, kv, s, c->num_sms, &c->rows);
+        if (st != MK_OK) { free_ctx(c); return st; }
+        PlanSizes z = rplan_sizes(s, c->num_sms);
+        c->h_tasks.resize(z.num_tasks);
+        c->h_queue.resize(z.num_tasks);
+        c->h_qoff.resize(c->num_sms + 1);
+        c->h_thresholds.resize(z.num_events);
+        Plan plan;
+        plan.tasks = c->h_tasks.data(); plan.queue = c->h_queue.data(); plan.qoff = c->h_qoff.data();
+        plan.thresholds = c->h_thresholds.data(); plan.bytes = nullptr;
+        rplan_build(s, c->num_sms, plan);
+        c->num_tasks = plan.num_tasks;
+        c->num_events = plan.num_events;
+        c->num_ops = plan.num_ops;
+        c->max_queue = plan.max_queue;
+        c->num_lm_tasks = plan.num_lm_tasks;
+        c->rp = rows_params(c->rows);
+        c->d_err = c->rp.err;
+        c->p.events = c->rp.events;
+        c->p.thresholds = c->rp.thresholds;
+        *out = c;
+        return MK_OK;
+    }
 
     // ---- task graph (host)
     PlanSizes z = plan_sizes(s, c->num_sms);
@@ -383,6 +439,11 @@ int mk_decode_step(mk_ctx *c, const int32_t *tokens, const int32_t *positions, i
     if (((uintptr_t)tokens & 3u) || ((uintptr_t)positions & 3u) || ((uintptr_t)next_tok_out & 3u) ||
         ((uintptr_t)logits_out & 3u))
         return MK_ERR_INVALID;
+    if (c->rows) {
+        const int st = rows_step(c->rows, tokens, positions, batch, logits_out, next_tok_out, (cudaStream_t)stream);
+        if (st == MK_OK) c->steps++;
+        return st;
+    }
     Params p = c->p;
     p.tokens = tokens;
     p.positions = positions;
@@ -399,6 +460,7 @@ int mk_generate(mk_ctx *c, const int32_t *tokens, int n_prompt, const int32_t *p
                 int n_steps, int32_t eos, int32_t *tokens_out, int32_t *next_tok_out, mk_stream_t stream) {
     if (!c) return MK_ERR_INVALID;
     if (c->failed) return MK_ERR_STATE;
+    if (c->rows) return MK_ERR_INVALID;   // one launch per generation: batch-1 contexts only
     if (batch < 1 || batch > c->s.Bmax || n_steps < 1 || n_steps > c->s.S) return MK_ERR_INVALID;
     if (n_prompt < 1 || n_prompt > n_steps) return MK_ERR_INVALID;
     if (!tokens || !positions || !tokens_out || !next_tok_out) return MK_ERR_INVALID;
@@ -421,6 +483,22 @@ int mk_generate(mk_ctx *c, const int32_t *tokens, int n_prompt, const int32_t *p
     return MK_OK;
 }
 
+int mk_prefill(mk_ctx *c, const int32_t *tokens, int n_tokens, int slot, int start_pos, float *logits_out,
+               int32_t *next_tok_out, mk_stream_t stream) {
+    if (!c) return MK_ERR_INVALID;
+    if (c->failed) return MK_ERR_STATE;
+    if (!c->rows) return MK_ERR_INVALID;
+    if (!tokens || !next_tok_out || n_tokens < 1 || slot < 0 || slot >= c->s.Bmax || start_pos < 0 ||
+        (long long)start_pos + n_tokens > c->s.S)
+        return MK_ERR_INVALID;
+    if (((uintptr_t)tokens & 3u) || ((uintptr_t)next_tok_out & 3u) || ((uintptr_t)logits_out & 3u))
+        return MK_ERR_INVALID;
+    const int st = rows_prefill(c->rows, tokens, n_tokens, slot, start_pos, logits_out, next_tok_out,
+                                (cudaStream_t)stream);
+    if (st == MK_OK) c->steps += (n_tokens + kRows - 1) / kRows;
+    return st;
+}
+
 int mk_sync(mk_ctx *c, mk_stream_t stream) {
     if (!c) return MK_ERR_INVALID;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MK_ERR_CUDA;
@@ -436,6 +514,12 @@ int mk_sync(mk_ctx *c, mk_stream_t stream) {
 int mk_reset(mk_ctx *c) {
     if (!c) return MK_ERR_INVALID;
     if (cudaDeviceSynchronize() != cudaSuccess) return MK_ERR_CUDA;
+    if (c->rows) {
+        if (rows_reset(c->rows) != MK_OK || cudaDeviceSynchronize() != cudaSuccess) return MK_ERR_CUDA;
+        c->steps = 0;
+        c->failed = false;
+        return MK_OK;
+    }
     const Params &p = c->p;
     if (cudaMemset(p.events, 0, sizeof(uint32_t) * c->num_events) != cudaSuccess ||
         cudaMemset(p.lm_cnt, 0, sizeof(uint32_t) * 4) != cudaSuccess ||
@@ -470,8 +554,8 @@ int mk_get_info(mk_ctx *c, mk_info *out) {
     out->num_ops = c->num_ops;
     out->attn_chunks = c->s.NC;
     out->max_queue = c->max_queue;
-    out->page_bytes = kPageBytes;
-    out->num_pages = kNumPages;
+    out->page_bytes = c->rows ? kRPageBytes : kPageBytes;
+    out->num_pages = c->rows ? kRStages : kNumPages;
     out->steps_run = c->steps;
     ErrWord ew;
     if (cudaMemcpy(&ew, c->d_err, sizeof ew, cudaMemcpyDeviceToHost) != cudaSuccess) return MK_ERR_CUDA;
@@ -495,6 +579,15 @@ int mk_get_event_counts(mk_ctx *c, uint32_t *counts_out, uint32_t *thresholds_ou
 int mk_read_buffer(mk_ctx *c, int which, float *host_out, size_t count) {
     if (!c || !host_out) return MK_ERR_INVALID;
     const Shape &s = c->s;
+    if (c->rows) {
+        // the residual stream after the last layer, rows [kRows][hidden] fp32
+        if (which != MK_BUF_HIDDEN || count > (size_t)kRows * s.H) return MK_ERR_INVALID;
+        RLayerBuf last;
+        if (cudaMemcpy(&last, c->rp.buf + (s.L - 1), sizeof last, cudaMemcpyDeviceToHost) != cudaSuccess ||
+            (count && cudaMemcpy(host_out, last.xb, sizeof(float) * count, cudaMemcpyDeviceToHost) != cudaSuccess))
+            return MK_ERR_CUDA;
+        return MK_OK;
+    }
     const TagLayout &tl = c->p.tl;
     const size_t last = (size_t)(s.L - 1) * tl.layer;
     size_t off = 0, n = 0;
@@ -518,7 +611,7 @@ int mk_read_buffer(mk_ctx *c, int which, float *host_out, size_t count) {
 }
 
 int mk_get_trace(mk_ctx *c, mk_trace_rec *host_out, int n) {
-    if (!c || !host_out || n < 0 || n > c->num_tasks) return MK_ERR_INVALID;
+    if (!c || !host_out || n < 0 || n > c->num_tasks || c->rows) return MK_ERR_INVALID;
     if (!c->p.trace) return MK_ERR_INVALID;
     static_assert(sizeof(mk_trace_rec) == sizeof(TraceRec), "trace record layout");
     if (cudaMemcpy(host_out, c->p.trace, sizeof(TraceRec) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
@@ -527,7 +620,7 @@ int mk_get_trace(mk_ctx *c, mk_trace_rec *host_out, int n) {
 }
 
 int mk_get_sm_stats(mk_ctx *c, uint64_t *host_out, int n) {
-    if (!c || !host_out || n < 0 || n > c->num_sms * kStatSlots) return MK_ERR_INVALID;
+    if (!c || !host_out || n < 0 || n > c->num_sms * kStatSlots || c->rows) return MK_ERR_INVALID;
     if (!c->p.sm_stats) return MK_ERR_INVALID;
     if (cudaMemcpy(host_out, c->p.sm_stats, sizeof(uint64_t) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
         return MK_ERR_CUDA;
@@ -556,7 +649,7 @@ int mk_debug_set_threshold(mk_ctx *c, int event, uint32_t threshold) {
 }
 
 int mk_debug_withhold_event(mk_ctx *c, int event) {
-    if (!c || event < -1 || event >= c->num_events) return MK_ERR_INVALID;
+    if (!c || event < -1 || event >= c->num_events || c->rows) return MK_ERR_INVALID;
     c->p.debug_withhold = event;
     return MK_OK;
 }

@@ -102,7 +102,8 @@ bool shape_ok(const mk_config *c, int num_sms, Shape &s) {
     if (c->layers < 1 || c->hidden < 8 || c->n_q_heads < 1 || c->n_kv_heads < 1 ||
         c->head_dim < 1 || c->ffn < 8 || c->vocab < 1 || c->max_seq < 1 || c->max_batch < 1)
         return false;
-    if (c->max_batch > MK_MAX_BATCH || c->n_q_heads % c->n_kv_heads != 0) return false;
+    // the batch-1 step on CUDA cores only (the batched step is not offered here)
+    if (c->max_batch > kMaxBatch || (c->flags & MK_FLAG_ROWS) || c->n_q_heads % c->n_kv_heads != 0) return false;
     const int G = c->n_q_heads / c->n_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return false;
     if (c->head_dim != 64 && c->head_dim != 128) return false;

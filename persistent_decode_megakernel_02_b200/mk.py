@@ -21,6 +21,8 @@ MK_FLAG_TRACE = 1
 MK_FLAG_NO_L2_PREFETCH = 2
 MK_FLAG_EVENT_WAIT = 4
 MK_FLAG_NO_TMEM_RING = 8
+MK_FLAG_ROWS = 16
+MAX_BATCH = 16
 MK_BUF_HIDDEN, MK_BUF_Q, MK_BUF_ATTN, MK_BUF_ACT = range(4)
 OP_NAMES = ["qkv", "attn", "oproj", "gateup", "down", "lmhead"]
 
@@ -99,12 +101,13 @@ _lib.mk_plan.argtypes = [C.POINTER(Config), C.c_int, C.POINTER(Info), _P, _P, _P
 _lib.mk_debug_set_threshold.argtypes = [_P, C.c_int, C.c_uint]
 _lib.mk_debug_withhold_event.argtypes = [_P, C.c_int]
 _lib.mk_generate.argtypes = [_P, _P, C.c_int, _P, C.c_int, C.c_int, C.c_int, _P, _P, _P]
+_lib.mk_prefill.argtypes = [_P, _P, C.c_int, C.c_int, C.c_int, _P, _P, _P]
 _lib.mk_decode_step_static.argtypes = [C.POINTER(Config), C.POINTER(PackedWeights), C.POINTER(KV),
                                        _P, _P, C.c_int, _P, _P, _P, _P]
 for _f in ("mk_create", "mk_decode_step", "mk_sync", "mk_reset", "mk_destroy", "mk_get_info",
            "mk_get_event_counts", "mk_read_buffer", "mk_get_trace", "mk_get_graph", "mk_plan",
            "mk_get_sm_stats", "mk_decode_step_static",
-           "mk_debug_set_threshold", "mk_debug_withhold_event", "mk_generate"):
+           "mk_debug_set_threshold", "mk_debug_withhold_event", "mk_generate", "mk_prefill"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -246,6 +249,17 @@ class Context:
         st = _lib.mk_generate(self._h, _ptr(tokens), n_prompt, _ptr(positions), b, int(n_steps),
                               int(eos), _ptr(tokens_out), _ptr(next_tok), _stream_ptr(stream))
         _check(st, "mk_generate")
+
+    def prefill(self, tokens, next_tok, logits=None, slot: int = 0, start_pos: int = 0, stream=None,
+                n_tokens=None):
+        """Enqueue a prompt as one launch (batched contexts): tokens int32 CUDA
+        tensor [n] at positions start_pos.., KV slot `slot`; next_tok int32
+        [1] and logits float32 [vocab] (or None) receive the last token's."""
+        n = int(tokens.numel()) if n_tokens is None else int(n_tokens)
+        st = _lib.mk_prefill(self._h, _ptr(tokens), n, int(slot), int(start_pos),
+                             _ptr(logits) if logits is not None else None, _ptr(next_tok),
+                             _stream_ptr(stream))
+        _check(st, "mk_prefill")
 
     def sync(self, stream=None) -> int:
         return _lib.mk_sync(self._h, _stream_ptr(stream))
