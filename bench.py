@@ -252,18 +252,152 @@ def run_oracle_steps(runner: OracleRunner, tokens, positions, n_warm: int, n_max
     return times
 
 
+def main_batched(args, world, rank, local, wk, W, K):
+    """Batched decode (the batched tensor-core step): wk.batch independent
+    sequences at start positions uniform in [32, 2048] over KV prefixes of
+    seeded N(0,1) values; every step decodes one token of every sequence at
+    its own position, each step's argmax feeding the next on the device."""
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from persistent_decode_megakernel_02_b200 import mk
+    shape, B = wk.shape, wk.batch
+    starts = wl.make_start_positions(B, seed=7)
+    max_seq = max(wk.max_seq, int(starts.max()) + W + K + 1)
+    metric = (f"decode ms/token @bs{B} ({shape.name}, staggered positions); achieved HBM GB/s vs roofline")
+    config = {"workload": f"{wk.name}: {shape.name} L{shape.layers} H{shape.hidden} {shape.n_q_heads}/"
+                          f"{shape.n_kv_heads} heads d{shape.head_dim} F{shape.ffn} V{shape.vocab}, {B} sequences "
+                          f"starting at positions uniform in [32, 2048] (KV prefix N(0,1))",
+              "batch": B, "start_positions": [int(x) for x in starts],
+              "l2": "weights exceed L2 (no flush needed)", "parallelism": f"replicas x{world}"}
+    weights = wl.make_weights(shape, seed=1234, device=dev)
+    kc, vc = wl.make_kv(shape, B, max_seq, device=dev, prefill_len=wk.prefill_len)
+    ctx = mk.Context(weights, kc, vc, max_seq, B)
+    stream = torch.cuda.Stream(device=dev)
+    pos = torch.tensor([[int(starts[b]) + i for b in range(B)] for i in range(W + K)], dtype=torch.int32,
+                       device=dev)
+    toks = torch.zeros(2, B, dtype=torch.int32, device=dev)
+    toks[0] = torch.from_numpy(wl.make_prompt(shape.vocab, B, seed=42)).to(dev)
+
+    def one(i):
+        ctx.decode_step(toks[i % 2], pos[i], toks[(i + 1) % 2], None, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            one(i)
+        stream.synchronize()
+        st = ctx.sync(stream)
+        if st != 0:
+            raise mk.MkError(st, "warm-up")
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            e0.record(stream)
+            for i in range(W, W + K):
+                one(i)
+            e1.record(stream)
+            stream.synchronize()
+        st = ctx.sync(stream)
+        if st != 0:
+            raise mk.MkError(st, "timed steps")
+        dev_ms = e0.elapsed_time(e1)
+    dev_ms = max_over_ranks(dev_ms, world, dev)
+    step_ms = dev_ms / K
+    value = step_ms / (B * world)
+    # roofline: every weight once per step (whatever the batch) plus every
+    # sequence's K/V of its C positions
+    contexts = np.array([[int(starts[b]) + i + 1 for b in range(B)] for i in range(W, W + K)])
+    alg_bytes = step_weight_bytes(shape) + step_kv_bytes(shape, contexts) / K
+    peaks = measured_peaks()
+    achieved = alg_bytes / (step_ms * 1e-3) / 1e9
+    flops = 2.0 * B * (step_weight_bytes(shape) / 2)   # one multiply-add per weight per row
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "peak_source": peaks["source"], "bytes_per_launch": int(alg_bytes),
+                "bound_ms": round(bandwidth_bound_ms(alg_bytes, peaks["hbm_gbs"]), 4),
+                "tensor_tflops": round(flops / (step_ms * 1e-3) / 1e12, 2)}
+    # end to end: tokens and positions from pinned host memory, next tokens back
+    e2e = None
+    if not args.no_e2e:
+        n = min(args.e2e_steps, K)
+        h_tok = torch.zeros(B, dtype=torch.int32).pin_memory()
+        h_pos = torch.zeros(B, dtype=torch.int32).pin_memory()
+        h_next = torch.zeros(B, dtype=torch.int32).pin_memory()
+        d_tok = torch.zeros(B, dtype=torch.int32, device=dev)
+        d_pos = torch.zeros(B, dtype=torch.int32, device=dev)
+        d_next = torch.zeros(B, dtype=torch.int32, device=dev)
+        h_tok.copy_(toks[(W + K) % 2].cpu())
+        with torch.cuda.stream(stream):
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            f0 = torch.cuda.Event(enable_timing=True)
+            f1 = torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for i in range(n):
+                h_pos.copy_(torch.from_numpy((starts + W + K + i).astype(np.int32)))
+                d_tok.copy_(h_tok, non_blocking=True)
+                d_pos.copy_(h_pos, non_blocking=True)
+                ctx.decode_step(d_tok, d_pos, d_next, None, stream=stream)
+                h_next.copy_(d_next, non_blocking=True)
+                stream.synchronize()
+                h_tok.copy_(h_next)
+            f1.record(stream)
+            stream.synchronize()
+            st = ctx.sync(stream)
+            if st != 0:
+                raise mk.MkError(st, "e2e steps")
+            e2e_ms = f0.elapsed_time(f1)
+        e2e_ms = max_over_ranks(e2e_ms, world, dev)
+        e2e = {"value": round(e2e_ms / (n * B * world), 5), "unit": UNIT, "h2d_bytes_per_step": 8 * B,
+               "d2h_bytes_per_step": 4 * B, "steps": n}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        runner = OracleRunner(shape, weights.numpy_bits(), max_seq, wk.prefill_len)
+        ptoks = toks[0].cpu().numpy()
+        with PinnedCore() as pin:
+            times = run_oracle_steps(runner, ptoks, [int(starts[0]) + i for i in range(len(ptoks))], 0, K,
+                                     args.cpu_sample_s)
+        cpu = {"value": round(float(np.mean(times)), 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "pinned_core": pin.core, "host_cores": host_cores(),
+               "sample": f"{len(times)} full oracle decode steps of one sequence (one token each; fp64 C, "
+                         f"single thread pinned to core {pin.core} of {host_cores()}) from position {int(starts[0])}"}
+    if rank == 0:
+        out = {"metric": metric, "value": round(value, 5), "unit": UNIT, "n_gpus": world, "steps": K,
+               "warmup": W, "ms_per_step": round(step_ms, 5), "higher_is_better": False, "scaling": "weak",
+               "vs_baseline": None, "dtype": "bf16 weights/KV, tcgen05 bf16 (high + low) x bf16, fp32 accumulate",
+               "data": "synthetic", "config": config, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+               "gpu_launches": K, "clocks": clk.summary(), "tokens_per_s": round(B * world / (step_ms * 1e-3), 1),
+               "achieved_gbs": round(achieved, 1)}
+        print(json.dumps(out), flush=True)
+    ctx.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 # ---------------------------------------------------------------------------
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=512)
     ap.add_argument("--warmup", type=int, default=39)
-    ap.add_argument("--workload", default="llama1b", choices=["llama1b", "llama8b", "longctx", "tiny"])
+    ap.add_argument("--workload", default="llama1b",
+                    choices=["llama1b", "llama8b", "longctx", "tiny", "batched4", "batched8", "batched16"])
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-generate", action="store_true",
                     help="skip the one-launch generation measurement")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prompt-in-one-launch measurement")
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--cpu-sample-s", type=float, default=8.0,
                     help="CPU baseline: time full oracle steps for about this long (at least 3)")
@@ -308,6 +442,8 @@ def main():
     W = max(3, args.warmup)
     K = max(1, args.steps)
     wk = wl.WORKLOADS[args.workload]
+    if wk.batch > 1:
+        return main_batched(args, world, rank, local, wk, W, K)
     shape = wk.shape
     prefill = wk.prefill_len
     start = prefill if prefill else 0
@@ -476,6 +612,54 @@ def main():
         gen = {"value": round(job_ms_per_token(gen_ms, K, world), 5), "unit": UNIT, "steps": K, "launches": 1,
                "api": "mk_generate"}
 
+    # ---- the prompt in one launch (mk_prefill on the batched tensor-core
+    # step: 16 tokens per kernel step, one weight read per 16 tokens) against
+    # the same prompt fed one token per launch through the batch-1 step
+    pre = None
+    if not args.no_prefill and wk.prompt_len > 1 and shape.hidden % 128 == 0:
+        n = wk.prompt_len
+        kc2, vc2 = wl.make_kv(shape, 1, max_seq, device=dev)
+        ctx2 = mk.Context(weights, kc2, vc2, max_seq, 1, flags=mk.MK_FLAG_ROWS)
+        ptok = torch.from_numpy(wl.make_prompt(shape.vocab, n, seed=42)).to(dev)
+        pnext = torch.zeros(1, dtype=torch.int32, device=dev)
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                ctx2.prefill(ptok, pnext, slot=0, start_pos=0, stream=stream)
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            p0 = torch.cuda.Event(enable_timing=True)
+            p1 = torch.cuda.Event(enable_timing=True)
+            reps = 5
+            p0.record(stream)
+            for _ in range(reps):
+                ctx2.prefill(ptok, pnext, slot=0, start_pos=0, stream=stream)
+            p1.record(stream)
+            stream.synchronize()
+            st = ctx2.sync(stream)
+            if st != 0:
+                raise mk.MkError(st, "prefill")
+            pf_ms = p0.elapsed_time(p1) / reps
+            # the same prompt one token per launch (batch-1 step, positions 0..n-1)
+            q0 = torch.cuda.Event(enable_timing=True)
+            q1 = torch.cuda.Event(enable_timing=True)
+            ppos = torch.arange(0, n, dtype=torch.int32, device=dev)
+            q0.record(stream)
+            for i in range(n):
+                ctx.decode_step(ptok[i:i + 1], ppos[i:i + 1], dummy_next, None, stream=stream)
+            q1.record(stream)
+            stream.synchronize()
+            st = ctx.sync(stream)
+            if st != 0:
+                raise mk.MkError(st, "prompt token by token")
+            tt_ms = q0.elapsed_time(q1)
+        pf_ms = max_over_ranks(pf_ms, world, dev)
+        tt_ms = max_over_ranks(tt_ms, world, dev)
+        pre = {"tokens": n, "ms": round(pf_ms, 4), "launches": 1, "api": "mk_prefill",
+               "ms_token_by_token": round(tt_ms, 4), "speedup": round(tt_ms / pf_ms, 2)}
+        ctx2.close()
+        del kc2, vc2
+
     # ---- CPU baseline: full oracle steps on one pinned core (rank 0, N=1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -500,7 +684,7 @@ def main():
                "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
                "dtype": "bf16 weights/KV, fp32 accumulate", "data": "synthetic",
                "config": config, "roofline": roofline, "cpu_baseline": cpu,
-               "e2e": e2e, "generate": gen, "gpu_launches": K, "clocks": clk.summary(),
+               "e2e": e2e, "generate": gen, "prefill": pre, "gpu_launches": K, "clocks": clk.summary(),
                "achieved_gbs": round(achieved, 1)}
         print(json.dumps(out), flush=True)
     ctx.close()

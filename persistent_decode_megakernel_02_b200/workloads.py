@@ -78,7 +78,9 @@ WORKLOADS = {
     "llama1b": Workload("llama1b", LLAMA_1B, 1, 39, 512, 560),
     "llama8b": Workload("llama8b", LLAMA_8B, 1, 39, 512, 560),
     "longctx": Workload("longctx", LLAMA_1B, 1, 0, 256, 16640, prefill_len=16384),
-    "batched16": Workload("batched16", LLAMA_1B, 16, 0, 128, 2048 + 136, staggered=True),
+    "batched4": Workload("batched4", LLAMA_1B, 4, 0, 128, 2048 + 136, prefill_len=2048, staggered=True),
+    "batched8": Workload("batched8", LLAMA_1B, 8, 0, 128, 2048 + 136, prefill_len=2048, staggered=True),
+    "batched16": Workload("batched16", LLAMA_1B, 16, 0, 128, 2048 + 136, prefill_len=2048, staggered=True),
 }
 
 
