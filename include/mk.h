@@ -251,11 +251,14 @@ int mk_generate(mk_ctx *ctx, const int32_t *tokens, int n_prompt, const int32_t 
  * multiples of 128; n_q_heads / n_kv_heads = 1, 2 or 4 with (n_q_heads /
  * n_kv_heads) * head_dim <= 512; attn_chunks: chunks of at least 1024
  * positions per (row, KV head), default ceil(max_seq / 1024).
- * MK_FLAG_TRACE, MK_FLAG_EVENT_WAIT (tasks always wait on event counters
- * here), mk_generate, mk_get_trace, mk_get_sm_stats and
- * mk_debug_withhold_event are not available on such contexts
- * (MK_ERR_INVALID); mk_read_buffer offers MK_BUF_HIDDEN as float
- * [16][hidden].
+ * MK_FLAG_EVENT_WAIT (tasks always wait on event counters here),
+ * mk_generate, mk_get_sm_stats and mk_debug_withhold_event are not
+ * available on such contexts (MK_ERR_INVALID); mk_read_buffer offers
+ * MK_BUF_HIDDEN as float [16][hidden].  With MK_FLAG_TRACE the trace
+ * records mean: t_ready the scheduler saw the dependency met, t_wait the
+ * MMA issuer began the task's pages, t_start the compute warps began,
+ * t_input the first accumulator (or the attention queries) was in hand,
+ * t_done the epilogue was done, t_end the completion was posted.
  *
  * mk_decode_step on such a context: sequence b (b < batch) is a row at its
  * own position, in KV slot b; any mix of positions.

@@ -316,6 +316,7 @@ __device__ void sched_role(const RParams &p, unsigned char *slabs, Ctl *c) {
             // what the producers wrote is read below by bulk copies (the
             // async proxy) and by the compute warps
             asm volatile("fence.proxy.async.global;" ::: "memory");
+            if (p.trace) p.trace[t.sm].t_ready = globaltimer();
             st_release_cta_shared(&c->ready_upto, (uint32_t)(step * qlen + (qi - q0) + 1));
             if (!is_gemv(t.kind) || !task_on(p, t, step)) continue;
             const RGemv g = rgemv(p.s, t.kind);
@@ -368,6 +369,7 @@ __device__ void mma_role(const RParams &p, unsigned char *ring, unsigned char *s
             continue;
         }
         if (!is_gemv(t.kind) || !task_on(p, t, step)) continue;
+        if (p.trace) p.trace[t.sm].t_wait = globaltimer();
         const RGemv g = rgemv(p.s, t.kind);
         for (int pg = t.begin; pg < t.end && ok;) {
             const int pe = seg_end(pg, t.end, g.slabs);
@@ -655,6 +657,7 @@ __device__ bool gemv_task(const RParams &p, Ctl *c, CState &cs, const Task &t) {
         const uint32_t acc = cs.segs & 1u;
         if (!wait_bar(&c->accfull[acc], (cs.segs >> 1) & 1u, p, c, W_ACC, (uint32_t)cs.task_id)) return false;
         tc_fence_after();
+        if (p.trace && m == 0 && pg == t.begin) p.trace[t.sm].t_input = globaltimer();
         uint32_t d[32];
         tmem_ld32(c->tmem_base + ((uint32_t)(32 * warp) << 16) + acc * kRAccCols, d);
         tmem_ld_wait();
@@ -817,6 +820,7 @@ __device__ bool attn_task(const RParams &p, unsigned char *ring, Ctl *c, CState 
         for (int i = tid; i < G * D; i += kComputeWarps * 32)
             c->at.q[i] = ldcg(B.q + (size_t)a.r * s.QD + (size_t)a.h * G * D + i);
     if (!group_sync(&c->cbar, cs.cph, p, c, (uint32_t)cs.task_id)) return false;
+    if (p.trace && tid == 0) p.trace[t.sm].t_input = globaltimer();
     float mx[G], l[G], o[G][DPL];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -954,6 +958,7 @@ __device__ void compute_role(const RParams &p, unsigned char *ring, Ctl *c) {
                 while (ld_acquire_cta_shared(&c->ready_upto) <= k)
                     if (!spin_ok(s, p, c, W_READY, (uint32_t)t.sm, 0u)) return;
             }
+            if (p.trace && tid == 0) p.trace[t.sm].t_start = globaltimer();
             bool ok = true;
             if (t.kind == ROP_ATTN) {
                 ok = p.s.d == 64 ? attn_dispatch<64>(p, ring, c, cs, t) : attn_dispatch<128>(p, ring, c, cs, t);
@@ -970,6 +975,7 @@ __device__ void compute_role(const RParams &p, unsigned char *ring, Ctl *c) {
             // every write of the task is done (and ordered before the bulk
             // copies that read it on other SMs) before its completion posts
             asm volatile("fence.proxy.async.global;" ::: "memory");
+            if (p.trace && tid == 0) p.trace[t.sm].t_done = globaltimer();
             if (!group_sync(&c->cbar, cs.cph, p, c, (uint32_t)t.sm)) return;
             if (t.kind == ROP_LMHEAD && task_on(p, t, step)) {
                 // the task's argmax partials, then (their writers fenced and
@@ -993,6 +999,7 @@ __device__ void compute_role(const RParams &p, unsigned char *ring, Ctl *c) {
                 if (c->last_flag && step + 1 == p.n_steps && warp == 0) lm_reduce(p, nrows);
             }
             if (tid == 0 && !post_done(p, c, t)) return;
+            if (p.trace && tid == 0) p.trace[t.sm].t_end = globaltimer();
         }
     }
 }

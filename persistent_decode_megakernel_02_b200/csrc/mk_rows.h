@@ -166,6 +166,11 @@ struct RParams {
     float *amax_val;            // [kRows][num_lm_tasks]
     int32_t *amax_idx;
     ErrWord *err;
+    TraceRec *trace;            // per-task timestamps of the last step (MK_FLAG_TRACE), or null:
+                                //  t_ready: the scheduler saw the dependency met; t_wait: the MMA
+                                //  issuer began the task's pages; t_start: the compute warps began;
+                                //  t_input: first accumulator (or attention queries) in hand;
+                                //  t_done: epilogue done; t_end: completion posted
     unsigned long long timeout_ns;
 };
 

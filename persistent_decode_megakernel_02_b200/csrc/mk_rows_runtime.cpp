@@ -232,6 +232,15 @@ int rows_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, cons
         RK_TRY(ralloc(c, &p.amax_val, (size_t)kRows * c->num_lm_tasks));
         RK_TRY(ralloc(c, &p.amax_idx, (size_t)kRows * c->num_lm_tasks));
     }
+    if (cfg->flags & MK_FLAG_TRACE) {
+        std::vector<TraceRec> tr(c->num_tasks);
+        for (int i = 0; i < c->num_tasks; ++i) {
+            const Task &t = c->h_tasks[i];
+            tr[i] = TraceRec{0, 0, 0, 0, 0, 0, t.sm, t.kind, t.layer, t.trig};
+        }
+        RK_TRY(ralloc(c, &p.trace, c->num_tasks));
+        RK_TRY(cudaMemcpy(p.trace, tr.data(), sizeof(TraceRec) * c->num_tasks, cudaMemcpyHostToDevice));
+    }
     RK_TRY(rows_prepare());
 #undef RK_TRY
 

@@ -106,7 +106,7 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
         s.tmem = 0;
         s.NC = c->attn_chunks > 0 ? c->attn_chunks : rows_default_chunks(s.S);
         if (s.NC > 4096 || !rows_shape_ok(s)) return MK_ERR_INVALID;
-        if (c->flags & (MK_FLAG_TRACE | MK_FLAG_EVENT_WAIT)) return MK_ERR_INVALID;
+        if (c->flags & MK_FLAG_EVENT_WAIT) return MK_ERR_INVALID;   // tasks always wait on events here
         return MK_OK;
     }
     s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nq, s.S);
@@ -611,7 +611,13 @@ int mk_read_buffer(mk_ctx *c, int which, float *host_out, size_t count) {
 }
 
 int mk_get_trace(mk_ctx *c, mk_trace_rec *host_out, int n) {
-    if (!c || !host_out || n < 0 || n > c->num_tasks || c->rows) return MK_ERR_INVALID;
+    if (!c || !host_out || n < 0 || n > c->num_tasks) return MK_ERR_INVALID;
+    if (c->rows) {
+        if (!c->rp.trace) return MK_ERR_INVALID;
+        if (cudaMemcpy(host_out, c->rp.trace, sizeof(TraceRec) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return MK_ERR_CUDA;
+        return MK_OK;
+    }
     if (!c->p.trace) return MK_ERR_INVALID;
     static_assert(sizeof(mk_trace_rec) == sizeof(TraceRec), "trace record layout");
     if (cudaMemcpy(host_out, c->p.trace, sizeof(TraceRec) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
