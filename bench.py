@@ -78,17 +78,31 @@ def bandwidth_bound_ms(bytes_per_step: float, gbs: float) -> float:
     return bytes_per_step / (gbs * 1e9) * 1e3
 
 
+STEP_KERNEL_SOURCES = ("mk_kernel.cu", "mk_internal.h", "mk_ptx.cuh")
+
+
+def step_kernel_digest() -> str:
+    """Hash of the sources the batch-1 step kernel is compiled from."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in STEP_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "persistent_decode_megakernel_02_b200", "csrc", name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def profiled_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu capture, only while the
-    library build is the one that was profiled (else None)."""
+    """DRAM bytes per launch from the committed ncu capture of the step
+    kernel, only while that kernel's sources are the ones profiled (else
+    None)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
-        with open(os.path.join(ROOT, "persistent_decode_megakernel_02_b200", "libmk.so.sha256")) as f:
-            digest = f.read().strip()
+        digest = step_kernel_digest()
     except (OSError, ValueError):
         return None
-    if t.get("workload") != workload or t.get("build_digest") != digest:
+    if t.get("workload") != workload or t.get("kernel_digest") != digest:
         return None
     return int(t["dram_bytes_read_per_launch"]) + int(t["dram_bytes_write_per_launch"])
 

@@ -92,6 +92,7 @@ struct __align__(16) Ctl {
         struct {
             float q[kMaxGD];                      // G query heads, head-major
             float st[kComputeWarps][kAttnSlot];   // per-warp G x (d output, m, l)
+            float4 pw[kComputeWarps][32];         // per warp: a block's softmax weights, 4 heads per position
         } at;
     };
 };
@@ -147,6 +148,19 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, const R
     return true;
 }
 
+// wait_bar that adds the time waited to *acc (trace mode; acc null: plain).
+__device__ __forceinline__ bool wait_bar_t(uint64_t *bar, uint32_t parity, const RParams &p, Ctl *c,
+                                           uint32_t where, uint32_t task, unsigned long long *acc) {
+    if (!acc) return wait_bar(bar, parity, p, c, where, task);
+    const unsigned long long t0 = globaltimer();
+    const bool ok = wait_bar(bar, parity, p, c, where, task);
+    *acc += globaltimer() - t0;
+    return ok;
+}
+__device__ __forceinline__ unsigned long long *stat_slot(const RParams &p, int which) {
+    return p.sm_stats ? p.sm_stats + (size_t)blockIdx.x * kRStats + which : nullptr;
+}
+
 // A barrier among `warps` warps (an mbarrier with that many arrivals, one
 // per warp): bounded, unlike bar.sync, so a warp that gave up on a wait
 // cannot leave the others blocked.
@@ -154,7 +168,7 @@ __device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &phase, const
                                            uint32_t task) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-    const bool ok = wait_bar(bar, phase, p, c, W_BAR, task);
+    const bool ok = wait_bar_t(bar, phase, p, c, W_BAR, task, threadIdx.x == 0 ? stat_slot(p, RS_CMP_SYNC) : nullptr);
     phase ^= 1u;
     return ok;
 }
@@ -192,7 +206,7 @@ __device__ __forceinline__ Item attn_item(const RParams &p, int step, int item) 
         a.P = rw.pos;
         a.slot = rw.slot;
         const int C = a.P + 1;
-        const int nc = min(s.NC, (C + kAttnChunkPositions - 1) / kAttnChunkPositions);
+        const int nc = min(s.NC, (C + kRAttnChunk - 1) / kRAttnChunk);
         const int Lc = (C + nc - 1) / nc;
         a.nc = nc;
         a.c0 = a.c * Lc;
@@ -235,7 +249,9 @@ __device__ __forceinline__ bool ring_acquire(const RParams &p, Ctl *c, Ring &r, 
     if (r.seq >= (uint32_t)kRStages) {
         const bool prev_m = (r.via_m >> slot) & 1u;
         const uint32_t par = (((prev_m ? r.odd_m : r.odd_c) >> slot) & 1u) ^ 1u;
-        if (!wait_bar(prev_m ? &c->empty_m[slot] : &c->empty_c[slot], par, p, c, W_EMPTY, task)) return false;
+        if (!wait_bar_t(prev_m ? &c->empty_m[slot] : &c->empty_c[slot], par, p, c, W_EMPTY, task,
+                        stat_slot(p, RS_LOAD_SLOT)))
+            return false;
     }
     if (for_mma) { r.via_m |= 1u << slot; r.odd_m ^= 1u << slot; }
     else { r.via_m &= ~(1u << slot); r.odd_c ^= 1u << slot; }
@@ -247,6 +263,7 @@ __device__ __forceinline__ bool ring_acquire(const RParams &p, Ctl *c, Ring &r, 
 
 __device__ void loader_role(const RParams &p, unsigned char *ring, Ctl *c) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
+    const unsigned long long t_begin = p.sm_stats ? globaltimer() : 0ull;
     const uint64_t pol = policy_evict_first();
     const int npp = rattn_pos_per_page(p.s.d);
     Ring rg;
@@ -280,6 +297,7 @@ __device__ void loader_role(const RParams &p, unsigned char *ring, Ctl *c) {
             }
         }
     }
+    if (p.sm_stats) *stat_slot(p, RS_LOAD_TOTAL) = globaltimer() - t_begin;
     // let every copy issued land before the CTA can exit
     const uint32_t used = rg.seq < (uint32_t)kRStages ? rg.seq : (uint32_t)kRStages;
     for (uint32_t sl = 0; sl < used; ++sl) {
@@ -311,8 +329,10 @@ __device__ void sched_role(const RParams &p, unsigned char *slabs, Ctl *c) {
             // the first op of a step waits for the previous step's last
             const uint32_t target = p.thresholds[t.dep] * (t.kind == ROP_EMBED ? ep - 1u : ep);
             Spin s;
+            const unsigned long long td = p.sm_stats ? globaltimer() : 0ull;
             while ((int32_t)(ld_acquire_gpu(&p.events[t.dep]) - target) < 0)
                 if (!spin_ok(s, p, c, W_DEP, (uint32_t)t.sm, (uint32_t)t.dep)) return;
+            if (p.sm_stats) *stat_slot(p, RS_SCHED_DEP) += globaltimer() - td;
             // what the producers wrote is read below by bulk copies (the
             // async proxy) and by the compute warps
             asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -324,7 +344,8 @@ __device__ void sched_role(const RParams &p, unsigned char *slabs, Ctl *c) {
             for (int pg = t.begin; pg < t.end; ++pg, ++bseq) {
                 const uint32_t slot = bseq % kRStages;
                 if (bseq >= (uint32_t)kRStages &&
-                    !wait_bar(&c->bempty[slot], ((bseq / kRStages) - 1u) & 1u, p, c, W_EMPTY, (uint32_t)t.sm))
+                    !wait_bar_t(&c->bempty[slot], ((bseq / kRStages) - 1u) & 1u, p, c, W_EMPTY, (uint32_t)t.sm,
+                                stat_slot(p, RS_SCHED_SLAB)))
                     return;
                 mbar_arrive_expect_tx(&c->bfull[slot], kRSlabBytes);
                 bulk_g2s(slabs + (size_t)slot * kRSlabBytes, x + (size_t)(pg % g.slabs) * kRSlabBytes, kRSlabBytes,
@@ -359,6 +380,7 @@ __device__ __forceinline__ int seg_end(int pg, int end, int slabs) {
 
 __device__ void mma_role(const RParams &p, unsigned char *ring, unsigned char *slabs, Ctl *c) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
+    const unsigned long long t_begin = p.sm_stats ? globaltimer() : 0ull;
     uint32_t aseq = 0, odd_m = 0, bseq = 0, segs = 0;
     bool ok = true;
     for (int step = 0; step < p.n_steps && ok; ++step)
@@ -374,7 +396,8 @@ __device__ void mma_role(const RParams &p, unsigned char *ring, unsigned char *s
         for (int pg = t.begin; pg < t.end && ok;) {
             const int pe = seg_end(pg, t.end, g.slabs);
             const uint32_t acc = segs & 1u;
-            if (segs >= 2u && !wait_bar(&c->accempty[acc], ((segs >> 1) - 1u) & 1u, p, c, W_ACC, (uint32_t)t.sm)) {
+            if (segs >= 2u && !wait_bar_t(&c->accempty[acc], ((segs >> 1) - 1u) & 1u, p, c, W_ACC, (uint32_t)t.sm,
+                                          stat_slot(p, RS_MMA_ACC))) {
                 ok = false;
                 break;
             }
@@ -382,8 +405,10 @@ __device__ void mma_role(const RParams &p, unsigned char *ring, unsigned char *s
             const uint32_t dt = c->tmem_base + acc * kRAccCols;
             for (int q = pg; q < pe; ++q) {
                 const uint32_t as = aseq % kRStages, bs = bseq % kRStages;
-                if (!wait_bar(&c->full_m[as], (odd_m >> as) & 1u, p, c, W_FULL, (uint32_t)t.sm) ||
-                    !wait_bar(&c->bfull[bs], (bseq / kRStages) & 1u, p, c, W_FULL, (uint32_t)t.sm)) {
+                if (!wait_bar_t(&c->full_m[as], (odd_m >> as) & 1u, p, c, W_FULL, (uint32_t)t.sm,
+                                stat_slot(p, RS_MMA_PAGE)) ||
+                    !wait_bar_t(&c->bfull[bs], (bseq / kRStages) & 1u, p, c, W_FULL, (uint32_t)t.sm,
+                                stat_slot(p, RS_MMA_SLAB))) {
                     ok = false;
                     break;
                 }
@@ -406,6 +431,7 @@ __device__ void mma_role(const RParams &p, unsigned char *ring, unsigned char *s
             pg = pe;
         }
     }
+    if (p.sm_stats) *stat_slot(p, RS_MMA_TOTAL) = globaltimer() - t_begin;
     // every contraction issued has completed before tensor memory is freed:
     // the last commit arrives only after all earlier tcgen05 operations
     if (segs > 0) {
@@ -655,7 +681,9 @@ __device__ bool gemv_task(const RParams &p, Ctl *c, CState &cs, const Task &t) {
         const int pe = seg_end(pg, t.end, g.slabs);
         const int tile = pg / g.slabs;
         const uint32_t acc = cs.segs & 1u;
-        if (!wait_bar(&c->accfull[acc], (cs.segs >> 1) & 1u, p, c, W_ACC, (uint32_t)cs.task_id)) return false;
+        if (!wait_bar_t(&c->accfull[acc], (cs.segs >> 1) & 1u, p, c, W_ACC, (uint32_t)cs.task_id,
+                        m == 0 ? stat_slot(p, RS_CMP_ACC) : nullptr))
+            return false;
         tc_fence_after();
         if (p.trace && m == 0 && pg == t.begin) p.trace[t.sm].t_input = globaltimer();
         uint32_t d[32];
@@ -729,10 +757,10 @@ __device__ bool embed_task(const RParams &p, Ctl *c, CState &cs, const Task &t) 
 // choice between a global-space load and a generic one of the same pointer
 // could be evaluated on both sides.
 template <int D, int G, bool GLOBAL>
-__device__ __forceinline__ void attn_block(const Ctl *c, const uint16_t *K, const uint16_t *V, int n,
+__device__ __forceinline__ void attn_block(Ctl *c, const uint16_t *K, const uint16_t *V, int n,
                                            float (&mx)[G], float (&l)[G], float (&o)[G][D / 32]) {
     constexpr int NCH = D / 8, DPL = D / 32;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float sc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) sc[g] = -INFINITY;
@@ -777,6 +805,14 @@ __device__ __forceinline__ void attn_block(const Ctl *c, const uint16_t *K, cons
         for (int i = 0; i < DPL; ++i) o[g][i] *= corr;
         mx[g] = mn;
     }
+    // the weights of position `lane` for every head, read back below by all
+    // lanes at once (one broadcast load per position instead of G shuffles)
+    float4 *pw = c->at.pw[warp];
+    float pv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int g = 0; g < G; ++g) pv[g] = pe[g];
+    pw[lane] = make_float4(pv[0], pv[1], pv[2], pv[3]);
+    __syncwarp();
     for (int k = 0; k < n; ++k) {
         const uint16_t *vr = V + (size_t)k * D + lane * DPL;
         float v[DPL];
@@ -791,13 +827,15 @@ __device__ __forceinline__ void attn_block(const Ctl *c, const uint16_t *K, cons
             else w = *reinterpret_cast<const uint2 *>(vr);
             v[0] = bf_lo(w.x); v[1] = bf_hi(w.x); v[2] = bf_lo(w.y); v[3] = bf_hi(w.y);
         }
+        const float4 pk4 = pw[k];
+        const float pk[4] = {pk4.x, pk4.y, pk4.z, pk4.w};
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const float pk = __shfl_sync(0xffffffffu, pe[g], k);
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) o[g][i] = fmaf(pk, v[i], o[g][i]);
+            for (int i = 0; i < DPL; ++i) o[g][i] = fmaf(pk[g], v[i], o[g][i]);
         }
     }
+    __syncwarp();   // the next block's weights overwrite pw
 }
 
 // One attention item (row r, KV head h, chunk c) on the 8 compute warps:
@@ -829,14 +867,20 @@ __device__ bool attn_task(const RParams &p, unsigned char *ring, Ctl *c, CState 
 #pragma unroll
         for (int i = 0; i < DPL; ++i) o[g][i] = 0.f;
     }
+    // the two halves of the warps take alternate pages (4 warps x 32
+    // positions = one page at head_dim 64); every warp still waits for every
+    // page in order, so its view of each slot's barrier phases stays exact
     for (int pg = 0; pg < npages; ++pg) {
         const uint32_t slot = cs.aseq % kRStages;
-        if (!wait_bar(&c->full_c[slot], (cs.odd_c >> slot) & 1u, p, c, W_FULL, (uint32_t)cs.task_id)) return false;
+        if (!wait_bar_t(&c->full_c[slot], (cs.odd_c >> slot) & 1u, p, c, W_FULL, (uint32_t)cs.task_id,
+                        tid == 0 ? stat_slot(p, RS_CMP_KV) : nullptr))
+            return false;
         const uint16_t *Kp = reinterpret_cast<const uint16_t *>(ring + (size_t)slot * kRPageBytes);
         const uint16_t *Vp = Kp + (size_t)npp * D;
         const int n = min(npp, a.nring - pg * npp);
-        for (int j0 = warp * 32; j0 < n; j0 += kComputeWarps * 32)
-            attn_block<D, G, false>(c, Kp + (size_t)j0 * D, Vp + (size_t)j0 * D, min(32, n - j0), mx, l, o);
+        if ((pg & 1) == (warp >> 2))
+            for (int j0 = (warp & 3) * 32; j0 < n; j0 += 4 * 32)
+                attn_block<D, G, false>(c, Kp + (size_t)j0 * D, Vp + (size_t)j0 * D, min(32, n - j0), mx, l, o);
         __syncwarp();
         if (lane == 0) mbar_arrive(&c->empty_c[slot]);
         cs.odd_c ^= 1u << slot;
@@ -944,6 +988,7 @@ __device__ void compute_role(const RParams &p, unsigned char *ring, Ctl *c) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     const int qlen = q1 - q0;
     const int tid = threadIdx.x, warp = tid >> 5;
+    const unsigned long long t_begin = p.sm_stats ? globaltimer() : 0ull;
     CState cs;
     for (int step = 0; step < p.n_steps; ++step) {
         cs.step = step;
@@ -955,9 +1000,13 @@ __device__ void compute_role(const RParams &p, unsigned char *ring, Ctl *c) {
                 // released by the scheduler once the dependency has fired
                 const uint32_t k = (uint32_t)(step * qlen + (qi - q0));
                 Spin s;
+                const unsigned long long tr = (p.sm_stats && tid == 0) ? globaltimer() : 0ull;
                 while (ld_acquire_cta_shared(&c->ready_upto) <= k)
                     if (!spin_ok(s, p, c, W_READY, (uint32_t)t.sm, 0u)) return;
+                if (p.sm_stats && tid == 0) *stat_slot(p, RS_CMP_READY) += globaltimer() - tr;
             }
+            const unsigned long long tb = (p.sm_stats && tid == 0) ? globaltimer() : 0ull;
+            const unsigned long long acc0 = (p.sm_stats && tid == 0) ? *stat_slot(p, RS_CMP_ACC) : 0ull;
             if (p.trace && tid == 0) p.trace[t.sm].t_start = globaltimer();
             bool ok = true;
             if (t.kind == ROP_ATTN) {
@@ -971,6 +1020,11 @@ __device__ void compute_role(const RParams &p, unsigned char *ring, Ctl *c) {
                 for (int pg = t.begin; pg < t.end; pg = seg_end(pg, t.end, g.slabs)) ++cs.segs;
             }
             if (!ok) return;
+            if (p.sm_stats && tid == 0) {
+                const unsigned long long dt = globaltimer() - tb;
+                if (t.kind == ROP_ATTN) *stat_slot(p, RS_CMP_ATTN) += dt;
+                else *stat_slot(p, RS_CMP_EPI) += dt - (*stat_slot(p, RS_CMP_ACC) - acc0);
+            }
             if (is_gemv(t.kind) && task_on(p, t, step)) cs.aseq += (uint32_t)(t.end - t.begin);
             // every write of the task is done (and ordered before the bulk
             // copies that read it on other SMs) before its completion posts
@@ -1002,6 +1056,7 @@ __device__ void compute_role(const RParams &p, unsigned char *ring, Ctl *c) {
             if (p.trace && tid == 0) p.trace[t.sm].t_end = globaltimer();
         }
     }
+    if (p.sm_stats && tid == 0) *stat_slot(p, RS_CMP_TOTAL) = globaltimer() - t_begin;
 }
 
 // ---------------------------------------------------------------------------

@@ -84,6 +84,9 @@ MK_HD inline size_t rx_elem(int n, int k) {
 
 // Attention positions per page (K block then V block).
 MK_HD inline int rattn_pos_per_page(int d) { return kRPageBytes / (4 * d); }
+// A row's positions are split into chunks of at least this many (one
+// attention item each); short contexts need no merge.
+constexpr int kRAttnChunk = 1024;
 
 // Per-layer device buffers of the rows step.
 //  xq, xo, xg, xd: the bf16 high/low inputs of QKV (rmsnorm gain folded in,
@@ -171,7 +174,28 @@ struct RParams {
                                 //  issuer began the task's pages; t_start: the compute warps began;
                                 //  t_input: first accumulator (or attention queries) in hand;
                                 //  t_done: epilogue done; t_end: completion posted
+    unsigned long long *sm_stats;   // [num_sms][16] ns spent per wait kind (MK_FLAG_TRACE), or null: RStat
     unsigned long long timeout_ns;
+};
+
+// Per-SM time accounting of the batched step (MK_FLAG_TRACE), ns.
+enum RStat {
+    RS_LOAD_SLOT = 0,    // loader waiting for a free page slot
+    RS_LOAD_TOTAL = 1,
+    RS_SCHED_DEP = 2,    // scheduler waiting on event counters
+    RS_SCHED_SLAB = 3,   // scheduler waiting for a free activation slab slot
+    RS_MMA_PAGE = 4,     // MMA issuer waiting for a weight page
+    RS_MMA_SLAB = 5,     // MMA issuer waiting for an activation slab
+    RS_MMA_ACC = 6,      // MMA issuer waiting for a free accumulator
+    RS_MMA_TOTAL = 7,
+    RS_CMP_READY = 8,    // compute warp 0 waiting for the scheduler
+    RS_CMP_ACC = 9,      // compute warp 0 waiting for an accumulator
+    RS_CMP_KV = 10,      // compute warp 0 waiting for a K/V page
+    RS_CMP_ATTN = 11,    // compute warp 0 in attention items (all of it)
+    RS_CMP_EPI = 12,     // compute warp 0 in GEMV tasks, accumulator waits excluded
+    RS_CMP_TOTAL = 13,
+    RS_CMP_SYNC = 14,    // compute warp 0 in group barriers
+    kRStats = 16
 };
 
 MK_HD inline int rrows_in_step(const RParams &p, int step) {

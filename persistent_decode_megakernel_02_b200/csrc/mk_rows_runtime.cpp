@@ -72,7 +72,7 @@ bool rows_shape_ok(const Shape &s) {
     return true;
 }
 
-int rows_default_chunks(int S) { return (S + kAttnChunkPositions - 1) / kAttnChunkPositions; }
+int rows_default_chunks(int S) { return (S + kRAttnChunk - 1) / kRAttnChunk; }
 
 void rows_destroy(RowsCtx *c) {
     if (!c) return;
@@ -239,6 +239,7 @@ int rows_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, cons
             tr[i] = TraceRec{0, 0, 0, 0, 0, 0, t.sm, t.kind, t.layer, t.trig};
         }
         RK_TRY(ralloc(c, &p.trace, c->num_tasks));
+        RK_TRY(ralloc(c, &p.sm_stats, (size_t)num_sms * kRStats, true));
         RK_TRY(cudaMemcpy(p.trace, tr.data(), sizeof(TraceRec) * c->num_tasks, cudaMemcpyHostToDevice));
     }
     RK_TRY(rows_prepare());

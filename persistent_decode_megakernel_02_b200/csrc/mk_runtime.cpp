@@ -626,7 +626,13 @@ int mk_get_trace(mk_ctx *c, mk_trace_rec *host_out, int n) {
 }
 
 int mk_get_sm_stats(mk_ctx *c, uint64_t *host_out, int n) {
-    if (!c || !host_out || n < 0 || n > c->num_sms * kStatSlots || c->rows) return MK_ERR_INVALID;
+    if (!c || !host_out || n < 0 || n > c->num_sms * kStatSlots) return MK_ERR_INVALID;
+    if (c->rows) {
+        if (!c->rp.sm_stats) return MK_ERR_INVALID;
+        if (cudaMemcpy(host_out, c->rp.sm_stats, sizeof(uint64_t) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return MK_ERR_CUDA;
+        return MK_OK;
+    }
     if (!c->p.sm_stats) return MK_ERR_INVALID;
     if (cudaMemcpy(host_out, c->p.sm_stats, sizeof(uint64_t) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
         return MK_ERR_CUDA;
