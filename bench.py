@@ -512,6 +512,8 @@ def main():
     weights = wl.make_weights(shape, seed=1234, device=dev)
     kc, vc = wl.make_kv(shape, 1, max_seq, device=dev, prefill_len=prefill)
     ctx = mk.Context(weights, kc, vc, max_seq, 1, flags=args.flags, attn_chunks=args.attn_chunks)
+    inf = ctx.info()
+    config["attention_items"] = {"q_heads_per_item": inf.attn_heads, "chunks": inf.attn_chunks}
     stream = torch.cuda.Stream(device=dev)
     prompt = torch.from_numpy(wl.make_prompt(shape.vocab, W, seed=42)).to(dev)
     toks = torch.zeros(W + K + 1, dtype=torch.int32, device=dev)

@@ -84,7 +84,21 @@ enum mk_flags {
     /* Run steps on the batched tensor-core kernel even with max_batch = 1,
      * which mk_prefill needs (contexts with max_batch > 1 always use it).
      * See "Batched steps" below. */
-    MK_FLAG_ROWS = 16
+    MK_FLAG_ROWS = 16,
+    /* Work items of the attention op (scaled dot-product attention over the
+     * KV cache, split into chunks of positions whose partial softmax states
+     * are merged exactly -- the chunked attention of the Flash-Decoding
+     * scheme the "Mirage Persistent Kernel" page's attention tasks follow).
+     * With MK_FLAG_ATTN_KV_ITEMS an item is (sequence, KV head, chunk) and
+     * computes every q head that shares the KV head (up to 512 / head_dim
+     * of them: a larger group is split), reading each K/V page once; with
+     * MK_FLAG_ATTN_Q_ITEMS an item is (sequence, q head, chunk).  Neither:
+     * KV-head items when a full cache would need more chunks per q head
+     * (ceil(max_seq / 1024)) than the SMs give (SMs / (max_batch *
+     * n_q_heads)), else q-head items.  Both: MK_ERR_INVALID.  The batched
+     * kernel always uses KV-head items. */
+    MK_FLAG_ATTN_KV_ITEMS = 32,
+    MK_FLAG_ATTN_Q_ITEMS = 64
 };
 
 /* Upper bounds of the shapes the kernel tiles. */
@@ -100,11 +114,12 @@ enum mk_flags {
  *  n_kv_heads: 1, 2, 4 or 8.  max_seq: KV capacity per sequence (positions
  *  0..max_seq-1).  max_batch: 1..MK_MAX_BATCH (above 1 see "Batched
  *  steps").  rms_eps > 0, rope_theta > 1.
- *  attn_chunks: most split-K chunks per (sequence, q head) in the
- *  attention op (a step uses ceil(context / 1024) of them, so contexts up
- *  to 1024 positions need no merge); 0 picks min(SMs / (max_batch *
- *  n_q_heads), ceil(max_seq / 1024)).  At most 4096 and chunks * (head_dim
- *  + 2) <= 8192.
+ *  attn_chunks: most split-K chunks per attention item (see
+ *  MK_FLAG_ATTN_KV_ITEMS; a step uses ceil(context / 1024) of them, so
+ *  contexts up to 1024 positions need no merge); 0 picks min(SMs /
+ *  (max_batch * items per chunk), ceil(max_seq / 1024)), items per chunk
+ *  being n_q_heads or n_q_heads / heads per item.  At most 4096 and chunks *
+ *  heads per item * (head_dim + 2) <= 8192.
  *  timeout_ns: bound on every device-side wait; 0 means 2 s.
  *  l2_lookahead_kb: how far (KiB of weights per SM) the loader bulk-
  *  prefetches into L2 beyond the pages it has copied into shared memory;
@@ -308,6 +323,7 @@ typedef struct mk_info {
     long long steps_run; /* decode steps enqueued since create/reset (mk_generate adds n_steps) */
     unsigned int err_code, err_info; /* device error word (0 = none); err_info = which wait << 24 | detail */
     unsigned int err_task;           /* task id the device error was raised in (0xffffffff: none) */
+    int attn_heads;                  /* q heads per attention item (MK_FLAG_ATTN_KV_ITEMS) */
 } mk_info;
 
 int mk_get_info(mk_ctx *ctx, mk_info *out);

@@ -14,20 +14,41 @@
 // so far, so the per-SM loaders see equal totals.
 //
 // No heap allocation: the caller sizes the arrays with plan_sizes().
+#include "mk.h"
 #include "mk_internal.h"
 
 namespace mk {
 
 static constexpr int kMaxSms = 1024;
 
-int default_attn_chunks(int num_sms, int Bmax, int nq, int S) {
-    int per = Bmax * nq;
-    int nc = per > 0 ? num_sms / per : 1;
-    if (nc < 1) nc = 1;
-    int cap = (S + kAttnChunkPositions - 1) / kAttnChunkPositions;   // chunks a full cache needs
+bool plan_attention(Shape &s, int num_sms, int flags, int attn_chunks) {
+    const bool kv = (flags & MK_FLAG_ATTN_KV_ITEMS) != 0, qi = (flags & MK_FLAG_ATTN_Q_ITEMS) != 0;
+    if (kv && qi) return false;
+    // q heads an item could take: the largest divisor of G whose heads fit
+    // the item's shared state
+    int hg = 1;
+    for (int h = s.G; h > 1; --h)
+        if (s.G % h == 0 && h * s.d <= kAttnHeadDims) { hg = h; break; }
+    int cap = (s.S + kAttnChunkPositions - 1) / kAttnChunkPositions;   // chunks a full cache needs
     if (cap < 1) cap = 1;
-    if (nc > cap) nc = cap;
-    return nc;
+    int per_q = num_sms / (s.Bmax * s.nq);                             // chunks per q head the SMs give
+    if (per_q < 1) per_q = 1;
+    s.HA = (kv || (!qi && cap > per_q)) ? hg : 1;
+    // chosen by default, KV-head items give way to q-head items where a
+    // given chunk count's partials would not fit the merge's staging area
+    if (!kv && s.HA > 1 && attn_chunks > 0 && (long long)attn_chunks * s.HA * (s.d + 2) > kStageFloats)
+        s.HA = 1;
+    int nc = attn_chunks;
+    if (nc <= 0) {
+        nc = num_sms / (s.Bmax * (s.nq / s.HA));
+        if (nc < 1) nc = 1;
+        if (nc > cap) nc = cap;
+        const int fit = kStageFloats / (s.HA * (s.d + 2));
+        if (nc > fit) nc = fit;
+    }
+    s.NC = nc;
+    // every head's chunk partials of an item must fit the merge's staging area
+    return nc <= 4096 && (long long)nc * s.HA * (s.d + 2) <= kStageFloats;
 }
 
 // Tiles per scheduling unit of a GEMV op: tasks of ops whose pages pass
@@ -128,7 +149,7 @@ struct Builder {
         OpTiles t = op_tiles(s);
         int per_chunk = (s.S + s.NC - 1) / s.NC;
         int64_t est = (int64_t)4 * s.d * per_chunk;   // K + V bf16 of one chunk at capacity
-        const int heads = s.Bmax * s.nq;              // items per chunk index
+        const int heads = s.Bmax * (s.nq / s.HA);     // items per chunk index
         for (int i = 0; i < t.attn_items; i += p.num_sms) {
             sort_by_load();
             int n = t.attn_items - i < p.num_sms ? t.attn_items - i : p.num_sms;

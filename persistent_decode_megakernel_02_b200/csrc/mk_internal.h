@@ -47,6 +47,9 @@ constexpr int kMaxBatch = 1;        // sequences per step (MK_MAX_BATCH)
 // chunks of at least this many positions (shorter contexts use fewer chunks;
 // one chunk needs no merge).
 constexpr int kAttnChunkPositions = 1024;
+// q heads of one attention item, times head_dim, at most (the item's
+// per-warp softmax states and queries live in the shared staging area).
+constexpr int kAttnHeadDims = 512;
 constexpr int kMaxHeadDim = 256;
 constexpr long long kL2Lookahead = 0;  // default L2 prefetch distance beyond the ring (0: off; measured no gain)
 constexpr int kStageFloats = 8192;  // shared staging: a GEMV input vector, or attention partials
@@ -93,6 +96,8 @@ struct Shape {
     int tmem;         // 1: GEMV pages of 2048-column rows pass through tensor memory
                       //    (weights in the TMEM page order, tasks start on page boundaries)
     int G;            // nq / nkv
+    int HA;           // q heads per attention item: 1, or a divisor of G (the
+                      //  q heads of one KV head share the item's K/V pages)
     int QD, KD;       // nq*d, nkv*d
     float theta, eps;
 };
@@ -109,7 +114,7 @@ struct OpTiles {
     int gateup;
     int down;
     int lmhead;
-    int attn_items;   // Bmax * nq * NC
+    int attn_items;   // Bmax * (nq / HA) * NC
 };
 
 MK_HD inline OpTiles op_tiles(const Shape &s) {
@@ -119,7 +124,7 @@ MK_HD inline OpTiles op_tiles(const Shape &s) {
     t.gateup = s.F / 8;
     t.down = s.H / 8;
     t.lmhead = (s.V + 7) / 8;
-    t.attn_items = s.Bmax * s.nq * s.NC;
+    t.attn_items = s.Bmax * (s.nq / s.HA) * s.NC;
     return t;
 }
 
@@ -340,6 +345,10 @@ PlanSizes plan_sizes(const Shape &s, int num_sms);
 void plan_build(const Shape &s, int num_sms, Plan &p);
 
 // Default number of attention chunks for a shape on `num_sms` SMs.
-int default_attn_chunks(int num_sms, int Bmax, int nq, int S);
+// Attention planning (mk_graph.cpp): sets s.HA and s.NC from the config
+// (flags MK_FLAG_ATTN_KV_ITEMS / MK_FLAG_ATTN_Q_ITEMS, attn_chunks) and the
+// SM count; false when the chunk partials of an item's heads would not fit
+// the merge's staging area.
+bool plan_attention(Shape &s, int num_sms, int flags, int attn_chunks);
 
 }  // namespace mk

@@ -222,8 +222,9 @@ struct AttnChunk {
 __device__ __forceinline__ AttnChunk attn_chunk(const Params &p, const SmemCtl *ctl, int step, int item) {
     const Shape &s = p.s;
     AttnChunk a;
-    a.b = item / (s.nq * s.NC);
-    a.h = (item / s.NC) % s.nq;
+    const int groups = s.nq / s.HA;          // items per (sequence, chunk)
+    a.b = item / (groups * s.NC);
+    a.h = ((item / s.NC) % groups) * s.HA;   // the item's first q head
     a.kvh = a.h / s.G;
     a.c = item % s.NC;
     a.active = a.b < p.batch;
@@ -652,12 +653,6 @@ __device__ __forceinline__ void release_tpage(SmemCtl *ctl, WState &w) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(&ctl->tempty[w.tslot]);
     if (++w.tslot == (uint32_t)kTmemSlots) { w.tslot = 0; w.tphase ^= 1u; }
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
 }
 
 // Sum of one float over the 256 worker threads (bounded barrier inside).
@@ -1597,6 +1592,8 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     phase_end(w, tp, WS_PRO);
     stamp_input(p, w);
 
+    // l: this lane's share of the softmax sum (m is warp-uniform, so the
+    // shares add up after the loop)
     float m = -INFINITY, l = 0.f, o[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) o[i] = 0.f;
@@ -1612,50 +1609,58 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
             float sc = -INFINITY;
             if (j < n) {
                 const uint4 *krow = reinterpret_cast<const uint4 *>(Kp + (size_t)j * D);
-                float2 acc = make_float2(0.f, 0.f);
+                float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < NCH; ++c) {
                     const int cc = (c + lane) & (NCH - 1);
                     const uint4 kw = krow[cc];
                     const float4 q0 = *reinterpret_cast<const float4 *>(qs + 12 * cc);
                     const float4 q1 = *reinterpret_cast<const float4 *>(qs + 12 * cc + 4);
-                    acc = ffma2(make_float2(bf_lo(kw.x), bf_hi(kw.x)), make_float2(q0.x, q0.y), acc);
-                    acc = ffma2(make_float2(bf_lo(kw.y), bf_hi(kw.y)), make_float2(q0.z, q0.w), acc);
-                    acc = ffma2(make_float2(bf_lo(kw.z), bf_hi(kw.z)), make_float2(q1.x, q1.y), acc);
-                    acc = ffma2(make_float2(bf_lo(kw.w), bf_hi(kw.w)), make_float2(q1.z, q1.w), acc);
+                    a0 = ffma2(make_float2(bf_lo(kw.x), bf_hi(kw.x)), make_float2(q0.x, q0.y), a0);
+                    a1 = ffma2(make_float2(bf_lo(kw.y), bf_hi(kw.y)), make_float2(q0.z, q0.w), a1);
+                    a0 = ffma2(make_float2(bf_lo(kw.z), bf_hi(kw.z)), make_float2(q1.x, q1.y), a0);
+                    a1 = ffma2(make_float2(bf_lo(kw.w), bf_hi(kw.w)), make_float2(q1.z, q1.w), a1);
                 }
-                sc = acc.x + acc.y;
+                sc = (a0.x + a0.y) + (a1.x + a1.y);
             }
-            float mb = sc;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
-            const float mn = fmaxf(m, mb);             // finite: lane 0's position is valid
+            const float mn = fmaxf(m, warp_max(sc));    // finite: lane 0's position is valid
             const float corr = expf(m - mn);
             const float pe = j < n ? expf(sc - mn) : 0.f;
-            l = l * corr + warp_sum(pe);
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) o[i] *= corr;
+            l = fmaf(l, corr, pe);
             m = mn;
-            const int cnt = min(32, n - j0);
             const uint16_t *vb = Vp + (size_t)j0 * D + lane * DPL;
-            for (int k = 0; k < cnt; ++k) {
+            // P·V over the block's positions, two independent sums
+            float ta[DPL], tb[DPL];
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) { ta[i] = 0.f; tb[i] = 0.f; }
+            auto pv = [&](int k, float *t) {
                 const float pk = __shfl_sync(0xffffffffu, pe, k);
                 if constexpr (DPL == 2) {
                     const uint32_t vw = *reinterpret_cast<const uint32_t *>(vb + (size_t)k * D);
-                    o[0] = fmaf(pk, bf_lo(vw), o[0]);
-                    o[1] = fmaf(pk, bf_hi(vw), o[1]);
+                    t[0] = fmaf(pk, bf_lo(vw), t[0]);
+                    t[1] = fmaf(pk, bf_hi(vw), t[1]);
                 } else {
                     const uint2 vw = *reinterpret_cast<const uint2 *>(vb + (size_t)k * D);
-                    o[0] = fmaf(pk, bf_lo(vw.x), o[0]);
-                    o[1] = fmaf(pk, bf_hi(vw.x), o[1]);
-                    o[2] = fmaf(pk, bf_lo(vw.y), o[2]);
-                    o[3] = fmaf(pk, bf_hi(vw.y), o[3]);
+                    t[0] = fmaf(pk, bf_lo(vw.x), t[0]);
+                    t[1] = fmaf(pk, bf_hi(vw.x), t[1]);
+                    t[2] = fmaf(pk, bf_lo(vw.y), t[2]);
+                    t[3] = fmaf(pk, bf_hi(vw.y), t[3]);
                 }
+            };
+            if (j0 + 32 <= n) {
+#pragma unroll
+                for (int k = 0; k < 32; k += 2) { pv(k, ta); pv(k + 1, tb); }
+            } else {
+                const int cnt = n - j0;
+                for (int k = 0; k < cnt; ++k) pv(k, ta);
             }
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) o[i] = fmaf(o[i], corr, ta[i] + tb[i]);
         }
         release_page(ctl, w, slot);
         phase_end(w, tp, WS_DOT);
     }
+    l = warp_sum(l);
     tp = phase_begin(w);
     if (new_warp) {
         float sc = 0.f;
@@ -1739,13 +1744,353 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     return true;
 }
 
+// Attention item of HA q heads sharing one KV head (MK_FLAG_ATTN_KV_ITEMS,
+// the default for long caches): the same chunk, pages and merge as
+// attn_task, but every K row a lane reads is scored against all HA queries
+// and every V row a lane reads feeds all HA outputs, so the item reads its
+// KV head's positions once for the group.  The block loop: lane j scores
+// position j for each head (rotated 16-byte chunk order against the padded
+// queries in shared memory), the warp takes the per-head maximum in one
+// instruction, the softmax weights go to a per-warp slot of shared memory,
+// and P·V broadcasts them from there (one vector load per position for all
+// heads) with lanes over head dims.  Softmax sums are kept per lane and
+// added up once after the pages.
+template <int D, int HA>   // head_dim 64 or 128; q heads per item, HA * D <= kAttnHeadDims
+__device__ bool attn_kv_task(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
+                             WState &w) {
+    const Shape &s = p.s;
+    constexpr int DPL = D / 32;                  // head dims per lane in P·V
+    constexpr int NCH = D / 8;                   // 16-byte chunks of a K row
+    constexpr int KP = DPL / 2;                  // tagged pairs of the new k (and v) per lane
+    constexpr int QST = 12 * NCH;                // floats of one head's padded query
+    constexpr int QN = HA * D / 2;               // rotation pairs of the item's queries
+    constexpr int QR = (QN + kWorkerThreads - 1) / kWorkerThreads;
+    constexpr int CMB = HA * (D + 2);            // per-warp combine slot: o of each head, then (m, l) pairs
+    constexpr int NB = 2 * QR + 2 * KP;          // pending bits of the input poll
+    static_assert(HA * D <= kAttnHeadDims, "item heads fit");
+    static_assert(kWorkerWarps * CMB + HA * QST + kWorkerWarps * 32 * HA <= kStageFloats, "stage");
+    static_assert(NB <= 32, "poll bits");
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const AttnChunk a = attn_chunk(p, ctl, ctl->wstep, t.begin);
+    const int npp = attn_pos_per_page(D);
+    if (!wait_ready(p, ctl, w)) return false;
+    unsigned long long tp = phase_begin(w);
+    const int npages = (a.npre + npp - 1) / npp;
+    float *qs = ctl->stage + kWorkerWarps * CMB;          // head hh, chunk c at qs + hh * QST + 12 c
+    float *pb = qs + HA * QST + warp * 32 * HA;           // this warp's weights [32 positions][HA]
+
+    // ---- the queries (thread i < QN takes element pair (e, e + D/2) of
+    // head i / (D/2), the pair RoPE rotates together) and the new k / v
+    // (warp 0), tagged, polled until fresh
+    const bool new_warp = a.has_new && warp == 0;
+    float kn[DPL], vn[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) { kn[i] = 0.f; vn[i] = 0.f; }
+    if (a.active) {
+        const uint64_t *qsrc = tag_buf(p, t.layer, p.tl.q) + (size_t)a.b * s.QD + (size_t)a.h * D;
+        const uint64_t *ksrc = tag_buf(p, t.layer, p.tl.kn) + (size_t)a.b * s.KD + (size_t)a.kvh * D + lane * DPL;
+        const uint64_t *vsrc = tag_buf(p, t.layer, p.tl.vn) + (size_t)a.b * s.KD + (size_t)a.kvh * D + lane * DPL;
+        float qv[2 * QR];
+#pragma unroll
+        for (int i = 0; i < 2 * QR; ++i) qv[i] = 0.f;
+        uint32_t pend = 0;
+        auto load = [&](int bit) {
+            bool ok;
+            if (bit < 2 * QR) {
+                const int i = tid + (bit >> 1) * kWorkerThreads;
+                const int hh = i / (D / 2), e = i % (D / 2);
+                const uint64_t v = ld_tag1(qsrc + hh * D + e + ((bit & 1) ? D / 2 : 0));
+                qv[bit] = tag_val(v);
+                ok = tag_ok(v, w.ep);
+            } else {
+                const int bb = bit - 2 * QR;
+                const bool isk = bb < KP;
+                const int h = isk ? bb : bb - KP;
+                const ulonglong2 v = ld_tag2((isk ? ksrc : vsrc) + 2 * h);
+                float *dst = isk ? kn : vn;
+                dst[2 * h] = tag_val(v.x);
+                dst[2 * h + 1] = tag_val(v.y);
+                ok = tag_ok(v.x, w.ep) && tag_ok(v.y, w.ep);
+            }
+            if (ok) pend &= ~(1u << bit);
+            else pend |= 1u << bit;
+        };
+#pragma unroll
+        for (int bit = 0; bit < NB; ++bit)
+            if (bit < 2 * QR ? tid + (bit >> 1) * kWorkerThreads < QN : new_warp) load(bit);
+        Spin sp;
+        while (__any_sync(0xffffffffu, pend != 0u)) {
+            if (!warp_spin_ok(sp, p, ctl, (uint32_t)w.task_id, 4u)) return false;
+#pragma unroll
+            for (int bit = 0; bit < NB; ++bit)
+                if (pend & (1u << bit)) load(bit);
+        }
+        const float scale = 1.0f / sqrtf((float)D);
+#pragma unroll
+        for (int r = 0; r < QR; ++r) {
+            const int i = tid + r * kWorkerThreads;
+            if (i < QN) {
+                const int hh = i / (D / 2), e = i % (D / 2), f = e + D / 2;
+                const float2 cs = p.rope[(size_t)a.P * (D / 2) + e];
+                float *qh = qs + hh * QST;
+                qh[12 * (e >> 3) + (e & 7)] = (qv[2 * r] * cs.x - qv[2 * r + 1] * cs.y) * scale;
+                qh[12 * (f >> 3) + (f & 7)] = (qv[2 * r + 1] * cs.x + qv[2 * r] * cs.y) * scale;
+            }
+        }
+        if (new_warp) {
+            // rotate the new key (the partner of an element sits D/2 further,
+            // in lane L ^ 16), round it to bf16 as the cache stores it; the
+            // item holding the group's first q head appends it
+            uint16_t kb[DPL];
+#pragma unroll
+            for (int j = 0; j < DPL; ++j) {
+                const float other = __shfl_xor_sync(0xffffffffu, kn[j], 16);
+                const int e = lane * DPL + j;
+                const int i = e % (D / 2);
+                const float2 cs = p.rope[(size_t)a.P * (D / 2) + i];
+                const float r = lane < 16 ? kn[j] * cs.x - other * cs.y : kn[j] * cs.x + other * cs.y;
+                kb[j] = f2bf(r);
+            }
+#pragma unroll
+            for (int j = 0; j < DPL; ++j) kn[j] = bf2f(kb[j]);
+            if (a.h % s.G == 0) {
+                uint16_t *kc = p.layers[t.layer].kc + (((size_t)a.b * s.nkv + a.kvh) * s.S + a.P) * D + lane * DPL;
+#pragma unroll
+                for (int j = 0; j < DPL; ++j) kc[j] = kb[j];
+            }
+        }
+    }
+    if (!worker_sync(p, ctl, w)) return false;   // queries visible to every warp
+    stamp_ready(p, w);
+    phase_end(w, tp, WS_PRO);
+    stamp_input(p, w);
+
+    float m[HA], l[HA], o[HA][DPL];   // l: this lane's share of the softmax sum
+#pragma unroll
+    for (int hh = 0; hh < HA; ++hh) {
+        m[hh] = -INFINITY;
+        l[hh] = 0.f;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) o[hh][i] = 0.f;
+    }
+    for (int pg = 0; pg < npages; ++pg) {
+        uint32_t slot;
+        if (!wait_page(p, ctl, w, slot)) return false;
+        tp = phase_begin(w);
+        const uint16_t *Kp = reinterpret_cast<const uint16_t *>(pages + (size_t)slot * kPageBytes);
+        const uint16_t *Vp = Kp + (size_t)npp * D;
+        const int n = min(npp, a.npre - pg * npp);
+        for (int j0 = warp * 32; j0 < n; j0 += kWorkerWarps * 32) {
+            const int j = j0 + lane;
+            float sc[HA];
+            if (j < n) {
+                const uint4 *krow = reinterpret_cast<const uint4 *>(Kp + (size_t)j * D);
+                float2 a0[HA], a1[HA];
+#pragma unroll
+                for (int hh = 0; hh < HA; ++hh) { a0[hh] = make_float2(0.f, 0.f); a1[hh] = make_float2(0.f, 0.f); }
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) {
+                    const int cc = (c + lane) & (NCH - 1);
+                    const uint4 kw = krow[cc];
+                    const float2 k01 = make_float2(bf_lo(kw.x), bf_hi(kw.x));
+                    const float2 k23 = make_float2(bf_lo(kw.y), bf_hi(kw.y));
+                    const float2 k45 = make_float2(bf_lo(kw.z), bf_hi(kw.z));
+                    const float2 k67 = make_float2(bf_lo(kw.w), bf_hi(kw.w));
+#pragma unroll
+                    for (int hh = 0; hh < HA; ++hh) {
+                        const float4 q0 = *reinterpret_cast<const float4 *>(qs + hh * QST + 12 * cc);
+                        const float4 q1 = *reinterpret_cast<const float4 *>(qs + hh * QST + 12 * cc + 4);
+                        a0[hh] = ffma2(k01, make_float2(q0.x, q0.y), a0[hh]);
+                        a1[hh] = ffma2(k23, make_float2(q0.z, q0.w), a1[hh]);
+                        a0[hh] = ffma2(k45, make_float2(q1.x, q1.y), a0[hh]);
+                        a1[hh] = ffma2(k67, make_float2(q1.z, q1.w), a1[hh]);
+                    }
+                }
+#pragma unroll
+                for (int hh = 0; hh < HA; ++hh) sc[hh] = (a0[hh].x + a0[hh].y) + (a1[hh].x + a1[hh].y);
+            } else {
+#pragma unroll
+                for (int hh = 0; hh < HA; ++hh) sc[hh] = -INFINITY;
+            }
+            float pe[HA], corr[HA];
+#pragma unroll
+            for (int hh = 0; hh < HA; ++hh) {
+                const float mn = fmaxf(m[hh], warp_max(sc[hh]));   // finite: lane 0's position is valid
+                corr[hh] = expf(m[hh] - mn);
+                pe[hh] = j < n ? expf(sc[hh] - mn) : 0.f;
+                l[hh] = fmaf(l[hh], corr[hh], pe[hh]);
+                m[hh] = mn;
+            }
+            if constexpr (HA % 4 == 0) {
+#pragma unroll
+                for (int hh = 0; hh < HA; hh += 4)
+                    *reinterpret_cast<float4 *>(pb + lane * HA + hh) = make_float4(pe[hh], pe[hh + 1], pe[hh + 2], pe[hh + 3]);
+            } else {
+                *reinterpret_cast<float2 *>(pb + lane * HA) = make_float2(pe[0], pe[1]);
+            }
+            __syncwarp();
+            const uint16_t *vb = Vp + (size_t)j0 * D + lane * DPL;
+            float tv[HA][DPL];
+#pragma unroll
+            for (int hh = 0; hh < HA; ++hh)
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) tv[hh][i] = 0.f;
+            auto pv = [&](int k) {
+                float pk[HA];
+                if constexpr (HA % 4 == 0) {
+#pragma unroll
+                    for (int hh = 0; hh < HA; hh += 4) {
+                        const float4 q = *reinterpret_cast<const float4 *>(pb + k * HA + hh);
+                        pk[hh] = q.x; pk[hh + 1] = q.y; pk[hh + 2] = q.z; pk[hh + 3] = q.w;
+                    }
+                } else {
+                    const float2 q = *reinterpret_cast<const float2 *>(pb + k * HA);
+                    pk[0] = q.x; pk[1] = q.y;
+                }
+                float v[DPL];
+                if constexpr (DPL == 2) {
+                    const uint32_t vw = *reinterpret_cast<const uint32_t *>(vb + (size_t)k * D);
+                    v[0] = bf_lo(vw); v[1] = bf_hi(vw);
+                } else {
+                    const uint2 vw = *reinterpret_cast<const uint2 *>(vb + (size_t)k * D);
+                    v[0] = bf_lo(vw.x); v[1] = bf_hi(vw.x); v[2] = bf_lo(vw.y); v[3] = bf_hi(vw.y);
+                }
+#pragma unroll
+                for (int hh = 0; hh < HA; ++hh)
+#pragma unroll
+                    for (int i = 0; i < DPL; ++i) tv[hh][i] = fmaf(pk[hh], v[i], tv[hh][i]);
+            };
+            if (j0 + 32 <= n) {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) pv(k);
+            } else {
+                const int cnt = n - j0;
+                for (int k = 0; k < cnt; ++k) pv(k);
+            }
+#pragma unroll
+            for (int hh = 0; hh < HA; ++hh)
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) o[hh][i] = fmaf(o[hh][i], corr[hh], tv[hh][i]);
+            __syncwarp();   // the weights slot is rewritten by the next block
+        }
+        release_page(ctl, w, slot);
+        phase_end(w, tp, WS_DOT);
+    }
+#pragma unroll
+    for (int hh = 0; hh < HA; ++hh) l[hh] = warp_sum(l[hh]);
+    tp = phase_begin(w);
+    if (new_warp) {
+#pragma unroll
+        for (int hh = 0; hh < HA; ++hh) {
+            float sc = 0.f;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) {
+                const int e = lane * DPL + i;
+                sc = fmaf(qs[hh * QST + 12 * (e >> 3) + (e & 7)], kn[i], sc);
+            }
+            sc = warp_sum(sc);
+            const float mn = fmaxf(m[hh], sc);
+            const float corr = expf(m[hh] - mn);
+            const float pe = expf(sc - mn);
+            l[hh] = l[hh] * corr + pe;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) o[hh][i] = fmaf(o[hh][i], corr, pe * vn[i]);
+            m[hh] = mn;
+        }
+    }
+
+    // ---- combine the warps' states
+    float *cw = ctl->stage + warp * CMB;
+#pragma unroll
+    for (int hh = 0; hh < HA; ++hh) {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) cw[hh * D + lane * DPL + i] = o[hh][i];
+        if (lane == 0) { cw[HA * D + 2 * hh] = m[hh]; cw[HA * D + 2 * hh + 1] = l[hh]; }
+    }
+    if (!worker_sync(p, ctl, w)) return false;
+    // the partials of q head h: [NC][D + 2] at part + (b * nq + h) * NC * (D + 2)
+    uint64_t *part = tag_buf(p, t.layer, p.tl.part) + ((size_t)a.b * s.nq + a.h) * s.NC * (D + 2);
+    uint64_t *attn = tag_buf(p, t.layer, p.tl.attn) + (size_t)a.b * s.QD + (size_t)a.h * D;
+    if (a.active && a.c < a.nc) {
+        for (int i = tid; i < HA * D; i += kWorkerThreads) {
+            const int hh = i / D, e = i % D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < kWorkerWarps; ++k) M = fmaxf(M, ctl->stage[k * CMB + HA * D + 2 * hh]);
+            float O = 0.f, L = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int k = 0; k < kWorkerWarps; ++k) {
+                    const float *ck = ctl->stage + k * CMB;
+                    const float f = expf(ck[HA * D + 2 * hh] - M);
+                    O = fmaf(f, ck[hh * D + e], O);
+                    L = fmaf(f, ck[HA * D + 2 * hh + 1], L);
+                }
+            }
+            if (a.nc == 1) {
+                st_tag_rep(attn + i, p.tl.rep_qd, O / L, w.ep_out);
+            } else {
+                uint64_t *dst = part + ((size_t)hh * s.NC + a.c) * (D + 2);
+                st_tag(dst + e, O, w.ep_out);
+                if (e == 0) {
+                    st_tag(dst + D, M, w.ep_out);
+                    st_tag(dst + D + 1, L, w.ep_out);
+                }
+            }
+        }
+    }
+    stamp_done(p, w);
+    if (a.active && a.nc > 1 && a.c == 0) {
+        // chunk 0's item merges the partials of its q heads: polls them into
+        // shared memory ([head][chunk][D + 2]; tagged, so it waits for
+        // exactly the chunks it reads), then combines them there
+        const int nc = a.nc;
+        if (!worker_sync(p, ctl, w)) return false;   // the combine above is done with the stage
+        if (!stage_partials(p, ctl, w, part, HA, nc * (D + 2), s.NC * (D + 2))) return false;
+        if (!worker_sync(p, ctl, w)) return false;
+        for (int i = tid; i < HA * D; i += kWorkerThreads) {
+            const int hh = i / D, e = i % D;
+            const float *sg = ctl->stage + (size_t)hh * nc * (D + 2);
+            float M = -INFINITY;
+            for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (D + 2) + D]);
+            float num = 0.f, den = 0.f;
+            for (int c = 0; c < nc; ++c) {
+                const float mc = sg[c * (D + 2) + D];
+                if (mc == -INFINITY) continue;
+                const float f = expf(mc - M);
+                num = fmaf(f, sg[c * (D + 2) + e], num);
+                den = fmaf(f, sg[c * (D + 2) + D + 1], den);
+            }
+            st_tag_rep(attn + i, p.tl.rep_qd, num / den, w.ep_out);
+        }
+    }
+    if (!worker_sync(p, ctl, w)) return false;
+    if (tid == 0) signal_event(p, ctl, t);
+    phase_end(w, tp, WS_ATT);
+    return true;
+}
+
 // ---------------------------------------------------------------------------
 // worker role
 // ---------------------------------------------------------------------------
+// KVI: the kernel instantiation with KV-head attention items (Shape::HA >
+// 1); the other one holds only the q-head body, so the code of the
+// short-context kernel does not grow with the long-context one's.
+template <bool KVI>
 __device__ bool run_task(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                          WState &w) {
-    if (t.kind == OP_ATTN)   // head_dim 64 or 128 (checked by mk_create)
-        return p.s.d == 64 ? attn_task<64>(p, t, pages, ctl, w) : attn_task<128>(p, t, pages, ctl, w);
+    if (t.kind == OP_ATTN) {   // head_dim 64 or 128, HA * head_dim <= 512 (checked by mk_create)
+        if constexpr (KVI) {
+            const int ha = p.s.HA;
+            if (p.s.d == 64)
+                return ha == 2 ? attn_kv_task<64, 2>(p, t, pages, ctl, w)
+                     : ha == 4 ? attn_kv_task<64, 4>(p, t, pages, ctl, w)
+                               : attn_kv_task<64, 8>(p, t, pages, ctl, w);
+            return ha == 2 ? attn_kv_task<128, 2>(p, t, pages, ctl, w) : attn_kv_task<128, 4>(p, t, pages, ctl, w);
+        } else {
+            return p.s.d == 64 ? attn_task<64>(p, t, pages, ctl, w) : attn_task<128>(p, t, pages, ctl, w);
+        }
+    }
     // Few instantiations on purpose: every body is inlined into the one
     // kernel, and more variants raise the register pressure of the whole and
     // spread the hot loop over more instruction-cache lines.
@@ -1802,6 +2147,7 @@ __device__ __noinline__ bool lm_reduce(const Params &p, SmemCtl *ctl, int step, 
     return true;
 }
 
+template <bool KVI>
 __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl) {
     const int q0 = p.qoff[blockIdx.x], q1 = p.qoff[blockIdx.x + 1];
     const int qlen = q1 - q0;
@@ -1849,7 +2195,7 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
         w.task_id = id;
         w.ep_out = t.trig == p.debug_withhold ? w.ep - 1u : w.ep;
         w.need = (uint32_t)(k + 1);   // the task body waits for it (counter-gated mode)
-        if (!run_task(p, t, pages, ctl, w)) return;
+        if (!run_task<KVI>(p, t, pages, ctl, w)) return;
         const unsigned long long te = phase_begin(w);
         if (t.kind != OP_ATTN) {
             // every output of the task is written (tile epilogues by threads < 8)
@@ -1897,6 +2243,7 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
+template <bool KVI>
 __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char *pages = smem;
@@ -1982,7 +2329,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     }
     if (warp < kWorkerWarps) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kWorkerRegs));
-        worker_role(p, pages, ctl);
+        worker_role<KVI>(p, pages, ctl);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
         if (warp == kLoaderWarp) {
@@ -2013,19 +2360,27 @@ size_t kernel_smem_bytes() { return kSmemBytes; }
 // Registers per thread the kernel was compiled to launch with; the register
 // split (setmaxnreg) is only valid when this equals kLaunchRegs.
 int kernel_launch_regs() {
-    cudaFuncAttributes a;
-    if (cudaFuncGetAttributes(&a, mk_step_kernel) != cudaSuccess) return -1;
-    return a.numRegs;
+    cudaFuncAttributes a, b;
+    if (cudaFuncGetAttributes(&a, mk_step_kernel<false>) != cudaSuccess) return -1;
+    if (cudaFuncGetAttributes(&b, mk_step_kernel<true>) != cudaSuccess) return -1;
+    return a.numRegs == b.numRegs ? a.numRegs : -1;
 }
 
 cudaError_t kernel_prepare() {
-    return cudaFuncSetAttribute(mk_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(mk_step_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(mk_step_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kSmemBytes);
 }
 
 cudaError_t kernel_occupancy(int *blocks_per_sm) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, mk_step_kernel, kThreads,
-                                                         kSmemBytes);
+    int a = 0, b = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, mk_step_kernel<false>, kThreads, kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, mk_step_kernel<true>, kThreads, kSmemBytes);
+    *blocks_per_sm = a < b ? a : b;
+    return e;
 }
 
 // Weights of a GEMV op into the TMEM page order (see tmem_page_src): `src`
@@ -2063,7 +2418,8 @@ cudaError_t kernel_launch(const Params &p, int grid, cudaStream_t stream) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, mk_step_kernel, p);
+    return p.s.HA > 1 ? cudaLaunchKernelEx(&cfg, mk_step_kernel<true>, p)
+                      : cudaLaunchKernelEx(&cfg, mk_step_kernel<false>, p);
 }
 
 }  // namespace mk

@@ -204,6 +204,21 @@ __device__ __forceinline__ float dot8(const uint4 w, const float *x) {
     return a;
 }
 // Packed two-lane fp32 FMA (sm_100): d = a * b + c element-wise on pairs.
+// Sum of v over the full warp (butterfly: every lane gets the total).
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Maximum of v over the full warp in one instruction (sm_100a; NaN inputs
+// are ignored, as by fmaxf).
+__device__ __forceinline__ float warp_max(float v) {
+    float r;
+    asm("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
+
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"

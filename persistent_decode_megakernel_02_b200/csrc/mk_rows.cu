@@ -788,21 +788,15 @@ __device__ __forceinline__ void attn_block(Ctl *c, const uint16_t *K, const uint
 #pragma unroll
         for (int g = 0; g < G; ++g) sc[g] = acc[g].x + acc[g].y;
     }
-    float pe[G];
+    // l: this lane's share of the softmax sum (mx is warp-uniform; the
+    // shares are added up once, after the item's positions)
+    float pe[G], corr[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        float mb = sc[g];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
-        const float mn = fmaxf(mx[g], mb);          // finite: position 0 of the block is valid
-        const float corr = expf(mx[g] - mn);
+        const float mn = fmaxf(mx[g], warp_max(sc[g]));   // finite: position 0 of the block is valid
+        corr[g] = expf(mx[g] - mn);
         pe[g] = lane < n ? expf(sc[g] - mn) : 0.f;
-        float ps = pe[g];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-        l[g] = l[g] * corr + ps;
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) o[g][i] *= corr;
+        l[g] = fmaf(l[g], corr[g], pe[g]);
         mx[g] = mn;
     }
     // the weights of position `lane` for every head, read back below by all
@@ -813,7 +807,12 @@ __device__ __forceinline__ void attn_block(Ctl *c, const uint16_t *K, const uint
     for (int g = 0; g < G; ++g) pv[g] = pe[g];
     pw[lane] = make_float4(pv[0], pv[1], pv[2], pv[3]);
     __syncwarp();
-    for (int k = 0; k < n; ++k) {
+    float tv[G][DPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) tv[g][i] = 0.f;
+    auto pvk = [&](int k) {
         const uint16_t *vr = V + (size_t)k * D + lane * DPL;
         float v[DPL];
         if constexpr (DPL == 2) {
@@ -832,9 +831,19 @@ __device__ __forceinline__ void attn_block(Ctl *c, const uint16_t *K, const uint
 #pragma unroll
         for (int g = 0; g < G; ++g) {
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) o[g][i] = fmaf(pk[g], v[i], o[g][i]);
+            for (int i = 0; i < DPL; ++i) tv[g][i] = fmaf(pk[g], v[i], tv[g][i]);
         }
+    };
+    if (n == 32) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) pvk(k);   // loads independent of the sums: all in flight
+    } else {
+        for (int k = 0; k < n; ++k) pvk(k);
     }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) o[g][i] = fmaf(o[g][i], corr[g], tv[g][i]);
     __syncwarp();   // the next block's weights overwrite pw
 }
 
@@ -892,6 +901,8 @@ __device__ bool attn_task(const RParams &p, unsigned char *ring, Ctl *c, CState 
         for (int j0 = a.c0 + a.nring + warp * 32; j0 < a.c1; j0 += kComputeWarps * 32)
             attn_block<D, G, true>(c, L.kc + (head + j0) * D, L.vc + (head + j0) * D, min(32, a.c1 - j0), mx, l, o);
     }
+#pragma unroll
+    for (int g = 0; g < G; ++g) l[g] = warp_sum(l[g]);
     // combine the warps' states: slot of warp w = G x (o[D], m, l)
     float *st = c->at.st[warp];
 #pragma unroll

@@ -104,15 +104,13 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     if (rows) {
         // the batched step: its own tiling, chunks of at least 1024 positions
         s.tmem = 0;
+        s.HA = s.G;   // items per (row, KV head, chunk)
         s.NC = c->attn_chunks > 0 ? c->attn_chunks : rows_default_chunks(s.S);
         if (s.NC > 4096 || !rows_shape_ok(s)) return MK_ERR_INVALID;
         if (c->flags & MK_FLAG_EVENT_WAIT) return MK_ERR_INVALID;   // tasks always wait on events here
         return MK_OK;
     }
-    s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nq, s.S);
-    if (s.NC > 4096) return MK_ERR_INVALID;
-    // one q head's chunk partials must fit the merge's shared staging area
-    if ((long long)s.NC * (s.d + 2) > kStageFloats) return MK_ERR_INVALID;
+    if (!plan_attention(s, num_sms, c->flags, c->attn_chunks)) return MK_ERR_INVALID;
     return MK_OK;
 }
 
@@ -170,6 +168,7 @@ int mk_plan(const mk_config *cfg, int num_sms, mk_info *info, int32_t *task_out,
         info->num_events = p.num_events;
         info->num_ops = p.num_ops;
         info->attn_chunks = s.NC;
+        info->attn_heads = s.HA;
         info->max_queue = p.max_queue;
         info->page_bytes = rows ? kRPageBytes : kPageBytes;
         info->num_pages = rows ? kRStages : kNumPages;
@@ -553,6 +552,7 @@ int mk_get_info(mk_ctx *c, mk_info *out) {
     out->num_events = c->num_events;
     out->num_ops = c->num_ops;
     out->attn_chunks = c->s.NC;
+    out->attn_heads = c->s.HA;
     out->max_queue = c->max_queue;
     out->page_bytes = c->rows ? kRPageBytes : kPageBytes;
     out->num_pages = c->rows ? kRStages : kNumPages;

@@ -81,11 +81,13 @@ uint64_t fnv1a(uint64_t h, const void *data, size_t n) {
     return h;
 }
 
-uint64_t shape_key(const mk_config *c, int num_sms) {
-    const long long f[] = {c->layers, c->hidden, c->n_q_heads, c->n_kv_heads, c->head_dim, c->ffn,
-                           c->vocab, c->max_seq, c->max_batch, c->attn_chunks, num_sms};
+// Keyed on the planned shape, not on the config: everything that decides the
+// task graph and the scratch layout (the attention items' heads and chunks
+// depend on the flags and the SM count as well as on the sizes).
+uint64_t shape_key(const Shape &s, int num_sms) {
+    const long long f[] = {s.L, s.H, s.nq, s.nkv, s.d, s.F, s.V, s.S, s.Bmax, s.NC, s.HA, s.tmem, num_sms};
     uint64_t h = fnv1a(1469598103934665603ull, f, sizeof f);
-    const float g[] = {c->rope_theta, c->rms_eps};
+    const float g[] = {s.theta, s.eps};
     return fnv1a(h, g, sizeof g);
 }
 
@@ -119,9 +121,7 @@ bool shape_ok(const mk_config *c, int num_sms, Shape &s) {
     s.G = G; s.QD = (int)QD; s.KD = c->n_kv_heads * c->head_dim;
     s.theta = c->rope_theta; s.eps = c->rms_eps;
     s.tmem = 0;   // weights come in the row-major packed layout: pages stay in shared memory
-    s.NC = c->attn_chunks > 0 ? c->attn_chunks : default_attn_chunks(num_sms, s.Bmax, s.nq, s.S);
-    if (s.NC > 4096 || (long long)s.NC * (s.d + 2) > kStageFloats) return false;
-    return true;
+    return plan_attention(s, num_sms, c->flags, c->attn_chunks);
 }
 
 Layout layout_for(const Shape &s, const PlanSizes &z, int num_sms, int num_lm_tasks) {
@@ -215,7 +215,7 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
         lw[l].kc = (uint16_t *)kv->k[l];
         lw[l].vc = (uint16_t *)kv->v[l];
     }
-    const uint64_t skey = shape_key(cfg, ds.num_sms);
+    const uint64_t skey = shape_key(s, ds.num_sms);
     const uint64_t lkey = fnv1a(skey, lw, sizeof(LayerW) * s.L);
     if (!sig.valid || sig.shape_key != skey) {
         // task graph and RoPE table for this shape, in static host storage

@@ -22,6 +22,8 @@ MK_FLAG_NO_L2_PREFETCH = 2
 MK_FLAG_EVENT_WAIT = 4
 MK_FLAG_NO_TMEM_RING = 8
 MK_FLAG_ROWS = 16
+MK_FLAG_ATTN_KV_ITEMS = 32
+MK_FLAG_ATTN_Q_ITEMS = 64
 MAX_BATCH = 16
 MK_BUF_HIDDEN, MK_BUF_Q, MK_BUF_ATTN, MK_BUF_ACT = range(4)
 OP_NAMES = ["qkv", "attn", "oproj", "gateup", "down", "lmhead"]
@@ -74,7 +76,7 @@ class Info(C.Structure):
                 ("num_ops", C.c_int), ("attn_chunks", C.c_int), ("max_queue", C.c_int),
                 ("page_bytes", C.c_int), ("num_pages", C.c_int),
                 ("steps_run", C.c_longlong), ("err_code", C.c_uint), ("err_info", C.c_uint),
-                ("err_task", C.c_uint)]
+                ("err_task", C.c_uint), ("attn_heads", C.c_int)]
 
 
 class TraceRec(C.Structure):

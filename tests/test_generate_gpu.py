@@ -40,7 +40,8 @@ def _generate(pair, first_tok, pos, n, eos=-1):
     return out[:, 0].cpu().numpy(), int(pair.nxt.item())
 
 
-@pytest.mark.parametrize("flags", [0, 4])
+# 32: MK_FLAG_ATTN_KV_ITEMS (the attention items of the long-cache kernel)
+@pytest.mark.parametrize("flags", [0, 4, 32])
 def test_generate_equals_step_by_step_and_oracle(flags):
     shape = wl.TINY
     n = 24

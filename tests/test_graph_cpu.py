@@ -63,7 +63,8 @@ def test_every_row_and_item_covered_once(planned):
             if (kind == LMHEAD) != (layer == shape.layers):
                 assert len(sel) == 0
                 continue
-            n = shape.n_q_heads * nc if kind == ATTN else tiles[kind]
+            ha = pl["info"].attn_heads
+            n = shape.n_q_heads // ha * nc if kind == ATTN else tiles[kind]
             cover = np.zeros(n, np.int32)
             for t in sel:
                 cover[t[4]:t[5]] += 1
@@ -161,21 +162,47 @@ def test_default_attention_chunks():
     # one task per (sequence, q head, chunk): as many chunks as fill the SMs
     # (148 // 32 q heads = 4), but no more than a full cache needs at 1024
     # positions per chunk
-    assert mk.plan(mk.make_config(wl.LLAMA_1B, 16640), SMS)["info"].attn_chunks == 4
-    assert mk.plan(mk.make_config(wl.LLAMA_1B, 560), SMS)["info"].attn_chunks == 1
-    assert mk.plan(mk.make_config(wl.TINY, 64), SMS)["info"].attn_chunks == 1
-    assert mk.plan(mk.make_config(wl.TINY, 4096), SMS)["info"].attn_chunks == 4
-    assert mk.plan(mk.make_config(wl.TINY, 64, attn_chunks=7), SMS)["info"].attn_chunks == 7
+    def info(shape, S, **kw):
+        return mk.plan(mk.make_config(shape, S, **kw), SMS)["info"]
+    assert (info(wl.LLAMA_1B, 560).attn_chunks, info(wl.LLAMA_1B, 560).attn_heads) == (1, 1)
+    assert (info(wl.TINY, 64).attn_chunks, info(wl.TINY, 64).attn_heads) == (1, 1)
+    assert (info(wl.TINY, 4096).attn_chunks, info(wl.TINY, 4096).attn_heads) == (4, 1)
+    assert info(wl.TINY, 64, attn_chunks=7).attn_chunks == 7
+    assert info(wl.LLAMA_1B, 4096).attn_heads == 1           # 4 chunks per q head reach 1024 positions
+    # a 16k cache needs 17 chunks, the SMs give 4 per q head: one task per
+    # (sequence, KV head, chunk) instead, its 4 q heads together, and
+    # 148 // 8 = 18 chunks, capped at the 17 a full cache needs
+    i = info(wl.LLAMA_1B, 16640)
+    assert (i.attn_heads, i.attn_chunks) == (4, 17)
+    i = info(wl.LLAMA_1B, 16640, flags=mk.MK_FLAG_ATTN_Q_ITEMS)
+    assert (i.attn_heads, i.attn_chunks) == (1, 4)
+    i = info(wl.LLAMA_1B, 560, flags=mk.MK_FLAG_ATTN_KV_ITEMS)
+    assert (i.attn_heads, i.attn_chunks) == (4, 1)
+    # 8B shape: G = 4 at head_dim 128 (4 x 128 <= 512); 16k: 17 chunks fit
+    # the stage only up to 8192 // (4 * 130) = 15
+    i = info(wl.LLAMA_8B, 16640)
+    assert (i.attn_heads, i.attn_chunks) == (4, 15)
+    # a group of 8 q heads of 128 dims is split in halves of 4
+    g8 = wl.ModelShape("g8", 2, 1024, 16, 2, 128, 2048, 4096, True, 1e4)
+    assert info(g8, 64, flags=mk.MK_FLAG_ATTN_KV_ITEMS).attn_heads == 4
+    g8s = wl.ModelShape("g8s", 2, 512, 8, 1, 64, 2048, 4096, True, 1e4)
+    assert info(g8s, 64, flags=mk.MK_FLAG_ATTN_KV_ITEMS).attn_heads == 8
+    # no grouping without shared KV heads
+    mha = wl.ModelShape("mha", 2, 256, 4, 4, 64, 768, 4096, True, 1e4)
+    assert info(mha, 16640, flags=mk.MK_FLAG_ATTN_KV_ITEMS).attn_heads == 1
+    with pytest.raises(mk.MkError):
+        info(wl.TINY, 64, flags=mk.MK_FLAG_ATTN_KV_ITEMS | mk.MK_FLAG_ATTN_Q_ITEMS)
 
 
+@pytest.mark.parametrize("flags", [0, mk.MK_FLAG_ATTN_KV_ITEMS])
 @pytest.mark.parametrize("sms,chunks", [(5, 7), (16, 8), (SMS, 0)])
-def test_attention_merger_runs_after_its_chunks(sms, chunks):
+def test_attention_merger_runs_after_its_chunks(sms, chunks, flags):
     """Chunk 0's task of every (sequence, KV head) merges the partials and
     waits for the other chunks' tagged outputs: on every queue it must come
     after each other chunk of its head, and the whole graph must run to
     completion when tasks wait on exactly their inputs."""
     shape = wl.TINY
-    cfg = mk.make_config(shape, 256, 1, attn_chunks=chunks)
+    cfg = mk.make_config(shape, 256, 1, attn_chunks=chunks, flags=flags)
     pl = mk.plan(cfg, sms)
     tasks, queue, qoff = pl["tasks"], pl["queue"], pl["qoff"]
     NC = pl["info"].attn_chunks
@@ -226,3 +253,15 @@ def test_plan_refuses_partials_that_overflow_the_merge_stage():
     with pytest.raises(mk.MkError) as ei:
         mk.plan(mk.make_config(shape, 64, 1, attn_chunks=125), SMS)
     assert ei.value.status == mk.MK_ERR_INVALID
+    # an item of 2 q heads (MK_FLAG_ATTN_KV_ITEMS, G = 2) stages both heads'
+    # partials: 62 chunks x 2 x 66 fit, 63 do not
+    kv = mk.MK_FLAG_ATTN_KV_ITEMS
+    assert mk.plan(mk.make_config(shape, 64, 1, attn_chunks=62, flags=kv), SMS)["info"].attn_chunks == 62
+    with pytest.raises(mk.MkError):
+        mk.plan(mk.make_config(shape, 64, 1, attn_chunks=63, flags=kv), SMS)
+    # chosen by default for a long cache, KV-head items give way to q-head
+    # items when the given chunk count would not fit with them
+    i = mk.plan(mk.make_config(shape, 126008, 1, attn_chunks=124), SMS)["info"]
+    assert (i.attn_heads, i.attn_chunks) == (1, 124)
+    i = mk.plan(mk.make_config(shape, 126008, 1, attn_chunks=62), SMS)["info"]
+    assert (i.attn_heads, i.attn_chunks) == (2, 62)

@@ -104,6 +104,62 @@ def test_many_active_attention_chunks_merged(head_dim, chunks, prefix):
     _check_hidden(pair, ref)
 
 
+# Attention items of one KV head's q heads together (MK_FLAG_ATTN_KV_ITEMS):
+# many merged chunks (the merge stages every head's partials: 62 chunks x 2
+# heads x 66 floats at head_dim 64, 31 x 2 x 130 at 128).
+KV = 32
+
+
+@pytest.mark.parametrize("head_dim,chunks,prefix", [(64, 13, 13000), (64, 62, 63000), (128, 31, 32000)])
+def test_kv_head_items_many_chunks_merged(head_dim, chunks, prefix):
+    shape = wl.TINY if head_dim == 64 else TINY_D128
+    S = prefix + 8
+    pair = Pair(shape, max_seq=S, prefill_len=prefix, attn_chunks=chunks, flags=KV)
+    assert (pair.ctx.info().attn_chunks, pair.ctx.info().attn_heads) == (chunks, 2)
+    toks = wl.make_prompt(shape.vocab, 2, seed=17)
+    for i, t in enumerate(toks):
+        pos = prefix + i
+        g_tok, g_log = pair.gpu_step(int(t), pos)
+        ref = pair.ref_step(int(t), pos, intermediates=True)
+        _check_step(pair, pos, g_tok, g_log, ref)
+        got = pair.ctx.read_buffer(pair.mk.MK_BUF_ATTN, ref["attn"].size).astype(np.float64)
+        assert rel_l2(got, ref["attn"]) <= 5e-3
+    _check_hidden(pair, ref)
+
+
+# Group sizes and head dims of the KV-head items: G = 4 and 8 at head_dim
+# 64 (4 and 8 heads per item), G = 4 at 128 (4 heads), and G = 8 at 128,
+# split into two items of 4 heads per KV head (only the first appends the
+# new key).  A prefix of 2600 positions (3 merged chunks), then decode.
+G4_D64 = wl.ModelShape("g4-d64", 2, 256, 8, 2, 64, 768, 4096, True, 1e4)
+G8_D64 = wl.ModelShape("g8-d64", 2, 512, 8, 1, 64, 768, 4096, False, 1e4)
+G4_D128 = wl.ModelShape("g4-d128", 2, 512, 4, 1, 128, 768, 4096, True, 1e4)
+G8_D128 = wl.ModelShape("g8-d128", 2, 1024, 8, 1, 128, 768, 4096, True, 1e4)
+
+
+@pytest.mark.parametrize("shape,heads", [(G4_D64, 4), (G8_D64, 8), (G4_D128, 4), (G8_D128, 4)],
+                         ids=["g4-d64", "g8-d64", "g4-d128", "g8-d128"])
+@pytest.mark.parametrize("flags", [KV, KV | 4])
+def test_kv_head_items_group_sizes(shape, heads, flags):
+    S = 2624
+    pair = Pair(shape, max_seq=S, prefill_len=2600, attn_chunks=3, flags=flags)
+    assert pair.ctx.info().attn_heads == heads
+    toks = wl.make_prompt(shape.vocab, 3, seed=19)
+    for i, t in enumerate(toks):
+        pos = 2600 + i
+        g_tok, g_log = pair.gpu_step(int(t), pos)
+        ref = pair.ref_step(int(t), pos, intermediates=True)
+        _check_step(pair, pos, g_tok, g_log, ref)
+        got = pair.ctx.read_buffer(pair.mk.MK_BUF_ATTN, ref["attn"].size).astype(np.float64)
+        assert rel_l2(got, ref["attn"]) <= 5e-3
+    _check_hidden(pair, ref)
+    # short contexts (one chunk, positions 0..): the same items, no merge
+    short = Pair(shape, max_seq=48, flags=flags)
+    for step, pos, g_tok, g_log, ref in short.teacher_forced(wl.make_prompt(shape.vocab, 20, seed=3), 20):
+        _check_step(short, step, g_tok, g_log, ref)
+    _check_events(short, 40)
+
+
 @pytest.mark.parametrize("chunks", [1, 3, 64])
 def test_short_contexts_with_more_chunks_than_positions(chunks):
     # contexts of at most 40 positions use one active chunk whatever the
@@ -270,10 +326,14 @@ def test_llama1b_shape_at_the_end_of_the_benchmark_range():
 
 
 @pytest.mark.slow
-def test_llama1b_long_context_prefilled():
+@pytest.mark.parametrize("flags,heads,chunks", [(0, 4, 17), (64, 1, 4)], ids=["kv-items", "q-items"])
+def test_llama1b_long_context_prefilled(flags, heads, chunks):
+    # the default at 16k: one item per (KV head, chunk) for its 4 q heads,
+    # 17 chunks; MK_FLAG_ATTN_Q_ITEMS: one per (q head, chunk), 4 chunks
     shape = wl.LLAMA_1B
     S = 16640
-    pair = Pair(shape, max_seq=S, prefill_len=16384)
+    pair = Pair(shape, max_seq=S, prefill_len=16384, flags=flags)
+    assert (pair.ctx.info().attn_heads, pair.ctx.info().attn_chunks) == (heads, chunks)
     prompt = wl.make_prompt(shape.vocab, 1, seed=5)
     for step, pos, g_tok, g_log, ref in pair.teacher_forced(prompt, 1, start_pos=16384):
         _check_step(pair, step, g_tok, g_log, ref)

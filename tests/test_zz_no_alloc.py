@@ -63,7 +63,8 @@ def _both(mk, ctx, cfg, packed, k_st, v_st, io, tok, pos):
     return int(io["nxt_b"].item()), io["log_b"][0].double().cpu().numpy()
 
 
-def test_static_step_matches_context_step_twice():
+@pytest.mark.parametrize("flags", [0, 32], ids=["q-items", "kv-items"])
+def test_static_step_matches_context_step_twice(flags):
     from persistent_decode_megakernel_02_b200 import mk
     shape = wl.TINY
     S = 48
@@ -71,8 +72,9 @@ def test_static_step_matches_context_step_twice():
     packed = _pack(w)
     k_ctx, v_ctx = wl.make_kv(shape, 1, S, device="cuda")
     k_st, v_st = wl.make_kv(shape, 1, S, device="cuda")
-    ctx = mk.Context(w, k_ctx, v_ctx, S, 1)
-    cfg = mk.make_config(shape, S, 1)
+    ctx = mk.Context(w, k_ctx, v_ctx, S, 1, flags=flags)
+    cfg = mk.make_config(shape, S, 1, flags=flags)
+    assert ctx.info().attn_heads == (2 if flags else 1)
     io = _io(shape.vocab)
     for p_, t_ in ((0, 17), (1, 4093)):
         _both(mk, ctx, cfg, packed, k_st, v_st, io, t_, p_)
@@ -89,14 +91,18 @@ def test_static_step_alternating_shapes_and_weights():
     from persistent_decode_megakernel_02_b200 import mk
     untied = wl.ModelShape("tiny-untied", 2, 256, 4, 2, 64, 768, 4096, False, 1e4)
     models = []
-    for shape, S, seed in ((wl.TINY, 48, 1), (untied, 40, 2), (wl.TINY, 48, 3)):
+    # model 3: model 0's sizes with the attention items of one KV head's q
+    # heads together (MK_FLAG_ATTN_KV_ITEMS): the same config sizes, another
+    # task graph and scratch layout
+    for shape, S, seed, flags in ((wl.TINY, 48, 1, 0), (untied, 40, 2, 0), (wl.TINY, 48, 3, 0),
+                                  (wl.TINY, 48, 4, 32)):
         w = wl.make_weights(shape, seed=seed, device="cuda")
         kc, vc = wl.make_kv(shape, 1, S, device="cuda")
         ks, vs = wl.make_kv(shape, 1, S, device="cuda")
-        models.append(dict(shape=shape, packed=_pack(w), ctx=mk.Context(w, kc, vc, S, 1),
-                           cfg=mk.make_config(shape, S, 1), k=ks, v=vs, pos=0,
+        models.append(dict(shape=shape, packed=_pack(w), ctx=mk.Context(w, kc, vc, S, 1, flags=flags),
+                           cfg=mk.make_config(shape, S, 1, flags=flags), k=ks, v=vs, pos=0,
                            io=_io(shape.vocab)))
-    for i, m in enumerate([0, 1, 0, 2, 1, 2, 0]):
+    for i, m in enumerate([0, 1, 0, 3, 2, 1, 3, 2, 0, 3]):
         M = models[m]
         _both(mk, M["ctx"], M["cfg"], M["packed"], M["k"], M["v"], M["io"], 100 + 7 * i, M["pos"])
         M["pos"] += 1
