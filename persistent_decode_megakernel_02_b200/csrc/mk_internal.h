@@ -187,6 +187,17 @@ MK_HD inline int rows_per_page(int K) {
     return p;
 }
 
+// KV-head attention items score positions with the queries in registers:
+// a warp's lanes are (position p, dim group g) pairs, NG = HA * d / 64
+// groups of NS = 8 / HA 16-byte chunks of the K row each (every lane holds
+// its chunks' slices of all HA queries: 64 floats).  Lane (p, g) reads its
+// chunks starting at attn_kv_rot(p, g, ...) (mod NS) so that the 8 lanes of
+// every quarter-warp hit 8 different bank groups (chunk index mod 8; K rows
+// are 128 or 256 bytes apart).
+MK_HD inline int attn_kv_rot(int p, int g, int ng, int ns, int d) {
+    return ((p % (8 / ng)) * (d / 64) + (g * ns) / 8) % ns;
+}
+
 // Attention positions per page (K block and V block of `n` positions).
 MK_HD inline int attn_pos_per_page(int d) { return kPageBytes / (4 * d); }
 

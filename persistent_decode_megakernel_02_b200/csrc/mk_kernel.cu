@@ -949,19 +949,17 @@ __device__ __forceinline__ void dot_tmem2(uint32_t ta, bool two, const float (&x
                                           float &acc_c) {
     static_assert(NVL == 8, "a TMEM page row is 2048 columns: 8 vectors per lane");
     float2 a = make_float2(0.f, 0.f), c = make_float2(0.f, 0.f);
+    // the second row's columns are read even when the page has one row (a
+    // trailing 8-row page): its result is then dropped.  All 64 columns of
+    // both rows, then one wait (it covers every load before it)
+    uint32_t ra[32], rc[32];
+    tmem_ld32(ta, ra);
+    tmem_ld32(ta + 64, rc);
+    tmem_ld_wait();
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        // the second row's columns are read even when the page has one
-        // row (a trailing 8-row page): its result is then dropped
-        uint32_t ra[8], rc[8];
-        tmem_ld8(ta + 8 * h, ra);
-        tmem_ld8(ta + 64 + 8 * h, rc);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            a = dot8x2(make_uint4(ra[4 * j], ra[4 * j + 1], ra[4 * j + 2], ra[4 * j + 3]), xr[2 * h + j], a);
-            c = dot8x2(make_uint4(rc[4 * j], rc[4 * j + 1], rc[4 * j + 2], rc[4 * j + 3]), xr[2 * h + j], c);
-        }
+    for (int j = 0; j < 8; ++j) {
+        a = dot8x2(make_uint4(ra[4 * j], ra[4 * j + 1], ra[4 * j + 2], ra[4 * j + 3]), xr[j], a);
+        c = dot8x2(make_uint4(rc[4 * j], rc[4 * j + 1], rc[4 * j + 2], rc[4 * j + 3]), xr[j], c);
     }
     acc_a = a.x + a.y;
     acc_c = two ? c.x + c.y : 0.f;
@@ -1744,17 +1742,43 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     return true;
 }
 
+// Reduce-scatter of CNT values over the lanes whose index differs in bits
+// OFF, OFF / 2, ..., 1 (the lanes of one position): at offset off the lane
+// keeps the upper half of its values if its g has that bit, adding the
+// partner's copy; once one value is left the remaining levels add it up.
+// Lane g ends with the full sum of value g / (2 OFF / CNT).
+template <int CNT, int OFF, int N>
+__device__ __forceinline__ void reduce_scatter(float (&v)[N], int g) {
+    if constexpr (OFF >= 1) {
+        if constexpr (CNT > 1) {
+            const bool up = (g & OFF) != 0;
+#pragma unroll
+            for (int i = 0; i < CNT / 2; ++i) {
+                const float send = up ? v[i] : v[i + CNT / 2];
+                const float keep = up ? v[i + CNT / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+            }
+            reduce_scatter<CNT / 2, OFF / 2>(v, g);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
+            reduce_scatter<1, OFF / 2>(v, g);
+        }
+    }
+}
+
 // Attention item of HA q heads sharing one KV head (MK_FLAG_ATTN_KV_ITEMS,
 // the default for long caches): the same chunk, pages and merge as
 // attn_task, but every K row a lane reads is scored against all HA queries
 // and every V row a lane reads feeds all HA outputs, so the item reads its
-// KV head's positions once for the group.  The block loop: lane j scores
-// position j for each head (rotated 16-byte chunk order against the padded
-// queries in shared memory), the warp takes the per-head maximum in one
-// instruction, the softmax weights go to a per-warp slot of shared memory,
-// and P·V broadcasts them from there (one vector load per position for all
-// heads) with lanes over head dims.  Softmax sums are kept per lane and
-// added up once after the pages.
+// KV head's positions once for the group.  The block loop keeps the
+// queries in registers: a lane is a (position, dim group) pair and holds its
+// group's slice of all HA queries (64 floats), so scoring reads only K rows
+// from shared memory (in a rotated chunk order free of bank conflicts,
+// attn_kv_rot) and the dim groups of a position add up with shuffles.  The
+// warp takes the per-head maximum in one instruction, the softmax weights go
+// to a per-warp slot of shared memory, and P·V broadcasts them from there
+// (one vector load per position for all heads) with lanes over head dims.
+// Softmax sums are kept per lane and added up once after the pages.
 template <int D, int HA>   // head_dim 64 or 128; q heads per item, HA * D <= kAttnHeadDims
 __device__ bool attn_kv_task(const Params &p, const Task &t, unsigned char *pages, SmemCtl *ctl,
                              WState &w) {
@@ -1865,11 +1889,36 @@ __device__ bool attn_kv_task(const Params &p, const Task &t, unsigned char *page
     phase_end(w, tp, WS_PRO);
     stamp_input(p, w);
 
-    float m[HA], l[HA], o[HA][DPL];   // l: this lane's share of the softmax sum
+    // ---- the block loop, queries in registers: lane (pp, g) scores
+    // position pp of each pass against its NS chunks of every head (the
+    // item's HA x 64-dim slice); the NG lanes of a position add up
+    constexpr int NG = HA * D / 64;            // lanes per position (dim groups)
+    constexpr int NS = 8 / HA;                 // 16-byte chunks per lane
+    constexpr int PPI = 32 / NG;               // positions per pass
+    constexpr int IT = NG;                     // passes per 32-position block
+    static_assert(NG * NS == NCH && NG <= 8, "dim groups");
+    constexpr int LPH = NG / HA;               // lanes per (position, head) after the reduce-scatter
+    const int g = lane % NG, pp = lane / NG, hg = g / LPH;
+    const int rot = attn_kv_rot(pp, g, NG, NS, D);
+    float2 qr[NS][HA][4];
+#pragma unroll
+    for (int k = 0; k < NS; ++k) {
+        const int cc = g * NS + (k + rot) % NS;
+#pragma unroll
+        for (int hh = 0; hh < HA; ++hh) {
+            const float4 q0 = *reinterpret_cast<const float4 *>(qs + hh * QST + 12 * cc);
+            const float4 q1 = *reinterpret_cast<const float4 *>(qs + hh * QST + 12 * cc + 4);
+            qr[k][hh][0] = make_float2(q0.x, q0.y);
+            qr[k][hh][1] = make_float2(q0.z, q0.w);
+            qr[k][hh][2] = make_float2(q1.x, q1.y);
+            qr[k][hh][3] = make_float2(q1.z, q1.w);
+        }
+    }
+    float m[HA], o[HA][DPL];
+    float lw = 0.f;   // lanes g % LPH == 0: this lane's share of head hg's softmax sum
 #pragma unroll
     for (int hh = 0; hh < HA; ++hh) {
         m[hh] = -INFINITY;
-        l[hh] = 0.f;
 #pragma unroll
         for (int i = 0; i < DPL; ++i) o[hh][i] = 0.f;
     }
@@ -1881,52 +1930,68 @@ __device__ bool attn_kv_task(const Params &p, const Task &t, unsigned char *page
         const uint16_t *Vp = Kp + (size_t)npp * D;
         const int n = min(npp, a.npre - pg * npp);
         for (int j0 = warp * 32; j0 < n; j0 += kWorkerWarps * 32) {
-            const int j = j0 + lane;
-            float sc[HA];
-            if (j < n) {
-                const uint4 *krow = reinterpret_cast<const uint4 *>(Kp + (size_t)j * D);
-                float2 a0[HA], a1[HA];
+            // per pass, the NG lanes of a position reduce-scatter their
+            // partial dots: lane g ends with head g / LPH's full score
+            float xs[IT];
 #pragma unroll
-                for (int hh = 0; hh < HA; ++hh) { a0[hh] = make_float2(0.f, 0.f); a1[hh] = make_float2(0.f, 0.f); }
+            for (int it = 0; it < IT; ++it) {
+                const int j = j0 + it * PPI + pp;
+                float2 acc[HA];
 #pragma unroll
-                for (int c = 0; c < NCH; ++c) {
-                    const int cc = (c + lane) & (NCH - 1);
-                    const uint4 kw = krow[cc];
-                    const float2 k01 = make_float2(bf_lo(kw.x), bf_hi(kw.x));
-                    const float2 k23 = make_float2(bf_lo(kw.y), bf_hi(kw.y));
-                    const float2 k45 = make_float2(bf_lo(kw.z), bf_hi(kw.z));
-                    const float2 k67 = make_float2(bf_lo(kw.w), bf_hi(kw.w));
+                for (int hh = 0; hh < HA; ++hh) acc[hh] = make_float2(0.f, 0.f);
+                if (j < n) {
+                    const uint4 *krow = reinterpret_cast<const uint4 *>(Kp + (size_t)j * D);
 #pragma unroll
-                    for (int hh = 0; hh < HA; ++hh) {
-                        const float4 q0 = *reinterpret_cast<const float4 *>(qs + hh * QST + 12 * cc);
-                        const float4 q1 = *reinterpret_cast<const float4 *>(qs + hh * QST + 12 * cc + 4);
-                        a0[hh] = ffma2(k01, make_float2(q0.x, q0.y), a0[hh]);
-                        a1[hh] = ffma2(k23, make_float2(q0.z, q0.w), a1[hh]);
-                        a0[hh] = ffma2(k45, make_float2(q1.x, q1.y), a0[hh]);
-                        a1[hh] = ffma2(k67, make_float2(q1.z, q1.w), a1[hh]);
+                    for (int k = 0; k < NS; ++k) {
+                        const uint4 kw = krow[g * NS + (k + rot) % NS];
+                        const float2 k01 = make_float2(bf_lo(kw.x), bf_hi(kw.x));
+                        const float2 k23 = make_float2(bf_lo(kw.y), bf_hi(kw.y));
+                        const float2 k45 = make_float2(bf_lo(kw.z), bf_hi(kw.z));
+                        const float2 k67 = make_float2(bf_lo(kw.w), bf_hi(kw.w));
+#pragma unroll
+                        for (int hh = 0; hh < HA; ++hh) {
+                            acc[hh] = ffma2(k01, qr[k][hh][0], acc[hh]);
+                            acc[hh] = ffma2(k23, qr[k][hh][1], acc[hh]);
+                            acc[hh] = ffma2(k45, qr[k][hh][2], acc[hh]);
+                            acc[hh] = ffma2(k67, qr[k][hh][3], acc[hh]);
+                        }
                     }
                 }
+                float v[HA];
 #pragma unroll
-                for (int hh = 0; hh < HA; ++hh) sc[hh] = (a0[hh].x + a0[hh].y) + (a1[hh].x + a1[hh].y);
-            } else {
-#pragma unroll
-                for (int hh = 0; hh < HA; ++hh) sc[hh] = -INFINITY;
+                for (int hh = 0; hh < HA; ++hh) v[hh] = acc[hh].x + acc[hh].y;
+                reduce_scatter<HA, NG / 2>(v, g);
+                xs[it] = j < n ? v[0] : -INFINITY;
             }
-            float pe[HA], corr[HA];
+            // head hg's block maximum: over the lane's passes, then over the
+            // lanes holding the same head (other positions, twin groups)
+            float mx = xs[0];
+#pragma unroll
+            for (int it = 1; it < IT; ++it) mx = fmaxf(mx, xs[it]);
+#pragma unroll
+            for (int off = 1; off < LPH; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+#pragma unroll
+            for (int off = NG; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            float corr[HA];
+            float mg = 0.f, cg = 0.f;   // head hg's new maximum and rescale
 #pragma unroll
             for (int hh = 0; hh < HA; ++hh) {
-                const float mn = fmaxf(m[hh], warp_max(sc[hh]));   // finite: lane 0's position is valid
+                const float mn = fmaxf(m[hh], __shfl_sync(0xffffffffu, mx, hh * LPH));   // finite: position j0 is valid
                 corr[hh] = expf(m[hh] - mn);
-                pe[hh] = j < n ? expf(sc[hh] - mn) : 0.f;
-                l[hh] = fmaf(l[hh], corr[hh], pe[hh]);
                 m[hh] = mn;
+                if (hg == hh) { mg = mn; cg = corr[hh]; }
             }
-            if constexpr (HA % 4 == 0) {
+            // one lane per (position, head): the weights go to the warp's
+            // slot for P·V, the sum stays in the lane
+            if (g % LPH == 0) {
+                float ls = 0.f;
 #pragma unroll
-                for (int hh = 0; hh < HA; hh += 4)
-                    *reinterpret_cast<float4 *>(pb + lane * HA + hh) = make_float4(pe[hh], pe[hh + 1], pe[hh + 2], pe[hh + 3]);
-            } else {
-                *reinterpret_cast<float2 *>(pb + lane * HA) = make_float2(pe[0], pe[1]);
+                for (int it = 0; it < IT; ++it) {
+                    const float pe = expf(xs[it] - mg);   // 0 for positions past n (x = -inf)
+                    ls += pe;
+                    pb[(it * PPI + pp) * HA + hg] = pe;
+                }
+                lw = fmaf(lw, cg, ls);
             }
             __syncwarp();
             const uint16_t *vb = Vp + (size_t)j0 * D + lane * DPL;
@@ -1976,8 +2041,12 @@ __device__ bool attn_kv_task(const Params &p, const Task &t, unsigned char *page
         release_page(ctl, w, slot);
         phase_end(w, tp, WS_DOT);
     }
+    // head h's softmax sum: the lanes of head h add up (lane h * LPH holds it)
 #pragma unroll
-    for (int hh = 0; hh < HA; ++hh) l[hh] = warp_sum(l[hh]);
+    for (int off = NG; off < 32; off <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+    float l[HA];
+#pragma unroll
+    for (int hh = 0; hh < HA; ++hh) l[hh] = __shfl_sync(0xffffffffu, lw, hh * LPH);
     tp = phase_begin(w);
     if (new_warp) {
 #pragma unroll

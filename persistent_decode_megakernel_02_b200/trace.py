@@ -86,6 +86,59 @@ def summarize(overhead: np.ndarray, kind: np.ndarray) -> dict:
     return out
 
 
+def critical_path(trace: np.ndarray, tasks: np.ndarray, layers=None) -> dict:
+    """How each op extends the step: for the ops in graph order (layer by
+    layer, then the LM head), `inc` = last t_done of the op - last t_done of
+    the op before it, split into `to_ready` (until the op's last task was
+    ready: its inputs fresh) and the rest; averaged per op kind over
+    `layers` (default: all but the first and last two).  Values in us."""
+    kind, layer = tasks[:, 0], tasks[:, 1]
+    done = trace["t_done"].astype(np.float64)
+    ready = trace["t_ready"].astype(np.float64)
+    L = int(layer[kind != 5].max()) + 1 if np.any(kind != 5) else 0
+    if layers is None:
+        layers = range(1, max(L - 2, 1))
+    rows = {}
+    prev = None
+    for l in range(L + 1):
+        for k in range(6):
+            sel = (kind == k) & (layer == l)
+            if not np.any(sel):
+                continue
+            last = done[sel].max()
+            if prev is not None and (l in layers or k == 5):
+                rows.setdefault(OP_NAMES[k], []).append(((last - prev), (ready[sel].max() - prev)))
+            prev = last
+    out = {}
+    for name, v in rows.items():
+        a = np.asarray(v) / 1e3
+        out[name] = {"inc_us": float(a[:, 0].mean()), "to_ready_us": float(a[:, 1].mean()), "n": len(v)}
+    return out
+
+
+def transitions(trace: np.ndarray, tasks: np.ndarray) -> dict:
+    """Per-SM task transitions: for consecutive tasks a, b on one SM (in
+    start order), medians (us) per kind of b of `tail` = t_end(a) - t_done(a)
+    (end barrier and completion post), `to_ready` = t_ready(b) - t_end(a)
+    (dispatch, prologue and the input round trip, waits included) and
+    `compute` = t_done(b) - t_input(b)."""
+    sm = tasks[:, 6]
+    f = {k: trace[k].astype(np.float64) for k in ("t_ready", "t_start", "t_input", "t_done", "t_end")}
+    rows = {}
+    for s in np.unique(sm):
+        idx = np.where(sm == s)[0]
+        idx = idx[np.argsort(f["t_start"][idx], kind="stable")]
+        for a, b in zip(idx[:-1], idx[1:]):
+            rows.setdefault(OP_NAMES[tasks[b, 0]], []).append(
+                (f["t_end"][a] - f["t_done"][a], f["t_ready"][b] - f["t_end"][a], f["t_done"][b] - f["t_input"][b]))
+    out = {}
+    for name, v in rows.items():
+        med = np.median(np.asarray(v), axis=0) / 1e3
+        out[name] = {"tail_us": float(med[0]), "to_ready_us": float(med[1]), "compute_us": float(med[2]),
+                     "n": len(v)}
+    return out
+
+
 def _measure(workload: str, flags: int, steps: int, warmup: int, traced: bool):
     """Run `warmup` + `steps` decode steps of `workload` (batch 1, synthetic
     weights) with mk_config.flags = flags; return (ms per step over the timed
@@ -113,7 +166,11 @@ def _measure(workload: str, flags: int, steps: int, warmup: int, traced: bool):
             ctx.decode_step(toks[i:i + 1], pos[i:i + 1], nxt)
             if ctx.sync() != 0:
                 raise RuntimeError("traced step failed")
-            per_step.append(task_overheads(ctx.trace(), g["tasks"], g["queue"], g["qoff"]))
+            tr = ctx.trace()
+            d = task_overheads(tr, g["tasks"], g["queue"], g["qoff"])
+            d["critical_path"] = critical_path(tr, g["tasks"])
+            d["transitions"] = transitions(tr, g["tasks"])
+            per_step.append(d)
         ms = None
     else:
         e0 = torch.cuda.Event(enable_timing=True)
@@ -134,7 +191,8 @@ def _measure(workload: str, flags: int, steps: int, warmup: int, traced: bool):
 def main(argv=None):
     """python -m persistent_decode_megakernel_02_b200.trace [--workload llama1b]
     [--steps N] [--warmup W]: per-task scheduling overhead in both wait modes
-    (one JSON line per mode) and the cost of trace mode (device time per
+    (one JSON line per mode), how each op extends the step (critical_path),
+    the per-SM task transitions, and the cost of trace mode (device time per
     step with and without MK_FLAG_TRACE)."""
     import argparse
     import json
@@ -150,9 +208,14 @@ def main(argv=None):
         _, steps = _measure(a.workload, mode | mk.MK_FLAG_TRACE, a.steps, a.warmup, True)
         ov = np.concatenate([s["overhead"] for s in steps])
         kind = np.concatenate([s["kind"] for s in steps])
+        def mean_of(key):
+            names = steps[0][key].keys()
+            return {n: {f: round(float(np.mean([s[key][n][f] for s in steps])), 3)
+                        for f in steps[0][key][n] if f != "n"} for n in names}
         out = {"workload": a.workload, "wait_mode": name, "traced_steps": a.steps,
                "ms_per_step": round(base_ms, 5), "ms_per_step_traced": round(tr_ms, 5),
-               "overhead": summarize(ov, kind)}
+               "overhead": summarize(ov, kind), "critical_path": mean_of("critical_path"),
+               "transitions": mean_of("transitions")}
         print(json.dumps(out), flush=True)
 
 

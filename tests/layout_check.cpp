@@ -3,7 +3,9 @@
 // shared-memory descriptor (leading byte offset 2048, stride byte offset
 // 128): TMEM lane r, columns 8c..8c+3 receive the 16 bytes at
 // 4096c + (r / 8) * 128 + (r % 8) * 16 of the page, columns 8c+4..8c+7 the
-// 16 bytes 2048 further.  Prints "ok" or the first violation.
+// 16 bytes 2048 further.  Also the chunk rotation of the KV-head attention
+// loop (attn_kv_rot): conflict-free shared-memory reads.  Prints "ok" or the
+// first violation.
 #include <cstdio>
 #include "../persistent_decode_megakernel_02_b200/csrc/mk_internal.h"
 
@@ -44,6 +46,31 @@ int main() {
                 }
             }
         }
+    // 4. the KV-head attention loop's chunk rotation: for every head_dim,
+    //    heads per item, pass s and quarter-warp, the 8 lanes read 8
+    //    distinct bank groups (chunk index mod 8), and each lane's NS
+    //    passes read its NS chunks once each
+    const int cases[5][2] = {{64, 2}, {64, 4}, {64, 8}, {128, 2}, {128, 4}};
+    for (const auto &cs : cases) {
+        const int d = cs[0], ha = cs[1], ng = ha * d / 64, ns = 8 / ha;
+        if (ng * ns != d / 8) { printf("groups x chunks != row chunks (d %d, ha %d)\n", d, ha); return 1; }
+        for (int lane = 0; lane < 32; ++lane) {
+            const int g = lane % ng, p = lane / ng;
+            int hit = 0;
+            for (int s = 0; s < ns; ++s) hit |= 1 << ((s + attn_kv_rot(p, g, ng, ns, d)) % ns);
+            if (hit != (1 << ns) - 1) { printf("lane %d misses a chunk (d %d, ha %d)\n", lane, d, ha); return 1; }
+        }
+        for (int s = 0; s < ns; ++s)
+            for (int q = 0; q < 4; ++q) {
+                int banks = 0;
+                for (int lane = 8 * q; lane < 8 * q + 8; ++lane) {
+                    const int g = lane % ng, p = lane / ng;
+                    const int c = g * ns + (s + attn_kv_rot(p, g, ng, ns, d)) % ns;
+                    banks |= 1 << (c % 8);
+                }
+                if (banks != 0xff) { printf("bank conflict: d %d ha %d pass %d quarter %d\n", d, ha, s, q); return 1; }
+            }
+    }
     printf("ok\n");
     return 0;
 }

@@ -65,3 +65,25 @@ def test_a_task_that_starts_before_its_event_fires_shows_a_negative_overhead():
     t["t_end"][0] = 250      # event 0 now fires at 250 (task 0)
     d = tr.task_overheads(t, tasks, queue, qoff)
     assert d["overhead"][3] == 240 - 250
+
+
+def test_critical_path_increments_and_transitions_by_hand():
+    t, tasks, queue, qoff = _graph()
+    t["t_ready"] = [100, 110, 290, 255, 690]
+    t["t_input"] = [120, 130, 310, 270, 720]
+    t["t_done"] = [190, 240, 390, 580, 790]
+    # layers=[0]: every op of layer 0 after the first counts
+    cp = tr.critical_path(t, tasks, layers=[0])
+    # QKV last done 240; attention last done 580 -> 340, last ready 290 -> 50;
+    # O-proj done 790 -> 210 after 580, ready 690 -> 110
+    assert cp["attn"] == {"inc_us": 0.34, "to_ready_us": 0.05, "n": 1}
+    assert cp["oproj"] == {"inc_us": 0.21, "to_ready_us": 0.11, "n": 1}
+    assert "qkv" not in cp
+    tv = tr.transitions(t, tasks)
+    # SM 0: 0 -> 2: tail 200-190 = 10, to_ready 290-200 = 90, compute 390-310 = 80
+    #        2 -> 4: tail 400-390 = 10, to_ready 690-400 = 290, compute 790-720 = 70
+    # SM 1: 1 -> 3: tail 250-240 = 10, to_ready 255-250 = 5, compute 580-270 = 310
+    assert tv["oproj"]["to_ready_us"] == 0.29 and tv["oproj"]["compute_us"] == 0.07
+    a = tv["attn"]     # medians of (90, 5) and (80, 310)
+    assert a["n"] == 2 and abs(a["to_ready_us"] - 0.0475) < 1e-12 and abs(a["compute_us"] - 0.195) < 1e-12
+    assert a["tail_us"] == 0.01
