@@ -34,21 +34,24 @@ bool plan_attention(Shape &s, int num_sms, int flags, int attn_chunks) {
     int per_q = num_sms / (s.Bmax * s.nq);                             // chunks per q head the SMs give
     if (per_q < 1) per_q = 1;
     s.HA = (kv || (!qi && cap > per_q)) ? hg : 1;
+    // the merge's shared staging: q-head items hold a head's chunk partials
+    // (d + 2 floats each); KV-head items those of all HA heads plus one
+    // weight per (head, chunk) and one sum per head
+    auto fits = [&](long long nc, int ha) {
+        return ha == 1 ? nc * (s.d + 2) <= kStageFloats : nc * ha * (s.d + 3) + ha <= kStageFloats;
+    };
     // chosen by default, KV-head items give way to q-head items where a
     // given chunk count's partials would not fit the merge's staging area
-    if (!kv && s.HA > 1 && attn_chunks > 0 && (long long)attn_chunks * s.HA * (s.d + 2) > kStageFloats)
-        s.HA = 1;
+    if (!kv && s.HA > 1 && attn_chunks > 0 && !fits(attn_chunks, s.HA)) s.HA = 1;
     int nc = attn_chunks;
     if (nc <= 0) {
         nc = num_sms / (s.Bmax * (s.nq / s.HA));
         if (nc < 1) nc = 1;
         if (nc > cap) nc = cap;
-        const int fit = kStageFloats / (s.HA * (s.d + 2));
-        if (nc > fit) nc = fit;
+        while (nc > 1 && !fits(nc, s.HA)) --nc;
     }
     s.NC = nc;
-    // every head's chunk partials of an item must fit the merge's staging area
-    return nc <= 4096 && (long long)nc * s.HA * (s.d + 2) <= kStageFloats;
+    return nc <= 4096 && fits(nc, s.HA);
 }
 
 // Tiles per scheduling unit of a GEMV op: tasks of ops whose pages pass

@@ -1742,30 +1742,6 @@ __device__ bool attn_task(const Params &p, const Task &t, unsigned char *pages, 
     return true;
 }
 
-// Reduce-scatter of CNT values over the lanes whose index differs in bits
-// OFF, OFF / 2, ..., 1 (the lanes of one position): at offset off the lane
-// keeps the upper half of its values if its g has that bit, adding the
-// partner's copy; once one value is left the remaining levels add it up.
-// Lane g ends with the full sum of value g / (2 OFF / CNT).
-template <int CNT, int OFF, int N>
-__device__ __forceinline__ void reduce_scatter(float (&v)[N], int g) {
-    if constexpr (OFF >= 1) {
-        if constexpr (CNT > 1) {
-            const bool up = (g & OFF) != 0;
-#pragma unroll
-            for (int i = 0; i < CNT / 2; ++i) {
-                const float send = up ? v[i] : v[i + CNT / 2];
-                const float keep = up ? v[i + CNT / 2] : v[i];
-                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
-            }
-            reduce_scatter<CNT / 2, OFF / 2>(v, g);
-        } else {
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
-            reduce_scatter<1, OFF / 2>(v, g);
-        }
-    }
-}
-
 // Attention item of HA q heads sharing one KV head (MK_FLAG_ATTN_KV_ITEMS,
 // the default for long caches): the same chunk, pages and merge as
 // attn_task, but every K row a lane reads is scored against all HA queries
@@ -2110,27 +2086,55 @@ __device__ bool attn_kv_task(const Params &p, const Task &t, unsigned char *page
     }
     stamp_done(p, w);
     if (a.active && a.nc > 1 && a.c == 0) {
-        // chunk 0's item merges the partials of its q heads: polls them into
-        // shared memory ([head][chunk][D + 2]; tagged, so it waits for
-        // exactly the chunks it reads), then combines them there
-        const int nc = a.nc;
+        // chunk 0's item merges the chunks' partials of its q heads (every
+        // other chunk's item sits ahead of it on its SM's queue, so the wait
+        // always ends): first the (m, l) words of every (head, chunk) until
+        // fresh (a few words per thread), then all partials in one pass into
+        // shared memory [head][chunk][D + 2] (the tags still checked)
         if (!worker_sync(p, ctl, w)) return false;   // the combine above is done with the stage
-        if (!stage_partials(p, ctl, w, part, HA, nc * (D + 2), s.NC * (D + 2))) return false;
-        if (!worker_sync(p, ctl, w)) return false;
-        for (int i = tid; i < HA * D; i += kWorkerThreads) {
-            const int hh = i / D, e = i % D;
-            const float *sg = ctl->stage + (size_t)hh * nc * (D + 2);
-            float M = -INFINITY;
-            for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (D + 2) + D]);
-            float num = 0.f, den = 0.f;
-            for (int c = 0; c < nc; ++c) {
-                const float mc = sg[c * (D + 2) + D];
-                if (mc == -INFINITY) continue;
-                const float f = expf(mc - M);
-                num = fmaf(f, sg[c * (D + 2) + e], num);
-                den = fmaf(f, sg[c * (D + 2) + D + 1], den);
+        for (int i = tid; i < HA * a.nc; i += kWorkerThreads) {
+            const uint64_t *src = part + ((size_t)(i / a.nc) * s.NC + i % a.nc) * (D + 2) + D;
+            ulonglong2 v = ld_tag2(src);
+            Spin sp;
+            while (!tag_ok(v.x, w.ep) || !tag_ok(v.y, w.ep)) {
+                if (!spin_ok(sp, p, ctl, W_TAG, (uint32_t)w.task_id, 6u)) return false;
+                v = ld_tag2(src);
             }
-            st_tag_rep(attn + i, p.tl.rep_qd, num / den, w.ep_out);
+        }
+        if (!worker_sync(p, ctl, w)) return false;
+        {
+            // the chunk weights exp(m_c - M) once per (head, chunk), then the sums
+            const int nc = a.nc;
+            if (!stage_partials(p, ctl, w, part, HA, nc * (D + 2), s.NC * (D + 2))) return false;
+            if (!worker_sync(p, ctl, w)) return false;
+            float *wt = ctl->stage + (size_t)HA * nc * (D + 2);   // [HA][nc] weights, then [HA] sums
+            if (tid < HA) {
+                const float *sg = ctl->stage + (size_t)tid * nc * (D + 2);
+                float M = -INFINITY;
+                for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (D + 2) + D]);
+                float den = 0.f;
+                for (int c = 0; c < nc; ++c) {
+                    const float mc = sg[c * (D + 2) + D];
+                    const float f = mc == -INFINITY ? 0.f : expf(mc - M);
+                    wt[tid * nc + c] = f;
+                    den = fmaf(f, sg[c * (D + 2) + D + 1], den);
+                }
+                wt[HA * nc + tid] = 1.0f / den;
+            }
+            if (!worker_sync(p, ctl, w)) return false;
+            for (int i = tid; i < HA * D; i += kWorkerThreads) {
+                const int hh = i / D, e = i % D;
+                const float *sg = ctl->stage + (size_t)hh * nc * (D + 2) + e;
+                const float *f = wt + hh * nc;
+                float n0 = 0.f, n1 = 0.f;
+                int c = 0;
+                for (; c + 1 < nc; c += 2) {
+                    n0 = fmaf(f[c], sg[c * (D + 2)], n0);
+                    n1 = fmaf(f[c + 1], sg[(c + 1) * (D + 2)], n1);
+                }
+                if (c < nc) n0 = fmaf(f[c], sg[c * (D + 2)], n0);
+                st_tag_rep(attn + i, p.tl.rep_qd, (n0 + n1) * wt[HA * nc + hh], w.ep_out);
+            }
         }
     }
     if (!worker_sync(p, ctl, w)) return false;
@@ -2271,7 +2275,7 @@ __device__ void worker_role(const Params &p, unsigned char *pages, SmemCtl *ctl)
             if (!worker_sync(p, ctl, w)) return;
             if (t.kind == OP_LMHEAD) {
                 if (tid == 0) {
-                    __threadfence();
+                    // after the barrier: a release that covers every thread's partials
                     const uint32_t old = atom_add_acqrel_gpu(p.lm_cnt, 1u);
                     const uint32_t last = (old + 1u == (uint32_t)p.num_lm_tasks * w.ep) ? 1u : 0u;
                     ctl->last_flag = last;

@@ -211,6 +211,30 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Reduce-scatter of CNT values over the lanes whose index differs in bits
+// OFF, OFF / 2, ..., 1 (the lanes of one position): at offset off the lane
+// keeps the upper half of its values if its g has that bit, adding the
+// partner's copy; once one value is left the remaining levels add it up.
+// Lane g ends with the full sum of value g / (2 OFF / CNT).
+template <int CNT, int OFF, int N>
+__device__ __forceinline__ void reduce_scatter(float (&v)[N], int g) {
+    if constexpr (OFF >= 1) {
+        if constexpr (CNT > 1) {
+            const bool up = (g & OFF) != 0;
+#pragma unroll
+            for (int i = 0; i < CNT / 2; ++i) {
+                const float send = up ? v[i] : v[i + CNT / 2];
+                const float keep = up ? v[i + CNT / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+            }
+            reduce_scatter<CNT / 2, OFF / 2>(v, g);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
+            reduce_scatter<1, OFF / 2>(v, g);
+        }
+    }
+}
+
 // Maximum of v over the full warp in one instruction (sm_100a; NaN inputs
 // are ignored, as by fmaxf).
 __device__ __forceinline__ float warp_max(float v) {

@@ -706,7 +706,8 @@ __device__ bool gemv_task(const RParams &p, Ctl *c, CState &cs, const Task &t) {
                 asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(a + r), "f"(y[r]), "f"(y[r + 1]),
                              "f"(y[r + 2]), "f"(y[r + 3])
                              : "memory");
-            __threadfence();
+            // the barrier puts every thread's adds before thread m == 0's
+            // release; the finisher's acquire puts all of them before its reads
             if (!group_sync(&c->ebar, cs.eph, p, c, (uint32_t)cs.task_id)) return false;
             if (m == 0) {
                 // a tile receives exactly `slabs` pages per step, and two
@@ -718,7 +719,6 @@ __device__ bool gemv_task(const RParams &p, Ctl *c, CState &cs, const Task &t) {
             if (!group_sync(&c->ebar, cs.eph, p, c, (uint32_t)cs.task_id)) return false;
             finish = c->last_flag != 0u;
             if (finish) {
-                __threadfence();
 #pragma unroll
                 for (int r = 0; r < kRows; r += 4) {
                     const float4 v = __ldcg(reinterpret_cast<const float4 *>(a + r));
@@ -748,70 +748,96 @@ __device__ bool embed_task(const RParams &p, Ctl *c, CState &cs, const Task &t) 
     return resid_out(p, c, cs, tile, m, x, nrows, p.x0, B.xq, p.layers[0].g_attn, B.ssq);
 }
 
-// One block of up to 32 positions for every query head of the item, lane j
-// holding position j: scores, the running softmax (m, l) per head and the
-// P.V sums (lane L: head dims DPL*L .. DPL*L + DPL - 1).  K rows and V rows
-// come from shared memory (a landed page) or, with GLOBAL, for positions
-// written during this launch, from global memory through L2 (ld.global.cg:
-// other SMs wrote them).  The two are separate instantiations: a runtime
-// choice between a global-space load and a generic one of the same pointer
-// could be evaluated on both sides.
+// One block of up to 32 positions of an attention item (G query heads of
+// one KV head), queries in registers: lane (pp, g) of the warp is position
+// pp of each pass and dim group g (NG = G * D / 64 groups of NS = 8 / G
+// 16-byte chunks; its query slices `qr` were loaded once per item), reading
+// K chunks in the rotated order of attn_kv_rot (no bank conflicts when K
+// sits in the ring); the NG lanes of a position reduce-scatter their partial
+// dots so each ends with one head's score.  The softmax weights go to the
+// warp's slot (4 heads per position), P·V reads them back with lanes over
+// head dims.  `lw`: this lane's share of head hg's softmax sum (lanes with
+// g % (NG / G) == 0).  K and V rows come from a landed page of the ring or,
+// with GLOBAL, for positions written during this launch, from global memory
+// through L2 (ld.global.cg: other SMs wrote them in this launch, so no
+// stale L1 line may be used).
 template <int D, int G, bool GLOBAL>
 __device__ __forceinline__ void attn_block(Ctl *c, const uint16_t *K, const uint16_t *V, int n,
-                                           float (&mx)[G], float (&l)[G], float (&o)[G][D / 32]) {
-    constexpr int NCH = D / 8, DPL = D / 32;
+                                           const float2 (&qr)[8 / G][G][4], int g, int pp, int rot,
+                                           float (&mx)[G], float &lw, float (&o)[G][D / 32]) {
+    constexpr int NG = G * D / 64, NS = 8 / G, PPI = 32 / NG, IT = NG, LPH = NG / G, DPL = D / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float sc[G];
+    const int hg = g / LPH;
+    float xs[IT];
 #pragma unroll
-    for (int g = 0; g < G; ++g) sc[g] = -INFINITY;
-    if (lane < n) {
+    for (int it = 0; it < IT; ++it) {
+        const int j = it * PPI + pp;
         float2 acc[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
-        const uint4 *krow = reinterpret_cast<const uint4 *>(K + (size_t)lane * D);
-#pragma unroll 4
-        for (int ch = 0; ch < NCH; ++ch) {
-            const int cc = (ch + lane) & (NCH - 1);   // rotated: the lanes of a phase hit different banks
-            uint4 kw;
-            if constexpr (GLOBAL) kw = __ldcg(krow + cc);
-            else kw = krow[cc];
+        for (int h = 0; h < G; ++h) acc[h] = make_float2(0.f, 0.f);
+        if (j < n) {
+            const uint4 *krow = reinterpret_cast<const uint4 *>(K + (size_t)j * D);
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float4 q0 = *reinterpret_cast<const float4 *>(c->at.q + g * D + 8 * cc);
-                const float4 q1 = *reinterpret_cast<const float4 *>(c->at.q + g * D + 8 * cc + 4);
-                acc[g] = ffma2(make_float2(bf_lo(kw.x), bf_hi(kw.x)), make_float2(q0.x, q0.y), acc[g]);
-                acc[g] = ffma2(make_float2(bf_lo(kw.y), bf_hi(kw.y)), make_float2(q0.z, q0.w), acc[g]);
-                acc[g] = ffma2(make_float2(bf_lo(kw.z), bf_hi(kw.z)), make_float2(q1.x, q1.y), acc[g]);
-                acc[g] = ffma2(make_float2(bf_lo(kw.w), bf_hi(kw.w)), make_float2(q1.z, q1.w), acc[g]);
+            for (int k = 0; k < NS; ++k) {
+                const int cc = g * NS + (k + rot) % NS;
+                uint4 kw;
+                if constexpr (GLOBAL) kw = __ldcg(krow + cc);
+                else kw = krow[cc];
+                const float2 k01 = make_float2(bf_lo(kw.x), bf_hi(kw.x));
+                const float2 k23 = make_float2(bf_lo(kw.y), bf_hi(kw.y));
+                const float2 k45 = make_float2(bf_lo(kw.z), bf_hi(kw.z));
+                const float2 k67 = make_float2(bf_lo(kw.w), bf_hi(kw.w));
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    acc[h] = ffma2(k01, qr[k][h][0], acc[h]);
+                    acc[h] = ffma2(k23, qr[k][h][1], acc[h]);
+                    acc[h] = ffma2(k45, qr[k][h][2], acc[h]);
+                    acc[h] = ffma2(k67, qr[k][h][3], acc[h]);
+                }
             }
         }
+        float v[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) sc[g] = acc[g].x + acc[g].y;
+        for (int h = 0; h < G; ++h) v[h] = acc[h].x + acc[h].y;
+        reduce_scatter<G, NG / 2>(v, g);
+        xs[it] = j < n ? v[0] : -INFINITY;
     }
-    // l: this lane's share of the softmax sum (mx is warp-uniform; the
-    // shares are added up once, after the item's positions)
-    float pe[G], corr[G];
+    // head hg's block maximum: the lane's passes, then the lanes holding the
+    // same head (twin dim groups, other positions)
+    float m = xs[0];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const float mn = fmaxf(mx[g], warp_max(sc[g]));   // finite: position 0 of the block is valid
-        corr[g] = expf(mx[g] - mn);
-        pe[g] = lane < n ? expf(sc[g] - mn) : 0.f;
-        l[g] = fmaf(l[g], corr[g], pe[g]);
-        mx[g] = mn;
+    for (int it = 1; it < IT; ++it) m = fmaxf(m, xs[it]);
+#pragma unroll
+    for (int off = 1; off < LPH; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+#pragma unroll
+    for (int off = NG; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float corr[G];
+    float mg = 0.f, cg = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        const float mn = fmaxf(mx[h], __shfl_sync(0xffffffffu, m, h * LPH));   // finite: position 0 is valid
+        corr[h] = expf(mx[h] - mn);
+        mx[h] = mn;
+        if (hg == h) { mg = mn; cg = corr[h]; }
     }
-    // the weights of position `lane` for every head, read back below by all
-    // lanes at once (one broadcast load per position instead of G shuffles)
-    float4 *pw = c->at.pw[warp];
-    float pv[4] = {0.f, 0.f, 0.f, 0.f};
+    float *pwf = reinterpret_cast<float *>(c->at.pw[warp]);   // [32 positions][4 heads]
+    if (g % LPH == 0) {
+        float ls = 0.f;
 #pragma unroll
-    for (int g = 0; g < G; ++g) pv[g] = pe[g];
-    pw[lane] = make_float4(pv[0], pv[1], pv[2], pv[3]);
+        for (int it = 0; it < IT; ++it) {
+            const float pe = expf(xs[it] - mg);   // 0 past n (xs = -inf)
+            ls += pe;
+            pwf[(it * PPI + pp) * 4 + hg] = pe;
+        }
+        lw = fmaf(lw, cg, ls);
+    }
     __syncwarp();
+    const float4 *pw = c->at.pw[warp];
     float tv[G][DPL];
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+    for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) tv[g][i] = 0.f;
+        for (int i = 0; i < DPL; ++i) tv[h][i] = 0.f;
     auto pvk = [&](int k) {
         const uint16_t *vr = V + (size_t)k * D + lane * DPL;
         float v[DPL];
@@ -829,9 +855,9 @@ __device__ __forceinline__ void attn_block(Ctl *c, const uint16_t *K, const uint
         const float4 pk4 = pw[k];
         const float pk[4] = {pk4.x, pk4.y, pk4.z, pk4.w};
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
+        for (int h = 0; h < G; ++h) {
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) tv[g][i] = fmaf(pk[g], v[i], tv[g][i]);
+            for (int i = 0; i < DPL; ++i) tv[h][i] = fmaf(pk[h], v[i], tv[h][i]);
         }
     };
     if (n == 32) {
@@ -841,9 +867,9 @@ __device__ __forceinline__ void attn_block(Ctl *c, const uint16_t *K, const uint
         for (int k = 0; k < n; ++k) pvk(k);
     }
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+    for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) o[g][i] = fmaf(o[g][i], corr[g], tv[g][i]);
+        for (int i = 0; i < DPL; ++i) o[h][i] = fmaf(o[h][i], corr[h], tv[h][i]);
     __syncwarp();   // the next block's weights overwrite pw
 }
 
@@ -868,11 +894,29 @@ __device__ bool attn_task(const RParams &p, unsigned char *ring, Ctl *c, CState 
             c->at.q[i] = ldcg(B.q + (size_t)a.r * s.QD + (size_t)a.h * G * D + i);
     if (!group_sync(&c->cbar, cs.cph, p, c, (uint32_t)cs.task_id)) return false;
     if (p.trace && tid == 0) p.trace[t.sm].t_input = globaltimer();
-    float mx[G], l[G], o[G][DPL];
+    // the lane's query slices (see attn_block), loaded once
+    constexpr int NG = G * D / 64, NS = 8 / G, LPH = NG / G;
+    const int gq = lane % NG, pq = lane / NG;
+    const int rot = attn_kv_rot(pq, gq, NG, NS, D);
+    float2 qr[NS][G][4];
+#pragma unroll
+    for (int k = 0; k < NS; ++k) {
+        const int cc = gq * NS + (k + rot) % NS;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float4 q0 = *reinterpret_cast<const float4 *>(c->at.q + h * D + 8 * cc);
+            const float4 q1 = *reinterpret_cast<const float4 *>(c->at.q + h * D + 8 * cc + 4);
+            qr[k][h][0] = make_float2(q0.x, q0.y);
+            qr[k][h][1] = make_float2(q0.z, q0.w);
+            qr[k][h][2] = make_float2(q1.x, q1.y);
+            qr[k][h][3] = make_float2(q1.z, q1.w);
+        }
+    }
+    float mx[G], o[G][DPL];
+    float lw = 0.f;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         mx[g] = -INFINITY;
-        l[g] = 0.f;
 #pragma unroll
         for (int i = 0; i < DPL; ++i) o[g][i] = 0.f;
     }
@@ -889,7 +933,8 @@ __device__ bool attn_task(const RParams &p, unsigned char *ring, Ctl *c, CState 
         const int n = min(npp, a.nring - pg * npp);
         if ((pg & 1) == (warp >> 2))
             for (int j0 = (warp & 3) * 32; j0 < n; j0 += 4 * 32)
-                attn_block<D, G, false>(c, Kp + (size_t)j0 * D, Vp + (size_t)j0 * D, min(32, n - j0), mx, l, o);
+                attn_block<D, G, false>(c, Kp + (size_t)j0 * D, Vp + (size_t)j0 * D, min(32, n - j0), qr, gq, pq,
+                                        rot, mx, lw, o);
         __syncwarp();
         if (lane == 0) mbar_arrive(&c->empty_c[slot]);
         cs.odd_c ^= 1u << slot;
@@ -899,10 +944,15 @@ __device__ bool attn_task(const RParams &p, unsigned char *ring, Ctl *c, CState 
         // positions written during this launch: straight from the cache
         const size_t head = ((size_t)a.slot * s.nkv + a.h) * s.S;
         for (int j0 = a.c0 + a.nring + warp * 32; j0 < a.c1; j0 += kComputeWarps * 32)
-            attn_block<D, G, true>(c, L.kc + (head + j0) * D, L.vc + (head + j0) * D, min(32, a.c1 - j0), mx, l, o);
+            attn_block<D, G, true>(c, L.kc + (head + j0) * D, L.vc + (head + j0) * D, min(32, a.c1 - j0), qr, gq,
+                                   pq, rot, mx, lw, o);
     }
+    // head h's softmax sum: the lanes of head h add up (lane h * LPH holds it)
 #pragma unroll
-    for (int g = 0; g < G; ++g) l[g] = warp_sum(l[g]);
+    for (int off = NG; off < 32; off <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+    float l[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) l[g] = __shfl_sync(0xffffffffu, lw, g * LPH);
     // combine the warps' states: slot of warp w = G x (o[D], m, l)
     float *st = c->at.st[warp];
 #pragma unroll
@@ -1043,18 +1093,17 @@ __device__ void compute_role(const RParams &p, unsigned char *ring, Ctl *c) {
             if (p.trace && tid == 0) p.trace[t.sm].t_done = globaltimer();
             if (!group_sync(&c->cbar, cs.cph, p, c, (uint32_t)t.sm)) return;
             if (t.kind == ROP_LMHEAD && task_on(p, t, step)) {
-                // the task's argmax partials, then (their writers fenced and
-                // met) its count: the task that completes a step's count
+                // the task's argmax partials, then (their writers met at the
+                // barrier) its count: the task that completes a step's count
                 // reduces every task's partials
                 const int nrows = rrows_in_step(p, step);
                 if (tid < nrows) {
                     p.amax_val[(size_t)tid * p.num_lm_tasks + t.slot] = c->bestv[tid];
                     p.amax_idx[(size_t)tid * p.num_lm_tasks + t.slot] = c->besti[tid];
-                    __threadfence();
                 }
                 if (!group_sync(&c->cbar, cs.cph, p, c, (uint32_t)t.sm)) return;
                 if (tid == 0) {
-                    __threadfence();
+                    // after the barrier: a release that covers every thread's partials
                     // the LM tasks of one step finish before any of the next
                     // step's start, so the count's multiples mark each step's last
                     const uint32_t old = atom_add_acqrel_gpu(p.lm_cnt, 1u);

@@ -50,7 +50,7 @@ int main() {
     //    heads per item, pass s and quarter-warp, the 8 lanes read 8
     //    distinct bank groups (chunk index mod 8), and each lane's NS
     //    passes read its NS chunks once each
-    const int cases[5][2] = {{64, 2}, {64, 4}, {64, 8}, {128, 2}, {128, 4}};
+    const int cases[7][2] = {{64, 1}, {64, 2}, {64, 4}, {64, 8}, {128, 1}, {128, 2}, {128, 4}};
     for (const auto &cs : cases) {
         const int d = cs[0], ha = cs[1], ng = ha * d / 64, ns = 8 / ha;
         if (ng * ns != d / 8) { printf("groups x chunks != row chunks (d %d, ha %d)\n", d, ha); return 1; }
