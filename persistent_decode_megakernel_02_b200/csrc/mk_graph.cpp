@@ -34,12 +34,9 @@ bool plan_attention(Shape &s, int num_sms, int flags, int attn_chunks) {
     int per_q = num_sms / (s.Bmax * s.nq);                             // chunks per q head the SMs give
     if (per_q < 1) per_q = 1;
     s.HA = (kv || (!qi && cap > per_q)) ? hg : 1;
-    // the merge's shared staging: q-head items hold a head's chunk partials
-    // (d + 2 floats each); KV-head items those of all HA heads plus one
-    // weight per (head, chunk) and one sum per head
-    auto fits = [&](long long nc, int ha) {
-        return ha == 1 ? nc * (s.d + 2) <= kStageFloats : nc * ha * (s.d + 3) + ha <= kStageFloats;
-    };
+    // the merge's shared staging holds the chunk partials (d + 2 floats
+    // each) of every q head of an item
+    auto fits = [&](long long nc, int ha) { return nc * ha * (s.d + 2) <= kStageFloats; };
     // chosen by default, KV-head items give way to q-head items where a
     // given chunk count's partials would not fit the merge's staging area
     if (!kv && s.HA > 1 && attn_chunks > 0 && !fits(attn_chunks, s.HA)) s.HA = 1;

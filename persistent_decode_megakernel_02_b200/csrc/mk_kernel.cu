@@ -2086,55 +2086,27 @@ __device__ bool attn_kv_task(const Params &p, const Task &t, unsigned char *page
     }
     stamp_done(p, w);
     if (a.active && a.nc > 1 && a.c == 0) {
-        // chunk 0's item merges the chunks' partials of its q heads (every
-        // other chunk's item sits ahead of it on its SM's queue, so the wait
-        // always ends): first the (m, l) words of every (head, chunk) until
-        // fresh (a few words per thread), then all partials in one pass into
-        // shared memory [head][chunk][D + 2] (the tags still checked)
+        // chunk 0's item merges the partials of its q heads: polls them into
+        // shared memory ([head][chunk][D + 2]; tagged, so it waits for
+        // exactly the chunks it reads), then combines them there
+        const int nc = a.nc;
         if (!worker_sync(p, ctl, w)) return false;   // the combine above is done with the stage
-        for (int i = tid; i < HA * a.nc; i += kWorkerThreads) {
-            const uint64_t *src = part + ((size_t)(i / a.nc) * s.NC + i % a.nc) * (D + 2) + D;
-            ulonglong2 v = ld_tag2(src);
-            Spin sp;
-            while (!tag_ok(v.x, w.ep) || !tag_ok(v.y, w.ep)) {
-                if (!spin_ok(sp, p, ctl, W_TAG, (uint32_t)w.task_id, 6u)) return false;
-                v = ld_tag2(src);
-            }
-        }
+        if (!stage_partials(p, ctl, w, part, HA, nc * (D + 2), s.NC * (D + 2))) return false;
         if (!worker_sync(p, ctl, w)) return false;
-        {
-            // the chunk weights exp(m_c - M) once per (head, chunk), then the sums
-            const int nc = a.nc;
-            if (!stage_partials(p, ctl, w, part, HA, nc * (D + 2), s.NC * (D + 2))) return false;
-            if (!worker_sync(p, ctl, w)) return false;
-            float *wt = ctl->stage + (size_t)HA * nc * (D + 2);   // [HA][nc] weights, then [HA] sums
-            if (tid < HA) {
-                const float *sg = ctl->stage + (size_t)tid * nc * (D + 2);
-                float M = -INFINITY;
-                for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (D + 2) + D]);
-                float den = 0.f;
-                for (int c = 0; c < nc; ++c) {
-                    const float mc = sg[c * (D + 2) + D];
-                    const float f = mc == -INFINITY ? 0.f : expf(mc - M);
-                    wt[tid * nc + c] = f;
-                    den = fmaf(f, sg[c * (D + 2) + D + 1], den);
-                }
-                wt[HA * nc + tid] = 1.0f / den;
+        for (int i = tid; i < HA * D; i += kWorkerThreads) {
+            const int hh = i / D, e = i % D;
+            const float *sg = ctl->stage + (size_t)hh * nc * (D + 2);
+            float M = -INFINITY;
+            for (int c = 0; c < nc; ++c) M = fmaxf(M, sg[c * (D + 2) + D]);
+            float num = 0.f, den = 0.f;
+            for (int c = 0; c < nc; ++c) {
+                const float mc = sg[c * (D + 2) + D];
+                if (mc == -INFINITY) continue;
+                const float f = expf(mc - M);
+                num = fmaf(f, sg[c * (D + 2) + e], num);
+                den = fmaf(f, sg[c * (D + 2) + D + 1], den);
             }
-            if (!worker_sync(p, ctl, w)) return false;
-            for (int i = tid; i < HA * D; i += kWorkerThreads) {
-                const int hh = i / D, e = i % D;
-                const float *sg = ctl->stage + (size_t)hh * nc * (D + 2) + e;
-                const float *f = wt + hh * nc;
-                float n0 = 0.f, n1 = 0.f;
-                int c = 0;
-                for (; c + 1 < nc; c += 2) {
-                    n0 = fmaf(f[c], sg[c * (D + 2)], n0);
-                    n1 = fmaf(f[c + 1], sg[(c + 1) * (D + 2)], n1);
-                }
-                if (c < nc) n0 = fmaf(f[c], sg[c * (D + 2)], n0);
-                st_tag_rep(attn + i, p.tl.rep_qd, (n0 + n1) * wt[HA * nc + hh], w.ep_out);
-            }
+            st_tag_rep(attn + i, p.tl.rep_qd, num / den, w.ep_out);
         }
     }
     if (!worker_sync(p, ctl, w)) return false;

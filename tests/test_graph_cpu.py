@@ -179,7 +179,7 @@ def test_default_attention_chunks():
     i = info(wl.LLAMA_1B, 560, flags=mk.MK_FLAG_ATTN_KV_ITEMS)
     assert (i.attn_heads, i.attn_chunks) == (4, 1)
     # 8B shape: G = 4 at head_dim 128 (4 x 128 <= 512); 16k: 17 chunks fit
-    # the stage only up to (8192 - 4) // (4 * 131) = 15
+    # the stage only up to 8192 // (4 * 130) = 15
     i = info(wl.LLAMA_8B, 16640)
     assert (i.attn_heads, i.attn_chunks) == (4, 15)
     # a group of 8 q heads of 128 dims is split in halves of 4
@@ -255,15 +255,14 @@ def test_plan_refuses_partials_that_overflow_the_merge_stage():
         mk.plan(mk.make_config(shape, 64, 1, attn_chunks=125), SMS)
     assert ei.value.status == mk.MK_ERR_INVALID
     # an item of 2 q heads (MK_FLAG_ATTN_KV_ITEMS, G = 2) stages both heads'
-    # partials plus a weight per (head, chunk) and a sum per head:
-    # 61 x 2 x 67 + 2 = 8176 fit, 62 x 2 x 67 + 2 = 8310 do not
+    # partials: 62 chunks x 2 x 66 fit, 63 do not
     kv = mk.MK_FLAG_ATTN_KV_ITEMS
-    assert mk.plan(mk.make_config(shape, 64, 1, attn_chunks=61, flags=kv), SMS)["info"].attn_chunks == 61
+    assert mk.plan(mk.make_config(shape, 64, 1, attn_chunks=62, flags=kv), SMS)["info"].attn_chunks == 62
     with pytest.raises(mk.MkError):
-        mk.plan(mk.make_config(shape, 64, 1, attn_chunks=62, flags=kv), SMS)
+        mk.plan(mk.make_config(shape, 64, 1, attn_chunks=63, flags=kv), SMS)
     # chosen by default for a long cache, KV-head items give way to q-head
     # items when the given chunk count would not fit with them
     i = mk.plan(mk.make_config(shape, 126008, 1, attn_chunks=124), SMS)["info"]
     assert (i.attn_heads, i.attn_chunks) == (1, 124)
-    i = mk.plan(mk.make_config(shape, 126008, 1, attn_chunks=61), SMS)["info"]
-    assert (i.attn_heads, i.attn_chunks) == (2, 61)
+    i = mk.plan(mk.make_config(shape, 126008, 1, attn_chunks=62), SMS)["info"]
+    assert (i.attn_heads, i.attn_chunks) == (2, 62)

@@ -105,13 +105,12 @@ def test_many_active_attention_chunks_merged(head_dim, chunks, prefix):
 
 
 # Attention items of one KV head's q heads together (MK_FLAG_ATTN_KV_ITEMS):
-# many merged chunks (chunk 0's item stages every head's partials and a
-# weight per chunk: 61 chunks x 2 heads x 67 floats at head_dim 64, 31 x 2 x
-# 131 at 128).
+# many merged chunks (chunk 0's item stages every head's partials: 62
+# chunks x 2 heads x 66 floats at head_dim 64, 31 x 2 x 130 at 128).
 KV = 32
 
 
-@pytest.mark.parametrize("head_dim,chunks,prefix", [(64, 13, 13000), (64, 61, 62000), (128, 31, 32000)])
+@pytest.mark.parametrize("head_dim,chunks,prefix", [(64, 13, 13000), (64, 62, 63000), (128, 31, 32000)])
 def test_kv_head_items_many_chunks_merged(head_dim, chunks, prefix):
     shape = wl.TINY if head_dim == 64 else TINY_D128
     S = prefix + 8
