@@ -15,12 +15,16 @@
 //    tasks (128 x 128 bf16 in the tcgen05 canonical layout, 32 KB each) and
 //    the cached K/V positions of its attention items into a ring of
 //    kRStages shared-memory pages, ahead of every dependency.
-//  * scheduler (warp 9, one thread): gates every task on its dependency's
-//    event counter (counter >= threshold x epoch, MPK's event model, the
-//    "显著提升小LLM的性能..." page, Figure 3 text), publishes the task to the
-//    compute warps, and for a GEMV task streams the activation slab that
-//    goes with every weight page (the bf16 high and low halves of the kRows
-//    input vectors, 128 columns, 8 KB) into a second ring.
+//  * scheduler (warp 9, one thread): gates the embedding and attention
+//    tasks on their dependency's event counter (counter >= threshold x
+//    epoch, MPK's event model, the "显著提升小LLM的性能..." page, Figure 3
+//    text), publishes every task to the compute warps, and for a GEMV task
+//    streams the activation slab that goes with every weight page (the bf16
+//    high and low halves of the kRows input vectors, 128 columns, 8 KB) into
+//    a second ring -- each slab as soon as its own writers have released it
+//    (a counter per input slab: the producing op's tile, or the attention
+//    items of its heads), so an op's first pages overlap the tail of the op
+//    before it instead of waiting for all of it.
 //  * MMA issuer (warp 10, one thread; the warp owns the tensor memory):
 //    per page, 8 tcgen05.mma (M = 128, N = 2 kRows, K = 16) into an fp32
 //    accumulator in tensor memory; a commit frees the page and the slab, and
@@ -326,27 +330,44 @@ __device__ void sched_role(const RParams &p, unsigned char *slabs, Ctl *c) {
         const uint32_t ep = c->ep + (uint32_t)step;
         for (int qi = q0; qi < q1; ++qi) {
             const Task t = p.qtasks[qi];
-            // the first op of a step waits for the previous step's last
-            const uint32_t target = p.thresholds[t.dep] * (t.kind == ROP_EMBED ? ep - 1u : ep);
-            Spin s;
-            const unsigned long long td = p.sm_stats ? globaltimer() : 0ull;
-            while ((int32_t)(ld_acquire_gpu(&p.events[t.dep]) - target) < 0)
-                if (!spin_ok(s, p, c, W_DEP, (uint32_t)t.sm, (uint32_t)t.dep)) return;
-            if (p.sm_stats) *stat_slot(p, RS_SCHED_DEP) += globaltimer() - td;
-            // what the producers wrote is read below by bulk copies (the
-            // async proxy) and by the compute warps
-            asm volatile("fence.proxy.async.global;" ::: "memory");
+            const bool gemv = is_gemv(t.kind);
+            if (!gemv) {
+                // embedding (the first op of a step waits for the previous
+                // step's last) and attention: the whole dependency op
+                const uint32_t target = p.thresholds[t.dep] * (t.kind == ROP_EMBED ? ep - 1u : ep);
+                Spin s;
+                const unsigned long long td = p.sm_stats ? globaltimer() : 0ull;
+                while ((int32_t)(ld_acquire_gpu(&p.events[t.dep]) - target) < 0)
+                    if (!spin_ok(s, p, c, W_DEP, (uint32_t)t.sm, (uint32_t)t.dep)) return;
+                if (p.sm_stats) *stat_slot(p, RS_SCHED_DEP) += globaltimer() - td;
+                // what the producers wrote is read by the compute warps
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+            }
+            // a GEMV task's compute warps only read what its accumulators
+            // depend on (through the slabs below) and what the producers of
+            // those slabs' inputs wrote before them, so they start at once
             if (p.trace) p.trace[t.sm].t_ready = globaltimer();
             st_release_cta_shared(&c->ready_upto, (uint32_t)(step * qlen + (qi - q0) + 1));
-            if (!is_gemv(t.kind) || !task_on(p, t, step)) continue;
+            if (!gemv || !task_on(p, t, step)) continue;
             const RGemv g = rgemv(p.s, t.kind);
             const char *x = reinterpret_cast<const char *>(gemv_input(p, t));
+            const uint32_t *rdy = t.kind == ROP_LMHEAD ? p.rdy_lm : p.buf[t.layer].rdy[rgemv_slot(t.kind)];
+            const uint32_t need = rslab_writers(p.s, t.kind) * ep;
             for (int pg = t.begin; pg < t.end; ++pg, ++bseq) {
                 const uint32_t slot = bseq % kRStages;
                 if (bseq >= (uint32_t)kRStages &&
                     !wait_bar_t(&c->bempty[slot], ((bseq / kRStages) - 1u) & 1u, p, c, W_EMPTY, (uint32_t)t.sm,
                                 stat_slot(p, RS_SCHED_SLAB)))
                     return;
+                {
+                    // the page's input slab is written (all its writers released)
+                    Spin s;
+                    const unsigned long long td = p.sm_stats ? globaltimer() : 0ull;
+                    while ((int32_t)(ld_acquire_gpu(&rdy[pg % g.slabs]) - need) < 0)
+                        if (!spin_ok(s, p, c, W_DEP, (uint32_t)t.sm, (uint32_t)(pg % g.slabs))) return;
+                    if (p.sm_stats) *stat_slot(p, RS_SCHED_DEP) += globaltimer() - td;
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                }
                 mbar_arrive_expect_tx(&c->bfull[slot], kRSlabBytes);
                 bulk_g2s(slabs + (size_t)slot * kRSlabBytes, x + (size_t)(pg % g.slabs) * kRSlabBytes, kRSlabBytes,
                          &c->bfull[slot]);
@@ -532,7 +553,7 @@ __device__ __forceinline__ bool load_rs(const RParams &p, Ctl *c, CState &cs, co
 // and summed into the per-tile sums of squares of the next RMSNorm.
 __device__ __forceinline__ bool resid_out(const RParams &p, Ctl *c, CState &cs, int tile, int m,
                                           const float (&x)[kRows], int nrows, float *x_out, uint16_t *x_next,
-                                          const uint16_t *gain, float *ss_out) {
+                                          const uint16_t *gain, float *ss_out, uint32_t *rdy_next) {
     const int R = tile * kRTile + m;
     const float g = __bfloat162float(__ushort_as_bfloat16(gain[R]));
     float sq[kRows];
@@ -543,9 +564,16 @@ __device__ __forceinline__ bool resid_out(const RParams &p, Ctl *c, CState &cs, 
         st_split(x_next, r, R, on ? x[r] * g : 0.f);
         sq[r] = on ? x[r] * x[r] : 0.f;
     }
+    // the slab is read by bulk copies (the async proxy) on other SMs
+    asm volatile("fence.proxy.async.global;" ::: "memory");
     float tot;
     if (!epi_rowsum(p, c, cs, sq, tot)) return false;
     if (threadIdx.x < kRows) ss_out[(size_t)tile * kRows + threadIdx.x] = tot;
+    // slab `tile` of the next op's input is written (every thread's part
+    // before the barrier in epi_rowsum, the row sums before the warp sync):
+    // one release lets that op's pages on it start
+    __syncwarp();
+    if (threadIdx.x == 0) red_release_gpu(rdy_next + tile, 1u);
     return true;
 }
 
@@ -597,7 +625,8 @@ __device__ bool tile_epilogue(const RParams &p, Ctl *c, CState &cs, const Task &
         float x[kRows];
 #pragma unroll
         for (int r = 0; r < kRows; ++r) x[r] = r < nrows ? ldcg(xin + (size_t)r * s.H + R) + y[r] : 0.f;
-        return resid_out(p, c, cs, tile, m, x, nrows, B.xa, B.xg, p.layers[t.layer].g_mlp, B.ssg);
+        return resid_out(p, c, cs, tile, m, x, nrows, B.xa, B.xg, p.layers[t.layer].g_mlp, B.ssg,
+                         B.rdy[rgemv_slot(ROP_GATEUP)]);
     }
     case ROP_GATEUP: {
         const RLayerBuf &B = p.buf[t.layer];
@@ -610,6 +639,11 @@ __device__ bool tile_epilogue(const RParams &p, Ctl *c, CState &cs, const Task &
 #pragma unroll
             for (int r = 0; r < kRows; ++r)
                 st_split(B.xd, r, j, r < nrows ? silu(y[r]) * c->xbuf[m + kRTile / 2][r] : 0.f);
+            // half of slab tile / 2 of the down projection's input: each
+            // writer warp releases its 32 columns (4 releases a slab)
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __syncwarp();
+            if ((m & 31) == 0) red_release_gpu(B.rdy[rgemv_slot(ROP_DOWN)] + tile / 2, 1u);
         }
         return true;
     }
@@ -621,7 +655,8 @@ __device__ bool tile_epilogue(const RParams &p, Ctl *c, CState &cs, const Task &
 #pragma unroll
         for (int r = 0; r < kRows; ++r) x[r] = r < nrows ? ldcg(B.xa + (size_t)r * s.H + R) + y[r] : 0.f;
         return resid_out(p, c, cs, tile, m, x, nrows, B.xb, last ? p.xlm : p.buf[t.layer + 1].xq,
-                         last ? p.g_final : p.layers[t.layer + 1].g_attn, last ? p.sslm : p.buf[t.layer + 1].ssq);
+                         last ? p.g_final : p.layers[t.layer + 1].g_attn, last ? p.sslm : p.buf[t.layer + 1].ssq,
+                         last ? p.rdy_lm : p.buf[t.layer + 1].rdy[rgemv_slot(ROP_QKV)]);
     }
     default: {   // ROP_LMHEAD
         if (!load_rs(p, c, cs, p.sslm)) return false;
@@ -745,7 +780,8 @@ __device__ bool embed_task(const RParams &p, Ctl *c, CState &cs, const Task &t) 
                                p.embed[(size_t)rrow(p, cs.step, r).tok * p.s.H + tile * kRTile + m]))
                          : 0.f;
     const RLayerBuf &B = p.buf[0];
-    return resid_out(p, c, cs, tile, m, x, nrows, p.x0, B.xq, p.layers[0].g_attn, B.ssq);
+    return resid_out(p, c, cs, tile, m, x, nrows, p.x0, B.xq, p.layers[0].g_attn, B.ssq,
+                     B.rdy[rgemv_slot(ROP_QKV)]);
 }
 
 // One block of up to 32 positions of an attention item (G query heads of
@@ -1092,6 +1128,17 @@ __device__ void compute_role(const RParams &p, unsigned char *ring, Ctl *c) {
             asm volatile("fence.proxy.async.global;" ::: "memory");
             if (p.trace && tid == 0) p.trace[t.sm].t_done = globaltimer();
             if (!group_sync(&c->cbar, cs.cph, p, c, (uint32_t)t.sm)) return;
+            if (t.kind == ROP_ATTN && tid == 0) {
+                // chunk 0's item of (row, KV head) has written the heads'
+                // outputs (directly or merged; nothing for an inactive row):
+                // it releases the O-projection input slabs they fall in
+                const Item a = attn_item(p, step, t.begin);
+                if (a.c == 0) {
+                    const int gd = p.s.G * p.s.d;
+                    uint32_t *rdy = p.buf[t.layer].rdy[rgemv_slot(ROP_OPROJ)];
+                    for (int sl = a.h * gd / kRSlab; sl <= (a.h * gd + gd - 1) / kRSlab; ++sl) red_release_gpu(rdy + sl, 1u);
+                }
+            }
             if (t.kind == ROP_LMHEAD && task_on(p, t, step)) {
                 // the task's argmax partials, then (their writers met at the
                 // barrier) its count: the task that completes a step's count

@@ -100,6 +100,9 @@ constexpr int kRAttnChunk = 1024;
 //  part: tagged attention partials [kRows][nkv][NC][G * (d + 2)]
 //  acc_*: split-tile accumulators [tiles][128][kRows] fp32 (zero between
 //    uses), cnt_*: pages accumulated per tile (epoch-scaled) [tiles]
+//  rdy_*: per input slab of the op, the releases of its writers so far
+//    (epoch-scaled) [K / 128]: a GEMV task's pages start on a slab as soon
+//    as that slab is written, not when the whole producing op is done
 struct RLayerBuf {
     uint16_t *xq, *xo, *xg, *xd;
     float *xa, *xb;
@@ -108,12 +111,28 @@ struct RLayerBuf {
     uint64_t *part;
     float *acc[4];          // QKV, OPROJ, GATEUP, DOWN (index: rgemv_slot)
     uint32_t *cnt[4];
+    uint32_t *rdy[4];       // per input slab of QKV, OPROJ, GATEUP, DOWN: writers that have
+                            //  released it (epoch-scaled: rslab_writers(op) per step)
 };
 
 // Index of a layer's GEMV op in RLayerBuf::acc / cnt (the attention op sits
 // between QKV and OPROJ in the op order, so the op values are not it).
 MK_HD inline int rgemv_slot(int op) {
     return op == ROP_QKV ? 0 : op == ROP_OPROJ ? 1 : op == ROP_GATEUP ? 2 : 3;
+}
+
+// Releases of one input slab (128 columns) of a GEMV op per step: one
+// producing tile for the QKV, gate/up and LM-head inputs (a residual
+// tile of the down projection, the O-projection or the embedding); two
+// gate/up tiles of 64 outputs, one release per writer warp each, for the
+// down projection's; one per row and KV head covering the slab for the
+// O-projection's (the attention output: every chunk-0 item of a (row, KV
+// head) releases, active or not, so the count is the same every step).
+MK_HD inline uint32_t rslab_writers(const Shape &s, int op) {
+    if (op == ROP_DOWN) return 4u;
+    if (op != ROP_OPROJ) return 1u;
+    const int gd = s.G * s.d;
+    return (uint32_t)kRows * (uint32_t)(gd >= kRSlab ? 1 : kRSlab / gd);
 }
 
 // Device pointers of one layer's weights (library copies in the page
@@ -163,6 +182,7 @@ struct RParams {
     const RLayerBuf *buf;       // [L]
     uint16_t *xlm;              // LM-head input [H / 128][8 KB]
     float *sslm;                // [H / 128][kRows]
+    uint32_t *rdy_lm;           // LM-head input slab releases (epoch-scaled) [H / 128]
     float *x0;                  // embedding rows [kRows][H] fp32
     float *lm_acc;              // [tiles][128][kRows]
     uint32_t *lm_tcnt;          // [tiles]

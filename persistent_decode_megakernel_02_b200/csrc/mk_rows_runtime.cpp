@@ -217,6 +217,7 @@ int rows_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, cons
                 const RGemv g = rgemv(s, op);
                 RK_TRY(ralloc(c, &b.acc[rgemv_slot(op)], (size_t)g.tiles * kRTile * kRows, true));
                 RK_TRY(ralloc(c, &b.cnt[rgemv_slot(op)], (size_t)g.tiles, true));
+                RK_TRY(ralloc(c, &b.rdy[rgemv_slot(op)], (size_t)g.slabs, true));
             }
         }
         RLayerBuf *d_buf;
@@ -225,6 +226,7 @@ int rows_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, cons
         p.buf = d_buf;
         RK_TRY(ralloc(c, &p.xlm, xh));
         RK_TRY(ralloc(c, &p.sslm, tiles_h * kRows));
+        RK_TRY(ralloc(c, &p.rdy_lm, (size_t)(s.H / kRSlab), true));
         RK_TRY(ralloc(c, &p.x0, (size_t)kRows * s.H));
         const RGemv glm = rgemv(s, ROP_LMHEAD);
         RK_TRY(ralloc(c, &p.lm_acc, (size_t)glm.tiles * kRTile * kRows, true));
