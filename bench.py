@@ -79,32 +79,44 @@ def bandwidth_bound_ms(bytes_per_step: float, gbs: float) -> float:
 
 
 STEP_KERNEL_SOURCES = ("mk_kernel.cu", "mk_internal.h", "mk_ptx.cuh")
+ROWS_KERNEL_SOURCES = ("mk_rows.cu", "mk_rows.h", "mk_internal.h", "mk_ptx.cuh")
 
 
-def step_kernel_digest() -> str:
-    """Hash of the sources the batch-1 step kernel is compiled from."""
+def kernel_digest(sources=STEP_KERNEL_SOURCES) -> str:
+    """Hash of the sources a kernel is compiled from."""
     import hashlib
     h = hashlib.sha256()
-    for name in STEP_KERNEL_SOURCES:
+    for name in sources:
         with open(os.path.join(ROOT, "persistent_decode_megakernel_02_b200", "csrc", name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
     return h.hexdigest()
 
 
+def step_kernel_digest() -> str:
+    """Hash of the sources the batch-1 step kernel is compiled from."""
+    return kernel_digest(STEP_KERNEL_SOURCES)
+
+
 def profiled_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu capture of the step
-    kernel, only while that kernel's sources are the ones profiled (else
-    None)."""
+    """DRAM bytes per launch from the committed ncu capture of the kernel
+    that runs `workload` (profiles/traffic.json, one record per workload),
+    only while that kernel's sources are the ones profiled (else None)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
-        digest = step_kernel_digest()
     except (OSError, ValueError):
         return None
-    if t.get("workload") != workload or t.get("kernel_digest") != digest:
-        return None
-    return int(t["dram_bytes_read_per_launch"]) + int(t["dram_bytes_write_per_launch"])
+    for e in t.get("entries", []):
+        if e.get("workload") != workload:
+            continue
+        try:
+            if e.get("kernel_digest") != kernel_digest(tuple(e.get("sources", STEP_KERNEL_SOURCES))):
+                return None
+        except OSError:
+            return None
+        return int(e["dram_bytes_read_per_launch"]) + int(e["dram_bytes_write_per_launch"])
+    return None
 
 
 def measured_peaks() -> dict:
@@ -334,7 +346,7 @@ def main_batched(args, world, rank, local, wk, W, K):
     achieved = alg_bytes / (step_ms * 1e-3) / 1e9
     flops = 2.0 * B * (step_weight_bytes(shape) / 2)   # one multiply-add per weight per row
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": profiled_traffic(wk.name),
                 "peak_source": peaks["source"], "bytes_per_launch": int(alg_bytes),
                 "bound_ms": round(bandwidth_bound_ms(alg_bytes, peaks["hbm_gbs"]), 4),
                 "tensor_tflops": round(flops / (step_ms * 1e-3) / 1e12, 2)}

@@ -415,8 +415,9 @@ int mk_plan(const mk_config *cfg, int num_sms, mk_info *info,
  * the tables is serialised by a lock, so host threads driving different
  * devices do not interfere.  The first call on a device looks up the
  * array's address and sets up the kernel for that device; a call whose shape
- * differs from the previous call's on that device uploads new task and RoPE
- * tables, and a call whose weight or KV pointers differ uploads a new layer
+ * differs from the previous call's on that device (its sizes, or the
+ * attention items its flags choose: MK_FLAG_ATTN_KV_ITEMS) uploads new task
+ * and RoPE tables, and a call whose weight or KV pointers differ uploads a new layer
  * table -- both synchronise the stream, so make such calls outside stream
  * capture (the first call on a device included).  The tables carry a key
  * that the kernel compares with the key its launch was set up with: a

@@ -20,9 +20,10 @@
 // host threads driving different devices do not mix their tables.  The first
 // call on a device looks up the array's device address with
 // cudaGetSymbolAddress (with that device current) and sets the kernel's
-// shared-memory attribute; a call whose shape, weights or KV cache differ
-// from the previous call's on that device uploads new tables and
-// synchronises the stream.  Make such calls outside stream capture.  The
+// shared-memory attribute; a call whose planned shape (the config's sizes
+// and the attention items its flags and the SM count choose), weights or KV
+// cache differ from the previous call's on that device uploads new tables
+// and synchronises the stream.  Make such calls outside stream capture.  The
 // uploaded tables carry a key the kernel checks against the key its launch
 // was set up with: a launch set up for tables that have been replaced since
 // (a replay of an earlier launch) runs nothing and reports MK_ERR_INVALID.

@@ -87,3 +87,31 @@ def test_oracle_baseline_times_full_steps_pinned_to_one_core():
     assert len(times) == 3 and all(t > 0 for t in times)
     # the runner's cache advanced through every step: position 4 was written
     assert any(np.any(k[:, 4] != 0) for k in runner.kc)
+
+
+def test_profiled_traffic_is_keyed_to_the_profiled_kernel_sources(tmp_path, monkeypatch):
+    import json
+    import bench
+    csrc = tmp_path / "persistent_decode_megakernel_02_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in set(bench.STEP_KERNEL_SOURCES) | set(bench.ROWS_KERNEL_SOURCES):
+        (csrc / name).write_text(f"// {name}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    entries = [{"workload": "llama1b", "sources": list(bench.STEP_KERNEL_SOURCES),
+                "kernel_digest": bench.kernel_digest(bench.STEP_KERNEL_SOURCES),
+                "dram_bytes_read_per_launch": 1000, "dram_bytes_write_per_launch": 24},
+               {"workload": "batched16", "sources": list(bench.ROWS_KERNEL_SOURCES),
+                "kernel_digest": bench.kernel_digest(bench.ROWS_KERNEL_SOURCES),
+                "dram_bytes_read_per_launch": 7, "dram_bytes_write_per_launch": 1}]
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"entries": entries}))
+    assert bench.profiled_traffic("llama1b") == 1024
+    assert bench.profiled_traffic("batched16") == 8
+    assert bench.profiled_traffic("longctx") is None          # no capture for it
+    # a change to the batched kernel's sources voids its record only
+    (csrc / "mk_rows.cu").write_text("// changed\n")
+    assert bench.profiled_traffic("batched16") is None
+    assert bench.profiled_traffic("llama1b") == 1024
+    # and a change to a shared header voids both
+    (csrc / "mk_ptx.cuh").write_text("// changed\n")
+    assert bench.profiled_traffic("llama1b") is None
