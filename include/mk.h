@@ -264,8 +264,8 @@ int mk_generate(mk_ctx *ctx, const int32_t *tokens, int n_prompt, const int32_t 
  * matrices are copied into a library-owned tile layout at create time.
  * Shape limits: hidden, n_q_heads*head_dim, n_kv_heads*head_dim and ffn
  * multiples of 128; n_q_heads / n_kv_heads = 1, 2 or 4 with (n_q_heads /
- * n_kv_heads) * head_dim <= 512; attn_chunks: chunks of at least 1024
- * positions per (row, KV head), default ceil(max_seq / 1024).
+ * n_kv_heads) * head_dim <= 512; attn_chunks: chunks of at least 4096
+ * positions per (row, KV head), default ceil(max_seq / 4096).
  * MK_FLAG_EVENT_WAIT (tasks always wait on event counters here),
  * mk_generate, mk_get_sm_stats and mk_debug_withhold_event are not
  * available on such contexts (MK_ERR_INVALID); mk_read_buffer offers

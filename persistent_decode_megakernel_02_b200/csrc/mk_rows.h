@@ -85,8 +85,12 @@ MK_HD inline size_t rx_elem(int n, int k) {
 // Attention positions per page (K block then V block).
 MK_HD inline int rattn_pos_per_page(int d) { return kRPageBytes / (4 * d); }
 // A row's positions are split into chunks of at least this many (one
-// attention item each); short contexts need no merge.
-constexpr int kRAttnChunk = 1024;
+// attention item each); contexts up to this long need no merge.  Longer
+// chunks measured faster at the batched workloads' positions (<= ~2200):
+// batch 16, 1024 / 2048 / 4096 positions: 1.816 / 1.652 / 1.591 ms/step --
+// a merge costs chunk 0's item a wait for the slowest chunk and an extra
+// pass, more than the longer items cost in balance.
+constexpr int kRAttnChunk = 4096;
 
 // Per-layer device buffers of the rows step.
 //  xq, xo, xg, xd: the bf16 high/low inputs of QKV (rmsnorm gain folded in,

@@ -7,7 +7,8 @@ of the weights with the rows on the tensor cores.
 * decode batches of 4, 8 and 16 sequences at staggered positions (start
   positions uniform in [32, 2048], KV prefixes of seeded N(0,1) values, the
   batched workload's recipe): every sequence's logits against the oracle's
-  step on that sequence, teacher-forced, at the stated tolerance;
+  step on that sequence, teacher-forced, at the stated tolerance; and 4
+  sequences at 4500..9000 positions, whose attention items are merged;
 * a prompt in one launch (mk_prefill, 16 tokens per kernel step, causal
   attention within the prompt): the KV entries it writes and the last
   token's logits against the oracle fed the same prompt token by token;
@@ -87,6 +88,26 @@ def test_batched_decode_staggered_positions(B):
             kg = bt.k[l][b, :, p0:p0 + 3].float().cpu().numpy()
             kr = torch.from_numpy(bt.kr[b][l][:, p0:p0 + 3].view(np.int16)).view(torch.bfloat16).float().numpy()
             assert np.abs(kg - kr).max() <= 2e-2 * np.abs(kr).max()
+
+
+def test_batched_decode_long_contexts_merged_chunks():
+    # a row's positions split into chunks of at least 4096 (one item each,
+    # chunk 0's item merges): start positions in [4500, 9000] give 2 or 3
+    # chunks per row, merged in every layer
+    shape = wl.TINY
+    B = 4
+    S = 9000 + 8
+    starts = wl.make_start_positions(B, seed=21, lo=4500, hi=9000)
+    bt = Batch(shape, B, S, prefill_len=9000)
+    assert bt.ctx.info().attn_chunks == 3
+    toks = [int(t) for t in wl.make_prompt(shape.vocab, B, seed=8)]
+    for step in range(2):
+        pos = [int(starts[b]) + step for b in range(B)]
+        g_tok, g_log = bt.gpu_step(toks, pos)
+        refs = [bt.ref_step(b, toks[b], pos[b]) for b in range(B)]
+        for b in range(B):
+            _check(g_log[b], g_tok[b], refs[b], f"step {step} seq {b} pos {pos[b]}")
+        toks = [r["next"] for r in refs]
 
 
 def test_batch_smaller_than_the_context_and_random_gains():
