@@ -102,7 +102,7 @@ int shape_from_config(const mk_config *c, int num_sms, Shape &s) {
     s.theta = c->rope_theta; s.eps = c->rms_eps;
     s.tmem = (c->flags & MK_FLAG_NO_TMEM_RING) ? 0 : 1;
     if (rows) {
-        // the batched step: its own tiling, chunks of at least 1024 positions
+        // the batched step: its own tiling, chunks of at least kRAttnChunk positions
         s.tmem = 0;
         s.HA = s.G;   // items per (row, KV head, chunk)
         s.NC = c->attn_chunks > 0 ? c->attn_chunks : rows_default_chunks(s.S);
