@@ -278,6 +278,83 @@ def run_oracle_steps(runner: OracleRunner, tokens, positions, n_warm: int, n_max
     return times
 
 
+def batched_workload(wk, W: int, K: int, world: int):
+    """Start positions, KV capacity, metric and config of a batched workload
+    (the same for the kernel's arm and the reference arm)."""
+    shape, B = wk.shape, wk.batch
+    starts = wl.make_start_positions(B, seed=7)
+    max_seq = max(wk.max_seq, int(starts.max()) + W + K + 1)
+    metric = (f"decode ms/token @bs{B} ({shape.name}, staggered positions); achieved HBM GB/s vs roofline")
+    config = {"workload": f"{wk.name}: {shape.name} L{shape.layers} H{shape.hidden} {shape.n_q_heads}/"
+                          f"{shape.n_kv_heads} heads d{shape.head_dim} F{shape.ffn} V{shape.vocab}, {B} sequences "
+                          f"starting at positions uniform in [32, 2048] (KV prefix N(0,1))",
+              "batch": B, "start_positions": [int(x) for x in starts],
+              "l2": "weights exceed L2 (no flush needed)", "parallelism": f"replicas x{world}"}
+    return starts, max_seq, metric, config
+
+
+def single_workload(wk, W: int, K: int, world: int):
+    """First position, KV capacity and config of a batch-1 workload."""
+    shape = wk.shape
+    prefill = wk.prefill_len
+    start = prefill if prefill else 0
+    max_seq = max(wk.max_seq, start + W + K + 1)
+    config = {"workload": f"{wk.name}: {shape.name} L{shape.layers} H{shape.hidden} "
+                          f"{shape.n_q_heads}/{shape.n_kv_heads} heads d{shape.head_dim} "
+                          f"F{shape.ffn} V{shape.vocab}" + (f", KV prefilled to {prefill}" if prefill else ""),
+              "batch": 1, "positions": [start + W, start + W + K - 1],
+              "l2": "weights exceed L2 (no flush needed)", "parallelism": f"replicas x{world}"}
+    return start, max_seq, config
+
+
+def main_reference(args, world, rank, wk, W, K):
+    """--impl reference: the oracle as it stands, full decode steps on one
+    pinned host core, for the same workload, metric and unit as the kernel's
+    arm; rank 0 alone (the other ranks exit at once).  A batched workload's
+    tokens are independent sequences, so its sample cycles through them:
+    oracle step j decodes one token of sequence j mod B at that sequence's
+    own position, and ms per oracle step is ms per token."""
+    if rank != 0:
+        return
+    import torch
+    shape = wk.shape
+    w_host = wl.make_weights(shape, seed=1234, device="cuda" if torch.cuda.is_available() else "cpu")
+    bits = w_host.numpy_bits()
+    del w_host
+    n_all = W + K
+    prompt = wl.make_prompt(shape.vocab, n_all, seed=42)
+    if wk.batch > 1:
+        B = wk.batch
+        starts, max_seq, metric, config = batched_workload(wk, W, K, world)
+        positions = np.array([int(starts[j % B]) + j // B for j in range(n_all)])
+        where = lambda n: f"step j decoding one token of sequence j mod {B} at its own position"
+    else:
+        start, max_seq, config = single_workload(wk, W, K, world)
+        metric = METRIC
+        positions = np.arange(start, start + n_all)
+        where = lambda n: f"positions {start + W}..{start + W + n - 1}"
+    runner = OracleRunner(shape, bits, max_seq, wk.prefill_len)
+    with PinnedCore() as pin:
+        t_run = time.perf_counter()
+        times = run_oracle_steps(runner, prompt, positions, W, K, args.ref_budget_s)
+        t_run = time.perf_counter() - t_run
+    n = len(times)
+    ms = float(np.mean(times))
+    sample = (f"{n} full oracle decode steps (every layer, every LM-head row; fp64 C, "
+              f"single thread pinned to core {pin.core} of {host_cores()}) after {W} untimed "
+              f"ones, {where(n)}"
+              + ("" if n == K else f"; {K} requested, capped by the {args.ref_budget_s:.0f} s budget"))
+    out = {"impl": "reference", "metric": metric, "value": ms, "unit": UNIT, "n_gpus": world,
+           "steps": n, "warmup": W, "ms_per_step": ms, "higher_is_better": False,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": config,
+           "cpu_baseline": {"value": ms, "unit": UNIT, "cores": 1, "kind": "oracle",
+                            "sample": sample, "pinned_core": pin.core, "host_cores": host_cores(),
+                            "wall_s": round(t_run, 2)},
+           "e2e": {"value": ms, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
 def main_batched(args, world, rank, local, wk, W, K):
     """Batched decode (the batched tensor-core step): wk.batch independent
     sequences at start positions uniform in [32, 2048] over KV prefixes of
@@ -293,14 +370,7 @@ def main_batched(args, world, rank, local, wk, W, K):
     torch.cuda.set_device(dev)
     from persistent_decode_megakernel_02_b200 import mk
     shape, B = wk.shape, wk.batch
-    starts = wl.make_start_positions(B, seed=7)
-    max_seq = max(wk.max_seq, int(starts.max()) + W + K + 1)
-    metric = (f"decode ms/token @bs{B} ({shape.name}, staggered positions); achieved HBM GB/s vs roofline")
-    config = {"workload": f"{wk.name}: {shape.name} L{shape.layers} H{shape.hidden} {shape.n_q_heads}/"
-                          f"{shape.n_kv_heads} heads d{shape.head_dim} F{shape.ffn} V{shape.vocab}, {B} sequences "
-                          f"starting at positions uniform in [32, 2048] (KV prefix N(0,1))",
-              "batch": B, "start_positions": [int(x) for x in starts],
-              "l2": "weights exceed L2 (no flush needed)", "parallelism": f"replicas x{world}"}
+    starts, max_seq, metric, config = batched_workload(wk, W, K, world)
     weights = wl.make_weights(shape, seed=1234, device=dev)
     kc, vc = wl.make_kv(shape, B, max_seq, device=dev, prefill_len=wk.prefill_len)
     ctx = mk.Context(weights, kc, vc, max_seq, B)
@@ -468,48 +538,13 @@ def main():
     W = max(3, args.warmup)
     K = max(1, args.steps)
     wk = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return main_reference(args, world, rank, wk, W, K)
     if wk.batch > 1:
         return main_batched(args, world, rank, local, wk, W, K)
     shape = wk.shape
     prefill = wk.prefill_len
-    start = prefill if prefill else 0
-    max_seq = max(wk.max_seq, start + W + K + 1)
-    config = {"workload": f"{wk.name}: {shape.name} L{shape.layers} H{shape.hidden} "
-                          f"{shape.n_q_heads}/{shape.n_kv_heads} heads d{shape.head_dim} "
-                          f"F{shape.ffn} V{shape.vocab}" + (f", KV prefilled to {prefill}" if prefill else ""),
-              "batch": 1, "positions": [start + W, start + W + K - 1],
-              "l2": "weights exceed L2 (no flush needed)", "parallelism": f"replicas x{world}"}
-
-    if args.impl == "reference":
-        if rank != 0:
-            return
-        import torch
-        w_host = wl.make_weights(shape, seed=1234, device="cuda" if torch.cuda.is_available() else "cpu")
-        bits = w_host.numpy_bits()
-        del w_host
-        runner = OracleRunner(shape, bits, max_seq, prefill)
-        prompt = wl.make_prompt(shape.vocab, W + K, seed=42)
-        positions = np.arange(start, start + W + K)
-        with PinnedCore() as pin:
-            t_run = time.perf_counter()
-            times = run_oracle_steps(runner, prompt, positions, W, K, args.ref_budget_s)
-            t_run = time.perf_counter() - t_run
-        n = len(times)
-        ms = float(np.mean(times))
-        sample = (f"{n} full oracle decode steps (every layer, every LM-head row; fp64 C, "
-                  f"single thread pinned to core {pin.core} of {host_cores()}) after {W} untimed "
-                  f"ones, positions {start + W}..{start + W + n - 1}"
-                  + ("" if n == K else f"; {K} requested, capped by the {args.ref_budget_s:.0f} s budget"))
-        out = {"impl": "reference", "metric": METRIC, "value": ms, "unit": UNIT, "n_gpus": world,
-               "steps": n, "warmup": W, "ms_per_step": ms, "higher_is_better": False,
-               "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-               "config": config,
-               "cpu_baseline": {"value": ms, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                "sample": sample, "pinned_core": pin.core, "host_cores": host_cores(),
-                                "wall_s": round(t_run, 2)},
-               "e2e": {"value": ms, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(out), flush=True)
-        return
+    start, max_seq, config = single_workload(wk, W, K, world)
 
     import torch
     if world > 1:

@@ -115,3 +115,30 @@ def test_profiled_traffic_is_keyed_to_the_profiled_kernel_sources(tmp_path, monk
     # and a change to a shared header voids both
     (csrc / "mk_ptx.cuh").write_text("// changed\n")
     assert bench.profiled_traffic("llama1b") is None
+
+
+def test_reference_arm_of_a_batched_workload_times_the_oracle(capsys):
+    # the reference arm of a batched workload reports the kernel arm's metric
+    # and config, and its oracle steps visit every sequence at its own
+    # staggered position (steps j, j + B, ... belong to sequence j)
+    import argparse
+    wk = wl.Workload("tiny4", wl.TINY, 4, 0, 8, 2112, prefill_len=2048, staggered=True)
+    args = argparse.Namespace(ref_budget_s=0.0)
+    seen = []
+    real = bench.OracleRunner.step_ms
+
+    def spy(self, token, pos):
+        seen.append(int(pos))
+        return real(self, token, pos)
+
+    bench.OracleRunner.step_ms = spy
+    try:
+        bench.main_reference(args, 1, 0, wk, 3, 5)
+    finally:
+        bench.OracleRunner.step_ms = real
+    rec = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    starts, _, metric, config = bench.batched_workload(wk, 3, 5, 1)
+    assert rec["impl"] == "reference" and rec["metric"] == metric and rec["config"] == config
+    assert rec["unit"] == "ms/token" and rec["value"] > 0 and rec["steps"] == 3
+    assert seen == [int(starts[j % 4]) + j // 4 for j in range(6)]
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["e2e"]["h2d_bytes_per_step"] == 0
