@@ -181,7 +181,9 @@ typedef struct mk_ctx mk_ctx;
  * task-graph generation by compile()), with the tasks placed in static per-SM queues (the Hazy page,
  * sfrk.com.cn/ruanjian/202506/86466, paragraph on the per-SM execution plan).
  * The device must be compute capability 10.0 (B200; the library holds sm_100a
- * code only): any other device gives MK_ERR_INVALID.
+ * code only), support cooperative launches and offer the kernel's shared
+ * memory per block: any other device gives MK_ERR_INVALID
+ * (mk_device_supported states the rule).
  * The q/k/v and gate/up matrices are copied into a library-owned layout
  * (rows in the order the kernel streams them, so every task reads one
  * contiguous range); unless MK_FLAG_NO_TMEM_RING is set, so are the other
@@ -393,6 +395,17 @@ int mk_get_graph(mk_ctx *ctx, int32_t *task_out, int32_t *queue_out, int32_t *qo
 int mk_plan(const mk_config *cfg, int num_sms, mk_info *info,
             int32_t *task_out, int32_t *queue_out, int32_t *qoff_out,
             uint32_t *thresholds_out, int64_t *bytes_out);
+
+/* Host-only (no GPU needed): whether mk_create and mk_decode_step_static
+ * accept a device with compute capability major.minor, cooperative-launch
+ * support (0 / 1) and `smem_optin_bytes` of opt-in shared memory per block
+ * (cudaDeviceProp.sharedMemPerBlockOptin), for the batched kernel (batched
+ * != 0: max_batch > 1 or MK_FLAG_ROWS) or the batch-1 kernel.  The library
+ * holds arch-specific sm_100a code, which runs on compute capability 10.0
+ * only.  Returns MK_OK or MK_ERR_INVALID; both entry points make exactly
+ * this check on the current device before anything else touches it. */
+int mk_device_supported(int major, int minor, int cooperative_launch, size_t smem_optin_bytes,
+                        int batched);
 
 /* ---- decode without allocating --------------------------------------- */
 

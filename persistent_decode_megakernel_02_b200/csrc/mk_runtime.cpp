@@ -131,7 +131,24 @@ bool is_rows(const mk_config *c) { return c->max_batch > 1 || (c->flags & MK_FLA
 
 }  // namespace
 
+namespace mk {
+// The devices the library runs on.  The binary holds sm_100a code only,
+// which is arch-specific: it runs on compute capability 10.0 exactly, not on
+// other Blackwell parts.  Both kernels are cooperative launches and take the
+// dynamic shared memory they were built for.
+int device_check(int major, int minor, int cooperative, size_t smem_optin, bool rows) {
+    if (major != 10 || minor != 0) return MK_ERR_INVALID;
+    if (!cooperative) return MK_ERR_INVALID;
+    if (smem_optin < (rows ? rows_smem_bytes() : kernel_smem_bytes())) return MK_ERR_INVALID;
+    return MK_OK;
+}
+}  // namespace mk
+
 extern "C" {
+
+int mk_device_supported(int major, int minor, int cooperative_launch, size_t smem_optin_bytes, int batched) {
+    return device_check(major, minor, cooperative_launch, smem_optin_bytes, batched != 0);
+}
 
 const char *mk_status_string(int status) {
     switch (status) {
@@ -197,16 +214,13 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv *kv, mk_ctx
     if (cudaGetDevice(&dev) != cudaSuccess) return MK_ERR_CUDA;
     cudaDeviceProp prop;
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MK_ERR_CUDA;
-    // the binary holds sm_100a code only (arch-specific: it runs on compute
-    // capability 10.0 exactly, not on other Blackwell parts)
-    if (prop.major != 10 || prop.minor != 0) return MK_ERR_INVALID;
-    if (!prop.cooperativeLaunch) return MK_ERR_INVALID;
-    if ((size_t)prop.sharedMemPerBlockOptin < (rows ? rows_smem_bytes() : kernel_smem_bytes())) return MK_ERR_INVALID;
+    int st = device_check(prop.major, prop.minor, prop.cooperativeLaunch, (size_t)prop.sharedMemPerBlockOptin, rows);
+    if (st != MK_OK) return st;
     // The worker/control register split is only safe with the launch
     // allocation it was computed for; refuse to launch anything else.
     if (kernel_launch_regs() != kLaunchRegs) return MK_ERR_INVALID;
     Shape s;
-    int st = shape_from_config(cfg, prop.multiProcessorCount, s);
+    st = shape_from_config(cfg, prop.multiProcessorCount, s);
     if (st != MK_OK) return st;
 
     // pointer checks

@@ -39,6 +39,7 @@
 
 namespace mk {
 size_t kernel_smem_bytes();
+int device_check(int major, int minor, int cooperative, size_t smem_optin, bool rows);
 int kernel_launch_regs();
 cudaError_t kernel_prepare();
 cudaError_t kernel_launch(const Params &p, int grid, cudaStream_t stream);
@@ -170,8 +171,9 @@ extern "C" int mk_decode_step_static(const mk_config *cfg, const mk_packed_weigh
         if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return MK_ERR_CUDA;
         cudaDeviceProp prop;
         if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MK_ERR_CUDA;
-        if (prop.major != 10 || prop.minor != 0 || !prop.cooperativeLaunch) return MK_ERR_INVALID;
-        if ((size_t)prop.sharedMemPerBlockOptin < kernel_smem_bytes()) return MK_ERR_INVALID;
+        const int st = device_check(prop.major, prop.minor, prop.cooperativeLaunch,
+                                    (size_t)prop.sharedMemPerBlockOptin, false);
+        if (st != MK_OK) return st;
         if (kernel_launch_regs() != kLaunchRegs) return MK_ERR_INVALID;
         if (kernel_prepare() != cudaSuccess) return MK_ERR_CUDA;
         ds.scratch = static_cast<unsigned char *>(ptr);

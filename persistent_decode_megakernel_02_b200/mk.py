@@ -100,6 +100,7 @@ _lib.mk_get_trace.argtypes = [_P, _P, C.c_int]
 _lib.mk_get_graph.argtypes = [_P, _P, _P, _P]
 _lib.mk_get_sm_stats.argtypes = [_P, _P, C.c_int]
 _lib.mk_plan.argtypes = [C.POINTER(Config), C.c_int, C.POINTER(Info), _P, _P, _P, _P, _P]
+_lib.mk_device_supported.argtypes = [C.c_int, C.c_int, C.c_int, C.c_size_t, C.c_int]
 _lib.mk_debug_set_threshold.argtypes = [_P, C.c_int, C.c_uint]
 _lib.mk_debug_withhold_event.argtypes = [_P, C.c_int]
 _lib.mk_generate.argtypes = [_P, _P, C.c_int, _P, C.c_int, C.c_int, C.c_int, _P, _P, _P]
@@ -115,6 +116,14 @@ for _f in ("mk_create", "mk_decode_step", "mk_sync", "mk_reset", "mk_destroy", "
 
 def status_string(status: int) -> str:
     return _lib.mk_status_string(int(status)).decode()
+
+
+def device_supported(major: int, minor: int, cooperative_launch: bool, smem_optin_bytes: int,
+                     batched: bool = False) -> int:
+    """mk_device_supported: MK_OK if mk_create would accept a device with
+    these properties (host-only)."""
+    return _lib.mk_device_supported(int(major), int(minor), int(bool(cooperative_launch)),
+                                    int(smem_optin_bytes), int(bool(batched)))
 
 
 def _check(status: int, what: str):

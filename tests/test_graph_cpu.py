@@ -34,6 +34,19 @@ def test_status_strings():
     assert mk.status_string(99) == "unknown status"
 
 
+def test_device_admission():
+    # mk_create and the no-allocation entry point run this check on the
+    # current device: B200 (compute capability 10.0, cooperative launches,
+    # 227 KB = 232448 bytes of opt-in shared memory per block) is accepted;
+    # the library's arch-specific sm_100a code runs on no other device
+    for batched in (False, True):
+        assert mk.device_supported(10, 0, True, 232448, batched) == 0
+        for major, minor in ((10, 1), (10, 3), (11, 0), (12, 0), (12, 1), (9, 0), (8, 0)):
+            assert mk.device_supported(major, minor, True, 232448, batched) == mk.MK_ERR_INVALID
+        assert mk.device_supported(10, 0, False, 232448, batched) == mk.MK_ERR_INVALID
+        assert mk.device_supported(10, 0, True, 200 * 1024, batched) == mk.MK_ERR_INVALID
+
+
 def _tiles(shape):
     d, H, F, V = shape.head_dim, shape.hidden, shape.ffn, shape.vocab
     # q/k/v tiles 8 rows, gate/up tiles 8 gate + 8 up rows, the others 8 rows
