@@ -304,12 +304,19 @@ int mk_sync(mk_ctx *ctx, mk_stream_t stream);
 
 /* Clear the device error state, the event counters and the tagged
  * activations, and restart the step count (blocks the host; no step may be
- * in flight).  Also turns off the mk_debug_withhold_event hook. */
+ * in flight).  Also turns off the mk_debug_withhold_event hook.  The
+ * context is usable again afterwards (also after MK_ERR_TIMEOUT or
+ * MK_ERR_INVALID from the device).  Errors: MK_ERR_INVALID (ctx NULL),
+ * MK_ERR_CUDA (a CUDA call failed). */
 int mk_reset(mk_ctx *ctx);
 
-/* Free the context's scratch (blocks the host).  NULL is accepted. */
+/* Wait for the device, then free the context's scratch and library-owned
+ * weight copies (blocks the host).  Caller buffers are not touched.  NULL is
+ * accepted.  Always returns MK_OK. */
 int mk_destroy(mk_ctx *ctx);
 
+/* A static description of a status code ("unknown status" for codes this
+ * header does not define); never NULL, never to be freed. */
 const char *mk_status_string(int status);
 
 /* ---- introspection (tests, tracing) ------------------------------------ */
@@ -328,11 +335,15 @@ typedef struct mk_info {
     int attn_heads;                  /* q heads per attention item (MK_FLAG_ATTN_KV_ITEMS) */
 } mk_info;
 
+/* Sizes of the context's task graph and its device error word (copied
+ * from the device: call after mk_sync for the status of finished steps).
+ * Errors: MK_ERR_INVALID (ctx or out NULL), MK_ERR_CUDA. */
 int mk_get_info(mk_ctx *ctx, mk_info *out);
 
-/* Copy the event counters (uint32 [num_events]) and thresholds to host.
- * After s successful steps every counter equals threshold * s (mod 2^32).
- * Blocks the host. */
+/* Copy the first n event counters (uint32) and thresholds to host (either
+ * pointer may be NULL).  After s successful steps every counter equals
+ * threshold * s (mod 2^32).  Blocks the host.  Errors: MK_ERR_INVALID (ctx
+ * NULL, n < 0 or n > num_events), MK_ERR_CUDA. */
 int mk_get_event_counts(mk_ctx *ctx, uint32_t *counts_out, uint32_t *thresholds_out, int n);
 
 /* Scratch buffers readable after a step (host copy, blocks the host):
@@ -342,6 +353,12 @@ int mk_get_event_counts(mk_ctx *ctx, uint32_t *counts_out, uint32_t *thresholds_
  * MK_BUF_ATTN float [max_batch][nq*head_dim] last layer's attention output;
  * MK_BUF_ACT float [max_batch][ffn] last layer's SiLU(gate)*up. */
 enum mk_buffer { MK_BUF_HIDDEN = 0, MK_BUF_Q = 1, MK_BUF_ATTN = 2, MK_BUF_ACT = 3 };
+/* Copies the first `count` floats of buffer `which` to host_out.
+ * Batched contexts (max_batch > 1 or MK_FLAG_ROWS) have MK_BUF_HIDDEN only
+ * (float [16][hidden]: the residual stream after the last layer, one row
+ * per row of the last kernel step).  Errors:
+ * MK_ERR_INVALID (ctx or host_out NULL, unknown or unavailable buffer,
+ * count beyond its size), MK_ERR_CUDA. */
 int mk_read_buffer(mk_ctx *ctx, int which, float *host_out, size_t count);
 
 /* Per-task trace of the last step (MK_FLAG_TRACE).  Records are
@@ -365,6 +382,9 @@ typedef struct mk_trace_rec {
 } mk_trace_rec;
 enum mk_op_kind { MK_OP_QKV = 0, MK_OP_ATTN = 1, MK_OP_OPROJ = 2, MK_OP_GATEUP = 3,
                   MK_OP_DOWN = 4, MK_OP_LMHEAD = 5 };
+/* Copies the first n records.  Errors: MK_ERR_INVALID (ctx or host_out
+ * NULL, n < 0 or n > num_tasks, or the context was created without
+ * MK_FLAG_TRACE), MK_ERR_CUDA. */
 int mk_get_trace(mk_ctx *ctx, mk_trace_rec *host_out, int n);
 
 /* Per-SM time accounting of the last step (MK_FLAG_TRACE): uint64
@@ -377,13 +397,17 @@ int mk_get_trace(mk_ctx *ctx, mk_trace_rec *host_out, int n);
  * task ends (barrier, completion post, argmax), tasks run, worker ns in
  * attention combine/merge tails, worker ns in the first page of each
  * column-split task, worker ns in its later pages}.  Worker figures are
- * those of thread 0 and some phases overlap the waits they contain. */
+ * those of thread 0 and some phases overlap the waits they contain.  Copies
+ * the first n values.  Errors: MK_ERR_INVALID (ctx or host_out NULL, n < 0
+ * or n > num_sms * 16, or no MK_FLAG_TRACE), MK_ERR_CUDA. */
 int mk_get_sm_stats(mk_ctx *ctx, uint64_t *host_out, int n);
 
 /* Static task graph as built by mk_create (host copy).  task_out: int32
  * [num_tasks][8] = {kind, layer, dep_event (-1 none), trig_event, begin,
  * end, sm, slot}; queue_out: int32 [num_tasks] task ids grouped by SM in
- * execution order; qoff_out: int32 [num_sms+1] offsets into queue_out. */
+ * execution order; qoff_out: int32 [num_sms+1] offsets into queue_out.
+ * Any of the arrays may be NULL; the sizes are in mk_get_info.  No device
+ * access.  Errors: MK_ERR_INVALID (ctx NULL). */
 int mk_get_graph(mk_ctx *ctx, int32_t *task_out, int32_t *queue_out, int32_t *qoff_out);
 
 /* Host-only planning (no GPU needed): build the task graph for `cfg` on a
@@ -391,7 +415,9 @@ int mk_get_graph(mk_ctx *ctx, int32_t *task_out, int32_t *queue_out, int32_t *qo
  * num_events, num_ops, attn_chunks, max_queue, page sizes), then fill the
  * arrays as mk_get_graph does (any of them may be NULL) plus thresholds_out
  * uint32 [num_events] and the per-task weight bytes bytes_out int64
- * [num_tasks].  Used to test the graph builder without a device. */
+ * [num_tasks].  Used to test the graph builder without a device.  Errors:
+ * MK_ERR_INVALID (cfg NULL, a shape or option mk_create would refuse,
+ * num_sms outside 1..1024). */
 int mk_plan(const mk_config *cfg, int num_sms, mk_info *info,
             int32_t *task_out, int32_t *queue_out, int32_t *qoff_out,
             uint32_t *thresholds_out, int64_t *bytes_out);
